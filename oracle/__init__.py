@@ -1,0 +1,152 @@
+"""CPU oracle for the packed 1-bit / balanced-ternary matmul (numpy wrappers).
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, by __graft_entry__.smoke() and by
+bench.py's CPU-baseline leg.  The product path (the CUDA library and its
+binding) never imports this package, and this package never imports it.
+
+Every function takes and returns host numpy arrays and calls the plain C++
+definitions in bnn_oracle.cpp (built on first use by oracle/build.py).  Which
+passage of the pages each definition follows is stated beside it there.
+"""
+from __future__ import annotations
+
+import ctypes as C
+
+import numpy as np
+
+from .build import build as _build
+
+_lib = None
+
+
+def _L():
+    global _lib
+    if _lib is None:
+        lib = C.CDLL(_build())
+        i64, vp = C.c_int64, C.c_void_p
+        sig = {
+            "oracle_pack_signs": ([vp, i64, i64, vp], None),
+            "oracle_unpack_signs": ([vp, i64, i64, vp], None),
+            "oracle_count_pad_bits": ([vp, i64, i64], i64),
+            "oracle_binary_gemm": ([vp, vp, vp, i64, i64, i64, vp, vp], None),
+            "oracle_binary_gemm_sampled": ([vp, vp, vp, i64, i64, i64, vp, vp, i64, vp, vp], None),
+            "oracle_twn_ternarize": ([vp, i64, i64, vp, vp, vp], None),
+            "oracle_base3_pack": ([vp, i64, i64, vp], None),
+            "oracle_base3_unpack": ([vp, i64, i64, vp], i64),
+            "oracle_ternary_gemm": ([vp, vp, vp, i64, i64, i64, vp, vp], None),
+            "oracle_ternary_gemm_sampled": ([vp, vp, vp, i64, i64, i64, vp, vp, i64, vp, vp], None),
+        }
+        for name, (args, res) in sig.items():
+            f = getattr(lib, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = lib
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(C.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def words_per_row(k: int) -> int:
+    return (k + 63) // 64
+
+
+def trit_words_per_row(k: int) -> int:
+    return (k + 9) // 10
+
+
+def pack_signs(x: np.ndarray, k: int | None = None) -> np.ndarray:
+    """fp32 [rows, k] -> uint64 [rows, ceil(k/64)]; bit 1 iff !(x > 0)."""
+    x = _c(x, np.float32)
+    x2 = x.reshape(-1, x.shape[-1]) if x.ndim > 1 else x.reshape(1, -1)
+    rows, kk = x2.shape
+    out = np.zeros((rows, words_per_row(kk)), dtype=np.uint64)
+    _L().oracle_pack_signs(_p(x2), rows, kk, _p(out))
+    return out
+
+
+def unpack_signs(p: np.ndarray, k: int) -> np.ndarray:
+    p = _c(p, np.uint64).reshape(-1, words_per_row(k)) if k else _c(p, np.uint64).reshape(-1, 0)
+    out = np.zeros((p.shape[0], k), dtype=np.int8)
+    _L().oracle_unpack_signs(_p(p), p.shape[0], k, _p(out))
+    return out
+
+
+def count_pad_bits(p: np.ndarray, k: int) -> int:
+    p = _c(p, np.uint64)
+    rows = p.shape[0] if p.ndim > 1 else 1
+    return int(_L().oracle_count_pad_bits(_p(p), rows, k))
+
+
+def binary_gemm(xp, wp, alpha, m: int, n: int, k: int):
+    """Returns (dots int32 [m,n], out float32 [m,n])."""
+    xp, wp, alpha = _c(xp, np.uint64), _c(wp, np.uint64), _c(alpha, np.float32)
+    dots = np.zeros((m, n), dtype=np.int32)
+    out = np.zeros((m, n), dtype=np.float32)
+    _L().oracle_binary_gemm(_p(xp), _p(wp), _p(alpha), m, n, k, _p(dots), _p(out))
+    return dots, out
+
+
+def binary_gemm_sampled(xp, wp, alpha, m: int, n: int, k: int, rows, cols):
+    xp, wp, alpha = _c(xp, np.uint64), _c(wp, np.uint64), _c(alpha, np.float32)
+    rows, cols = _c(rows, np.int64), _c(cols, np.int64)
+    assert rows.shape == cols.shape
+    assert rows.size == 0 or (rows.min() >= 0 and rows.max() < m and cols.min() >= 0 and cols.max() < n)
+    dots = np.zeros(rows.shape, dtype=np.int32)
+    out = np.zeros(rows.shape, dtype=np.float32)
+    _L().oracle_binary_gemm_sampled(_p(xp), _p(wp), _p(alpha), m, n, k, _p(rows), _p(cols),
+                                    rows.size, _p(dots), _p(out))
+    return dots, out
+
+
+def twn_ternarize(w: np.ndarray):
+    """fp32 [n,k] -> (trits int8 [n,k], scale float32 [n], delta float32)."""
+    w = _c(w, np.float32)
+    n, k = w.shape
+    trits = np.zeros((n, k), dtype=np.int8)
+    scale = np.zeros(n, dtype=np.float32)
+    delta = np.zeros(1, dtype=np.float32)
+    _L().oracle_twn_ternarize(_p(w), n, k, _p(trits), _p(scale), _p(delta))
+    return trits, scale, np.float32(delta[0])
+
+
+def base3_pack(trits: np.ndarray) -> np.ndarray:
+    trits = _c(trits, np.int8)
+    n, k = trits.shape
+    out = np.zeros((n, trit_words_per_row(k)), dtype=np.uint16)
+    _L().oracle_base3_pack(_p(trits), n, k, _p(out))
+    return out
+
+
+def base3_unpack(packed: np.ndarray, k: int):
+    """-> (trits int8 [n,k], number of words >= 3^10)."""
+    packed = _c(packed, np.uint16)
+    n = packed.shape[0]
+    trits = np.zeros((n, k), dtype=np.int8)
+    bad = _L().oracle_base3_unpack(_p(packed), n, k, _p(trits))
+    return trits, int(bad)
+
+
+def ternary_gemm(x_bf16, packed, scale, m: int, n: int, k: int):
+    """Returns (y float64 [m,n], mag float64 [m,n])."""
+    x_bf16, packed, scale = _c(x_bf16, np.uint16), _c(packed, np.uint16), _c(scale, np.float32)
+    y = np.zeros((m, n), dtype=np.float64)
+    mag = np.zeros((m, n), dtype=np.float64)
+    _L().oracle_ternary_gemm(_p(x_bf16), _p(packed), _p(scale), m, n, k, _p(y), _p(mag))
+    return y, mag
+
+
+def ternary_gemm_sampled(x_bf16, packed, scale, m: int, n: int, k: int, rows, cols):
+    x_bf16, packed, scale = _c(x_bf16, np.uint16), _c(packed, np.uint16), _c(scale, np.float32)
+    rows, cols = _c(rows, np.int64), _c(cols, np.int64)
+    assert rows.size == 0 or (rows.min() >= 0 and rows.max() < m and cols.min() >= 0 and cols.max() < n)
+    y = np.zeros(rows.shape, dtype=np.float64)
+    mag = np.zeros(rows.shape, dtype=np.float64)
+    _L().oracle_ternary_gemm_sampled(_p(x_bf16), _p(packed), _p(scale), m, n, k, _p(rows), _p(cols),
+                                     rows.size, _p(y), _p(mag))
+    return y, mag

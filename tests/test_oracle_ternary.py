@@ -1,0 +1,188 @@
+"""Pins for the oracle's ternary path: exhaustive base-3 round trip over all
+3^10 codes, closed-form words, hand-worked TWN cases, least-squares
+optimality, N(0,1) statistics with known closed forms, and the ternary matmul
+against numpy float64 matmul and special cases.
+
+Page: "BalancedTernaryEngine" README, sections "Features" (TWN threshold,
+least-squares per-channel scale, 10 trits per 16-bit word in base 3),
+".tbin Format" and Layer.forward in "Module Overview"."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from conftest import golden_lines
+from ternary_neural_net_b200 import synth
+
+
+def all_trit_vectors():
+    """All 3^10 trit vectors, as an independent enumeration (itertools order)."""
+    import itertools
+    return np.array(list(itertools.product((-1, 0, 1), repeat=10)), dtype=np.int8)
+
+
+def test_base3_exhaustive_bijection():
+    t = all_trit_vectors()                        # 59049 x 10
+    words = oracle.base3_pack(t).reshape(-1)       # one word per vector
+    assert words.dtype == np.uint16
+    assert words.max() == 59048 and words.min() == 0
+    assert np.unique(words).size == 59049          # injective onto 0..59048
+    back, bad = oracle.base3_unpack(words.reshape(-1, 1), 10)
+    assert bad == 0 and np.array_equal(back, t)
+    all_words = np.arange(59049, dtype=np.uint16).reshape(-1, 1)
+    t2, bad2 = oracle.base3_unpack(all_words, 10)
+    assert bad2 == 0
+    assert np.array_equal(oracle.base3_pack(t2).reshape(-1), all_words.reshape(-1))
+
+
+def test_base3_words_above_range_are_flagged():
+    w = np.array([[59049], [65535], [59048]], dtype=np.uint16)
+    _, bad = oracle.base3_unpack(w, 10)
+    assert bad == 2
+
+
+def test_base3_golden_words():
+    for line in golden_lines("base3_words.txt"):
+        f = line.split()
+        word, t = int(f[0]), np.array([[int(v) for v in f[1:]]], dtype=np.int8)
+        assert int(oracle.base3_pack(t)[0, 0]) == word
+        back, bad = oracle.base3_unpack(np.array([[word]], np.uint16), 10)
+        assert bad == 0 and np.array_equal(back, t)
+
+
+@pytest.mark.parametrize("k", [1, 9, 10, 11, 19, 20, 21, 4096])
+def test_base3_row_padding(k):
+    """Rows are packed independently; trits past k are 0 (digit 1)."""
+    rng = np.random.default_rng(k)
+    t = rng.integers(-1, 2, (3, k)).astype(np.int8)
+    p = oracle.base3_pack(t)
+    assert p.shape == (3, (k + 9) // 10)
+    back, bad = oracle.base3_unpack(p, k)
+    assert bad == 0 and np.array_equal(back, t)
+    padded = np.zeros((3, 10 * p.shape[1]), np.int8)
+    padded[:, :k] = t
+    back_full, _ = oracle.base3_unpack(p, 10 * p.shape[1])
+    assert np.array_equal(back_full, padded)
+    # word j depends only on trits 10j..10j+9: one word per 10-trit slice
+    for j in range(p.shape[1]):
+        assert np.array_equal(oracle.base3_pack(padded[:, 10 * j: 10 * j + 10])[:, 0], p[:, j])
+
+
+def _twn_cases():
+    lines = list(golden_lines("twn_small.txt"))
+    i = 0
+    while i < len(lines):
+        _, name, rows, cols = lines[i].split()
+        rows, cols = int(rows), int(cols)
+        w = np.array([[float(v) for v in lines[i + 1 + r].split()] for r in range(rows)], np.float32)
+        d = lines[i + 1 + rows].split()[1]
+        tr, sc = [], []
+        for r in range(rows):
+            a, b = lines[i + 2 + rows + r].split("|")
+            tr.append([int(v) for v in a.split()])
+            sc.append(float(b))
+        yield name, w, (None if d == "-" else int(d, 16)), np.array(tr, np.int8), np.array(sc, np.float32)
+        i += 2 + 2 * rows
+
+
+@pytest.mark.parametrize("case", list(_twn_cases()), ids=lambda c: c[0])
+def test_twn_golden(case):
+    _, w, delta_bits, trits, scales = case
+    t, s, d = oracle.twn_ternarize(w)
+    if delta_bits is not None:
+        assert int(np.array([d], np.float32).view(np.uint32)[0]) == delta_bits
+    assert np.array_equal(t, trits)
+    assert np.array_equal(s, scales)
+
+
+def test_twn_constant_magnitude_rows_reconstruct_exactly():
+    rng = np.random.default_rng(21)
+    c = np.float32(rng.random() * 4 + 0.1)
+    signs = np.where(rng.random((5, 33)) < 0.5, 1, -1).astype(np.float32)
+    w = c * signs
+    t, s, d = oracle.twn_ternarize(w)
+    assert np.array_equal(t, signs.astype(np.int8))
+    assert np.all(s == c)
+    assert d == np.float32(0.7 * np.float64(c))
+
+
+def test_twn_least_squares_optimal():
+    """For the oracle's trits, its scale minimises sum (w - s t)^2 per row: a
+    perturbation either way does not lower the error (textbook LS)."""
+    w = synth.normal_f32(3, 1, (16, 300)).astype(np.float64)
+    t, s, _ = oracle.twn_ternarize(w.astype(np.float32))
+    t = t.astype(np.float64)
+    for r in range(16):
+        def err(sc):
+            return float(((w[r] - sc * t[r]) ** 2).sum())
+        s_ls = float((w[r] * t[r]).sum() / (t[r] * t[r]).sum())   # numpy normal equations
+        assert abs(float(s[r]) - s_ls) <= 2e-7 * s_ls
+        for eps in (1e-3, 1e-5):
+            assert err(float(s[r])) <= err(float(s[r]) * (1 + eps))
+            assert err(float(s[r])) <= err(float(s[r]) * (1 - eps))
+
+
+def test_twn_gaussian_statistics():
+    """For W ~ N(0,1): mean|W| -> sqrt(2/pi), Delta -> 0.7 sqrt(2/pi), the zero
+    fraction -> erf(Delta/sqrt 2), and the mean scale -> E[|w| : |w| > Delta]
+    = phi(Delta) / (1 - Phi(Delta))."""
+    w = synth.normal_f32(4, 2, (512, 4096))
+    t, s, d = oracle.twn_ternarize(w)
+    delta_inf = 0.7 * math.sqrt(2 / math.pi)
+    assert abs(float(d) - delta_inf) < 3e-3
+    zero_frac = float((t == 0).mean())
+    assert abs(zero_frac - math.erf(float(d) / math.sqrt(2))) < 3e-3
+    phi = math.exp(-float(d) ** 2 / 2) / math.sqrt(2 * math.pi)
+    tail = 0.5 * math.erfc(float(d) / math.sqrt(2))
+    assert abs(float(s.mean()) - phi / tail) < 5e-3
+    # trits agree with the sign of w wherever they are not zero, and |w| > Delta there
+    nz = t != 0
+    assert np.all(np.sign(w[nz]) == t[nz])
+    assert np.all(np.abs(w[nz]) > d) and np.all(np.abs(w[~nz]) <= d)
+
+
+def _bf16(x):
+    return synth.bf16_bits_from_f32(np.asarray(x, np.float32))
+
+
+def _bf16_to_f64_torch(bits):
+    """Independent widening: torch's own bfloat16 -> float64 conversion."""
+    t = torch.from_numpy(np.asarray(bits, np.uint16).astype(np.int16)).view(torch.bfloat16)
+    return t.to(torch.float64).numpy()
+
+
+def test_ternary_gemm_special_cases():
+    k = 37
+    xb = _bf16(synth.normal_f32(5, 1, (2, k)))
+    xd = _bf16_to_f64_torch(xb)
+    trits = np.zeros((4, k), np.int8)
+    trits[0] = 1                 # all +1 -> s * sum x
+    trits[2, 11] = 1             # one-hot +1 at 11 -> s * x_11
+    trits[3, 30] = -1            # one-hot -1 at 30 -> -s * x_30
+    scale = np.array([1.25, 3.0, 0.5, 2.0], np.float32)
+    y, mag = oracle.ternary_gemm(xb, oracle.base3_pack(trits), scale, 2, 4, k)
+    for i in range(2):
+        assert y[i, 0] == pytest.approx(1.25 * xd[i].sum(), rel=1e-15, abs=1e-15)
+        assert mag[i, 0] == pytest.approx(1.25 * np.abs(xd[i]).sum(), rel=1e-15)
+        assert y[i, 1] == 0.0 and mag[i, 1] == 0.0
+        assert y[i, 2] == 0.5 * xd[i, 11]
+        assert y[i, 3] == -2.0 * xd[i, 30]
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 5, 10), (3, 7, 23), (4, 2, 95), (2, 3, 1)])
+def test_ternary_gemm_against_numpy(m, n, k):
+    rng = np.random.default_rng(m * 100 + n * 10 + k)
+    trits = rng.integers(-1, 2, (n, k)).astype(np.int8)
+    scale = (rng.random(n) + 0.5).astype(np.float32)
+    xb = _bf16(rng.standard_normal((m, k)))
+    y, mag = oracle.ternary_gemm(xb, oracle.base3_pack(trits), scale, m, n, k)
+    xd = _bf16_to_f64_torch(xb)
+    want = (xd @ trits.T.astype(np.float64)) * scale.astype(np.float64)[None, :]
+    np.testing.assert_allclose(y, want, rtol=1e-12, atol=1e-12)
+    want_mag = (np.abs(xd) @ np.abs(trits.T).astype(np.float64)) * scale.astype(np.float64)[None, :]
+    np.testing.assert_allclose(mag, want_mag, rtol=1e-12, atol=1e-12)
+    rows, cols = rng.integers(0, m, 9), rng.integers(0, n, 9)
+    ys, ms = oracle.ternary_gemm_sampled(xb, oracle.base3_pack(trits), scale, m, n, k, rows, cols)
+    assert np.array_equal(ys, y[rows, cols]) and np.array_equal(ms, mag[rows, cols])
