@@ -1,0 +1,153 @@
+/*
+ * bnn.h -- C ABI of the packed 1-bit / balanced-ternary matmul for NVIDIA B200
+ * (sm_100a).  Library: libbnn.so (built in-tree by ternary_neural_net_b200/build.py).
+ *
+ * Sources the operations are defined by (page title, section):
+ *   [BME] "Binary Math Effectiveness -- why / how / when", section 1 "The core
+ *         identity": bit 0 encodes +1 and bit 1 encodes -1; <x,w> = n - 2d with
+ *         d = popcount(x XOR w) over the logical n; "Edge cases": pad bits
+ *         encode +1 and do not count, n = 0 gives 0, a channel scale alpha = 0
+ *         gives 0, inputs <= 0 project to -1 and > 0 to +1.
+ *   [ADR] "Architecture Decision Record", section "Decision": binary_gemm_u64,
+ *         the packed XNOR/XOR + popcount matmul over uint64 words.
+ *   [BTE] "BalancedTernaryEngine" README, section "Features": TWN threshold
+ *         Delta = 0.7 * mean|W|, least-squares per-channel scale, 10 trits per
+ *         16-bit word in base 3; "Module Overview": Layer.forward.
+ *
+ * Conventions shared by every call:
+ *   - Layout.  Every matrix is row-major with the reduction dimension k
+ *     contiguous: activations X[m,k], weights W[n,k] (the nn.Linear weight
+ *     layout), outputs [m,n].  A packed sign row is kw = ceil(k/64) uint64
+ *     words; element e of the row is bit (e mod 64) of word e/64 (least
+ *     significant bit first), bits at positions >= k are 0.  A packed trit row
+ *     is kt = ceil(k/10) uint16 words; word j holds trits 10j..10j+9, trit
+ *     10j+i contributing (trit + 1) * 3^i, trits past k being 0 (digit 1).
+ *     Rows are stored back to back with no extra pitch.
+ *   - Pointers are DEVICE pointers (memory the caller allocated with any CUDA
+ *     allocator, e.g. PyTorch's).  The caller owns every buffer; the library
+ *     keeps no pointer after a call returns.  Buffers must not overlap.
+ *   - Every call is asynchronous and ordered on the stream `s` it is given
+ *     (0 = the legacy default stream).  It returns after enqueueing its
+ *     kernels; the status covers argument checks and the launch only.  It
+ *     never synchronises the device or the stream.
+ *   - Errors.  BNN_ERR_INVALID_ARG: a size is negative or too large, or a
+ *     required pointer is NULL.  BNN_ERR_MISALIGNED: a pointer is not aligned
+ *     to its element size (8 bytes for uint64, 4 for float/int32, 2 for
+ *     uint16).  BNN_ERR_CUDA: a CUDA runtime call or a kernel launch failed
+ *     (bnn_last_cuda_error() gives the cudaError_t of the calling thread's
+ *     last failure).  Nothing is written when a call fails its argument
+ *     checks.  Sizes of 0 are valid and return BNN_OK.
+ *   - Threads.  Calls are re-entrant; concurrent calls on different streams
+ *     are independent.
+ */
+#ifndef BNN_H
+#define BNN_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BNN_OK = 0,
+  BNN_ERR_INVALID_ARG = 1,
+  BNN_ERR_MISALIGNED = 2,
+  BNN_ERR_CUDA = 3,
+  BNN_ERR_UNSUPPORTED = 4
+} bnn_status;
+
+/* Largest logical reduction length accepted by the binary matmul: with
+ * |dot| <= k <= 2^24 every dot is exact in float32, so the alpha epilogue is a
+ * single correctly rounded float32 multiply. */
+#define BNN_MAX_K_BINARY (1 << 24)
+
+/*
+ * bnn_pack_signs -- sign-pack float32 rows into uint64 words.  [BME] section 1
+ * encoding table and "Edge cases" (<= 0 -> -1, > 0 -> +1; pad bits +1).
+ *
+ *   x     float32 [rows, k], device, 4-byte aligned.
+ *   rows  number of rows, >= 0.
+ *   k     logical row length, >= 0.
+ *   out   uint64 [rows, ceil(k/64)], device, 8-byte aligned.  Bit e of a row
+ *         is 1 exactly when !(x[e] > 0), so +-0, NaN and -inf give -1 (bit 1)
+ *         and denormals keep their sign (no flush to zero).  Pad bits are 0.
+ */
+bnn_status bnn_pack_signs(const float* x, int64_t rows, int64_t k, uint64_t* out,
+                          cudaStream_t s);
+
+/*
+ * bnn_binary_gemm -- packed XOR + popcount matmul with a per-output-channel
+ * scale.  [ADR] "Decision" (binary_gemm_u64); [BME] section 1 (identity and
+ * "Edge cases").
+ *
+ *   xp     uint64 [m, ceil(k/64)] packed activations, device, 8-byte aligned.
+ *   wp     uint64 [n, ceil(k/64)] packed weights, device, 8-byte aligned.
+ *          Pad bits of xp and wp must be 0 (bnn_pack_signs guarantees it);
+ *          they are not masked.
+ *   alpha  float32 [n] per-output-channel scale, device; may be NULL only
+ *          when out is NULL.
+ *   m, n   output shape, >= 0.
+ *   k      logical reduction length, 0 <= k <= BNN_MAX_K_BINARY.
+ *   dots   int32 [m, n] or NULL: dots[i,j] = k - 2 * popcount(xp_i XOR wp_j),
+ *          the exact +-1 dot product.
+ *   out    float32 [m, n] or NULL: out[i,j] = alpha[j] * (float)dots[i,j], one
+ *          IEEE float32 multiply, round to nearest even.
+ *   At least one of dots and out must be non-NULL.  With k = 0 every dot is 0
+ *   and out is alpha * 0.
+ */
+bnn_status bnn_binary_gemm(const uint64_t* xp, const uint64_t* wp, const float* alpha,
+                           int64_t m, int64_t n, int64_t k, int32_t* dots, float* out,
+                           cudaStream_t s);
+
+/*
+ * bnn_ternary_pack -- TWN ternarisation, least-squares per-row scale and base-3
+ * packing of a float32 weight matrix.  [BTE] "Features".
+ *
+ *   w       float32 [n, k] weights, device, 4-byte aligned.
+ *   n, k    shape, >= 0, n * k < 2^40.
+ *   packed  uint16 [n, ceil(k/10)] base-3 words (see Layout), device, 2-byte aligned.
+ *   scale   float32 [n], device: scale[r] = float32(mean of |w[r,e]| over the
+ *           e with a non-zero trit), 0 for a row whose trits are all 0; the
+ *           least-squares scale for the row's trits.
+ *   delta   float32 [1], device: Delta = float32(0.7 * mean|W|), the mean
+ *           taken over all n*k weights in float64 (0 when n*k = 0).
+ *   Trit of w[r,e]: +1 if |w| > Delta and w > 0, -1 if |w| > Delta and w < 0,
+ *   else 0 (a tie |w| == Delta gives 0; NaN gives 0).
+ *   Scratch: the float64 partial sums of |W| (8 bytes per 65536 weights) are
+ *   taken from the stream-ordered allocator (cudaMallocAsync / cudaFreeAsync
+ *   on s); BNN_ERR_CUDA if that allocation fails.  The reduction order is
+ *   fixed, so results are bitwise reproducible from run to run.
+ */
+bnn_status bnn_ternary_pack(const float* w, int64_t n, int64_t k, uint16_t* packed,
+                            float* scale, float* delta, cudaStream_t s);
+
+/*
+ * bnn_ternary_gemm -- ternary layer forward: base-3 unpack and accumulate.
+ * [BTE] "Module Overview" (Layer.forward) with the "Features" encoding.
+ *
+ *   x_bf16  bfloat16 [m, k] activations as raw 16-bit patterns, device,
+ *           2-byte aligned.
+ *   packed  uint16 [n, ceil(k/10)] base-3 words, device, 2-byte aligned; every
+ *           word must be < 3^10 = 59049 (not checked on the hot path).
+ *   scale   float32 [n], device.
+ *   m, n, k shape, >= 0.
+ *   out     float32 [m, n], device: out[i,j] = scale[j] * sum_e x[i,e] * t[j,e],
+ *           the products exact, the sum accumulated in float32 (in an order
+ *           the library chooses), the scale applied once after the sum.
+ */
+bnn_status bnn_ternary_gemm(const uint16_t* x_bf16, const uint16_t* packed, const float* scale,
+                            int64_t m, int64_t n, int64_t k, float* out, cudaStream_t s);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* bnn_status_string(bnn_status st);
+
+/* cudaError_t (as int) of the calling thread's most recent BNN_ERR_CUDA, or 0. */
+int bnn_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BNN_H */

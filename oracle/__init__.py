@@ -31,6 +31,8 @@ def _L():
             "oracle_binary_gemm": ([vp, vp, vp, i64, i64, i64, vp, vp], None),
             "oracle_binary_gemm_sampled": ([vp, vp, vp, i64, i64, i64, vp, vp, i64, vp, vp], None),
             "oracle_twn_ternarize": ([vp, i64, i64, vp, vp, vp], None),
+            "oracle_twn_delta": ([vp, i64], C.c_float),
+            "oracle_twn_apply": ([vp, i64, i64, C.c_float, vp, vp], None),
             "oracle_base3_pack": ([vp, i64, i64, vp], None),
             "oracle_base3_unpack": ([vp, i64, i64, vp], i64),
             "oracle_ternary_gemm": ([vp, vp, vp, i64, i64, i64, vp, vp], None),
@@ -113,6 +115,21 @@ def twn_ternarize(w: np.ndarray):
     delta = np.zeros(1, dtype=np.float32)
     _L().oracle_twn_ternarize(_p(w), n, k, _p(trits), _p(scale), _p(delta))
     return trits, scale, np.float32(delta[0])
+
+
+def twn_delta(w: np.ndarray) -> np.float32:
+    w = _c(w, np.float32)
+    return np.float32(_L().oracle_twn_delta(_p(w), w.size))
+
+
+def twn_apply(w: np.ndarray, delta) -> tuple:
+    """Trits and least-squares scales for a given threshold Delta (float32)."""
+    w = _c(w, np.float32)
+    n, k = w.shape
+    trits = np.zeros((n, k), dtype=np.int8)
+    scale = np.zeros(n, dtype=np.float32)
+    _L().oracle_twn_apply(_p(w), n, k, C.c_float(np.float32(delta)), _p(trits), _p(scale))
+    return trits, scale
 
 
 def base3_pack(trits: np.ndarray) -> np.ndarray:

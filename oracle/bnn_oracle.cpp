@@ -128,17 +128,19 @@ void oracle_binary_gemm_sampled(const uint64_t* xp, const uint64_t* wp, const fl
 }
 
 // [BTE] "Features": TWN threshold Delta = 0.7 * mean|W| over the whole tensor,
-// trit = sign(w) where |w| > Delta else 0, and a per-channel least-squares
-// scale.  For fixed trits t the least-squares scale of row r minimises
-// sum_e (w_e - s * t_e)^2, i.e. s = <w,t>/<t,t> = mean of |w| over t != 0.
-void oracle_twn_ternarize(const float* w, int64_t n, int64_t k, int8_t* trits,
-                          float* scale, float* delta) {
-  const int64_t total = n * k;
+// the mean summed in float64 in element order and Delta rounded once to float32.
+float oracle_twn_delta(const float* w, int64_t total) {
   double sum_abs = 0.0;
   for (int64_t e = 0; e < total; ++e) sum_abs += std::fabs(double(w[e]));
   const double mean_abs = total > 0 ? sum_abs / double(total) : 0.0;
-  const float d = float(0.7 * mean_abs);
-  *delta = d;
+  return float(0.7 * mean_abs);
+}
+
+// [BTE] "Features": trit = sign(w) where |w| > Delta else 0 (the comparison in
+// float32), and a per-channel least-squares scale.  For fixed trits t the
+// least-squares scale of row r minimises sum_e (w_e - s * t_e)^2, i.e.
+// s = <w,t>/<t,t> = mean of |w| over t != 0 (0 for a row with no non-zero trit).
+void oracle_twn_apply(const float* w, int64_t n, int64_t k, float d, int8_t* trits, float* scale) {
   for (int64_t r = 0; r < n; ++r) {
     double kept = 0.0;
     int64_t nonzero = 0;
@@ -154,6 +156,14 @@ void oracle_twn_ternarize(const float* w, int64_t n, int64_t k, int8_t* trits,
     }
     scale[r] = nonzero > 0 ? float(kept / double(nonzero)) : 0.0f;
   }
+}
+
+// The two steps above in order: Delta from the whole tensor, then trits and scales.
+void oracle_twn_ternarize(const float* w, int64_t n, int64_t k, int8_t* trits,
+                          float* scale, float* delta) {
+  const float d = oracle_twn_delta(w, n * k);
+  *delta = d;
+  oracle_twn_apply(w, n, k, d, trits, scale);
 }
 
 // [BTE] "Features": 10 trits per 16-bit word, base 3.  Word j of a row holds

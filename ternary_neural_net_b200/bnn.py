@@ -1,0 +1,176 @@
+"""Python binding of libbnn (the C ABI declared in include/bnn.h).
+
+Argument marshalling only: every function checks shapes and dtypes, allocates
+outputs with PyTorch when the caller does not pass them, and calls the
+library entry point of the same name with raw device pointers and the current
+CUDA stream.  Every step of the computation runs in the library's kernels;
+there is no fallback.  Importing this module loads libbnn.so and raises
+ImportError when it is missing (build it with
+``python -m ternary_neural_net_b200.build``).
+
+dtype conventions (PyTorch has no general-purpose unsigned tensors, so the
+unsigned words travel in signed tensors of the same width, bit for bit):
+  packed sign words   torch.int64  [rows, ceil(k/64)]   (uint64 in the ABI)
+  base-3 trit words   torch.int16  [n, ceil(k/10)]      (uint16 in the ABI)
+  bf16 activations    torch.bfloat16 [m, k]             (uint16 bit patterns in the ABI)
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbnn.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libbnn.so not found at {LIB_PATH}; build it with "
+                      "`python -m ternary_neural_net_b200.build` (needs nvcc)")
+_lib = C.CDLL(LIB_PATH)
+
+_vp, _i64, _int = C.c_void_p, C.c_int64, C.c_int
+_SIGS = {
+    "bnn_pack_signs": [_vp, _i64, _i64, _vp, _vp],
+    "bnn_binary_gemm": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp],
+    "bnn_ternary_pack": [_vp, _i64, _i64, _vp, _vp, _vp, _vp],
+    "bnn_ternary_gemm": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
+}
+for _name, _args in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.argtypes = _args
+    _f.restype = _int
+_lib.bnn_status_string.argtypes = [_int]
+_lib.bnn_status_string.restype = C.c_char_p
+_lib.bnn_last_cuda_error.argtypes = []
+_lib.bnn_last_cuda_error.restype = _int
+
+# Exported symbol names, as declared in include/bnn.h.
+ABI_SYMBOLS = tuple(_SIGS) + ("bnn_status_string", "bnn_last_cuda_error")
+
+BNN_OK, BNN_ERR_INVALID_ARG, BNN_ERR_MISALIGNED, BNN_ERR_CUDA, BNN_ERR_UNSUPPORTED = range(5)
+MAX_K_BINARY = 1 << 24
+
+
+class BnnError(RuntimeError):
+    def __init__(self, status: int, call: str):
+        msg = _lib.bnn_status_string(status).decode()
+        if status == BNN_ERR_CUDA:
+            msg += f" (cudaError {_lib.bnn_last_cuda_error()})"
+        super().__init__(f"{call}: {msg}")
+        self.status = status
+
+
+def lib() -> C.CDLL:
+    """The loaded libbnn handle (for raw-pointer calls)."""
+    return _lib
+
+
+def _check(st: int, call: str):
+    if st != BNN_OK:
+        raise BnnError(st, call)
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(device):
+    return C.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None, ndim=2):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must be {ndim}-D, got shape {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def words_per_row(k: int) -> int:
+    return (k + 63) // 64
+
+
+def trit_words_per_row(k: int) -> int:
+    return (k + 9) // 10
+
+
+def bnn_pack_signs(x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """float32 [rows, k] -> packed int64 [rows, ceil(k/64)] (bit 1 iff !(x > 0))."""
+    _dev(x, "x", torch.float32)
+    rows, k = x.shape
+    if out is None:
+        out = torch.empty((rows, words_per_row(k)), dtype=torch.int64, device=x.device)
+    else:
+        _dev(out, "out", torch.int64)
+        if tuple(out.shape) != (rows, words_per_row(k)):
+            raise ValueError("out has the wrong shape")
+    _check(_lib.bnn_pack_signs(_ptr(x), rows, k, _ptr(out), _stream(x.device)), "bnn_pack_signs")
+    return out
+
+
+def bnn_binary_gemm(xp: torch.Tensor, wp: torch.Tensor, alpha: torch.Tensor | None, k: int,
+                    want_dots: bool = True, want_out: bool = True,
+                    dots: torch.Tensor | None = None, out: torch.Tensor | None = None):
+    """Packed XOR+popcount matmul.  Returns (dots int32 [m,n] or None, out float32 [m,n] or None)."""
+    _dev(xp, "xp", torch.int64)
+    _dev(wp, "wp", torch.int64)
+    m, n = xp.shape[0], wp.shape[0]
+    if xp.shape[1] != words_per_row(k) or wp.shape[1] != words_per_row(k):
+        raise ValueError("packed rows must hold ceil(k/64) words")
+    dev = xp.device
+    if want_dots and dots is None:
+        dots = torch.empty((m, n), dtype=torch.int32, device=dev)
+    if want_out and out is None:
+        out = torch.empty((m, n), dtype=torch.float32, device=dev)
+    if dots is not None:
+        _dev(dots, "dots", torch.int32)
+    if out is not None:
+        _dev(out, "out", torch.float32)
+        _dev(alpha, "alpha", torch.float32, ndim=1)
+    _check(_lib.bnn_binary_gemm(_ptr(xp), _ptr(wp), _ptr(alpha), m, n, k, _ptr(dots), _ptr(out),
+                                _stream(dev)), "bnn_binary_gemm")
+    return dots, out
+
+
+def bnn_ternary_pack(w: torch.Tensor, packed: torch.Tensor | None = None,
+                     scale: torch.Tensor | None = None, delta: torch.Tensor | None = None):
+    """float32 [n, k] -> (packed int16 [n, ceil(k/10)], scale float32 [n], delta float32 [1])."""
+    _dev(w, "w", torch.float32)
+    n, k = w.shape
+    dev = w.device
+    if packed is None:
+        packed = torch.empty((n, trit_words_per_row(k)), dtype=torch.int16, device=dev)
+    if scale is None:
+        scale = torch.empty((n,), dtype=torch.float32, device=dev)
+    if delta is None:
+        delta = torch.empty((1,), dtype=torch.float32, device=dev)
+    _dev(packed, "packed", torch.int16)
+    _dev(scale, "scale", torch.float32, ndim=1)
+    _dev(delta, "delta", torch.float32, ndim=1)
+    _check(_lib.bnn_ternary_pack(_ptr(w), n, k, _ptr(packed), _ptr(scale), _ptr(delta), _stream(dev)),
+           "bnn_ternary_pack")
+    return packed, scale, delta
+
+
+def bnn_ternary_gemm(x: torch.Tensor, packed: torch.Tensor, scale: torch.Tensor, k: int | None = None,
+                     out: torch.Tensor | None = None) -> torch.Tensor:
+    """bf16 [m, k] x base-3 packed [n, ceil(k/10)] -> float32 [m, n] (scale applied)."""
+    _dev(x, "x", torch.bfloat16)
+    _dev(packed, "packed", torch.int16)
+    _dev(scale, "scale", torch.float32, ndim=1)
+    m, kk = x.shape
+    k = kk if k is None else k
+    if k != kk or packed.shape[1] != trit_words_per_row(k):
+        raise ValueError("packed rows must hold ceil(k/10) words")
+    n = packed.shape[0]
+    if out is None:
+        out = torch.empty((m, n), dtype=torch.float32, device=x.device)
+    _dev(out, "out", torch.float32)
+    _check(_lib.bnn_ternary_gemm(_ptr(x), _ptr(packed), _ptr(scale), m, n, k, _ptr(out), _stream(x.device)),
+           "bnn_ternary_gemm")
+    return out

@@ -1,0 +1,33 @@
+// Internal helpers shared by the libbnn CUDA sources (not part of the ABI).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "bnn.h"
+
+namespace bnn {
+
+// Records a failed CUDA call for bnn_last_cuda_error() and maps it to a status.
+bnn_status cuda_fail(cudaError_t e);
+
+inline bnn_status check_launch() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? BNN_OK : cuda_fail(e);
+}
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+__host__ __device__ inline int64_t words64(int64_t k) { return (k + 63) / 64; }
+__host__ __device__ inline int64_t words10(int64_t k) { return (k + 9) / 10; }
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+}  // namespace bnn
+
+#define BNN_TRY(expr)                              \
+  do {                                             \
+    cudaError_t bnn_e_ = (expr);                   \
+    if (bnn_e_ != cudaSuccess) return bnn::cuda_fail(bnn_e_); \
+  } while (0)

@@ -1,0 +1,84 @@
+"""The C-ABI library loads and exports every symbol include/bnn.h declares,
+and its host-side argument checks reject bad calls before any CUDA work (these
+calls never reach a kernel, so they run without a GPU)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "bnn.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bnn_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def bnn():
+    from ternary_neural_net_b200 import bnn as mod
+    return mod
+
+
+def test_header_declares_the_four_calls():
+    syms = declared_symbols()
+    for name in ("bnn_pack_signs", "bnn_binary_gemm", "bnn_ternary_pack", "bnn_ternary_gemm",
+                 "bnn_status_string", "bnn_last_cuda_error"):
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol(bnn):
+    lib = C.CDLL(bnn.LIB_PATH)
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    assert set(bnn.ABI_SYMBOLS) <= set(declared_symbols())
+
+
+def test_status_strings(bnn):
+    lib = bnn.lib()
+    for st in range(5):
+        assert lib.bnn_status_string(st)
+    assert b"INVALID" in lib.bnn_status_string(1)
+    assert b"UNKNOWN" in lib.bnn_status_string(99)
+
+
+def test_host_argument_checks(bnn):
+    lib = bnn.lib()
+    P = C.c_void_p
+    good8 = P(0x1000)
+    good2 = P(0x1002)
+    # negative sizes
+    assert lib.bnn_pack_signs(good8, -1, 5, good8, None) == bnn.BNN_ERR_INVALID_ARG
+    assert lib.bnn_binary_gemm(good8, good8, good8, 1, 1, -3, good8, good8, None) == bnn.BNN_ERR_INVALID_ARG
+    assert lib.bnn_ternary_pack(good8, -1, 3, good8, good8, good8, None) == bnn.BNN_ERR_INVALID_ARG
+    assert lib.bnn_ternary_gemm(good8, good8, good8, 1, -1, 3, good8, None) == bnn.BNN_ERR_INVALID_ARG
+    # k beyond the exact-float32 bound
+    assert lib.bnn_binary_gemm(good8, good8, good8, 1, 1, (1 << 24) + 1, good8, None, None) == bnn.BNN_ERR_INVALID_ARG
+    # no output at all / out without alpha
+    assert lib.bnn_binary_gemm(good8, good8, good8, 1, 1, 64, None, None, None) == bnn.BNN_ERR_INVALID_ARG
+    assert lib.bnn_binary_gemm(good8, good8, None, 1, 1, 64, None, good8, None) == bnn.BNN_ERR_INVALID_ARG
+    # null required pointers
+    assert lib.bnn_pack_signs(None, 2, 5, good8, None) == bnn.BNN_ERR_INVALID_ARG
+    assert lib.bnn_ternary_gemm(None, good8, good8, 1, 1, 3, good8, None) == bnn.BNN_ERR_INVALID_ARG
+    assert lib.bnn_ternary_pack(good8, 2, 3, good8, good8, None, None) == bnn.BNN_ERR_INVALID_ARG
+    # misaligned pointers
+    assert lib.bnn_pack_signs(P(0x1001), 2, 5, good8, None) == bnn.BNN_ERR_MISALIGNED
+    assert lib.bnn_pack_signs(good8, 2, 5, P(0x1004), None) == bnn.BNN_ERR_MISALIGNED
+    assert lib.bnn_binary_gemm(P(0x1004), good8, good8, 1, 1, 64, good8, None, None) == bnn.BNN_ERR_MISALIGNED
+    assert lib.bnn_ternary_gemm(P(0x1001), good2, good8, 1, 1, 3, good8, None) == bnn.BNN_ERR_MISALIGNED
+    assert lib.bnn_ternary_pack(good8, 1, 3, P(0x1001), good8, good8, None) == bnn.BNN_ERR_MISALIGNED
+    # empty problems are valid and launch nothing
+    assert lib.bnn_pack_signs(None, 0, 5, None, None) == bnn.BNN_OK
+    assert lib.bnn_pack_signs(good8, 3, 0, good8, None) == bnn.BNN_OK
+    assert lib.bnn_binary_gemm(None, None, None, 0, 5, 64, good8, None, None) == bnn.BNN_OK
+    assert lib.bnn_ternary_gemm(None, None, None, 4, 0, 10, good8, None) == bnn.BNN_OK
+
+
+def test_binding_rejects_host_tensors(bnn):
+    import torch
+    with pytest.raises(ValueError):
+        bnn.bnn_pack_signs(torch.zeros(2, 3))

@@ -1,0 +1,188 @@
+"""GPU parity of the binary path (sign-pack, XOR+popcount matmul, alpha
+epilogue) against the CPU oracle: bit-exact packing and int32 dots, bitwise
+float32 outputs.  Every call goes through the C ABI (libbnn.so) via the
+binding."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from conftest import golden_lines
+from gpu_util import assert_bits_equal, host_u64, to_dev_f32, to_dev_u64
+from ternary_neural_net_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def bnn(cuda_device):
+    from ternary_neural_net_b200 import bnn as mod
+    return mod
+
+
+def test_pack_special_values(bnn):
+    bits = []
+    vals = []
+    for line in golden_lines("sign_pack_special.txt"):
+        h, b = line.split()[:2]
+        vals.append(int(h, 16))
+        bits.append(int(b))
+    x = np.array(vals, dtype=np.uint32).view(np.float32).reshape(1, -1)
+    got = host_u64(bnn.bnn_pack_signs(to_dev_f32(x)))
+    want = sum(b << i for i, b in enumerate(bits))
+    assert int(got[0, 0]) == want
+
+
+@pytest.mark.parametrize("rows,k", [(1, 1), (3, 63), (5, 64), (7, 65), (2, 1000), (33, 4096 + 17),
+                                    (256, 4096), (1, 8192), (300, 129), (4, 2047)])
+def test_pack_matches_oracle(bnn, rows, k):
+    x = synth.normal_f32(rows * 7 + k, 1, (rows, k))
+    x[:, ::13] = 0.0
+    special = np.array([-0.0, np.nan, np.inf, -np.inf, 1e-45], np.float32)
+    x[0, :min(5, k)] = special[:min(5, k)]
+    got = host_u64(bnn.bnn_pack_signs(to_dev_f32(x)))
+    assert_bits_equal(got, oracle.pack_signs(x), f"pack {rows}x{k}")
+
+
+def test_pack_empty(bnn):
+    out = bnn.bnn_pack_signs(torch.empty((0, 100), device="cuda"))
+    assert out.shape == (0, 2)
+    out = bnn.bnn_pack_signs(torch.empty((4, 0), device="cuda"))
+    assert out.shape == (4, 0)
+
+
+def _gemm_case(bnn, m, n, k, seed, offset_words=0):
+    xp = synth.fair_coin_words(seed, 1, m, k)
+    wp = synth.fair_coin_words(seed, 2, n, k)
+    alpha = synth.uniform_f32(seed, 3, (n,), -1.0, 2.0)
+    if n > 2:
+        alpha[1] = 0.0
+    if offset_words:
+        # place the operands 8 bytes past a 16-byte boundary to exercise the 8-byte path
+        kw = synth.words_per_row(k)
+        bx = torch.zeros(m * kw + offset_words, dtype=torch.int64, device="cuda")
+        bw = torch.zeros(n * kw + offset_words, dtype=torch.int64, device="cuda")
+        bx[offset_words:] = to_dev_u64(xp).reshape(-1)
+        bw[offset_words:] = to_dev_u64(wp).reshape(-1)
+        dxp, dwp = bx[offset_words:].view(m, kw), bw[offset_words:].view(n, kw)
+    else:
+        dxp, dwp = to_dev_u64(xp), to_dev_u64(wp)
+    dots, out = bnn.bnn_binary_gemm(dxp, dwp, to_dev_f32(alpha), k)
+    torch.cuda.synchronize()
+    want_d, want_o = oracle.binary_gemm(xp, wp, alpha, m, n, k)
+    assert_bits_equal(dots.cpu().numpy(), want_d, f"dots {m}x{n}x{k}")
+    assert_bits_equal(out.cpu().numpy(), want_o, f"out {m}x{n}x{k}")
+
+
+@pytest.mark.parametrize("m", [1, 2, 3, 4, 5, 8])
+@pytest.mark.parametrize("n,k", [(1, 1), (17, 63), (130, 64), (129, 65), (1000, 1000), (64, 4096 + 64 * 3 + 5)])
+def test_skinny_matches_oracle(bnn, m, n, k):
+    _gemm_case(bnn, m, n, k, seed=m * 1000 + n + k)
+
+
+@pytest.mark.parametrize("m,n,k", [(9, 33, 64), (64, 64, 128), (130, 257, 1000), (300, 129, 4096 + 100),
+                                   (129, 1000, 63), (512, 640, 512), (17, 3, 130)])
+def test_tiled_matches_oracle(bnn, m, n, k):
+    _gemm_case(bnn, m, n, k, seed=m + 7 * n + k)
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 100, 200), (3, 50, 640), (40, 70, 128), (200, 300, 1024)])
+def test_unaligned_operands_use_the_8_byte_path(bnn, m, n, k):
+    _gemm_case(bnn, m, n, k, seed=99 + m, offset_words=1)
+
+
+def test_k_zero_gives_zero_and_alpha_times_zero(bnn):
+    for m in (1, 20):
+        xp = torch.empty((m, 0), dtype=torch.int64, device="cuda")
+        wp = torch.empty((5, 0), dtype=torch.int64, device="cuda")
+        alpha = to_dev_f32(np.array([1.0, -2.0, 0.0, 3.5, 1e-3], np.float32))
+        dots, out = bnn.bnn_binary_gemm(xp, wp, alpha, 0)
+        assert torch.all(dots == 0) and torch.all(out == 0)
+
+
+def test_dots_only_and_out_only(bnn):
+    m, n, k = 6, 40, 300
+    xp, wp = synth.fair_coin_words(5, 1, m, k), synth.fair_coin_words(5, 2, n, k)
+    alpha = synth.uniform_f32(5, 3, (n,), 0.5, 1.5)
+    want_d, want_o = oracle.binary_gemm(xp, wp, alpha, m, n, k)
+    d, o = bnn.bnn_binary_gemm(to_dev_u64(xp), to_dev_u64(wp), None, k, want_out=False)
+    assert o is None and np.array_equal(d.cpu().numpy(), want_d)
+    d, o = bnn.bnn_binary_gemm(to_dev_u64(xp), to_dev_u64(wp), to_dev_f32(alpha), k, want_dots=False)
+    assert d is None
+    assert_bits_equal(o.cpu().numpy(), want_o, "out only")
+
+
+def test_identity_special_rows(bnn):
+    """x = w gives k, x = -w gives -k, for k across word boundaries."""
+    for k in (1, 63, 64, 65, 127, 128, 129, 1000):
+        w = synth.fair_coin_words(k, 1, 2, k)
+        mask = synth.fair_coin_words(0, 0, 1, k)
+        mask[:] = np.uint64(0xFFFFFFFFFFFFFFFF)
+        kw = synth.words_per_row(k)
+        if k % 64:
+            mask[0, kw - 1] = np.uint64((1 << (k % 64)) - 1)
+        x = np.stack([w[0], w[0] ^ mask[0]])
+        dots, _ = bnn.bnn_binary_gemm(to_dev_u64(x), to_dev_u64(w[:1]), None, k, want_out=False)
+        d = dots.cpu().numpy()
+        assert d[0, 0] == k and d[1, 0] == -k
+
+
+# ---------------------------------------------------------------------------
+# The five workloads at their full sizes, in the launch configuration the bench
+# times; outputs the oracle can compute one by one are sampled.
+# ---------------------------------------------------------------------------
+def _samples(m, n, count, seed):
+    rng = np.random.default_rng(seed)
+    rows = np.concatenate([rng.integers(0, m, count), np.zeros(n, np.int64) if n <= 4096 else np.zeros(0, np.int64),
+                           np.arange(min(m, 4096))])
+    cols = np.concatenate([rng.integers(0, n, count), np.arange(n) if n <= 4096 else np.zeros(0, np.int64),
+                           np.zeros(min(m, 4096), np.int64)])
+    return rows.astype(np.int64), cols.astype(np.int64)
+
+
+def test_workload_gemv_small_full(bnn):
+    c = synth.gemv_small(1)
+    dots, out = bnn.bnn_binary_gemm(to_dev_u64(c["xp"]), to_dev_u64(c["wp"]), to_dev_f32(c["alpha"]), c["k"])
+    want_d, want_o = oracle.binary_gemm(c["xp"], c["wp"], c["alpha"], c["m"], c["n"], c["k"])
+    assert_bits_equal(dots.cpu().numpy(), want_d, "cfg1 dots")
+    assert_bits_equal(out.cpu().numpy(), want_o, "cfg1 out")
+
+
+def test_workload_gemm_fused_pack(bnn):
+    c = synth.gemm_fused_pack(1)
+    xp = bnn.bnn_pack_signs(to_dev_f32(c["x"]))
+    wp = bnn.bnn_pack_signs(to_dev_f32(c["w"]))
+    dots, out = bnn.bnn_binary_gemm(xp, wp, to_dev_f32(c["alpha"]), c["k"])
+    hx, hw = host_u64(xp), host_u64(wp)
+    assert_bits_equal(hx, oracle.pack_signs(c["x"]), "cfg2 x pack")
+    assert_bits_equal(hw, oracle.pack_signs(c["w"]), "cfg2 w pack")
+    rows, cols = _samples(c["m"], c["n"], 4096, 2)
+    sd, so = oracle.binary_gemm_sampled(hx, hw, c["alpha"], c["m"], c["n"], c["k"], rows, cols)
+    assert_bits_equal(dots.cpu().numpy()[rows, cols], sd, "cfg2 dots")
+    assert_bits_equal(out.cpu().numpy()[rows, cols], so, "cfg2 out")
+
+
+def test_workload_gemv_ffn(bnn):
+    c = synth.gemv_ffn(1)
+    xp = bnn.bnn_pack_signs(to_dev_f32(c["x"]))
+    _, out = bnn.bnn_binary_gemm(xp, to_dev_u64(c["wp"]), to_dev_f32(c["alpha"]), c["k"], want_dots=False)
+    hx = host_u64(xp)
+    assert_bits_equal(hx, oracle.pack_signs(c["x"]), "cfg3 x pack")
+    _, want_o = oracle.binary_gemm(hx, c["wp"], c["alpha"], 1, c["n"], c["k"])  # 2.3e8 MAC: full
+    assert_bits_equal(out.cpu().numpy(), want_o, "cfg3 out")
+
+
+def test_workload_gemm_large(bnn):
+    c = synth.gemm_large(1)
+    dots, out = bnn.bnn_binary_gemm(to_dev_u64(c["xp"]), to_dev_u64(c["wp"]), to_dev_f32(c["alpha"]), c["k"])
+    torch.cuda.synchronize()
+    rows, cols = _samples(c["m"], c["n"], 2048, 4)
+    sd, so = oracle.binary_gemm_sampled(c["xp"], c["wp"], c["alpha"], c["m"], c["n"], c["k"], rows, cols)
+    d = dots.cpu().numpy()
+    assert_bits_equal(d[rows, cols], sd, "cfg4 dots")
+    assert_bits_equal(out.cpu().numpy()[rows, cols], so, "cfg4 out")
+    # properties at every output: parity of k, range, and out = alpha * dot
+    k = c["k"]
+    assert np.all((d - k) % 2 == 0) and np.abs(d).max() <= k
+    o = out.cpu().numpy()
+    assert_bits_equal(o, c["alpha"][None, :] * d.astype(np.float32), "cfg4 epilogue everywhere")

@@ -1,0 +1,142 @@
+"""GPU parity of the ternary path (TWN ternarise + least-squares scale +
+base-3 pack, and the ternary matmul) against the CPU oracle.  Trits/words are
+bit-exact given the same threshold; scales within 1 ulp (float64 sums in a
+different order, rounded once); matmul outputs within 1e-3 of scale*sum|x t|."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import assert_bits_equal, assert_ternary_close, host_u16, to_dev_bf16, to_dev_f32, to_dev_u16
+from ternary_neural_net_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def bnn(cuda_device):
+    from ternary_neural_net_b200 import bnn as mod
+    return mod
+
+
+def _ulp_diff(a: np.ndarray, b: np.ndarray) -> int:
+    ia = a.astype(np.float32).view(np.int32).astype(np.int64)
+    ib = b.astype(np.float32).view(np.int32).astype(np.int64)
+    return int(np.abs(ia - ib).max()) if a.size else 0
+
+
+def _check_pack(bnn, w: np.ndarray, what: str):
+    n, k = w.shape
+    packed, scale, delta = bnn.bnn_ternary_pack(to_dev_f32(w))
+    torch.cuda.synchronize()
+    gp, gs, gd = host_u16(packed), scale.cpu().numpy(), np.float32(delta.cpu().numpy()[0])
+    od = oracle.twn_delta(w)
+    if gd != od:
+        # float64 sums in another order rounded to a different float32 Delta:
+        # compare against the oracle run at the GPU's Delta, and say how many
+        # weights lie between the two thresholds.
+        lo, hi = min(gd, od), max(gd, od)
+        between = int(((np.abs(w) > lo) & (np.abs(w) <= hi)).sum())
+        print(f"{what}: Delta differs (gpu {gd!r}, oracle {od!r}); {between} weights in between")
+        assert abs(float(gd) - float(od)) <= 2 * np.spacing(np.float32(od))
+    trits, oscale = oracle.twn_apply(w, gd)
+    assert_bits_equal(gp, oracle.base3_pack(trits), f"{what} words")
+    assert _ulp_diff(gs, oscale) <= 1, f"{what} scales"
+    return gp, gs, gd
+
+
+@pytest.mark.parametrize("n,k", [(1, 1), (3, 10), (5, 23), (2, 9), (7, 4096), (64, 1000), (300, 4096 + 7)])
+def test_pack_matches_oracle(bnn, n, k):
+    w = synth.normal_f32(n + k, 5, (n, k))
+    w[0, :3] = [0.0, -0.0, np.float32(1e-30)][: min(3, k)]
+    _check_pack(bnn, w, f"pack {n}x{k}")
+
+
+def test_pack_golden_tie_and_empty_rows(bnn):
+    w = np.array([[-7, 13, -10, 10]], np.float32)  # Delta = 7 exactly, |-7| is not > Delta
+    packed, scale, delta = bnn.bnn_ternary_pack(to_dev_f32(w))
+    t, bad = oracle.base3_unpack(host_u16(packed), 4)
+    assert bad == 0 and t.tolist() == [[0, 1, -1, 1]]
+    assert float(delta.cpu()[0]) == 7.0 and float(scale.cpu()[0]) == 11.0
+    w = np.array([[0.1, -0.1, 0.1, -0.1], [5, -5, 5, -5]], np.float32)
+    packed, scale, _ = bnn.bnn_ternary_pack(to_dev_f32(w))
+    t, _ = oracle.base3_unpack(host_u16(packed), 4)
+    assert t.tolist() == [[0, 0, 0, 0], [1, -1, 1, -1]] and scale.cpu().tolist() == [0.0, 5.0]
+    w = np.zeros((3, 11), np.float32)
+    packed, scale, delta = bnn.bnn_ternary_pack(to_dev_f32(w))
+    assert np.all(host_u16(packed)[:, 0] == 29524) and float(delta.cpu()[0]) == 0.0
+    assert torch.all(scale == 0)
+
+
+def test_pack_empty_shapes(bnn):
+    packed, scale, delta = bnn.bnn_ternary_pack(torch.empty((0, 5), device="cuda"))
+    torch.cuda.synchronize()
+    assert packed.shape == (0, 1) and float(delta.cpu()[0]) == 0.0
+    packed, scale, delta = bnn.bnn_ternary_pack(torch.empty((4, 0), device="cuda"))
+    torch.cuda.synchronize()
+    assert packed.shape == (4, 0) and torch.all(scale == 0) and float(delta.cpu()[0]) == 0.0
+
+
+def test_pack_is_reproducible(bnn):
+    w = to_dev_f32(synth.normal_f32(3, 3, (513, 777)))
+    a = [t.clone() for t in bnn.bnn_ternary_pack(w)]
+    b = bnn.bnn_ternary_pack(w)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def _gemm_case(bnn, m, n, k, seed, trits=None):
+    rng = np.random.default_rng(seed)
+    if trits is None:
+        trits = rng.integers(-1, 2, (n, k)).astype(np.int8)
+    packed = oracle.base3_pack(trits)
+    scale = synth.uniform_f32(seed, 1, (n,), 0.25, 2.0)
+    xb = synth.bf16_bits_from_f32(synth.normal_f32(seed, 2, (m, k)))
+    out = bnn.bnn_ternary_gemm(to_dev_bf16(xb), to_dev_u16(packed), to_dev_f32(scale), k)
+    ref, mag = oracle.ternary_gemm(xb, packed, scale, m, n, k)
+    return assert_ternary_close(out.cpu().numpy(), ref, mag, f"ternary {m}x{n}x{k}")
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 7, 10), (1, 100, 4096), (2, 33, 95), (4, 65, 161), (8, 64, 1000),
+                                   (1, 5, 1), (3, 9, 9)])
+def test_gemv_matches_oracle(bnn, m, n, k):
+    _gemm_case(bnn, m, n, k, seed=m * 31 + n + k)
+
+
+@pytest.mark.parametrize("m,n,k", [(9, 65, 161), (64, 64, 160), (64, 200, 4096), (100, 130, 1001),
+                                   (130, 70, 33), (65, 1, 10)])
+def test_gemm_matches_oracle(bnn, m, n, k):
+    _gemm_case(bnn, m, n, k, seed=m * 17 + n + k)
+
+
+@pytest.mark.parametrize("m", [1, 64])
+def test_every_base3_word_decodes(bnn, m):
+    """One weight row holding all 3^10 words once (k = 590490): every code goes
+    through the kernel's decoder."""
+    words = np.arange(59049, dtype=np.uint16).reshape(1, -1)
+    trits, bad = oracle.base3_unpack(words, 590490)
+    assert bad == 0
+    rows = np.concatenate([trits, -trits, np.zeros_like(trits)])
+    _gemm_case(bnn, m, 3, 590490, seed=5 + m, trits=rows)
+
+
+def test_zero_trits_give_exact_zero(bnn):
+    k = 300
+    packed = np.full((4, 30), 29524, np.uint16)
+    xb = synth.bf16_bits_from_f32(synth.normal_f32(1, 1, (3, k)))
+    for m in (1, 3):
+        out = bnn.bnn_ternary_gemm(to_dev_bf16(xb[:m]), to_dev_u16(packed), to_dev_f32(np.ones(4, np.float32)), k)
+        assert torch.all(out == 0)
+
+
+@pytest.mark.parametrize("m", [1, 64])
+def test_workload_ternary_full(bnn, m):
+    c = synth.ternary(1, m=m)
+    gp, gs, gd = _check_pack(bnn, c["w"], "cfg5 pack")
+    zero_frac = float((oracle.base3_unpack(gp, c["k"])[0] == 0).mean())
+    print(f"cfg5: Delta={gd} zero fraction={zero_frac:.4f}")
+    assert 0.40 < zero_frac < 0.45
+    out = bnn.bnn_ternary_gemm(to_dev_bf16(c["x_bf16"]), to_dev_u16(gp), to_dev_f32(gs), c["k"])
+    ref, mag = oracle.ternary_gemm(c["x_bf16"], gp, gs, m, c["n"], c["k"])
+    worst = assert_ternary_close(out.cpu().numpy(), ref, mag, f"cfg5 m={m}")
+    print(f"cfg5 m={m}: worst |err|/mag = {worst:.3e}")

@@ -186,3 +186,14 @@ def test_ternary_gemm_against_numpy(m, n, k):
     rows, cols = rng.integers(0, m, 9), rng.integers(0, n, 9)
     ys, ms = oracle.ternary_gemm_sampled(xb, oracle.base3_pack(trits), scale, m, n, k, rows, cols)
     assert np.array_equal(ys, y[rows, cols]) and np.array_equal(ms, mag[rows, cols])
+
+
+def test_twn_steps_compose():
+    w = synth.normal_f32(9, 3, (7, 45))
+    t, s, d = oracle.twn_ternarize(w)
+    assert oracle.twn_delta(w) == d
+    t2, s2 = oracle.twn_apply(w, d)
+    assert np.array_equal(t, t2) and np.array_equal(s, s2)
+    # a larger threshold can only zero more trits
+    t3, _ = oracle.twn_apply(w, np.float32(d * 2))
+    assert np.all((t3 == 0) | (t3 == t)) and (t3 == 0).sum() >= (t == 0).sum()
