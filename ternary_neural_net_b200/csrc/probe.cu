@@ -1,0 +1,49 @@
+// bnn_probe_popc: integer-pipe rate probe (measurement helper, see bnn_probe.h).
+#include "bnn_internal.cuh"
+#include "bnn_probe.h"
+
+namespace {
+
+constexpr int kChains = 8;
+
+__global__ void __launch_bounds__(256) probe_popc_kernel(int mode, int64_t iters, int32_t* __restrict__ sink) {
+  const uint32_t tid = blockIdx.x * blockDim.x + threadIdx.x;
+  uint32_t a[kChains], b[kChains];
+#pragma unroll
+  for (int c = 0; c < kChains; ++c) {
+    a[c] = tid * 2654435761u + c * 40503u;
+    b[c] = tid ^ (c * 0x9E3779B9u);
+  }
+  if (mode == 0) {
+    for (int64_t i = 0; i < iters; ++i) {
+#pragma unroll
+      for (int c = 0; c < kChains; ++c) a[c] = __popc(a[c]) + b[c] + a[c];
+    }
+  } else {
+    for (int64_t i = 0; i < iters; ++i) {
+#pragma unroll
+      for (int c = 0; c < kChains; ++c) {
+        // one 64-bit word pair: XOR both halves, popcount both, accumulate
+        const uint32_t lo = a[c] ^ b[c];
+        const uint32_t hi = a[c] ^ (b[c] + 0x5bd1e995u);
+        a[c] = a[c] + __popc(lo) + __popc(hi);
+      }
+    }
+  }
+  uint32_t r = 0;
+#pragma unroll
+  for (int c = 0; c < kChains; ++c) r ^= a[c];
+  sink[tid] = static_cast<int32_t>(r);
+}
+
+}  // namespace
+
+extern "C" bnn_status bnn_probe_popc(int mode, int64_t blocks, int64_t iters, int32_t* sink, double* ops,
+                                     cudaStream_t s) {
+  if ((mode != 0 && mode != 1) || blocks <= 0 || blocks > (1 << 22) || iters < 0 || !sink || !ops)
+    return BNN_ERR_INVALID_ARG;
+  if (!bnn::aligned(sink, 4)) return BNN_ERR_MISALIGNED;
+  *ops = static_cast<double>(blocks) * 256.0 * static_cast<double>(iters) * kChains;
+  probe_popc_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(mode, iters, sink);
+  return bnn::check_launch();
+}
