@@ -57,7 +57,9 @@ def parse_args():
     p.add_argument("--steps", type=int, default=2000)
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["bnn", "reference"], default="bnn")
-    p.add_argument("--workloads", choices=["all", "headline"], default="all")
+    p.add_argument("--workloads", default="all",
+                   help="all, or a comma list of: headline, gemv_small, gemv_ffn, gemm_large, ternary "
+                        "(without 'headline' no JSON headline is measured: for profiling runs)")
     p.add_argument("--seed", type=int, default=1)
     return p.parse_args()
 
@@ -235,36 +237,48 @@ def run_headline(cu: Cuda, args, dist: Dist):
     XP = [torch.empty((m, kw), dtype=torch.int64, device=dev) for _ in range(R)]
     D = [torch.empty((m, n), dtype=torch.int32, device=dev) for _ in range(R)]
     O = [torch.empty((m, n), dtype=torch.float32, device=dev) for _ in range(R)]
-    lib, s = cu.lib, cu.s
-    pack_args = [(C.c_void_p(X[r].data_ptr()), m, k, C.c_void_p(XP[r].data_ptr()), s) for r in range(R)]
+    lib = cu.lib
+    cap = torch.cuda.Stream(dev)
+    cs = C.c_void_p(cap.cuda_stream)
+    pack_args = [(C.c_void_p(X[r].data_ptr()), m, k, C.c_void_p(XP[r].data_ptr()), cs) for r in range(R)]
     gemm_args = [(C.c_void_p(XP[r].data_ptr()), C.c_void_p(WP[r].data_ptr()), C.c_void_p(alpha.data_ptr()),
-                  m, n, k, C.c_void_p(D[r].data_ptr()), C.c_void_p(O[r].data_ptr()), s) for r in range(R)]
+                  m, n, k, C.c_void_p(D[r].data_ptr()), C.c_void_p(O[r].data_ptr()), cs) for r in range(R)]
 
     def step(i, ev=None):
         r = i % R
         if ev:
-            ev[0].record(cu.stream)
+            ev[0].record(cap)
         st1 = lib.bnn_pack_signs(*pack_args[r])
         if ev:
-            ev[1].record(cu.stream)
+            ev[1].record(cap)
         st2 = lib.bnn_binary_gemm(*gemm_args[r])
         if ev:
-            ev[2].record(cu.stream)
+            ev[2].record(cap)
         if st1 or st2:
             cu.check(st1 or st2, "headline step")
 
-    for i in range(args.warmup):
-        step(i)
+    # W eager warm-up steps, then the K timed steps captured once into a CUDA
+    # graph (so host launch overhead cannot leave gaps between kernels), with
+    # external timing events between the kernels of every step.
+    cap.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(cap):
+        for i in range(args.warmup):
+            step(i)
+    torch.cuda.synchronize(dev)
     K = args.steps
-    evs = [cu.events(3) for _ in range(K)]
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(K)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cap):
+        for i in range(K):
+            step(args.warmup + i, evs[i])
+    g.replay()                                   # upload the graph (untimed)
     t0, t1 = cu.events(2)
     torch.cuda.synchronize(dev)
     dist.barrier(dev)
     torch.cuda.synchronize(dev)
     with ClockSampler(dev.index) as clocks:
         t0.record(cu.stream)
-        for i in range(K):
-            step(args.warmup + i, evs[i])
+        g.replay()
         t1.record(cu.stream)
         torch.cuda.synchronize(dev)
     dist.barrier(dev)
@@ -273,9 +287,14 @@ def run_headline(cu: Cuda, args, dist: Dist):
     ms = dist.max(ms_local, dev)
     pack_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
     gemm_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    del g
     macs = float(m) * n * k
     res = dict(m=m, n=n, k=k, R=R, ms_total=ms, ms_per_step=ms / K, pack_ms=pack_ms, gemm_ms=gemm_ms,
                macs=macs, clocks=clocks.summary())
+
+    # the same GEMM with the popcount kernel family (for its own roofline)
+    popc_args = [a[:-1] + (C.c_int(1), a[-1]) for a in gemm_args]
+    res["gemm_popc_ms"] = graph_time(cu, lambda i: lib.bnn_binary_gemm_algo(*popc_args[i % R]), 200, cap)
 
     # end to end through the public API: pinned host activations in, dots and outputs back to pinned host
     xh = x_host.pin_memory()
@@ -306,6 +325,34 @@ def run_headline(cu: Cuda, args, dist: Dist):
     for lst in (X, WP, XP, D, O):
         lst.clear()
     return res
+
+
+def graph_time(cu: Cuda, fn, iters: int, stream=None) -> float:
+    """ms per call of fn(i) (fn launches on `stream`), from a CUDA graph of
+    `iters` calls replayed once untimed and once between events."""
+    torch = cu.torch
+    dev = cu.device
+    stream = stream or torch.cuda.Stream(dev)
+    stream.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            st = fn(i)
+            if st:
+                cu.check(st, "warm-up")
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(iters):
+            fn(3 + i)
+    g.replay()
+    a, b = cu.events(2)
+    torch.cuda.synchronize(dev)
+    a.record(cu.stream)
+    g.replay()
+    b.record(cu.stream)
+    torch.cuda.synchronize(dev)
+    del g
+    return a.elapsed_time(b) / iters
 
 
 def popc_probe(cu: Cuda, dev):
@@ -340,6 +387,7 @@ def popc_probe(cu: Cuda, dev):
 # the other workloads (after the headline's timed region)
 # ----------------------------------------------------------------------------
 def time_calls(cu, fn, iters, warm=3):
+    """ms per call of eager launches on the current stream (host launch cost included)."""
     torch = cu.torch
     for i in range(warm):
         fn(i)
@@ -354,11 +402,29 @@ def time_calls(cu, fn, iters, warm=3):
 
 
 def run_workloads(cu: Cuda, args, peaks, popc_peak_macs):
-    torch, dev, lib, s = cu.torch, cu.device, cu.lib, cu.s
+    torch, dev, lib = cu.torch, cu.device, cu.lib
     P = lambda t: C.c_void_p(t.data_ptr()) if t is not None else None  # noqa: E731
     hbm = peaks["hbm_gbs"]
+    st = torch.cuda.Stream(dev)
+    s = C.c_void_p(st.cuda_stream)
     out = {}
 
+    want = set(args.workloads.split(",")) if args.workloads != "all" else {"gemv_small", "gemv_ffn", "gemm_large",
+                                                                           "ternary"}
+    if "gemv_small" in want:
+        out.update(wl_gemv_small(cu, args, P, st, s))
+    if "gemv_ffn" in want:
+        out.update(wl_gemv_ffn(cu, args, P, st, s, hbm))
+    if "gemm_large" in want:
+        out.update(wl_gemm_large(cu, args, P, st, s, popc_peak_macs))
+    if "ternary" in want:
+        out.update(wl_ternary(cu, args, P, st, s, hbm, peaks))
+    return out
+
+
+def wl_gemv_small(cu, args, P, st, s):
+    torch, dev, lib = cu.torch, cu.device, cu.lib
+    out = {}
     # 1. GEMV small: M=1, K=1000, N=1024 (launch-latency bound)
     c = synth.gemv_small(args.seed)
     xp = torch.from_numpy(c["xp"].view(np.int64)).to(dev)
@@ -366,22 +432,19 @@ def run_workloads(cu: Cuda, args, peaks, popc_peak_macs):
     al = torch.from_numpy(c["alpha"]).to(dev)
     d = torch.empty((1, c["n"]), dtype=torch.int32, device=dev)
     o = torch.empty((1, c["n"]), dtype=torch.float32, device=dev)
-    ms = time_calls(cu, lambda i: lib.bnn_binary_gemm(P(xp), P(wp), P(al), 1, c["n"], c["k"], P(d), P(o), s), 2000)
-    g = torch.cuda.CUDAGraph()
-    side = torch.cuda.Stream(dev)
-    with torch.cuda.stream(side):
-        gs = C.c_void_p(side.cuda_stream)
-        lib.bnn_binary_gemm(P(xp), P(wp), P(al), 1, c["n"], c["k"], P(d), P(o), gs)
-        torch.cuda.synchronize(dev)
-        with torch.cuda.graph(g, stream=side):
-            for _ in range(100):
-                lib.bnn_binary_gemm(P(xp), P(wp), P(al), 1, c["n"], c["k"], P(d), P(o),
-                                    C.c_void_p(torch.cuda.current_stream(dev).cuda_stream))
-    ms_graph = time_calls(cu, lambda i: g.replay(), 50) / 100
-    bytes1 = c["n"] * 16 * 8 + 16 * 8 + c["n"] * 12
-    out["gemv_small_m1_n1024_k1000"] = dict(us_per_call=ms * 1e3, us_per_call_graph=ms_graph * 1e3,
+    ms_eager = time_calls(cu, lambda i: lib.bnn_binary_gemm(P(xp), P(wp), P(al), 1, c["n"], c["k"], P(d), P(o),
+                                                            cu.s), 2000)
+    ms_graph = graph_time(cu, lambda i: lib.bnn_binary_gemm(P(xp), P(wp), P(al), 1, c["n"], c["k"], P(d), P(o), s),
+                          200, st)
+    bytes1 = c["n"] * 16 * 8 + 16 * 8 + c["n"] * 4 * 3
+    out["gemv_small_m1_n1024_k1000"] = dict(us_per_call_eager=ms_eager * 1e3, us_per_call_graph=ms_graph * 1e3,
                                             gbs_graph=bytes1 / (ms_graph * 1e-3) / 1e9)
-    del g
+    return out
+
+
+def wl_gemv_ffn(cu, args, P, st, s, hbm):
+    torch, dev, lib = cu.torch, cu.device, cu.lib
+    out = {}
 
     # 3. GEMV FFN: M=1, K=8192, N=28672 (HBM-bound weight stream), x packed on device
     c = synth.gemv_ffn(args.seed)
@@ -389,18 +452,20 @@ def run_workloads(cu: Cuda, args, peaks, popc_peak_macs):
     kw = synth.words_per_row(k)
     wp_bytes = n * kw * 8
     R = rotation_copies(wp_bytes)
-    WP = [torch.from_numpy(c["wp"].view(np.int64)).to(dev) for _ in range(1)]
+    WP = [torch.from_numpy(c["wp"].view(np.int64)).to(dev)]
     WP += [WP[0].clone() for _ in range(R - 1)]
     x = torch.from_numpy(c["x"]).to(dev)
     xp = torch.empty((1, kw), dtype=torch.int64, device=dev)
     al = torch.from_numpy(c["alpha"]).to(dev)
     o = torch.empty((1, n), dtype=torch.float32, device=dev)
-    ms_gemv = time_calls(cu, lambda i: lib.bnn_binary_gemm(P(xp), P(WP[i % R]), P(al), 1, n, k, None, P(o), s), 300)
+    lib.bnn_pack_signs(P(x), 1, k, P(xp), cu.s)
+    ms_gemv = graph_time(cu, lambda i: lib.bnn_binary_gemm(P(xp), P(WP[i % R]), P(al), 1, n, k, None, P(o), s),
+                         300, st)
 
     def step3(i):
-        lib.bnn_pack_signs(P(x), 1, k, P(xp), s)
-        lib.bnn_binary_gemm(P(xp), P(WP[i % R]), P(al), 1, n, k, None, P(o), s)
-    ms_step = time_calls(cu, step3, 300)
+        return lib.bnn_pack_signs(P(x), 1, k, P(xp), s) or \
+            lib.bnn_binary_gemm(P(xp), P(WP[i % R]), P(al), 1, n, k, None, P(o), s)
+    ms_step = graph_time(cu, step3, 300, st)
     alg_kernel = wp_bytes + kw * 8 + n * 4 + n * 4
     alg_step = alg_kernel + k * 4 + kw * 8
     out["gemv_ffn_m1_n28672_k8192"] = dict(
@@ -409,8 +474,14 @@ def run_workloads(cu: Cuda, args, peaks, popc_peak_macs):
         us_step=ms_step * 1e3, step_gbs=alg_step / (ms_step * 1e-3) / 1e9, rotation=R,
         gemv_traffic_bytes=traffic_for("binary_gemv", "ternary_neural_net_b200/csrc/binary_gemm.cu"))
     del WP
+    return out
 
-    # 4. GEMM large: M=N=K=8192 pre-packed (integer pipe)
+
+def wl_gemm_large(cu, args, P, st, s, popc_peak_macs):
+    torch, dev, lib = cu.torch, cu.device, cu.lib
+    out = {}
+
+    # 4. GEMM large: M=N=K=8192 pre-packed, both kernel families
     c = synth.gemm_large(args.seed)
     m, n, k = c["m"], c["n"], c["k"]
     xp = torch.from_numpy(c["xp"].view(np.int64)).to(dev)
@@ -418,13 +489,23 @@ def run_workloads(cu: Cuda, args, peaks, popc_peak_macs):
     al = torch.from_numpy(c["alpha"]).to(dev)
     d = torch.empty((m, n), dtype=torch.int32, device=dev)
     o = torch.empty((m, n), dtype=torch.float32, device=dev)
-    with ClockSampler(dev.index) as clk:
-        ms = time_calls(cu, lambda i: lib.bnn_binary_gemm(P(xp), P(wp), P(al), m, n, k, P(d), P(o), s), 10, warm=2)
     macs = float(m) * n * k
-    out["gemm_large_8192"] = dict(ms=ms, gmacs=macs / (ms * 1e-3) / 1e9,
-                                  frac_of_popc_peak=macs / (ms * 1e-3) / 1e12 / popc_peak_macs,
-                                  clocks=clk.summary())
+    res4 = {}
+    for algo, name in ((2, "mma_s8"), (1, "popc")):
+        with ClockSampler(dev.index) as clk:
+            ms = graph_time(cu, lambda i: lib.bnn_binary_gemm_algo(P(xp), P(wp), P(al), m, n, k, P(d), P(o), algo, s),
+                            10 if algo == 2 else 5, st)
+        res4[name] = dict(ms=ms, gmacs=macs / (ms * 1e-3) / 1e9, clocks=clk.summary())
+    res4["popc"]["frac_of_popc_peak"] = res4["popc"]["gmacs"] / 1e3 / popc_peak_macs
+    res4["mma_s8"]["x_popc_peak"] = res4["mma_s8"]["gmacs"] / 1e3 / popc_peak_macs
+    out["gemm_large_8192"] = res4
     del d, o, xp, wp
+    return out
+
+
+def wl_ternary(cu, args, P, st, s, hbm, peaks):
+    torch, dev, lib = cu.torch, cu.device, cu.lib
+    out = {}
 
     # 5. Ternary: TWN pack of N=11008 x K=4096 (offline), then M=1 and M=64
     c = synth.ternary(args.seed, m=64)
@@ -434,7 +515,8 @@ def run_workloads(cu: Cuda, args, peaks, popc_peak_macs):
     packed = torch.empty((n, kt), dtype=torch.int16, device=dev)
     scale = torch.empty((n,), dtype=torch.float32, device=dev)
     delta = torch.empty((1,), dtype=torch.float32, device=dev)
-    ms_pack = time_calls(cu, lambda i: lib.bnn_ternary_pack(P(w), n, k, P(packed), P(scale), P(delta), s), 5, warm=1)
+    ms_pack = time_calls(cu, lambda i: lib.bnn_ternary_pack(P(w), n, k, P(packed), P(scale), P(delta), cu.s), 5,
+                         warm=1)
     del w
     pbytes = n * kt * 2
     R = rotation_copies(pbytes)
@@ -442,8 +524,9 @@ def run_workloads(cu: Cuda, args, peaks, popc_peak_macs):
     xb = torch.from_numpy(c["x_bf16"].view(np.int16)).to(dev).view(torch.bfloat16)
     o1 = torch.empty((1, n), dtype=torch.float32, device=dev)
     o64 = torch.empty((64, n), dtype=torch.float32, device=dev)
-    ms1 = time_calls(cu, lambda i: lib.bnn_ternary_gemm(P(xb), P(PK[i % R]), P(scale), 1, n, k, P(o1), s), 300)
-    ms64 = time_calls(cu, lambda i: lib.bnn_ternary_gemm(P(xb), P(PK[i % R]), P(scale), 64, n, k, P(o64), s), 100)
+    ms1 = graph_time(cu, lambda i: lib.bnn_ternary_gemm(P(xb), P(PK[i % R]), P(scale), 1, n, k, P(o1), s), 300, st)
+    ms64 = graph_time(cu, lambda i: lib.bnn_ternary_gemm(P(xb), P(PK[i % R]), P(scale), 64, n, k, P(o64), s), 100,
+                      st)
     alg1 = pbytes + k * 2 + n * 4 + n * 4
     flops64 = 2.0 * 64 * n * k
     out["ternary_n11008_k4096"] = dict(
@@ -541,18 +624,26 @@ def main():
     cu = Cuda(torch, dev)
     peaks, peak_src = measured_peaks()
 
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    with_headline = args.workloads == "all" or "headline" in args.workloads.split(",")
+    if not with_headline:   # profiling runs of single workloads: no headline line
+        popc_peak_macs = sms * POPC32_PER_CLK_PER_SM * 32 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+        print(json.dumps({"workloads": run_workloads(cu, args, peaks, popc_peak_macs)}), flush=True)
+        dist.close()
+        return 0
     res = run_headline(cu, args, dist)
     probe = popc_probe(cu, dev)
-    sms = torch.cuda.get_device_properties(dev).multi_processor_count
     max_mhz = res["clocks"]["sm_max_mhz"] or peaks.get("sm_max_mhz", 1965.0)
     popc_peak_macs = sms * POPC32_PER_CLK_PER_SM * 32 * max_mhz * 1e6 / 1e12  # TMAC/s at max clock
-    workloads = run_workloads(cu, args, peaks, popc_peak_macs) if args.workloads == "all" else {}
+    int8_peak = 2.0 * peaks["bf16_tflops"]                                     # TOP/s (1 MAC = 2 ops)
+    workloads = run_workloads(cu, args, peaks, popc_peak_macs) if args.workloads != "headline" else {}
     torch.cuda.synchronize(dev)
 
     K, W, N = args.steps, args.warmup, dist.world
     ms_step = res["ms_per_step"]
     value = N * res["macs"] / (ms_step * 1e-3) / 1e9
-    gemm_achieved = res["macs"] / (res["gemm_ms"] * 1e-3) / 1e12
+    gemm_achieved = res["macs"] / (res["gemm_ms"] * 1e-3) / 1e12           # TMAC/s
+    popc_achieved = res["macs"] / (res["gemm_popc_ms"] * 1e-3) / 1e12
     cpu = oracle_sample_rate(args.seed, 10.0) if (dist.rank == 0 and N == 1) else None
     e2e = res["e2e"]
     line = {
@@ -565,20 +656,31 @@ def main():
                    "m": res["m"], "n": res["n"], "k": res["k"],
                    "l2": f"inputs and outputs rotate through {res['R']} copies (> 2x L2) so each step starts cold",
                    "parallelism": f"replicas x{N} (independent problems per GPU)"},
-        "roofline": {"bound": "alu", "kernel": "bnn_binary_gemm (XOR+popcount tiled)",
-                     "achieved": gemm_achieved, "peak": popc_peak_macs, "unit": "TMAC/s",
-                     "frac": gemm_achieved / popc_peak_macs,
-                     "traffic": traffic_for("binary_gemm_tiled_4x4",
-                                            "ternary_neural_net_b200/csrc/binary_gemm.cu"),
-                     "peak_basis": f"{sms} SMs x {POPC32_PER_CLK_PER_SM} popc32/clk x 32 bit-MAC x {max_mhz} MHz "
-                                   f"(max SM clock); probe measured {probe['popc32']['per_sm_per_clk']:.2f} "
-                                   f"popc32/clk/SM and {probe['word_step']['per_sm_per_clk']:.2f} word-steps/clk/SM"},
-        "kernels_ms": {"bnn_pack_signs": res["pack_ms"], "bnn_binary_gemm": res["gemm_ms"]},
+        "roofline": {"bound": "tensor", "kernel": "binary_gemm_mma_kernel (bnn_binary_gemm, m > 8: packed bits -> "
+                                                  "+-1 int8 in registers, m16n8k32 s8 MMA)",
+                     "achieved": 2 * gemm_achieved, "peak": int8_peak, "unit": "TOP/s",
+                     "frac": 2 * gemm_achieved / int8_peak,
+                     "traffic": traffic_for("binary_gemm_mma_64x64", "ternary_neural_net_b200/csrc/binary_gemm.cu"),
+                     "peak_basis": f"int8 dense tensor peak = measured bf16 {peaks['bf16_tflops']} TFLOP/s x 2 "
+                                   f"(nominal int8:bf16 ratio 4.5:2.25 PFLOP/s), {peak_src}"},
+        "roofline_popc": {"bound": "alu", "kernel": "binary_gemm_tiled_kernel (bnn_binary_gemm_algo POPC)",
+                          "achieved": popc_achieved, "peak": popc_peak_macs, "unit": "TMAC/s",
+                          "frac": popc_achieved / popc_peak_macs,
+                          "traffic": traffic_for("binary_gemm_tiled_4x4",
+                                                 "ternary_neural_net_b200/csrc/binary_gemm.cu"),
+                          "peak_basis": f"{sms} SMs x {POPC32_PER_CLK_PER_SM} popc32/clk x 32 bit-MAC x {max_mhz} MHz "
+                                        f"(max SM clock); probe measured {probe['popc32']['per_sm_per_clk']:.2f} "
+                                        f"popc32/clk/SM and {probe['word_step']['per_sm_per_clk']:.2f} "
+                                        f"word-steps/clk/SM"},
+        "kernels_ms": {"bnn_pack_signs": res["pack_ms"], "bnn_binary_gemm": res["gemm_ms"],
+                       "bnn_binary_gemm_algo(POPC)": res["gemm_popc_ms"]},
         "cpu_baseline": cpu,
         "e2e": {"value": N * res["macs"] / (e2e["ms_per_step"] * 1e-3) / 1e9, "unit": "GMAC/s",
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                 "ms_per_step": e2e["ms_per_step"]},
         "gpu_launches": 2 * K,
+        "timing": "K steps captured in one CUDA graph (external events between kernels), replayed once untimed "
+                  "to upload, then once between events",
         "clocks": res["clocks"],
         "peaks": {"source": peak_src, "hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"]},
         "popc_probe": probe,

@@ -101,6 +101,26 @@ bnn_status bnn_binary_gemm(const uint64_t* xp, const uint64_t* wp, const float* 
                            int64_t m, int64_t n, int64_t k, int32_t* dots, float* out,
                            cudaStream_t s);
 
+/* Kernel family for bnn_binary_gemm_algo.  All give bit-identical results. */
+typedef enum {
+  BNN_ALGO_AUTO = 0,   /* what bnn_binary_gemm uses: POPC GEMV for m <= 8, MMA_S8 otherwise */
+  BNN_ALGO_POPC = 1,   /* XOR + 64-bit popcount on the integer pipe (skinny GEMV for m <= 8,
+                          register-tiled GEMM otherwise) */
+  BNN_ALGO_MMA_S8 = 2  /* packed bits expanded in registers to +-1 int8 and summed exactly by
+                          m16n8k32 s8 tensor-core MMAs into int32 */
+} bnn_binary_algo;
+
+/*
+ * bnn_binary_gemm_algo -- bnn_binary_gemm with an explicit kernel family
+ * (same arguments, outputs and errors; BNN_ERR_INVALID_ARG for an unknown
+ * algo).  The identity it evaluates is the same in every family: the MMA
+ * family sums the +-1 products directly, which equals k - 2*popcount(x XOR w)
+ * exactly.
+ */
+bnn_status bnn_binary_gemm_algo(const uint64_t* xp, const uint64_t* wp, const float* alpha,
+                                int64_t m, int64_t n, int64_t k, int32_t* dots, float* out,
+                                bnn_binary_algo algo, cudaStream_t s);
+
 /*
  * bnn_ternary_pack -- TWN ternarisation, least-squares per-row scale and base-3
  * packing of a float32 weight matrix.  [BTE] "Features".

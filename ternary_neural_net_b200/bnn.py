@@ -33,6 +33,7 @@ _vp, _i64, _int = C.c_void_p, C.c_int64, C.c_int
 _SIGS = {
     "bnn_pack_signs": [_vp, _i64, _i64, _vp, _vp],
     "bnn_binary_gemm": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp],
+    "bnn_binary_gemm_algo": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _int, _vp],
     "bnn_ternary_pack": [_vp, _i64, _i64, _vp, _vp, _vp, _vp],
     "bnn_ternary_gemm": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
 }
@@ -49,6 +50,7 @@ _lib.bnn_last_cuda_error.restype = _int
 ABI_SYMBOLS = tuple(_SIGS) + ("bnn_status_string", "bnn_last_cuda_error")
 
 BNN_OK, BNN_ERR_INVALID_ARG, BNN_ERR_MISALIGNED, BNN_ERR_CUDA, BNN_ERR_UNSUPPORTED = range(5)
+ALGO_AUTO, ALGO_POPC, ALGO_MMA_S8 = 0, 1, 2
 MAX_K_BINARY = 1 << 24
 
 
@@ -115,8 +117,9 @@ def bnn_pack_signs(x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Te
 
 def bnn_binary_gemm(xp: torch.Tensor, wp: torch.Tensor, alpha: torch.Tensor | None, k: int,
                     want_dots: bool = True, want_out: bool = True,
-                    dots: torch.Tensor | None = None, out: torch.Tensor | None = None):
-    """Packed XOR+popcount matmul.  Returns (dots int32 [m,n] or None, out float32 [m,n] or None)."""
+                    dots: torch.Tensor | None = None, out: torch.Tensor | None = None, algo: int = ALGO_AUTO):
+    """Packed XOR+popcount matmul.  Returns (dots int32 [m,n] or None, out float32 [m,n] or None).
+    `algo` selects the kernel family (ALGO_AUTO, ALGO_POPC, ALGO_MMA_S8); all are bit-identical."""
     _dev(xp, "xp", torch.int64)
     _dev(wp, "wp", torch.int64)
     m, n = xp.shape[0], wp.shape[0]
@@ -132,8 +135,12 @@ def bnn_binary_gemm(xp: torch.Tensor, wp: torch.Tensor, alpha: torch.Tensor | No
     if out is not None:
         _dev(out, "out", torch.float32)
         _dev(alpha, "alpha", torch.float32, ndim=1)
-    _check(_lib.bnn_binary_gemm(_ptr(xp), _ptr(wp), _ptr(alpha), m, n, k, _ptr(dots), _ptr(out),
-                                _stream(dev)), "bnn_binary_gemm")
+    if algo == ALGO_AUTO:
+        st = _lib.bnn_binary_gemm(_ptr(xp), _ptr(wp), _ptr(alpha), m, n, k, _ptr(dots), _ptr(out), _stream(dev))
+    else:
+        st = _lib.bnn_binary_gemm_algo(_ptr(xp), _ptr(wp), _ptr(alpha), m, n, k, _ptr(dots), _ptr(out),
+                                       int(algo), _stream(dev))
+    _check(st, "bnn_binary_gemm")
     return dots, out
 
 

@@ -6,7 +6,7 @@
 // gives 0, alpha = 0 gives 0.  "Architecture Decision Record", "Decision":
 // binary_gemm_u64 over uint64 words.
 //
-// Two kernels:
+// Three kernels:
 //  * skinny (m <= 8): batch-1 GEMV shapes are HBM-bound on the weight stream.
 //    A group of LPR lanes owns one weight row, reads it with 16-byte loads
 //    (8-byte when the rows are not 16-byte aligned), XORs it with the
@@ -19,6 +19,19 @@
 //    tiles of BK words per row staged through shared memory with cp.async in a
 //    STAGES-deep ring (rows padded to an odd multiple of 16 bytes), int32
 //    accumulators, fused k - 2d and alpha epilogue.
+//  * int8 tensor-core (m > 8, the default there): the same packed words are
+//    staged through shared memory, and each thread expands the bits it needs
+//    straight into the registers of an m16n8k32 s8 MMA fragment as 0/-1 bytes
+//    (one shift and one sign-replicating byte permute per 4 values); the MMA
+//    sums popc(a AND b) exactly in int32 on the tensor cores and the epilogue
+//    forms <x,w> = k - 2 popc(a) - 2 popc(b) + 4 popc(a AND b).
+//    On B200 the s8 mma.sync path issues 3.7x the popcount rate of the
+//    integer pipe, while the b1 XOR-popcount MMA issues below it.  Because the
+//    dot product is a sum over k, any fixed bijection between the 32 bits of a
+//    word and the 32 k-slots of the MMA gives the same result as long as both
+//    operands use it; the one used here lets each thread build its fragment
+//    bytes from byte-aligned sign bits.  Pad bits and zero-filled tail words
+//    are 0 in both operands and add nothing to any count.
 #include "bnn_internal.cuh"
 
 namespace {
@@ -261,17 +274,271 @@ bnn_status launch_tiled(const uint64_t* xp, const uint64_t* wp, const float* alp
   if (gx > 2147483647LL || gy > 65535) return BNN_ERR_INVALID_ARG;
   const size_t smem = static_cast<size_t>(kStages) * (BM + BN) * kPitch * sizeof(uint64_t);
   auto kern = binary_gemm_tiled_kernel<TM, TN, VEC>;
-  BNN_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
+  BNN_TRY(bnn::ensure_smem(kern, smem));
   kern<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), 256, smem, s>>>(xp, wp, alpha, m, n, k, kw, dots, out);
   return bnn::check_launch();
 }
 
+
+// ---------------------------------------------------------------------------
+// int8 tensor-core kernel
+// ---------------------------------------------------------------------------
+constexpr int kMBKW = 4;               // uint64 words per stage per row (256 bits = 8 k32 steps)
+constexpr int kMPitch = 6;             // 48-byte rows: 8 consecutive rows hit distinct 16-byte slots
+constexpr int kMStages = 4;
+
+// Bytes j of the result are -1 (0xFF) where bit 8j+7-s of w is set, else 0;
+// mul = 2^s.  The shift is a multiply so that it issues on the FMA pipe and
+// leaves the integer pipe to the byte permute.
+__device__ __forceinline__ uint32_t expand_neg(uint32_t w, uint32_t mul) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %1, 0xBA98;\n" : "=r"(r) : "r"(w * mul));
+  return r;
+}
+
+__device__ __forceinline__ void mma_s8_16832(int* c, const uint32_t* a, const uint32_t* b) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// CTA = WARPS_M x WARPS_N warps; each warp owns WM m16 tiles x WN n8 tiles.
+//
+// With sign bits a (activation) and b (weight), x = 1 - 2a and w = 1 - 2b, so
+//   <x, w> = k - 2 popc(a) - 2 popc(b) + 4 popc(a AND b).
+// The MMA operands are the bytes -a and -b (0 or -1: one shift and one
+// sign-replicating byte permute per 4 values), whose products sum to
+// popc(a AND b) exactly; the row popcounts are accumulated on the side from
+// the same shared-memory words by one lane per row.  Zero bits (pad bits,
+// zero-filled tail words and rows) add nothing to any of the three counts.
+// KSPLIT groups of WARPS_M x WARPS_N warps split the words of every stage
+// between them (more warps per SM for the same tile); their partial counts
+// are added through shared memory before the epilogue.
+template <int WM, int WN, int WARPS_M, int WARPS_N, int KSPLIT, int VEC, int MINB>
+__global__ void __launch_bounds__(WARPS_M * WARPS_N * KSPLIT * 32, MINB)
+binary_gemm_mma_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restrict__ wp,
+                       const float* __restrict__ alpha, int64_t m, int64_t n, int k, int kw,
+                       int32_t* __restrict__ dots, float* __restrict__ out) {
+  constexpr int THREADS = WARPS_M * WARPS_N * KSPLIT * 32;
+  constexpr int GROUP = WARPS_M * WARPS_N * 32;         // threads per K group
+  constexpr int BM = 16 * WM * WARPS_M;
+  constexpr int BN = 8 * WN * WARPS_N;
+  constexpr int CH = kMBKW / VEC;                       // copy chunks per row per stage
+  static_assert(kMBKW % KSPLIT == 0, "KSPLIT must divide the words per stage");
+  extern __shared__ __align__(16) uint64_t smem[];
+  uint64_t* As = smem;                                  // [kMStages][BM][kMPitch]
+  uint64_t* Bs = smem + kMStages * BM * kMPitch;        // [kMStages][BN][kMPitch]
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = (tid % GROUP) >> 5;
+  const int kg = tid / GROUP;                           // K group of this thread
+  const int gid = lane >> 2, tq = lane & 3;
+  const int wm = warp % WARPS_M, wn = warp / WARPS_M;
+  const int64_t m0 = static_cast<int64_t>(blockIdx.y) * BM;
+  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * BN;
+  const int ktiles = (kw + kMBKW - 1) / kMBKW;
+  const uint32_t s0 = 1u << (2 * tq), s1 = 2u << (2 * tq);
+  const bool count_a = (wn == 0) && (tq == 0);   // one lane per activation row and K group
+  const bool count_b = (wm == 0) && (tq == 0);   // one lane per weight row and K group
+
+  auto load_stage = [&](int stage, int kt) {
+    const int kbase = kt * kMBKW;
+    for (int c = tid; c < BM * CH; c += THREADS) {
+      const int row = c / CH, col = (c % CH) * VEC;
+      const int64_t gm = m0 + row;
+      const bool valid = gm < m && kbase + col < kw;
+      const uint64_t* src = valid ? xp + gm * kw + kbase + col : xp;
+      uint64_t* dst = As + (stage * BM + row) * kMPitch + col;
+      if constexpr (VEC == 2) cp_async_16(dst, src, valid); else cp_async_8(dst, src, valid);
+    }
+    for (int c = tid; c < BN * CH; c += THREADS) {
+      const int row = c / CH, col = (c % CH) * VEC;
+      const int64_t gn = n0 + row;
+      const bool valid = gn < n && kbase + col < kw;
+      const uint64_t* src = valid ? wp + gn * kw + kbase + col : wp;
+      uint64_t* dst = Bs + (stage * BN + row) * kMPitch + col;
+      if constexpr (VEC == 2) cp_async_16(dst, src, valid); else cp_async_8(dst, src, valid);
+    }
+  };
+
+  int acc[WM][WN][4];
+#pragma unroll
+  for (int i = 0; i < WM; ++i)
+#pragma unroll
+    for (int j = 0; j < WN; ++j)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[i][j][c] = 0;
+  int pa[WM][2], pb[WN];
+#pragma unroll
+  for (int i = 0; i < WM; ++i) pa[i][0] = pa[i][1] = 0;
+#pragma unroll
+  for (int j = 0; j < WN; ++j) pb[j] = 0;
+
+#pragma unroll
+  for (int st = 0; st < kMStages - 1; ++st) {
+    if (st < ktiles) load_stage(st, st);
+    cp_async_commit();
+  }
+
+  for (int kt = 0; kt < ktiles; ++kt) {
+    cp_async_wait<kMStages - 2>();
+    __syncthreads();
+    const int stage = kt % kMStages;
+    const uint64_t* A = As + (stage * BM + wm * 16 * WM + gid) * kMPitch;
+    const uint64_t* B = Bs + (stage * BN + wn * 8 * WN + gid) * kMPitch;
+#pragma unroll
+    for (int kq = 0; kq < kMBKW / KSPLIT; ++kq) {
+      const int kk = kq * KSPLIT + kg;
+      // one uint64 word = two k32 MMA steps
+      uint2 aw[WM][2], bw[WN];
+#pragma unroll
+      for (int i = 0; i < WM; ++i) {
+        aw[i][0] = *reinterpret_cast<const uint2*>(A + (16 * i) * kMPitch + kk);
+        aw[i][1] = *reinterpret_cast<const uint2*>(A + (16 * i + 8) * kMPitch + kk);
+      }
+#pragma unroll
+      for (int j = 0; j < WN; ++j) bw[j] = *reinterpret_cast<const uint2*>(B + (8 * j) * kMPitch + kk);
+      if (count_a) {
+#pragma unroll
+        for (int i = 0; i < WM; ++i)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) pa[i][h] += __popc(aw[i][h].x) + __popc(aw[i][h].y);
+      }
+      if (count_b) {
+#pragma unroll
+        for (int j = 0; j < WN; ++j) pb[j] += __popc(bw[j].x) + __popc(bw[j].y);
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t bf[WN][2];
+#pragma unroll
+        for (int j = 0; j < WN; ++j) {
+          const uint32_t w = h ? bw[j].y : bw[j].x;
+          bf[j][0] = expand_neg(w, s0);
+          bf[j][1] = expand_neg(w, s1);
+        }
+#pragma unroll
+        for (int i = 0; i < WM; ++i) {
+          const uint32_t w0 = h ? aw[i][0].y : aw[i][0].x;
+          const uint32_t w1 = h ? aw[i][1].y : aw[i][1].x;
+          const uint32_t af[4] = {expand_neg(w0, s0), expand_neg(w1, s0), expand_neg(w0, s1),
+                                  expand_neg(w1, s1)};
+#pragma unroll
+          for (int j = 0; j < WN; ++j) mma_s8_16832(acc[i][j], af, bf[j]);
+        }
+      }
+    }
+    const int next = kt + kMStages - 1;
+    if (next < ktiles) load_stage(next % kMStages, next);
+    cp_async_commit();
+  }
+  cp_async_wait<0>();
+  __syncthreads();  // every warp is done with the operand tiles: reuse the space
+
+  if constexpr (KSPLIT > 1) {
+    // groups 1.. hand their partial AND-counts to group 0 (fixed order: exact integers anyway)
+    int* xs = reinterpret_cast<int*>(smem);  // [KSPLIT-1][GROUP][WM*WN*4]
+    constexpr int PER = WM * WN * 4;
+    if (kg > 0) {
+      int* dst = xs + ((kg - 1) * GROUP + (tid % GROUP)) * PER;
+#pragma unroll
+      for (int i = 0; i < WM; ++i)
+#pragma unroll
+        for (int j = 0; j < WN; ++j)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) dst[(i * WN + j) * 4 + c] = acc[i][j][c];
+    }
+    __syncthreads();
+    if (kg == 0) {
+      for (int g = 1; g < KSPLIT; ++g) {
+        const int* src = xs + ((g - 1) * GROUP + tid) * PER;
+#pragma unroll
+        for (int i = 0; i < WM; ++i)
+#pragma unroll
+          for (int j = 0; j < WN; ++j)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[i][j][c] += src[(i * WN + j) * 4 + c];
+      }
+    }
+    __syncthreads();
+  }
+
+  int* pa_s = reinterpret_cast<int*>(smem);  // [BM]
+  int* pb_s = pa_s + BM;                      // [BN]
+  for (int i = tid; i < BM + BN; i += THREADS) pa_s[i] = 0;
+  __syncthreads();
+  if (count_a) {
+#pragma unroll
+    for (int i = 0; i < WM; ++i)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) atomicAdd(&pa_s[wm * 16 * WM + 16 * i + 8 * h + gid], pa[i][h]);
+  }
+  if (count_b) {
+#pragma unroll
+    for (int j = 0; j < WN; ++j) atomicAdd(&pb_s[wn * 8 * WN + 8 * j + gid], pb[j]);
+  }
+  __syncthreads();
+  if (kg != 0) return;
+
+#pragma unroll
+  for (int i = 0; i < WM; ++i) {
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const int lr = wm * 16 * WM + 16 * i + gid + 8 * hr;
+      const int64_t gm = m0 + lr;
+      if (gm >= m) continue;
+      const int base = k - 2 * pa_s[lr];
+#pragma unroll
+      for (int j = 0; j < WN; ++j) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int lc = wn * 8 * WN + 8 * j + 2 * tq + c;
+          const int64_t gn = n0 + lc;
+          if (gn >= n) continue;
+          const int32_t d = base - 2 * pb_s[lc] + 4 * acc[i][j][2 * hr + c];
+          if (dots) dots[gm * n + gn] = d;
+          if (out) out[gm * n + gn] = __ldg(alpha + gn) * static_cast<float>(d);
+        }
+      }
+    }
+  }
+}
+
+template <int WM, int WN, int WARPS_M, int WARPS_N, int KSPLIT, int VEC, int MINB>
+bnn_status launch_mma(const uint64_t* xp, const uint64_t* wp, const float* alpha, int64_t m, int64_t n,
+                      int k, int kw, int32_t* dots, float* out, cudaStream_t s) {
+  constexpr int BM = 16 * WM * WARPS_M, BN = 8 * WN * WARPS_N;
+  const int64_t gx = (n + BN - 1) / BN, gy = (m + BM - 1) / BM;
+  if (gx > 2147483647LL || gy > 65535) return BNN_ERR_INVALID_ARG;
+  constexpr int THREADS = WARPS_M * WARPS_N * KSPLIT * 32;
+  const size_t tiles = static_cast<size_t>(kMStages) * (BM + BN) * kMPitch * sizeof(uint64_t);
+  const size_t xchg = static_cast<size_t>(KSPLIT - 1) * WARPS_M * WARPS_N * 32 * WM * WN * 4 * sizeof(int);
+  const size_t smem = tiles > xchg ? tiles : xchg;
+  auto kern = binary_gemm_mma_kernel<WM, WN, WARPS_M, WARPS_N, KSPLIT, VEC, MINB>;
+  BNN_TRY(bnn::ensure_smem(kern, smem));
+  kern<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), THREADS, smem, s>>>(
+      xp, wp, alpha, m, n, k, kw, dots, out);
+  return bnn::check_launch();
+}
+
+template <int VEC>
+bnn_status dispatch_mma(const uint64_t* xp, const uint64_t* wp, const float* alpha, int64_t m, int64_t n,
+                        int k, int kw, int32_t* dots, float* out, cudaStream_t s) {
+  const int64_t big_tiles = ((m + 127) / 128) * ((n + 127) / 128);
+  if (big_tiles >= 2LL * bnn::sm_count())
+    return launch_mma<4, 4, 2, 4, 1, VEC, 1>(xp, wp, alpha, m, n, k, kw, dots, out, s);  // 128 x 128, 8 warps
+  return launch_mma<2, 4, 2, 2, 2, VEC, 2>(xp, wp, alpha, m, n, k, kw, dots, out, s);    // 64 x 64, 2 x 4 warps
+}
+
 }  // namespace
 
-extern "C" bnn_status bnn_binary_gemm(const uint64_t* xp, const uint64_t* wp, const float* alpha,
-                                      int64_t m, int64_t n, int64_t k, int32_t* dots, float* out,
-                                      cudaStream_t s) {
+extern "C" bnn_status bnn_binary_gemm_algo(const uint64_t* xp, const uint64_t* wp, const float* alpha,
+                                           int64_t m, int64_t n, int64_t k, int32_t* dots, float* out,
+                                           bnn_binary_algo algo, cudaStream_t s) {
   if (m < 0 || n < 0 || k < 0 || k > BNN_MAX_K_BINARY) return BNN_ERR_INVALID_ARG;
+  if (algo != BNN_ALGO_AUTO && algo != BNN_ALGO_POPC && algo != BNN_ALGO_MMA_S8) return BNN_ERR_INVALID_ARG;
   if (!dots && !out) return BNN_ERR_INVALID_ARG;
   if (out && !alpha) return BNN_ERR_INVALID_ARG;
   if (m == 0 || n == 0) return BNN_OK;
@@ -284,6 +551,10 @@ extern "C" bnn_status bnn_binary_gemm(const uint64_t* xp, const uint64_t* wp, co
   const bool vec2 = (kw % 2 == 0) && bnn::aligned(xp, 16) && bnn::aligned(wp, 16);
   const int ki = static_cast<int>(k);
 
+  if (algo == BNN_ALGO_MMA_S8 || (algo == BNN_ALGO_AUTO && m > 8)) {
+    return vec2 ? dispatch_mma<2>(xp, wp, alpha, m, n, ki, kw, dots, out, s)
+                : dispatch_mma<1>(xp, wp, alpha, m, n, ki, kw, dots, out, s);
+  }
   if (m <= 8) {
     if (vec2) dispatch_gemv<2>(xp, wp, alpha, static_cast<int>(m), n, ki, kw, dots, out, s);
     else dispatch_gemv<1>(xp, wp, alpha, static_cast<int>(m), n, ki, kw, dots, out, s);
@@ -298,4 +569,10 @@ extern "C" bnn_status bnn_binary_gemm(const uint64_t* xp, const uint64_t* wp, co
   }
   return vec2 ? launch_tiled<4, 4, 2>(xp, wp, alpha, m, n, ki, kw, dots, out, s)
               : launch_tiled<4, 4, 1>(xp, wp, alpha, m, n, ki, kw, dots, out, s);
+}
+
+extern "C" bnn_status bnn_binary_gemm(const uint64_t* xp, const uint64_t* wp, const float* alpha,
+                                      int64_t m, int64_t n, int64_t k, int32_t* dots, float* out,
+                                      cudaStream_t s) {
+  return bnn_binary_gemm_algo(xp, wp, alpha, m, n, k, dots, out, BNN_ALGO_AUTO, s);
 }

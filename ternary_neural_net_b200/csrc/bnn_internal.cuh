@@ -24,6 +24,23 @@ __host__ __device__ inline int64_t words10(int64_t k) { return (k + 9) / 10; }
 // Number of SMs of the current device (cached per device).
 int sm_count();
 
+// Current device index (0 if the query fails).
+int current_device();
+
+// Raises a kernel's dynamic shared-memory limit to `bytes` once per device and
+// process, so that later calls (including calls made while a stream is being
+// captured into a CUDA graph) only launch.
+template <typename Kernel>
+cudaError_t ensure_smem(Kernel kern, size_t bytes) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  static size_t done[64] = {0};
+  const int dev = current_device();
+  if (dev >= 0 && dev < 64 && done[dev] >= bytes) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = bytes;
+  return e;
+}
+
 }  // namespace bnn
 
 #define BNN_TRY(expr)                              \

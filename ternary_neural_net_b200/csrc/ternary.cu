@@ -169,6 +169,130 @@ ternary_gemv_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Ternary GEMV, m = 1: activation pair tables + base-9 digits.
+//
+// Each base-9 digit v of a word (v = d_{2q} + 3 d_{2q+1}, q = 0..4) covers two
+// consecutive trits, so for the activation pair (x_{2P}, x_{2P+1}) at pair
+// index P = 5j + q a 9-entry table T_P[v] = x_{2P} (v mod 3 - 1) + x_{2P+1}
+// (v div 3 - 1) turns two multiply-adds into one shared-memory load and one
+// add.  The digit is the high word of 9F and the next fraction its low word
+// (taken with __umulhi and a 32-bit multiply).
+// Lanes of a half-warp own 16 consecutive weight rows and walk the same word
+// index, so the 16 lanes read within one 9-entry table (at most 9 distinct
+// addresses, one per bank: no bank conflicts); the two half-warps work on
+// K-slices whose tables sit in disjoint banks.  The 16-row chunk of packed
+// words is contiguous in memory and is brought into shared memory with
+// 16-byte cp.async (double-buffered across the chunks this CTA owns); the
+// per-slice partial sums are added in a fixed order, then scaled once.  The
+// chunk copies run kLutStages - 1 chunks ahead of the compute (the copy
+// latency from HBM is several times one chunk's compute).
+// ---------------------------------------------------------------------------
+constexpr int kLutRows = 16;
+constexpr int kLutStages = 4;
+
+template <int SLICES>
+__global__ void __launch_bounds__(kLutRows * SLICES, 1)
+ternary_gemv_lut_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ packed,
+                        const float* __restrict__ scale, int64_t n, int k, int kt, int slice_words,
+                        float* __restrict__ out) {
+  constexpr int THREADS = kLutRows * SLICES;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int npairs = 5 * kt;
+  float* T = reinterpret_cast<float*>(smem_raw);                                   // [npairs][9]
+  const size_t t_bytes = (static_cast<size_t>(npairs) * 9 * sizeof(float) + 15) & ~static_cast<size_t>(15);
+  const size_t chunk_bytes = (static_cast<size_t>(kLutRows) * kt * 2 + 15) & ~static_cast<size_t>(15);
+  uint16_t* const buf0 = reinterpret_cast<uint16_t*>(smem_raw + t_bytes);         // [kLutStages][chunk]
+  const size_t chunk_elems = chunk_bytes / 2;
+  float* red = reinterpret_cast<float*>(smem_raw + t_bytes + kLutStages * chunk_bytes);  // [SLICES][kLutRows]
+
+  const int tid = threadIdx.x;
+  const int64_t nchunks = (n + kLutRows - 1) / kLutRows;
+
+  auto issue_chunk = [&](int64_t c, uint16_t* dst) {
+    const int64_t rows = n - c * kLutRows < kLutRows ? n - c * kLutRows : kLutRows;
+    const int64_t bytes = rows * kt * 2;
+    const unsigned char* src = reinterpret_cast<const unsigned char*>(packed + c * kLutRows * kt);
+    for (int64_t off = static_cast<int64_t>(tid) * 16; off < bytes; off += THREADS * 16) {
+      const int64_t left = bytes - off;
+      const int sz = left < 16 ? static_cast<int>(left) : 16;
+      const unsigned saddr = static_cast<unsigned>(__cvta_generic_to_shared(reinterpret_cast<unsigned char*>(dst) + off));
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(saddr), "l"(src + off), "r"(sz));
+    }
+  };
+
+  // Prefetch the first kLutStages - 1 chunks of this CTA (one commit group each).
+#pragma unroll
+  for (int st = 0; st < kLutStages - 1; ++st) {
+    const int64_t cc = blockIdx.x + static_cast<int64_t>(st) * gridDim.x;
+    if (cc < nchunks) issue_chunk(cc, buf0 + st * chunk_elems);
+    asm volatile("cp.async.commit_group;\n" ::);
+  }
+  int64_t c = blockIdx.x;
+
+  // Pair tables from the activation row (exact products, one rounding per entry).
+  for (int p = tid; p < npairs; p += THREADS) {
+    const float x0 = 2 * p < k ? __uint_as_float(static_cast<uint32_t>(__ldg(x + 2 * p)) << 16) : 0.0f;
+    const float x1 = 2 * p + 1 < k ? __uint_as_float(static_cast<uint32_t>(__ldg(x + 2 * p + 1)) << 16) : 0.0f;
+#pragma unroll
+    for (int v = 0; v < 9; ++v)
+      T[p * 9 + v] = x0 * static_cast<float>(v % 3 - 1) + x1 * static_cast<float>(v / 3 - 1);
+  }
+
+  const int row = tid % kLutRows;
+  const int sl = tid / kLutRows;
+  const int j0 = sl * slice_words;
+  const int j1 = j0 + slice_words < kt ? j0 + slice_words : kt;
+
+  for (int it = 0; c < nchunks; c += gridDim.x, ++it) {
+    // chunk `it` was the (it+1)-th commit group: allow the kLutStages-2 newer ones to be pending
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(kLutStages - 2));
+    __syncthreads();
+
+    const uint16_t* rowp = buf0 + (it % kLutStages) * chunk_elems + row * kt;
+    float acc0 = 0.0f, acc1 = 0.0f;
+#pragma unroll 2
+    for (int j = j0; j < j1; ++j) {
+      uint32_t F = static_cast<uint32_t>(rowp[j]) * kFixMul;
+      const float* Tj = T + (5 * j) * 9;
+#pragma unroll
+      for (int q = 4; q >= 0; --q) {
+        // high and low words of 9F: the digit and the next fraction
+        const uint32_t v = __umulhi(F, 9u);
+        F *= 9u;
+        if (q & 1) acc1 += Tj[q * 9 + v]; else acc0 += Tj[q * 9 + v];
+      }
+    }
+    red[sl * kLutRows + row] = acc0 + acc1;
+    __syncthreads();
+    if (tid < kLutRows) {
+      const int64_t r = c * kLutRows + tid;
+      if (r < n) {
+        float s = 0.0f;
+#pragma unroll 4
+        for (int q = 0; q < SLICES; ++q) s += red[q * kLutRows + tid];
+        out[r] = __ldg(scale + r) * s;
+      }
+    }
+    // The buffer of chunk it + kLutStages - 1 (the one computed in the previous
+    // iteration) and red are rewritten only after this barrier.
+    __syncthreads();
+    const int64_t cn = c + static_cast<int64_t>(kLutStages - 1) * gridDim.x;
+    if (cn < nchunks) issue_chunk(cn, buf0 + ((it + kLutStages - 1) % kLutStages) * chunk_elems);
+    asm volatile("cp.async.commit_group;\n" ::);
+  }
+  asm volatile("cp.async.wait_group 0;\n" ::);
+}
+
+constexpr int kLutSlices = 32;
+
+size_t lut_smem_bytes(int64_t kt) {
+  const size_t t_bytes = (static_cast<size_t>(5 * kt) * 9 * sizeof(float) + 15) & ~static_cast<size_t>(15);
+  const size_t chunk_bytes = (static_cast<size_t>(kLutRows) * kt * 2 + 15) & ~static_cast<size_t>(15);
+  return t_bytes + kLutStages * chunk_bytes + static_cast<size_t>(kLutSlices) * kLutRows * sizeof(float);
+}
+
 // ---------------------------------------------------------------------------
 // Ternary GEMM (m > 8): decode trits to bf16 tiles in shared memory, bf16
 // mma.sync m16n8k16 with fp32 accumulation.
@@ -331,6 +455,17 @@ extern "C" bnn_status bnn_ternary_gemm(const uint16_t* x_bf16, const uint16_t* p
       !bnn::aligned(out, 4))
     return BNN_ERR_MISALIGNED;
   const int64_t kt = bnn::words10(k);
+  if (m == 1 && kt > 0 && bnn::aligned(packed, 16) && lut_smem_bytes(kt) <= 200 * 1024) {
+    const size_t smem = lut_smem_bytes(kt);
+    auto kern = ternary_gemv_lut_kernel<kLutSlices>;
+    BNN_TRY(bnn::ensure_smem(kern, smem));
+    int slice_words = static_cast<int>((kt + kLutSlices - 1) / kLutSlices);
+    const int64_t nchunks = (n + kLutRows - 1) / kLutRows;
+    const int grid = static_cast<int>(nchunks < bnn::sm_count() ? nchunks : bnn::sm_count());
+    kern<<<grid, kLutRows * kLutSlices, smem, s>>>(x_bf16, packed, scale, n, static_cast<int>(k), static_cast<int>(kt),
+                                                  slice_words, out);
+    return bnn::check_launch();
+  }
   if (m <= 8) {
     const int64_t warps_per_block = 8;
     const int64_t blocks_needed = (n + warps_per_block - 1) / warps_per_block;

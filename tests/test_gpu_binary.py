@@ -51,7 +51,7 @@ def test_pack_empty(bnn):
     assert out.shape == (4, 0)
 
 
-def _gemm_case(bnn, m, n, k, seed, offset_words=0):
+def _gemm_case(bnn, m, n, k, seed, offset_words=0, algos=(0, 1, 2)):
     xp = synth.fair_coin_words(seed, 1, m, k)
     wp = synth.fair_coin_words(seed, 2, n, k)
     alpha = synth.uniform_f32(seed, 3, (n,), -1.0, 2.0)
@@ -67,11 +67,12 @@ def _gemm_case(bnn, m, n, k, seed, offset_words=0):
         dxp, dwp = bx[offset_words:].view(m, kw), bw[offset_words:].view(n, kw)
     else:
         dxp, dwp = to_dev_u64(xp), to_dev_u64(wp)
-    dots, out = bnn.bnn_binary_gemm(dxp, dwp, to_dev_f32(alpha), k)
-    torch.cuda.synchronize()
     want_d, want_o = oracle.binary_gemm(xp, wp, alpha, m, n, k)
-    assert_bits_equal(dots.cpu().numpy(), want_d, f"dots {m}x{n}x{k}")
-    assert_bits_equal(out.cpu().numpy(), want_o, f"out {m}x{n}x{k}")
+    for algo in algos:
+        dots, out = bnn.bnn_binary_gemm(dxp, dwp, to_dev_f32(alpha), k, algo=algo)
+        torch.cuda.synchronize()
+        assert_bits_equal(dots.cpu().numpy(), want_d, f"dots {m}x{n}x{k} algo {algo}")
+        assert_bits_equal(out.cpu().numpy(), want_o, f"out {m}x{n}x{k} algo {algo}")
 
 
 @pytest.mark.parametrize("m", [1, 2, 3, 4, 5, 8])
@@ -81,7 +82,8 @@ def test_skinny_matches_oracle(bnn, m, n, k):
 
 
 @pytest.mark.parametrize("m,n,k", [(9, 33, 64), (64, 64, 128), (130, 257, 1000), (300, 129, 4096 + 100),
-                                   (129, 1000, 63), (512, 640, 512), (17, 3, 130)])
+                                   (129, 1000, 63), (512, 640, 512), (17, 3, 130), (16, 8, 32), (1000, 2500, 257),
+                                   (2400, 2500, 640)])
 def test_tiled_matches_oracle(bnn, m, n, k):
     _gemm_case(bnn, m, n, k, seed=m + 7 * n + k)
 
@@ -93,11 +95,12 @@ def test_unaligned_operands_use_the_8_byte_path(bnn, m, n, k):
 
 def test_k_zero_gives_zero_and_alpha_times_zero(bnn):
     for m in (1, 20):
-        xp = torch.empty((m, 0), dtype=torch.int64, device="cuda")
-        wp = torch.empty((5, 0), dtype=torch.int64, device="cuda")
-        alpha = to_dev_f32(np.array([1.0, -2.0, 0.0, 3.5, 1e-3], np.float32))
-        dots, out = bnn.bnn_binary_gemm(xp, wp, alpha, 0)
-        assert torch.all(dots == 0) and torch.all(out == 0)
+        for algo in (0, 1, 2):
+            xp = torch.empty((m, 0), dtype=torch.int64, device="cuda")
+            wp = torch.empty((5, 0), dtype=torch.int64, device="cuda")
+            alpha = to_dev_f32(np.array([1.0, -2.0, 0.0, 3.5, 1e-3], np.float32))
+            dots, out = bnn.bnn_binary_gemm(xp, wp, alpha, 0, algo=algo)
+            assert torch.all(dots == 0) and torch.all(out == 0)
 
 
 def test_dots_only_and_out_only(bnn):
@@ -148,11 +151,12 @@ def test_workload_gemv_small_full(bnn):
     assert_bits_equal(out.cpu().numpy(), want_o, "cfg1 out")
 
 
-def test_workload_gemm_fused_pack(bnn):
+@pytest.mark.parametrize("algo", [0, 1, 2])
+def test_workload_gemm_fused_pack(bnn, algo):
     c = synth.gemm_fused_pack(1)
     xp = bnn.bnn_pack_signs(to_dev_f32(c["x"]))
     wp = bnn.bnn_pack_signs(to_dev_f32(c["w"]))
-    dots, out = bnn.bnn_binary_gemm(xp, wp, to_dev_f32(c["alpha"]), c["k"])
+    dots, out = bnn.bnn_binary_gemm(xp, wp, to_dev_f32(c["alpha"]), c["k"], algo=algo)
     hx, hw = host_u64(xp), host_u64(wp)
     assert_bits_equal(hx, oracle.pack_signs(c["x"]), "cfg2 x pack")
     assert_bits_equal(hw, oracle.pack_signs(c["w"]), "cfg2 w pack")
@@ -172,9 +176,11 @@ def test_workload_gemv_ffn(bnn):
     assert_bits_equal(out.cpu().numpy(), want_o, "cfg3 out")
 
 
-def test_workload_gemm_large(bnn):
+@pytest.mark.parametrize("algo", [0, 1])
+def test_workload_gemm_large(bnn, algo):
     c = synth.gemm_large(1)
-    dots, out = bnn.bnn_binary_gemm(to_dev_u64(c["xp"]), to_dev_u64(c["wp"]), to_dev_f32(c["alpha"]), c["k"])
+    dots, out = bnn.bnn_binary_gemm(to_dev_u64(c["xp"]), to_dev_u64(c["wp"]), to_dev_f32(c["alpha"]), c["k"],
+                                    algo=algo)
     torch.cuda.synchronize()
     rows, cols = _samples(c["m"], c["n"], 2048, 4)
     sd, so = oracle.binary_gemm_sampled(c["xp"], c["wp"], c["alpha"], c["m"], c["n"], c["k"], rows, cols)
@@ -186,3 +192,22 @@ def test_workload_gemm_large(bnn):
     assert np.all((d - k) % 2 == 0) and np.abs(d).max() <= k
     o = out.cpu().numpy()
     assert_bits_equal(o, c["alpha"][None, :] * d.astype(np.float32), "cfg4 epilogue everywhere")
+
+
+def test_algos_agree_bitwise_on_random_shapes(bnn):
+    """Every kernel family gives the same bits on ragged shapes (m from 1 to 300)."""
+    rng = np.random.default_rng(77)
+    for _ in range(12):
+        m, n, k = int(rng.integers(1, 300)), int(rng.integers(1, 300)), int(rng.integers(1, 700))
+        xp = to_dev_u64(synth.fair_coin_words(int(m + n + k), 1, m, k))
+        wp = to_dev_u64(synth.fair_coin_words(int(m + n + k), 2, n, k))
+        alpha = to_dev_f32(synth.uniform_f32(3, 3, (n,), -2.0, 2.0))
+        res = [bnn.bnn_binary_gemm(xp, wp, alpha, k, algo=a) for a in (0, 1, 2)]
+        for d, o in res[1:]:
+            assert torch.equal(d, res[0][0]) and torch.equal(o.view(torch.int32), res[0][1].view(torch.int32))
+
+
+def test_unknown_algo_rejected(bnn):
+    xp = torch.zeros((2, 1), dtype=torch.int64, device="cuda")
+    with pytest.raises(bnn.BnnError):
+        bnn.bnn_binary_gemm(xp, xp, None, 64, want_out=False, algo=7)
