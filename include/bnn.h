@@ -144,6 +144,38 @@ bnn_status bnn_ternary_pack(const float* w, int64_t n, int64_t k, uint16_t* pack
                             float* scale, float* delta, cudaStream_t s);
 
 /*
+ * bnn_ternary_pack_noalloc -- bnn_ternary_pack for callers that must not
+ * allocate device memory.  The pages have no counterpart to this call: it is
+ * an interface choice of this library.
+ *
+ * Some callers cannot allocate when they pack weights: a serving runtime that
+ * reserves all device memory up front under its own allocator and forbids
+ * allocation on its request path, a process whose device or driver setup has
+ * no stream-ordered memory pools (cudaMallocAsync unavailable), or a
+ * latency-bound loop that cannot risk an allocator call blocking or failing.
+ * This entry point computes exactly what bnn_ternary_pack computes (same
+ * kernels, same reduction order, bitwise the same outputs) and takes the
+ * same arguments, but keeps its float64 partial sums in a fixed 64 KiB array
+ * compiled into libbnn.so instead of allocating them.  It calls no
+ * cudaMalloc, cudaMallocAsync, cudaFree or other allocating routine.
+ *
+ *   Limit: n * k <= 2^29 (536,870,912 weights, one partial sum per 65536
+ *   weights in an array of 8192); larger sizes return BNN_ERR_INVALID_ARG
+ *   with nothing written.
+ *   Set-up: the first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current) and caches it; make
+ *   that first call before any stream capture on the device.
+ *   Sharing: every GPU that loads the library holds the array until the
+ *   process exits, and all calls on a device share it.  Each call writes
+ *   every slot it reads before reading it, so nothing needs clearing between
+ *   calls, but two calls that overlap on the GPU (e.g. on streams with no
+ *   ordering between them) race on the array and may both produce wrong
+ *   results: order such calls on one stream or with events.
+ */
+bnn_status bnn_ternary_pack_noalloc(const float* w, int64_t n, int64_t k, uint16_t* packed,
+                                    float* scale, float* delta, cudaStream_t s);
+
+/*
  * bnn_ternary_gemm -- ternary layer forward: base-3 unpack and accumulate.
  * [BTE] "Module Overview" (Layer.forward) with the "Features" encoding.
  *

@@ -13,6 +13,8 @@
 // (base 9 works the same way with 9F, giving trit pairs).
 #include <cuda_bf16.h>
 
+#include <mutex>
+
 #include "bnn_internal.cuh"
 
 namespace {
@@ -480,5 +482,72 @@ extern "C" bnn_status bnn_ternary_gemm(const uint16_t* x_bf16, const uint16_t* p
   if (gx > 2147483647LL || gy > 65535) return BNN_ERR_INVALID_ARG;
   ternary_gemm_mma_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), 256, 0, s>>>(
       x_bf16, packed, scale, m, n, k, kt, out);
+  return bnn::check_launch();
+}
+
+// ---------------------------------------------------------------------------
+// bnn_ternary_pack_noalloc: the same TWN pack with its scratch in a fixed
+// device array instead of memory taken from an allocator.
+//
+// The float64 partial sums of |W| (one per 65536 weights) live in the
+// file-scope array below, which every GPU that loads this library holds
+// until the process exits.  Its host-side name is only a stand-in for the
+// symbol; the device address comes from cudaGetSymbolAddress, looked up once
+// per device (with that device current) on the first call and cached.
+// ---------------------------------------------------------------------------
+constexpr int64_t kNoAllocMaxParts = 8192;  // 64 KiB of float64: up to 8192 * 65536 = 2^29 weights
+
+static __device__ __align__(256) double g_twn_noalloc_partials[kNoAllocMaxParts];
+
+namespace {
+
+constexpr int kNoAllocMaxDevices = 64;
+double* g_noalloc_ptr[kNoAllocMaxDevices] = {nullptr};
+std::mutex g_noalloc_mu;
+
+// Device address of g_twn_noalloc_partials on the current device.
+bnn_status noalloc_scratch(double** out) {
+  int dev = -1;
+  BNN_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return BNN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_twn_noalloc_partials);
+    if (e != cudaSuccess) return bnn::cuda_fail(e);
+    g_noalloc_ptr[dev] = static_cast<double*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return BNN_OK;
+}
+
+}  // namespace
+
+extern "C" bnn_status bnn_ternary_pack_noalloc(const float* w, int64_t n, int64_t k, uint16_t* packed,
+                                               float* scale, float* delta, cudaStream_t s) {
+  if (n < 0 || k < 0) return BNN_ERR_INVALID_ARG;
+  if (!delta) return BNN_ERR_INVALID_ARG;
+  if (n > 0 && !scale) return BNN_ERR_INVALID_ARG;
+  if (n > 0 && k > 0 && (!w || !packed)) return BNN_ERR_INVALID_ARG;
+  if (k > 0 && n > (int64_t(1) << 40) / k) return BNN_ERR_INVALID_ARG;
+  if ((w && !bnn::aligned(w, 4)) || (packed && !bnn::aligned(packed, 2)) || (scale && !bnn::aligned(scale, 4)) ||
+      !bnn::aligned(delta, 4))
+    return BNN_ERR_MISALIGNED;
+  const int64_t total = n * k;
+  const int64_t nparts = (total + kChunk - 1) / kChunk;
+  if (nparts > kNoAllocMaxParts) return BNN_ERR_INVALID_ARG;  // more than 2^29 weights
+  double* partial = nullptr;
+  if (nparts > 0) {
+    const bnn_status st = noalloc_scratch(&partial);
+    if (st != BNN_OK) return st;
+    // Every slot the second kernel reads is written by the first kernel of the
+    // same call, so nothing left by an earlier call needs clearing.
+    twn_abs_partial_kernel<<<static_cast<unsigned>(nparts), kRedThreads, 0, s>>>(w, total, partial);
+    const bnn_status st2 = bnn::check_launch();
+    if (st2 != BNN_OK) return st2;
+  }
+  const int64_t cap = static_cast<int64_t>(bnn::sm_count()) * 8;
+  const int grid = static_cast<int>(n < 1 ? 1 : (n < cap ? n : cap));
+  twn_pack_rows_kernel<<<grid, kRedThreads, 0, s>>>(w, n, k, partial, nparts, total, packed, scale, delta);
   return bnn::check_launch();
 }
