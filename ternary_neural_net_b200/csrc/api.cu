@@ -1,4 +1,6 @@
 // Status strings, error bookkeeping and device queries for libbnn.
+#include <mutex>
+
 #include "bnn_internal.cuh"
 
 namespace {
@@ -12,6 +14,35 @@ namespace bnn {
 bnn_status cuda_fail(cudaError_t e) {
   g_last_cuda_error = static_cast<int>(e);
   return BNN_ERR_CUDA;
+}
+
+namespace {
+struct SmemEntry {
+  const void* kernel;
+  int device;
+  size_t bytes;
+};
+constexpr int kMaxSmemEntries = 256;
+SmemEntry g_smem[kMaxSmemEntries];
+int g_smem_count = 0;
+std::mutex g_smem_mu;
+}  // namespace
+
+cudaError_t ensure_smem_raw(const void* kernel, size_t bytes) {
+  const int dev = current_device();
+  std::lock_guard<std::mutex> lock(g_smem_mu);
+  for (int i = 0; i < g_smem_count; ++i)
+    if (g_smem[i].kernel == kernel && g_smem[i].device == dev && g_smem[i].bytes >= bytes) return cudaSuccess;
+  const cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (e != cudaSuccess) return e;
+  for (int i = 0; i < g_smem_count; ++i)
+    if (g_smem[i].kernel == kernel && g_smem[i].device == dev) {
+      g_smem[i].bytes = bytes;
+      return cudaSuccess;
+    }
+  if (g_smem_count < kMaxSmemEntries) g_smem[g_smem_count++] = SmemEntry{kernel, dev, bytes};
+  return cudaSuccess;
 }
 
 int current_device() {

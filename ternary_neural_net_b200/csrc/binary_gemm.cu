@@ -39,13 +39,14 @@ namespace {
 // ---------------------------------------------------------------------------
 // skinny kernel
 // ---------------------------------------------------------------------------
-template <int VEC, int LPR, int R, int MT>
-__global__ void __launch_bounds__(256)
+template <int VEC, int LPR, int R, int MT, int P>
+__global__ void __launch_bounds__(256, MT == 1 ? 8 : 4)
 binary_gemv_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restrict__ wp,
                    const float* __restrict__ alpha, int m, int64_t n, int k, int kw,
                    int32_t* __restrict__ dots, float* __restrict__ out) {
   static_assert(VEC == 1 || VEC == 2, "VEC");
   constexpr int GROUPS_PER_WARP = 32 / LPR;
+  constexpr int SPAN = LPR * VEC;             // words a row group covers in one pass
   const int lane = threadIdx.x & 31;
   const int sub = lane % LPR;                 // lane within its row group
   const int grp = lane / LPR;                 // row group within the warp
@@ -60,40 +61,50 @@ binary_gemv_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restrict__
 #pragma unroll
       for (int t = 0; t < MT; ++t) acc[r][t] = 0;
 
-    for (int w = sub * VEC; w < kw; w += LPR * VEC) {
-      uint64_t wv[R][VEC];
+    for (int wb = sub * VEC; wb < kw; wb += SPAN * P) {
+      // all R x P loads of this step are issued before any is used
+      uint64_t wv[R][P][VEC];
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const int64_t row = row0 + static_cast<int64_t>(r) * GROUPS_PER_WARP + grp;
-        if (row < n) {
-          const uint64_t* p = wp + row * kw + w;
-          if constexpr (VEC == 2) {
-            const ulonglong2 v = __ldcs(reinterpret_cast<const ulonglong2*>(p));
-            wv[r][0] = v.x;
-            wv[r][VEC - 1] = v.y;
+      for (int p = 0; p < P; ++p) {
+        const int w = wb + p * SPAN;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const int64_t row = row0 + static_cast<int64_t>(r) * GROUPS_PER_WARP + grp;
+          if (row < n && w < kw) {
+            const uint64_t* ptr = wp + row * kw + w;
+            if constexpr (VEC == 2) {
+              const ulonglong2 v = __ldcs(reinterpret_cast<const ulonglong2*>(ptr));
+              wv[r][p][0] = v.x;
+              wv[r][p][VEC - 1] = v.y;
+            } else {
+              wv[r][p][0] = __ldcs(ptr);
+            }
           } else {
-            wv[r][0] = __ldcs(p);
-          }
-        } else {
 #pragma unroll
-          for (int v = 0; v < VEC; ++v) wv[r][v] = 0;
+            for (int v = 0; v < VEC; ++v) wv[r][p][v] = 0;
+          }
         }
       }
 #pragma unroll
-      for (int t = 0; t < MT; ++t) {
-        if (t < m) {
-          uint64_t xv[VEC];
-          if constexpr (VEC == 2) {
-            const ulonglong2 v = __ldg(reinterpret_cast<const ulonglong2*>(xp + static_cast<int64_t>(t) * kw + w));
-            xv[0] = v.x;
-            xv[VEC - 1] = v.y;
-          } else {
-            xv[0] = __ldg(xp + static_cast<int64_t>(t) * kw + w);
+      for (int p = 0; p < P; ++p) {
+        const int w = wb + p * SPAN;
+        if (w >= kw) continue;
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+          if (t < m) {
+            uint64_t xv[VEC];
+            if constexpr (VEC == 2) {
+              const ulonglong2 v = __ldg(reinterpret_cast<const ulonglong2*>(xp + static_cast<int64_t>(t) * kw + w));
+              xv[0] = v.x;
+              xv[VEC - 1] = v.y;
+            } else {
+              xv[0] = __ldg(xp + static_cast<int64_t>(t) * kw + w);
+            }
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+              for (int v = 0; v < VEC; ++v) acc[r][t] += __popcll(wv[r][p][v] ^ xv[v]);
           }
-#pragma unroll
-          for (int r = 0; r < R; ++r)
-#pragma unroll
-            for (int v = 0; v < VEC; ++v) acc[r][t] += __popcll(wv[r][v] ^ xv[v]);
         }
       }
     }
@@ -123,7 +134,7 @@ binary_gemv_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restrict__
   }
 }
 
-template <int VEC, int LPR, int R, int MT>
+template <int VEC, int LPR, int R, int MT, int P = 1>
 void launch_gemv(const uint64_t* xp, const uint64_t* wp, const float* alpha, int m, int64_t n, int k,
                  int kw, int32_t* dots, float* out, cudaStream_t s) {
   constexpr int threads = 256;
@@ -131,7 +142,7 @@ void launch_gemv(const uint64_t* xp, const uint64_t* wp, const float* alpha, int
   const int64_t blocks_needed = (n + rows_per_block - 1) / rows_per_block;
   const int64_t cap = static_cast<int64_t>(bnn::sm_count()) * 8;
   const int grid = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
-  binary_gemv_kernel<VEC, LPR, R, MT><<<grid, threads, 0, s>>>(xp, wp, alpha, m, n, k, kw, dots, out);
+  binary_gemv_kernel<VEC, LPR, R, MT, P><<<grid, threads, 0, s>>>(xp, wp, alpha, m, n, k, kw, dots, out);
 }
 
 template <int VEC>
@@ -142,7 +153,7 @@ void dispatch_gemv(const uint64_t* xp, const uint64_t* wp, const float* alpha, i
   if (m <= 1) {
     if (chunks <= 8) launch_gemv<VEC, 8, 2, 1>(xp, wp, alpha, m, n, k, kw, dots, out, s);
     else if (chunks <= 16) launch_gemv<VEC, 16, 2, 1>(xp, wp, alpha, m, n, k, kw, dots, out, s);
-    else launch_gemv<VEC, 32, 2, 1>(xp, wp, alpha, m, n, k, kw, dots, out, s);
+    else launch_gemv<VEC, 32, 2, 1, 2>(xp, wp, alpha, m, n, k, kw, dots, out, s);  // 4 loads in flight per lane
   } else if (m <= 2) {
     if (chunks <= 8) launch_gemv<VEC, 8, 2, 2>(xp, wp, alpha, m, n, k, kw, dots, out, s);
     else launch_gemv<VEC, 32, 2, 2>(xp, wp, alpha, m, n, k, kw, dots, out, s);
@@ -283,13 +294,15 @@ bnn_status launch_tiled(const uint64_t* xp, const uint64_t* wp, const float* alp
 // ---------------------------------------------------------------------------
 // int8 tensor-core kernel
 // ---------------------------------------------------------------------------
-constexpr int kMBKW = 4;               // uint64 words per stage per row (256 bits = 8 k32 steps)
-constexpr int kMPitch = 6;             // 48-byte rows: 8 consecutive rows hit distinct 16-byte slots
+constexpr int kMBKW = 8;               // uint64 words per stage per row (512 bits = 16 k32 steps)
+constexpr int kMPitch = 10;            // 80-byte rows: 8 consecutive rows hit distinct 16-byte slots
 constexpr int kMStages = 4;
 
 // Bytes j of the result are -1 (0xFF) where bit 8j+7-s of w is set, else 0;
 // mul = 2^s.  The shift is a multiply so that it issues on the FMA pipe and
-// leaves the integer pipe to the byte permute.
+// leaves the integer pipe to the byte permute; the multipliers come from a
+// constant table so that the compiler does not turn them back into shifts.
+__constant__ uint32_t kShiftMul[8] = {1u, 2u, 4u, 8u, 16u, 32u, 64u, 128u};
 __device__ __forceinline__ uint32_t expand_neg(uint32_t w, uint32_t mul) {
   uint32_t r;
   asm("prmt.b32 %0, %1, %1, 0xBA98;\n" : "=r"(r) : "r"(w * mul));
@@ -339,7 +352,7 @@ binary_gemm_mma_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restri
   const int64_t m0 = static_cast<int64_t>(blockIdx.y) * BM;
   const int64_t n0 = static_cast<int64_t>(blockIdx.x) * BN;
   const int ktiles = (kw + kMBKW - 1) / kMBKW;
-  const uint32_t s0 = 1u << (2 * tq), s1 = 2u << (2 * tq);
+  const uint32_t s0 = kShiftMul[2 * tq], s1 = kShiftMul[2 * tq + 1];
   const bool count_a = (wn == 0) && (tq == 0);   // one lane per activation row and K group
   const bool count_b = (wm == 0) && (tq == 0);   // one lane per weight row and K group
 
@@ -439,27 +452,27 @@ binary_gemm_mma_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restri
 
   if constexpr (KSPLIT > 1) {
     // groups 1.. hand their partial AND-counts to group 0 (fixed order: exact integers anyway)
-    int* xs = reinterpret_cast<int*>(smem);  // [KSPLIT-1][GROUP][WM*WN*4]
+    int* xs = reinterpret_cast<int*>(smem);  // [KSPLIT-1][WM*WN*4][GROUP]: lanes hit consecutive banks
     constexpr int PER = WM * WN * 4;
     if (kg > 0) {
-      int* dst = xs + ((kg - 1) * GROUP + (tid % GROUP)) * PER;
+      int* dst = xs + (kg - 1) * PER * GROUP + (tid % GROUP);
 #pragma unroll
       for (int i = 0; i < WM; ++i)
 #pragma unroll
         for (int j = 0; j < WN; ++j)
 #pragma unroll
-          for (int c = 0; c < 4; ++c) dst[(i * WN + j) * 4 + c] = acc[i][j][c];
+          for (int c = 0; c < 4; ++c) dst[((i * WN + j) * 4 + c) * GROUP] = acc[i][j][c];
     }
     __syncthreads();
     if (kg == 0) {
       for (int g = 1; g < KSPLIT; ++g) {
-        const int* src = xs + ((g - 1) * GROUP + tid) * PER;
+        const int* src = xs + (g - 1) * PER * GROUP + tid;
 #pragma unroll
         for (int i = 0; i < WM; ++i)
 #pragma unroll
           for (int j = 0; j < WN; ++j)
 #pragma unroll
-            for (int c = 0; c < 4; ++c) acc[i][j][c] += src[(i * WN + j) * 4 + c];
+            for (int c = 0; c < 4; ++c) acc[i][j][c] += src[((i * WN + j) * 4 + c) * GROUP];
       }
     }
     __syncthreads();

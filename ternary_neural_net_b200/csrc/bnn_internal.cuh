@@ -27,18 +27,15 @@ int sm_count();
 // Current device index (0 if the query fails).
 int current_device();
 
-// Raises a kernel's dynamic shared-memory limit to `bytes` once per device and
-// process, so that later calls (including calls made while a stream is being
-// captured into a CUDA graph) only launch.
+// Raises a kernel's dynamic shared-memory limit to `bytes` once per kernel,
+// device and process, so that later calls (including calls made while a
+// stream is being captured into a CUDA graph) only launch.
+cudaError_t ensure_smem_raw(const void* kernel, size_t bytes);
+
 template <typename Kernel>
 cudaError_t ensure_smem(Kernel kern, size_t bytes) {
   if (bytes <= 48 * 1024) return cudaSuccess;
-  static size_t done[64] = {0};
-  const int dev = current_device();
-  if (dev >= 0 && dev < 64 && done[dev] >= bytes) return cudaSuccess;
-  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
-  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = bytes;
-  return e;
+  return ensure_smem_raw(reinterpret_cast<const void*>(kern), bytes);
 }
 
 }  // namespace bnn

@@ -11,6 +11,7 @@
 // [w / 3^10, w / 3^10 + 1/3^10), so repeatedly taking the high word of 3F
 // yields the digits most significant first, exactly, for every valid word
 // (base 9 works the same way with 9F, giving trit pairs).
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 
 #include <mutex>
@@ -296,14 +297,26 @@ size_t lut_smem_bytes(int64_t kt) {
 }
 
 // ---------------------------------------------------------------------------
-// Ternary GEMM (m > 8): decode trits to bf16 tiles in shared memory, bf16
+// Ternary GEMM (m > 8): trits decoded to bf16 tiles in shared memory, bf16
 // mma.sync m16n8k16 with fp32 accumulation.
+//
+// A cluster of kTK CTAs computes one kTBM x kTBN output tile; CTA r of the
+// cluster takes the r-th quarter of the packed words, so four times as many
+// CTAs share the GPU and each reads only its quarter of the activations.  The
+// partial tiles are added through distributed shared memory in rank order
+// (0 + 1 + 2 + 3) by rank 0, which applies the scale once and writes out.
+// Per 8-word (80-trit, 5 x k16) chunk: the activation tile is copied with
+// 16-byte cp.async (double-buffered), and each weight word is decoded by one
+// thread: five base-9 digits, each a 9-entry table lookup giving the bf16
+// pair (t_2q, t_2q+1), stored as one 32-bit word.
 // ---------------------------------------------------------------------------
-constexpr int kTBM = 64;           // activation rows per CTA
-constexpr int kTBN = 64;           // weight rows per CTA
-constexpr int kTBKW = 16;          // base-3 words per K chunk
-constexpr int kTBK = 10 * kTBKW;   // 160 trits per chunk (a multiple of 16)
-constexpr int kTPitch = kTBK + 8;  // bf16 elements per smem row (336 bytes)
+constexpr int kTBM = 64;             // activation rows per CTA
+constexpr int kTBN = 64;             // weight rows per CTA
+constexpr int kTK = 4;               // CTAs per cluster, splitting the packed words
+constexpr int kTCW = 8;              // words per chunk (80 trits = 5 k16 steps)
+constexpr int kTCK = 10 * kTCW;      // 80 trits per chunk
+constexpr int kTPitch = kTCK + 8;    // bf16 per smem row: 176 bytes, an odd multiple of 16
+constexpr int kTThreads = 256;
 
 __device__ __forceinline__ void ldmatrix_x4(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3,
                                             const void* p) {
@@ -311,10 +324,6 @@ __device__ __forceinline__ void ldmatrix_x4(uint32_t& r0, uint32_t& r1, uint32_t
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                : "r"(a));
-}
-__device__ __forceinline__ void ldmatrix_x2(uint32_t& r0, uint32_t& r1, const void* p) {
-  const unsigned a = static_cast<unsigned>(__cvta_generic_to_shared(p));
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];\n" : "=r"(r0), "=r"(r1) : "r"(a));
 }
 __device__ __forceinline__ void mma_bf16_16816(float* c, const uint32_t* a, const uint32_t* b) {
   asm volatile(
@@ -324,18 +333,79 @@ __device__ __forceinline__ void mma_bf16_16816(float* c, const uint32_t* a, cons
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-__global__ void __launch_bounds__(256)
+template <bool VECX>
+__global__ void __cluster_dims__(kTK, 1, 1) __launch_bounds__(kTThreads)
 ternary_gemm_mma_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ packed,
                         const float* __restrict__ scale, int64_t m, int64_t n, int64_t k, int64_t kt,
-                        float* __restrict__ out) {
-  __shared__ __align__(16) uint16_t Xs[kTBM * kTPitch];
-  __shared__ __align__(16) uint16_t Ws[kTBN * kTPitch];
+                        int64_t slice_words, float* __restrict__ out) {
+  __shared__ __align__(16) uint16_t Xs[2][kTBM * kTPitch];
+  __shared__ __align__(16) uint16_t Ws[2][kTBN * kTPitch];
+  __shared__ uint32_t lut[9];
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   const int wm = warp & 1;   // 2 warps along M (32 rows each)
   const int wn = warp >> 1;  // 4 warps along N (16 cols each)
+  const int rank = static_cast<int>(cluster.block_rank());
   const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kTBM;
-  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kTBN;
+  const int64_t n0 = static_cast<int64_t>(blockIdx.x / kTK) * kTBN;
+  const int64_t w_begin = rank * slice_words;
+  const int64_t w_end = w_begin + slice_words < kt ? w_begin + slice_words : kt;
+  const int64_t nchunks = w_end > w_begin ? (w_end - w_begin + kTCW - 1) / kTCW : 0;
+
+  if (tid < 9) {
+    // bf16 bit patterns of (t_lo, t_hi) for base-9 digit v = (t_lo + 1) + 3 (t_hi + 1)
+    const int lo = tid % 3, hi = tid / 3;  // digit = trit + 1
+    const uint32_t blo = lo == 0 ? 0xBF80u : (lo == 2 ? 0x3F80u : 0u);
+    const uint32_t bhi = hi == 0 ? 0xBF80u : (hi == 2 ? 0x3F80u : 0u);
+    lut[tid] = blo | (bhi << 16);
+  }
+
+  auto load_x = [&](int64_t ch, int buf) {
+    const int64_t kb = 10 * (w_begin + ch * kTCW);  // first trit of the chunk
+    if constexpr (VECX) {
+      // 64 rows x 10 pieces of 16 bytes; pieces past k are zero-filled
+      for (int c = tid; c < kTBM * (kTCK / 8); c += kTThreads) {
+        const int row = c / (kTCK / 8), piece = c % (kTCK / 8);
+        const int64_t gm = m0 + row, gk = kb + 8 * piece;
+        int bytes = 0;
+        if (gm < m && gk < k) bytes = static_cast<int>((k - gk < 8 ? k - gk : 8) * 2);
+        const uint16_t* src = bytes ? x + gm * k + gk : x;
+        const unsigned saddr = static_cast<unsigned>(__cvta_generic_to_shared(&Xs[buf][row * kTPitch + 8 * piece]));
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(saddr), "l"(src), "r"(bytes) : "memory");
+      }
+    } else {
+      for (int c = tid; c < kTBM * kTCK; c += kTThreads) {
+        const int row = c / kTCK, col = c % kTCK;
+        const int64_t gm = m0 + row, gk = kb + col;
+        Xs[buf][row * kTPitch + col] = (gm < m && gk < k) ? __ldg(x + gm * k + gk) : static_cast<uint16_t>(0);
+      }
+    }
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+  };
+
+  auto decode_w = [&](int64_t ch, int buf) {
+    const int64_t wb = w_begin + ch * kTCW;
+    for (int c = tid; c < kTBN * kTCW; c += kTThreads) {
+      const int row = c / kTCW, wj = c % kTCW;
+      const int64_t gn = n0 + row, gw = wb + wj;
+      uint32_t* dst = reinterpret_cast<uint32_t*>(&Ws[buf][row * kTPitch + 10 * wj]);
+      if (gn < n && gw < w_end) {
+        uint32_t F = static_cast<uint32_t>(__ldg(packed + gn * kt + gw)) * kFixMul;
+#pragma unroll
+        for (int q = 4; q >= 0; --q) {
+          const uint32_t v = __umulhi(F, 9u);
+          F *= 9u;
+          dst[q] = lut[v];
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 5; ++q) dst[q] = 0u;
+      }
+    }
+  };
 
   float acc[2][2][4];
 #pragma unroll
@@ -345,72 +415,72 @@ ternary_gemm_mma_kernel(const uint16_t* __restrict__ x, const uint16_t* __restri
 #pragma unroll
       for (int c = 0; c < 4; ++c) acc[a][b][c] = 0.0f;
 
-  const int64_t nchunks = (kt + kTBKW - 1) / kTBKW;
+  __syncthreads();  // lut ready
+  if (nchunks > 0) {
+    load_x(0, 0);
+    decode_w(0, 0);
+  }
   for (int64_t ch = 0; ch < nchunks; ++ch) {
-    const int64_t kbase = ch * kTBK;
-    // Activations: kTBM rows x kTBK bf16, zero outside [m) x [k).
-    for (int idx = tid; idx < kTBM * kTBK; idx += 256) {
-      const int row = idx / kTBK, col = idx % kTBK;
-      const int64_t gm = m0 + row, gk = kbase + col;
-      Xs[row * kTPitch + col] = (gm < m && gk < k) ? __ldg(x + gm * k + gk) : static_cast<uint16_t>(0);
+    const int buf = static_cast<int>(ch & 1);
+    if (ch + 1 < nchunks) {
+      load_x(ch + 1, buf ^ 1);
+      asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;\n" ::: "memory");
     }
-    // Weights: kTBN rows x kTBKW words, each decoded to 10 bf16 trits.
-    for (int idx = tid; idx < kTBN * kTBKW; idx += 256) {
-      const int row = idx / kTBKW, wj = idx % kTBKW;
-      const int64_t gn = n0 + row, gj = ch * kTBKW + wj;
-      uint16_t* dst = Ws + row * kTPitch + 10 * wj;
-      if (gn < n && gj < kt) {
-        uint32_t F = static_cast<uint32_t>(__ldg(packed + gn * kt + gj)) * kFixMul;
+    __syncthreads();  // chunk ch's activations landed and its weights are decoded
 #pragma unroll
-        for (int i = 9; i >= 0; --i) {
-          const uint32_t d = __umulhi(F, 3u);
-          F *= 3u;
-          dst[i] = d == 0u ? static_cast<uint16_t>(0xBF80u) : (d == 2u ? static_cast<uint16_t>(0x3F80u) : static_cast<uint16_t>(0));
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 10; ++i) dst[i] = 0;
-      }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int ks = 0; ks < kTBK; ks += 16) {
-      uint32_t af[2][4], bfr[2][2];
+    for (int ks = 0; ks < kTCK; ks += 16) {
+      uint32_t af[2][4], bfr[4];
 #pragma unroll
       for (int mi = 0; mi < 2; ++mi) {
         const int row = wm * 32 + mi * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
         const int col = ks + 8 * (lane >> 4);
-        ldmatrix_x4(af[mi][0], af[mi][1], af[mi][2], af[mi][3], Xs + row * kTPitch + col);
+        ldmatrix_x4(af[mi][0], af[mi][1], af[mi][2], af[mi][3], &Xs[buf][row * kTPitch + col]);
       }
-#pragma unroll
-      for (int ni = 0; ni < 2; ++ni) {
-        const int row = wn * 16 + ni * 8 + (lane & 7);
+      {
+        // matrices: (n 0-7, k 0-7), (n 0-7, k 8-15), (n 8-15, k 0-7), (n 8-15, k 8-15)
+        const int row = wn * 16 + (lane & 7) + 8 * (lane >> 4);
         const int col = ks + 8 * ((lane >> 3) & 1);
-        ldmatrix_x2(bfr[ni][0], bfr[ni][1], Ws + row * kTPitch + col);
+        ldmatrix_x4(bfr[0], bfr[1], bfr[2], bfr[3], &Ws[buf][row * kTPitch + col]);
       }
 #pragma unroll
-      for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-        for (int ni = 0; ni < 2; ++ni) mma_bf16_16816(acc[mi][ni], af[mi], bfr[ni]);
+      for (int mi = 0; mi < 2; ++mi) {
+        mma_bf16_16816(acc[mi][0], af[mi], &bfr[0]);
+        mma_bf16_16816(acc[mi][1], af[mi], &bfr[2]);
+      }
     }
-    __syncthreads();
+    if (ch + 1 < nchunks) decode_w(ch + 1, buf ^ 1);
+    __syncthreads();  // everyone is done with buffer `buf` before it is refilled
   }
 
+  // Partial tile -> own shared memory; rank 0 adds the cluster's partials in rank order.
+  float* part = reinterpret_cast<float*>(&Xs[0][0]);  // kTBM x kTBN floats (16 KiB) fit in Xs
   const int g = lane >> 2, tq = lane & 3;
 #pragma unroll
   for (int mi = 0; mi < 2; ++mi)
 #pragma unroll
     for (int ni = 0; ni < 2; ++ni)
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int64_t gm = m0 + wm * 32 + mi * 16 + g + 8 * h;
-        if (gm >= m) continue;
+      for (int h = 0; h < 2; ++h)
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-          const int64_t gn = n0 + wn * 16 + ni * 8 + 2 * tq + c;
-          if (gn < n) out[gm * n + gn] = __ldg(scale + gn) * acc[mi][ni][2 * h + c];
+          const int r = wm * 32 + mi * 16 + g + 8 * h;
+          const int col = wn * 16 + ni * 8 + 2 * tq + c;
+          part[r * kTBN + col] = acc[mi][ni][2 * h + c];
         }
-      }
+  cluster.sync();
+  if (rank == 0) {
+    for (int idx = tid; idx < kTBM * kTBN; idx += kTThreads) {
+      const int r = idx / kTBN, col = idx % kTBN;
+      const int64_t gm = m0 + r, gn = n0 + col;
+      float s = part[idx];
+#pragma unroll
+      for (int q = 1; q < kTK; ++q) s += cluster.map_shared_rank(part, q)[idx];
+      if (gm < m && gn < n) out[gm * n + gn] = __ldg(scale + gn) * s;
+    }
+  }
+  cluster.sync();  // keep every CTA's partial tile alive until rank 0 has read it
 }
 
 }  // namespace
@@ -478,10 +548,16 @@ extern "C" bnn_status bnn_ternary_gemm(const uint16_t* x_bf16, const uint16_t* p
     else ternary_gemv_kernel<8><<<grid, 256, 0, s>>>(x_bf16, packed, scale, static_cast<int>(m), n, k, kt, out);
     return bnn::check_launch();
   }
-  const int64_t gx = (n + kTBN - 1) / kTBN, gy = (m + kTBM - 1) / kTBM;
-  if (gx > 2147483647LL || gy > 65535) return BNN_ERR_INVALID_ARG;
-  ternary_gemm_mma_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), 256, 0, s>>>(
-      x_bf16, packed, scale, m, n, k, kt, out);
+  const int64_t ntiles = (n + kTBN - 1) / kTBN, gy = (m + kTBM - 1) / kTBM;
+  if (ntiles * kTK > 2147483647LL || gy > 65535) return BNN_ERR_INVALID_ARG;
+  // each cluster rank takes a whole number of 8-word chunks
+  const int64_t per = (kt + kTK - 1) / kTK;
+  const int64_t slice_words = (per + kTCW - 1) / kTCW * kTCW;
+  const dim3 grid(static_cast<unsigned>(ntiles * kTK), static_cast<unsigned>(gy));
+  if (k % 8 == 0 && bnn::aligned(x_bf16, 16))
+    ternary_gemm_mma_kernel<true><<<grid, kTThreads, 0, s>>>(x_bf16, packed, scale, m, n, k, kt, slice_words, out);
+  else
+    ternary_gemm_mma_kernel<false><<<grid, kTThreads, 0, s>>>(x_bf16, packed, scale, m, n, k, kt, slice_words, out);
   return bnn::check_launch();
 }
 
