@@ -143,6 +143,34 @@ bnn_status bnn_binary_gemm_algo(const uint64_t* xp, const uint64_t* wp, const fl
 bnn_status bnn_ternary_pack(const float* w, int64_t n, int64_t k, uint16_t* packed,
                             float* scale, float* delta, cudaStream_t s);
 
+/* Ternarisation rules for bnn_ternary_pack_mode. */
+typedef enum {
+  BNN_TERNARY_TWN = 0,      /* Delta = float32(0.7 mean|W|); trit = sign(w) where |w| > Delta */
+  BNN_TERNARY_ABSMEAN = 1,  /* gamma = float32(mean|W|); trit = clamp(round-half-even(w / gamma), -1, 1) */
+  BNN_TERNARY_DELTA = 2     /* a given threshold F >= 0; trit = sign(w) where |w| > F */
+} bnn_ternary_mode;
+
+/*
+ * bnn_ternary_pack_mode -- ternarise, scale and pack with one of the three
+ * quantisation modes of [BTE] "Features" ("twn", "absmean" -- the BitNet
+ * b1.58 absmean scale of "Binary Math Effectiveness", section 5 -- and
+ * "delta", a fixed threshold with MSE-optimal scales).  Every mode writes
+ * the per-row least-squares scale (mean |w| over the row's non-zero trits, 0
+ * for none) and base-3 words exactly as bnn_ternary_pack does.
+ *
+ *   mode        a bnn_ternary_mode; BNN_ERR_INVALID_ARG otherwise.
+ *   threshold   F for BNN_TERNARY_DELTA (must be >= 0, not NaN); ignored
+ *               by the other modes.
+ *   thresh_out  float32 [1], device: Delta (TWN), gamma (ABSMEAN) or F (DELTA).
+ *   In ABSMEAN the quotient w / gamma is one IEEE float32 division and a
+ *   quotient of exactly +-0.5 rounds to 0; gamma = 0 gives all-zero trits.
+ *   TWN is bnn_ternary_pack itself; ABSMEAN takes its float64 partial sums
+ *   from the stream-ordered allocator like bnn_ternary_pack; DELTA allocates
+ *   nothing.  Other arguments, layouts and errors as bnn_ternary_pack.
+ */
+bnn_status bnn_ternary_pack_mode(const float* w, int64_t n, int64_t k, int mode, float threshold,
+                                 uint16_t* packed, float* scale, float* thresh_out, cudaStream_t s);
+
 /*
  * bnn_ternary_pack_noalloc -- bnn_ternary_pack for callers that must not
  * allocate device memory.  The pages have no counterpart to this call: it is

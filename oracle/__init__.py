@@ -32,6 +32,7 @@ def _L():
             "oracle_binary_gemm_sampled": ([vp, vp, vp, i64, i64, i64, vp, vp, i64, vp, vp], None),
             "oracle_twn_ternarize": ([vp, i64, i64, vp, vp, vp], None),
             "oracle_twn_delta": ([vp, i64], C.c_float),
+            "oracle_absmean_ternarize": ([vp, i64, i64, vp, vp, vp], None),
             "oracle_twn_apply": ([vp, i64, i64, C.c_float, vp, vp], None),
             "oracle_base3_pack": ([vp, i64, i64, vp], None),
             "oracle_base3_unpack": ([vp, i64, i64, vp], i64),
@@ -130,6 +131,22 @@ def twn_apply(w: np.ndarray, delta) -> tuple:
     scale = np.zeros(n, dtype=np.float32)
     _L().oracle_twn_apply(_p(w), n, k, C.c_float(np.float32(delta)), _p(trits), _p(scale))
     return trits, scale
+
+
+def absmean_ternarize(w: np.ndarray):
+    """fp32 [n,k] -> (trits int8 [n,k], scale float32 [n], gamma float32)."""
+    w = _c(w, np.float32)
+    n, k = w.shape
+    trits = np.zeros((n, k), dtype=np.int8)
+    scale = np.zeros(n, dtype=np.float32)
+    gamma = np.zeros(1, dtype=np.float32)
+    _L().oracle_absmean_ternarize(_p(w), n, k, _p(trits), _p(scale), _p(gamma))
+    return trits, scale, np.float32(gamma[0])
+
+
+def delta_ternarize(w: np.ndarray, threshold) -> tuple:
+    """Mode 'delta': a given threshold F and least-squares scales (twn_apply at F)."""
+    return twn_apply(w, threshold)
 
 
 def base3_pack(trits: np.ndarray) -> np.ndarray:

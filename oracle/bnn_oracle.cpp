@@ -166,6 +166,41 @@ void oracle_twn_ternarize(const float* w, int64_t n, int64_t k, int8_t* trits,
   oracle_twn_apply(w, n, k, d, trits, scale);
 }
 
+// [BME] section 5 "Ternary math" (absmean scale gamma = mean|w|, BitNet
+// b1.58) and [BTE] "Features" (mode absmean): gamma = float32 of mean|W| over
+// the whole tensor (float64 sum), q = w / gamma in float32, trit =
+// RoundClip(q, -1, 1) = clamp(round-half-to-even(q), -1, 1); so |q| > 0.5
+// gives sign(q) and |q| <= 0.5 (ties included) gives 0.  gamma = 0 gives all
+// zero trits.  Scales are the per-row least-squares scales of oracle_twn_apply
+// ([BTE] "Features": per-channel least-squares scaling).
+void oracle_absmean_ternarize(const float* w, int64_t n, int64_t k, int8_t* trits, float* scale,
+                              float* gamma_out) {
+  const int64_t total = n * k;
+  double sum_abs = 0.0;
+  for (int64_t e = 0; e < total; ++e) sum_abs += std::fabs(double(w[e]));
+  const float g = float(total > 0 ? sum_abs / double(total) : 0.0);
+  *gamma_out = g;
+  for (int64_t r = 0; r < n; ++r) {
+    double kept = 0.0;
+    int64_t nonzero = 0;
+    for (int64_t e = 0; e < k; ++e) {
+      const float v = w[r * k + e];
+      int8_t t = 0;
+      if (g > 0.0f) {
+        const float q = v / g;
+        const float rounded = std::nearbyint(q);  // default rounding mode: to nearest, ties to even
+        t = rounded > 0.0f ? int8_t(+1) : (rounded < 0.0f ? int8_t(-1) : int8_t(0));
+      }
+      trits[r * k + e] = t;
+      if (t != 0) {
+        kept += std::fabs(double(v));
+        ++nonzero;
+      }
+    }
+    scale[r] = nonzero > 0 ? float(kept / double(nonzero)) : 0.0f;
+  }
+}
+
 // [BTE] "Features": 10 trits per 16-bit word, base 3.  Word j of a row holds
 // trits 10j .. 10j+9; trit 10j+i contributes (trit + 1) * 3^i.  Missing trits
 // past k count as 0 (digit 1).

@@ -36,6 +36,8 @@ _SIGS = {
     "bnn_binary_gemm_algo": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _int, _vp],
     "bnn_ternary_pack": [_vp, _i64, _i64, _vp, _vp, _vp, _vp],
     "bnn_ternary_gemm": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
+    "bnn_ternary_pack_mode": [_vp, _i64, _i64, _int, C.c_float, _vp, _vp, _vp, _vp],
+    "bnn_ternary_pack_noalloc": [_vp, _i64, _i64, _vp, _vp, _vp, _vp],
 }
 for _name, _args in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -51,6 +53,7 @@ ABI_SYMBOLS = tuple(_SIGS) + ("bnn_status_string", "bnn_last_cuda_error")
 
 BNN_OK, BNN_ERR_INVALID_ARG, BNN_ERR_MISALIGNED, BNN_ERR_CUDA, BNN_ERR_UNSUPPORTED = range(5)
 ALGO_AUTO, ALGO_POPC, ALGO_MMA_S8 = 0, 1, 2
+TERNARY_TWN, TERNARY_ABSMEAN, TERNARY_DELTA = 0, 1, 2
 MAX_K_BINARY = 1 << 24
 
 
@@ -162,6 +165,20 @@ def bnn_ternary_pack(w: torch.Tensor, packed: torch.Tensor | None = None,
     _check(_lib.bnn_ternary_pack(_ptr(w), n, k, _ptr(packed), _ptr(scale), _ptr(delta), _stream(dev)),
            "bnn_ternary_pack")
     return packed, scale, delta
+
+
+def bnn_ternary_pack_mode(w: torch.Tensor, mode: int, threshold: float = 0.0):
+    """Ternarise with TERNARY_TWN / TERNARY_ABSMEAN / TERNARY_DELTA (threshold = F).
+    Returns (packed int16 [n, ceil(k/10)], scale float32 [n], threshold used float32 [1])."""
+    _dev(w, "w", torch.float32)
+    n, k = w.shape
+    dev = w.device
+    packed = torch.empty((n, trit_words_per_row(k)), dtype=torch.int16, device=dev)
+    scale = torch.empty((n,), dtype=torch.float32, device=dev)
+    thresh = torch.empty((1,), dtype=torch.float32, device=dev)
+    _check(_lib.bnn_ternary_pack_mode(_ptr(w), n, k, int(mode), float(threshold), _ptr(packed), _ptr(scale),
+                                      _ptr(thresh), _stream(dev)), "bnn_ternary_pack_mode")
+    return packed, scale, thresh
 
 
 def bnn_ternary_gemm(x: torch.Tensor, packed: torch.Tensor, scale: torch.Tensor, k: int | None = None,

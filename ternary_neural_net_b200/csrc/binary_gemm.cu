@@ -323,9 +323,10 @@ __device__ __forceinline__ void mma_s8_16832(int* c, const uint32_t* a, const ui
 //   <x, w> = k - 2 popc(a) - 2 popc(b) + 4 popc(a AND b).
 // The MMA operands are the bytes -a and -b (0 or -1: one shift and one
 // sign-replicating byte permute per 4 values), whose products sum to
-// popc(a AND b) exactly; the row popcounts are accumulated on the side from
-// the same shared-memory words by one lane per row.  Zero bits (pad bits,
-// zero-filled tail words and rows) add nothing to any of the three counts.
+// popc(a AND b) exactly; the row popcounts are taken from the same staged
+// tiles, every thread of the CTA owning one row (or a fixed share of one) so
+// the side work is spread evenly.  Zero bits (pad bits, zero-filled tail
+// words and rows) add nothing to any count.
 // KSPLIT groups of WARPS_M x WARPS_N warps split the words of every stage
 // between them (more warps per SM for the same tile); their partial counts
 // are added through shared memory before the epilogue.
@@ -353,8 +354,15 @@ binary_gemm_mma_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restri
   const int64_t n0 = static_cast<int64_t>(blockIdx.x) * BN;
   const int ktiles = (kw + kMBKW - 1) / kMBKW;
   const uint32_t s0 = kShiftMul[2 * tq], s1 = kShiftMul[2 * tq + 1];
-  const bool count_a = (wn == 0) && (tq == 0);   // one lane per activation row and K group
-  const bool count_b = (wm == 0) && (tq == 0);   // one lane per weight row and K group
+  // side popcounts: thread -> (row of the A/B tile stack, share of its words)
+  constexpr int PROWS = BM + BN;
+  static_assert(THREADS % PROWS == 0, "threads must cover the tile rows evenly");
+  constexpr int TPR = THREADS / PROWS;          // threads per row
+  static_assert(kMBKW % TPR == 0, "row words must split evenly");
+  constexpr int WPT = kMBKW / TPR;              // words per thread per stage
+  const int prow = tid % PROWS;
+  const int pw0 = (tid / PROWS) * WPT;
+  int pcount = 0;
 
   auto load_stage = [&](int stage, int kt) {
     const int kbase = kt * kMBKW;
@@ -383,11 +391,6 @@ binary_gemm_mma_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restri
     for (int j = 0; j < WN; ++j)
 #pragma unroll
       for (int c = 0; c < 4; ++c) acc[i][j][c] = 0;
-  int pa[WM][2], pb[WN];
-#pragma unroll
-  for (int i = 0; i < WM; ++i) pa[i][0] = pa[i][1] = 0;
-#pragma unroll
-  for (int j = 0; j < WN; ++j) pb[j] = 0;
 
 #pragma unroll
   for (int st = 0; st < kMStages - 1; ++st) {
@@ -399,6 +402,12 @@ binary_gemm_mma_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restri
     cp_async_wait<kMStages - 2>();
     __syncthreads();
     const int stage = kt % kMStages;
+    {
+      const uint64_t* prow_ptr = prow < BM ? As + (stage * BM + prow) * kMPitch
+                                           : Bs + (stage * BN + (prow - BM)) * kMPitch;
+#pragma unroll
+      for (int q = 0; q < WPT; ++q) pcount += __popcll(prow_ptr[pw0 + q]);
+    }
     const uint64_t* A = As + (stage * BM + wm * 16 * WM + gid) * kMPitch;
     const uint64_t* B = Bs + (stage * BN + wn * 8 * WN + gid) * kMPitch;
 #pragma unroll
@@ -413,16 +422,6 @@ binary_gemm_mma_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restri
       }
 #pragma unroll
       for (int j = 0; j < WN; ++j) bw[j] = *reinterpret_cast<const uint2*>(B + (8 * j) * kMPitch + kk);
-      if (count_a) {
-#pragma unroll
-        for (int i = 0; i < WM; ++i)
-#pragma unroll
-          for (int h = 0; h < 2; ++h) pa[i][h] += __popc(aw[i][h].x) + __popc(aw[i][h].y);
-      }
-      if (count_b) {
-#pragma unroll
-        for (int j = 0; j < WN; ++j) pb[j] += __popc(bw[j].x) + __popc(bw[j].y);
-      }
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t bf[WN][2];
@@ -480,18 +479,9 @@ binary_gemm_mma_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restri
 
   int* pa_s = reinterpret_cast<int*>(smem);  // [BM]
   int* pb_s = pa_s + BM;                      // [BN]
-  for (int i = tid; i < BM + BN; i += THREADS) pa_s[i] = 0;
+  for (int i = tid; i < PROWS; i += THREADS) pa_s[i] = 0;
   __syncthreads();
-  if (count_a) {
-#pragma unroll
-    for (int i = 0; i < WM; ++i)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) atomicAdd(&pa_s[wm * 16 * WM + 16 * i + 8 * h + gid], pa[i][h]);
-  }
-  if (count_b) {
-#pragma unroll
-    for (int j = 0; j < WN; ++j) atomicAdd(&pb_s[wn * 8 * WN + 8 * j + gid], pb[j]);
-  }
+  atomicAdd(&pa_s[prow], pcount);  // integer adds: the order does not matter
   __syncthreads();
   if (kg != 0) return;
 

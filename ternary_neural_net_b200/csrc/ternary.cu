@@ -67,19 +67,32 @@ twn_abs_partial_kernel(const float* __restrict__ w, int64_t total, double* __res
   if (threadIdx.x == 0) partial[blockIdx.x] = s;
 }
 
-// Every block derives Delta from the partial sums (same order in every block),
-// then ternarises, scales and packs whole rows.
+// Ternarisation rules (BNN_TERNARY_* in bnn.h):
+//   TWN:     Delta = float32(0.7 mean|W|), trit = sign(w) where |w| > Delta;
+//   ABSMEAN: gamma = float32(mean|W|), trit = clamp(round-half-even(w / gamma), -1, 1)
+//            ("Binary Math Effectiveness", section 5; BitNet b1.58), i.e.
+//            sign(w) where |w / gamma| > 0.5, 0 at or below (ties round to 0);
+//   DELTA:   a given threshold F, trit = sign(w) where |w| > F.
+// Every mode takes the per-row least-squares scale.
+enum { kModeTWN = 0, kModeAbsmean = 1, kModeDelta = 2 };
+
+// Every block derives the threshold from the partial sums (same order in every
+// block), then ternarises, scales and packs whole rows.
+template <int MODE>
 __global__ void __launch_bounds__(kRedThreads)
 twn_pack_rows_kernel(const float* __restrict__ w, int64_t n, int64_t k, const double* __restrict__ partial,
                      int64_t nparts, int64_t total, uint16_t* __restrict__ packed, float* __restrict__ scale,
-                     float* __restrict__ delta_out) {
+                     float* __restrict__ delta_out, float fixed_threshold = 0.0f) {
   __shared__ double shd[kRedThreads];
   __shared__ long long shl[kRedThreads];
-  double ps = 0.0;
-  for (int64_t i = threadIdx.x; i < nparts; i += kRedThreads) ps += partial[i];
-  const double sum_abs = block_sum_f64(ps, shd);
-  const double mean_abs = total > 0 ? sum_abs / static_cast<double>(total) : 0.0;
-  const float delta = __double2float_rn(0.7 * mean_abs);
+  float delta = fixed_threshold;
+  if constexpr (MODE != kModeDelta) {
+    double ps = 0.0;
+    for (int64_t i = threadIdx.x; i < nparts; i += kRedThreads) ps += partial[i];
+    const double sum_abs = block_sum_f64(ps, shd);
+    const double mean_abs = total > 0 ? sum_abs / static_cast<double>(total) : 0.0;
+    delta = __double2float_rn(MODE == kModeTWN ? 0.7 * mean_abs : mean_abs);
+  }
   if (blockIdx.x == 0 && threadIdx.x == 0) *delta_out = delta;
 
   const int64_t kt = bnn::words10(k);
@@ -96,7 +109,13 @@ twn_pack_rows_kernel(const float* __restrict__ w, int64_t n, int64_t k, const do
         if (e < k) {
           const float v = __ldg(row + e);
           const float a = fabsf(v);
-          if (a > delta) {
+          bool keep;
+          if constexpr (MODE == kModeAbsmean) {
+            keep = delta > 0.0f && fabsf(__fdiv_rn(v, delta)) > 0.5f;  // |round-half-even(q)| >= 1
+          } else {
+            keep = a > delta;
+          }
+          if (keep) {
             digit = v > 0.0f ? 2u : 0u;
             kept += static_cast<double>(a);
             ++nz;
@@ -184,8 +203,10 @@ ternary_gemv_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__
 // (taken with __umulhi and a 32-bit multiply).
 // Lanes of a half-warp own 16 consecutive weight rows and walk the same word
 // index, so the 16 lanes read within one 9-entry table (at most 9 distinct
-// addresses, one per bank: no bank conflicts); the two half-warps work on
-// K-slices whose tables sit in disjoint banks.  The 16-row chunk of packed
+// addresses, one per bank: no bank conflicts); the two half-warps take
+// neighbouring words, whose tables (45 floats apart) sit in disjoint banks.
+// Words are dealt to the SLICES thread groups round-robin, so every group
+// gets the same number of words to within one.  The 16-row chunk of packed
 // words is contiguous in memory and is brought into shared memory with
 // 16-byte cp.async (double-buffered across the chunks this CTA owns); the
 // per-slice partial sums are added in a fixed order, then scaled once.  The
@@ -244,9 +265,8 @@ ternary_gemv_lut_kernel(const uint16_t* __restrict__ x, const uint16_t* __restri
   }
 
   const int row = tid % kLutRows;
-  const int sl = tid / kLutRows;
-  const int j0 = sl * slice_words;
-  const int j1 = j0 + slice_words < kt ? j0 + slice_words : kt;
+  const int sl = tid / kLutRows;   // this thread takes words sl, sl + SLICES, ...
+  (void)slice_words;
 
   for (int it = 0; c < nchunks; c += gridDim.x, ++it) {
     // chunk `it` was the (it+1)-th commit group: allow the kLutStages-2 newer ones to be pending
@@ -256,7 +276,7 @@ ternary_gemv_lut_kernel(const uint16_t* __restrict__ x, const uint16_t* __restri
     const uint16_t* rowp = buf0 + (it % kLutStages) * chunk_elems + row * kt;
     float acc0 = 0.0f, acc1 = 0.0f;
 #pragma unroll 2
-    for (int j = j0; j < j1; ++j) {
+    for (int j = sl; j < kt; j += SLICES) {
       uint32_t F = static_cast<uint32_t>(rowp[j]) * kFixMul;
       const float* Tj = T + (5 * j) * 9;
 #pragma unroll
@@ -338,9 +358,10 @@ __global__ void __cluster_dims__(kTK, 1, 1) __launch_bounds__(kTThreads)
 ternary_gemm_mma_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ packed,
                         const float* __restrict__ scale, int64_t m, int64_t n, int64_t k, int64_t kt,
                         int64_t slice_words, float* __restrict__ out) {
-  __shared__ __align__(16) uint16_t Xs[2][kTBM * kTPitch];
-  __shared__ __align__(16) uint16_t Ws[2][kTBN * kTPitch];
-  __shared__ uint32_t lut[9];
+  extern __shared__ __align__(16) uint16_t tsm[];
+  uint16_t (*Xs)[kTBM * kTPitch] = reinterpret_cast<uint16_t (*)[kTBM * kTPitch]>(tsm);                // [2]
+  uint16_t (*Ws)[kTBN * kTPitch] = reinterpret_cast<uint16_t (*)[kTBN * kTPitch]>(tsm + 2 * kTBM * kTPitch);  // [2]
+  uint32_t* lut = reinterpret_cast<uint32_t*>(tsm + 2 * (kTBM + kTBN) * kTPitch);                     // [9]
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
 
@@ -509,7 +530,7 @@ extern "C" bnn_status bnn_ternary_pack(const float* w, int64_t n, int64_t k, uin
   }
   const int64_t cap = static_cast<int64_t>(bnn::sm_count()) * 8;
   const int grid = static_cast<int>(n < 1 ? 1 : (n < cap ? n : cap));
-  twn_pack_rows_kernel<<<grid, kRedThreads, 0, s>>>(w, n, k, partial, nparts, total, packed, scale, delta);
+  twn_pack_rows_kernel<kModeTWN><<<grid, kRedThreads, 0, s>>>(w, n, k, partial, nparts, total, packed, scale, delta);
   bnn_status st = bnn::check_launch();
   if (partial) {
     const cudaError_t e = cudaFreeAsync(partial, s);
@@ -550,14 +571,18 @@ extern "C" bnn_status bnn_ternary_gemm(const uint16_t* x_bf16, const uint16_t* p
   }
   const int64_t ntiles = (n + kTBN - 1) / kTBN, gy = (m + kTBM - 1) / kTBM;
   if (ntiles * kTK > 2147483647LL || gy > 65535) return BNN_ERR_INVALID_ARG;
-  // each cluster rank takes a whole number of 8-word chunks
+  // each cluster rank takes a whole number of chunks
   const int64_t per = (kt + kTK - 1) / kTK;
   const int64_t slice_words = (per + kTCW - 1) / kTCW * kTCW;
   const dim3 grid(static_cast<unsigned>(ntiles * kTK), static_cast<unsigned>(gy));
-  if (k % 8 == 0 && bnn::aligned(x_bf16, 16))
-    ternary_gemm_mma_kernel<true><<<grid, kTThreads, 0, s>>>(x_bf16, packed, scale, m, n, k, kt, slice_words, out);
-  else
-    ternary_gemm_mma_kernel<false><<<grid, kTThreads, 0, s>>>(x_bf16, packed, scale, m, n, k, kt, slice_words, out);
+  const size_t smem = 2 * static_cast<size_t>(kTBM + kTBN) * kTPitch * sizeof(uint16_t) + 9 * sizeof(uint32_t);
+  if (k % 8 == 0 && bnn::aligned(x_bf16, 16)) {
+    BNN_TRY(bnn::ensure_smem(ternary_gemm_mma_kernel<true>, smem));
+    ternary_gemm_mma_kernel<true><<<grid, kTThreads, smem, s>>>(x_bf16, packed, scale, m, n, k, kt, slice_words, out);
+  } else {
+    BNN_TRY(bnn::ensure_smem(ternary_gemm_mma_kernel<false>, smem));
+    ternary_gemm_mma_kernel<false><<<grid, kTThreads, smem, s>>>(x_bf16, packed, scale, m, n, k, kt, slice_words, out);
+  }
   return bnn::check_launch();
 }
 
@@ -624,6 +649,51 @@ extern "C" bnn_status bnn_ternary_pack_noalloc(const float* w, int64_t n, int64_
   }
   const int64_t cap = static_cast<int64_t>(bnn::sm_count()) * 8;
   const int grid = static_cast<int>(n < 1 ? 1 : (n < cap ? n : cap));
-  twn_pack_rows_kernel<<<grid, kRedThreads, 0, s>>>(w, n, k, partial, nparts, total, packed, scale, delta);
+  twn_pack_rows_kernel<kModeTWN><<<grid, kRedThreads, 0, s>>>(w, n, k, partial, nparts, total, packed, scale, delta);
   return bnn::check_launch();
+}
+
+// ---------------------------------------------------------------------------
+// bnn_ternary_pack_mode: the other ternarisation rules of the pages.
+// ---------------------------------------------------------------------------
+extern "C" bnn_status bnn_ternary_pack_mode(const float* w, int64_t n, int64_t k, int mode, float threshold,
+                                            uint16_t* packed, float* scale, float* thresh_out, cudaStream_t s) {
+  if (mode != kModeTWN && mode != kModeAbsmean && mode != kModeDelta) return BNN_ERR_INVALID_ARG;
+  if (mode == kModeTWN) return bnn_ternary_pack(w, n, k, packed, scale, thresh_out, s);
+  if (mode == kModeDelta && !(threshold >= 0.0f)) return BNN_ERR_INVALID_ARG;  // NaN or negative
+  if (n < 0 || k < 0) return BNN_ERR_INVALID_ARG;
+  if (!thresh_out) return BNN_ERR_INVALID_ARG;
+  if (n > 0 && !scale) return BNN_ERR_INVALID_ARG;
+  if (n > 0 && k > 0 && (!w || !packed)) return BNN_ERR_INVALID_ARG;
+  if (k > 0 && n > (int64_t(1) << 40) / k) return BNN_ERR_INVALID_ARG;
+  if ((w && !bnn::aligned(w, 4)) || (packed && !bnn::aligned(packed, 2)) || (scale && !bnn::aligned(scale, 4)) ||
+      !bnn::aligned(thresh_out, 4))
+    return BNN_ERR_MISALIGNED;
+  const int64_t total = n * k;
+  const int64_t cap = static_cast<int64_t>(bnn::sm_count()) * 8;
+  const int grid = static_cast<int>(n < 1 ? 1 : (n < cap ? n : cap));
+  if (mode == kModeDelta) {
+    twn_pack_rows_kernel<kModeDelta><<<grid, kRedThreads, 0, s>>>(w, n, k, nullptr, 0, total, packed, scale,
+                                                                  thresh_out, threshold);
+    return bnn::check_launch();
+  }
+  const int64_t nparts = (total + kChunk - 1) / kChunk;
+  double* partial = nullptr;
+  if (nparts > 0) {
+    BNN_TRY(cudaMallocAsync(reinterpret_cast<void**>(&partial), static_cast<size_t>(nparts) * sizeof(double), s));
+    twn_abs_partial_kernel<<<static_cast<unsigned>(nparts), kRedThreads, 0, s>>>(w, total, partial);
+    const bnn_status st = bnn::check_launch();
+    if (st != BNN_OK) {
+      cudaFreeAsync(partial, s);
+      return st;
+    }
+  }
+  twn_pack_rows_kernel<kModeAbsmean><<<grid, kRedThreads, 0, s>>>(w, n, k, partial, nparts, total, packed, scale,
+                                                                  thresh_out);
+  bnn_status st = bnn::check_launch();
+  if (partial) {
+    const cudaError_t e = cudaFreeAsync(partial, s);
+    if (st == BNN_OK && e != cudaSuccess) st = bnn::cuda_fail(e);
+  }
+  return st;
 }

@@ -140,3 +140,48 @@ def test_workload_ternary_full(bnn, m):
     ref, mag = oracle.ternary_gemm(c["x_bf16"], gp, gs, m, c["n"], c["k"])
     worst = assert_ternary_close(out.cpu().numpy(), ref, mag, f"cfg5 m={m}")
     print(f"cfg5 m={m}: worst |err|/mag = {worst:.3e}")
+
+
+@pytest.mark.parametrize("n,k", [(7, 4096), (64, 1000), (300, 4096 + 7), (1, 1)])
+def test_pack_mode_absmean_matches_oracle(bnn, n, k):
+    w = synth.normal_f32(n * 3 + k, 7, (n, k))
+    packed, scale, gamma = bnn.bnn_ternary_pack_mode(to_dev_f32(w), bnn.TERNARY_ABSMEAN)
+    torch.cuda.synchronize()
+    ot, os_, og = oracle.absmean_ternarize(w)
+    gg = np.float32(gamma.cpu().numpy()[0])
+    if gg == og:
+        assert_bits_equal(host_u16(packed), oracle.base3_pack(ot), f"absmean {n}x{k} words")
+        assert _ulp_diff(scale.cpu().numpy(), os_) <= 1
+    else:  # float64 sums in another order rounded to a neighbouring float32
+        assert abs(float(gg) - float(og)) <= 2 * np.spacing(np.float32(og))
+
+
+@pytest.mark.parametrize("F", [0.0, 0.5, 1.3])
+def test_pack_mode_delta_matches_oracle(bnn, F):
+    w = synth.normal_f32(5, 8, (33, 777))
+    w[0, :3] = [0.5, -0.5, 1.3]  # ties at the thresholds
+    packed, scale, thr = bnn.bnn_ternary_pack_mode(to_dev_f32(w), bnn.TERNARY_DELTA, F)
+    torch.cuda.synchronize()
+    ot, os_ = oracle.delta_ternarize(w, np.float32(F))
+    assert float(thr.cpu()[0]) == np.float32(F)
+    assert_bits_equal(host_u16(packed), oracle.base3_pack(ot), f"delta F={F}")
+    assert _ulp_diff(scale.cpu().numpy(), os_) <= 1
+
+
+def test_pack_mode_twn_is_bnn_ternary_pack(bnn):
+    w = to_dev_f32(synth.normal_f32(6, 9, (40, 500)))
+    a = bnn.bnn_ternary_pack(w)
+    b = bnn.bnn_ternary_pack_mode(w, bnn.TERNARY_TWN)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_pack_mode_golden_absmean_ties(bnn):
+    w = np.array([[1, -1, 3, -3]], np.float32)   # gamma = 2: +-0.5 ties round to 0, +-1.5 clip to +-1
+    packed, scale, gamma = bnn.bnn_ternary_pack_mode(to_dev_f32(w), bnn.TERNARY_ABSMEAN)
+    t, _ = oracle.base3_unpack(host_u16(packed), 4)
+    assert t.tolist() == [[0, 0, 1, -1]] and float(gamma.cpu()[0]) == 2.0 and float(scale.cpu()[0]) == 3.0
+    with pytest.raises(bnn.BnnError):
+        bnn.bnn_ternary_pack_mode(to_dev_f32(w), 7)
+    with pytest.raises(bnn.BnnError):
+        bnn.bnn_ternary_pack_mode(to_dev_f32(w), bnn.TERNARY_DELTA, -1.0)

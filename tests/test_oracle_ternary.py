@@ -197,3 +197,65 @@ def test_twn_steps_compose():
     # a larger threshold can only zero more trits
     t3, _ = oracle.twn_apply(w, np.float32(d * 2))
     assert np.all((t3 == 0) | (t3 == t)) and (t3 == 0).sum() >= (t == 0).sum()
+
+
+def _mode_cases():
+    lines = list(golden_lines("absmean_delta_small.txt"))
+    i = 0
+    while i < len(lines):
+        _, name, rows, cols, param = lines[i].split()
+        rows, cols = int(rows), int(cols)
+        w = np.array([[float(v) for v in lines[i + 1 + r].split()] for r in range(rows)], np.float32)
+        th = int(lines[i + 1 + rows].split()[1], 16)
+        tr, sc = [], []
+        for r in range(rows):
+            a, b = lines[i + 2 + rows + r].split("|")
+            tr.append([int(v) for v in a.split()])
+            sc.append(float(b))
+        yield name, w, (None if param == "-" else np.float32(param)), th, np.array(tr, np.int8), np.array(sc, np.float32)
+        i += 2 + 2 * rows
+
+
+@pytest.mark.parametrize("case", list(_mode_cases()), ids=lambda c: c[0])
+def test_absmean_and_delta_golden(case):
+    name, w, param, th_bits, trits, scales = case
+    if param is None:
+        t, s, g = oracle.absmean_ternarize(w)
+        assert int(np.array([g], np.float32).view(np.uint32)[0]) == th_bits
+    else:
+        assert int(np.array([param], np.float32).view(np.uint32)[0]) == th_bits
+        t, s = oracle.delta_ternarize(w, param)
+    assert np.array_equal(t, trits)
+    assert np.array_equal(s, scales)
+
+
+def test_absmean_is_roundclip_of_numpy():
+    """The absmean trits equal numpy's own RoundClip (np.round is half-to-even)
+    of the float32 quotient, with gamma the float64 mean rounded to float32."""
+    w = synth.normal_f32(11, 4, (64, 777))
+    t, s, g = oracle.absmean_ternarize(w)
+    g_np = np.float32(np.abs(w.astype(np.float64)).mean())
+    assert g == g_np
+    q = (w / g_np).astype(np.float32)
+    want = np.clip(np.round(q), -1, 1).astype(np.int8)
+    assert np.array_equal(t, want)
+    _, s_ls = oracle.twn_apply(w, np.float32(0))  # same LS rule, given the trits below
+    kept = np.abs(w.astype(np.float64)) * (t != 0)
+    cnt = (t != 0).sum(axis=1)
+    want_s = np.where(cnt > 0, kept.sum(axis=1) / np.maximum(cnt, 1), 0).astype(np.float32)
+    assert np.array_equal(s, want_s)
+
+
+def test_absmean_gaussian_statistics():
+    """For N(0,1): gamma -> sqrt(2/pi) and the zero fraction -> erf(gamma / (2 sqrt 2))."""
+    w = synth.normal_f32(12, 5, (512, 4096))
+    t, s, g = oracle.absmean_ternarize(w)
+    assert abs(float(g) - math.sqrt(2 / math.pi)) < 3e-3
+    assert abs(float((t == 0).mean()) - math.erf(float(g) / (2 * math.sqrt(2)))) < 3e-3
+
+
+def test_delta_mode_equals_threshold_rule():
+    w = synth.normal_f32(13, 6, (9, 100))
+    F = np.float32(0.8)
+    t, s = oracle.delta_ternarize(w, F)
+    assert np.array_equal(t, (np.sign(w) * (np.abs(w) > F)).astype(np.int8))
