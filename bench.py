@@ -306,6 +306,10 @@ def run_headline(cu: Cuda, args, dist: Dist):
     # the same GEMM with the popcount kernel family (for its own roofline)
     popc_args = [a[:-1] + (C.c_int(1), a[-1]) for a in gemm_args]
     res["gemm_popc_ms"] = graph_time(cu, lambda i: lib.bnn_binary_gemm_algo(*popc_args[i % R]), 200, cap)
+    tc_args = [a[:-1] + (C.c_int(3), a[-1]) for a in gemm_args]
+    res["gemm_tc_ms"] = graph_time(cu, lambda i: lib.bnn_binary_gemm_algo(*tc_args[i % R]), 200, cap)
+    mma_args = [a[:-1] + (C.c_int(2), a[-1]) for a in gemm_args]
+    res["gemm_mma_ms"] = graph_time(cu, lambda i: lib.bnn_binary_gemm_algo(*mma_args[i % R]), 200, cap)
     # each kernel alone, back to back in a graph without events in between
     res["pack_graph_ms"] = graph_time(cu, lambda i: lib.bnn_pack_signs(*pack_args[i % R]), 200, cap)
     res["gemm_graph_ms"] = graph_time(cu, lambda i: lib.bnn_binary_gemm(*gemm_args[i % R]), 200, cap)
@@ -505,13 +509,14 @@ def wl_gemm_large(cu, args, P, st, s, popc_peak_macs):
     o = torch.empty((m, n), dtype=torch.float32, device=dev)
     macs = float(m) * n * k
     res4 = {}
-    for algo, name in ((2, "mma_s8"), (1, "popc")):
+    for algo, name in ((3, "tc"), (2, "mma_s8"), (1, "popc")):
         with ClockSampler(dev.index) as clk:
             ms = graph_time(cu, lambda i: lib.bnn_binary_gemm_algo(P(xp), P(wp), P(al), m, n, k, P(d), P(o), algo, s),
                             10 if algo == 2 else 5, st)
         res4[name] = dict(ms=ms, gmacs=macs / (ms * 1e-3) / 1e9, clocks=clk.summary())
     res4["popc"]["frac_of_popc_peak"] = res4["popc"]["gmacs"] / 1e3 / popc_peak_macs
     res4["mma_s8"]["x_popc_peak"] = res4["mma_s8"]["gmacs"] / 1e3 / popc_peak_macs
+    res4["tc"]["x_popc_peak"] = res4["tc"]["gmacs"] / 1e3 / popc_peak_macs
     out["gemm_large_8192"] = res4
     del d, o, xp, wp
     return out
@@ -697,6 +702,8 @@ def main():
                                         f"word-steps/clk/SM"},
         "kernels_ms": {"bnn_pack_signs": res["pack_ms"], "bnn_binary_gemm": res["gemm_ms"],
                        "bnn_binary_gemm_algo(POPC)": res["gemm_popc_ms"],
+                       "bnn_binary_gemm_algo(TC)": res["gemm_tc_ms"],
+                       "bnn_binary_gemm_algo(MMA_S8)": res["gemm_mma_ms"],
                        "bnn_pack_signs(graph, alone)": res["pack_graph_ms"],
                        "bnn_binary_gemm(graph, alone)": res["gemm_graph_ms"]},
         "cpu_baseline": cpu,

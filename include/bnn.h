@@ -106,8 +106,10 @@ typedef enum {
   BNN_ALGO_AUTO = 0,   /* what bnn_binary_gemm uses: POPC GEMV for m <= 8, MMA_S8 otherwise */
   BNN_ALGO_POPC = 1,   /* XOR + 64-bit popcount on the integer pipe (skinny GEMV for m <= 8,
                           register-tiled GEMM otherwise) */
-  BNN_ALGO_MMA_S8 = 2  /* packed bits expanded in registers to +-1 int8 and summed exactly by
-                          m16n8k32 s8 tensor-core MMAs into int32 */
+  BNN_ALGO_MMA_S8 = 2, /* packed bits expanded in registers to 0/-1 int8 fragments of
+                          m16n8k32 s8 mma.sync; popc(a AND b) summed exactly in int32 */
+  BNN_ALGO_TC = 3      /* packed bits expanded to +-1 int8 in shared memory and summed exactly
+                          by tcgen05.mma kind::i8 into an int32 tensor-memory accumulator */
 } bnn_binary_algo;
 
 /*
@@ -219,6 +221,29 @@ bnn_status bnn_ternary_pack_noalloc(const float* w, int64_t n, int64_t k, uint16
  */
 bnn_status bnn_ternary_gemm(const uint16_t* x_bf16, const uint16_t* packed, const float* scale,
                             int64_t m, int64_t n, int64_t k, float* out, cudaStream_t s);
+
+/* Number of bounded device-side waits that ran out since the last reset
+ * (a kernel that gives up a wait leaves its outputs unspecified and counts it
+ * here); reset != 0 clears the count.  Synchronous; -1 if the query fails.
+ * No counterpart on the pages: a diagnostic of this library. */
+int bnn_device_error_count(int reset);
+
+/* Kernel family for bnn_ternary_gemm_algo.  Results agree within the
+ * tolerance of bnn_ternary_gemm (float32 accumulation in different orders). */
+typedef enum {
+  BNN_TALGO_AUTO = 0,        /* what bnn_ternary_gemm uses: CUDA-core GEMV for m <= 8, MMA otherwise */
+  BNN_TALGO_CUDA_CORES = 1,  /* CUDA-core GEMV kernels (m <= 8 only; BNN_ERR_UNSUPPORTED beyond) */
+  BNN_TALGO_MMA = 2,         /* trits decoded to bf16 tiles, bf16 mma.sync m16n8k16 */
+  BNN_TALGO_TC = 3           /* trits decoded to bf16 tiles, tcgen05.mma kind::f16 into tensor memory */
+} bnn_ternary_algo;
+
+/*
+ * bnn_ternary_gemm_algo -- bnn_ternary_gemm with an explicit kernel family
+ * (a bnn_ternary_algo; BNN_ERR_INVALID_ARG for an unknown one).  Same
+ * arguments, outputs and errors as bnn_ternary_gemm.
+ */
+bnn_status bnn_ternary_gemm_algo(const uint16_t* x_bf16, const uint16_t* packed, const float* scale,
+                                 int64_t m, int64_t n, int64_t k, float* out, int algo, cudaStream_t s);
 
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* bnn_status_string(bnn_status st);

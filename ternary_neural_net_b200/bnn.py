@@ -37,6 +37,7 @@ _SIGS = {
     "bnn_ternary_pack": [_vp, _i64, _i64, _vp, _vp, _vp, _vp],
     "bnn_ternary_gemm": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
     "bnn_ternary_pack_mode": [_vp, _i64, _i64, _int, C.c_float, _vp, _vp, _vp, _vp],
+    "bnn_ternary_gemm_algo": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _int, _vp],
     "bnn_ternary_pack_noalloc": [_vp, _i64, _i64, _vp, _vp, _vp, _vp],
 }
 for _name, _args in _SIGS.items():
@@ -47,13 +48,21 @@ _lib.bnn_status_string.argtypes = [_int]
 _lib.bnn_status_string.restype = C.c_char_p
 _lib.bnn_last_cuda_error.argtypes = []
 _lib.bnn_last_cuda_error.restype = _int
+_lib.bnn_device_error_count.argtypes = [_int]
+_lib.bnn_device_error_count.restype = _int
 
 # Exported symbol names, as declared in include/bnn.h.
-ABI_SYMBOLS = tuple(_SIGS) + ("bnn_status_string", "bnn_last_cuda_error")
+ABI_SYMBOLS = tuple(_SIGS) + ("bnn_status_string", "bnn_last_cuda_error", "bnn_device_error_count")
+
+
+def device_error_count(reset: bool = False) -> int:
+    """Bounded device-side waits that ran out since the last reset (0 when all is well)."""
+    return int(_lib.bnn_device_error_count(1 if reset else 0))
 
 BNN_OK, BNN_ERR_INVALID_ARG, BNN_ERR_MISALIGNED, BNN_ERR_CUDA, BNN_ERR_UNSUPPORTED = range(5)
-ALGO_AUTO, ALGO_POPC, ALGO_MMA_S8 = 0, 1, 2
+ALGO_AUTO, ALGO_POPC, ALGO_MMA_S8, ALGO_TC = 0, 1, 2, 3
 TERNARY_TWN, TERNARY_ABSMEAN, TERNARY_DELTA = 0, 1, 2
+TALGO_AUTO, TALGO_CUDA_CORES, TALGO_MMA, TALGO_TC = 0, 1, 2, 3
 MAX_K_BINARY = 1 << 24
 
 
@@ -122,7 +131,7 @@ def bnn_binary_gemm(xp: torch.Tensor, wp: torch.Tensor, alpha: torch.Tensor | No
                     want_dots: bool = True, want_out: bool = True,
                     dots: torch.Tensor | None = None, out: torch.Tensor | None = None, algo: int = ALGO_AUTO):
     """Packed XOR+popcount matmul.  Returns (dots int32 [m,n] or None, out float32 [m,n] or None).
-    `algo` selects the kernel family (ALGO_AUTO, ALGO_POPC, ALGO_MMA_S8); all are bit-identical."""
+    `algo` selects the kernel family (ALGO_AUTO, ALGO_POPC, ALGO_MMA_S8, ALGO_TC); all are bit-identical."""
     _dev(xp, "xp", torch.int64)
     _dev(wp, "wp", torch.int64)
     m, n = xp.shape[0], wp.shape[0]
@@ -182,8 +191,9 @@ def bnn_ternary_pack_mode(w: torch.Tensor, mode: int, threshold: float = 0.0):
 
 
 def bnn_ternary_gemm(x: torch.Tensor, packed: torch.Tensor, scale: torch.Tensor, k: int | None = None,
-                     out: torch.Tensor | None = None) -> torch.Tensor:
-    """bf16 [m, k] x base-3 packed [n, ceil(k/10)] -> float32 [m, n] (scale applied)."""
+                     out: torch.Tensor | None = None, algo: int = TALGO_AUTO) -> torch.Tensor:
+    """bf16 [m, k] x base-3 packed [n, ceil(k/10)] -> float32 [m, n] (scale applied).
+    `algo` selects the kernel family (TALGO_AUTO, TALGO_CUDA_CORES, TALGO_MMA, TALGO_TC)."""
     _dev(x, "x", torch.bfloat16)
     _dev(packed, "packed", torch.int16)
     _dev(scale, "scale", torch.float32, ndim=1)
@@ -195,6 +205,10 @@ def bnn_ternary_gemm(x: torch.Tensor, packed: torch.Tensor, scale: torch.Tensor,
     if out is None:
         out = torch.empty((m, n), dtype=torch.float32, device=x.device)
     _dev(out, "out", torch.float32)
-    _check(_lib.bnn_ternary_gemm(_ptr(x), _ptr(packed), _ptr(scale), m, n, k, _ptr(out), _stream(x.device)),
-           "bnn_ternary_gemm")
+    if algo == TALGO_AUTO:
+        st = _lib.bnn_ternary_gemm(_ptr(x), _ptr(packed), _ptr(scale), m, n, k, _ptr(out), _stream(x.device))
+    else:
+        st = _lib.bnn_ternary_gemm_algo(_ptr(x), _ptr(packed), _ptr(scale), m, n, k, _ptr(out), int(algo),
+                                        _stream(x.device))
+    _check(st, "bnn_ternary_gemm")
     return out

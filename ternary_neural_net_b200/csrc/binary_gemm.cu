@@ -541,7 +541,8 @@ extern "C" bnn_status bnn_binary_gemm_algo(const uint64_t* xp, const uint64_t* w
                                            int64_t m, int64_t n, int64_t k, int32_t* dots, float* out,
                                            bnn_binary_algo algo, cudaStream_t s) {
   if (m < 0 || n < 0 || k < 0 || k > BNN_MAX_K_BINARY) return BNN_ERR_INVALID_ARG;
-  if (algo != BNN_ALGO_AUTO && algo != BNN_ALGO_POPC && algo != BNN_ALGO_MMA_S8) return BNN_ERR_INVALID_ARG;
+  if (algo != BNN_ALGO_AUTO && algo != BNN_ALGO_POPC && algo != BNN_ALGO_MMA_S8 && algo != BNN_ALGO_TC)
+    return BNN_ERR_INVALID_ARG;
   if (!dots && !out) return BNN_ERR_INVALID_ARG;
   if (out && !alpha) return BNN_ERR_INVALID_ARG;
   if (m == 0 || n == 0) return BNN_OK;
@@ -554,6 +555,7 @@ extern "C" bnn_status bnn_binary_gemm_algo(const uint64_t* xp, const uint64_t* w
   const bool vec2 = (kw % 2 == 0) && bnn::aligned(xp, 16) && bnn::aligned(wp, 16);
   const int ki = static_cast<int>(k);
 
+  if (algo == BNN_ALGO_TC) return bnn::binary_gemm_tc(xp, wp, alpha, m, n, ki, kw, dots, out, s);
   if (algo == BNN_ALGO_MMA_S8 || (algo == BNN_ALGO_AUTO && m > 8)) {
     return vec2 ? dispatch_mma<2>(xp, wp, alpha, m, n, ki, kw, dots, out, s)
                 : dispatch_mma<1>(xp, wp, alpha, m, n, ki, kw, dots, out, s);

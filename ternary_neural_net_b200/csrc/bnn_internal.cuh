@@ -38,6 +38,17 @@ cudaError_t ensure_smem(Kernel kern, size_t bytes) {
   return ensure_smem_raw(reinterpret_cast<const void*>(kern), bytes);
 }
 
+// Tensor-core (tcgen05 kind::i8) binary GEMM, in binary_gemm_tc.cu.
+bnn_status binary_gemm_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha, int64_t m, int64_t n, int k,
+                          int kw, int32_t* dots, float* out, cudaStream_t s);
+
+// Bounded waits that ran out in the ternary tensor-core kernel (reset != 0 clears).
+int ternary_tc_error_count(int reset);
+
+// Tensor-core (tcgen05 kind::f16) ternary GEMM, in ternary_gemm_tc.cu.
+bnn_status ternary_gemm_tc(const uint16_t* x_bf16, const uint16_t* packed, const float* scale, int64_t m, int64_t n,
+                           int64_t k, float* out, cudaStream_t s);
+
 }  // namespace bnn
 
 #define BNN_TRY(expr)                              \

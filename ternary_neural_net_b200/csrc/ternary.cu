@@ -539,8 +539,11 @@ extern "C" bnn_status bnn_ternary_pack(const float* w, int64_t n, int64_t k, uin
   return st;
 }
 
-extern "C" bnn_status bnn_ternary_gemm(const uint16_t* x_bf16, const uint16_t* packed, const float* scale,
-                                       int64_t m, int64_t n, int64_t k, float* out, cudaStream_t s) {
+extern "C" bnn_status bnn_ternary_gemm_algo(const uint16_t* x_bf16, const uint16_t* packed, const float* scale,
+                                            int64_t m, int64_t n, int64_t k, float* out, int algo, cudaStream_t s) {
+  if (algo != BNN_TALGO_AUTO && algo != BNN_TALGO_CUDA_CORES && algo != BNN_TALGO_MMA && algo != BNN_TALGO_TC)
+    return BNN_ERR_INVALID_ARG;
+  if (algo == BNN_TALGO_CUDA_CORES && m > 8) return BNN_ERR_UNSUPPORTED;
   if (m < 0 || n < 0 || k < 0) return BNN_ERR_INVALID_ARG;
   if (m == 0 || n == 0) return BNN_OK;
   if (!scale || !out || (k > 0 && (!x_bf16 || !packed))) return BNN_ERR_INVALID_ARG;
@@ -548,7 +551,8 @@ extern "C" bnn_status bnn_ternary_gemm(const uint16_t* x_bf16, const uint16_t* p
       !bnn::aligned(out, 4))
     return BNN_ERR_MISALIGNED;
   const int64_t kt = bnn::words10(k);
-  if (m == 1 && kt > 0 && bnn::aligned(packed, 16) && lut_smem_bytes(kt) <= 200 * 1024) {
+  if (algo == BNN_TALGO_TC) return bnn::ternary_gemm_tc(x_bf16, packed, scale, m, n, k, out, s);
+  if (algo != BNN_TALGO_MMA && m == 1 && kt > 0 && bnn::aligned(packed, 16) && lut_smem_bytes(kt) <= 200 * 1024) {
     const size_t smem = lut_smem_bytes(kt);
     auto kern = ternary_gemv_lut_kernel<kLutSlices>;
     BNN_TRY(bnn::ensure_smem(kern, smem));
@@ -559,7 +563,7 @@ extern "C" bnn_status bnn_ternary_gemm(const uint16_t* x_bf16, const uint16_t* p
                                                   slice_words, out);
     return bnn::check_launch();
   }
-  if (m <= 8) {
+  if (algo != BNN_TALGO_MMA && m <= 8) {
     const int64_t warps_per_block = 8;
     const int64_t blocks_needed = (n + warps_per_block - 1) / warps_per_block;
     const int64_t cap = static_cast<int64_t>(bnn::sm_count()) * 8;
@@ -584,6 +588,11 @@ extern "C" bnn_status bnn_ternary_gemm(const uint16_t* x_bf16, const uint16_t* p
     ternary_gemm_mma_kernel<false><<<grid, kTThreads, smem, s>>>(x_bf16, packed, scale, m, n, k, kt, slice_words, out);
   }
   return bnn::check_launch();
+}
+
+extern "C" bnn_status bnn_ternary_gemm(const uint16_t* x_bf16, const uint16_t* packed, const float* scale,
+                                       int64_t m, int64_t n, int64_t k, float* out, cudaStream_t s) {
+  return bnn_ternary_gemm_algo(x_bf16, packed, scale, m, n, k, out, BNN_TALGO_AUTO, s);
 }
 
 // ---------------------------------------------------------------------------

@@ -51,7 +51,7 @@ def test_pack_empty(bnn):
     assert out.shape == (4, 0)
 
 
-def _gemm_case(bnn, m, n, k, seed, offset_words=0, algos=(0, 1, 2)):
+def _gemm_case(bnn, m, n, k, seed, offset_words=0, algos=(0, 1, 2, 3)):
     xp = synth.fair_coin_words(seed, 1, m, k)
     wp = synth.fair_coin_words(seed, 2, n, k)
     alpha = synth.uniform_f32(seed, 3, (n,), -1.0, 2.0)
@@ -95,7 +95,7 @@ def test_unaligned_operands_use_the_8_byte_path(bnn, m, n, k):
 
 def test_k_zero_gives_zero_and_alpha_times_zero(bnn):
     for m in (1, 20):
-        for algo in (0, 1, 2):
+        for algo in (0, 1, 2, 3):
             xp = torch.empty((m, 0), dtype=torch.int64, device="cuda")
             wp = torch.empty((5, 0), dtype=torch.int64, device="cuda")
             alpha = to_dev_f32(np.array([1.0, -2.0, 0.0, 3.5, 1e-3], np.float32))
@@ -151,7 +151,7 @@ def test_workload_gemv_small_full(bnn):
     assert_bits_equal(out.cpu().numpy(), want_o, "cfg1 out")
 
 
-@pytest.mark.parametrize("algo", [0, 1, 2])
+@pytest.mark.parametrize("algo", [0, 1, 2, 3])
 def test_workload_gemm_fused_pack(bnn, algo):
     c = synth.gemm_fused_pack(1)
     xp = bnn.bnn_pack_signs(to_dev_f32(c["x"]))
@@ -176,7 +176,7 @@ def test_workload_gemv_ffn(bnn):
     assert_bits_equal(out.cpu().numpy(), want_o, "cfg3 out")
 
 
-@pytest.mark.parametrize("algo", [0, 1])
+@pytest.mark.parametrize("algo", [0, 1, 3])
 def test_workload_gemm_large(bnn, algo):
     c = synth.gemm_large(1)
     dots, out = bnn.bnn_binary_gemm(to_dev_u64(c["xp"]), to_dev_u64(c["wp"]), to_dev_f32(c["alpha"]), c["k"],
@@ -202,7 +202,7 @@ def test_algos_agree_bitwise_on_random_shapes(bnn):
         xp = to_dev_u64(synth.fair_coin_words(int(m + n + k), 1, m, k))
         wp = to_dev_u64(synth.fair_coin_words(int(m + n + k), 2, n, k))
         alpha = to_dev_f32(synth.uniform_f32(3, 3, (n,), -2.0, 2.0))
-        res = [bnn.bnn_binary_gemm(xp, wp, alpha, k, algo=a) for a in (0, 1, 2)]
+        res = [bnn.bnn_binary_gemm(xp, wp, alpha, k, algo=a) for a in (0, 1, 2, 3)]
         for d, o in res[1:]:
             assert torch.equal(d, res[0][0]) and torch.equal(o.view(torch.int32), res[0][1].view(torch.int32))
 
@@ -211,3 +211,9 @@ def test_unknown_algo_rejected(bnn):
     xp = torch.zeros((2, 1), dtype=torch.int64, device="cuda")
     with pytest.raises(bnn.BnnError):
         bnn.bnn_binary_gemm(xp, xp, None, 64, want_out=False, algo=7)
+
+
+def test_no_device_wait_ran_out(bnn):
+    """Every bounded wait of the tensor-core kernels completed in this run."""
+    torch.cuda.synchronize()
+    assert bnn.device_error_count() == 0

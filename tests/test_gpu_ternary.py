@@ -85,16 +85,19 @@ def test_pack_is_reproducible(bnn):
         assert torch.equal(x, y)
 
 
-def _gemm_case(bnn, m, n, k, seed, trits=None):
+def _gemm_case(bnn, m, n, k, seed, trits=None, algos=(0,)):
     rng = np.random.default_rng(seed)
     if trits is None:
         trits = rng.integers(-1, 2, (n, k)).astype(np.int8)
     packed = oracle.base3_pack(trits)
     scale = synth.uniform_f32(seed, 1, (n,), 0.25, 2.0)
     xb = synth.bf16_bits_from_f32(synth.normal_f32(seed, 2, (m, k)))
-    out = bnn.bnn_ternary_gemm(to_dev_bf16(xb), to_dev_u16(packed), to_dev_f32(scale), k)
     ref, mag = oracle.ternary_gemm(xb, packed, scale, m, n, k)
-    return assert_ternary_close(out.cpu().numpy(), ref, mag, f"ternary {m}x{n}x{k}")
+    worst = 0.0
+    for algo in algos:
+        out = bnn.bnn_ternary_gemm(to_dev_bf16(xb), to_dev_u16(packed), to_dev_f32(scale), k, algo=algo)
+        worst = max(worst, assert_ternary_close(out.cpu().numpy(), ref, mag, f"ternary {m}x{n}x{k} algo {algo}"))
+    return worst
 
 
 @pytest.mark.parametrize("m,n,k", [(1, 7, 10), (1, 100, 4096), (2, 33, 95), (4, 65, 161), (8, 64, 1000),
@@ -104,9 +107,9 @@ def test_gemv_matches_oracle(bnn, m, n, k):
 
 
 @pytest.mark.parametrize("m,n,k", [(9, 65, 161), (64, 64, 160), (64, 200, 4096), (100, 130, 1001),
-                                   (130, 70, 33), (65, 1, 10)])
+                                   (130, 70, 33), (65, 1, 10), (64, 300, 640), (1, 129, 64), (3, 140, 700)])
 def test_gemm_matches_oracle(bnn, m, n, k):
-    _gemm_case(bnn, m, n, k, seed=m * 17 + n + k)
+    _gemm_case(bnn, m, n, k, seed=m * 17 + n + k, algos=(0, 2, 3))
 
 
 @pytest.mark.parametrize("m", [1, 64])
@@ -117,7 +120,7 @@ def test_every_base3_word_decodes(bnn, m):
     trits, bad = oracle.base3_unpack(words, 590490)
     assert bad == 0
     rows = np.concatenate([trits, -trits, np.zeros_like(trits)])
-    _gemm_case(bnn, m, 3, 590490, seed=5 + m, trits=rows)
+    _gemm_case(bnn, m, 3, 590490, seed=5 + m, trits=rows, algos=(0, 3) if m > 1 else (0,))
 
 
 def test_zero_trits_give_exact_zero(bnn):
@@ -136,10 +139,12 @@ def test_workload_ternary_full(bnn, m):
     zero_frac = float((oracle.base3_unpack(gp, c["k"])[0] == 0).mean())
     print(f"cfg5: Delta={gd} zero fraction={zero_frac:.4f}")
     assert 0.40 < zero_frac < 0.45
-    out = bnn.bnn_ternary_gemm(to_dev_bf16(c["x_bf16"]), to_dev_u16(gp), to_dev_f32(gs), c["k"])
     ref, mag = oracle.ternary_gemm(c["x_bf16"], gp, gs, m, c["n"], c["k"])
-    worst = assert_ternary_close(out.cpu().numpy(), ref, mag, f"cfg5 m={m}")
-    print(f"cfg5 m={m}: worst |err|/mag = {worst:.3e}")
+    for algo in ((0,) if m == 1 else (0, 2, 3)):
+        out = bnn.bnn_ternary_gemm(to_dev_bf16(c["x_bf16"]), to_dev_u16(gp), to_dev_f32(gs), c["k"], algo=algo)
+        worst = assert_ternary_close(out.cpu().numpy(), ref, mag, f"cfg5 m={m} algo {algo}")
+        print(f"cfg5 m={m} algo {algo}: worst |err|/mag = {worst:.3e}")
+    assert bnn.device_error_count() == 0
 
 
 @pytest.mark.parametrize("n,k", [(7, 4096), (64, 1000), (300, 4096 + 7), (1, 1)])
