@@ -540,6 +540,14 @@ def wl_ternary(cu, args, P, st, s, hbm, peaks):
                                              C.c_void_p]
     ms_pack_na = time_calls(cu, lambda i: lib.bnn_ternary_pack_noalloc(P(w), n, k, P(packed), P(scale), P(delta),
                                                                         cu.s), 20, warm=3)
+    lib.bnn_ternary_pack_mode.argtypes = [C.c_void_p, C.c_int64, C.c_int64, C.c_int, C.c_float, C.c_void_p,
+                                          C.c_void_p, C.c_void_p, C.c_void_p]
+    ms_modes = {}
+    for mode, name, thr in ((1, "absmean", 0.0), (2, "delta", 0.5)):
+        ms_modes[name] = time_calls(cu, lambda i: lib.bnn_ternary_pack_mode(P(w), n, k, mode, thr, P(packed), P(scale),
+                                                                            P(delta), cu.s), 10, warm=2)
+    # the TWN pack is what the layer below uses
+    lib.bnn_ternary_pack_noalloc(P(w), n, k, P(packed), P(scale), P(delta), cu.s)
     del w
     pbytes = n * kt * 2
     R = rotation_copies(pbytes)
@@ -550,13 +558,21 @@ def wl_ternary(cu, args, P, st, s, hbm, peaks):
     ms1 = graph_time(cu, lambda i: lib.bnn_ternary_gemm(P(xb), P(PK[i % R]), P(scale), 1, n, k, P(o1), s), 300, st)
     ms64 = graph_time(cu, lambda i: lib.bnn_ternary_gemm(P(xb), P(PK[i % R]), P(scale), 64, n, k, P(o64), s), 100,
                       st)
+    lib.bnn_ternary_gemm_algo.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int64, C.c_int64, C.c_int64,
+                                          C.c_void_p, C.c_int, C.c_void_p]
+    ms64_alg = {}
+    for algo, name in ((2, "mma"), (3, "tc")):
+        ms64_alg[name] = graph_time(
+            cu, lambda i: lib.bnn_ternary_gemm_algo(P(xb), P(PK[i % R]), P(scale), 64, n, k, P(o64), algo, s), 100, st)
     alg1 = pbytes + k * 2 + n * 4 + n * 4
     flops64 = 2.0 * 64 * n * k
     out["ternary_n11008_k4096"] = dict(
-        pack_ms=ms_pack, pack_noalloc_ms=ms_pack_na, pack_gbs=(2 * n * k * 4 + pbytes) / (ms_pack_na * 1e-3) / 1e9,
+        pack_ms=ms_pack, pack_noalloc_ms=ms_pack_na, pack_mode_ms=ms_modes, pack_gbs=(2 * n * k * 4 + pbytes) / (ms_pack_na * 1e-3) / 1e9,
         m1_us=ms1 * 1e3, m1_gbs=alg1 / (ms1 * 1e-3) / 1e9,
         m1_frac_of_hbm=alg1 / (ms1 * 1e-3) / 1e9 / hbm,
         m64_us=ms64 * 1e3, m64_tflops=flops64 / (ms64 * 1e-3) / 1e12,
+        m64_us_by_algo={a: v * 1e3 for a, v in ms64_alg.items()},
+        m64_tflops_by_algo={a: flops64 / (v * 1e-3) / 1e12 for a, v in ms64_alg.items()},
         m64_frac_of_bf16=flops64 / (ms64 * 1e-3) / 1e12 / peaks["bf16_tflops"], rotation=R)
     return out
 
