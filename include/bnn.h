@@ -103,13 +103,16 @@ bnn_status bnn_binary_gemm(const uint64_t* xp, const uint64_t* wp, const float* 
 
 /* Kernel family for bnn_binary_gemm_algo.  All give bit-identical results. */
 typedef enum {
-  BNN_ALGO_AUTO = 0,   /* what bnn_binary_gemm uses: POPC GEMV for m <= 8, MMA_S8 otherwise */
+  BNN_ALGO_AUTO = 0,   /* what bnn_binary_gemm uses: POPC GEMV for m <= 8, MMA_S8 for
+                          9 <= m <= 63, TC for m >= 64 */
   BNN_ALGO_POPC = 1,   /* XOR + 64-bit popcount on the integer pipe (skinny GEMV for m <= 8,
                           register-tiled GEMM otherwise) */
   BNN_ALGO_MMA_S8 = 2, /* packed bits expanded in registers to 0/-1 int8 fragments of
                           m16n8k32 s8 mma.sync; popc(a AND b) summed exactly in int32 */
-  BNN_ALGO_TC = 3      /* packed bits expanded to +-1 int8 in shared memory and summed exactly
-                          by tcgen05.mma kind::i8 into an int32 tensor-memory accumulator */
+  BNN_ALGO_TC = 3      /* packed bits expanded to 0/1 bytes in shared memory; tcgen05.mma
+                          kind::i8 sums popc(a AND b) exactly into an int32 tensor-memory
+                          accumulator, and k - 2 popc(a) - 2 popc(b) + 4 popc(a AND b) is
+                          the dot */
 } bnn_binary_algo;
 
 /*

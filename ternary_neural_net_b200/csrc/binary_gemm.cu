@@ -555,7 +555,10 @@ extern "C" bnn_status bnn_binary_gemm_algo(const uint64_t* xp, const uint64_t* w
   const bool vec2 = (kw % 2 == 0) && bnn::aligned(xp, 16) && bnn::aligned(wp, 16);
   const int ki = static_cast<int>(k);
 
-  if (algo == BNN_ALGO_TC) return bnn::binary_gemm_tc(xp, wp, alpha, m, n, ki, kw, dots, out, s);
+  // AUTO: tcgen05 from 64 activation rows up (measured faster than mma.sync from
+  // the 64 x 4096 x 4096 layer to 8192^3), mma.sync for 9..63 rows, GEMV below.
+  if (algo == BNN_ALGO_TC || (algo == BNN_ALGO_AUTO && m >= 64))
+    return bnn::binary_gemm_tc(xp, wp, alpha, m, n, ki, kw, dots, out, s);
   if (algo == BNN_ALGO_MMA_S8 || (algo == BNN_ALGO_AUTO && m > 8)) {
     return vec2 ? dispatch_mma<2>(xp, wp, alpha, m, n, ki, kw, dots, out, s)
                 : dispatch_mma<1>(xp, wp, alpha, m, n, ki, kw, dots, out, s);

@@ -1,28 +1,46 @@
 // bnn_binary_gemm on the 5th-generation tensor cores (tcgen05, sm_100a).
 //
 // "Binary Math Effectiveness -- why / how / when", section 1: for +-1 vectors
-// packed with bit 1 = -1, <x,w> = sum_e x_e w_e = n - 2 popcount(x XOR w).
-// +-1 is exact in int8 and the sum is exact in int32, so an int8 MMA over the
-// expanded signs computes the same dot as the XOR + popcount identity.
+// packed with bit 1 = -1, <x,w> = n - 2 popcount(x XOR w).  Writing a and b
+// for the bits of x and w, popcount(x XOR w) = pa + pb - 2 popcount(a AND b),
+// so <x,w> = k - 2 pa - 2 pb + 4 popcount(a AND b), where pa and pb are the
+// row popcounts.  popcount(a AND b) is the dot product of the rows' bits as
+// 0/1 bytes, which an int8 MMA sums exactly into int32.  Pad bits are 0 in
+// both rows and so add nothing to any of the three counts.
 //
-// Per CTA: a 128 x BN output tile (UMMA M = 128 activation rows, N = BN weight
-// rows), K in stages of 128 bits.  Every thread owns one row of the stacked
-// (activation, weight) tile: it loads the row's two 64-bit words of the stage
-// (prefetched kTcPre stages ahead in registers), expands the 128 signs to 128
-// +-1 bytes in the 128-byte-swizzled K-major shared-memory layout the tensor
-// core reads (per 4 bytes: a shift, a sign-replicating byte permute and an
-// OR), and one thread issues 4 tcgen05.mma.kind::i8 (K = 32 each) into an
-// int32 accumulator in tensor memory, committing to the stage's mbarrier so
-// the buffer is refilled only after the tensor core has read it.  Any fixed
-// bijection between bits and k-slots gives the same dot when both operands
-// use it; the one used makes every 4-byte group a byte permute of one
-// shifted 32-bit half-word.  Bits past k (pad bits and zero-filled words)
-// are 0 in both operands and each adds exactly +1; the epilogue subtracts
-// their count, reads the accumulator back with tcgen05.ld and applies alpha.
+// Tile: UMMA M = 128 weight rows (operand A) x N = BN activation rows (operand
+// B), K in stages of 128 bits.  Roles inside a CTA:
+//   - producer threads, two per row of the stacked (weight, activation) tile,
+//     each owning one 64-bit word of the row per stage: load it (prefetched
+//     kPre stages ahead in registers), count its bits, and write its 64 0/1
+//     bytes (per 4 bytes a shift and an AND) in the 128-byte-swizzled K-major
+//     layout the tensor core reads, then arrive on the stage's "full" mbarrier;
+//   - one MMA thread: waits for "full", issues 4 tcgen05.mma.kind::i8 (K = 32)
+//     into the int32 accumulator in tensor memory and commits to the stage's
+//     "empty" mbarrier, which the producers wait on before refilling it;
+//   - the epilogue (warps 0-7; warp w reads tensor-memory lanes 32(w%4).. and
+//     half w/4 of the columns): tcgen05.ld, the popcount correction, alpha,
+//     and stores in which the 32 lanes of a warp write 32 consecutive weight
+//     columns of one output row.
+// Any bijection between the 128 bits and the 128 k-slots of a stage gives the
+// same sum when both operands use it; here byte j of word s of 16-byte chunk
+// 2h+q holds bit 32h + 8j + 4q + s.
+// Narrow tiles (BN = 64) keep 96 KB of stages so that two CTAs share an SM:
+// the producers' shift/AND/store chains need many warps to hide their latency.
 //
-// Every wait on an mbarrier is bounded; a wait that runs out sets a
-// device-side error count (bnn_device_error_count) and the CTA drains its
-// MMAs (again bounded), frees its tensor memory and returns.
+// Split K: a cluster of KS CTAs shares one output tile, each taking a
+// contiguous share of the stages.  Each CTA turns its accumulator into its
+// share of the dot (-2 pa - 2 pb + 4 S over its stages) and stores it straight
+// into the shared memory of the CTA that owns that output row (distributed
+// shared memory); CTA r adds the KS shares of its BN/KS output rows and writes
+// them.  Integer addition makes the result independent of the order.
+//
+// Every wait on an mbarrier is bounded.  A wait that runs out bumps a
+// device-side error count (bnn_device_error_count) and raises a CTA-wide abort
+// flag that ends the other waits; the CTA then skips its stores, waits
+// (bounded) for the MMAs it issued, frees its tensor memory and returns.
+#include <cooperative_groups.h>
+
 #include "bnn_internal.cuh"
 
 // Bounded waits that ran out in this file's kernels (read by bnn_device_error_count).
@@ -30,9 +48,8 @@ __device__ unsigned int g_bnn_device_errors = 0;
 
 namespace {
 
-constexpr int kTcStages = 4;
-constexpr int kTcPre = 8;                  // stages of words prefetched in registers
-constexpr int kTcBM = 128;
+constexpr int kTm = 128;                   // weight rows per tile (UMMA M)
+constexpr int kPre = 8;                    // stages of packed words prefetched in registers
 constexpr uint32_t kSpinLimit = 1u << 24;  // bounded mbarrier waits
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -51,59 +68,118 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
   return d;
 }
 
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait; false when it ran out (counted, abort raised) or when another
+// thread of the CTA raised the abort flag.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
   for (uint32_t it = 0; it < kSpinLimit; ++it) {
-    uint32_t ok;
-    asm volatile(
-        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    if (ok) return true;
+    if (mbar_try(bar, parity)) return true;
+    if ((it & 255u) == 255u && *abort_flag) return false;
   }
+  *abort_flag = 1;
+  atomicAdd(&g_bnn_device_errors, 1u);
   return false;
 }
 
-// 4 bytes, byte j = -1 where bit 8j+7-s of w is set, else +1.
-__device__ __forceinline__ uint32_t pm1_bytes(uint32_t w, int s) {
-  uint32_t r;
-  asm("prmt.b32 %0, %1, %1, 0xBA98;\n" : "=r"(r) : "r"(w << s));
-  return r | 0x01010101u;
+// Bounded wait that ignores the abort flag (used for the final drain).
+__device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity) {
+  for (uint32_t it = 0; it < kSpinLimit; ++it)
+    if (mbar_try(bar, parity)) return true;
+  atomicAdd(&g_bnn_device_errors, 1u);
+  return false;
 }
 
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
+}
+
+// 32 columns of this warp's 32 tensor-memory lanes
+__device__ __forceinline__ void tmem_ld32(uint32_t addr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(addr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+}
+
+// operand stages per CTA: 4 x 24 KB for BN = 64 (two CTAs per SM), 4 x 48 KB for BN = 256
 template <int BN>
-__global__ void __launch_bounds__(kTcBM + BN, 1)
+__host__ __device__ constexpr int stages_for() {
+  return 4;
+}
+template <int BN>
+__host__ __device__ constexpr int stage_smem() {
+  return stages_for<BN>() * (kTm + BN) * 128;
+}
+template <int BN>
+__host__ __device__ constexpr int threads_for() {
+  return 2 * (kTm + BN) + 32;
+}
+
+// grid: x = KS * (weight tiles of 128 rows), y = activation tiles of BN rows;
+// clusters of KS CTAs along x
+template <int BN, int KS>
+__global__ void __launch_bounds__(threads_for<BN>(), BN <= 64 ? 2 : 1)
 binary_gemm_tc_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restrict__ wp,
                       const float* __restrict__ alpha, int64_t m, int64_t n, int k, int kw,
                       int32_t* __restrict__ dots, float* __restrict__ out) {
+  constexpr int S = stages_for<BN>();
+  constexpr int kRows = kTm + BN;
+  constexpr int kProducers = 2 * kRows;
+  constexpr uint32_t kStageBytes = static_cast<uint32_t>(kRows) * 128u;
+  static_assert(S >= 2, "at least two operand stages");
+  static_assert(KS == 1 || BN * kTm * 4 <= stage_smem<BN>(), "split-K shares must fit the stage memory");
+  static_assert(BN % KS == 0, "activation columns split evenly across the cluster");
+
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bars[kTcStages];
+  __shared__ __align__(8) uint64_t full_bar[S];
+  __shared__ __align__(8) uint64_t empty_bar[S];
+  __shared__ __align__(8) uint64_t done_bar;
   __shared__ uint32_t tmem_holder;
+  __shared__ volatile int abort_flag;
+  __shared__ int any_bad;    // split K: some CTA of the cluster aborted
+  __shared__ int pop_w[kTm];  // popcount of each weight row over this CTA's stages
+  __shared__ int pop_x[BN];   // popcount of each activation row over this CTA's stages
   // the 128-byte swizzle repeats every 1024 bytes of address: align the tiles to it
   uint8_t* const smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
   const int tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31;
-  const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kTcBM;
-  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * BN;
-  const int ktiles = (kw + 1) / 2;                 // 2 words (128 bits) per stage
+  const int warp = tid >> 5;
+  const int rank = KS > 1 ? static_cast<int>(blockIdx.x % KS) : 0;
+  const int64_t j0 = static_cast<int64_t>(blockIdx.x / KS) * kTm;  // first weight row
+  const int64_t i0 = static_cast<int64_t>(blockIdx.y) * BN;        // first activation row
+  const int ktiles = (kw + 1) / 2;                                 // 2 words (128 bits) per stage
+  const int share = (ktiles + KS - 1) / KS;
+  const int kb = rank * share < ktiles ? rank * share : ktiles;
+  const int ke = kb + share < ktiles ? kb + share : ktiles;
+  const int nst = ke - kb;
+  const uint32_t smem_base = smem_u32(smem);
 
-  // this thread's row of the stacked tile
-  const bool is_a = tid < kTcBM;
-  const int64_t grow = is_a ? m0 + tid : n0 + (tid - kTcBM);
-  const bool live = grow < (is_a ? m : n);
-  const uint64_t* src = (is_a ? xp : wp) + (live ? grow : 0) * static_cast<int64_t>(kw);
-  const uint32_t row_off = is_a ? tid * 128u : kTcBM * 128u * kTcStages + (tid - kTcBM) * 128u;
-  // A region: kTcStages x [128 rows x 128 B]; B region after it: kTcStages x [BN rows x 128 B]
-  const uint32_t a_stage = kTcBM * 128u, b_stage = BN * 128u;
-  const uint32_t swz = static_cast<uint32_t>(tid & 7);
-
+  for (int i = tid; i < kRows; i += blockDim.x) (i < kTm ? pop_w[i] : pop_x[i - kTm]) = 0;
   if (tid == 0) {
-    for (int i = 0; i < kTcStages; ++i)
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_u32(&bars[i])));
+    for (int i = 0; i < S; ++i) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(&full_bar[i])), "r"(kProducers));
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_u32(&empty_bar[i])));
+    }
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_u32(&done_bar)));
+    abort_flag = 0;
+    any_bad = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
-  if (warp == 0) {
+  if (warp == kProducers / 32) {  // the MMA warp owns the tensor memory
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(&tmem_holder)),
                  "r"(BN));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::);
@@ -113,141 +189,216 @@ binary_gemm_tc_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restric
   asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
   const uint32_t tmem = tmem_holder;
 
-  // instruction descriptor: D s32, A and B s8, both K-major, N = BN, M = 128
-  const uint32_t idesc = (2u << 4) | (1u << 7) | (1u << 10) | ((static_cast<uint32_t>(BN) >> 3) << 17) |
-                         ((static_cast<uint32_t>(kTcBM) >> 4) << 24);
-  const uint32_t smem_base = smem_u32(smem);
+  if (tid < kProducers) {
+    // ------------------------------------------------------------ producers
+    const int r2 = tid >> 1, part = tid & 1;  // stacked row, word of the stage
+    const bool is_w = r2 < kTm;
+    const int row = is_w ? r2 : r2 - kTm;
+    const int64_t grow = is_w ? j0 + row : i0 + row;
+    const bool live = grow < (is_w ? n : m);
+    const uint64_t* src = (is_w ? wp : xp) + (live ? grow : 0) * static_cast<int64_t>(kw) + part;
+    const uint32_t row_off = static_cast<uint32_t>(r2) * 128u;  // weight rows first, then activation rows
+    const uint32_t swz = static_cast<uint32_t>(row & 7);
 
-  // this row's words, prefetched kTcPre stages ahead into a register ring
-  // (the k-loop is unrolled by kTcPre so that every ring index is static)
-  auto fetch = [&](int kt, uint64_t& lo, uint64_t& hi) {
-    const int w0 = 2 * kt;
-    lo = (live && w0 < kw) ? __ldg(src + w0) : 0ull;
-    hi = (live && w0 + 1 < kw) ? __ldg(src + w0 + 1) : 0ull;
-  };
-  uint64_t ring_lo[kTcPre], ring_hi[kTcPre];
+    auto fetch = [&](int jj) -> uint64_t {
+      const int w = 2 * (kb + jj) + part;
+      return (live && jj < nst && w < kw) ? __ldg(src + 2 * (kb + jj)) : 0ull;
+    };
+    uint64_t ring[kPre];
 #pragma unroll
-  for (int u = 0; u < kTcPre; ++u) fetch(u, ring_lo[u], ring_hi[u]);
+    for (int u = 0; u < kPre; ++u) ring[u] = fetch(u);
 
-  bool ok = true;
-  int committed = -1;  // last stage whose MMAs were committed (uniform across the CTA)
-  for (int kt0 = 0; kt0 < ktiles && ok; kt0 += kTcPre) {
+    int my_pop = 0;
+    bool ok = true;
+    for (int js = 0; js < nst && ok; js += kPre) {
 #pragma unroll
-    for (int u = 0; u < kTcPre; ++u) {
-      const int kt = kt0 + u;
-      if (kt >= ktiles || !ok) break;
-      const int b = kt % kTcStages;
-      // the tensor core must be done with this buffer (stage kt - kTcStages)
-      const bool free_ok =
-          kt < kTcStages || mbar_wait(smem_u32(&bars[b]), static_cast<uint32_t>((kt / kTcStages - 1) & 1));
-      const uint64_t cur[2] = {ring_lo[u], ring_hi[u]};
-      if (kt + kTcPre < ktiles) fetch(kt + kTcPre, ring_lo[u], ring_hi[u]);
-      if (free_ok) {
-        // expand 128 bits -> 128 bytes: half-word h fills 16-byte chunks 2h and 2h+1
-        uint8_t* row_ptr = smem + row_off + (is_a ? b * a_stage : b * b_stage);
+      for (int u = 0; u < kPre; ++u) {
+        const int j = js + u;
+        if (j >= nst) break;
+        const int b = j % S;
+        // refill only after the tensor core has read the previous fill of this buffer
+        if (j >= S && !mbar_wait(smem_u32(&empty_bar[b]), static_cast<uint32_t>((j / S + 1) & 1), &abort_flag)) {
+          ok = false;
+          break;
+        }
+        const uint64_t cw = ring[u];
+        ring[u] = fetch(j + kPre);
+        my_pop += __popcll(cw);
+        uint8_t* dst = smem + b * kStageBytes + row_off;
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const uint32_t hw = static_cast<uint32_t>(cur[h >> 1] >> (32 * (h & 1)));
+        for (int hh = 0; hh < 2; ++hh) {
+          const int h = 2 * part + hh;  // half-word of the stage's 128 bits
+          const uint32_t hw = static_cast<uint32_t>(cw >> (32 * hh));
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
             uint4 v;
-            v.x = pm1_bytes(hw, 4 * q + 0);
-            v.y = pm1_bytes(hw, 4 * q + 1);
-            v.z = pm1_bytes(hw, 4 * q + 2);
-            v.w = pm1_bytes(hw, 4 * q + 3);
+            v.x = (hw >> (4 * q + 0)) & 0x01010101u;
+            v.y = (hw >> (4 * q + 1)) & 0x01010101u;
+            v.z = (hw >> (4 * q + 2)) & 0x01010101u;
+            v.w = (hw >> (4 * q + 3)) & 0x01010101u;
             const uint32_t chunk = static_cast<uint32_t>(2 * h + q);
-            *reinterpret_cast<uint4*>(row_ptr + ((chunk ^ swz) << 4)) = v;
+            *reinterpret_cast<uint4*>(dst + ((chunk ^ swz) << 4)) = v;
+          }
+        }
+        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+        mbar_arrive(smem_u32(&full_bar[b]));
+      }
+    }
+    atomicAdd(is_w ? &pop_w[row] : &pop_x[row], my_pop);
+  } else if (tid == kProducers) {
+    // ------------------------------------------------------------ MMA issue
+    // instruction descriptor: D s32, A and B 8-bit integers (0/1 bytes read
+    // the same signed or unsigned), both K-major, N = BN, M = 128
+    const uint32_t idesc = (2u << 4) | (1u << 7) | (1u << 10) | ((static_cast<uint32_t>(BN) >> 3) << 17) |
+                           ((static_cast<uint32_t>(kTm) >> 4) << 24);
+    for (int j = 0; j < nst; ++j) {
+      const int b = j % S;
+      if (!mbar_wait(smem_u32(&full_bar[b]), static_cast<uint32_t>((j / S) & 1), &abort_flag)) break;
+      asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+      const uint64_t ad = sw128_desc(smem_base + b * kStageBytes);
+      const uint64_t bd = sw128_desc(smem_base + b * kStageBytes + kTm * 128u);  // activation rows
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+        asm volatile(
+            "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+            "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem),
+            "l"(ad + static_cast<uint64_t>(2 * kk)), "l"(bd + static_cast<uint64_t>(2 * kk)), "r"(idesc), "r"(acc));
+      }
+      asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
+                       smem_u32(&empty_bar[b]))
+                   : "memory");
+    }
+    // arrives once every MMA issued above has completed
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
+                     smem_u32(&done_bar))
+                 : "memory");
+  }
+  __syncwarp();
+
+  // -------------------------------------------------------------- epilogue
+  // every producer is past its loop (row popcounts added); the accumulator is final
+  // once done_bar completes
+  if (tid < kProducers) asm volatile("bar.sync 1, %0;\n" ::"r"(kProducers) : "memory");
+  bool drained = true;
+  if (warp < 8) {
+    drained = mbar_drain(smem_u32(&done_bar), 0u);
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+  }
+  const bool good = __syncthreads_and(drained && abort_flag == 0) != 0;
+
+  // epilogue warps 0-7: warp w reads tensor-memory lanes 32(w%4).. (weight rows)
+  // and half w/4 of the BN accumulator columns (activation rows)
+  const int erow = 32 * (warp & 3) + (tid & 31);
+  const int ecol0 = (warp >> 2) * (BN / 2);
+  const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+  if constexpr (KS == 1) {
+    if (warp < 8 && good) {
+      const int64_t jrow = j0 + erow;
+      const bool jlive = jrow < n;
+      const float a_j = (out && jlive) ? __ldg(alpha + jrow) : 0.0f;
+      const int base = k - 2 * pop_w[erow];
+      for (int c0 = ecol0; c0 < ecol0 + BN / 2; c0 += 32) {
+        uint32_t r[32];
+        if (nst > 0) {
+          tmem_ld32(taddr + static_cast<uint32_t>(c0), r);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) r[c] = 0u;
+        }
+        const int64_t rows_left = m - (i0 + c0);
+        if (jlive && rows_left > 0) {
+          const int nc = rows_left < 32 ? static_cast<int>(rows_left) : 32;
+          const int64_t off = (i0 + c0) * n + jrow;
+          int32_t* dp = dots ? dots + off : nullptr;
+          float* op = out ? out + off : nullptr;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            if (c < nc) {
+              const int32_t d = base - 2 * pop_x[c0 + c] + 4 * static_cast<int32_t>(r[c]);
+              if (dp) *dp = d;
+              if (op) *op = a_j * static_cast<float>(d);
+            }
+            dp += n;
+            op += n;
           }
         }
       }
-      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-      ok = __syncthreads_and(free_ok) != 0;  // one decision for the whole CTA
-      if (!ok) break;
-      if (tid == 0) {
-        asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-        const uint64_t ad = sw128_desc(smem_base + b * a_stage);
-        const uint64_t bd = sw128_desc(smem_base + kTcBM * 128u * kTcStages + b * b_stage);
+    }
+  } else {
+    // Split K: CTA q of the cluster owns accumulator columns [q kCols, (q+1) kCols).
+    // Every CTA pushes its share of each column to the owner's receive buffer
+    // [source rank][column][weight row] (remote stores, no round trip), then
+    // each owner adds the KS shares of its columns.
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    constexpr int kCols = BN / KS;
+    int* recv = reinterpret_cast<int*>(smem);
+    cluster.sync();  // every CTA's tensor core is done with its stage memory
+    if (tid == 0 && !good)  // this CTA's shares will be missing: no CTA of the cluster writes
+      for (int q = 0; q < KS; ++q) atomicExch(cluster.map_shared_rank(&any_bad, q), 1);
+    if (warp < 8 && good) {
+      const int base = -2 * pop_w[erow];
+      for (int c0 = ecol0; c0 < ecol0 + BN / 2; c0 += 32) {
+        uint32_t r[32];
+        if (nst > 0) {
+          tmem_ld32(taddr + static_cast<uint32_t>(c0), r);
+        } else {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint32_t acc = (kt > 0 || kk > 0) ? 1u : 0u;
-          asm volatile(
-              "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
-              "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem),
-              "l"(ad + static_cast<uint64_t>(2 * kk)), "l"(bd + static_cast<uint64_t>(2 * kk)), "r"(idesc), "r"(acc));
+          for (int c = 0; c < 32; ++c) r[c] = 0u;
         }
-        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
-                         smem_u32(&bars[b]))
-                     : "memory");
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const int col = c0 + c;
+          int* dst = cluster.map_shared_rank(recv, col / kCols);
+          dst[(rank * kCols + col % kCols) * kTm + erow] = base - 2 * pop_x[col] + 4 * static_cast<int32_t>(r[c]);
+        }
       }
-      committed = kt;
+    }
+    cluster.sync();  // every share has landed
+    if (any_bad == 0) {
+      for (int e = tid; e < kCols * kTm; e += blockDim.x) {
+        const int cl = e / kTm, row = e % kTm;
+        const int64_t gi = i0 + rank * kCols + cl, jrow = j0 + row;
+        if (gi < m && jrow < n) {
+          int32_t d = k;
+#pragma unroll
+          for (int q = 0; q < KS; ++q) d += recv[(q * kCols + cl) * kTm + row];
+          if (dots) dots[gi * n + jrow] = d;
+          if (out) out[gi * n + jrow] = __ldg(alpha + jrow) * static_cast<float>(d);
+        }
+      }
     }
   }
-  // the last commit covers every MMA issued before it (second bounded wait after a timeout)
-  bool drained = true;
-  if (committed >= 0) {
-    const uint32_t bar = smem_u32(&bars[committed % kTcStages]);
-    const uint32_t par = static_cast<uint32_t>((committed / kTcStages) & 1);
-    drained = mbar_wait(bar, par) || mbar_wait(bar, par);
-  }
-  const bool good = __syncthreads_and(ok && drained) != 0;
-  if (!good && tid == 0) atomicAdd(&g_bnn_device_errors, 1u);
-  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
 
-  // epilogue: warps 0-3 own TMEM lanes 32w..32w+31 = tile rows; each 32x32
-  // block is transposed through shared memory so the stores are row-coalesced
-  if (warp < 4 && good) {
-    const int pad = ktiles * 128 - k;
-    int* tr = reinterpret_cast<int*>(smem) + warp * 32 * 33;  // operand tiles are no longer read
-    for (int c0 = 0; c0 < BN; c0 += 32) {
-      uint32_t r[32];
-      if (ktiles > 0) {
-        const uint32_t a = tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(c0);
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-            "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
-            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-              "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-              "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-              "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-            : "r"(a));
-        asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
-      } else {
-#pragma unroll
-        for (int c = 0; c < 32; ++c) r[c] = 0u;
-      }
-#pragma unroll
-      for (int c = 0; c < 32; ++c) tr[lane * 33 + c] = static_cast<int>(r[c]) - pad;  // [row][col]
-      __syncwarp();
-      const int64_t gn = n0 + c0 + lane;
-      const float a_n = (out && gn < n) ? __ldg(alpha + gn) : 0.0f;
-#pragma unroll 4
-      for (int i = 0; i < 32; ++i) {
-        const int64_t gm = m0 + warp * 32 + i;
-        if (gm < m && gn < n) {
-          const int32_t d = tr[i * 33 + lane];
-          if (dots) dots[gm * n + gn] = d;
-          if (out) out[gm * n + gn] = a_n * static_cast<float>(d);
-        }
-      }
-      __syncwarp();
-    }
-  }
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
   __syncthreads();
-  if (warp == 0)
+  if (warp == kProducers / 32)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(BN));
 }
 
-template <int BN>
+template <int BN, int KS>
 bnn_status launch_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha, int64_t m, int64_t n, int k, int kw,
                      int32_t* dots, float* out, cudaStream_t s) {
-  const int64_t gx = (n + BN - 1) / BN, gy = (m + kTcBM - 1) / kTcBM;
+  const int64_t gx = KS * ((n + kTm - 1) / kTm), gy = (m + BN - 1) / BN;
   if (gx > 2147483647LL || gy > 65535) return BNN_ERR_INVALID_ARG;
-  const size_t smem = static_cast<size_t>(kTcStages) * (kTcBM + BN) * 128 + 1024;  // + 1024-byte alignment slack
-  auto kern = binary_gemm_tc_kernel<BN>;
+  const size_t smem = static_cast<size_t>(stage_smem<BN>()) + 1024;  // + 1024-byte alignment slack
+  auto kern = binary_gemm_tc_kernel<BN, KS>;
   BNN_TRY(bnn::ensure_smem(kern, smem));
-  kern<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), kTcBM + BN, smem, s>>>(xp, wp, alpha, m, n, k,
-                                                                                          kw, dots, out);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
+  cfg.blockDim = dim3(threads_for<BN>());
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = KS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = KS > 1 ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, xp, wp, alpha, m, n, k, kw, dots, out);
+  if (e != cudaSuccess) return bnn::cuda_fail(e);
   return bnn::check_launch();
 }
 
@@ -255,13 +406,33 @@ bnn_status launch_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha,
 
 namespace bnn {
 
-// Tensor-core (tcgen05) binary GEMM; picks the tile width by problem size.
+// Tensor-core (tcgen05) binary GEMM.  m > 128 takes 256-row activation tiles
+// (one CTA per SM; the widest MMA, fewest re-expansions of the operands);
+// smaller m takes 64-row tiles (two CTAs per SM).  When the tiles alone would
+// leave SMs idle, a cluster of 2 or 4 CTAs splits each tile's stages (at least
+// 4 stages per CTA).
 bnn_status binary_gemm_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha, int64_t m, int64_t n, int k,
                           int kw, int32_t* dots, float* out, cudaStream_t s) {
-  const int64_t mt = (m + kTcBM - 1) / kTcBM;
-  if (mt * ((n + 255) / 256) >= 2LL * sm_count()) return launch_tc<256>(xp, wp, alpha, m, n, k, kw, dots, out, s);
-  if (mt * ((n + 127) / 128) >= sm_count()) return launch_tc<128>(xp, wp, alpha, m, n, k, kw, dots, out, s);
-  return launch_tc<64>(xp, wp, alpha, m, n, k, kw, dots, out, s);
+  const int64_t wt = (n + kTm - 1) / kTm;
+  const int64_t sms = sm_count();
+  const int ktiles = (kw + 1) / 2;
+  auto pick_ks = [&](int64_t tiles, int64_t capacity) {
+    if (tiles * 4 <= capacity && ktiles >= 16) return 4;
+    if (tiles * 2 <= capacity && ktiles >= 8) return 2;
+    return 1;
+  };
+  if (m > 128) {
+    switch (pick_ks(wt * ((m + 255) / 256), sms)) {
+      case 4: return launch_tc<256, 4>(xp, wp, alpha, m, n, k, kw, dots, out, s);
+      case 2: return launch_tc<256, 2>(xp, wp, alpha, m, n, k, kw, dots, out, s);
+      default: return launch_tc<256, 1>(xp, wp, alpha, m, n, k, kw, dots, out, s);
+    }
+  }
+  switch (pick_ks(wt * ((m + 63) / 64), 2 * sms)) {
+    case 4: return launch_tc<64, 4>(xp, wp, alpha, m, n, k, kw, dots, out, s);
+    case 2: return launch_tc<64, 2>(xp, wp, alpha, m, n, k, kw, dots, out, s);
+    default: return launch_tc<64, 1>(xp, wp, alpha, m, n, k, kw, dots, out, s);
+  }
 }
 
 }  // namespace bnn
