@@ -53,6 +53,8 @@ binary_gemv_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restrict__
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   const int64_t rows_per_warp_iter = static_cast<int64_t>(GROUPS_PER_WARP) * R;
+  bnn::pdl_trigger();
+  bool waited = false;  // launched with launch_pdl: the first weight loads overlap the preceding kernel
 
   for (int64_t row0 = warp * rows_per_warp_iter; row0 < n; row0 += nwarps * rows_per_warp_iter) {
     uint32_t acc[R][MT];
@@ -85,6 +87,10 @@ binary_gemv_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restrict__
           }
         }
       }
+      if (!waited) {
+        bnn::pdl_wait();  // x may come from the preceding kernel
+        waited = true;
+      }
 #pragma unroll
       for (int p = 0; p < P; ++p) {
         const int w = wb + p * SPAN;
@@ -115,6 +121,10 @@ binary_gemv_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restrict__
       for (int t = 0; t < MT; ++t)
 #pragma unroll
         for (int off = LPR / 2; off > 0; off >>= 1) acc[r][t] += __shfl_xor_sync(0xffffffffu, acc[r][t], off);
+    if (!waited) {
+      bnn::pdl_wait();  // the outputs are written after the preceding kernel
+      waited = true;
+    }
     if (sub == 0) {
 #pragma unroll
       for (int r = 0; r < R; ++r) {
@@ -142,7 +152,8 @@ void launch_gemv(const uint64_t* xp, const uint64_t* wp, const float* alpha, int
   const int64_t blocks_needed = (n + rows_per_block - 1) / rows_per_block;
   const int64_t cap = static_cast<int64_t>(bnn::sm_count()) * 8;
   const int grid = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
-  binary_gemv_kernel<VEC, LPR, R, MT, P><<<grid, threads, 0, s>>>(xp, wp, alpha, m, n, k, kw, dots, out);
+  bnn::launch_pdl(binary_gemv_kernel<VEC, LPR, R, MT, P>, dim3(grid), dim3(threads), 0, s, 1, xp, wp, alpha, m, n,
+                  k, kw, dots, out);
 }
 
 template <int VEC>

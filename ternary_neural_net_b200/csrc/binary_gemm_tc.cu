@@ -10,14 +10,21 @@
 //
 // Tile: UMMA M = 128 weight rows (operand A) x N = BN activation rows (operand
 // B), K in stages of 128 bits.  Roles inside a CTA:
+//   - a TMA thread (when every row is 16-byte aligned): copies the packed words
+//     of 4 stages of all the tile's rows (a 64-byte-swizzled box of each
+//     operand) into a double-buffered chunk ring, signalling an mbarrier with
+//     the byte count;
 //   - producer threads, two per row of the stacked (weight, activation) tile,
-//     each owning one 64-bit word of the row per stage: load it (prefetched
-//     kPre stages ahead in registers), count its bits, and write its 64 0/1
-//     bytes (per 4 bytes a shift and an AND) in the 128-byte-swizzled K-major
-//     layout the tensor core reads, then arrive on the stage's "full" mbarrier;
+//     each owning one 64-bit word of the row per stage: read it (from the
+//     chunk ring, or without TMA straight from global memory, prefetched kPre
+//     stages ahead in registers), count its bits, and write its 64 0/1 bytes
+//     (per 4 bytes a shift and an AND) in the 128-byte-swizzled K-major layout
+//     the tensor core reads, then arrive on the stage's "full" mbarrier;
 //   - one MMA thread: waits for "full", issues 4 tcgen05.mma.kind::i8 (K = 32)
-//     into the int32 accumulator in tensor memory and commits to the stage's
-//     "empty" mbarrier, which the producers wait on before refilling it;
+//     into the int32 accumulator(s) in tensor memory and commits to the
+//     stage's "empty" mbarrier, which the producers wait on before refilling
+//     it.  With ACC = 2 consecutive K = 32 blocks alternate between two
+//     accumulators, so that back-to-back MMAs do not depend on each other;
 //   - the epilogue (warps 0-7; warp w reads tensor-memory lanes 32(w%4).. and
 //     half w/4 of the columns): tcgen05.ld, the popcount correction, alpha,
 //     and stores in which the 32 lanes of a warp write 32 consecutive weight
@@ -25,15 +32,14 @@
 // Any bijection between the 128 bits and the 128 k-slots of a stage gives the
 // same sum when both operands use it; here byte j of word s of 16-byte chunk
 // 2h+q holds bit 32h + 8j + 4q + s.
-// Narrow tiles (BN = 64) keep 96 KB of stages so that two CTAs share an SM:
-// the producers' shift/AND/store chains need many warps to hide their latency.
 //
 // Split K: a cluster of KS CTAs shares one output tile, each taking a
 // contiguous share of the stages.  Each CTA turns its accumulator into its
-// share of the dot (-2 pa - 2 pb + 4 S over its stages) and stores it straight
-// into the shared memory of the CTA that owns that output row (distributed
-// shared memory); CTA r adds the KS shares of its BN/KS output rows and writes
-// them.  Integer addition makes the result independent of the order.
+// share of the dot (-2 pa - 2 pb + 4 S over its stages) and stores it, four
+// columns per 16-byte store, straight into the shared memory of the CTA that
+// owns those output rows (distributed shared memory); CTA r adds the KS shares
+// of its BN/KS output rows and writes them.  Integer addition makes the
+// result independent of the order.
 //
 // Every wait on an mbarrier is bounded.  A wait that runs out bumps a
 // device-side error count (bnn_device_error_count) and raises a CTA-wide abort
@@ -49,8 +55,22 @@ __device__ unsigned int g_bnn_device_errors = 0;
 namespace {
 
 constexpr int kTm = 128;                   // weight rows per tile (UMMA M)
-constexpr int kPre = 8;                    // stages of packed words prefetched in registers
+constexpr int kPre = 8;                    // without TMA: stages of words prefetched in registers
+constexpr int kChunkStages = 4;            // with TMA: stages per packed chunk (64 bytes of every row)
 constexpr uint32_t kSpinLimit = 1u << 24;  // bounded mbarrier waits
+
+template <int BN, bool TMA>
+struct TcCfg {
+  static constexpr int kRows = kTm + BN;                             // stacked weight + activation rows
+  static constexpr uint32_t kStageBytes = kRows * 128u;              // one expanded stage
+  static constexpr uint32_t kChunkBytes = kRows * 16u * kChunkStages; // one packed chunk (2 words per stage)
+  static constexpr int S = TMA ? 3 : 4;                              // expanded stages
+  static constexpr int P = TMA ? 2 : 0;                              // packed chunks
+  static constexpr uint32_t kSmem = S * kStageBytes + P * kChunkBytes;
+  static constexpr int kProducers = 2 * kRows;
+  static constexpr int kThreads = kProducers + 64;                   // + MMA warp + TMA warp
+  static constexpr int kMinBlocks = BN <= 64 ? 2 : 1;
+};
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -90,7 +110,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   return false;
 }
 
-// Bounded wait that ignores the abort flag (used for the final drain).
+// Bounded wait that ignores the abort flag (used for the final drains).
 __device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity) {
   for (uint32_t it = 0; it < kSpinLimit; ++it)
     if (mbar_try(bar, parity)) return true;
@@ -102,59 +122,85 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
 }
 
-// 32 columns of this warp's 32 tensor-memory lanes
-__device__ __forceinline__ void tmem_ld32(uint32_t addr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(addr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
 }
 
-// operand stages per CTA: 4 x 24 KB for BN = 64 (two CTAs per SM), 4 x 48 KB for BN = 256
-template <int BN>
-__host__ __device__ constexpr int stages_for() {
-  return 4;
+// 2-D tiled TMA load of one box into this CTA's shared memory (x = packed word,
+// y = row), completing `bytes` on the mbarrier.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
 }
-template <int BN>
-__host__ __device__ constexpr int stage_smem() {
-  return stages_for<BN>() * (kTm + BN) * 128;
+
+// 16 columns of this warp's 32 tensor-memory lanes
+__device__ __forceinline__ void tmem_ld16(uint32_t addr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(addr));
 }
-template <int BN>
-__host__ __device__ constexpr int threads_for() {
-  return 2 * (kTm + BN) + 32;
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+
+// 4 bytes per 16-byte chunk word: byte j of word s holds bit 8j + s of hw
+__device__ __forceinline__ void expand_word(uint8_t* dst_row, uint32_t swz, int part, uint64_t cw) {
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    const int h = 2 * part + hh;  // half-word of the stage's 128 bits
+    const uint32_t hw = static_cast<uint32_t>(cw >> (32 * hh));
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      uint4 v;
+      v.x = (hw >> (4 * q + 0)) & 0x01010101u;
+      v.y = (hw >> (4 * q + 1)) & 0x01010101u;
+      v.z = (hw >> (4 * q + 2)) & 0x01010101u;
+      v.w = (hw >> (4 * q + 3)) & 0x01010101u;
+      const uint32_t chunk = static_cast<uint32_t>(2 * h + q);
+      *reinterpret_cast<uint4*>(dst_row + ((chunk ^ swz) << 4)) = v;
+    }
+  }
 }
 
 // grid: x = KS * (weight tiles of 128 rows), y = activation tiles of BN rows;
 // clusters of KS CTAs along x
-template <int BN, int KS>
-__global__ void __launch_bounds__(threads_for<BN>(), BN <= 64 ? 2 : 1)
-binary_gemm_tc_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restrict__ wp,
+template <int BN, int KS, int ACC, bool TMA>
+__global__ void __launch_bounds__(TcCfg<BN, TMA>::kThreads, TcCfg<BN, TMA>::kMinBlocks)
+binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
+                      const uint64_t* __restrict__ xp, const uint64_t* __restrict__ wp,
                       const float* __restrict__ alpha, int64_t m, int64_t n, int k, int kw,
                       int32_t* __restrict__ dots, float* __restrict__ out) {
-  constexpr int S = stages_for<BN>();
-  constexpr int kRows = kTm + BN;
-  constexpr int kProducers = 2 * kRows;
-  constexpr uint32_t kStageBytes = static_cast<uint32_t>(kRows) * 128u;
+  using Cfg = TcCfg<BN, TMA>;
+  constexpr int S = Cfg::S;
+  constexpr int P = TMA ? Cfg::P : 1;
+  constexpr int kRows = Cfg::kRows;
+  constexpr int kProducers = Cfg::kProducers;
+  constexpr uint32_t kStageBytes = Cfg::kStageBytes;
+  constexpr int kCols = BN / KS;          // split K: accumulator columns each CTA owns
+  constexpr int kPitch = kCols + 4;       // split K: padded receive row (ints)
   static_assert(S >= 2, "at least two operand stages");
-  static_assert(KS == 1 || BN * kTm * 4 <= stage_smem<BN>(), "split-K shares must fit the stage memory");
-  static_assert(BN % KS == 0, "activation columns split evenly across the cluster");
+  static_assert(BN % KS == 0 && kCols % 4 == 0, "activation columns split evenly, four at a time");
+  static_assert(KS == 1 || KS * kTm * kPitch * 4 <= Cfg::kSmem, "split-K shares must fit the stage memory");
+  static_assert(ACC * BN <= 512, "tensor-memory columns");
 
   extern __shared__ __align__(16) uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[S];
   __shared__ __align__(8) uint64_t empty_bar[S];
+  __shared__ __align__(8) uint64_t chunk_full[P];
+  __shared__ __align__(8) uint64_t chunk_empty[P];
   __shared__ __align__(8) uint64_t done_bar;
   __shared__ uint32_t tmem_holder;
   __shared__ volatile int abort_flag;
-  __shared__ int any_bad;    // split K: some CTA of the cluster aborted
-  __shared__ int pop_w[kTm];  // popcount of each weight row over this CTA's stages
-  __shared__ int pop_x[BN];   // popcount of each activation row over this CTA's stages
+  __shared__ int any_bad;      // split K: some CTA of the cluster aborted
+  __shared__ int pop_w[kTm];   // popcount of each weight row over this CTA's stages
+  __shared__ int pop_x[BN];    // popcount of each activation row over this CTA's stages
   // the 128-byte swizzle repeats every 1024 bytes of address: align the tiles to it
   uint8_t* const smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* const chunks = smem + S * kStageBytes;  // TMA: packed chunk ring
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -167,6 +213,7 @@ binary_gemm_tc_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restric
   const int ke = kb + share < ktiles ? kb + share : ktiles;
   const int nst = ke - kb;
   const uint32_t smem_base = smem_u32(smem);
+  constexpr int kMmaWarp = kProducers / 32, kTmaWarp = kMmaWarp + 1;
 
   for (int i = tid; i < kRows; i += blockDim.x) (i < kTm ? pop_w[i] : pop_x[i - kTm]) = 0;
   if (tid == 0) {
@@ -174,78 +221,93 @@ binary_gemm_tc_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restric
       asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(&full_bar[i])), "r"(kProducers));
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_u32(&empty_bar[i])));
     }
+    for (int i = 0; i < P; ++i) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_u32(&chunk_full[i])));
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(&chunk_empty[i])), "r"(kProducers));
+    }
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_u32(&done_bar)));
     abort_flag = 0;
     any_bad = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
-  if (warp == kProducers / 32) {  // the MMA warp owns the tensor memory
+  if (warp == kMmaWarp) {  // the MMA warp owns the tensor memory
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(&tmem_holder)),
-                 "r"(BN));
+                 "r"(ACC * BN));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::);
   }
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
   const uint32_t tmem = tmem_holder;
+  bnn::pdl_trigger();
 
   if (tid < kProducers) {
     // ------------------------------------------------------------ producers
     const int r2 = tid >> 1, part = tid & 1;  // stacked row, word of the stage
     const bool is_w = r2 < kTm;
     const int row = is_w ? r2 : r2 - kTm;
-    const int64_t grow = is_w ? j0 + row : i0 + row;
-    const bool live = grow < (is_w ? n : m);
-    const uint64_t* src = (is_w ? wp : xp) + (live ? grow : 0) * static_cast<int64_t>(kw) + part;
     const uint32_t row_off = static_cast<uint32_t>(r2) * 128u;  // weight rows first, then activation rows
     const uint32_t swz = static_cast<uint32_t>(row & 7);
-
-    auto fetch = [&](int jj) -> uint64_t {
-      const int w = 2 * (kb + jj) + part;
-      return (live && jj < nst && w < kw) ? __ldg(src + 2 * (kb + jj)) : 0ull;
-    };
-    uint64_t ring[kPre];
-#pragma unroll
-    for (int u = 0; u < kPre; ++u) ring[u] = fetch(u);
-
     int my_pop = 0;
     bool ok = true;
-    for (int js = 0; js < nst && ok; js += kPre) {
-#pragma unroll
-      for (int u = 0; u < kPre; ++u) {
-        const int j = js + u;
-        if (j >= nst) break;
+    if constexpr (TMA) {
+      // this thread's word of stage s of a chunk: row r2 (64 bytes), 16-byte unit
+      // s under the 64-byte swizzle (unit ^ bits 7-8 of the address), half `part`
+      const uint32_t rd_off = static_cast<uint32_t>(r2) * 64u + 8u * static_cast<uint32_t>(part);
+      const uint32_t rd_swz = static_cast<uint32_t>((r2 >> 1) & 3);
+      for (int j = 0; j < nst; ++j) {
+        const int c = j / kChunkStages, s = j % kChunkStages, pb = c % P;
+        if (s == 0 && !mbar_wait(smem_u32(&chunk_full[pb]), static_cast<uint32_t>((c / P) & 1), &abort_flag)) {
+          ok = false;
+          break;
+        }
+        const uint64_t cw = *reinterpret_cast<const uint64_t*>(
+            chunks + pb * Cfg::kChunkBytes + rd_off + ((static_cast<uint32_t>(s) ^ rd_swz) << 4));
+        if (s == kChunkStages - 1 || j == nst - 1) mbar_arrive(smem_u32(&chunk_empty[pb]));
         const int b = j % S;
         // refill only after the tensor core has read the previous fill of this buffer
         if (j >= S && !mbar_wait(smem_u32(&empty_bar[b]), static_cast<uint32_t>((j / S + 1) & 1), &abort_flag)) {
           ok = false;
           break;
         }
-        const uint64_t cw = ring[u];
-        ring[u] = fetch(j + kPre);
         my_pop += __popcll(cw);
-        uint8_t* dst = smem + b * kStageBytes + row_off;
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int h = 2 * part + hh;  // half-word of the stage's 128 bits
-          const uint32_t hw = static_cast<uint32_t>(cw >> (32 * hh));
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            uint4 v;
-            v.x = (hw >> (4 * q + 0)) & 0x01010101u;
-            v.y = (hw >> (4 * q + 1)) & 0x01010101u;
-            v.z = (hw >> (4 * q + 2)) & 0x01010101u;
-            v.w = (hw >> (4 * q + 3)) & 0x01010101u;
-            const uint32_t chunk = static_cast<uint32_t>(2 * h + q);
-            *reinterpret_cast<uint4*>(dst + ((chunk ^ swz) << 4)) = v;
-          }
-        }
+        expand_word(smem + b * kStageBytes + row_off, swz, part, cw);
         asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
         mbar_arrive(smem_u32(&full_bar[b]));
       }
+    } else {
+      const int64_t grow = is_w ? j0 + row : i0 + row;
+      const bool live = grow < (is_w ? n : m);
+      const uint64_t* src = (is_w ? wp : xp) + (live ? grow : 0) * static_cast<int64_t>(kw) + part;
+      if (!is_w) bnn::pdl_wait();  // the activations may come from the preceding kernel
+      auto fetch = [&](int jj) -> uint64_t {
+        const int w = 2 * (kb + jj) + part;
+        return (live && jj < nst && w < kw) ? __ldg(src + 2 * (kb + jj)) : 0ull;
+      };
+      uint64_t ring[kPre];
+#pragma unroll
+      for (int u = 0; u < kPre; ++u) ring[u] = fetch(u);
+      for (int js = 0; js < nst && ok; js += kPre) {
+#pragma unroll
+        for (int u = 0; u < kPre; ++u) {
+          const int j = js + u;
+          if (j >= nst) break;
+          const int b = j % S;
+          if (j >= S && !mbar_wait(smem_u32(&empty_bar[b]), static_cast<uint32_t>((j / S + 1) & 1), &abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint64_t cw = ring[u];
+          ring[u] = fetch(j + kPre);
+          my_pop += __popcll(cw);
+          expand_word(smem + b * kStageBytes + row_off, swz, part, cw);
+          asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+          mbar_arrive(smem_u32(&full_bar[b]));
+        }
+      }
     }
     atomicAdd(is_w ? &pop_w[row] : &pop_x[row], my_pop);
-  } else if (tid == kProducers) {
+  } else if (tid == kMmaWarp * 32) {
     // ------------------------------------------------------------ MMA issue
     // instruction descriptor: D s32, A and B 8-bit integers (0/1 bytes read
     // the same signed or unsigned), both K-major, N = BN, M = 128
@@ -259,10 +321,11 @@ binary_gemm_tc_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restric
       const uint64_t bd = sw128_desc(smem_base + b * kStageBytes + kTm * 128u);  // activation rows
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
-        const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+        const uint32_t d = tmem + static_cast<uint32_t>((kk % ACC) * BN);
+        const uint32_t acc = (j > 0 || kk >= ACC) ? 1u : 0u;
         asm volatile(
             "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
-            "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem),
+            "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
             "l"(ad + static_cast<uint64_t>(2 * kk)), "l"(bd + static_cast<uint64_t>(2 * kk)), "r"(idesc), "r"(acc));
       }
       asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
@@ -273,12 +336,43 @@ binary_gemm_tc_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restric
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
                      smem_u32(&done_bar))
                  : "memory");
+  } else if (TMA && tid == kTmaWarp * 32) {
+    // ------------------------------------------------------------ TMA copies
+    const int nch = (nst + kChunkStages - 1) / kChunkStages;
+    const int pre = nch < P ? nch : P;
+    auto chunk_x = [&](int c) { return 2 * kb + 2 * kChunkStages * c; };  // first word (even: 16-byte aligned)
+    // the weights do not depend on the preceding kernel: their first chunks
+    // are copied before waiting for it, the activations after
+    for (int c = 0; c < pre; ++c) {
+      mbar_expect_tx(smem_u32(&chunk_full[c]), Cfg::kChunkBytes);
+      tma_load_2d(smem_u32(chunks + c * Cfg::kChunkBytes), &tmap_w, chunk_x(c), static_cast<int>(j0),
+                  smem_u32(&chunk_full[c]));
+    }
+    bnn::pdl_wait();
+    for (int c = 0; c < pre; ++c)
+      tma_load_2d(smem_u32(chunks + c * Cfg::kChunkBytes) + kTm * 16u * kChunkStages, &tmap_x, chunk_x(c),
+                  static_cast<int>(i0), smem_u32(&chunk_full[c]));
+    int issued = pre;
+    for (int c = pre; c < nch; ++c) {
+      const int pb = c % P;
+      if (!mbar_wait(smem_u32(&chunk_empty[pb]), static_cast<uint32_t>((c / P + 1) & 1), &abort_flag)) break;
+      const uint32_t dst = smem_u32(chunks + pb * Cfg::kChunkBytes);
+      const uint32_t bar = smem_u32(&chunk_full[pb]);
+      mbar_expect_tx(bar, Cfg::kChunkBytes);
+      tma_load_2d(dst, &tmap_w, chunk_x(c), static_cast<int>(j0), bar);
+      tma_load_2d(dst + kTm * 16u * kChunkStages, &tmap_x, chunk_x(c), static_cast<int>(i0), bar);
+      issued = c + 1;
+    }
+    // the CTA must not retire with copies in flight (producers that aborted no
+    // longer wait for them): wait for the last chunk issued into each buffer
+    for (int c = issued - P; c < issued; ++c)
+      if (c >= 0) mbar_drain(smem_u32(&chunk_full[c % P]), static_cast<uint32_t>((c / P) & 1));
   }
   __syncwarp();
 
   // -------------------------------------------------------------- epilogue
-  // every producer is past its loop (row popcounts added); the accumulator is final
-  // once done_bar completes
+  // every producer is past its loop (row popcounts added); the accumulator is
+  // final once done_bar completes
   if (tid < kProducers) asm volatile("bar.sync 1, %0;\n" ::"r"(kProducers) : "memory");
   bool drained = true;
   if (warp < 8) {
@@ -292,28 +386,41 @@ binary_gemm_tc_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restric
   const int erow = 32 * (warp & 3) + (tid & 31);
   const int ecol0 = (warp >> 2) * (BN / 2);
   const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+  // the tile's accumulated popc(a AND b) for 16 columns from c0 (sum of the accumulators)
+  auto load16 = [&](int c0, uint32_t (&r)[16]) {
+    if (nst > 0) {
+      tmem_ld16(taddr + static_cast<uint32_t>(c0), r);
+      if constexpr (ACC == 2) {
+        uint32_t r2[16];
+        tmem_ld16(taddr + static_cast<uint32_t>(BN + c0), r2);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 16; ++c) r[c] += r2[c];
+      } else {
+        tmem_wait_ld();
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 16; ++c) r[c] = 0u;
+    }
+  };
   if constexpr (KS == 1) {
     if (warp < 8 && good) {
       const int64_t jrow = j0 + erow;
       const bool jlive = jrow < n;
       const float a_j = (out && jlive) ? __ldg(alpha + jrow) : 0.0f;
       const int base = k - 2 * pop_w[erow];
-      for (int c0 = ecol0; c0 < ecol0 + BN / 2; c0 += 32) {
-        uint32_t r[32];
-        if (nst > 0) {
-          tmem_ld32(taddr + static_cast<uint32_t>(c0), r);
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) r[c] = 0u;
-        }
+      for (int c0 = ecol0; c0 < ecol0 + BN / 2; c0 += 16) {
+        uint32_t r[16];
+        load16(c0, r);
         const int64_t rows_left = m - (i0 + c0);
         if (jlive && rows_left > 0) {
-          const int nc = rows_left < 32 ? static_cast<int>(rows_left) : 32;
+          const int nc = rows_left < 16 ? static_cast<int>(rows_left) : 16;
           const int64_t off = (i0 + c0) * n + jrow;
           int32_t* dp = dots ? dots + off : nullptr;
           float* op = out ? out + off : nullptr;
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
+          for (int c = 0; c < 16; ++c) {
             if (c < nc) {
               const int32_t d = base - 2 * pop_x[c0 + c] + 4 * static_cast<int32_t>(r[c]);
               if (dp) *dp = d;
@@ -328,44 +435,57 @@ binary_gemm_tc_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restric
   } else {
     // Split K: CTA q of the cluster owns accumulator columns [q kCols, (q+1) kCols).
     // Every CTA pushes its share of each column to the owner's receive buffer
-    // [source rank][column][weight row] (remote stores, no round trip), then
-    // each owner adds the KS shares of its columns.
+    // [source rank][weight row][column, padded] (16-byte remote stores, no
+    // round trip), then each owner adds the KS shares of its columns.
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
-    constexpr int kCols = BN / KS;
     int* recv = reinterpret_cast<int*>(smem);
     cluster.sync();  // every CTA's tensor core is done with its stage memory
     if (tid == 0 && !good)  // this CTA's shares will be missing: no CTA of the cluster writes
       for (int q = 0; q < KS; ++q) atomicExch(cluster.map_shared_rank(&any_bad, q), 1);
     if (warp < 8 && good) {
       const int base = -2 * pop_w[erow];
-      for (int c0 = ecol0; c0 < ecol0 + BN / 2; c0 += 32) {
-        uint32_t r[32];
-        if (nst > 0) {
-          tmem_ld32(taddr + static_cast<uint32_t>(c0), r);
-        } else {
+      for (int c0 = ecol0; c0 < ecol0 + BN / 2; c0 += 16) {
+        uint32_t r[16];
+        load16(c0, r);
 #pragma unroll
-          for (int c = 0; c < 32; ++c) r[c] = 0u;
-        }
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const int col = c0 + c;
+        for (int g = 0; g < 4; ++g) {
+          const int col = c0 + 4 * g;
+          int4 v;
+          v.x = base - 2 * pop_x[col + 0] + 4 * static_cast<int32_t>(r[4 * g + 0]);
+          v.y = base - 2 * pop_x[col + 1] + 4 * static_cast<int32_t>(r[4 * g + 1]);
+          v.z = base - 2 * pop_x[col + 2] + 4 * static_cast<int32_t>(r[4 * g + 2]);
+          v.w = base - 2 * pop_x[col + 3] + 4 * static_cast<int32_t>(r[4 * g + 3]);
           int* dst = cluster.map_shared_rank(recv, col / kCols);
-          dst[(rank * kCols + col % kCols) * kTm + erow] = base - 2 * pop_x[col] + 4 * static_cast<int32_t>(r[c]);
+          *reinterpret_cast<int4*>(dst + (rank * kTm + erow) * kPitch + col % kCols) = v;
         }
       }
     }
     cluster.sync();  // every share has landed
     if (any_bad == 0) {
-      for (int e = tid; e < kCols * kTm; e += blockDim.x) {
-        const int cl = e / kTm, row = e % kTm;
-        const int64_t gi = i0 + rank * kCols + cl, jrow = j0 + row;
-        if (gi < m && jrow < n) {
-          int32_t d = k;
+      for (int e = tid; e < kTm * (kCols / 4); e += blockDim.x) {
+        const int row = e % kTm, cl = 4 * (e / kTm);
+        const int64_t jrow = j0 + row;
+        if (jrow < n) {
+          int4 d = make_int4(k, k, k, k);
 #pragma unroll
-          for (int q = 0; q < KS; ++q) d += recv[(q * kCols + cl) * kTm + row];
-          if (dots) dots[gi * n + jrow] = d;
-          if (out) out[gi * n + jrow] = __ldg(alpha + jrow) * static_cast<float>(d);
+          for (int q = 0; q < KS; ++q) {
+            const int4 v = *reinterpret_cast<const int4*>(recv + (q * kTm + row) * kPitch + cl);
+            d.x += v.x;
+            d.y += v.y;
+            d.z += v.z;
+            d.w += v.w;
+          }
+          const float a_j = out ? __ldg(alpha + jrow) : 0.0f;
+          const int dv[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int64_t gi = i0 + rank * kCols + cl + t;
+            if (gi < m) {
+              if (dots) dots[gi * n + jrow] = dv[t];
+              if (out) out[gi * n + jrow] = a_j * static_cast<float>(dv[t]);
+            }
+          }
         }
       }
     }
@@ -373,31 +493,33 @@ binary_gemm_tc_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restric
 
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
   __syncthreads();
-  if (warp == kProducers / 32)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(BN));
+  if (warp == kMmaWarp)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(ACC * BN));
 }
 
-template <int BN, int KS>
+template <int BN, int KS, int ACC>
 bnn_status launch_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha, int64_t m, int64_t n, int k, int kw,
                      int32_t* dots, float* out, cudaStream_t s) {
   const int64_t gx = KS * ((n + kTm - 1) / kTm), gy = (m + BN - 1) / BN;
   if (gx > 2147483647LL || gy > 65535) return BNN_ERR_INVALID_ARG;
-  const size_t smem = static_cast<size_t>(stage_smem<BN>()) + 1024;  // + 1024-byte alignment slack
-  auto kern = binary_gemm_tc_kernel<BN, KS>;
+  // TMA needs 16-byte aligned rows (even kw, aligned bases) and coordinates that fit int32
+  CUtensorMap tw, tx;
+  bool tma = kw > 0 && kw % 2 == 0 && bnn::aligned(xp, 16) && bnn::aligned(wp, 16) && n < (1LL << 31) &&
+             m < (1LL << 31);
+  if (tma)
+    tma = bnn::encode_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT64, wp, static_cast<uint64_t>(kw),
+                              static_cast<uint64_t>(n), static_cast<uint64_t>(kw) * 8u, 2 * kChunkStages, kTm,
+                              CU_TENSOR_MAP_SWIZZLE_64B) &&
+          bnn::encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT64, xp, static_cast<uint64_t>(kw),
+                              static_cast<uint64_t>(m), static_cast<uint64_t>(kw) * 8u, 2 * kChunkStages, BN,
+                              CU_TENSOR_MAP_SWIZZLE_64B);
+  if (!tma) memset(&tw, 0, sizeof(tw)), memset(&tx, 0, sizeof(tx));
+  const size_t smem = static_cast<size_t>(tma ? TcCfg<BN, true>::kSmem : TcCfg<BN, false>::kSmem) + 1024;
+  auto kern = tma ? binary_gemm_tc_kernel<BN, KS, ACC, true> : binary_gemm_tc_kernel<BN, KS, ACC, false>;
   BNN_TRY(bnn::ensure_smem(kern, smem));
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
-  cfg.blockDim = dim3(threads_for<BN>());
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = KS;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = KS > 1 ? 1 : 0;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, xp, wp, alpha, m, n, k, kw, dots, out);
+  const cudaError_t e = bnn::launch_pdl(kern, dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)),
+                                        dim3(tma ? TcCfg<BN, true>::kThreads : TcCfg<BN, false>::kThreads), smem, s,
+                                        KS, tw, tx, xp, wp, alpha, m, n, k, kw, dots, out);
   if (e != cudaSuccess) return bnn::cuda_fail(e);
   return bnn::check_launch();
 }
@@ -406,33 +528,22 @@ bnn_status launch_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha,
 
 namespace bnn {
 
-// Tensor-core (tcgen05) binary GEMM.  m > 128 takes 256-row activation tiles
-// (one CTA per SM; the widest MMA, fewest re-expansions of the operands);
-// smaller m takes 64-row tiles (two CTAs per SM).  When the tiles alone would
-// leave SMs idle, a cluster of 2 or 4 CTAs splits each tile's stages (at least
-// 4 stages per CTA).
+// Tensor-core (tcgen05) binary GEMM.  With at least a full wave of 256-row
+// activation tiles the kernel takes those (one CTA per SM; the widest MMA and
+// the fewest re-expansions of the operands); otherwise 64-row tiles (two CTAs
+// per SM), with a cluster of 4 CTAs splitting each tile's stages when that
+// still leaves at most one CTA per SM, else of 2 when the CTAs fit in one
+// wave (at least 4 stages per CTA either way).
 bnn_status binary_gemm_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha, int64_t m, int64_t n, int k,
                           int kw, int32_t* dots, float* out, cudaStream_t s) {
   const int64_t wt = (n + kTm - 1) / kTm;
   const int64_t sms = sm_count();
   const int ktiles = (kw + 1) / 2;
-  auto pick_ks = [&](int64_t tiles, int64_t capacity) {
-    if (tiles * 4 <= capacity && ktiles >= 16) return 4;
-    if (tiles * 2 <= capacity && ktiles >= 8) return 2;
-    return 1;
-  };
-  if (m > 128) {
-    switch (pick_ks(wt * ((m + 255) / 256), sms)) {
-      case 4: return launch_tc<256, 4>(xp, wp, alpha, m, n, k, kw, dots, out, s);
-      case 2: return launch_tc<256, 2>(xp, wp, alpha, m, n, k, kw, dots, out, s);
-      default: return launch_tc<256, 1>(xp, wp, alpha, m, n, k, kw, dots, out, s);
-    }
-  }
-  switch (pick_ks(wt * ((m + 63) / 64), 2 * sms)) {
-    case 4: return launch_tc<64, 4>(xp, wp, alpha, m, n, k, kw, dots, out, s);
-    case 2: return launch_tc<64, 2>(xp, wp, alpha, m, n, k, kw, dots, out, s);
-    default: return launch_tc<64, 1>(xp, wp, alpha, m, n, k, kw, dots, out, s);
-  }
+  if (wt * ((m + 255) / 256) >= sms) return launch_tc<256, 1, 1>(xp, wp, alpha, m, n, k, kw, dots, out, s);
+  const int64_t tiles = wt * ((m + 63) / 64);
+  if (tiles * 4 <= sms && ktiles >= 16) return launch_tc<64, 4, 1>(xp, wp, alpha, m, n, k, kw, dots, out, s);
+  if (tiles * 2 <= 2 * sms && ktiles >= 8) return launch_tc<64, 2, 1>(xp, wp, alpha, m, n, k, kw, dots, out, s);
+  return launch_tc<64, 1, 1>(xp, wp, alpha, m, n, k, kw, dots, out, s);
 }
 
 }  // namespace bnn

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>  // CUtensorMap and its enums (the encoder is fetched from the driver at run time)
 #include <cuda_runtime.h>
 
 #include "bnn.h"
@@ -36,6 +37,42 @@ template <typename Kernel>
 cudaError_t ensure_smem(Kernel kern, size_t bytes) {
   if (bytes <= 48 * 1024) return cudaSuccess;
   return ensure_smem_raw(reinterpret_cast<const void*>(kern), bytes);
+}
+
+// Fills a 2-D TMA descriptor for a row-major matrix of `rows` rows of `inner`
+// elements, rows `row_bytes` apart, copied in boxes of box_inner x box_rows
+// elements with the given shared-memory swizzle; elements outside the matrix
+// read as zero.  False when the driver rejects it (alignment, sizes) or the
+// encoder is unavailable.
+bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType type, const void* base, uint64_t inner, uint64_t rows,
+                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swizzle);
+
+// Programmatic dependent launch.  A kernel launched with launch_pdl may start
+// while the preceding kernel on the stream is still running; it must call
+// pdl_wait() before it reads anything that kernel writes and before its own
+// first global store.  pdl_trigger() lets the next such kernel start early (a
+// no-op when the next kernel was launched normally).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, unsigned cluster_x,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster_x;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = cluster_x > 1 ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
 }
 
 // Tensor-core (tcgen05 kind::i8) binary GEMM, in binary_gemm_tc.cu.

@@ -25,6 +25,7 @@ pack_signs_kernel(const float* __restrict__ x, int64_t k, int64_t kw, int64_t un
   const int lane = threadIdx.x & 31;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
+  bnn::pdl_trigger();  // a matmul launched after this kernel may start its weight copies now
   for (int64_t u0 = warp; u0 < units; u0 += nwarps * kUnroll) {
     float a[kUnroll][kWords], b[kUnroll][kWords];
     int64_t row[kUnroll], j0[kUnroll];
