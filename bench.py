@@ -434,7 +434,7 @@ def run_workloads(cu: Cuda, args, peaks, popc_peak_macs):
     if "gemv_ffn" in want:
         out.update(wl_gemv_ffn(cu, args, P, st, s, hbm))
     if "gemm_large" in want:
-        out.update(wl_gemm_large(cu, args, P, st, s, popc_peak_macs))
+        out.update(wl_gemm_large(cu, args, P, st, s, popc_peak_macs, peaks))
     if "ternary" in want:
         out.update(wl_ternary(cu, args, P, st, s, hbm, peaks))
     return out
@@ -495,7 +495,7 @@ def wl_gemv_ffn(cu, args, P, st, s, hbm):
     return out
 
 
-def wl_gemm_large(cu, args, P, st, s, popc_peak_macs):
+def wl_gemm_large(cu, args, P, st, s, popc_peak_macs, peaks):
     torch, dev, lib = cu.torch, cu.device, cu.lib
     out = {}
 
@@ -517,6 +517,9 @@ def wl_gemm_large(cu, args, P, st, s, popc_peak_macs):
     res4["popc"]["frac_of_popc_peak"] = res4["popc"]["gmacs"] / 1e3 / popc_peak_macs
     res4["mma_s8"]["x_popc_peak"] = res4["mma_s8"]["gmacs"] / 1e3 / popc_peak_macs
     res4["tc"]["x_popc_peak"] = res4["tc"]["gmacs"] / 1e3 / popc_peak_macs
+    int8_peak = 2.0 * peaks["bf16_tflops"]  # TOP/s: nominal int8:bf16 ratio 2 x the measured bf16 rate
+    res4["tc"]["frac_of_int8_peak"] = 2.0 * res4["tc"]["gmacs"] / 1e3 / int8_peak
+    res4["tc"]["traffic_bytes"] = traffic_for("binary_gemm_tc_256x1", "ternary_neural_net_b200/csrc/binary_gemm_tc.cu")
     out["gemm_large_8192"] = res4
     del d, o, xp, wp
     return out
@@ -696,16 +699,16 @@ def main():
                    "m": res["m"], "n": res["n"], "k": res["k"],
                    "l2": f"inputs and outputs rotate through {res['R']} copies (> 2x L2) so each step starts cold",
                    "parallelism": f"replicas x{N} (independent problems per GPU)"},
-        "roofline": {"bound": "tensor", "kernel": "binary_gemm_tc_kernel<256,4> (bnn_binary_gemm, m >= 64: packed "
-                                                  "bits -> 0/1 bytes in swizzled smem, tcgen05.mma kind::i8 into "
-                                                  "TMEM, 4-CTA cluster split-K)",
+        "roofline": {"bound": "tensor", "kernel": "binary_gemm_tc_kernel<64,2,1,TMA> (bnn_binary_gemm, m >= 64: "
+                                                  "TMA-fed packed chunks -> 0/1 bytes in swizzled smem, tcgen05.mma "
+                                                  "kind::i8 into TMEM, 2-CTA cluster split-K)",
                      "achieved": 2 * gemm_achieved, "peak": int8_peak, "unit": "TOP/s",
                      "frac": 2 * gemm_achieved / int8_peak,
                      "achieved_back_to_back": 2 * res["macs"] / (res["gemm_graph_ms"] * 1e-3) / 1e12,
                      "achieved_basis": "achieved: CUDA events around the kernel on every 16th step of the timed "
                                        "graph (includes the event nodes' serialisation); achieved_back_to_back: "
                                        "a graph of the kernel alone launched back to back",
-                     "traffic": traffic_for("binary_gemm_tc_256x4", "ternary_neural_net_b200/csrc/binary_gemm_tc.cu"),
+                     "traffic": traffic_for("binary_gemm_tc_64x2", "ternary_neural_net_b200/csrc/binary_gemm_tc.cu"),
                      "peak_basis": f"int8 dense tensor peak = measured bf16 {peaks['bf16_tflops']} TFLOP/s x 2 "
                                    f"(nominal int8:bf16 ratio 4.5:2.25 PFLOP/s), {peak_src}"},
         "roofline_popc": {"bound": "alu", "kernel": "binary_gemm_tiled_kernel (bnn_binary_gemm_algo POPC)",
