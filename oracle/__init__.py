@@ -30,6 +30,8 @@ def _L():
             "oracle_count_pad_bits": ([vp, i64, i64], i64),
             "oracle_binary_gemm": ([vp, vp, vp, i64, i64, i64, vp, vp], None),
             "oracle_binary_gemm_sampled": ([vp, vp, vp, i64, i64, i64, vp, vp, i64, vp, vp], None),
+            "oracle_binary_linear": ([vp, vp, vp, vp, i64, i64, i64, vp, vp, vp], None),
+            "oracle_ternary_linear": ([vp, vp, vp, vp, i64, i64, i64, vp, vp], None),
             "oracle_twn_ternarize": ([vp, i64, i64, vp, vp, vp], None),
             "oracle_twn_delta": ([vp, i64], C.c_float),
             "oracle_absmean_ternarize": ([vp, i64, i64, vp, vp, vp], None),
@@ -105,6 +107,28 @@ def binary_gemm_sampled(xp, wp, alpha, m: int, n: int, k: int, rows, cols):
     _L().oracle_binary_gemm_sampled(_p(xp), _p(wp), _p(alpha), m, n, k, _p(rows), _p(cols),
                                     rows.size, _p(dots), _p(out))
     return dots, out
+
+
+def binary_linear(xp, wp, alpha, bias, m: int, n: int, k: int):
+    """One binarised layer: (dots int32 [m,n], y float32 [m,n], next uint64 [m, ceil(n/64)]),
+    y = fl32(fl32(alpha*dot) + bias) (bias may be None), next = sign pack of y."""
+    xp, wp, alpha = _c(xp, np.uint64), _c(wp, np.uint64), _c(alpha, np.float32)
+    bias = None if bias is None else _c(bias, np.float32)
+    dots = np.zeros((m, n), dtype=np.int32)
+    y = np.zeros((m, n), dtype=np.float32)
+    nxt = np.zeros((m, words_per_row(n)), dtype=np.uint64)
+    _L().oracle_binary_linear(_p(xp), _p(wp), _p(alpha), _p(bias), m, n, k, _p(dots), _p(y), _p(nxt))
+    return dots, y, nxt
+
+
+def ternary_linear(x_bf16, packed, scale, bias, m: int, n: int, k: int):
+    """Ternary layer with bias, float64: (y [m,n], mag [m,n])."""
+    x_bf16, packed, scale = _c(x_bf16, np.uint16), _c(packed, np.uint16), _c(scale, np.float32)
+    bias = None if bias is None else _c(bias, np.float32)
+    y = np.zeros((m, n), dtype=np.float64)
+    mag = np.zeros((m, n), dtype=np.float64)
+    _L().oracle_ternary_linear(_p(x_bf16), _p(packed), _p(scale), _p(bias), m, n, k, _p(y), _p(mag))
+    return y, mag
 
 
 def twn_ternarize(w: np.ndarray):

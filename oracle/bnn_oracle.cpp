@@ -127,6 +127,37 @@ void oracle_binary_gemm_sampled(const uint64_t* xp, const uint64_t* wp, const fl
                dots ? dots + s : nullptr, out ? out + s : nullptr);
 }
 
+// One binarised linear layer followed by the next layer's input packing
+// ([BTE] ".tbin Format": a ternary/binary record carries a per-channel bias;
+// "binary_nn" README, FFN stacks of BinaryLinear: binary activations from layer
+// to layer).  In this order: the +-1 dot (as oracle_binary_gemm), the channel
+// scale y = fl32(alpha_j * dot), the bias y = fl32(y + bias_j) (an IEEE float32
+// addition, skipped when bias is null), then the sign pack of the row of y
+// exactly as oracle_pack_signs (bit = !(y > 0), pad bits 0) into
+// next[i, 0 .. ceil(n/64)).  Any output pointer may be null.
+void oracle_binary_linear(const uint64_t* xp, const uint64_t* wp, const float* alpha, const float* bias,
+                          int64_t m, int64_t n, int64_t k, int32_t* dots, float* y, uint64_t* next) {
+  const int64_t kw = words64(k);
+  const int64_t nw = words64(n);
+  float* row = new float[n > 0 ? n : 1];
+  for (int64_t i = 0; i < m; ++i) {
+    for (int64_t j = 0; j < n; ++j) {
+      int32_t d = 0;
+      float v = 0.0f;
+      binary_one(xp + i * kw, wp + j * kw, k, alpha, j, &d, &v);
+      if (bias) {
+        const float b = bias[j];
+        v = v + b;  // binary32 addition, round to nearest even (built with -ffp-contract=off)
+      }
+      row[j] = v;
+      if (dots) dots[i * n + j] = d;
+      if (y) y[i * n + j] = v;
+    }
+    if (next) oracle_pack_signs(row, 1, n, next + i * nw);
+  }
+  delete[] row;
+}
+
 // [BTE] "Features": TWN threshold Delta = 0.7 * mean|W| over the whole tensor,
 // the mean summed in float64 in element order and Delta rounded once to float32.
 float oracle_twn_delta(const float* w, int64_t total) {
@@ -268,6 +299,20 @@ void oracle_ternary_gemm(const uint16_t* x_bf16, const uint16_t* packed, const f
       ternary_one(x_bf16 + i * k, t, k, scale[j], out + i * n + j, mag ? mag + i * n + j : nullptr);
   }
   delete[] t;
+}
+
+// The ternary layer with its per-channel bias ([BTE] ".tbin Format" biases,
+// "Module Overview" Layer.forward): y = scale_j * sum + bias_j in float64, and
+// mag = |scale_j| * sum |x t| + |bias_j| (the magnitude the tolerance scales with).
+void oracle_ternary_linear(const uint16_t* x_bf16, const uint16_t* packed, const float* scale, const float* bias,
+                           int64_t m, int64_t n, int64_t k, double* out, double* mag) {
+  oracle_ternary_gemm(x_bf16, packed, scale, m, n, k, out, mag);
+  if (!bias) return;
+  for (int64_t i = 0; i < m; ++i)
+    for (int64_t j = 0; j < n; ++j) {
+      out[i * n + j] += double(bias[j]);
+      if (mag) mag[i * n + j] += std::fabs(double(bias[j]));
+    }
 }
 
 void oracle_ternary_gemm_sampled(const uint16_t* x_bf16, const uint16_t* packed,

@@ -19,6 +19,8 @@ void oracle_binary_gemm(const uint64_t* xp, const uint64_t* wp, const float* alp
 void oracle_binary_gemm_sampled(const uint64_t* xp, const uint64_t* wp, const float* alpha,
                                 int64_t m, int64_t n, int64_t k, const int64_t* rows,
                                 const int64_t* cols, int64_t count, int32_t* dots, float* out);
+void oracle_binary_linear(const uint64_t* xp, const uint64_t* wp, const float* alpha, const float* bias,
+                          int64_t m, int64_t n, int64_t k, int32_t* dots, float* y, uint64_t* next);
 float oracle_twn_delta(const float* w, int64_t total);
 void oracle_twn_apply(const float* w, int64_t n, int64_t k, float delta, int8_t* trits, float* scale);
 void oracle_twn_ternarize(const float* w, int64_t n, int64_t k, int8_t* trits,
@@ -29,6 +31,8 @@ void oracle_base3_pack(const int8_t* trits, int64_t n, int64_t k, uint16_t* pack
 int64_t oracle_base3_unpack(const uint16_t* packed, int64_t n, int64_t k, int8_t* trits);
 void oracle_ternary_gemm(const uint16_t* x_bf16, const uint16_t* packed, const float* scale,
                          int64_t m, int64_t n, int64_t k, double* out, double* mag);
+void oracle_ternary_linear(const uint16_t* x_bf16, const uint16_t* packed, const float* scale, const float* bias,
+                           int64_t m, int64_t n, int64_t k, double* out, double* mag);
 void oracle_ternary_gemm_sampled(const uint16_t* x_bf16, const uint16_t* packed,
                                  const float* scale, int64_t m, int64_t n, int64_t k,
                                  const int64_t* rows, const int64_t* cols, int64_t count,

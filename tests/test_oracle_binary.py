@@ -148,3 +148,55 @@ def test_pad_bit_counter_sees_planted_bit():
     assert oracle.count_pad_bits(xp, 70) == 0
     xp[0, 1] |= np.uint64(1) << np.uint64(9)
     assert oracle.count_pad_bits(xp, 70) == 1
+
+
+# ---------------------------------------------------------------------------
+# Fused layer epilogue: y = fl32(fl32(alpha * dot) + bias), next = sign pack of y
+# ---------------------------------------------------------------------------
+def test_linear_without_bias_is_the_gemm_and_its_pack():
+    rng = np.random.default_rng(21)
+    m, n, k = 5, 70, 200   # n past one word: pad bits in `next`
+    xp, wp = np_pack(rand_pm1(rng, m, k)), np_pack(rand_pm1(rng, n, k))
+    alpha = (rng.random(n) * 2 - 0.5).astype(np.float32)
+    d, y, nxt = oracle.binary_linear(xp, wp, alpha, None, m, n, k)
+    gd, go = oracle.binary_gemm(xp, wp, alpha, m, n, k)
+    assert np.array_equal(d, gd) and np.array_equal(y.view(np.uint32), go.view(np.uint32))
+    # the next layer's input, by an independent packer: bit j = !(y_j > 0)
+    assert np.array_equal(nxt, np_pack(np.where(y > 0, 1, -1)))
+    assert oracle.count_pad_bits(nxt, n) == 0
+
+
+def test_linear_bias_special_cases():
+    rng = np.random.default_rng(22)
+    m, n, k = 3, 6, 129
+    xp, wp = np_pack(rand_pm1(rng, m, k)), np_pack(rand_pm1(rng, n, k))
+    alpha = (rng.random(n) + 0.5).astype(np.float32)
+    _, y0, _ = oracle.binary_linear(xp, wp, alpha, None, m, n, k)
+    # bias cancelling row 0 exactly: y = +0 there, which packs as -1 (0 is not > 0)
+    bias = -y0[0].copy()
+    _, y, nxt = oracle.binary_linear(xp, wp, alpha, bias, m, n, k)
+    assert np.all(y[0] == 0.0) and not np.any(np.signbit(y[0]))
+    assert int(nxt[0, 0]) == (1 << n) - 1
+    # huge positive / negative bias forces every sign
+    _, y, nxt = oracle.binary_linear(xp, wp, alpha, np.full(n, 1e30, np.float32), m, n, k)
+    assert np.all(nxt == 0) and np.all(y == np.float32(1e30))
+    _, _, nxt = oracle.binary_linear(xp, wp, alpha, np.full(n, -np.inf, np.float32), m, n, k)
+    assert np.all(nxt[:, 0] == (1 << n) - 1)
+    # one float32 addition after the rounded product: a bias below half an ulp of
+    # y leaves y unchanged (no fused multiply-add)
+    tiny = np.full(n, 1e-30, np.float32)
+    _, yt, _ = oracle.binary_linear(xp, wp, alpha, tiny, m, n, k)
+    assert np.array_equal(yt[y0 != 0], y0[y0 != 0])
+
+
+def test_linear_bias_is_one_float32_addition():
+    rng = np.random.default_rng(23)
+    m, n, k = 4, 33, 300
+    xp, wp = np_pack(rand_pm1(rng, m, k)), np_pack(rand_pm1(rng, n, k))
+    alpha = (rng.random(n) * 3 - 1).astype(np.float32)
+    bias = rng.standard_normal(n).astype(np.float32) * 20
+    d, y, nxt = oracle.binary_linear(xp, wp, alpha, bias, m, n, k)
+    want = (alpha[None, :] * d.astype(np.float32)) + bias[None, :]
+    assert want.dtype == np.float32
+    assert np.array_equal(y.view(np.uint32), want.view(np.uint32))
+    assert np.array_equal(nxt, np_pack(np.where(want > 0, 1, -1)))

@@ -259,3 +259,21 @@ def test_delta_mode_equals_threshold_rule():
     F = np.float32(0.8)
     t, s = oracle.delta_ternarize(w, F)
     assert np.array_equal(t, (np.sign(w) * (np.abs(w) > F)).astype(np.int8))
+
+
+def test_ternary_linear_adds_the_bias():
+    k = 31
+    xb = _bf16(synth.normal_f32(6, 1, (2, k)))
+    trits = np.zeros((3, k), np.int8)
+    trits[0] = 1
+    trits[2, 5] = -1
+    scale = np.array([1.5, 2.0, 0.25], np.float32)
+    bias = np.array([0.5, -3.0, 8.0], np.float32)
+    packed = oracle.base3_pack(trits)
+    y0, m0 = oracle.ternary_gemm(xb, packed, scale, 2, 3, k)
+    y, mag = oracle.ternary_linear(xb, packed, scale, bias, 2, 3, k)
+    assert np.array_equal(y, y0 + bias.astype(np.float64)[None, :])
+    assert np.array_equal(mag, m0 + np.abs(bias).astype(np.float64)[None, :])
+    assert np.all(y[:, 1] == -3.0)          # all-zero trits: the bias alone
+    yn, mn = oracle.ternary_linear(xb, packed, scale, None, 2, 3, k)
+    assert np.array_equal(yn, y0) and np.array_equal(mn, m0)
