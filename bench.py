@@ -428,7 +428,7 @@ def run_workloads(cu: Cuda, args, peaks, popc_peak_macs):
     out = {}
 
     want = set(args.workloads.split(",")) if args.workloads != "all" else {"gemv_small", "gemv_ffn", "gemm_large",
-                                                                           "ternary"}
+                                                                           "ternary", "stack"}
     if "gemv_small" in want:
         out.update(wl_gemv_small(cu, args, P, st, s))
     if "gemv_ffn" in want:
@@ -437,7 +437,51 @@ def run_workloads(cu: Cuda, args, peaks, popc_peak_macs):
         out.update(wl_gemm_large(cu, args, P, st, s, popc_peak_macs, peaks))
     if "ternary" in want:
         out.update(wl_ternary(cu, args, P, st, s, hbm, peaks))
+    if "stack" in want:
+        out.update(wl_stack(cu, args, P, st, s))
     return out
+
+
+def wl_stack(cu, args, P, st, s):
+    """Two binarised 4096 -> 4096 layers on a 256-row batch (the headline layer
+    twice): fused (bnn_binary_linear: bias + the next layer's sign pack in the
+    first layer's epilogue) against unfused (GEMM, then bnn_pack_signs of its
+    float32 output, then the second GEMM)."""
+    torch, dev, lib = cu.torch, cu.device, cu.lib
+    m, n, k = 256, 4096, 4096
+    kw = synth.words_per_row(k)
+    c = synth.gemm_fused_pack(args.seed)
+    x = torch.from_numpy(c["x"]).to(dev)
+    w1 = torch.empty((n, kw), dtype=torch.int64, device=dev)
+    lib.bnn_pack_signs(P(torch.from_numpy(c["w"]).to(dev)), n, k, P(w1), cu.s)
+    w2 = torch.from_numpy(synth.fair_coin_words(args.seed + 7, 2, n, n).view(np.int64)).to(dev)
+    a1 = torch.from_numpy(c["alpha"]).to(dev)
+    a2 = torch.from_numpy(synth.uniform_f32(args.seed + 7, 3, (n,), 0.5, 1.5)).to(dev)
+    b1 = torch.from_numpy(synth.normal_f32(args.seed + 7, 4, (n,))).to(dev)
+    xp = torch.empty((m, kw), dtype=torch.int64, device=dev)
+    h = torch.empty((m, kw), dtype=torch.int64, device=dev)
+    y1 = torch.empty((m, n), dtype=torch.float32, device=dev)
+    y2 = torch.empty((m, n), dtype=torch.float32, device=dev)
+    torch.cuda.synchronize(dev)
+
+    def fused(i):
+        return lib.bnn_pack_signs(P(x), m, k, P(xp), s) or \
+            lib.bnn_binary_linear(P(xp), P(w1), P(a1), P(b1), m, n, k, None, None, P(h), s) or \
+            lib.bnn_binary_linear(P(h), P(w2), P(a2), None, m, n, n, None, P(y2), None, s)
+
+    def unfused(i):
+        return lib.bnn_pack_signs(P(x), m, k, P(xp), s) or \
+            lib.bnn_binary_gemm(P(xp), P(w1), P(a1), m, n, k, None, P(y1), s) or \
+            lib.bnn_pack_signs(P(y1), m, n, P(h), s) or \
+            lib.bnn_binary_gemm(P(h), P(w2), P(a2), m, n, n, None, P(y2), s)
+    ms_f = graph_time(cu, fused, 200, st)
+    ms_u = graph_time(cu, unfused, 200, st)
+    macs = 2.0 * m * n * k
+    return {"stack_2x_m256_n4096_k4096": dict(
+        us_fused=ms_f * 1e3, us_unfused=ms_u * 1e3, tmacs_fused=macs / (ms_f * 1e-3) / 1e12,
+        tmacs_unfused=macs / (ms_u * 1e-3) / 1e12,
+        note="fused: pack x, layer 1 with bias and the sign pack of its output in the epilogue, layer 2 "
+             "(float32 out); unfused: pack x, GEMM, pack of the float32 layer-1 output, GEMM (no bias)")}
 
 
 def wl_gemv_small(cu, args, P, st, s):

@@ -127,6 +127,32 @@ bnn_status bnn_binary_gemm_algo(const uint64_t* xp, const uint64_t* wp, const fl
                                 bnn_binary_algo algo, cudaStream_t s);
 
 /*
+ * bnn_binary_linear -- one binarised linear layer with its epilogue fused:
+ * the packed matmul of bnn_binary_gemm, the channel scale, an optional
+ * per-channel bias ([BTE] ".tbin Format": records carry per-channel biases)
+ * and the sign pack of the layer output as the next layer's packed input
+ * (binary activations from layer to layer, as in the FFN stacks of
+ * BinaryLinear layers of the "binary_nn" README).
+ *
+ *   xp, wp, m, n, k   as for bnn_binary_gemm.
+ *   alpha  float32 [n], device; required when out or next is non-NULL.
+ *   bias   float32 [n], device, or NULL for no bias.
+ *   y[i,j] = fl32(alpha[j] * (float)dot[i,j]), then, with a bias,
+ *            fl32(y[i,j] + bias[j]): two IEEE float32 operations, round to
+ *            nearest even, never fused into one multiply-add.
+ *   dots   int32 [m, n] or NULL: the exact dots (as bnn_binary_gemm).
+ *   out    float32 [m, n] or NULL: y.
+ *   next   uint64 [m, ceil(n/64)] or NULL, 8-byte aligned: row i is
+ *          bnn_pack_signs of row i of y (bit j = !(y[i,j] > 0), pad bits 0).
+ *   At least one of dots, out and next must be non-NULL.  Runs on the
+ *   tensor-core kernel family (BNN_ALGO_TC) for every m.  Errors as for
+ *   bnn_binary_gemm.
+ */
+bnn_status bnn_binary_linear(const uint64_t* xp, const uint64_t* wp, const float* alpha,
+                             const float* bias, int64_t m, int64_t n, int64_t k, int32_t* dots,
+                             float* out, uint64_t* next, cudaStream_t s);
+
+/*
  * bnn_ternary_pack -- TWN ternarisation, least-squares per-row scale and base-3
  * packing of a float32 weight matrix.  [BTE] "Features".
  *
@@ -247,6 +273,22 @@ typedef enum {
  */
 bnn_status bnn_ternary_gemm_algo(const uint16_t* x_bf16, const uint16_t* packed, const float* scale,
                                  int64_t m, int64_t n, int64_t k, float* out, int algo, cudaStream_t s);
+
+/*
+ * bnn_ternary_linear -- bnn_ternary_gemm with the layer's per-channel bias
+ * added in the epilogue ([BTE] ".tbin Format": each record carries per-channel
+ * biases; "Module Overview": Layer.forward).
+ *
+ *   bias   float32 [n], device, 4-byte aligned, or NULL (then identical to
+ *          bnn_ternary_gemm).
+ *   out[i,j] = scale[j] * sum_e x[i,e] t[j,e] + bias[j], fp32 accumulation;
+ *          within 1e-3 of |scale[j]| * sum |x t| + |bias[j]| of the exact value.
+ *   Other arguments, kernels (the AUTO family) and errors as for
+ *   bnn_ternary_gemm.
+ */
+bnn_status bnn_ternary_linear(const uint16_t* x_bf16, const uint16_t* packed, const float* scale,
+                              const float* bias, int64_t m, int64_t n, int64_t k, float* out,
+                              cudaStream_t s);
 
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* bnn_status_string(bnn_status st);

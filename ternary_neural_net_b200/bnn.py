@@ -34,11 +34,13 @@ _SIGS = {
     "bnn_pack_signs": [_vp, _i64, _i64, _vp, _vp],
     "bnn_binary_gemm": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp],
     "bnn_binary_gemm_algo": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _int, _vp],
+    "bnn_binary_linear": [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp],
     "bnn_ternary_pack": [_vp, _i64, _i64, _vp, _vp, _vp, _vp],
     "bnn_ternary_gemm": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
     "bnn_ternary_pack_mode": [_vp, _i64, _i64, _int, C.c_float, _vp, _vp, _vp, _vp],
     "bnn_ternary_gemm_algo": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _int, _vp],
     "bnn_ternary_pack_noalloc": [_vp, _i64, _i64, _vp, _vp, _vp, _vp],
+    "bnn_ternary_linear": [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
 }
 for _name, _args in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -156,6 +158,40 @@ def bnn_binary_gemm(xp: torch.Tensor, wp: torch.Tensor, alpha: torch.Tensor | No
     return dots, out
 
 
+def bnn_binary_linear(xp: torch.Tensor, wp: torch.Tensor, alpha: torch.Tensor | None,
+                      bias: torch.Tensor | None, k: int, want_dots: bool = False, want_out: bool = True,
+                      want_next: bool = True, dots: torch.Tensor | None = None,
+                      out: torch.Tensor | None = None, nxt: torch.Tensor | None = None):
+    """One binarised layer with the fused epilogue: returns (dots int32 [m,n] or None,
+    y float32 [m,n] or None, next int64 [m, ceil(n/64)] or None), y = alpha*dot (+ bias),
+    next = the sign pack of y (the next layer's packed input)."""
+    _dev(xp, "xp", torch.int64)
+    _dev(wp, "wp", torch.int64)
+    m, n = xp.shape[0], wp.shape[0]
+    if xp.shape[1] != words_per_row(k) or wp.shape[1] != words_per_row(k):
+        raise ValueError("packed rows must hold ceil(k/64) words")
+    dev = xp.device
+    if want_dots and dots is None:
+        dots = torch.empty((m, n), dtype=torch.int32, device=dev)
+    if want_out and out is None:
+        out = torch.empty((m, n), dtype=torch.float32, device=dev)
+    if want_next and nxt is None:
+        nxt = torch.empty((m, words_per_row(n)), dtype=torch.int64, device=dev)
+    if dots is not None:
+        _dev(dots, "dots", torch.int32)
+    if out is not None:
+        _dev(out, "out", torch.float32)
+    if nxt is not None:
+        _dev(nxt, "next", torch.int64)
+    if out is not None or nxt is not None:
+        _dev(alpha, "alpha", torch.float32, ndim=1)
+    if bias is not None:
+        _dev(bias, "bias", torch.float32, ndim=1)
+    _check(_lib.bnn_binary_linear(_ptr(xp), _ptr(wp), _ptr(alpha), _ptr(bias), m, n, k, _ptr(dots), _ptr(out),
+                                  _ptr(nxt), _stream(dev)), "bnn_binary_linear")
+    return dots, out, nxt
+
+
 def bnn_ternary_pack(w: torch.Tensor, packed: torch.Tensor | None = None,
                      scale: torch.Tensor | None = None, delta: torch.Tensor | None = None):
     """float32 [n, k] -> (packed int16 [n, ceil(k/10)], scale float32 [n], delta float32 [1])."""
@@ -211,4 +247,24 @@ def bnn_ternary_gemm(x: torch.Tensor, packed: torch.Tensor, scale: torch.Tensor,
         st = _lib.bnn_ternary_gemm_algo(_ptr(x), _ptr(packed), _ptr(scale), m, n, k, _ptr(out), int(algo),
                                         _stream(x.device))
     _check(st, "bnn_ternary_gemm")
+    return out
+
+
+def bnn_ternary_linear(x: torch.Tensor, packed: torch.Tensor, scale: torch.Tensor, bias: torch.Tensor | None,
+                       out: torch.Tensor | None = None) -> torch.Tensor:
+    """bnn_ternary_gemm plus the per-channel bias: float32 [m, n]."""
+    _dev(x, "x", torch.bfloat16)
+    _dev(packed, "packed", torch.int16)
+    _dev(scale, "scale", torch.float32, ndim=1)
+    m, k = x.shape
+    if packed.shape[1] != trit_words_per_row(k):
+        raise ValueError("packed rows must hold ceil(k/10) words")
+    n = packed.shape[0]
+    if bias is not None:
+        _dev(bias, "bias", torch.float32, ndim=1)
+    if out is None:
+        out = torch.empty((m, n), dtype=torch.float32, device=x.device)
+    _dev(out, "out", torch.float32)
+    _check(_lib.bnn_ternary_linear(_ptr(x), _ptr(packed), _ptr(scale), _ptr(bias), m, n, k, _ptr(out),
+                                   _stream(x.device)), "bnn_ternary_linear")
     return out

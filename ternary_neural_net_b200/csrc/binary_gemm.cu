@@ -569,7 +569,7 @@ extern "C" bnn_status bnn_binary_gemm_algo(const uint64_t* xp, const uint64_t* w
   // AUTO: tcgen05 from 64 activation rows up (measured faster than mma.sync from
   // the 64 x 4096 x 4096 layer to 8192^3), mma.sync for 9..63 rows, GEMV below.
   if (algo == BNN_ALGO_TC || (algo == BNN_ALGO_AUTO && m >= 64))
-    return bnn::binary_gemm_tc(xp, wp, alpha, m, n, ki, kw, dots, out, s);
+    return bnn::binary_gemm_tc(xp, wp, alpha, nullptr, m, n, ki, kw, dots, out, nullptr, s);
   if (algo == BNN_ALGO_MMA_S8 || (algo == BNN_ALGO_AUTO && m > 8)) {
     return vec2 ? dispatch_mma<2>(xp, wp, alpha, m, n, ki, kw, dots, out, s)
                 : dispatch_mma<1>(xp, wp, alpha, m, n, ki, kw, dots, out, s);
@@ -588,6 +588,22 @@ extern "C" bnn_status bnn_binary_gemm_algo(const uint64_t* xp, const uint64_t* w
   }
   return vec2 ? launch_tiled<4, 4, 2>(xp, wp, alpha, m, n, ki, kw, dots, out, s)
               : launch_tiled<4, 4, 1>(xp, wp, alpha, m, n, ki, kw, dots, out, s);
+}
+
+extern "C" bnn_status bnn_binary_linear(const uint64_t* xp, const uint64_t* wp, const float* alpha,
+                                        const float* bias, int64_t m, int64_t n, int64_t k, int32_t* dots,
+                                        float* out, uint64_t* next, cudaStream_t s) {
+  if (m < 0 || n < 0 || k < 0 || k > BNN_MAX_K_BINARY) return BNN_ERR_INVALID_ARG;
+  if (!dots && !out && !next) return BNN_ERR_INVALID_ARG;
+  if ((out || next) && !alpha) return BNN_ERR_INVALID_ARG;
+  if (m == 0 || n == 0) return BNN_OK;
+  if (k > 0 && (!xp || !wp)) return BNN_ERR_INVALID_ARG;
+  if ((xp && !bnn::aligned(xp, 8)) || (wp && !bnn::aligned(wp, 8)) || (alpha && !bnn::aligned(alpha, 4)) ||
+      (bias && !bnn::aligned(bias, 4)) || (dots && !bnn::aligned(dots, 4)) || (out && !bnn::aligned(out, 4)) ||
+      (next && !bnn::aligned(next, 8)))
+    return BNN_ERR_MISALIGNED;
+  return bnn::binary_gemm_tc(xp, wp, alpha, bias, m, n, static_cast<int>(k), static_cast<int>(bnn::words64(k)),
+                             dots, out, next, s);
 }
 
 extern "C" bnn_status bnn_binary_gemm(const uint64_t* xp, const uint64_t* wp, const float* alpha,

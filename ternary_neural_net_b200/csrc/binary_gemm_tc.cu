@@ -27,8 +27,10 @@
 //     accumulators, so that back-to-back MMAs do not depend on each other;
 //   - the epilogue (warps 0-7; warp w reads tensor-memory lanes 32(w%4).. and
 //     half w/4 of the columns): tcgen05.ld, the popcount correction, alpha,
-//     and stores in which the 32 lanes of a warp write 32 consecutive weight
-//     columns of one output row.
+//     the optional bias, and stores in which the 32 lanes of a warp write 32
+//     consecutive weight columns of one output row.  Those 32 columns are also
+//     one 32-bit half of a word of the next layer's packed input, so the
+//     optional sign pack of the layer output is one __ballot_sync per row.
 // Any bijection between the 128 bits and the 128 k-slots of a stage gives the
 // same sum when both operands use it; here byte j of word s of 16-byte chunk
 // 2h+q holds bit 32h + 8j + 4q + s.
@@ -172,8 +174,9 @@ template <int BN, int KS, int ACC, bool TMA>
 __global__ void __launch_bounds__(TcCfg<BN, TMA>::kThreads, TcCfg<BN, TMA>::kMinBlocks)
 binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                       const uint64_t* __restrict__ xp, const uint64_t* __restrict__ wp,
-                      const float* __restrict__ alpha, int64_t m, int64_t n, int k, int kw,
-                      int32_t* __restrict__ dots, float* __restrict__ out) {
+                      const float* __restrict__ alpha, const float* __restrict__ bias, int64_t m, int64_t n,
+                      int k, int kw, int32_t* __restrict__ dots, float* __restrict__ out,
+                      uint32_t* __restrict__ next, int64_t next_w32) {
   using Cfg = TcCfg<BN, TMA>;
   constexpr int S = Cfg::S;
   constexpr int P = TMA ? Cfg::P : 1;
@@ -404,31 +407,47 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
       for (int c = 0; c < 16; ++c) r[c] = 0u;
     }
   };
+  // y = fl32(alpha * dot), then fl32(y + bias) when there is a bias (two
+  // roundings: no fused multiply-add); the next layer's input bit is !(y > 0)
+  auto layer_y = [&](float a, float b, int32_t d) {
+    const float y = __fmul_rn(a, static_cast<float>(d));
+    return bias ? __fadd_rn(y, b) : y;
+  };
+  const bool need_y = out || next;
   if constexpr (KS == 1) {
     if (warp < 8 && good) {
       const int64_t jrow = j0 + erow;
       const bool jlive = jrow < n;
-      const float a_j = (out && jlive) ? __ldg(alpha + jrow) : 0.0f;
+      const float a_j = (need_y && jlive) ? __ldg(alpha + jrow) : 0.0f;
+      const float b_j = (bias && jlive) ? __ldg(bias + jrow) : 0.0f;
       const int base = k - 2 * pop_w[erow];
+      // this warp's 32 weight rows form one 32-bit half of a packed word of `next`
+      const int64_t half = (j0 + 32 * (warp & 3)) / 32;
+      const bool pack = next && half < next_w32;  // uniform across the warp
       for (int c0 = ecol0; c0 < ecol0 + BN / 2; c0 += 16) {
         uint32_t r[16];
         load16(c0, r);
         const int64_t rows_left = m - (i0 + c0);
-        if (jlive && rows_left > 0) {
-          const int nc = rows_left < 16 ? static_cast<int>(rows_left) : 16;
-          const int64_t off = (i0 + c0) * n + jrow;
-          int32_t* dp = dots ? dots + off : nullptr;
-          float* op = out ? out + off : nullptr;
+        const int nc = rows_left <= 0 ? 0 : (rows_left < 16 ? static_cast<int>(rows_left) : 16);
+        const int64_t off = (i0 + c0) * n + jrow;
+        int32_t* dp = dots ? dots + off : nullptr;
+        float* op = out ? out + off : nullptr;
+        uint32_t* np = pack ? next + (i0 + c0) * next_w32 + half : nullptr;
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            if (c < nc) {
-              const int32_t d = base - 2 * pop_x[c0 + c] + 4 * static_cast<int32_t>(r[c]);
-              if (dp) *dp = d;
-              if (op) *op = a_j * static_cast<float>(d);
-            }
-            dp += n;
-            op += n;
+        for (int c = 0; c < 16; ++c) {
+          const int32_t d = base - 2 * pop_x[c0 + c] + 4 * static_cast<int32_t>(r[c]);
+          const float y = layer_y(a_j, b_j, d);
+          if (c < nc && jlive) {
+            if (dp) *dp = d;
+            if (op) *op = y;
           }
+          if (np) {
+            const unsigned bits = __ballot_sync(0xffffffffu, jlive && !(y > 0.0f));
+            if ((tid & 31) == 0 && c < nc) *np = bits;
+            np += next_w32;
+          }
+          dp += n;
+          op += n;
         }
       }
     }
@@ -463,28 +482,37 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
     }
     cluster.sync();  // every share has landed
     if (any_bad == 0) {
+      // a warp's 32 lanes take 32 consecutive weight rows (one 32-bit half of a
+      // packed word of `next`) and the same four activation rows
       for (int e = tid; e < kTm * (kCols / 4); e += blockDim.x) {
         const int row = e % kTm, cl = 4 * (e / kTm);
         const int64_t jrow = j0 + row;
-        if (jrow < n) {
-          int4 d = make_int4(k, k, k, k);
+        const bool jlive = jrow < n;
+        int4 d = make_int4(k, k, k, k);
 #pragma unroll
-          for (int q = 0; q < KS; ++q) {
-            const int4 v = *reinterpret_cast<const int4*>(recv + (q * kTm + row) * kPitch + cl);
-            d.x += v.x;
-            d.y += v.y;
-            d.z += v.z;
-            d.w += v.w;
+        for (int q = 0; q < KS; ++q) {
+          const int4 v = *reinterpret_cast<const int4*>(recv + (q * kTm + row) * kPitch + cl);
+          d.x += v.x;
+          d.y += v.y;
+          d.z += v.z;
+          d.w += v.w;
+        }
+        const float a_j = (need_y && jlive) ? __ldg(alpha + jrow) : 0.0f;
+        const float b_j = (bias && jlive) ? __ldg(bias + jrow) : 0.0f;
+        const int64_t half = (j0 + row - (tid & 31)) / 32;
+        const bool pack = next && half < next_w32;  // uniform across the warp
+        const int dv[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int64_t gi = i0 + rank * kCols + cl + t;
+          const float y = layer_y(a_j, b_j, dv[t]);
+          if (gi < m && jlive) {
+            if (dots) dots[gi * n + jrow] = dv[t];
+            if (out) out[gi * n + jrow] = y;
           }
-          const float a_j = out ? __ldg(alpha + jrow) : 0.0f;
-          const int dv[4] = {d.x, d.y, d.z, d.w};
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const int64_t gi = i0 + rank * kCols + cl + t;
-            if (gi < m) {
-              if (dots) dots[gi * n + jrow] = dv[t];
-              if (out) out[gi * n + jrow] = a_j * static_cast<float>(dv[t]);
-            }
+          if (pack) {
+            const unsigned bits = __ballot_sync(0xffffffffu, jlive && !(y > 0.0f));
+            if ((tid & 31) == 0 && gi < m) next[gi * next_w32 + half] = bits;
           }
         }
       }
@@ -498,8 +526,8 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
 }
 
 template <int BN, int KS, int ACC>
-bnn_status launch_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha, int64_t m, int64_t n, int k, int kw,
-                     int32_t* dots, float* out, cudaStream_t s) {
+bnn_status launch_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha, const float* bias, int64_t m,
+                     int64_t n, int k, int kw, int32_t* dots, float* out, uint64_t* next, cudaStream_t s) {
   const int64_t gx = KS * ((n + kTm - 1) / kTm), gy = (m + BN - 1) / BN;
   if (gx > 2147483647LL || gy > 65535) return BNN_ERR_INVALID_ARG;
   // TMA needs 16-byte aligned rows (even kw, aligned bases) and coordinates that fit int32
@@ -519,7 +547,8 @@ bnn_status launch_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha,
   BNN_TRY(bnn::ensure_smem(kern, smem));
   const cudaError_t e = bnn::launch_pdl(kern, dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)),
                                         dim3(tma ? TcCfg<BN, true>::kThreads : TcCfg<BN, false>::kThreads), smem, s,
-                                        KS, tw, tx, xp, wp, alpha, m, n, k, kw, dots, out);
+                                        KS, tw, tx, xp, wp, alpha, bias, m, n, k, kw, dots, out,
+                                        reinterpret_cast<uint32_t*>(next), 2 * bnn::words64(n));
   if (e != cudaSuccess) return bnn::cuda_fail(e);
   return bnn::check_launch();
 }
@@ -534,16 +563,19 @@ namespace bnn {
 // per SM), with a cluster of 4 CTAs splitting each tile's stages when that
 // still leaves at most one CTA per SM, else of 2 when the CTAs fit in one
 // wave (at least 4 stages per CTA either way).
-bnn_status binary_gemm_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha, int64_t m, int64_t n, int k,
-                          int kw, int32_t* dots, float* out, cudaStream_t s) {
+bnn_status binary_gemm_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha, const float* bias, int64_t m,
+                          int64_t n, int k, int kw, int32_t* dots, float* out, uint64_t* next, cudaStream_t s) {
   const int64_t wt = (n + kTm - 1) / kTm;
   const int64_t sms = sm_count();
   const int ktiles = (kw + 1) / 2;
-  if (wt * ((m + 255) / 256) >= sms) return launch_tc<256, 1, 1>(xp, wp, alpha, m, n, k, kw, dots, out, s);
+  if (wt * ((m + 255) / 256) >= sms)
+    return launch_tc<256, 1, 1>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
   const int64_t tiles = wt * ((m + 63) / 64);
-  if (tiles * 4 <= sms && ktiles >= 16) return launch_tc<64, 4, 1>(xp, wp, alpha, m, n, k, kw, dots, out, s);
-  if (tiles * 2 <= 2 * sms && ktiles >= 8) return launch_tc<64, 2, 1>(xp, wp, alpha, m, n, k, kw, dots, out, s);
-  return launch_tc<64, 1, 1>(xp, wp, alpha, m, n, k, kw, dots, out, s);
+  if (tiles * 4 <= sms && ktiles >= 16)
+    return launch_tc<64, 4, 1>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
+  if (tiles * 2 <= 2 * sms && ktiles >= 8)
+    return launch_tc<64, 2, 1>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
+  return launch_tc<64, 1, 1>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
 }
 
 }  // namespace bnn

@@ -75,16 +75,18 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
 }
 
-// Tensor-core (tcgen05 kind::i8) binary GEMM, in binary_gemm_tc.cu.
-bnn_status binary_gemm_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha, int64_t m, int64_t n, int k,
-                          int kw, int32_t* dots, float* out, cudaStream_t s);
+// Tensor-core (tcgen05 kind::i8) binary GEMM, in binary_gemm_tc.cu, with the
+// optional layer epilogue: bias (may be null) and the sign-packed output for
+// the next layer (next, may be null; ceil(n/64) words per row).
+bnn_status binary_gemm_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha, const float* bias, int64_t m,
+                          int64_t n, int k, int kw, int32_t* dots, float* out, uint64_t* next, cudaStream_t s);
 
 // Bounded waits that ran out in the ternary tensor-core kernel (reset != 0 clears).
 int ternary_tc_error_count(int reset);
 
 // Tensor-core (tcgen05 kind::f16) ternary GEMM, in ternary_gemm_tc.cu.
-bnn_status ternary_gemm_tc(const uint16_t* x_bf16, const uint16_t* packed, const float* scale, int64_t m, int64_t n,
-                           int64_t k, float* out, cudaStream_t s);
+bnn_status ternary_gemm_tc(const uint16_t* x_bf16, const uint16_t* packed, const float* scale, const float* bias,
+                           int64_t m, int64_t n, int64_t k, float* out, cudaStream_t s);
 
 }  // namespace bnn
 

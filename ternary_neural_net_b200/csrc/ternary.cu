@@ -154,7 +154,7 @@ template <int MT>
 __global__ void __launch_bounds__(256)
 ternary_gemv_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ packed,
                     const float* __restrict__ scale, int m, int64_t n, int64_t k, int64_t kt,
-                    float* __restrict__ out) {
+                    float* __restrict__ out, const float* __restrict__ bias) {
   const int lane = threadIdx.x & 31;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
@@ -186,7 +186,7 @@ ternary_gemv_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__
       const float s = __ldg(scale + r);
 #pragma unroll
       for (int t = 0; t < MT; ++t)
-        if (t < m) out[static_cast<int64_t>(t) * n + r] = s * acc[t];
+        if (t < m) out[static_cast<int64_t>(t) * n + r] = bias ? s * acc[t] + __ldg(bias + r) : s * acc[t];
     }
   }
 }
@@ -220,7 +220,7 @@ template <int SLICES>
 __global__ void __launch_bounds__(kLutRows * SLICES, 1)
 ternary_gemv_lut_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ packed,
                         const float* __restrict__ scale, int64_t n, int k, int kt, int slice_words,
-                        float* __restrict__ out) {
+                        float* __restrict__ out, const float* __restrict__ bias) {
   constexpr int THREADS = kLutRows * SLICES;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int npairs = 5 * kt;
@@ -295,7 +295,7 @@ ternary_gemv_lut_kernel(const uint16_t* __restrict__ x, const uint16_t* __restri
         float s = 0.0f;
 #pragma unroll 4
         for (int q = 0; q < SLICES; ++q) s += red[q * kLutRows + tid];
-        out[r] = __ldg(scale + r) * s;
+        out[r] = bias ? __ldg(scale + r) * s + __ldg(bias + r) : __ldg(scale + r) * s;
       }
     }
     // The buffer of chunk it + kLutStages - 1 (the one computed in the previous
@@ -357,7 +357,7 @@ template <bool VECX>
 __global__ void __cluster_dims__(kTK, 1, 1) __launch_bounds__(kTThreads)
 ternary_gemm_mma_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ packed,
                         const float* __restrict__ scale, int64_t m, int64_t n, int64_t k, int64_t kt,
-                        int64_t slice_words, float* __restrict__ out) {
+                        int64_t slice_words, float* __restrict__ out, const float* __restrict__ bias) {
   extern __shared__ __align__(16) uint16_t tsm[];
   uint16_t (*Xs)[kTBM * kTPitch] = reinterpret_cast<uint16_t (*)[kTBM * kTPitch]>(tsm);                // [2]
   uint16_t (*Ws)[kTBN * kTPitch] = reinterpret_cast<uint16_t (*)[kTBN * kTPitch]>(tsm + 2 * kTBM * kTPitch);  // [2]
@@ -498,7 +498,7 @@ ternary_gemm_mma_kernel(const uint16_t* __restrict__ x, const uint16_t* __restri
       float s = part[idx];
 #pragma unroll
       for (int q = 1; q < kTK; ++q) s += cluster.map_shared_rank(part, q)[idx];
-      if (gm < m && gn < n) out[gm * n + gn] = __ldg(scale + gn) * s;
+      if (gm < m && gn < n) out[gm * n + gn] = bias ? __ldg(scale + gn) * s + __ldg(bias + gn) : __ldg(scale + gn) * s;
     }
   }
   cluster.sync();  // keep every CTA's partial tile alive until rank 0 has read it
@@ -539,8 +539,9 @@ extern "C" bnn_status bnn_ternary_pack(const float* w, int64_t n, int64_t k, uin
   return st;
 }
 
-extern "C" bnn_status bnn_ternary_gemm_algo(const uint16_t* x_bf16, const uint16_t* packed, const float* scale,
-                                            int64_t m, int64_t n, int64_t k, float* out, int algo, cudaStream_t s) {
+namespace {
+bnn_status ternary_gemm_impl(const uint16_t* x_bf16, const uint16_t* packed, const float* scale, const float* bias,
+                             int64_t m, int64_t n, int64_t k, float* out, int algo, cudaStream_t s) {
   if (algo != BNN_TALGO_AUTO && algo != BNN_TALGO_CUDA_CORES && algo != BNN_TALGO_MMA && algo != BNN_TALGO_TC)
     return BNN_ERR_INVALID_ARG;
   if (algo == BNN_TALGO_CUDA_CORES && m > 8) return BNN_ERR_UNSUPPORTED;
@@ -548,10 +549,10 @@ extern "C" bnn_status bnn_ternary_gemm_algo(const uint16_t* x_bf16, const uint16
   if (m == 0 || n == 0) return BNN_OK;
   if (!scale || !out || (k > 0 && (!x_bf16 || !packed))) return BNN_ERR_INVALID_ARG;
   if ((x_bf16 && !bnn::aligned(x_bf16, 2)) || (packed && !bnn::aligned(packed, 2)) || !bnn::aligned(scale, 4) ||
-      !bnn::aligned(out, 4))
+      !bnn::aligned(out, 4) || (bias && !bnn::aligned(bias, 4)))
     return BNN_ERR_MISALIGNED;
   const int64_t kt = bnn::words10(k);
-  if (algo == BNN_TALGO_TC) return bnn::ternary_gemm_tc(x_bf16, packed, scale, m, n, k, out, s);
+  if (algo == BNN_TALGO_TC) return bnn::ternary_gemm_tc(x_bf16, packed, scale, bias, m, n, k, out, s);
   if (algo != BNN_TALGO_MMA && m == 1 && kt > 0 && bnn::aligned(packed, 16) && lut_smem_bytes(kt) <= 200 * 1024) {
     const size_t smem = lut_smem_bytes(kt);
     auto kern = ternary_gemv_lut_kernel<kLutSlices>;
@@ -560,7 +561,7 @@ extern "C" bnn_status bnn_ternary_gemm_algo(const uint16_t* x_bf16, const uint16
     const int64_t nchunks = (n + kLutRows - 1) / kLutRows;
     const int grid = static_cast<int>(nchunks < bnn::sm_count() ? nchunks : bnn::sm_count());
     kern<<<grid, kLutRows * kLutSlices, smem, s>>>(x_bf16, packed, scale, n, static_cast<int>(k), static_cast<int>(kt),
-                                                  slice_words, out);
+                                                  slice_words, out, bias);
     return bnn::check_launch();
   }
   if (algo != BNN_TALGO_MMA && m <= 8) {
@@ -568,9 +569,10 @@ extern "C" bnn_status bnn_ternary_gemm_algo(const uint16_t* x_bf16, const uint16
     const int64_t blocks_needed = (n + warps_per_block - 1) / warps_per_block;
     const int64_t cap = static_cast<int64_t>(bnn::sm_count()) * 8;
     const int grid = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
-    if (m == 1) ternary_gemv_kernel<1><<<grid, 256, 0, s>>>(x_bf16, packed, scale, 1, n, k, kt, out);
-    else if (m <= 4) ternary_gemv_kernel<4><<<grid, 256, 0, s>>>(x_bf16, packed, scale, static_cast<int>(m), n, k, kt, out);
-    else ternary_gemv_kernel<8><<<grid, 256, 0, s>>>(x_bf16, packed, scale, static_cast<int>(m), n, k, kt, out);
+    if (m == 1) ternary_gemv_kernel<1><<<grid, 256, 0, s>>>(x_bf16, packed, scale, 1, n, k, kt, out, bias);
+    else if (m <= 4)
+      ternary_gemv_kernel<4><<<grid, 256, 0, s>>>(x_bf16, packed, scale, static_cast<int>(m), n, k, kt, out, bias);
+    else ternary_gemv_kernel<8><<<grid, 256, 0, s>>>(x_bf16, packed, scale, static_cast<int>(m), n, k, kt, out, bias);
     return bnn::check_launch();
   }
   const int64_t ntiles = (n + kTBN - 1) / kTBN, gy = (m + kTBM - 1) / kTBM;
@@ -582,12 +584,26 @@ extern "C" bnn_status bnn_ternary_gemm_algo(const uint16_t* x_bf16, const uint16
   const size_t smem = 2 * static_cast<size_t>(kTBM + kTBN) * kTPitch * sizeof(uint16_t) + 9 * sizeof(uint32_t);
   if (k % 8 == 0 && bnn::aligned(x_bf16, 16)) {
     BNN_TRY(bnn::ensure_smem(ternary_gemm_mma_kernel<true>, smem));
-    ternary_gemm_mma_kernel<true><<<grid, kTThreads, smem, s>>>(x_bf16, packed, scale, m, n, k, kt, slice_words, out);
+    ternary_gemm_mma_kernel<true><<<grid, kTThreads, smem, s>>>(x_bf16, packed, scale, m, n, k, kt, slice_words, out,
+                                                                bias);
   } else {
     BNN_TRY(bnn::ensure_smem(ternary_gemm_mma_kernel<false>, smem));
-    ternary_gemm_mma_kernel<false><<<grid, kTThreads, smem, s>>>(x_bf16, packed, scale, m, n, k, kt, slice_words, out);
+    ternary_gemm_mma_kernel<false><<<grid, kTThreads, smem, s>>>(x_bf16, packed, scale, m, n, k, kt, slice_words, out,
+                                                                 bias);
   }
   return bnn::check_launch();
+}
+}  // namespace
+
+extern "C" bnn_status bnn_ternary_gemm_algo(const uint16_t* x_bf16, const uint16_t* packed, const float* scale,
+                                            int64_t m, int64_t n, int64_t k, float* out, int algo, cudaStream_t s) {
+  return ternary_gemm_impl(x_bf16, packed, scale, nullptr, m, n, k, out, algo, s);
+}
+
+extern "C" bnn_status bnn_ternary_linear(const uint16_t* x_bf16, const uint16_t* packed, const float* scale,
+                                         const float* bias, int64_t m, int64_t n, int64_t k, float* out,
+                                         cudaStream_t s) {
+  return ternary_gemm_impl(x_bf16, packed, scale, bias, m, n, k, out, BNN_TALGO_AUTO, s);
 }
 
 extern "C" bnn_status bnn_ternary_gemm(const uint16_t* x_bf16, const uint16_t* packed, const float* scale,

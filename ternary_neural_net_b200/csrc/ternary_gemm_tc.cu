@@ -77,7 +77,7 @@ template <bool VECX>
 __global__ void __cluster_dims__(kTcK, 1, 1) __launch_bounds__(kTcThreads)
 ternary_gemm_tc_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ packed,
                        const float* __restrict__ scale, int64_t m, int64_t n, int64_t k, int64_t kt,
-                       int64_t slice_stages, float* __restrict__ out) {
+                       int64_t slice_stages, float* __restrict__ out, const float* __restrict__ bias) {
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ __align__(16) uint8_t tsm_raw[];
@@ -284,7 +284,7 @@ ternary_gemm_tc_kernel(const uint16_t* __restrict__ x, const uint16_t* __restric
 #pragma unroll
       for (int q = 1; q < kTcK; ++q) sum += cluster.map_shared_rank(part, q)[wr * PP + xr];
       const int64_t gn = n0 + wr, gm = m0 + xr;
-      if (gn < n && gm < m) out[gm * n + gn] = __ldg(scale + gn) * sum;
+      if (gn < n && gm < m) out[gm * n + gn] = bias ? __ldg(scale + gn) * sum + __ldg(bias + gn) : __ldg(scale + gn) * sum;
     }
   }
   cluster.sync();  // partial tiles stay alive until rank 0 has read them
@@ -307,8 +307,8 @@ int ternary_tc_error_count(int reset) {
   return static_cast<int>(v);
 }
 
-bnn_status ternary_gemm_tc(const uint16_t* x_bf16, const uint16_t* packed, const float* scale, int64_t m, int64_t n,
-                           int64_t k, float* out, cudaStream_t s) {
+bnn_status ternary_gemm_tc(const uint16_t* x_bf16, const uint16_t* packed, const float* scale, const float* bias,
+                           int64_t m, int64_t n, int64_t k, float* out, cudaStream_t s) {
   const int64_t kt = words10(k);
   const int64_t ntiles = (n + kTcMW - 1) / kTcMW, gy = (m + kTcNX - 1) / kTcNX;
   if (ntiles * kTcK > 2147483647LL || gy > 65535) return BNN_ERR_INVALID_ARG;
@@ -318,11 +318,12 @@ bnn_status ternary_gemm_tc(const uint16_t* x_bf16, const uint16_t* packed, const
   const dim3 grid(static_cast<unsigned>(ntiles * kTcK), static_cast<unsigned>(gy));
   if (k % 8 == 0 && aligned(x_bf16, 16)) {
     BNN_TRY(ensure_smem(ternary_gemm_tc_kernel<true>, smem));
-    ternary_gemm_tc_kernel<true><<<grid, kTcThreads, smem, s>>>(x_bf16, packed, scale, m, n, k, kt, slice_stages, out);
+    ternary_gemm_tc_kernel<true><<<grid, kTcThreads, smem, s>>>(x_bf16, packed, scale, m, n, k, kt, slice_stages, out,
+                                                                bias);
   } else {
     BNN_TRY(ensure_smem(ternary_gemm_tc_kernel<false>, smem));
     ternary_gemm_tc_kernel<false><<<grid, kTcThreads, smem, s>>>(x_bf16, packed, scale, m, n, k, kt, slice_stages,
-                                                                 out);
+                                                                 out, bias);
   }
   return check_launch();
 }

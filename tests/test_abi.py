@@ -82,3 +82,32 @@ def test_binding_rejects_host_tensors(bnn):
     import torch
     with pytest.raises(ValueError):
         bnn.bnn_pack_signs(torch.zeros(2, 3))
+
+
+def test_binary_linear_host_checks(bnn):
+    lib = bnn.lib()
+    P = C.c_void_p
+    g = P(0x1000)
+    # no output at all; out or next without alpha
+    assert lib.bnn_binary_linear(g, g, g, None, 1, 1, 64, None, None, None, None) == bnn.BNN_ERR_INVALID_ARG
+    assert lib.bnn_binary_linear(g, g, None, None, 1, 1, 64, None, g, None, None) == bnn.BNN_ERR_INVALID_ARG
+    assert lib.bnn_binary_linear(g, g, None, None, 1, 1, 64, None, None, g, None) == bnn.BNN_ERR_INVALID_ARG
+    # dots alone need no alpha; sizes and k bound as for the GEMM
+    assert lib.bnn_binary_linear(g, g, None, None, 1, -1, 64, g, None, None, None) == bnn.BNN_ERR_INVALID_ARG
+    assert lib.bnn_binary_linear(g, g, g, None, 1, 1, (1 << 24) + 1, g, None, None, None) == bnn.BNN_ERR_INVALID_ARG
+    # misaligned next (8 bytes) and bias (4 bytes)
+    assert lib.bnn_binary_linear(g, g, g, None, 1, 1, 64, None, None, P(0x1004), None) == bnn.BNN_ERR_MISALIGNED
+    assert lib.bnn_binary_linear(g, g, g, P(0x1002), 1, 1, 64, None, g, None, None) == bnn.BNN_ERR_MISALIGNED
+    # empty problems launch nothing
+    assert lib.bnn_binary_linear(None, None, None, None, 0, 7, 64, g, None, None, None) == bnn.BNN_OK
+    assert lib.bnn_binary_linear(None, None, g, None, 3, 0, 64, None, None, g, None) == bnn.BNN_OK
+
+
+def test_ternary_linear_host_checks(bnn):
+    lib = bnn.lib()
+    P = C.c_void_p
+    g = P(0x1000)
+    assert lib.bnn_ternary_linear(g, g, g, g, 1, -1, 3, g, None) == bnn.BNN_ERR_INVALID_ARG
+    assert lib.bnn_ternary_linear(g, g, None, g, 1, 1, 3, g, None) == bnn.BNN_ERR_INVALID_ARG
+    assert lib.bnn_ternary_linear(g, g, g, P(0x1002), 1, 1, 3, g, None) == bnn.BNN_ERR_MISALIGNED
+    assert lib.bnn_ternary_linear(None, None, None, None, 0, 3, 3, g, None) == bnn.BNN_OK
