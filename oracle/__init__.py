@@ -32,6 +32,10 @@ def _L():
             "oracle_binary_gemm_sampled": ([vp, vp, vp, i64, i64, i64, vp, vp, i64, vp, vp], None),
             "oracle_binary_linear": ([vp, vp, vp, vp, i64, i64, i64, vp, vp, vp], None),
             "oracle_ternary_linear": ([vp, vp, vp, vp, i64, i64, i64, vp, vp], None),
+            "oracle_sparse_count": ([vp, i64, i64, vp], i64),
+            "oracle_sparse_encode": ([vp, i64, i64, vp, vp], None),
+            "oracle_sparse_decode": ([vp, vp, i64, i64, vp], i64),
+            "oracle_sparse_gemm": ([vp, vp, vp, vp, vp, i64, i64, i64, vp, vp], None),
             "oracle_twn_ternarize": ([vp, i64, i64, vp, vp, vp], None),
             "oracle_twn_delta": ([vp, i64], C.c_float),
             "oracle_absmean_ternarize": ([vp, i64, i64, vp, vp, vp], None),
@@ -128,6 +132,38 @@ def ternary_linear(x_bf16, packed, scale, bias, m: int, n: int, k: int):
     y = np.zeros((m, n), dtype=np.float64)
     mag = np.zeros((m, n), dtype=np.float64)
     _L().oracle_ternary_linear(_p(x_bf16), _p(packed), _p(scale), _p(bias), m, n, k, _p(y), _p(mag))
+    return y, mag
+
+
+def sparse_encode(trits):
+    """int8 trits [n,k] -> (row_ptr int64 [n+1], entries uint16 [nnz]): index + sign
+    entries (position in bits 0..14, bit 15 for -1), rows in order."""
+    trits = _c(trits, np.int8)
+    n, k = trits.shape
+    row_ptr = np.zeros(n + 1, dtype=np.int64)
+    nnz = int(_L().oracle_sparse_count(_p(trits), n, k, _p(row_ptr)))
+    entries = np.zeros(max(nnz, 1), dtype=np.uint16)
+    _L().oracle_sparse_encode(_p(trits), n, k, _p(row_ptr), _p(entries))
+    return row_ptr, entries[:nnz]
+
+
+def sparse_decode(row_ptr, entries, n: int, k: int):
+    """Inverse of sparse_encode: (trits int8 [n,k], count of malformed entries)."""
+    row_ptr, entries = _c(row_ptr, np.int64), _c(entries, np.uint16)
+    trits = np.zeros((n, k), dtype=np.int8)
+    bad = _L().oracle_sparse_decode(_p(row_ptr), _p(entries if entries.size else np.zeros(1, np.uint16)), n, k,
+                                    _p(trits))
+    return trits, int(bad)
+
+
+def sparse_gemm(x_bf16, row_ptr, entries, scale, bias, m: int, n: int, k: int):
+    """Sparse ternary layer in float64: (y [m,n], mag [m,n])."""
+    x_bf16, row_ptr, scale = _c(x_bf16, np.uint16), _c(row_ptr, np.int64), _c(scale, np.float32)
+    entries = _c(entries, np.uint16) if len(entries) else np.zeros(1, np.uint16)
+    bias = None if bias is None else _c(bias, np.float32)
+    y = np.zeros((m, n), dtype=np.float64)
+    mag = np.zeros((m, n), dtype=np.float64)
+    _L().oracle_sparse_gemm(_p(x_bf16), _p(row_ptr), _p(entries), _p(scale), _p(bias), m, n, k, _p(y), _p(mag))
     return y, mag
 
 

@@ -315,6 +315,70 @@ void oracle_ternary_linear(const uint16_t* x_bf16, const uint16_t* packed, const
     }
 }
 
+// [BTE] "Features" (sparse encoding: an index + sign format for high-sparsity
+// layers) and "Module Overview" (Packer.pack_sparse).  Reading: for each weight
+// row, the positions of its non-zero trits in increasing order, one 16-bit
+// entry each -- the position in bits 0..14 (so k <= 32768) and bit 15 set when
+// the trit is -1; row j's entries are entries[row_ptr[j] .. row_ptr[j+1]),
+// row_ptr[0] = 0.
+int64_t oracle_sparse_count(const int8_t* trits, int64_t n, int64_t k, int64_t* row_ptr) {
+  row_ptr[0] = 0;
+  for (int64_t j = 0; j < n; ++j) {
+    int64_t c = 0;
+    for (int64_t e = 0; e < k; ++e) c += trits[j * k + e] != 0 ? 1 : 0;
+    row_ptr[j + 1] = row_ptr[j] + c;
+  }
+  return row_ptr[n];
+}
+
+void oracle_sparse_encode(const int8_t* trits, int64_t n, int64_t k, const int64_t* row_ptr, uint16_t* entries) {
+  for (int64_t j = 0; j < n; ++j) {
+    int64_t at = row_ptr[j];
+    for (int64_t e = 0; e < k; ++e) {
+      const int8_t t = trits[j * k + e];
+      if (t != 0) entries[at++] = uint16_t(uint16_t(e) | (t < 0 ? 0x8000u : 0u));
+    }
+  }
+}
+
+// Inverse of oracle_sparse_encode; returns the number of malformed entries
+// (position >= k, or positions not strictly increasing within a row).
+int64_t oracle_sparse_decode(const int64_t* row_ptr, const uint16_t* entries, int64_t n, int64_t k, int8_t* trits) {
+  int64_t bad = 0;
+  for (int64_t e = 0; e < n * k; ++e) trits[e] = 0;
+  for (int64_t j = 0; j < n; ++j) {
+    int64_t prev = -1;
+    for (int64_t q = row_ptr[j]; q < row_ptr[j + 1]; ++q) {
+      const int64_t pos = entries[q] & 0x7FFF;
+      if (pos >= k || pos <= prev) {
+        ++bad;
+        continue;
+      }
+      prev = pos;
+      trits[j * k + pos] = (entries[q] & 0x8000) ? -1 : 1;
+    }
+  }
+  return bad;
+}
+
+// The sparse layer: y[i,j] = scale_j * sum over row j's entries of (+-1) *
+// x[i, position] (+ bias_j), in float64, with mag as in oracle_ternary_linear.
+void oracle_sparse_gemm(const uint16_t* x_bf16, const int64_t* row_ptr, const uint16_t* entries, const float* scale,
+                        const float* bias, int64_t m, int64_t n, int64_t k, double* out, double* mag) {
+  (void)k;
+  for (int64_t i = 0; i < m; ++i)
+    for (int64_t j = 0; j < n; ++j) {
+      double acc = 0.0, acc_abs = 0.0;
+      for (int64_t q = row_ptr[j]; q < row_ptr[j + 1]; ++q) {
+        const double v = bf16_to_double(x_bf16[i * k + (entries[q] & 0x7FFF)]);
+        acc += (entries[q] & 0x8000) ? -v : v;
+        acc_abs += std::fabs(v);
+      }
+      out[i * n + j] = double(scale[j]) * acc + (bias ? double(bias[j]) : 0.0);
+      if (mag) mag[i * n + j] = std::fabs(double(scale[j])) * acc_abs + (bias ? std::fabs(double(bias[j])) : 0.0);
+    }
+}
+
 void oracle_ternary_gemm_sampled(const uint16_t* x_bf16, const uint16_t* packed,
                                  const float* scale, int64_t m, int64_t n, int64_t k,
                                  const int64_t* rows, const int64_t* cols, int64_t count,

@@ -33,6 +33,11 @@ void oracle_ternary_gemm(const uint16_t* x_bf16, const uint16_t* packed, const f
                          int64_t m, int64_t n, int64_t k, double* out, double* mag);
 void oracle_ternary_linear(const uint16_t* x_bf16, const uint16_t* packed, const float* scale, const float* bias,
                            int64_t m, int64_t n, int64_t k, double* out, double* mag);
+int64_t oracle_sparse_count(const int8_t* trits, int64_t n, int64_t k, int64_t* row_ptr);
+void oracle_sparse_encode(const int8_t* trits, int64_t n, int64_t k, const int64_t* row_ptr, uint16_t* entries);
+int64_t oracle_sparse_decode(const int64_t* row_ptr, const uint16_t* entries, int64_t n, int64_t k, int8_t* trits);
+void oracle_sparse_gemm(const uint16_t* x_bf16, const int64_t* row_ptr, const uint16_t* entries, const float* scale,
+                        const float* bias, int64_t m, int64_t n, int64_t k, double* out, double* mag);
 void oracle_ternary_gemm_sampled(const uint16_t* x_bf16, const uint16_t* packed,
                                  const float* scale, int64_t m, int64_t n, int64_t k,
                                  const int64_t* rows, const int64_t* cols, int64_t count,

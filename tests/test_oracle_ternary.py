@@ -277,3 +277,50 @@ def test_ternary_linear_adds_the_bias():
     assert np.all(y[:, 1] == -3.0)          # all-zero trits: the bias alone
     yn, mn = oracle.ternary_linear(xb, packed, scale, None, 2, 3, k)
     assert np.array_equal(yn, y0) and np.array_equal(mn, m0)
+
+
+# ---------------------------------------------------------------------------
+# Index + sign sparse encoding ("Features": sparse encoding for high-sparsity
+# layers; Packer.pack_sparse)
+# ---------------------------------------------------------------------------
+def test_sparse_encoding_by_hand():
+    trits = np.zeros((3, 20), np.int8)
+    trits[0, [0, 5, 19]] = [1, -1, 1]
+    trits[2, 7] = -1               # row 1 empty
+    row_ptr, ent = oracle.sparse_encode(trits)
+    assert row_ptr.tolist() == [0, 3, 3, 4]
+    assert ent.tolist() == [0, 5 | 0x8000, 19, 7 | 0x8000]
+
+
+@pytest.mark.parametrize("n,k,density", [(5, 1, 0.5), (7, 33, 0.1), (4, 4096, 0.58), (3, 32768, 0.02),
+                                         (6, 100, 1.0), (2, 50, 0.0)])
+def test_sparse_round_trip_and_counts(n, k, density):
+    rng = np.random.default_rng(n * k)
+    trits = (rng.integers(0, 2, (n, k)) * 2 - 1).astype(np.int8) * (rng.random((n, k)) < density)
+    row_ptr, ent = oracle.sparse_encode(trits)
+    assert row_ptr[0] == 0 and np.all(np.diff(row_ptr) == (trits != 0).sum(axis=1))
+    back, bad = oracle.sparse_decode(row_ptr, ent, n, k)
+    assert bad == 0 and np.array_equal(back, trits)
+
+
+def test_sparse_decode_flags_malformed_entries():
+    row_ptr = np.array([0, 3], np.int64)
+    ent = np.array([4, 4, 9], np.uint16)        # repeated position, position >= k
+    _, bad = oracle.sparse_decode(row_ptr, ent, 1, 8)
+    assert bad == 2
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 9, 130), (3, 5, 4096), (2, 4, 1)])
+def test_sparse_gemm_equals_dense_ternary_layer(m, n, k):
+    """The sparse layer over the entries of a trit matrix is the dense ternary
+    layer over the same trits (the dense oracle is pinned above)."""
+    rng = np.random.default_rng(m + n + k)
+    trits = rng.integers(-1, 2, (n, k)).astype(np.int8) * (rng.random((n, k)) < 0.3)
+    scale = (rng.random(n) + 0.5).astype(np.float32)
+    bias = rng.standard_normal(n).astype(np.float32)
+    xb = _bf16(rng.standard_normal((m, k)))
+    row_ptr, ent = oracle.sparse_encode(trits)
+    y, mag = oracle.sparse_gemm(xb, row_ptr, ent, scale, bias, m, n, k)
+    yd, md = oracle.ternary_linear(xb, oracle.base3_pack(trits), scale, bias, m, n, k)
+    np.testing.assert_allclose(y, yd, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(mag, md, rtol=1e-12, atol=1e-12)
