@@ -290,6 +290,46 @@ bnn_status bnn_ternary_linear(const uint16_t* x_bf16, const uint16_t* packed, co
                               const float* bias, int64_t m, int64_t n, int64_t k, float* out,
                               cudaStream_t s);
 
+/*
+ * Index + sign sparse ternary layers.  [BTE] "Features" (sparse encoding:
+ * index + sign format for high-sparsity layers), "Module Overview"
+ * (Packer.pack_sparse).  Format: row j's non-zero trits are entries
+ * [row_ptr[j], row_ptr[j+1]) of a uint16 array, in increasing position order,
+ * each the position (bits 0..14) with bit 15 set for -1; row_ptr[0] = 0.
+ * Positions need 15 bits, so k <= BNN_MAX_K_SPARSE.
+ */
+#define BNN_MAX_K_SPARSE 32768
+
+/*
+ * bnn_ternary_sparse_count -- row_ptr of the sparse form of base-3 packed
+ * weights.
+ *   packed   uint16 [n, ceil(k/10)] base-3 words (see Layout), device.
+ *   row_ptr  int64 [n + 1], device, 8-byte aligned: row_ptr[j+1] - row_ptr[j]
+ *            = number of non-zero trits of row j; row_ptr[n] = total entries
+ *            (read it back to size `entries`).
+ */
+bnn_status bnn_ternary_sparse_count(const uint16_t* packed, int64_t n, int64_t k, int64_t* row_ptr,
+                                    cudaStream_t s);
+
+/*
+ * bnn_ternary_sparse_encode -- write the entries of the sparse form.
+ *   row_ptr  as produced by bnn_ternary_sparse_count for the same packed.
+ *   entries  uint16 [row_ptr[n]], device, 2-byte aligned (may be NULL only
+ *            when n or k is 0).
+ */
+bnn_status bnn_ternary_sparse_encode(const uint16_t* packed, int64_t n, int64_t k, const int64_t* row_ptr,
+                                     uint16_t* entries, cudaStream_t s);
+
+/*
+ * bnn_ternary_sparse_gemm -- the ternary layer over the sparse form:
+ *   out[i,j] = scale[j] * sum_{e in row j} (+-1) x[i, pos_e] (+ bias[j]),
+ *   x bf16 [m, k], float32 accumulation; scale float32 [n]; bias float32 [n]
+ *   or NULL; out float32 [m, n].  Same tolerance as bnn_ternary_gemm.
+ */
+bnn_status bnn_ternary_sparse_gemm(const uint16_t* x_bf16, const int64_t* row_ptr, const uint16_t* entries,
+                                   const float* scale, const float* bias, int64_t m, int64_t n, int64_t k,
+                                   float* out, cudaStream_t s);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* bnn_status_string(bnn_status st);
 

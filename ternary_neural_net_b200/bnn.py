@@ -41,6 +41,9 @@ _SIGS = {
     "bnn_ternary_gemm_algo": [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _int, _vp],
     "bnn_ternary_pack_noalloc": [_vp, _i64, _i64, _vp, _vp, _vp, _vp],
     "bnn_ternary_linear": [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
+    "bnn_ternary_sparse_count": [_vp, _i64, _i64, _vp, _vp],
+    "bnn_ternary_sparse_encode": [_vp, _i64, _i64, _vp, _vp, _vp],
+    "bnn_ternary_sparse_gemm": [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
 }
 for _name, _args in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -66,6 +69,7 @@ ALGO_AUTO, ALGO_POPC, ALGO_MMA_S8, ALGO_TC = 0, 1, 2, 3
 TERNARY_TWN, TERNARY_ABSMEAN, TERNARY_DELTA = 0, 1, 2
 TALGO_AUTO, TALGO_CUDA_CORES, TALGO_MMA, TALGO_TC = 0, 1, 2, 3
 MAX_K_BINARY = 1 << 24
+MAX_K_SPARSE = 1 << 15
 
 
 class BnnError(RuntimeError):
@@ -190,6 +194,42 @@ def bnn_binary_linear(xp: torch.Tensor, wp: torch.Tensor, alpha: torch.Tensor | 
     _check(_lib.bnn_binary_linear(_ptr(xp), _ptr(wp), _ptr(alpha), _ptr(bias), m, n, k, _ptr(dots), _ptr(out),
                                   _ptr(nxt), _stream(dev)), "bnn_binary_linear")
     return dots, out, nxt
+
+
+def bnn_ternary_sparse_encode(packed: torch.Tensor, k: int):
+    """Base-3 packed [n, ceil(k/10)] -> (row_ptr int64 [n+1], entries int16 [nnz]) of the index +
+    sign sparse form.  Reads the entry count back from the device (one synchronisation)."""
+    _dev(packed, "packed", torch.int16)
+    n = packed.shape[0]
+    if packed.shape[1] != trit_words_per_row(k):
+        raise ValueError("packed rows must hold ceil(k/10) words")
+    dev = packed.device
+    row_ptr = torch.empty((n + 1,), dtype=torch.int64, device=dev)
+    _check(_lib.bnn_ternary_sparse_count(_ptr(packed), n, k, _ptr(row_ptr), _stream(dev)), "bnn_ternary_sparse_count")
+    nnz = int(row_ptr[n].item())
+    entries = torch.empty((max(nnz, 1),), dtype=torch.int16, device=dev)
+    _check(_lib.bnn_ternary_sparse_encode(_ptr(packed), n, k, _ptr(row_ptr), _ptr(entries), _stream(dev)),
+           "bnn_ternary_sparse_encode")
+    return row_ptr, entries[:nnz]
+
+
+def bnn_ternary_sparse_gemm(x: torch.Tensor, row_ptr: torch.Tensor, entries: torch.Tensor, scale: torch.Tensor,
+                            bias: torch.Tensor | None = None, out: torch.Tensor | None = None) -> torch.Tensor:
+    """bf16 [m, k] x sparse ternary [n, k] -> float32 [m, n] (scale and bias applied)."""
+    _dev(x, "x", torch.bfloat16)
+    _dev(row_ptr, "row_ptr", torch.int64, ndim=1)
+    _dev(scale, "scale", torch.float32, ndim=1)
+    m, k = x.shape
+    n = row_ptr.shape[0] - 1
+    if bias is not None:
+        _dev(bias, "bias", torch.float32, ndim=1)
+    if out is None:
+        out = torch.empty((m, n), dtype=torch.float32, device=x.device)
+    _dev(out, "out", torch.float32)
+    ent = _ptr(entries) if entries.numel() else None
+    _check(_lib.bnn_ternary_sparse_gemm(_ptr(x), _ptr(row_ptr), ent, _ptr(scale), _ptr(bias), m, n, k, _ptr(out),
+                                        _stream(x.device)), "bnn_ternary_sparse_gemm")
+    return out
 
 
 def bnn_ternary_pack(w: torch.Tensor, packed: torch.Tensor | None = None,

@@ -111,3 +111,19 @@ def test_ternary_linear_host_checks(bnn):
     assert lib.bnn_ternary_linear(g, g, None, g, 1, 1, 3, g, None) == bnn.BNN_ERR_INVALID_ARG
     assert lib.bnn_ternary_linear(g, g, g, P(0x1002), 1, 1, 3, g, None) == bnn.BNN_ERR_MISALIGNED
     assert lib.bnn_ternary_linear(None, None, None, None, 0, 3, 3, g, None) == bnn.BNN_OK
+
+
+def test_sparse_host_checks(bnn):
+    lib = bnn.lib()
+    P = C.c_void_p
+    g = P(0x1000)
+    assert lib.bnn_ternary_sparse_count(g, 2, (1 << 15) + 1, g, None) == bnn.BNN_ERR_INVALID_ARG
+    assert lib.bnn_ternary_sparse_count(g, 2, 10, None, None) == bnn.BNN_ERR_INVALID_ARG
+    assert lib.bnn_ternary_sparse_count(g, 2, 10, P(0x1004), None) == bnn.BNN_ERR_MISALIGNED
+    assert lib.bnn_ternary_sparse_encode(g, 2, 10, g, None, None) == bnn.BNN_ERR_INVALID_ARG
+    assert lib.bnn_ternary_sparse_encode(g, 2, 10, g, P(0x1001), None) == bnn.BNN_ERR_MISALIGNED
+    assert lib.bnn_ternary_sparse_encode(None, 0, 10, g, None, None) == bnn.BNN_OK
+    assert lib.bnn_ternary_sparse_gemm(g, g, g, g, None, 1, 1, -1, g, None) == bnn.BNN_ERR_INVALID_ARG
+    assert lib.bnn_ternary_sparse_gemm(g, g, g, None, None, 1, 1, 10, g, None) == bnn.BNN_ERR_INVALID_ARG
+    assert lib.bnn_ternary_sparse_gemm(g, g, g, g, P(0x1002), 1, 1, 10, g, None) == bnn.BNN_ERR_MISALIGNED
+    assert lib.bnn_ternary_sparse_gemm(None, None, None, None, None, 0, 4, 10, None, None) == bnn.BNN_OK
