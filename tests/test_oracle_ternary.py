@@ -324,3 +324,54 @@ def test_sparse_gemm_equals_dense_ternary_layer(m, n, k):
     yd, md = oracle.ternary_linear(xb, oracle.base3_pack(trits), scale, bias, m, n, k)
     np.testing.assert_allclose(y, yd, rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(mag, md, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# .tbin files ("BalancedTernaryEngine" README, ".tbin Format")
+# ---------------------------------------------------------------------------
+def golden_tbin_files():
+    files, cur = {}, None
+    for line in golden_lines("tbin_small.txt"):
+        if line.startswith("file "):
+            cur = line.split()[1]
+            files[cur] = bytearray()
+        else:
+            files[cur] += bytes.fromhex(line.split("#")[0])
+    return {k: bytes(v) for k, v in files.items()}
+
+
+def test_tbin_golden_files():
+    from oracle import tbin
+    f = golden_tbin_files()
+    ver, meta, recs = tbin.read(f["v2"])
+    assert ver == 2 and meta == b"{}" and len(recs) == 2
+    t, r = recs
+    assert (t["kind"], t["name"], t["out_feat"], t["in_feat"]) == ("ternary", "ab", 1, 3)
+    assert t["delta"] == 0.5 and t["sparsity"] == 0.0 and t["biases"] is None
+    assert t["scales"].tolist() == [1.0] and t["words"].tolist() == [5]
+    assert oracle.base3_unpack(t["words"].reshape(1, 1), 3)[0].tolist() == [[1, 0, -1]]
+    assert (r["kind"], r["name"], r["dims"], r["data"].tolist()) == ("raw", "n", [2], [1.0, -2.0])
+    ver, meta, recs = tbin.read(f["v1"])
+    (t,) = recs
+    assert ver == 1 and meta == b"" and (t["name"], t["out_feat"], t["in_feat"]) == ("w", 2, 11)
+    assert t["delta"] == np.float32(0.1) and t["sparsity"] == 0.25
+    assert t["scales"].tolist() == [2.0, 0.5] and t["biases"].tolist() == [1.0, -1.0]
+    trits, bad = oracle.base3_unpack(t["words"].reshape(2, 2), 11)
+    assert bad == 0
+    assert trits[0].tolist() == [1, 1, -1, -1, 0, 0, 0, 0, 0, 0, 1]
+    assert trits[1].tolist() == [-1, -1, 1, 0, 1, -1, -1, -1, -1, -1, -1]
+    # the writer reproduces both files byte for byte
+    assert tbin.write([dict(kind="ternary", name="ab", out_feat=1, in_feat=3, delta=0.5, sparsity=0.0,
+                            scales=[1.0], biases=None, words=[5]),
+                       dict(kind="raw", name="n", dims=[2], data=[1.0, -2.0])]) == f["v2"]
+    assert tbin.write([dict(kind="ternary", name="w", out_feat=2, in_feat=11, delta=np.float32(0.1), sparsity=0.25,
+                            scales=[2.0, 0.5], biases=[1.0, -1.0], words=[29492, 29525, 207, 29523])],
+                      metadata=b"", version=1) == f["v1"]
+
+
+def test_tbin_rejects_malformed_files():
+    from oracle import tbin
+    f = golden_tbin_files()["v2"]
+    for bad in (b"XBN\0" + f[4:], f[:-1], f[:20]):
+        with pytest.raises((ValueError, IndexError, Exception)):
+            tbin.read(bad)
