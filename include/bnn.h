@@ -330,6 +330,61 @@ bnn_status bnn_ternary_sparse_gemm(const uint16_t* x_bf16, const int64_t* row_pt
                                    const float* scale, const float* bias, int64_t m, int64_t n, int64_t k,
                                    float* out, cudaStream_t s);
 
+/*
+ * .tbin ternary model files.  [BTE] ".tbin Format": header (magic "TBN\0",
+ * version 1 or 2, num_layers, meta_len, JSON metadata), then records (kind
+ * byte in version 2: 0 ternary, 1 raw float16; size; payload).  All fields
+ * little-endian.  A ternary record holds out_features float16 scales, then 0
+ * or out_features float16 biases (the record size decides), then
+ * out_features x ceil(in_features/10) base-3 words.
+ */
+#define BNN_TBIN_MAX_DIMS 8
+
+typedef struct bnn_tbin_record {
+  uint32_t kind;            /* 0 ternary, 1 raw float16 */
+  uint32_t name_len;        /* UTF-8 name: name_len bytes at name_offset */
+  uint64_t name_offset;
+  /* kind 0 */
+  uint32_t out_features, in_features;
+  float delta, sparsity;
+  uint32_t num_biases;      /* 0 or out_features */
+  uint32_t reserved;
+  uint64_t scales_offset;   /* out_features float16 */
+  uint64_t biases_offset;   /* num_biases float16 (0 when there are none) */
+  uint64_t weights_offset;  /* weights_words uint16 base-3 words */
+  uint64_t weights_words;
+  /* kind 1 */
+  uint32_t ndims;
+  uint32_t dims[BNN_TBIN_MAX_DIMS];
+  uint64_t data_offset;     /* data_elems float16 */
+  uint64_t data_elems;
+} bnn_tbin_record;
+
+/*
+ * bnn_tbin_parse -- read the record table of a .tbin file held in HOST memory
+ * (file, len bytes); nothing is copied and no CUDA call is made.  *count =
+ * num_layers; the first min(capacity, num_layers) records are written to
+ * records (all byte offsets are from the start of the file).  version,
+ * meta_offset and meta_len may be NULL.  BNN_ERR_INVALID_ARG for a bad magic
+ * or version, a truncated file or a record whose size does not fit its fields.
+ */
+bnn_status bnn_tbin_parse(const uint8_t* file, uint64_t len, uint32_t* version, uint64_t* meta_offset,
+                          uint64_t* meta_len, bnn_tbin_record* records, int64_t capacity, int64_t* count);
+
+/*
+ * bnn_tbin_load_ternary -- copy one ternary record out of the file's bytes in
+ * DEVICE memory (file_dev, len bytes, any alignment) into the buffers the
+ * ternary calls take: packed uint16 [out_features, ceil(in_features/10)],
+ * scale float32 [out_features] (may be NULL), bias float32 [out_features] (may
+ * be NULL; zeros when the record has no biases).  float16 -> float32 is exact.
+ */
+bnn_status bnn_tbin_load_ternary(const uint8_t* file_dev, uint64_t len, const bnn_tbin_record* rec,
+                                 uint16_t* packed, float* scale, float* bias, cudaStream_t s);
+
+/* bnn_tbin_load_raw -- a raw float16 record's data as float32 [data_elems]. */
+bnn_status bnn_tbin_load_raw(const uint8_t* file_dev, uint64_t len, const bnn_tbin_record* rec, float* out,
+                             cudaStream_t s);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* bnn_status_string(bnn_status st);
 

@@ -45,6 +45,22 @@ _SIGS = {
     "bnn_ternary_sparse_encode": [_vp, _i64, _i64, _vp, _vp, _vp],
     "bnn_ternary_sparse_gemm": [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp],
 }
+class TbinRecord(C.Structure):
+    """bnn_tbin_record (include/bnn.h)."""
+    _fields_ = [("kind", C.c_uint32), ("name_len", C.c_uint32), ("name_offset", C.c_uint64),
+                ("out_features", C.c_uint32), ("in_features", C.c_uint32), ("delta", C.c_float),
+                ("sparsity", C.c_float), ("num_biases", C.c_uint32), ("reserved", C.c_uint32),
+                ("scales_offset", C.c_uint64), ("biases_offset", C.c_uint64), ("weights_offset", C.c_uint64),
+                ("weights_words", C.c_uint64), ("ndims", C.c_uint32), ("dims", C.c_uint32 * 8),
+                ("data_offset", C.c_uint64), ("data_elems", C.c_uint64)]
+
+
+_SIGS.update({
+    "bnn_tbin_parse": [_vp, C.c_uint64, _vp, _vp, _vp, _vp, _i64, _vp],
+    "bnn_tbin_load_ternary": [_vp, C.c_uint64, _vp, _vp, _vp, _vp, _vp],
+    "bnn_tbin_load_raw": [_vp, C.c_uint64, _vp, _vp, _vp],
+})
+
 for _name, _args in _SIGS.items():
     _f = getattr(_lib, _name)
     _f.argtypes = _args
@@ -230,6 +246,46 @@ def bnn_ternary_sparse_gemm(x: torch.Tensor, row_ptr: torch.Tensor, entries: tor
     _check(_lib.bnn_ternary_sparse_gemm(_ptr(x), _ptr(row_ptr), ent, _ptr(scale), _ptr(bias), m, n, k, _ptr(out),
                                         _stream(x.device)), "bnn_ternary_sparse_gemm")
     return out
+
+
+def bnn_tbin_parse(data: bytes):
+    """Parse a .tbin file held in host memory: (version, metadata bytes, [TbinRecord, ...])."""
+    buf = C.create_string_buffer(bytes(data), len(data))
+    ver, moff, mlen, count = C.c_uint32(), C.c_uint64(), C.c_uint64(), C.c_int64()
+    _check(_lib.bnn_tbin_parse(buf, len(data), C.byref(ver), C.byref(moff), C.byref(mlen), None, 0,
+                               C.byref(count)), "bnn_tbin_parse")
+    recs = (TbinRecord * max(count.value, 1))()
+    _check(_lib.bnn_tbin_parse(buf, len(data), None, None, None, recs, count.value, C.byref(count)),
+           "bnn_tbin_parse")
+    meta = bytes(data[moff.value:moff.value + mlen.value])
+    return ver.value, meta, [recs[i] for i in range(count.value)]
+
+
+def tbin_record_name(data: bytes, rec: TbinRecord) -> str:
+    return bytes(data[rec.name_offset:rec.name_offset + rec.name_len]).decode()
+
+
+def bnn_tbin_load_ternary(file_dev: torch.Tensor, rec: TbinRecord):
+    """A ternary record from the file's bytes on the device (uint8 tensor) ->
+    (packed int16 [out, ceil(in/10)], scale float32 [out], bias float32 [out] or None)."""
+    _dev(file_dev, "file", torch.uint8, ndim=1)
+    dev = file_dev.device
+    out_f, kt = rec.out_features, trit_words_per_row(rec.in_features)
+    packed = torch.empty((out_f, kt), dtype=torch.int16, device=dev)
+    scale = torch.empty((out_f,), dtype=torch.float32, device=dev)
+    bias = torch.empty((out_f,), dtype=torch.float32, device=dev) if rec.num_biases else None
+    _check(_lib.bnn_tbin_load_ternary(_ptr(file_dev), file_dev.numel(), C.byref(rec), _ptr(packed), _ptr(scale),
+                                      _ptr(bias), _stream(dev)), "bnn_tbin_load_ternary")
+    return packed, scale, bias
+
+
+def bnn_tbin_load_raw(file_dev: torch.Tensor, rec: TbinRecord) -> torch.Tensor:
+    """A raw float16 record from the file's bytes on the device -> float32 tensor of its dims."""
+    _dev(file_dev, "file", torch.uint8, ndim=1)
+    out = torch.empty((int(rec.data_elems),), dtype=torch.float32, device=file_dev.device)
+    _check(_lib.bnn_tbin_load_raw(_ptr(file_dev), file_dev.numel(), C.byref(rec), _ptr(out),
+                                  _stream(file_dev.device)), "bnn_tbin_load_raw")
+    return out.view(*[int(rec.dims[d]) for d in range(rec.ndims)]) if rec.ndims else out
 
 
 def bnn_ternary_pack(w: torch.Tensor, packed: torch.Tensor | None = None,
