@@ -263,7 +263,8 @@ typedef enum {
   BNN_TALGO_AUTO = 0,        /* what bnn_ternary_gemm uses: CUDA-core GEMV for m <= 8, MMA otherwise */
   BNN_TALGO_CUDA_CORES = 1,  /* CUDA-core GEMV kernels (m <= 8 only; BNN_ERR_UNSUPPORTED beyond) */
   BNN_TALGO_MMA = 2,         /* trits decoded to bf16 tiles, bf16 mma.sync m16n8k16 */
-  BNN_TALGO_TC = 3           /* trits decoded to bf16 tiles, tcgen05.mma kind::f16 into tensor memory */
+  BNN_TALGO_TC = 3           /* trits decoded to bf16 tiles, tcgen05.mma kind::f16 into tensor memory
+                                (activations by TMA when k % 8 == 0 and x is 16-byte aligned) */
 } bnn_ternary_algo;
 
 /*

@@ -50,16 +50,25 @@
 #include <cooperative_groups.h>
 
 #include "bnn_internal.cuh"
+#include "tc_common.cuh"
 
 // Bounded waits that ran out in this file's kernels (read by bnn_device_error_count).
 __device__ unsigned int g_bnn_device_errors = 0;
 
 namespace {
 
+using bnn::tc::mbar_arrive;
+using bnn::tc::mbar_expect_tx;
+using bnn::tc::mbar_try;
+using bnn::tc::smem_u32;
+using bnn::tc::sw128_desc;
+using bnn::tc::tma_load_2d;
+using bnn::tc::tmem_ld16;
+using bnn::tc::tmem_wait_ld;
+
 constexpr int kTm = 128;                   // weight rows per tile (UMMA M)
 constexpr int kPre = 8;                    // without TMA: stages of words prefetched in registers
 constexpr int kChunkStages = 4;            // with TMA: stages per packed chunk (64 bytes of every row)
-constexpr uint32_t kSpinLimit = 1u << 24;  // bounded mbarrier waits
 
 template <int BN, bool TMA>
 struct TcCfg {
@@ -73,81 +82,6 @@ struct TcCfg {
   static constexpr int kThreads = kProducers + 64;                   // + MMA warp + TMA warp
   static constexpr int kMinBlocks = BN <= 64 ? 2 : 1;
 };
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, 8-row
-// groups 1024 bytes apart.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);  // start address (16-byte units)
-  d |= static_cast<uint64_t>(1) << 16;                 // leading-dimension offset (unused for this layout)
-  d |= static_cast<uint64_t>(1024 >> 4) << 32;         // stride between 8-row groups
-  d |= static_cast<uint64_t>(1) << 46;                 // descriptor version
-  d |= static_cast<uint64_t>(2) << 61;                 // 128-byte swizzle
-  return d;
-}
-
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait; false when it ran out (counted, abort raised) or when another
-// thread of the CTA raised the abort flag.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-  for (uint32_t it = 0; it < kSpinLimit; ++it) {
-    if (mbar_try(bar, parity)) return true;
-    if ((it & 255u) == 255u && *abort_flag) return false;
-  }
-  *abort_flag = 1;
-  atomicAdd(&g_bnn_device_errors, 1u);
-  return false;
-}
-
-// Bounded wait that ignores the abort flag (used for the final drains).
-__device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity) {
-  for (uint32_t it = 0; it < kSpinLimit; ++it)
-    if (mbar_try(bar, parity)) return true;
-  atomicAdd(&g_bnn_device_errors, 1u);
-  return false;
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
-}
-
-// 2-D tiled TMA load of one box into this CTA's shared memory (x = packed word,
-// y = row), completing `bytes` on the mbarrier.
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(
-          dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
-
-// 16 columns of this warp's 32 tensor-memory lanes
-__device__ __forceinline__ void tmem_ld16(uint32_t addr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(addr));
-}
-
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
 
 // 4 bytes per 16-byte chunk word: byte j of word s holds bit 8j + s of hw
 __device__ __forceinline__ void expand_word(uint8_t* dst_row, uint32_t swz, int part, uint64_t cw) {
@@ -260,7 +194,8 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
       const uint32_t rd_swz = static_cast<uint32_t>((r2 >> 1) & 3);
       for (int j = 0; j < nst; ++j) {
         const int c = j / kChunkStages, s = j % kChunkStages, pb = c % P;
-        if (s == 0 && !mbar_wait(smem_u32(&chunk_full[pb]), static_cast<uint32_t>((c / P) & 1), &abort_flag)) {
+        if (s == 0 && !bnn::tc::mbar_wait(smem_u32(&chunk_full[pb]), static_cast<uint32_t>((c / P) & 1), &abort_flag,
+                                          &g_bnn_device_errors)) {
           ok = false;
           break;
         }
@@ -269,7 +204,8 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
         if (s == kChunkStages - 1 || j == nst - 1) mbar_arrive(smem_u32(&chunk_empty[pb]));
         const int b = j % S;
         // refill only after the tensor core has read the previous fill of this buffer
-        if (j >= S && !mbar_wait(smem_u32(&empty_bar[b]), static_cast<uint32_t>((j / S + 1) & 1), &abort_flag)) {
+        if (j >= S && !bnn::tc::mbar_wait(smem_u32(&empty_bar[b]), static_cast<uint32_t>((j / S + 1) & 1), &abort_flag,
+                                          &g_bnn_device_errors)) {
           ok = false;
           break;
         }
@@ -296,7 +232,8 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
           const int j = js + u;
           if (j >= nst) break;
           const int b = j % S;
-          if (j >= S && !mbar_wait(smem_u32(&empty_bar[b]), static_cast<uint32_t>((j / S + 1) & 1), &abort_flag)) {
+          if (j >= S && !bnn::tc::mbar_wait(smem_u32(&empty_bar[b]), static_cast<uint32_t>((j / S + 1) & 1), &abort_flag,
+                                          &g_bnn_device_errors)) {
             ok = false;
             break;
           }
@@ -318,7 +255,9 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
                            ((static_cast<uint32_t>(kTm) >> 4) << 24);
     for (int j = 0; j < nst; ++j) {
       const int b = j % S;
-      if (!mbar_wait(smem_u32(&full_bar[b]), static_cast<uint32_t>((j / S) & 1), &abort_flag)) break;
+      if (!bnn::tc::mbar_wait(smem_u32(&full_bar[b]), static_cast<uint32_t>((j / S) & 1), &abort_flag,
+                              &g_bnn_device_errors))
+        break;
       asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
       const uint64_t ad = sw128_desc(smem_base + b * kStageBytes);
       const uint64_t bd = sw128_desc(smem_base + b * kStageBytes + kTm * 128u);  // activation rows
@@ -358,7 +297,9 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
     int issued = pre;
     for (int c = pre; c < nch; ++c) {
       const int pb = c % P;
-      if (!mbar_wait(smem_u32(&chunk_empty[pb]), static_cast<uint32_t>((c / P + 1) & 1), &abort_flag)) break;
+      if (!bnn::tc::mbar_wait(smem_u32(&chunk_empty[pb]), static_cast<uint32_t>((c / P + 1) & 1), &abort_flag,
+                              &g_bnn_device_errors))
+        break;
       const uint32_t dst = smem_u32(chunks + pb * Cfg::kChunkBytes);
       const uint32_t bar = smem_u32(&chunk_full[pb]);
       mbar_expect_tx(bar, Cfg::kChunkBytes);
@@ -369,7 +310,7 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
     // the CTA must not retire with copies in flight (producers that aborted no
     // longer wait for them): wait for the last chunk issued into each buffer
     for (int c = issued - P; c < issued; ++c)
-      if (c >= 0) mbar_drain(smem_u32(&chunk_full[c % P]), static_cast<uint32_t>((c / P) & 1));
+      if (c >= 0) bnn::tc::mbar_drain(smem_u32(&chunk_full[c % P]), static_cast<uint32_t>((c / P) & 1), &g_bnn_device_errors);
   }
   __syncwarp();
 
@@ -379,7 +320,7 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
   if (tid < kProducers) asm volatile("bar.sync 1, %0;\n" ::"r"(kProducers) : "memory");
   bool drained = true;
   if (warp < 8) {
-    drained = mbar_drain(smem_u32(&done_bar), 0u);
+    drained = bnn::tc::mbar_drain(smem_u32(&done_bar), 0u, &g_bnn_device_errors);
     asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
   }
   const bool good = __syncthreads_and(drained && abort_flag == 0) != 0;

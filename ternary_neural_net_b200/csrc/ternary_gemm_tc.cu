@@ -24,6 +24,7 @@
 #include <cooperative_groups.h>
 
 #include "bnn_internal.cuh"
+#include "tc_common.cuh"
 
 // Bounded waits that ran out in this file's kernels (read by bnn_device_error_count).
 __device__ unsigned int g_bnn_tc_ternary_errors = 0;
@@ -293,6 +294,335 @@ ternary_gemm_tc_kernel(const uint16_t* __restrict__ x, const uint16_t* __restric
   if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kTcNX));
 }
 
+
+// ---------------------------------------------------------------------------
+// Warp-specialised version (activation rows 16-byte aligned: TMA).
+//
+// Roles: one thread copies the stage's 64 x 64 bf16 activation box by TMA
+// straight into the 128-byte-swizzled tile; 512 producer threads copy the
+// stage's 8-word window of each weight row into shared memory (coalesced along
+// the rows, one stage ahead) and then decode: warp w takes quarter w % 4 (16
+// trits, 8 pairs) of 32 weight rows, reads the (up to) three words covering
+// them and writes two 16-byte chunks; one thread issues 4
+// tcgen05.mma.kind::f16 (K = 16) per stage; warps 0-7 read the float32
+// accumulator.  A pair's word and base-9 digit depend only on the phase (first
+// trit mod 10, one of 0, 2, 4, 6, 8), which is the same for every lane of a
+// warp, so the decode is specialised per phase without divergence: per pair one
+// multiply by a constant power of 9, one __umulhi and one 9-entry table load.
+// The producers meet at one named barrier per stage (with an AND of their
+// wait results, so that a wait that ran out stops all of them together); the
+// rest is synchronised by mbarriers.  A cluster of KS CTAs
+// splits the stages; each CTA pushes its partial sums (float4 stores into
+// distributed shared memory) to the CTA owning those activation rows, which
+// adds them in rank order (deterministic), scales and adds the bias.
+// ---------------------------------------------------------------------------
+constexpr int kT2M = 128;                            // weight rows (UMMA M)
+constexpr int kT2N = 64;                             // activation rows (UMMA N)
+constexpr int kT2S = 4;                              // stages of 64 trits
+constexpr int kT2Prod = 4 * kT2M;                    // producer threads
+constexpr int kT2Threads = kT2Prod + 64;             // + MMA warp + TMA warp
+constexpr uint32_t kT2AStage = kT2M * 128u, kT2Stage = kT2AStage + kT2N * 128u;
+constexpr int kT2Pre = 4;                            // stages of words prefetched in registers
+constexpr uint32_t kZeroWord = 29524u;               // all ten trits 0 (every digit 1)
+
+// floor(v / 10) for any 32-bit v (multiply-high by ceil(2^35 / 10))
+__device__ __forceinline__ uint32_t div10(uint32_t v) { return __umulhi(v, 0xCCCCCCCDu) >> 3; }
+
+// 9^p (p <= 4)
+__host__ __device__ constexpr uint32_t pow9(int p) { return p <= 0 ? 1u : 9u * pow9(p - 1); }
+
+// the 8 bf16 pairs of 16 trits starting at phase R10 of word 0 (F[i] = word_i * kFix)
+template <int R10>
+__device__ __forceinline__ void decode16(const uint32_t (&F)[3], const uint32_t* lut, uint4& lo, uint4& hi) {
+  uint32_t v[8];
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    const int kp = R10 / 2 + p;       // pair index counted from word 0
+    const int j = kp / 5, q = kp % 5;  // word, base-9 digit (q = 4: trits 8, 9)
+    // the digit is the integer part of 9 x (fraction of word / 9^5 scaled by 9^(4-q))
+    v[p] = lut[__umulhi(F[j] * pow9(4 - q), 9u)];
+  }
+  lo = make_uint4(v[0], v[1], v[2], v[3]);
+  hi = make_uint4(v[4], v[5], v[6], v[7]);
+}
+
+template <int KS>
+__global__ void __launch_bounds__(kT2Threads, 2)
+ternary_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t* __restrict__ packed,
+                        const float* __restrict__ scale, const float* __restrict__ bias, int64_t m, int64_t n,
+                        int64_t k, int64_t kt, float* __restrict__ out) {
+  using namespace bnn::tc;
+  constexpr int kCols = kT2N / KS;
+  constexpr int kPitch = kCols + 4;  // padded receive row (floats)
+  static_assert(KS * kT2M * kPitch * 4 <= kT2S * kT2Stage, "split-K shares must fit the stage memory");
+
+  extern __shared__ __align__(16) uint8_t t2_raw[];
+  __shared__ __align__(8) uint64_t full_bar[kT2S];
+  __shared__ __align__(8) uint64_t empty_bar[kT2S];
+  __shared__ __align__(8) uint64_t done_bar;
+  __shared__ uint32_t tmem_holder;
+  __shared__ volatile int abort_flag;
+  __shared__ int any_bad;
+  __shared__ uint32_t lut[9];
+  __shared__ uint32_t wtile[2][kT2M][9];  // packed words of a stage's window, 9-word pitch (odd: no bank conflicts)
+  uint8_t* const smem = t2_raw + ((1024u - (smem_u32(t2_raw) & 1023u)) & 1023u);
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int rank = KS > 1 ? static_cast<int>(blockIdx.x % KS) : 0;
+  const int64_t j0 = static_cast<int64_t>(blockIdx.x / KS) * kT2M;  // first weight row
+  const int64_t i0 = static_cast<int64_t>(blockIdx.y) * kT2N;        // first activation row
+  const int64_t total = (10 * kt + 63) / 64;                         // 64-trit stages covering every word
+  const int64_t share = (total + KS - 1) / KS;
+  const int64_t sb = rank * share < total ? rank * share : total;
+  const int64_t se = sb + share < total ? sb + share : total;
+  const int nst = static_cast<int>(se - sb);
+  constexpr int kMmaWarp = kT2Prod / 32, kTmaWarp = kMmaWarp + 1;
+
+  if (tid < 9) {
+    const int lo = tid % 3, hi = tid / 3;  // digit = trit + 1
+    const uint32_t blo = lo == 0 ? 0xBF80u : (lo == 2 ? 0x3F80u : 0u);
+    const uint32_t bhi = hi == 0 ? 0xBF80u : (hi == 2 ? 0x3F80u : 0u);
+    lut[tid] = blo | (bhi << 16);
+  }
+  if (tid == 0) {
+    for (int i = 0; i < kT2S; ++i) {
+      mbar_init(smem_u32(&full_bar[i]), kT2Prod + 1);  // producers + the TMA thread's expect_tx
+      mbar_init(smem_u32(&empty_bar[i]), 1);
+    }
+    mbar_init(smem_u32(&done_bar), 1);
+    abort_flag = 0;
+    any_bad = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(&tmem_holder)),
+                 "r"(kT2N));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::);
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+  const uint32_t tmem = tmem_holder;
+  bnn::pdl_trigger();
+
+  if (tid < kT2Prod) {
+    // ------------------------------------------------------------ producers
+    // Copy: producer p stages words 2(p%4), 2(p%4)+1 of the stage's 8-word
+    // window of weight row p/4 (coalesced along the row) into wtile, one stage
+    // ahead, from registers loaded kT2Pre stages ahead.
+    const int crow = tid >> 2, cw = 2 * (tid & 3);
+    const int64_t cgn = j0 + crow;
+    const bool clive = cgn < n;
+    const uint16_t* csrc = packed + (clive ? cgn : 0) * kt;
+    const uint32_t kt32 = static_cast<uint32_t>(kt), se32 = static_cast<uint32_t>(se);
+    auto fetch = [&](uint32_t s, uint32_t& w0, uint32_t& w1) {
+      const uint32_t j = div10(64u * s) + static_cast<uint32_t>(cw);
+      w0 = (clive && s < se32 && j < kt32) ? static_cast<uint32_t>(__ldg(csrc + j)) : kZeroWord;
+      w1 = (clive && s < se32 && j + 1 < kt32) ? static_cast<uint32_t>(__ldg(csrc + j + 1)) : kZeroWord;
+    };
+    auto stage_words = [&](int buf, uint32_t w0, uint32_t w1) {
+      wtile[buf][crow][cw] = w0;
+      wtile[buf][crow][cw + 1] = w1;
+    };
+    // Decode: warp w takes quarter w % 4 (trits 16q..16q+15 of the stage) of
+    // 32 weight rows, so the word phase of a stage is the same for the whole warp.
+    const int quarter = warp & 3, row = 32 * (warp >> 2) + (tid & 31);
+    const uint32_t row_off = static_cast<uint32_t>(row) * 128u, swz = static_cast<uint32_t>(row & 7);
+
+    const uint32_t sb32 = static_cast<uint32_t>(sb);
+    uint32_t ring[kT2Pre][2];
+#pragma unroll
+    for (int u = 0; u < kT2Pre; ++u) fetch(sb32 + 1 + u, ring[u][0], ring[u][1]);
+    {
+      uint32_t w0, w1;
+      fetch(sb32, w0, w1);
+      stage_words(0, w0, w1);
+    }
+    bool ok = bnn::tc::producer_barrier_and(true, kT2Prod);
+    for (int js = 0; js < nst && ok; js += kT2Pre) {
+#pragma unroll
+      for (int u = 0; u < kT2Pre; ++u) {
+        const int jj = js + u;
+        if (jj >= nst) break;
+        // the next stage's window (ring[u] holds stage sb + jj + 1)
+        stage_words((jj + 1) & 1, ring[u][0], ring[u][1]);
+        fetch(sb32 + jj + 1 + kT2Pre, ring[u][0], ring[u][1]);
+        const int b = jj % kT2S;
+        const bool fine = jj < kT2S || mbar_wait(smem_u32(&empty_bar[b]),
+                                                 static_cast<uint32_t>((jj / kT2S + 1) & 1), &abort_flag,
+                                                 &g_bnn_tc_ternary_errors);
+        if (fine) {
+          const uint32_t s64 = 64u * (sb32 + jj), t0 = s64 + 16u * quarter;  // trit positions (< 2^31)
+          const uint32_t jt = div10(t0);
+          const uint32_t jrel = jt - div10(s64);
+          const uint32_t* wr = wtile[jj & 1][row];
+          const uint32_t F[3] = {wr[jrel] * kFix, wr[jrel + 1] * kFix, wr[jrel + 2] * kFix};
+          uint4 lo, hi;
+          switch (t0 - 10u * jt) {  // the phase, warp-uniform
+            case 0: decode16<0>(F, lut, lo, hi); break;
+            case 2: decode16<2>(F, lut, lo, hi); break;
+            case 4: decode16<4>(F, lut, lo, hi); break;
+            case 6: decode16<6>(F, lut, lo, hi); break;
+            default: decode16<8>(F, lut, lo, hi); break;
+          }
+          uint8_t* dst = smem + b * kT2Stage + row_off;
+          *reinterpret_cast<uint4*>(dst + (((2u * quarter) ^ swz) << 4)) = lo;
+          *reinterpret_cast<uint4*>(dst + (((2u * quarter + 1u) ^ swz) << 4)) = hi;
+          asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+          mbar_arrive(smem_u32(&full_bar[b]));
+        }
+        // one decision for all producers: the staged window is complete and the
+        // decoded one may be overwritten; a wait that ran out stops them all
+        ok = bnn::tc::producer_barrier_and(fine, kT2Prod);
+        if (!ok) break;
+      }
+    }
+  } else if (tid == kMmaWarp * 32) {
+    // ------------------------------------------------------------ MMA issue
+    // D f32, A and B bf16, both K-major, N = 64, M = 128
+    const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((static_cast<uint32_t>(kT2N) >> 3) << 17) |
+                           ((static_cast<uint32_t>(kT2M) >> 4) << 24);
+    const uint32_t base = smem_u32(smem);
+    for (int jj = 0; jj < nst; ++jj) {
+      const int b = jj % kT2S;
+      if (!mbar_wait(smem_u32(&full_bar[b]), static_cast<uint32_t>((jj / kT2S) & 1), &abort_flag,
+                     &g_bnn_tc_ternary_errors))
+        break;
+      asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+      const uint64_t ad = sw128_desc(base + b * kT2Stage), bd = sw128_desc(base + b * kT2Stage + kT2AStage);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint32_t acc = (jj > 0 || kk > 0) ? 1u : 0u;
+        asm volatile(
+            "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem),
+            "l"(ad + static_cast<uint64_t>(2 * kk)), "l"(bd + static_cast<uint64_t>(2 * kk)), "r"(idesc), "r"(acc));
+      }
+      mma_commit(smem_u32(&empty_bar[b]));
+    }
+    mma_commit(smem_u32(&done_bar));
+  } else if (tid == kTmaWarp * 32) {
+    // ------------------------------------------------------------ TMA copies of the activations
+    bnn::pdl_wait();  // x may come from the preceding kernel
+    for (int jj = 0; jj < nst; ++jj) {
+      const int b = jj % kT2S;
+      if (jj >= kT2S && !mbar_wait(smem_u32(&empty_bar[b]), static_cast<uint32_t>((jj / kT2S + 1) & 1),
+                                   &abort_flag, &g_bnn_tc_ternary_errors))
+        break;
+      const uint32_t bar = smem_u32(&full_bar[b]);
+      mbar_expect_tx(bar, kT2N * 128u);
+      tma_load_2d(smem_u32(smem + b * kT2Stage + kT2AStage), &tmap_x, static_cast<int>(64 * (sb + jj)),
+                  static_cast<int>(i0), bar);
+    }
+  }
+  __syncwarp();
+
+  // -------------------------------------------------------------- epilogue
+  bool drained = true;
+  if (warp < 8) {
+    drained = mbar_drain(smem_u32(&done_bar), 0u, &g_bnn_tc_ternary_errors);
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+  }
+  const bool good = __syncthreads_and(drained && abort_flag == 0) != 0;
+  const int erow = 32 * (warp & 3) + (tid & 31);       // weight row (tensor-memory lane)
+  const int ecol0 = (warp >> 2) * (kT2N / 2);          // half of the activation columns
+  const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+  const int64_t jrow = j0 + erow;
+  if constexpr (KS == 1) {
+    if (warp < 8 && good) {
+      const bool jlive = jrow < n;
+      const float sc = jlive ? __ldg(scale + jrow) : 0.0f, bv = (bias && jlive) ? __ldg(bias + jrow) : 0.0f;
+      for (int c0 = ecol0; c0 < ecol0 + kT2N / 2; c0 += 16) {
+        uint32_t r[16];
+        if (nst > 0) {  // every lane of the warp takes part in the collective load
+          tmem_ld16(taddr + static_cast<uint32_t>(c0), r);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) r[c] = 0u;
+        }
+        if (jlive) {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int64_t gi = i0 + c0 + c;
+            const float acc = __uint_as_float(r[c]);
+            if (gi < m) out[gi * n + jrow] = bias ? sc * acc + bv : sc * acc;
+          }
+        }
+      }
+    }
+  } else {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    float* recv = reinterpret_cast<float*>(smem);  // [source rank][weight row][column, padded]
+    cluster.sync();                               // every CTA's tensor core is done with its stages
+    if (tid == 0 && !good)
+      for (int q = 0; q < KS; ++q) atomicExch(cluster.map_shared_rank(&any_bad, q), 1);
+    if (warp < 8 && good) {
+      for (int c0 = ecol0; c0 < ecol0 + kT2N / 2; c0 += 16) {
+        uint32_t r[16];
+        if (nst > 0) {
+          tmem_ld16(taddr + static_cast<uint32_t>(c0), r);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) r[c] = 0u;
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const int col = c0 + 4 * g;
+          float* dst = cluster.map_shared_rank(recv, col / kCols);
+          *reinterpret_cast<float4*>(dst + (rank * kT2M + erow) * kPitch + col % kCols) =
+              make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]), __uint_as_float(r[4 * g + 2]),
+                          __uint_as_float(r[4 * g + 3]));
+        }
+      }
+    }
+    cluster.sync();  // every share has landed
+    if (any_bad == 0) {
+      for (int e = tid; e < kT2M * (kCols / 4); e += blockDim.x) {
+        const int wr = e % kT2M, cl = 4 * (e / kT2M);
+        const int64_t gj = j0 + wr;
+        if (gj >= n) continue;
+        float4 a = *reinterpret_cast<const float4*>(recv + wr * kPitch + cl);
+#pragma unroll
+        for (int q = 1; q < KS; ++q) {  // rank order
+          const float4 v = *reinterpret_cast<const float4*>(recv + (q * kT2M + wr) * kPitch + cl);
+          a.x += v.x;
+          a.y += v.y;
+          a.z += v.z;
+          a.w += v.w;
+        }
+        const float sc = __ldg(scale + gj), bv = bias ? __ldg(bias + gj) : 0.0f;
+        const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int64_t gi = i0 + rank * kCols + cl + t;
+          if (gi < m) out[gi * n + gj] = bias ? sc * av[t] + bv : sc * av[t];
+        }
+      }
+    }
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+  __syncthreads();
+  if (warp == kMmaWarp)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kT2N));
+}
+
+template <int KS>
+bnn_status launch_tc2(const CUtensorMap& tx, const uint16_t* packed, const float* scale, const float* bias, int64_t m,
+                      int64_t n, int64_t k, int64_t kt, float* out, cudaStream_t s) {
+  const int64_t gx = KS * ((n + kT2M - 1) / kT2M), gy = (m + kT2N - 1) / kT2N;
+  if (gx > 2147483647LL || gy > 65535) return BNN_ERR_INVALID_ARG;
+  const size_t smem = static_cast<size_t>(kT2S) * kT2Stage + 1024;
+  auto kern = ternary_gemm_tc2_kernel<KS>;
+  BNN_TRY(bnn::ensure_smem(kern, smem));
+  const cudaError_t e = bnn::launch_pdl(kern, dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)),
+                                   dim3(kT2Threads), smem, s, KS, tx, packed, scale, bias, m, n, k, kt, out);
+  if (e != cudaSuccess) return bnn::cuda_fail(e);
+  return bnn::check_launch();
+}
+
 }  // namespace
 
 namespace bnn {
@@ -310,6 +640,18 @@ int ternary_tc_error_count(int reset) {
 bnn_status ternary_gemm_tc(const uint16_t* x_bf16, const uint16_t* packed, const float* scale, const float* bias,
                            int64_t m, int64_t n, int64_t k, float* out, cudaStream_t s) {
   const int64_t kt = words10(k);
+  // activation rows TMA can copy (16-byte aligned): the warp-specialised kernel
+  CUtensorMap tx;
+  if (k > 0 && k % 8 == 0 && k < (1LL << 31) && aligned(x_bf16, 16) && m < (1LL << 31) &&
+      encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x_bf16, static_cast<uint64_t>(k), static_cast<uint64_t>(m),
+                     static_cast<uint64_t>(k) * 2u, 64, kT2N, CU_TENSOR_MAP_SWIZZLE_128B)) {
+    const int64_t tiles = ((n + kT2M - 1) / kT2M) * ((m + kT2N - 1) / kT2N);
+    const int64_t stages = (10 * kt + 63) / 64;
+    const int64_t slots = 2LL * sm_count();  // two CTAs per SM
+    if (tiles * 4 <= slots && stages >= 16) return launch_tc2<4>(tx, packed, scale, bias, m, n, k, kt, out, s);
+    if (tiles * 2 <= slots && stages >= 8) return launch_tc2<2>(tx, packed, scale, bias, m, n, k, kt, out, s);
+    return launch_tc2<1>(tx, packed, scale, bias, m, n, k, kt, out, s);
+  }
   const int64_t ntiles = (n + kTcMW - 1) / kTcMW, gy = (m + kTcNX - 1) / kTcNX;
   if (ntiles * kTcK > 2147483647LL || gy > 65535) return BNN_ERR_INVALID_ARG;
   const int64_t total_stages = (10 * kt + 63) / 64;

@@ -123,6 +123,25 @@ def test_every_base3_word_decodes(bnn, m):
     _gemm_case(bnn, m, 3, 590490, seed=5 + m, trits=rows, algos=(0, 3) if m > 1 else (0,))
 
 
+# Shapes for the warp-specialised tensor-core kernel (k a multiple of 8): the
+# stages split over 4, 2 and 1 CTAs, ragged m and n, and m = 1.
+@pytest.mark.parametrize("m,n,k", [(64, 300, 4096), (200, 1000, 640), (128, 9600, 160), (1, 129, 64),
+                                   (70, 130, 4096 + 8), (33, 255, 2400)])
+def test_tc_warp_specialised_configs(bnn, m, n, k):
+    _gemm_case(bnn, m, n, k, seed=m * 5 + n + k, algos=(3,))
+
+
+def test_every_base3_word_decodes_tma_path(bnn):
+    """All 3^10 words in one row with k a multiple of 8 (the TMA kernel), then
+    a zero-trit word: every code goes through the phase-specialised decoder."""
+    k = 590496
+    words = np.concatenate([np.arange(59049, dtype=np.uint16), np.array([29524], np.uint16)]).reshape(1, -1)
+    trits, bad = oracle.base3_unpack(words, k)
+    assert bad == 0
+    rows = np.concatenate([trits, -trits, np.zeros_like(trits)])
+    _gemm_case(bnn, 64, 3, k, seed=17, trits=rows, algos=(3,))
+
+
 def test_zero_trits_give_exact_zero(bnn):
     k = 300
     packed = np.full((4, 30), 29524, np.uint16)
