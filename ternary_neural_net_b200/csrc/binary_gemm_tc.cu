@@ -70,17 +70,20 @@ constexpr int kTm = 128;                   // weight rows per tile (UMMA M)
 constexpr int kPre = 8;                    // without TMA: stages of words prefetched in registers
 constexpr int kChunkStages = 4;            // with TMA: stages per packed chunk (64 bytes of every row)
 
-template <int BN, bool TMA>
+// WIDE (64-row tiles only): one CTA per SM, twice the expanded stages in
+// flight; otherwise 64-row tiles keep 96 KB so that two CTAs share an SM.
+template <int BN, bool TMA, bool WIDE>
 struct TcCfg {
+  static_assert(!WIDE || BN == 64, "deep rings for the 64-row tile only");
   static constexpr int kRows = kTm + BN;                             // stacked weight + activation rows
   static constexpr uint32_t kStageBytes = kRows * 128u;              // one expanded stage
   static constexpr uint32_t kChunkBytes = kRows * 16u * kChunkStages; // one packed chunk (2 words per stage)
-  static constexpr int S = TMA ? 3 : 4;                              // expanded stages
+  static constexpr int S = (TMA ? 3 : 4) * (WIDE ? 2 : 1);           // expanded stages
   static constexpr int P = TMA ? 2 : 0;                              // packed chunks
   static constexpr uint32_t kSmem = S * kStageBytes + P * kChunkBytes;
   static constexpr int kProducers = 2 * kRows;
   static constexpr int kThreads = kProducers + 64;                   // + MMA warp + TMA warp
-  static constexpr int kMinBlocks = BN <= 64 ? 2 : 1;
+  static constexpr int kMinBlocks = (BN <= 64 && !WIDE) ? 2 : 1;
 };
 
 // 4 bytes per 16-byte chunk word: byte j of word s holds bit 8j + s of hw
@@ -104,14 +107,14 @@ __device__ __forceinline__ void expand_word(uint8_t* dst_row, uint32_t swz, int 
 
 // grid: x = KS * (weight tiles of 128 rows), y = activation tiles of BN rows;
 // clusters of KS CTAs along x
-template <int BN, int KS, int ACC, bool TMA>
-__global__ void __launch_bounds__(TcCfg<BN, TMA>::kThreads, TcCfg<BN, TMA>::kMinBlocks)
+template <int BN, int KS, int ACC, bool TMA, bool WIDE>
+__global__ void __launch_bounds__(TcCfg<BN, TMA, WIDE>::kThreads, TcCfg<BN, TMA, WIDE>::kMinBlocks)
 binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                       const uint64_t* __restrict__ xp, const uint64_t* __restrict__ wp,
                       const float* __restrict__ alpha, const float* __restrict__ bias, int64_t m, int64_t n,
                       int k, int kw, int32_t* __restrict__ dots, float* __restrict__ out,
                       uint32_t* __restrict__ next, int64_t next_w32) {
-  using Cfg = TcCfg<BN, TMA>;
+  using Cfg = TcCfg<BN, TMA, WIDE>;
   constexpr int S = Cfg::S;
   constexpr int P = TMA ? Cfg::P : 1;
   constexpr int kRows = Cfg::kRows;
@@ -466,7 +469,7 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(ACC * BN));
 }
 
-template <int BN, int KS, int ACC>
+template <int BN, int KS, int ACC, bool WIDE = false>
 bnn_status launch_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha, const float* bias, int64_t m,
                      int64_t n, int k, int kw, int32_t* dots, float* out, uint64_t* next, cudaStream_t s) {
   const int64_t gx = KS * ((n + kTm - 1) / kTm), gy = (m + BN - 1) / BN;
@@ -483,11 +486,13 @@ bnn_status launch_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha,
                               static_cast<uint64_t>(m), static_cast<uint64_t>(kw) * 8u, 2 * kChunkStages, BN,
                               CU_TENSOR_MAP_SWIZZLE_64B);
   if (!tma) memset(&tw, 0, sizeof(tw)), memset(&tx, 0, sizeof(tx));
-  const size_t smem = static_cast<size_t>(tma ? TcCfg<BN, true>::kSmem : TcCfg<BN, false>::kSmem) + 1024;
-  auto kern = tma ? binary_gemm_tc_kernel<BN, KS, ACC, true> : binary_gemm_tc_kernel<BN, KS, ACC, false>;
+  const size_t smem =
+      static_cast<size_t>(tma ? TcCfg<BN, true, WIDE>::kSmem : TcCfg<BN, false, WIDE>::kSmem) + 1024;
+  auto kern = tma ? binary_gemm_tc_kernel<BN, KS, ACC, true, WIDE> : binary_gemm_tc_kernel<BN, KS, ACC, false, WIDE>;
   BNN_TRY(bnn::ensure_smem(kern, smem));
   const cudaError_t e = bnn::launch_pdl(kern, dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)),
-                                        dim3(tma ? TcCfg<BN, true>::kThreads : TcCfg<BN, false>::kThreads), smem, s,
+                                        dim3(tma ? TcCfg<BN, true, WIDE>::kThreads : TcCfg<BN, false, WIDE>::kThreads),
+                                        smem, s,
                                         KS, tw, tx, xp, wp, alpha, bias, m, n, k, kw, dots, out,
                                         reinterpret_cast<uint32_t*>(next), 2 * bnn::words64(n));
   if (e != cudaSuccess) return bnn::cuda_fail(e);
@@ -500,10 +505,11 @@ namespace bnn {
 
 // Tensor-core (tcgen05) binary GEMM.  With at least a full wave of 256-row
 // activation tiles the kernel takes those (one CTA per SM; the widest MMA and
-// the fewest re-expansions of the operands); otherwise 64-row tiles (two CTAs
-// per SM), with a cluster of 4 CTAs splitting each tile's stages when that
-// still leaves at most one CTA per SM, else of 2 when the CTAs fit in one
-// wave (at least 4 stages per CTA either way).
+// the fewest re-expansions of the operands); otherwise 64-row tiles.  When the
+// tiles leave SMs idle a cluster of 4 or 2 CTAs splits each tile's stages (at
+// least 4 stages per CTA).  Whenever the CTAs fit one per SM they take the deep
+// ring (twice the stages in flight); otherwise two CTAs share an SM.  Chosen
+// from a sweep over M = 64 .. 8192 at N = K = 4096 (and 8192^3).
 bnn_status binary_gemm_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha, const float* bias, int64_t m,
                           int64_t n, int k, int kw, int32_t* dots, float* out, uint64_t* next, cudaStream_t s) {
   const int64_t wt = (n + kTm - 1) / kTm;
@@ -513,10 +519,13 @@ bnn_status binary_gemm_tc(const uint64_t* xp, const uint64_t* wp, const float* a
     return launch_tc<256, 1, 1>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
   const int64_t tiles = wt * ((m + 63) / 64);
   if (tiles * 4 <= sms && ktiles >= 16)
-    return launch_tc<64, 4, 1>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
+    return launch_tc<64, 4, 1, true>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
+  if (tiles * 2 <= sms && ktiles >= 8)
+    return launch_tc<64, 2, 1, true>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
   if (tiles * 2 <= 2 * sms && ktiles >= 8)
-    return launch_tc<64, 2, 1>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
-  return launch_tc<64, 1, 1>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
+    return launch_tc<64, 2, 1, false>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
+  if (tiles <= sms) return launch_tc<64, 1, 1, true>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
+  return launch_tc<64, 1, 1, false>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
 }
 
 }  // namespace bnn
