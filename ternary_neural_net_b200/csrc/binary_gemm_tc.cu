@@ -170,6 +170,10 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
     any_bad = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
+  if (TMA && tid == kTmaWarp * 32) {  // bring both descriptors on chip while the CTA sets up
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tmap_w)) : "memory");
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
+  }
   if (warp == kMmaWarp) {  // the MMA warp owns the tensor memory
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(&tmem_holder)),
                  "r"(ACC * BN));

@@ -394,6 +394,8 @@ ternary_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16
     any_bad = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
+  if (tid == kTmaWarp * 32)
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
   if (warp == kMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(&tmem_holder)),
                  "r"(kT2N));
