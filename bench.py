@@ -805,7 +805,7 @@ def main():
                    "m": res["m"], "n": res["n"], "k": res["k"],
                    "l2": f"inputs and outputs rotate through {res['R']} copies (> 2x L2) so each step starts cold",
                    "parallelism": f"replicas x{N} (independent problems per GPU)"},
-        "roofline": {"bound": "tensor", "kernel": "binary_gemm_tc_kernel<64,2,1,TMA> (bnn_binary_gemm, m >= 64: "
+        "roofline": {"bound": "tensor", "kernel": "binary_gemm_tc_kernel<128,2,1,TMA,deep> (bnn_binary_gemm, m >= 64: "
                                                   "TMA-fed packed chunks -> 0/1 bytes in swizzled smem, tcgen05.mma "
                                                   "kind::i8 into TMEM, 2-CTA cluster split-K)",
                      "achieved": 2 * gemm_achieved, "peak": int8_peak, "unit": "TOP/s",
@@ -814,7 +814,7 @@ def main():
                      "achieved_basis": "achieved: CUDA events around the kernel on every 16th step of the timed "
                                        "graph (includes the event nodes' serialisation); achieved_back_to_back: "
                                        "a graph of the kernel alone launched back to back",
-                     "traffic": traffic_for("binary_gemm_tc_64x2", "ternary_neural_net_b200/csrc/binary_gemm_tc.cu"),
+                     "traffic": traffic_for("binary_gemm_tc_128x2", "ternary_neural_net_b200/csrc/binary_gemm_tc.cu"),
                      "peak_basis": f"int8 dense tensor peak = measured bf16 {peaks['bf16_tflops']} TFLOP/s x 2 "
                                    f"(nominal int8:bf16 ratio 4.5:2.25 PFLOP/s), {peak_src}"},
         "roofline_popc": {"bound": "alu", "kernel": "binary_gemm_tiled_kernel (bnn_binary_gemm_algo POPC)",

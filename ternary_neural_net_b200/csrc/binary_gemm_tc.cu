@@ -70,15 +70,16 @@ constexpr int kTm = 128;                   // weight rows per tile (UMMA M)
 constexpr int kPre = 8;                    // without TMA: stages of words prefetched in registers
 constexpr int kChunkStages = 4;            // with TMA: stages per packed chunk (64 bytes of every row)
 
-// WIDE (64-row tiles only): one CTA per SM, twice the expanded stages in
-// flight; otherwise 64-row tiles keep 96 KB so that two CTAs share an SM.
+// WIDE (64- and 128-row tiles): one CTA per SM with a deeper ring of expanded
+// stages; otherwise 64-row tiles keep 96 KB so that two CTAs share an SM.
 template <int BN, bool TMA, bool WIDE>
 struct TcCfg {
-  static_assert(!WIDE || BN == 64, "deep rings for the 64-row tile only");
+  static_assert(!WIDE || BN <= 128, "deep rings for the 64- and 128-row tiles");
   static constexpr int kRows = kTm + BN;                             // stacked weight + activation rows
   static constexpr uint32_t kStageBytes = kRows * 128u;              // one expanded stage
   static constexpr uint32_t kChunkBytes = kRows * 16u * kChunkStages; // one packed chunk (2 words per stage)
-  static constexpr int S = (TMA ? 3 : 4) * (WIDE ? 2 : 1);           // expanded stages
+  static constexpr int S = !WIDE ? (TMA ? 3 : 4)                     // expanded stages
+                                 : (BN == 64 ? (TMA ? 6 : 8) : (TMA ? 5 : 6));
   static constexpr int P = TMA ? 2 : 0;                              // packed chunks
   static constexpr uint32_t kSmem = S * kStageBytes + P * kChunkBytes;
   static constexpr int kProducers = 2 * kRows;
@@ -507,20 +508,27 @@ bnn_status launch_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha,
 
 namespace bnn {
 
-// Tensor-core (tcgen05) binary GEMM.  With at least a full wave of 256-row
-// activation tiles the kernel takes those (one CTA per SM; the widest MMA and
-// the fewest re-expansions of the operands); otherwise 64-row tiles.  When the
+// Tensor-core (tcgen05) binary GEMM; tiles chosen from a sweep over M = 64 ..
+// 8192 at N = K = 4096 and 8192.  m <= 128: 64-row activation tiles.  Larger
+// m: 256-row tiles (the widest MMA, the fewest re-expansions of the operands)
+// once they make three quarters of a wave, otherwise 128-row tiles.  When the
 // tiles leave SMs idle a cluster of 4 or 2 CTAs splits each tile's stages (at
-// least 4 stages per CTA).  Whenever the CTAs fit one per SM they take the deep
-// ring (twice the stages in flight); otherwise two CTAs share an SM.  Chosen
-// from a sweep over M = 64 .. 8192 at N = K = 4096 (and 8192^3).
+// least 4 stages per CTA).  CTAs that fit one per SM take the deep ring (more
+// stages in flight); otherwise 64-row-tile CTAs pair up on an SM.
 bnn_status binary_gemm_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha, const float* bias, int64_t m,
                           int64_t n, int k, int kw, int32_t* dots, float* out, uint64_t* next, cudaStream_t s) {
   const int64_t wt = (n + kTm - 1) / kTm;
   const int64_t sms = sm_count();
   const int ktiles = (kw + 1) / 2;
-  if (wt * ((m + 255) / 256) >= sms)
-    return launch_tc<256, 1, 1>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
+  if (m > 128) {
+    if (4 * wt * ((m + 255) / 256) >= 3 * sms)
+      return launch_tc<256, 1, 1>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
+    const int64_t t128 = wt * ((m + 127) / 128);
+    if (t128 * 2 <= sms && ktiles >= 8)
+      return launch_tc<128, 2, 1, true>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
+    if (t128 <= sms) return launch_tc<128, 1, 1, true>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
+    return launch_tc<128, 1, 1, false>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
+  }
   const int64_t tiles = wt * ((m + 63) / 64);
   if (tiles * 4 <= sms && ktiles >= 16)
     return launch_tc<64, 4, 1, true>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);

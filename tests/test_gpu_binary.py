@@ -88,14 +88,15 @@ def test_tiled_matches_oracle(bnn, m, n, k):
     _gemm_case(bnn, m, n, k, seed=m + 7 * n + k)
 
 
-# Shapes that reach each tensor-core configuration: 64-row activation tiles
-# with the stages split over 1, 2 or 4 CTAs of a cluster, with the deep ring
-# (one CTA per SM) and without, 256-row tiles, TMA copies (even word count) and
-# plain loads (odd), and ragged m, n and k.
+# Shapes that reach each tensor-core configuration: 64- and 128-row activation
+# tiles with the stages split over 1, 2 or 4 CTAs of a cluster, with the deep
+# ring (one CTA per SM) and without, 256-row tiles, TMA copies (even word
+# count) and plain loads (odd), and ragged m, n and k.
 @pytest.mark.parametrize("m,n,k", [(40, 300, 2048 + 37), (64, 1000, 1000), (100, 500, 4096), (128, 129, 1100),
                                    (70, 9600, 512), (65, 2, 64 * 20 + 1), (256, 4096 + 3, 4096 - 64),
                                    (257, 383, 2048 * 2 + 64), (2304, 4219, 130), (600, 9000, 760), (50, 700, 2000),
-                                   (64, 1000, 300), (64, 2000, 500)])
+                                   (64, 1000, 300), (64, 2000, 500), (200, 1000, 2048), (300, 3000, 256),
+                                   (384, 6400, 128), (250, 700, 2048 + 130)])
 def test_tc_tile_configs(bnn, m, n, k):
     _gemm_case(bnn, m, n, k, seed=5 * m + n + 3 * k, algos=(3,))
 
