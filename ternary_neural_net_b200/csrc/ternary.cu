@@ -201,120 +201,88 @@ ternary_gemv_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__
 // (v div 3 - 1) turns two multiply-adds into one shared-memory load and one
 // add.  The digit is the high word of 9F and the next fraction its low word
 // (taken with __umulhi and a 32-bit multiply).
-// Lanes of a half-warp own 16 consecutive weight rows and walk the same word
-// index, so the 16 lanes read within one 9-entry table (at most 9 distinct
-// addresses, one per bank: no bank conflicts); the two half-warps take
-// neighbouring words, whose tables (45 floats apart) sit in disjoint banks.
-// Words are dealt to the SLICES thread groups round-robin, so every group
-// gets the same number of words to within one.  The 16-row chunk of packed
-// words is contiguous in memory and is brought into shared memory with
-// 16-byte cp.async (double-buffered across the chunks this CTA owns); the
-// per-slice partial sums are added in a fixed order, then scaled once.  The
-// chunk copies run kLutStages - 1 chunks ahead of the compute (the copy
-// latency from HBM is several times one chunk's compute).
+// One CTA per SM builds the tables once and takes a contiguous block of
+// weight rows; each warp takes one row at a time, its lanes walking the row's
+// words (lane l: words l, l + 32, ... -- 64-byte coalesced loads, the next
+// row's words prefetched in registers while this row is decoded).  A word's
+// tables are 45 floats apart, an odd bank stride, so the lanes' loads rarely
+// share a bank.  The lanes' sums are added by a shuffle tree (a fixed order)
+// and scaled once.  No block barrier after the table build.  Launched with
+// programmatic dependent launch: the first row's words are read before
+// waiting for the kernel that produced x.
 // ---------------------------------------------------------------------------
-constexpr int kLutRows = 16;
-constexpr int kLutStages = 4;
+constexpr int kRowThreads = 1024;
+constexpr int kRowWords = 16;  // words per lane per pass over a row (512 words per warp pass)
 
-template <int SLICES>
-__global__ void __launch_bounds__(kLutRows * SLICES, 1)
-ternary_gemv_lut_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ packed,
-                        const float* __restrict__ scale, int64_t n, int k, int kt, int slice_words,
-                        float* __restrict__ out, const float* __restrict__ bias) {
-  constexpr int THREADS = kLutRows * SLICES;
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  const int npairs = 5 * kt;
-  float* T = reinterpret_cast<float*>(smem_raw);                                   // [npairs][9]
-  const size_t t_bytes = (static_cast<size_t>(npairs) * 9 * sizeof(float) + 15) & ~static_cast<size_t>(15);
-  const size_t chunk_bytes = (static_cast<size_t>(kLutRows) * kt * 2 + 15) & ~static_cast<size_t>(15);
-  uint16_t* const buf0 = reinterpret_cast<uint16_t*>(smem_raw + t_bytes);         // [kLutStages][chunk]
-  const size_t chunk_elems = chunk_bytes / 2;
-  float* red = reinterpret_cast<float*>(smem_raw + t_bytes + kLutStages * chunk_bytes);  // [SLICES][kLutRows]
+__global__ void __launch_bounds__(kRowThreads, 1)
+ternary_gemv_rows_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ packed,
+                         const float* __restrict__ scale, int64_t n, int k, int kt, float* __restrict__ out,
+                         const float* __restrict__ bias) {
+  extern __shared__ float T[];  // [5 kt pairs][9]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int kWarps = kRowThreads / 32;
+  const int64_t r_begin = n * blockIdx.x / gridDim.x, r_end = n * (blockIdx.x + 1) / gridDim.x;
+  bnn::pdl_trigger();
 
-  const int tid = threadIdx.x;
-  const int64_t nchunks = (n + kLutRows - 1) / kLutRows;
-
-  auto issue_chunk = [&](int64_t c, uint16_t* dst) {
-    const int64_t rows = n - c * kLutRows < kLutRows ? n - c * kLutRows : kLutRows;
-    const int64_t bytes = rows * kt * 2;
-    const unsigned char* src = reinterpret_cast<const unsigned char*>(packed + c * kLutRows * kt);
-    for (int64_t off = static_cast<int64_t>(tid) * 16; off < bytes; off += THREADS * 16) {
-      const int64_t left = bytes - off;
-      const int sz = left < 16 ? static_cast<int>(left) : 16;
-      const unsigned saddr = static_cast<unsigned>(__cvta_generic_to_shared(reinterpret_cast<unsigned char*>(dst) + off));
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(saddr), "l"(src + off), "r"(sz));
+  // the words of (row r, pass p) for this lane, 0xFFFF past the row
+  auto fetch = [&](int64_t r, int p, uint32_t (&w)[kRowWords]) {
+#pragma unroll
+    for (int i = 0; i < kRowWords; ++i) {
+      const int j = p * 32 * kRowWords + lane + 32 * i;
+      w[i] = (r < r_end && j < kt) ? static_cast<uint32_t>(__ldcs(packed + r * kt + j)) : 0xFFFFu;
     }
   };
+  const int passes = (kt + 32 * kRowWords - 1) / (32 * kRowWords);
+  int64_t r = r_begin + warp;
+  int p = 0;
+  uint32_t cur[kRowWords];
+  fetch(r, p, cur);  // weights do not depend on the preceding kernel
 
-  // Prefetch the first kLutStages - 1 chunks of this CTA (one commit group each).
+  bnn::pdl_wait();  // x may come from it
+  for (int q = tid; q < 5 * kt; q += kRowThreads) {
+    const float x0 = 2 * q < k ? __uint_as_float(static_cast<uint32_t>(__ldg(x + 2 * q)) << 16) : 0.0f;
+    const float x1 = 2 * q + 1 < k ? __uint_as_float(static_cast<uint32_t>(__ldg(x + 2 * q + 1)) << 16) : 0.0f;
 #pragma unroll
-  for (int st = 0; st < kLutStages - 1; ++st) {
-    const int64_t cc = blockIdx.x + static_cast<int64_t>(st) * gridDim.x;
-    if (cc < nchunks) issue_chunk(cc, buf0 + st * chunk_elems);
-    asm volatile("cp.async.commit_group;\n" ::);
+    for (int v = 0; v < 9; ++v) T[q * 9 + v] = x0 * static_cast<float>(v % 3 - 1) + x1 * static_cast<float>(v / 3 - 1);
   }
-  int64_t c = blockIdx.x;
+  __syncthreads();
 
-  // Pair tables from the activation row (exact products, one rounding per entry).
-  for (int p = tid; p < npairs; p += THREADS) {
-    const float x0 = 2 * p < k ? __uint_as_float(static_cast<uint32_t>(__ldg(x + 2 * p)) << 16) : 0.0f;
-    const float x1 = 2 * p + 1 < k ? __uint_as_float(static_cast<uint32_t>(__ldg(x + 2 * p + 1)) << 16) : 0.0f;
+  float acc0 = 0.0f, acc1 = 0.0f;
+  while (r < r_end) {
+    // the next (row, pass) while this one is decoded
+    const int pn = p + 1 < passes ? p + 1 : 0;
+    const int64_t rn = p + 1 < passes ? r : r + kWarps;
+    uint32_t nxt[kRowWords];
+    fetch(rn, pn, nxt);
 #pragma unroll
-    for (int v = 0; v < 9; ++v)
-      T[p * 9 + v] = x0 * static_cast<float>(v % 3 - 1) + x1 * static_cast<float>(v / 3 - 1);
-  }
-
-  const int row = tid % kLutRows;
-  const int sl = tid / kLutRows;   // this thread takes words sl, sl + SLICES, ...
-  (void)slice_words;
-
-  for (int it = 0; c < nchunks; c += gridDim.x, ++it) {
-    // chunk `it` was the (it+1)-th commit group: allow the kLutStages-2 newer ones to be pending
-    asm volatile("cp.async.wait_group %0;\n" ::"n"(kLutStages - 2));
-    __syncthreads();
-
-    const uint16_t* rowp = buf0 + (it % kLutStages) * chunk_elems + row * kt;
-    float acc0 = 0.0f, acc1 = 0.0f;
-#pragma unroll 2
-    for (int j = sl; j < kt; j += SLICES) {
-      uint32_t F = static_cast<uint32_t>(rowp[j]) * kFixMul;
-      const float* Tj = T + (5 * j) * 9;
+    for (int i = 0; i < kRowWords; ++i) {
+      if (cur[i] != 0xFFFFu) {
+        const int j = p * 32 * kRowWords + lane + 32 * i;
+        const float* Tj = T + 45 * j;
+        uint32_t F = cur[i] * kFixMul;
 #pragma unroll
-      for (int q = 4; q >= 0; --q) {
-        // high and low words of 9F: the digit and the next fraction
-        const uint32_t v = __umulhi(F, 9u);
-        F *= 9u;
-        if (q & 1) acc1 += Tj[q * 9 + v]; else acc0 += Tj[q * 9 + v];
+        for (int q = 4; q >= 0; --q) {
+          const uint32_t v = __umulhi(F, 9u);  // base-9 digit q (trits 2q, 2q+1)
+          F *= 9u;
+          if (q & 1) acc1 += Tj[q * 9 + v]; else acc0 += Tj[q * 9 + v];
+        }
       }
     }
-    red[sl * kLutRows + row] = acc0 + acc1;
-    __syncthreads();
-    if (tid < kLutRows) {
-      const int64_t r = c * kLutRows + tid;
-      if (r < n) {
-        float s = 0.0f;
-#pragma unroll 4
-        for (int q = 0; q < SLICES; ++q) s += red[q * kLutRows + tid];
-        out[r] = bias ? __ldg(scale + r) * s + __ldg(bias + r) : __ldg(scale + r) * s;
-      }
+    if (pn == 0) {  // the row is complete
+      float sum = acc0 + acc1;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+      if (lane == 0) out[r] = bias ? __ldg(scale + r) * sum + __ldg(bias + r) : __ldg(scale + r) * sum;
+      acc0 = acc1 = 0.0f;
     }
-    // The buffer of chunk it + kLutStages - 1 (the one computed in the previous
-    // iteration) and red are rewritten only after this barrier.
-    __syncthreads();
-    const int64_t cn = c + static_cast<int64_t>(kLutStages - 1) * gridDim.x;
-    if (cn < nchunks) issue_chunk(cn, buf0 + ((it + kLutStages - 1) % kLutStages) * chunk_elems);
-    asm volatile("cp.async.commit_group;\n" ::);
+    r = rn;
+    p = pn;
+#pragma unroll
+    for (int i = 0; i < kRowWords; ++i) cur[i] = nxt[i];
   }
-  asm volatile("cp.async.wait_group 0;\n" ::);
 }
 
-constexpr int kLutSlices = 32;
-
-size_t lut_smem_bytes(int64_t kt) {
-  const size_t t_bytes = (static_cast<size_t>(5 * kt) * 9 * sizeof(float) + 15) & ~static_cast<size_t>(15);
-  const size_t chunk_bytes = (static_cast<size_t>(kLutRows) * kt * 2 + 15) & ~static_cast<size_t>(15);
-  return t_bytes + kLutStages * chunk_bytes + static_cast<size_t>(kLutSlices) * kLutRows * sizeof(float);
-}
+size_t rows_smem_bytes(int64_t kt) { return static_cast<size_t>(5 * kt) * 9 * sizeof(float); }
 
 // ---------------------------------------------------------------------------
 // Ternary GEMM (m > 8): trits decoded to bf16 tiles in shared memory, bf16
@@ -553,15 +521,13 @@ bnn_status ternary_gemm_impl(const uint16_t* x_bf16, const uint16_t* packed, con
     return BNN_ERR_MISALIGNED;
   const int64_t kt = bnn::words10(k);
   if (algo == BNN_TALGO_TC) return bnn::ternary_gemm_tc(x_bf16, packed, scale, bias, m, n, k, out, s);
-  if (algo != BNN_TALGO_MMA && m == 1 && kt > 0 && bnn::aligned(packed, 16) && lut_smem_bytes(kt) <= 200 * 1024) {
-    const size_t smem = lut_smem_bytes(kt);
-    auto kern = ternary_gemv_lut_kernel<kLutSlices>;
-    BNN_TRY(bnn::ensure_smem(kern, smem));
-    int slice_words = static_cast<int>((kt + kLutSlices - 1) / kLutSlices);
-    const int64_t nchunks = (n + kLutRows - 1) / kLutRows;
-    const int grid = static_cast<int>(nchunks < bnn::sm_count() ? nchunks : bnn::sm_count());
-    kern<<<grid, kLutRows * kLutSlices, smem, s>>>(x_bf16, packed, scale, n, static_cast<int>(k), static_cast<int>(kt),
-                                                  slice_words, out, bias);
+  if (algo != BNN_TALGO_MMA && m == 1 && kt > 0 && rows_smem_bytes(kt) <= 200 * 1024) {
+    const size_t smem = rows_smem_bytes(kt);
+    BNN_TRY(bnn::ensure_smem(ternary_gemv_rows_kernel, smem));
+    const int64_t sms = bnn::sm_count();
+    const int grid = static_cast<int>(n < sms ? n : sms);
+    BNN_TRY(bnn::launch_pdl(ternary_gemv_rows_kernel, dim3(grid), dim3(kRowThreads), smem, s, 1, x_bf16, packed,
+                            scale, n, static_cast<int>(k), static_cast<int>(kt), out, bias));
     return bnn::check_launch();
   }
   if (algo != BNN_TALGO_MMA && m <= 8) {

@@ -142,6 +142,16 @@ def test_every_base3_word_decodes_tma_path(bnn):
     _gemm_case(bnn, 64, 3, k, seed=17, trits=rows, algos=(3,))
 
 
+def test_every_base3_word_decodes_row_kernel(bnn):
+    """All 3^10 words spread over 60 rows of 1000 words (k = 10000, the m = 1
+    pair-table kernel), every code through its decoder, with a bias."""
+    k = 10000
+    words = (np.arange(60000) % 59049).astype(np.uint16).reshape(60, 1000)
+    trits, bad = oracle.base3_unpack(words, k)
+    assert bad == 0
+    _gemm_case(bnn, 1, 60, k, seed=23, trits=trits, algos=(0, 1))
+
+
 def test_zero_trits_give_exact_zero(bnn):
     k = 300
     packed = np.full((4, 30), 29524, np.uint16)
