@@ -805,7 +805,7 @@ def main():
                    "m": res["m"], "n": res["n"], "k": res["k"],
                    "l2": f"inputs and outputs rotate through {res['R']} copies (> 2x L2) so each step starts cold",
                    "parallelism": f"replicas x{N} (independent problems per GPU)"},
-        "roofline": {"bound": "tensor", "kernel": "binary_gemm_tc_kernel<128,2,1,TMA,deep> (bnn_binary_gemm, m >= 64: "
+        "roofline": {"bound": "tensor", "kernel": "binary_gemm_tc_kernel<128,2,TMA,deep> (bnn_binary_gemm, m >= 64: "
                                                   "TMA-fed packed chunks -> 0/1 bytes in swizzled smem, tcgen05.mma "
                                                   "kind::i8 into TMEM, 2-CTA cluster split-K)",
                      "achieved": 2 * gemm_achieved, "peak": int8_peak, "unit": "TOP/s",

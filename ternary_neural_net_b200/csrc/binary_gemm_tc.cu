@@ -21,10 +21,8 @@
 //     (per 4 bytes a shift and an AND) in the 128-byte-swizzled K-major layout
 //     the tensor core reads, then arrive on the stage's "full" mbarrier;
 //   - one MMA thread: waits for "full", issues 4 tcgen05.mma.kind::i8 (K = 32)
-//     into the int32 accumulator(s) in tensor memory and commits to the
-//     stage's "empty" mbarrier, which the producers wait on before refilling
-//     it.  With ACC = 2 consecutive K = 32 blocks alternate between two
-//     accumulators, so that back-to-back MMAs do not depend on each other;
+//     into the int32 accumulator in tensor memory and commits to the stage's
+//     "empty" mbarrier, which the producers wait on before refilling it;
 //   - the epilogue (warps 0-7; warp w reads tensor-memory lanes 32(w%4).. and
 //     half w/4 of the columns): tcgen05.ld, the popcount correction, alpha,
 //     the optional bias, and stores in which the 32 lanes of a warp write 32
@@ -108,7 +106,7 @@ __device__ __forceinline__ void expand_word(uint8_t* dst_row, uint32_t swz, int 
 
 // grid: x = KS * (weight tiles of 128 rows), y = activation tiles of BN rows;
 // clusters of KS CTAs along x
-template <int BN, int KS, int ACC, bool TMA, bool WIDE>
+template <int BN, int KS, bool TMA, bool WIDE>
 __global__ void __launch_bounds__(TcCfg<BN, TMA, WIDE>::kThreads, TcCfg<BN, TMA, WIDE>::kMinBlocks)
 binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                       const uint64_t* __restrict__ xp, const uint64_t* __restrict__ wp,
@@ -126,7 +124,6 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
   static_assert(S >= 2, "at least two operand stages");
   static_assert(BN % KS == 0 && kCols % 4 == 0, "activation columns split evenly, four at a time");
   static_assert(KS == 1 || KS * kTm * kPitch * 4 <= Cfg::kSmem, "split-K shares must fit the stage memory");
-  static_assert(ACC * BN <= 512, "tensor-memory columns");
 
   extern __shared__ __align__(16) uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[S];
@@ -177,7 +174,7 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
   }
   if (warp == kMmaWarp) {  // the MMA warp owns the tensor memory
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(&tmem_holder)),
-                 "r"(ACC * BN));
+                 "r"(BN));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::);
   }
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
@@ -271,11 +268,10 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
       const uint64_t bd = sw128_desc(smem_base + b * kStageBytes + kTm * 128u);  // activation rows
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
-        const uint32_t d = tmem + static_cast<uint32_t>((kk % ACC) * BN);
-        const uint32_t acc = (j > 0 || kk >= ACC) ? 1u : 0u;
+        const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
         asm volatile(
             "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
-            "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
+            "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem),
             "l"(ad + static_cast<uint64_t>(2 * kk)), "l"(bd + static_cast<uint64_t>(2 * kk)), "r"(idesc), "r"(acc));
       }
       asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
@@ -338,19 +334,11 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
   const int erow = 32 * (warp & 3) + (tid & 31);
   const int ecol0 = (warp >> 2) * (BN / 2);
   const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
-  // the tile's accumulated popc(a AND b) for 16 columns from c0 (sum of the accumulators)
+  // the tile's accumulated popc(a AND b) for 16 columns from c0
   auto load16 = [&](int c0, uint32_t (&r)[16]) {
     if (nst > 0) {
       tmem_ld16(taddr + static_cast<uint32_t>(c0), r);
-      if constexpr (ACC == 2) {
-        uint32_t r2[16];
-        tmem_ld16(taddr + static_cast<uint32_t>(BN + c0), r2);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 16; ++c) r[c] += r2[c];
-      } else {
-        tmem_wait_ld();
-      }
+      tmem_wait_ld();
     } else {
 #pragma unroll
       for (int c = 0; c < 16; ++c) r[c] = 0u;
@@ -471,10 +459,10 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
   __syncthreads();
   if (warp == kMmaWarp)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(ACC * BN));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(BN));
 }
 
-template <int BN, int KS, int ACC, bool WIDE = false>
+template <int BN, int KS, bool WIDE = false>
 bnn_status launch_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha, const float* bias, int64_t m,
                      int64_t n, int k, int kw, int32_t* dots, float* out, uint64_t* next, cudaStream_t s) {
   const int64_t gx = KS * ((n + kTm - 1) / kTm), gy = (m + BN - 1) / BN;
@@ -493,7 +481,7 @@ bnn_status launch_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha,
   if (!tma) memset(&tw, 0, sizeof(tw)), memset(&tx, 0, sizeof(tx));
   const size_t smem =
       static_cast<size_t>(tma ? TcCfg<BN, true, WIDE>::kSmem : TcCfg<BN, false, WIDE>::kSmem) + 1024;
-  auto kern = tma ? binary_gemm_tc_kernel<BN, KS, ACC, true, WIDE> : binary_gemm_tc_kernel<BN, KS, ACC, false, WIDE>;
+  auto kern = tma ? binary_gemm_tc_kernel<BN, KS, true, WIDE> : binary_gemm_tc_kernel<BN, KS, false, WIDE>;
   BNN_TRY(bnn::ensure_smem(kern, smem));
   const cudaError_t e = bnn::launch_pdl(kern, dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)),
                                         dim3(tma ? TcCfg<BN, true, WIDE>::kThreads : TcCfg<BN, false, WIDE>::kThreads),
@@ -522,22 +510,22 @@ bnn_status binary_gemm_tc(const uint64_t* xp, const uint64_t* wp, const float* a
   const int ktiles = (kw + 1) / 2;
   if (m > 128) {
     if (4 * wt * ((m + 255) / 256) >= 3 * sms)
-      return launch_tc<256, 1, 1>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
+      return launch_tc<256, 1>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
     const int64_t t128 = wt * ((m + 127) / 128);
     if (t128 * 2 <= sms && ktiles >= 8)
-      return launch_tc<128, 2, 1, true>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
-    if (t128 <= sms) return launch_tc<128, 1, 1, true>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
-    return launch_tc<128, 1, 1, false>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
+      return launch_tc<128, 2, true>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
+    if (t128 <= sms) return launch_tc<128, 1, true>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
+    return launch_tc<128, 1, false>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
   }
   const int64_t tiles = wt * ((m + 63) / 64);
   if (tiles * 4 <= sms && ktiles >= 16)
-    return launch_tc<64, 4, 1, true>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
+    return launch_tc<64, 4, true>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
   if (tiles * 2 <= sms && ktiles >= 8)
-    return launch_tc<64, 2, 1, true>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
+    return launch_tc<64, 2, true>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
   if (tiles * 2 <= 2 * sms && ktiles >= 8)
-    return launch_tc<64, 2, 1, false>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
-  if (tiles <= sms) return launch_tc<64, 1, 1, true>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
-  return launch_tc<64, 1, 1, false>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
+    return launch_tc<64, 2, false>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
+  if (tiles <= sms) return launch_tc<64, 1, true>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
+  return launch_tc<64, 1, false>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
 }
 
 }  // namespace bnn
