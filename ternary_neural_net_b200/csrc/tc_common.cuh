@@ -49,6 +49,21 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   return false;
 }
 
+// mbar_wait for threads that only wait (MMA issue, copies): between polls the
+// thread sleeps, leaving the issue slots of its SM sub-partition to the warps
+// that compute.
+__device__ __forceinline__ bool mbar_wait_idle(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                               unsigned int* errors) {
+  for (uint32_t it = 0; it < (kSpinLimit >> 4); ++it) {
+    if (mbar_try(bar, parity)) return true;
+    if ((it & 15u) == 15u && *abort_flag) return false;
+    __nanosleep(32);
+  }
+  *abort_flag = 1;
+  atomicAdd(errors, 1u);
+  return false;
+}
+
 // Bounded wait that ignores the abort flag (the final drains).
 __device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity, unsigned int* errors) {
   for (uint32_t it = 0; it < kSpinLimit; ++it)

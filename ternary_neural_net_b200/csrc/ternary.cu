@@ -204,49 +204,64 @@ ternary_gemv_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__
 // One CTA per SM builds the tables once and takes a contiguous block of
 // weight rows; each warp takes one row at a time, its lanes walking the row's
 // words (lane l: words l, l + 32, ... -- 64-byte coalesced loads, the next
-// row's words prefetched in registers while this row is decoded).  A word's
-// tables are 45 floats apart, an odd bank stride, so the lanes' loads rarely
-// share a bank.  The lanes' sums are added by a shuffle tree (a fixed order)
-// and scaled once.  No block barrier after the table build.  Launched with
+// row's words prefetched in registers while this row is decoded).  The tables
+// are stored entry-major, word-minor: entry (q, v) of word j sits at
+// (9q + v) * ktp + j with ktp a multiple of 32, so the 32 lanes (32
+// consecutive words) always hit 32 different banks whatever digits they
+// decode.  The lanes' sums are added by a shuffle tree (a fixed order) and
+// scaled once.  No block barrier after the table build.  Launched with
 // programmatic dependent launch: the first row's words are read before
 // waiting for the kernel that produced x.
 // ---------------------------------------------------------------------------
 constexpr int kRowThreads = 1024;
 constexpr int kRowWords = 16;  // words per lane per pass over a row (512 words per warp pass)
 
+__host__ __device__ constexpr int table_pitch(int kt) { return (kt + 31) & ~31; }
+
 __global__ void __launch_bounds__(kRowThreads, 1)
 ternary_gemv_rows_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ packed,
                          const float* __restrict__ scale, int64_t n, int k, int kt, float* __restrict__ out,
                          const float* __restrict__ bias) {
-  extern __shared__ float T[];  // [5 kt pairs][9]
+  extern __shared__ float T[];  // [45][ktp]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int kWarps = kRowThreads / 32;
+  constexpr int kPassWords = 32 * kRowWords;
+  const int ktp = table_pitch(kt);
   const int64_t r_begin = n * blockIdx.x / gridDim.x, r_end = n * (blockIdx.x + 1) / gridDim.x;
   bnn::pdl_trigger();
 
-  // the words of (row r, pass p) for this lane, 0xFFFF past the row
+  // the words of (row r, pass p) for this lane (words p * kPassWords + lane + 32 i), 0xFFFF past the row
   auto fetch = [&](int64_t r, int p, uint32_t (&w)[kRowWords]) {
+    const bool live = r < r_end;
+    const int lim = live ? kt - p * kPassWords - lane : 0;
+    const uint16_t* src = packed + (live ? r : r_begin) * kt + p * kPassWords + lane;
 #pragma unroll
     for (int i = 0; i < kRowWords; ++i) {
-      const int j = p * 32 * kRowWords + lane + 32 * i;
-      w[i] = (r < r_end && j < kt) ? static_cast<uint32_t>(__ldcs(packed + r * kt + j)) : 0xFFFFu;
+      w[i] = 0xFFFFu;
+      if (32 * i < lim) w[i] = __ldcs(src + 32 * i);
     }
   };
-  const int passes = (kt + 32 * kRowWords - 1) / (32 * kRowWords);
+  const int passes = (kt + kPassWords - 1) / kPassWords;
   int64_t r = r_begin + warp;
   int p = 0;
   uint32_t cur[kRowWords];
   fetch(r, p, cur);  // weights do not depend on the preceding kernel
 
   bnn::pdl_wait();  // x may come from it
-  for (int q = tid; q < 5 * kt; q += kRowThreads) {
-    const float x0 = 2 * q < k ? __uint_as_float(static_cast<uint32_t>(__ldg(x + 2 * q)) << 16) : 0.0f;
-    const float x1 = 2 * q + 1 < k ? __uint_as_float(static_cast<uint32_t>(__ldg(x + 2 * q + 1)) << 16) : 0.0f;
+  for (int e = tid; e < 5 * kt; e += kRowThreads) {
+    const int q = e / kt, j = e - q * kt;  // consecutive threads: consecutive words, distinct banks
+    const int P = 5 * j + q;
+    const float x0 = 2 * P < k ? __uint_as_float(static_cast<uint32_t>(__ldg(x + 2 * P)) << 16) : 0.0f;
+    const float x1 = 2 * P + 1 < k ? __uint_as_float(static_cast<uint32_t>(__ldg(x + 2 * P + 1)) << 16) : 0.0f;
 #pragma unroll
-    for (int v = 0; v < 9; ++v) T[q * 9 + v] = x0 * static_cast<float>(v % 3 - 1) + x1 * static_cast<float>(v / 3 - 1);
+    for (int v = 0; v < 9; ++v)
+      T[(9 * q + v) * ktp + j] = x0 * static_cast<float>(v % 3 - 1) + x1 * static_cast<float>(v / 3 - 1);
   }
   __syncthreads();
 
+  // shared-memory byte addresses: entry (q, v) of word j at tq[q] + v * stride + 4 j'
+  const uint32_t stride = 4u * static_cast<uint32_t>(ktp);
+  const uint32_t t0 = static_cast<uint32_t>(__cvta_generic_to_shared(T)) + 4u * static_cast<uint32_t>(lane);
   float acc0 = 0.0f, acc1 = 0.0f;
   while (r < r_end) {
     // the next (row, pass) while this one is decoded
@@ -254,17 +269,22 @@ ternary_gemv_rows_kernel(const uint16_t* __restrict__ x, const uint16_t* __restr
     const int64_t rn = p + 1 < passes ? r : r + kWarps;
     uint32_t nxt[kRowWords];
     fetch(rn, pn, nxt);
+    uint32_t tq[5];
+#pragma unroll
+    for (int q = 0; q < 5; ++q) tq[q] = t0 + 4u * static_cast<uint32_t>(p * kPassWords) + 9u * q * stride;
 #pragma unroll
     for (int i = 0; i < kRowWords; ++i) {
       if (cur[i] != 0xFFFFu) {
-        const int j = p * 32 * kRowWords + lane + 32 * i;
-        const float* Tj = T + 45 * j;
         uint32_t F = cur[i] * kFixMul;
 #pragma unroll
         for (int q = 4; q >= 0; --q) {
-          const uint32_t v = __umulhi(F, 9u);  // base-9 digit q (trits 2q, 2q+1)
-          F *= 9u;
-          if (q & 1) acc1 += Tj[q * 9 + v]; else acc0 += Tj[q * 9 + v];
+          // base-9 digit q (trits 2q, 2q+1) in the high word of 9F, the rest in the low word
+          const uint64_t P9 = static_cast<uint64_t>(F) * 9u;
+          const uint32_t v = static_cast<uint32_t>(P9 >> 32);
+          F = static_cast<uint32_t>(P9);
+          float t;
+          asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(t) : "r"(tq[q] + v * stride + 128u * i));
+          if (q & 1) acc1 += t; else acc0 += t;
         }
       }
     }
@@ -282,7 +302,9 @@ ternary_gemv_rows_kernel(const uint16_t* __restrict__ x, const uint16_t* __restr
   }
 }
 
-size_t rows_smem_bytes(int64_t kt) { return static_cast<size_t>(5 * kt) * 9 * sizeof(float); }
+size_t rows_smem_bytes(int64_t kt) {
+  return static_cast<size_t>(45) * static_cast<size_t>((kt + 31) & ~int64_t{31}) * sizeof(float);
+}
 
 // ---------------------------------------------------------------------------
 // Ternary GEMM (m > 8): trits decoded to bf16 tiles in shared memory, bf16
@@ -521,6 +543,10 @@ bnn_status ternary_gemm_impl(const uint16_t* x_bf16, const uint16_t* packed, con
     return BNN_ERR_MISALIGNED;
   const int64_t kt = bnn::words10(k);
   if (algo == BNN_TALGO_TC) return bnn::ternary_gemm_tc(x_bf16, packed, scale, bias, m, n, k, out, s);
+  // one activation tile (decode-bound): the kernel that decodes into tensor memory
+  if (algo == BNN_TALGO_AUTO && m > 8 && m <= 64 && k % 8 == 0 && bnn::aligned(x_bf16, 16) &&
+      bnn::aligned(packed, 4))
+    return bnn::ternary_gemm_tc(x_bf16, packed, scale, bias, m, n, k, out, s);
   if (algo != BNN_TALGO_MMA && m == 1 && kt > 0 && rows_smem_bytes(kt) <= 200 * 1024) {
     const size_t smem = rows_smem_bytes(kt);
     BNN_TRY(bnn::ensure_smem(ternary_gemv_rows_kernel, smem));

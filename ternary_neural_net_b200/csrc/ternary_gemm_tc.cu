@@ -23,6 +23,8 @@
 // bnn_device_error_count).
 #include <cooperative_groups.h>
 
+#include <mutex>
+
 #include "bnn_internal.cuh"
 #include "tc_common.cuh"
 
@@ -328,8 +330,10 @@ constexpr uint32_t kZeroWord = 29524u;               // all ten trits 0 (every d
 // floor(v / 10) for any 32-bit v (multiply-high by ceil(2^35 / 10))
 __device__ __forceinline__ uint32_t div10(uint32_t v) { return __umulhi(v, 0xCCCCCCCDu) >> 3; }
 
-// 9^p (p <= 4)
-__host__ __device__ constexpr uint32_t pow9(int p) { return p <= 0 ? 1u : 9u * pow9(p - 1); }
+// 9^p (0 <= p <= 4); not recursive, so that it folds to a constant in unrolled code
+__host__ __device__ __forceinline__ constexpr uint32_t pow9(int p) {
+  return p <= 0 ? 1u : (p == 1 ? 9u : (p == 2 ? 81u : (p == 3 ? 729u : 6561u)));
+}
 
 // the 8 bf16 pairs of 16 trits starting at phase R10 of word 0 (F[i] = word_i * kFix)
 template <int R10>
@@ -386,7 +390,7 @@ ternary_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16
   }
   if (tid == 0) {
     for (int i = 0; i < kT2S; ++i) {
-      mbar_init(smem_u32(&full_bar[i]), kT2Prod + 1);  // producers + the TMA thread's expect_tx
+      mbar_init(smem_u32(&full_bar[i]), 2);  // one producer after their barrier + the TMA thread's expect_tx
       mbar_init(smem_u32(&empty_bar[i]), 1);
     }
     mbar_init(smem_u32(&done_bar), 1);
@@ -471,12 +475,13 @@ ternary_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16
           *reinterpret_cast<uint4*>(dst + (((2u * quarter) ^ swz) << 4)) = lo;
           *reinterpret_cast<uint4*>(dst + (((2u * quarter + 1u) ^ swz) << 4)) = hi;
           asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-          mbar_arrive(smem_u32(&full_bar[b]));
         }
         // one decision for all producers: the staged window is complete and the
-        // decoded one may be overwritten; a wait that ran out stops them all
+        // decoded one may be overwritten; a wait that ran out stops them all.
+        // After it one thread tells the tensor core that the stage is written.
         ok = bnn::tc::producer_barrier_and(fine, kT2Prod);
         if (!ok) break;
+        if (tid == 0) mbar_arrive(smem_u32(&full_bar[b]));
       }
     }
   } else if (tid == kMmaWarp * 32) {
@@ -625,6 +630,427 @@ bnn_status launch_tc2(const CUtensorMap& tx, const uint16_t* packed, const float
   return bnn::check_launch();
 }
 
+// ---------------------------------------------------------------------------
+// Decode-bound shapes (at most 64 activation rows): the decoded trits go to
+// tensor memory.
+//
+// With one activation tile every packed word is decoded exactly once, so the
+// decode is the whole cost.  Here it writes no shared memory: each producer
+// thread owns one weight row (its tensor-memory lane) and one 64-trit quarter
+// of a 256-trit stage, decodes its 32 bf16 pairs into registers (five base-9
+// digit phases, warp-uniform, as above) and stores them with one
+// tcgen05.st.32x32b.x32 into the stage's A slot of tensor memory; the MMA reads
+// A from there ([a-tmem] operand) and B, the activations, from shared memory
+// (four TMA boxes of 64 x 64 bf16 per stage, 128-byte swizzle).  The packed
+// words reach shared memory without passing through registers: four loader
+// warps copy, per group of five stages (1280 trits = 128 words, 129 when the
+// group starts inside a word), every row's window as 4-byte cp.async units
+// (the row's bytes from the 4-byte boundary at or below its first word; units
+// past the end of the matrix are zero-filled) into a [row][65 units] buffer
+// (odd stride: a warp's 32 rows read 32 different banks), double-buffered and
+// completed on an mbarrier by cp.async.mbarrier.arrive.  Per stage a producer
+// waits for its slot to be free, decodes, stores, waits for the store and
+// arrives once per warp; one thread waits for the A slot and the B tile and
+// issues 16 tcgen05.mma (K = 16).  A cluster of KS CTAs splits the stages;
+// the partial tiles are added in rank order through distributed shared
+// memory, each CTA owning a block of activation columns (multiples of 4).
+// ---------------------------------------------------------------------------
+constexpr int kT3M = 128;                              // weight rows = tensor-memory lanes
+constexpr int kT3N = 64;                               // activation rows (UMMA N)
+constexpr int kT3K = 256;                              // trits per stage
+constexpr int kT3S = 3;                                // stages in flight
+constexpr int kT3G = 5;                                // stages per word group (1280 trits)
+constexpr int kT3GU = 65;                              // 4-byte units staged per row and group (129 words + offset)
+constexpr int kT3Prod = 512;                           // producer threads (16 warps)
+constexpr int kT3Load = 128;                           // loader threads (4 warps)
+constexpr int kT3Threads = kT3Prod + 64 + kT3Load;     // + MMA warp + TMA warp + loaders
+constexpr uint32_t kT3BAtom = kT3N * 128u;             // one 64-trit box of activations
+constexpr uint32_t kT3BStage = 4 * kT3BAtom;
+constexpr uint32_t kT3WBuf = kT3M * kT3GU * 4u;        // one group's words
+constexpr uint32_t kT3Cols = 512;                      // D (64 columns) + kT3S A slots of 128
+constexpr int kT3Units = kT3N / 4;                     // activation columns in units of 4
+static_assert(kT3N + 128 * kT3S <= static_cast<int>(kT3Cols), "tensor-memory columns");
+static_assert(2 * kT3GU * 4 >= 2 + 2 * (kT3G * kT3K / 10 + 1) + 2, "a group's window fits its units");
+
+// the 32 bf16 pairs of 64 trits starting at phase PH of word 0 (F[i] = word_i * kFix)
+template <int PH>
+__device__ __forceinline__ void decode64(const uint32_t (&F)[8], const uint32_t* lut, uint32_t (&a)[32]) {
+#pragma unroll
+  for (int p = 0; p < 32; ++p) {
+    const int kp = PH / 2 + p;         // pair index counted from word 0
+    const int j = kp / 5, q = kp % 5;  // word, base-9 digit
+    a[p] = lut[__umulhi(F[j] * pow9(4 - q), 9u)];
+  }
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t addr, const uint32_t (&a)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n" ::"r"(addr),
+      "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a[4]), "r"(a[5]), "r"(a[6]), "r"(a[7]), "r"(a[8]), "r"(a[9]),
+      "r"(a[10]), "r"(a[11]), "r"(a[12]), "r"(a[13]), "r"(a[14]), "r"(a[15]), "r"(a[16]), "r"(a[17]), "r"(a[18]),
+      "r"(a[19]), "r"(a[20]), "r"(a[21]), "r"(a[22]), "r"(a[23]), "r"(a[24]), "r"(a[25]), "r"(a[26]), "r"(a[27]),
+      "r"(a[28]), "r"(a[29]), "r"(a[30]), "r"(a[31])
+      : "memory");
+}
+
+// 4 bytes from global to shared (src_bytes of them read, the rest zero)
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+
+// first activation column owned by cluster rank q (blocks of whole units of 4)
+template <int KS>
+__device__ __forceinline__ int t3_col_begin(int q) { return 4 * ((kT3Units * q) / KS); }
+
+template <int KS>
+__global__ void __launch_bounds__(kT3Threads, 1)
+ternary_gemm_tmem_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t* __restrict__ packed,
+                         const float* __restrict__ scale, const float* __restrict__ bias, int64_t m, int64_t n,
+                         int64_t kt, int rows_cta, float* __restrict__ out) {
+  using namespace bnn::tc;
+  constexpr int kMaxCols = 4 * ((kT3Units + KS - 1) / KS);
+  constexpr int kPitch = kMaxCols + 4;  // padded receive row (floats)
+  static_assert(KS * kT3M * kPitch * 4 <= kT3S * kT3BStage, "split-K shares must fit the activation stages");
+
+  extern __shared__ __align__(16) uint8_t t3_raw[];
+  __shared__ __align__(8) uint64_t a_full[kT3S];   // one arrive per producer warp
+  __shared__ __align__(8) uint64_t b_full[kT3S];   // the TMA thread's expect_tx + bytes
+  __shared__ __align__(8) uint64_t empty_bar[kT3S];
+  __shared__ __align__(8) uint64_t w_full[2];      // the loaders' copies of a group's words
+  __shared__ __align__(8) uint64_t w_empty[2];     // one arrive per producer warp after the group
+  __shared__ __align__(8) uint64_t done_bar;
+  __shared__ uint32_t tmem_holder;
+  __shared__ volatile int abort_flag;
+  __shared__ int any_bad;
+  __shared__ uint32_t lut[9];
+  uint8_t* const bsm = t3_raw + ((1024u - (smem_u32(t3_raw) & 1023u)) & 1023u);  // kT3S activation stages
+  uint8_t* const wbuf = bsm + kT3S * kT3BStage;                                   // [2][kT3M][kT3GU] units
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int rank = KS > 1 ? static_cast<int>(blockIdx.x % KS) : 0;
+  const int64_t j0 = static_cast<int64_t>(blockIdx.x / KS) * rows_cta;  // first weight row (rows_cta: 32..128)
+  const int64_t i0 = static_cast<int64_t>(blockIdx.y) * kT3N;        // first activation row
+  const int64_t total = (10 * kt + kT3K - 1) / kT3K;                 // stages covering every word
+  const int64_t share = (total + KS - 1) / KS;
+  const int64_t sb = rank * share < total ? rank * share : total;
+  const int64_t se = sb + share < total ? sb + share : total;
+  const int nst = static_cast<int>(se - sb);
+  const int ngroups = (nst + kT3G - 1) / kT3G;
+  constexpr int kMmaWarp = kT3Prod / 32, kTmaWarp = kMmaWarp + 1, kLoadWarp0 = kMmaWarp + 2;
+  const int prod_warps = 4 * (rows_cta / 32);  // producer warps with rows: 4 quarters of the stage per 32 rows
+  const int64_t rows_live = n - j0 < rows_cta ? n - j0 : rows_cta;
+
+  if (tid < 9) {
+    const int lo = tid % 3, hi = tid / 3;  // digit = trit + 1
+    const uint32_t blo = lo == 0 ? 0xBF80u : (lo == 2 ? 0x3F80u : 0u);
+    const uint32_t bhi = hi == 0 ? 0xBF80u : (hi == 2 ? 0x3F80u : 0u);
+    lut[tid] = blo | (bhi << 16);
+  }
+  if (tid == 0) {
+    for (int i = 0; i < kT3S; ++i) {
+      mbar_init(smem_u32(&a_full[i]), prod_warps);
+      mbar_init(smem_u32(&b_full[i]), 1);
+      mbar_init(smem_u32(&empty_bar[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&w_full[i]), kT3Load);
+      mbar_init(smem_u32(&w_empty[i]), prod_warps);
+    }
+    mbar_init(smem_u32(&done_bar), 1);
+    abort_flag = 0;
+    any_bad = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  if (tid == kTmaWarp * 32)
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(&tmem_holder)),
+                 "r"(kT3Cols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::);
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+  const uint32_t tmem = tmem_holder;  // D: columns [0, 64); A slot i: columns [64 + 128 i, 192 + 128 i)
+  bnn::pdl_trigger();
+
+  if (tid < kT3Prod) {
+    // ------------------------------------------------------------ producers
+    // (warps whose 32 rows lie past rows_cta have nothing to do: their lanes
+    // of the accumulator are never stored)
+    const int row = 32 * (warp & 3) + lane;  // weight row of the tile = tensor-memory lane
+    const int qk = warp >> 2;                // 64-trit quarter of each stage
+    const uint32_t lane_field = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    bool ok = 32 * (warp & 3) < rows_cta;
+    for (int g = 0; g < ngroups && ok; ++g) {
+      const int buf = g & 1;
+      bool fine = mbar_wait(smem_u32(&w_full[buf]), static_cast<uint32_t>((g >> 1) & 1), &abort_flag,
+                            &g_bnn_tc_ternary_errors);
+      if (!__all_sync(0xffffffffu, fine)) break;
+      const int64_t s0 = sb + kT3G * static_cast<int64_t>(g);  // first stage of the group
+      const int64_t w0 = (kT3K * s0) / 10;                     // first word staged
+      // this row's words in the buffer: its first staged byte sits at the row's
+      // byte offset mod 4 within its units
+      const int64_t rbyte = ((j0 + row) * kt + w0) * 2;
+      const uint16_t* wrow =
+          reinterpret_cast<const uint16_t*>(wbuf + buf * kT3WBuf + row * (kT3GU * 4) + (rbyte & 3));
+      for (int u = 0; u < kT3G; ++u) {
+        const int jj = kT3G * g + u;
+        if (jj >= nst) break;
+        const int slot = jj % kT3S;
+        fine = jj < kT3S || mbar_wait(smem_u32(&empty_bar[slot]), static_cast<uint32_t>((jj / kT3S + 1) & 1),
+                                      &abort_flag, &g_bnn_tc_ternary_errors);
+        if (!__all_sync(0xffffffffu, fine)) {  // the tensor-memory store below is warp-collective
+          ok = false;
+          break;
+        }
+        asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+        const int64_t t0 = kT3K * (sb + jj) + 64 * qk;  // first trit of this quarter
+        const int64_t jw = t0 / 10;
+        const uint16_t* wr = wrow + (jw - w0);
+        uint32_t F[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) F[i] = static_cast<uint32_t>(wr[i]) * kFix;
+        uint32_t av[32];
+        switch (static_cast<int>(t0 - 10 * jw)) {  // the phase, warp-uniform
+          case 0: decode64<0>(F, lut, av); break;
+          case 2: decode64<2>(F, lut, av); break;
+          case 4: decode64<4>(F, lut, av); break;
+          case 6: decode64<6>(F, lut, av); break;
+          default: decode64<8>(F, lut, av); break;
+        }
+        tmem_st32(tmem + lane_field + static_cast<uint32_t>(kT3N + 128 * slot + 32 * qk), av);
+        asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
+        asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&a_full[slot]));
+      }
+      __syncwarp();
+      if (ok && lane == 0) mbar_arrive(smem_u32(&w_empty[buf]));  // this warp is done with the group's words
+    }
+  } else if (warp >= kLoadWarp0) {
+    // ------------------------------------------------------------ loaders of the packed words
+    const int lt = tid - kLoadWarp0 * 32;
+    const uint8_t* gbase = reinterpret_cast<const uint8_t*>(packed);
+    const int64_t total_bytes = n * kt * 2;
+    for (int g = 0; g < ngroups; ++g) {
+      const int buf = g & 1;
+      if (g >= 2 && !mbar_wait_idle(smem_u32(&w_empty[buf]), static_cast<uint32_t>(((g >> 1) + 1) & 1), &abort_flag,
+                               &g_bnn_tc_ternary_errors))
+        break;
+      const int64_t w0 = (kT3K * (sb + kT3G * static_cast<int64_t>(g))) / 10;
+      const uint32_t dbase = smem_u32(wbuf + buf * kT3WBuf);
+      for (int idx = lt; idx < rows_cta * kT3GU; idx += kT3Load) {
+        const int r = idx / kT3GU, un = idx - r * kT3GU;
+        const int64_t a = ((((j0 + r) * kt + w0) * 2) & ~int64_t{3}) + 4 * un;  // 4-byte unit of the matrix
+        const int64_t left = r < rows_live ? total_bytes - a : 0;
+        const uint32_t bytes = left >= 4 ? 4u : (left > 0 ? static_cast<uint32_t>(left) : 0u);
+        cp_async4(dbase + static_cast<uint32_t>(idx) * 4u, gbase + (bytes ? a : 0), bytes);
+      }
+      asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(smem_u32(&w_full[buf])) : "memory");
+    }
+    asm volatile("cp.async.wait_all;\n" ::: "memory");  // no copy in flight when the CTA retires
+  } else if (tid == kMmaWarp * 32) {
+    // ------------------------------------------------------------ MMA issue
+    // D f32, A (tensor memory) and B bf16, K-major, N = 64, M = 128
+    const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((static_cast<uint32_t>(kT3N) >> 3) << 17) |
+                           ((static_cast<uint32_t>(kT3M) >> 4) << 24);
+    const uint32_t base = smem_u32(bsm);
+    for (int jj = 0; jj < nst; ++jj) {
+      const int slot = jj % kT3S;
+      const uint32_t par = static_cast<uint32_t>((jj / kT3S) & 1);
+      if (!mbar_wait_idle(smem_u32(&b_full[slot]), par, &abort_flag, &g_bnn_tc_ternary_errors) ||
+          !mbar_wait_idle(smem_u32(&a_full[slot]), par, &abort_flag, &g_bnn_tc_ternary_errors))
+        break;
+      asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+#pragma unroll
+      for (int kk = 0; kk < 16; ++kk) {
+        const uint64_t bd = sw128_desc(base + slot * kT3BStage + (kk >> 2) * kT3BAtom) +
+                            static_cast<uint64_t>(2 * (kk & 3));
+        const uint32_t at = tmem + static_cast<uint32_t>(kT3N + 128 * slot + 8 * kk);
+        const uint32_t acc = (jj > 0 || kk > 0) ? 1u : 0u;
+        asm volatile(
+            "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(tmem),
+            "r"(at), "l"(bd), "r"(idesc), "r"(acc));
+      }
+      mma_commit(smem_u32(&empty_bar[slot]));
+    }
+    mma_commit(smem_u32(&done_bar));
+  } else if (tid == kTmaWarp * 32) {
+    // ------------------------------------------------------------ TMA copies of the activations
+    bnn::pdl_wait();  // x may come from the preceding kernel
+    int issued = 0;
+    for (int jj = 0; jj < nst; ++jj) {
+      const int slot = jj % kT3S;
+      if (jj >= kT3S && !mbar_wait_idle(smem_u32(&empty_bar[slot]), static_cast<uint32_t>((jj / kT3S + 1) & 1),
+                                        &abort_flag, &g_bnn_tc_ternary_errors))
+        break;
+      const uint32_t bar = smem_u32(&b_full[slot]);
+      const uint32_t dst = smem_u32(bsm + slot * kT3BStage);
+      mbar_expect_tx(bar, kT3BStage);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        tma_load_2d(dst + q * kT3BAtom, &tmap_x, static_cast<int>(kT3K * (sb + jj) + 64 * q), static_cast<int>(i0),
+                    bar);
+      issued = jj + 1;
+    }
+    // no copy may still be in flight when the CTA retires
+    for (int jj = issued - kT3S; jj < issued; ++jj)
+      if (jj >= 0)
+        mbar_drain(smem_u32(&b_full[jj % kT3S]), static_cast<uint32_t>((jj / kT3S) & 1), &g_bnn_tc_ternary_errors);
+  }
+  __syncwarp();
+
+  // -------------------------------------------------------------- epilogue
+  bool drained = true;
+  if (warp < 8) {
+    drained = mbar_drain(smem_u32(&done_bar), 0u, &g_bnn_tc_ternary_errors);
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+  }
+  const bool good = __syncthreads_and(drained && abort_flag == 0) != 0;
+  const int erow = 32 * (warp & 3) + lane;       // weight row (tensor-memory lane)
+  const int ecol0 = (warp >> 2) * (kT3N / 2);    // half of the activation columns
+  const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+  const int64_t jrow = j0 + erow;
+  if constexpr (KS == 1) {
+    if (warp < 8 && good) {
+      const bool jlive = erow < rows_live;
+      const float sc = jlive ? __ldg(scale + jrow) : 0.0f, bv = (bias && jlive) ? __ldg(bias + jrow) : 0.0f;
+      for (int c0 = ecol0; c0 < ecol0 + kT3N / 2; c0 += 16) {
+        uint32_t r[16];
+        if (nst > 0) {  // every lane of the warp takes part in the collective load
+          tmem_ld16(taddr + static_cast<uint32_t>(c0), r);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) r[c] = 0u;
+        }
+        if (jlive) {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int64_t gi = i0 + c0 + c;
+            const float acc = __uint_as_float(r[c]);
+            if (gi < m) out[gi * n + jrow] = bias ? sc * acc + bv : sc * acc;
+          }
+        }
+      }
+    }
+  } else {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    float* recv = reinterpret_cast<float*>(bsm);  // [source rank][weight row][owned column, padded]
+    cluster.sync();                              // every CTA's tensor core is done with its stages
+    if (tid == 0 && !good)
+      for (int q = 0; q < KS; ++q) atomicExch(cluster.map_shared_rank(&any_bad, q), 1);
+    if (warp < 8 && good) {
+      for (int c0 = ecol0; c0 < ecol0 + kT3N / 2; c0 += 16) {
+        uint32_t r[16];
+        if (nst > 0) {
+          tmem_ld16(taddr + static_cast<uint32_t>(c0), r);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) r[c] = 0u;
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const int col = c0 + 4 * g;
+          int q = 0;
+#pragma unroll
+          for (int t = 1; t < KS; ++t) q += col >= t3_col_begin<KS>(t) ? 1 : 0;
+          float* dst = cluster.map_shared_rank(recv, q);
+          *reinterpret_cast<float4*>(dst + (rank * kT3M + erow) * kPitch + (col - t3_col_begin<KS>(q))) =
+              make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]), __uint_as_float(r[4 * g + 2]),
+                          __uint_as_float(r[4 * g + 3]));
+        }
+      }
+    }
+    cluster.sync();  // every share has landed
+    if (any_bad == 0) {
+      const int cb = t3_col_begin<KS>(rank), ncols = t3_col_begin<KS>(rank + 1) - cb;
+      for (int e = tid; e < kT3M * (ncols / 4); e += blockDim.x) {
+        const int wr = e % kT3M, cl = 4 * (e / kT3M);
+        const int64_t gj = j0 + wr;
+        if (wr >= rows_live) continue;
+        float4 a = *reinterpret_cast<const float4*>(recv + wr * kPitch + cl);
+#pragma unroll
+        for (int q = 1; q < KS; ++q) {  // rank order
+          const float4 v = *reinterpret_cast<const float4*>(recv + (q * kT3M + wr) * kPitch + cl);
+          a.x += v.x;
+          a.y += v.y;
+          a.z += v.z;
+          a.w += v.w;
+        }
+        const float sc = __ldg(scale + gj), bv = bias ? __ldg(bias + gj) : 0.0f;
+        const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int64_t gi = i0 + cb + cl + t;
+          if (gi < m) out[gi * n + gj] = bias ? sc * av[t] + bv : sc * av[t];
+        }
+      }
+    }
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+  __syncthreads();
+  if (warp == kMmaWarp)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kT3Cols));
+}
+
+// dynamic shared memory: 1024-byte alignment slack, the activation stages, two
+// word buffers and 16 bytes past them (a producer may read, and not use, the
+// word after its row's window)
+size_t tmem_smem_bytes() { return 1024 + static_cast<size_t>(kT3S) * kT3BStage + 2u * kT3WBuf + 16; }
+
+// clusters of KS CTAs of the tensor-memory kernel that can run at once (0 when unknown)
+template <int KS>
+int tmem_active_clusters() {
+  static std::mutex mu;
+  static int cached[64] = {};
+  const int dev = bnn::current_device();
+  if (dev < 0 || dev >= 64) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached[dev] != 0) return cached[dev] > 0 ? cached[dev] : 0;
+  auto kern = ternary_gemm_tmem_kernel<KS>;
+  int num = 0;
+  if (bnn::ensure_smem(kern, tmem_smem_bytes()) == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(KS * 128, 1, 1);
+    cfg.blockDim = dim3(kT3Threads, 1, 1);
+    cfg.dynamicSmemBytes = tmem_smem_bytes();
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = KS;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&num, kern, &cfg) != cudaSuccess) {
+      (void)cudaGetLastError();
+      num = 0;
+    }
+  }
+  cached[dev] = num > 0 ? num : -1;
+  return num > 0 ? num : 0;
+}
+
+template <int KS>
+bnn_status launch_tmem(const CUtensorMap& tx, const uint16_t* packed, const float* scale, const float* bias, int64_t m,
+                       int64_t n, int64_t kt, int rows_cta, float* out, cudaStream_t s) {
+  const int64_t gx = KS * ((n + rows_cta - 1) / rows_cta), gy = (m + kT3N - 1) / kT3N;
+  if (gx > 2147483647LL || gy > 65535) return BNN_ERR_INVALID_ARG;
+  auto kern = ternary_gemm_tmem_kernel<KS>;
+  const size_t smem = tmem_smem_bytes();
+  BNN_TRY(bnn::ensure_smem(kern, smem));
+  const cudaError_t e = bnn::launch_pdl(kern, dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)),
+                                        dim3(kT3Threads), smem, s, KS, tx, packed, scale, bias, m, n, kt, rows_cta,
+                                        out);
+  if (e != cudaSuccess) return bnn::cuda_fail(e);
+  return bnn::check_launch();
+}
+
 }  // namespace
 
 namespace bnn {
@@ -647,6 +1073,39 @@ bnn_status ternary_gemm_tc(const uint16_t* x_bf16, const uint16_t* packed, const
   if (k > 0 && k % 8 == 0 && k < (1LL << 31) && aligned(x_bf16, 16) && m < (1LL << 31) &&
       encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x_bf16, static_cast<uint64_t>(k), static_cast<uint64_t>(m),
                      static_cast<uint64_t>(k) * 2u, 64, kT2N, CU_TENSOR_MAP_SWIZZLE_128B)) {
+    if (m <= kT3N && aligned(packed, 4)) {
+      // one activation tile: decode-bound.  Choose the rows per CTA (32..128)
+      // and the cluster split of the stages for the fewest waves times the
+      // time of a CTA, in units of a 128-row stage / 128: the decode scales with
+      // the rows (not below 64: fewer warps hide less latency), and every CTA
+      // pays about two stages of start-up (its first words), plus two for the
+      // exchange of a split.  CTAs of a cluster take whole SMs, so few clusters
+      // of 3 or 4 run at once.
+      const int64_t stages3 = (10 * kt + kT3K - 1) / kT3K;
+      const int active[5] = {0, tmem_active_clusters<1>(), tmem_active_clusters<2>(), tmem_active_clusters<3>(),
+                             tmem_active_clusters<4>()};
+      int best_ks = 1, best_rows = kT3M;
+      int64_t best_cost = INT64_MAX;
+      for (int rows = kT3M; rows >= 32; rows -= 32) {
+        const int64_t tiles3 = (n + rows - 1) / rows;
+        for (int ks = 1; ks <= 4; ++ks) {
+          if (active[ks] <= 0 || (ks > 1 && stages3 < 2 * ks)) continue;
+          const int64_t waves = (tiles3 + active[ks] - 1) / active[ks];
+          const int64_t cost = waves * ((rows < 64 ? 64 : rows) * ((stages3 + ks - 1) / ks) + 256 + (ks > 1 ? 256 : 32));
+          if (cost < best_cost) {
+            best_cost = cost;
+            best_ks = ks;
+            best_rows = rows;
+          }
+        }
+      }
+      switch (best_ks) {
+        case 4: return launch_tmem<4>(tx, packed, scale, bias, m, n, kt, best_rows, out, s);
+        case 3: return launch_tmem<3>(tx, packed, scale, bias, m, n, kt, best_rows, out, s);
+        case 2: return launch_tmem<2>(tx, packed, scale, bias, m, n, kt, best_rows, out, s);
+        default: return launch_tmem<1>(tx, packed, scale, bias, m, n, kt, best_rows, out, s);
+      }
+    }
     const int64_t tiles = ((n + kT2M - 1) / kT2M) * ((m + kT2N - 1) / kT2N);
     const int64_t stages = (10 * kt + 63) / 64;
     const int64_t slots = 2LL * sm_count();  // two CTAs per SM

@@ -123,10 +123,13 @@ def test_every_base3_word_decodes(bnn, m):
     _gemm_case(bnn, m, 3, 590490, seed=5 + m, trits=rows, algos=(0, 3) if m > 1 else (0,))
 
 
-# Shapes for the warp-specialised tensor-core kernel (k a multiple of 8): the
-# stages split over 4, 2 and 1 CTAs, ragged m and n, and m = 1.
+# Shapes for the warp-specialised tensor-core kernels (k a multiple of 8): the
+# stages split over 4, 3, 2 and 1 CTAs, ragged m and n, word groups cut short,
+# a single stage, and m = 1.  m <= 64 takes the kernel that decodes into
+# tensor memory, larger m the one that decodes into shared memory.
 @pytest.mark.parametrize("m,n,k", [(64, 300, 4096), (200, 1000, 640), (128, 9600, 160), (1, 129, 64),
-                                   (70, 130, 4096 + 8), (33, 255, 2400)])
+                                   (70, 130, 4096 + 8), (33, 255, 2400), (50, 10000, 1600), (40, 385, 1288),
+                                   (64, 129, 8)])
 def test_tc_warp_specialised_configs(bnn, m, n, k):
     _gemm_case(bnn, m, n, k, seed=m * 5 + n + k, algos=(3,))
 
