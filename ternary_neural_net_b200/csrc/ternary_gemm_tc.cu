@@ -1,5 +1,11 @@
 // bnn_ternary_gemm on the 5th-generation tensor cores (tcgen05, sm_100a).
 //
+// Three kernels: ternary_gemm_tmem_kernel (at most 64 activation rows, k a
+// multiple of 8: the decoded trits are stored to tensor memory),
+// ternary_gemm_tc2_kernel (more rows, k a multiple of 8: warp-specialised,
+// decoded trits in shared memory) and ternary_gemm_tc_kernel (any shape,
+// described first below).
+//
 // "BalancedTernaryEngine" README, "Module Overview" (Layer.forward) with the
 // "Features" encoding: y[i,j] = scale_j * sum_e x[i,e] t[j,e], trits packed 10
 // per 16-bit word in base 3.
@@ -670,7 +676,7 @@ constexpr uint32_t kT3WBuf = kT3M * kT3GU * 4u;        // one group's words
 constexpr uint32_t kT3Cols = 512;                      // D (64 columns) + kT3S A slots of 128
 constexpr int kT3Units = kT3N / 4;                     // activation columns in units of 4
 static_assert(kT3N + 128 * kT3S <= static_cast<int>(kT3Cols), "tensor-memory columns");
-static_assert(2 * kT3GU * 4 >= 2 + 2 * (kT3G * kT3K / 10 + 1) + 2, "a group's window fits its units");
+static_assert(kT3GU * 4 >= 2 + 2 * (kT3G * kT3K / 10 + 1), "a group's words (from a 2-byte offset) fit its units");
 
 // the 32 bf16 pairs of 64 trits starting at phase PH of word 0 (F[i] = word_i * kFix)
 template <int PH>
