@@ -222,3 +222,36 @@ def test_pack_mode_golden_absmean_ties(bnn):
         bnn.bnn_ternary_pack_mode(to_dev_f32(w), 7)
     with pytest.raises(bnn.BnnError):
         bnn.bnn_ternary_pack_mode(to_dev_f32(w), bnn.TERNARY_DELTA, -1.0)
+
+
+def test_auto_one_tile_edge_cases(bnn):
+    """AUTO for 9 <= m <= 64 takes the tensor-memory kernel only when k % 8 == 0,
+    x is 16-byte and the packed words 4-byte aligned: an empty K gives
+    scale * 0, and operands 2 bytes off those alignments take the mma.sync
+    kernel with the same results."""
+    n = 70
+    x0 = torch.empty((20, 0), dtype=torch.bfloat16, device="cuda")
+    p0 = torch.empty((n, 0), dtype=torch.int16, device="cuda")
+    out = bnn.bnn_ternary_gemm(x0, p0, to_dev_f32(np.ones(n, np.float32)), 0)
+    assert torch.all(out == 0)
+
+    m, k = 24, 640
+    rng = np.random.default_rng(41)
+    trits = rng.integers(-1, 2, (n, k)).astype(np.int8)
+    packed = oracle.base3_pack(trits)
+    scale = synth.uniform_f32(41, 1, (n,), 0.25, 2.0)
+    xb = synth.bf16_bits_from_f32(synth.normal_f32(41, 2, (m, k)))
+    ref, mag = oracle.ternary_gemm(xb, packed, scale, m, n, k)
+    # 2-byte offsets: a view one element into a larger buffer
+    pbuf = torch.empty(packed.size + 1, dtype=torch.int16, device="cuda")
+    pbuf[1:] = to_dev_u16(packed).reshape(-1)
+    p_off = pbuf[1:].view(packed.shape)
+    xbuf = torch.empty(xb.size + 1, dtype=torch.int16, device="cuda")
+    xbuf[1:] = to_dev_u16(xb).reshape(-1)
+    x_off = xbuf[1:].view(torch.bfloat16).view(m, k)
+    assert p_off.data_ptr() % 4 == 2 and x_off.data_ptr() % 16 == 2
+    sc = to_dev_f32(scale)
+    for xd, pd, what in ((to_dev_bf16(xb), to_dev_u16(packed), "aligned"), (to_dev_bf16(xb), p_off, "packed +2"),
+                         (x_off, to_dev_u16(packed), "x +2")):
+        out = bnn.bnn_ternary_gemm(xd, pd, sc, k)
+        assert_ternary_close(out.cpu().numpy(), ref, mag, f"AUTO one tile, {what}")
