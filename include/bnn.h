@@ -39,6 +39,19 @@
  *     checks.  Sizes of 0 are valid and return BNN_OK.
  *   - Threads.  Calls are re-entrant; concurrent calls on different streams
  *     are independent.
+ *   - Weights are static data.  The matmul calls (bnn_binary_gemm*,
+ *     bnn_binary_linear, bnn_ternary_gemm*, bnn_ternary_linear,
+ *     bnn_ternary_sparse_gemm) are launched with programmatic dependent
+ *     launch: they may start, and read their WEIGHT operands (packed sign or
+ *     trit rows; the sparse row_ptr and entries), while the kernel before them
+ *     on the stream is still running.  Activations, scales, biases and outputs
+ *     keep plain stream order.  So a weight operand must be complete before
+ *     the stream reaches the matmuls that read it: after preparing it (with
+ *     bnn_pack_signs, bnn_ternary_pack*, bnn_ternary_sparse_encode,
+ *     bnn_tbin_load_ternary or any other kernel), synchronise the stream or
+ *     the device, or prepare it on another stream and make this one wait on
+ *     an event recorded there.  Activations packed or produced right before a
+ *     matmul on the same stream need nothing.
  */
 #ifndef BNN_H
 #define BNN_H

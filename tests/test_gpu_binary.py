@@ -167,8 +167,9 @@ def test_workload_gemv_small_full(bnn):
 @pytest.mark.parametrize("algo", [0, 1, 2, 3])
 def test_workload_gemm_fused_pack(bnn, algo):
     c = synth.gemm_fused_pack(1)
-    xp = bnn.bnn_pack_signs(to_dev_f32(c["x"]))
     wp = bnn.bnn_pack_signs(to_dev_f32(c["w"]))
+    torch.cuda.synchronize()  # weights are complete before a matmul reads them (bnn.h, "Weights are static data")
+    xp = bnn.bnn_pack_signs(to_dev_f32(c["x"]))
     dots, out = bnn.bnn_binary_gemm(xp, wp, to_dev_f32(c["alpha"]), c["k"], algo=algo)
     hx, hw = host_u64(xp), host_u64(wp)
     assert_bits_equal(hx, oracle.pack_signs(c["x"]), "cfg2 x pack")

@@ -95,8 +95,9 @@ def test_two_layer_stack_headline_size(bnn):
     whole packed intermediate against the oracle's pack of layer 1's y."""
     m, n, k = 256, 4096, 4096
     c = synth.gemm_fused_pack(1)
-    x = bnn.bnn_pack_signs(to_dev_f32(c["x"]))
     w1 = bnn.bnn_pack_signs(to_dev_f32(c["w"]))
+    torch.cuda.synchronize()  # weights are complete before a matmul reads them
+    x = bnn.bnn_pack_signs(to_dev_f32(c["x"]))
     w2p = synth.fair_coin_words(11, 2, n, n)
     b1 = synth.normal_f32(11, 5, (n,))
     a2 = synth.uniform_f32(11, 6, (n,), 0.5, 1.5)

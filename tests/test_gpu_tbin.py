@@ -57,6 +57,7 @@ def test_loaded_layer_runs(bnn):
     _, _, (rec,) = bnn.bnn_tbin_parse(data)
     dev = torch.from_numpy(np.frombuffer(data, np.uint8).copy()).cuda()
     packed, sc, bi = bnn.bnn_tbin_load_ternary(dev, rec)
+    torch.cuda.synchronize()  # weights are complete before a matmul reads them
     for m in (1, 64):
         xb = synth.bf16_bits_from_f32(synth.normal_f32(5 + m, 3, (m, k)))
         got = bnn.bnn_ternary_linear(to_dev_bf16(xb), packed, sc, bi)
