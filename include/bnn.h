@@ -274,8 +274,7 @@ int bnn_device_error_count(int reset);
  * tolerance of bnn_ternary_gemm (float32 accumulation in different orders). */
 typedef enum {
   BNN_TALGO_AUTO = 0,        /* what bnn_ternary_gemm uses: CUDA-core GEMV for m <= 8; TC for
-                                9 <= m <= 64 when k % 8 == 0, x is 16-byte and packed 4-byte aligned;
-                                MMA otherwise */
+                                m > 8 when k % 8 == 0 and x is 16-byte aligned; MMA otherwise */
   BNN_TALGO_CUDA_CORES = 1,  /* CUDA-core GEMV kernels (m <= 8 only; BNN_ERR_UNSUPPORTED beyond) */
   BNN_TALGO_MMA = 2,         /* trits decoded to bf16 tiles, bf16 mma.sync m16n8k16 */
   BNN_TALGO_TC = 3           /* trits decoded to bf16, tcgen05.mma kind::f16 accumulating in tensor

@@ -543,9 +543,9 @@ bnn_status ternary_gemm_impl(const uint16_t* x_bf16, const uint16_t* packed, con
     return BNN_ERR_MISALIGNED;
   const int64_t kt = bnn::words10(k);
   if (algo == BNN_TALGO_TC) return bnn::ternary_gemm_tc(x_bf16, packed, scale, bias, m, n, k, out, s);
-  // one activation tile (decode-bound): the kernel that decodes into tensor memory
-  if (algo == BNN_TALGO_AUTO && m > 8 && m <= 64 && k % 8 == 0 && bnn::aligned(x_bf16, 16) &&
-      bnn::aligned(packed, 4))
+  // activations TMA can copy: the tcgen05 kernels (decoding into tensor memory
+  // for one activation tile, into shared memory above that)
+  if (algo == BNN_TALGO_AUTO && m > 8 && k % 8 == 0 && bnn::aligned(x_bf16, 16))
     return bnn::ternary_gemm_tc(x_bf16, packed, scale, bias, m, n, k, out, s);
   if (algo != BNN_TALGO_MMA && m == 1 && kt > 0 && rows_smem_bytes(kt) <= 200 * 1024) {
     const size_t smem = rows_smem_bytes(kt);

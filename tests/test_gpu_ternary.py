@@ -227,8 +227,8 @@ def test_pack_mode_golden_absmean_ties(bnn):
 def test_auto_one_tile_edge_cases(bnn):
     """AUTO for 9 <= m <= 64 takes the tensor-memory kernel only when k % 8 == 0,
     x is 16-byte and the packed words 4-byte aligned: an empty K gives
-    scale * 0, and operands 2 bytes off those alignments take the mma.sync
-    kernel with the same results."""
+    scale * 0, packed words 2 bytes off take the shared-memory tcgen05 kernel
+    and activations 2 bytes off the mma.sync kernel, with the same results."""
     n = 70
     x0 = torch.empty((20, 0), dtype=torch.bfloat16, device="cuda")
     p0 = torch.empty((n, 0), dtype=torch.int16, device="cuda")
