@@ -33,6 +33,21 @@ extern "C" {
 bnn_status bnn_probe_popc(int mode, int64_t blocks, int64_t iters, int32_t* sink, double* ops,
                           cudaStream_t s);
 
+/*
+ * bnn_probe_ternary_plan -- the launch plan bnn_ternary_gemm uses for one
+ * activation tile (1 <= m <= 64, k % 8 == 0, aligned operands: the kernel that
+ * decodes into tensor memory), computed on the host from given occupancy:
+ *   n, k    weight rows and logical reduction length (both >= 1);
+ *   active  host int[4]: how many clusters of 1, 2, 3 and 4 CTAs of that
+ *           kernel fit the GPU at once (0 excludes that cluster size); the
+ *           library itself asks the CUDA occupancy API;
+ *   rows    host out: weight rows per CTA (32, 64, 96 or 128);
+ *   ks      host out: CTAs per cluster splitting the 256-trit stages (1..4).
+ * Host only, no CUDA call; BNN_ERR_INVALID_ARG for bad arguments.  A
+ * diagnostic of this library (no counterpart on the pages).
+ */
+bnn_status bnn_probe_ternary_plan(int64_t n, int64_t k, const int* active, int* rows, int* ks);
+
 #ifdef __cplusplus
 }
 #endif

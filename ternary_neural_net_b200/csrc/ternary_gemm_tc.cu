@@ -1071,6 +1071,33 @@ int ternary_tc_error_count(int reset) {
   return static_cast<int>(v);
 }
 
+// Choose the rows per CTA (32..128) and the cluster split of the stages for
+// the fewest waves times the time of a CTA, in units of a 128-row stage / 128:
+// the decode scales with the rows (not below 64: fewer warps hide less
+// latency), and every CTA pays about two stages of start-up (its first words),
+// plus two for the exchange of a split.  CTAs of a cluster take whole SMs, so
+// few clusters of 3 or 4 run at once.
+void ternary_tmem_plan(int64_t n, int64_t kt, const int active[4], int* rows, int* ks) {
+  const int64_t stages = (10 * kt + kT3K - 1) / kT3K;
+  int best_ks = 1, best_rows = kT3M;
+  int64_t best_cost = INT64_MAX;
+  for (int r = kT3M; r >= 32; r -= 32) {
+    const int64_t tiles = (n + r - 1) / r;
+    for (int c = 1; c <= 4; ++c) {
+      if (active[c - 1] <= 0 || (c > 1 && stages < 2 * c)) continue;
+      const int64_t waves = (tiles + active[c - 1] - 1) / active[c - 1];
+      const int64_t cost = waves * ((r < 64 ? 64 : r) * ((stages + c - 1) / c) + 256 + (c > 1 ? 256 : 32));
+      if (cost < best_cost) {
+        best_cost = cost;
+        best_ks = c;
+        best_rows = r;
+      }
+    }
+  }
+  *rows = best_rows;
+  *ks = best_ks;
+}
+
 bnn_status ternary_gemm_tc(const uint16_t* x_bf16, const uint16_t* packed, const float* scale, const float* bias,
                            int64_t m, int64_t n, int64_t k, float* out, cudaStream_t s) {
   const int64_t kt = words10(k);
@@ -1080,36 +1107,16 @@ bnn_status ternary_gemm_tc(const uint16_t* x_bf16, const uint16_t* packed, const
       encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x_bf16, static_cast<uint64_t>(k), static_cast<uint64_t>(m),
                      static_cast<uint64_t>(k) * 2u, 64, kT2N, CU_TENSOR_MAP_SWIZZLE_128B)) {
     if (m <= kT3N && aligned(packed, 4)) {
-      // one activation tile: decode-bound.  Choose the rows per CTA (32..128)
-      // and the cluster split of the stages for the fewest waves times the
-      // time of a CTA, in units of a 128-row stage / 128: the decode scales with
-      // the rows (not below 64: fewer warps hide less latency), and every CTA
-      // pays about two stages of start-up (its first words), plus two for the
-      // exchange of a split.  CTAs of a cluster take whole SMs, so few clusters
-      // of 3 or 4 run at once.
-      const int64_t stages3 = (10 * kt + kT3K - 1) / kT3K;
-      const int active[5] = {0, tmem_active_clusters<1>(), tmem_active_clusters<2>(), tmem_active_clusters<3>(),
+      // one activation tile: decode-bound
+      const int active[4] = {tmem_active_clusters<1>(), tmem_active_clusters<2>(), tmem_active_clusters<3>(),
                              tmem_active_clusters<4>()};
-      int best_ks = 1, best_rows = kT3M;
-      int64_t best_cost = INT64_MAX;
-      for (int rows = kT3M; rows >= 32; rows -= 32) {
-        const int64_t tiles3 = (n + rows - 1) / rows;
-        for (int ks = 1; ks <= 4; ++ks) {
-          if (active[ks] <= 0 || (ks > 1 && stages3 < 2 * ks)) continue;
-          const int64_t waves = (tiles3 + active[ks] - 1) / active[ks];
-          const int64_t cost = waves * ((rows < 64 ? 64 : rows) * ((stages3 + ks - 1) / ks) + 256 + (ks > 1 ? 256 : 32));
-          if (cost < best_cost) {
-            best_cost = cost;
-            best_ks = ks;
-            best_rows = rows;
-          }
-        }
-      }
-      switch (best_ks) {
-        case 4: return launch_tmem<4>(tx, packed, scale, bias, m, n, kt, best_rows, out, s);
-        case 3: return launch_tmem<3>(tx, packed, scale, bias, m, n, kt, best_rows, out, s);
-        case 2: return launch_tmem<2>(tx, packed, scale, bias, m, n, kt, best_rows, out, s);
-        default: return launch_tmem<1>(tx, packed, scale, bias, m, n, kt, best_rows, out, s);
+      int rows = kT3M, ks = 1;
+      ternary_tmem_plan(n, kt, active, &rows, &ks);
+      switch (ks) {
+        case 4: return launch_tmem<4>(tx, packed, scale, bias, m, n, kt, rows, out, s);
+        case 3: return launch_tmem<3>(tx, packed, scale, bias, m, n, kt, rows, out, s);
+        case 2: return launch_tmem<2>(tx, packed, scale, bias, m, n, kt, rows, out, s);
+        default: return launch_tmem<1>(tx, packed, scale, bias, m, n, kt, rows, out, s);
       }
     }
     const int64_t tiles = ((n + kT2M - 1) / kT2M) * ((m + kT2N - 1) / kT2N);

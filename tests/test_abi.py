@@ -10,12 +10,15 @@ import pytest
 from conftest import ROOT
 
 HEADER = os.path.join(ROOT, "include", "bnn.h")
+HEADERS = [HEADER, os.path.join(ROOT, "include", "bnn_probe.h")]
 
 
-def declared_symbols():
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(bnn_[a-z0-9_]+)\s*\(", text)))
+def declared_symbols(paths=(HEADER,)):
+    names = set()
+    for path in paths:
+        text = re.sub(r"/\*.*?\*/", "", open(path).read(), flags=re.S)
+        names |= set(re.findall(r"\b(bnn_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
 
 
 @pytest.fixture(scope="module")
@@ -33,7 +36,7 @@ def test_header_declares_the_four_calls():
 
 def test_library_exports_every_declared_symbol(bnn):
     lib = C.CDLL(bnn.LIB_PATH)
-    for name in declared_symbols():
+    for name in declared_symbols(HEADERS):
         assert hasattr(lib, name), name
     assert set(bnn.ABI_SYMBOLS) <= set(declared_symbols())
 
@@ -127,3 +130,44 @@ def test_sparse_host_checks(bnn):
     assert lib.bnn_ternary_sparse_gemm(g, g, g, None, None, 1, 1, 10, g, None) == bnn.BNN_ERR_INVALID_ARG
     assert lib.bnn_ternary_sparse_gemm(g, g, g, g, P(0x1002), 1, 1, 10, g, None) == bnn.BNN_ERR_MISALIGNED
     assert lib.bnn_ternary_sparse_gemm(None, None, None, None, None, 0, 4, 10, None, None) == bnn.BNN_OK
+
+
+def _plan(lib, n, k, active):
+    f = lib.bnn_probe_ternary_plan
+    f.argtypes = [C.c_int64, C.c_int64, C.POINTER(C.c_int), C.POINTER(C.c_int), C.POINTER(C.c_int)]
+    f.restype = C.c_int
+    act = (C.c_int * 4)(*active)
+    rows, ks = C.c_int(0), C.c_int(0)
+    st = f(n, k, act, C.byref(rows), C.byref(ks))
+    return st, rows.value, ks.value
+
+
+# clusters of 1..4 CTAs of the tensor-memory kernel that fit a 148-SM B200 at
+# once (cudaOccupancyMaxActiveClusters on that GPU)
+B200_ACTIVE = (148, 74, 45, 33)
+
+
+def test_ternary_plan_cases(bnn):
+    """The plan of the decode-into-tensor-memory ternary kernel: 115 CTAs of
+    96 rows in one wave for the 11008 x 4096 layer (3-CTA clusters would need
+    two waves); small layers split K over clusters; no split without clusters
+    or without enough stages."""
+    lib = bnn.lib()
+    assert _plan(lib, 11008, 4096, B200_ACTIVE) == (bnn.BNN_OK, 96, 1)
+    assert _plan(lib, 300, 4096, B200_ACTIVE) == (bnn.BNN_OK, 64, 4)
+    assert _plan(lib, 385, 1288, B200_ACTIVE) == (bnn.BNN_OK, 64, 3)
+    assert _plan(lib, 300, 4096, (148, 0, 0, 0)) == (bnn.BNN_OK, 64, 1)
+    assert _plan(lib, 129, 8, B200_ACTIVE) == (bnn.BNN_OK, 64, 1)  # one stage: no split
+    assert _plan(lib, 0, 4096, B200_ACTIVE)[0] == bnn.BNN_ERR_INVALID_ARG
+    assert _plan(lib, 10, 0, B200_ACTIVE)[0] == bnn.BNN_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("n", [1, 31, 32, 97, 1000, 4096, 11008, 28672, 100000])
+@pytest.mark.parametrize("k", [8, 640, 4096, 16384])
+def test_ternary_plan_is_valid(bnn, n, k):
+    lib = bnn.lib()
+    st, rows, ks = _plan(lib, n, k, B200_ACTIVE)
+    assert st == bnn.BNN_OK
+    assert rows in (32, 64, 96, 128) and 1 <= ks <= 4
+    stages = -(-10 * (-(-k // 10)) // 256)
+    assert ks == 1 or stages >= 2 * ks  # every CTA of a split keeps at least two stages
