@@ -111,8 +111,9 @@ extern "C" bnn_status bnn_tbin_parse(const uint8_t* file, uint64_t len, uint32_t
       uint64_t elems = 1;
       for (uint8_t d = 0; d < nd; ++d) {
         if (!rdv(file, end, q + 1 + 4ull * d, rec.dims[d])) return BNN_ERR_INVALID_ARG;
+        // the product never exceeds the file's length, so it cannot wrap
+        if (rec.dims[d] != 0 && elems > len / rec.dims[d]) return BNN_ERR_INVALID_ARG;
         elems *= rec.dims[d];
-        if (elems > len) return BNN_ERR_INVALID_ARG;
       }
       q += 1 + 4ull * nd;
       if (end - q != 2 * elems) return BNN_ERR_INVALID_ARG;

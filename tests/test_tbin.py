@@ -75,3 +75,22 @@ def test_malformed_files_are_rejected(bnn):
     for data in bad:
         with pytest.raises(bnn.BnnError):
             bnn.bnn_tbin_parse(data)
+
+
+def test_raw_record_dims_must_match_its_data(bnn):
+    """A raw record's dims must multiply to its float16 count: a product larger
+    than the file (whatever its wrap-around modulo 2^64) or different from the
+    payload is rejected; a matching one parses."""
+    import struct
+
+    def raw_file(dims, n_data):
+        name = b"t"
+        p = struct.pack("<H", len(name)) + name + struct.pack("<B", len(dims))
+        p += struct.pack("<%dI" % len(dims), *dims) + b"\0\0" * n_data
+        return b"TBN\0" + struct.pack("<III", 2, 1, 0) + struct.pack("<BI", 1, len(p)) + p
+
+    _, _, (rec,) = bnn.bnn_tbin_parse(raw_file([3, 5], 15))
+    assert rec.data_elems == 15 and rec.ndims == 2
+    for dims, n in (([3, 5], 14), ([65536, 65536, 65536, 65536], 0), ([0xFFFFFFFF, 2], 2), ([2 ** 31, 2], 0)):
+        with pytest.raises(bnn.BnnError):
+            bnn.bnn_tbin_parse(raw_file(dims, n))
