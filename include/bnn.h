@@ -235,8 +235,11 @@ bnn_status bnn_ternary_pack_mode(const float* w, int64_t n, int64_t k, int mode,
  *   weights in an array of 8192); larger sizes return BNN_ERR_INVALID_ARG
  *   with nothing written.
  *   Set-up: the first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress, with that device current) and caches it; make
- *   that first call before any stream capture on the device.
+ *   (cudaGetSymbolAddress, with that device current) and caches it for the
+ *   device's current CUDA context; make that first call before any stream
+ *   capture on the device.  After a device reset (a new context) the next
+ *   call looks the address up again, so it too should come before any
+ *   capture.
  *   Sharing: every GPU that loads the library holds the array until the
  *   process exits, and all calls on a device share it.  Each call writes
  *   every slot it reads before reading it, so nothing needs clearing between

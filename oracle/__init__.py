@@ -39,6 +39,7 @@ def _L():
             "oracle_twn_ternarize": ([vp, i64, i64, vp, vp, vp], None),
             "oracle_twn_delta": ([vp, i64], C.c_float),
             "oracle_absmean_ternarize": ([vp, i64, i64, vp, vp, vp], None),
+            "oracle_absmean_apply": ([vp, i64, i64, C.c_float, vp, vp], None),
             "oracle_twn_apply": ([vp, i64, i64, C.c_float, vp, vp], None),
             "oracle_base3_pack": ([vp, i64, i64, vp], None),
             "oracle_base3_unpack": ([vp, i64, i64, vp], i64),
@@ -202,6 +203,16 @@ def absmean_ternarize(w: np.ndarray):
     gamma = np.zeros(1, dtype=np.float32)
     _L().oracle_absmean_ternarize(_p(w), n, k, _p(trits), _p(scale), _p(gamma))
     return trits, scale, np.float32(gamma[0])
+
+
+def absmean_apply(w: np.ndarray, gamma) -> tuple:
+    """Mode 'absmean' at a given gamma (float32): (trits int8 [n,k], scale float32 [n])."""
+    w = _c(w, np.float32)
+    n, k = w.shape
+    trits = np.zeros((n, k), dtype=np.int8)
+    scale = np.zeros(n, dtype=np.float32)
+    _L().oracle_absmean_apply(_p(w), n, k, C.c_float(np.float32(gamma)), _p(trits), _p(scale))
+    return trits, scale
 
 
 def delta_ternarize(w: np.ndarray, threshold) -> tuple:

@@ -198,19 +198,13 @@ void oracle_twn_ternarize(const float* w, int64_t n, int64_t k, int8_t* trits,
 }
 
 // [BME] section 5 "Ternary math" (absmean scale gamma = mean|w|, BitNet
-// b1.58) and [BTE] "Features" (mode absmean): gamma = float32 of mean|W| over
-// the whole tensor (float64 sum), q = w / gamma in float32, trit =
-// RoundClip(q, -1, 1) = clamp(round-half-to-even(q), -1, 1); so |q| > 0.5
-// gives sign(q) and |q| <= 0.5 (ties included) gives 0.  gamma = 0 gives all
-// zero trits.  Scales are the per-row least-squares scales of oracle_twn_apply
-// ([BTE] "Features": per-channel least-squares scaling).
-void oracle_absmean_ternarize(const float* w, int64_t n, int64_t k, int8_t* trits, float* scale,
-                              float* gamma_out) {
-  const int64_t total = n * k;
-  double sum_abs = 0.0;
-  for (int64_t e = 0; e < total; ++e) sum_abs += std::fabs(double(w[e]));
-  const float g = float(total > 0 ? sum_abs / double(total) : 0.0);
-  *gamma_out = g;
+// b1.58) and [BTE] "Features" (mode absmean), the trit rule for a given gamma:
+// q = w / gamma in float32, trit = RoundClip(q, -1, 1) = clamp(round-half-to-
+// even(q), -1, 1); so |q| > 0.5 gives sign(q) and |q| <= 0.5 (ties included)
+// gives 0.  gamma = 0 gives all zero trits.  Scales are the per-row
+// least-squares scales of oracle_twn_apply ([BTE] "Features": per-channel
+// least-squares scaling).
+void oracle_absmean_apply(const float* w, int64_t n, int64_t k, float g, int8_t* trits, float* scale) {
   for (int64_t r = 0; r < n; ++r) {
     double kept = 0.0;
     int64_t nonzero = 0;
@@ -230,6 +224,18 @@ void oracle_absmean_ternarize(const float* w, int64_t n, int64_t k, int8_t* trit
     }
     scale[r] = nonzero > 0 ? float(kept / double(nonzero)) : 0.0f;
   }
+}
+
+// The absmean mode in order: gamma = float32 of mean|W| over the whole tensor
+// (float64 sum in element order, rounded once), then the trit rule above.
+void oracle_absmean_ternarize(const float* w, int64_t n, int64_t k, int8_t* trits, float* scale,
+                              float* gamma_out) {
+  const int64_t total = n * k;
+  double sum_abs = 0.0;
+  for (int64_t e = 0; e < total; ++e) sum_abs += std::fabs(double(w[e]));
+  const float g = float(total > 0 ? sum_abs / double(total) : 0.0);
+  *gamma_out = g;
+  oracle_absmean_apply(w, n, k, g, trits, scale);
 }
 
 // [BTE] "Features": 10 trits per 16-bit word, base 3.  Word j of a row holds

@@ -25,6 +25,7 @@ float oracle_twn_delta(const float* w, int64_t total);
 void oracle_twn_apply(const float* w, int64_t n, int64_t k, float delta, int8_t* trits, float* scale);
 void oracle_twn_ternarize(const float* w, int64_t n, int64_t k, int8_t* trits,
                           float* scale, float* delta);
+void oracle_absmean_apply(const float* w, int64_t n, int64_t k, float gamma, int8_t* trits, float* scale);
 void oracle_absmean_ternarize(const float* w, int64_t n, int64_t k, int8_t* trits, float* scale,
                               float* gamma_out);
 void oracle_base3_pack(const int8_t* trits, int64_t n, int64_t k, uint16_t* packed);

@@ -214,7 +214,10 @@ def bnn_binary_linear(xp: torch.Tensor, wp: torch.Tensor, alpha: torch.Tensor | 
 
 def bnn_ternary_sparse_encode(packed: torch.Tensor, k: int):
     """Base-3 packed [n, ceil(k/10)] -> (row_ptr int64 [n+1], entries int16 [nnz]) of the index +
-    sign sparse form.  Reads the entry count back from the device (one synchronisation)."""
+    sign sparse form.  An offline weight-preparation step: it reads the entry count back from
+    the device between its two kernels, and synchronises the stream again after the encode, so
+    the returned tensors are complete when it returns (the sparse matmul reads its weight
+    operands before waiting for the kernel ahead of it; see "Weights are static data" in bnn.h)."""
     _dev(packed, "packed", torch.int16)
     n = packed.shape[0]
     if packed.shape[1] != trit_words_per_row(k):
@@ -226,6 +229,7 @@ def bnn_ternary_sparse_encode(packed: torch.Tensor, k: int):
     entries = torch.empty((max(nnz, 1),), dtype=torch.int16, device=dev)
     _check(_lib.bnn_ternary_sparse_encode(_ptr(packed), n, k, _ptr(row_ptr), _ptr(entries), _stream(dev)),
            "bnn_ternary_sparse_encode")
+    torch.cuda.current_stream(dev).synchronize()
     return row_ptr, entries[:nnz]
 
 

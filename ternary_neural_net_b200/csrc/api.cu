@@ -17,9 +17,40 @@ bnn_status cuda_fail(cudaError_t e) {
 }
 
 namespace {
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+CtxGetCurrentFn g_ctx_current = nullptr;
+CtxGetIdFn g_ctx_id = nullptr;
+std::once_flag g_ctx_once;
+
+void* driver_entry(const char* name) {
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &fn, cudaEnableDefault, &q) == cudaSuccess && q == cudaDriverEntryPointSuccess)
+    return fn;
+  return nullptr;
+}
+}  // namespace
+
+uint64_t context_id() {
+  std::call_once(g_ctx_once, [] {
+    g_ctx_current = reinterpret_cast<CtxGetCurrentFn>(driver_entry("cuCtxGetCurrent"));
+    g_ctx_id = reinterpret_cast<CtxGetIdFn>(driver_entry("cuCtxGetId"));
+  });
+  if (!g_ctx_current || !g_ctx_id) return 0;
+  CUcontext ctx = nullptr;
+  if (g_ctx_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  unsigned long long id = 0;
+  if (g_ctx_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return static_cast<uint64_t>(id) + 1;
+}
+
+namespace {
+// One entry per (kernel, context): a context created after a device reset
+// starts with default attributes, so it gets an entry of its own.
 struct SmemEntry {
   const void* kernel;
-  int device;
+  uint64_t ctx;
   size_t bytes;
 };
 constexpr int kMaxSmemEntries = 256;
@@ -29,19 +60,22 @@ std::mutex g_smem_mu;
 }  // namespace
 
 cudaError_t ensure_smem_raw(const void* kernel, size_t bytes) {
-  const int dev = current_device();
   std::lock_guard<std::mutex> lock(g_smem_mu);
-  for (int i = 0; i < g_smem_count; ++i)
-    if (g_smem[i].kernel == kernel && g_smem[i].device == dev && g_smem[i].bytes >= bytes) return cudaSuccess;
+  uint64_t ctx = context_id();
+  if (ctx != 0)
+    for (int i = 0; i < g_smem_count; ++i)
+      if (g_smem[i].kernel == kernel && g_smem[i].ctx == ctx && g_smem[i].bytes >= bytes) return cudaSuccess;
   const cudaError_t e =
       cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
   if (e != cudaSuccess) return e;
+  ctx = context_id();  // the call above made the device's context current if it was not yet
+  if (ctx == 0) return cudaSuccess;  // no context id available: set the attribute on every call
   for (int i = 0; i < g_smem_count; ++i)
-    if (g_smem[i].kernel == kernel && g_smem[i].device == dev) {
+    if (g_smem[i].kernel == kernel && g_smem[i].ctx == ctx) {
       g_smem[i].bytes = bytes;
       return cudaSuccess;
     }
-  if (g_smem_count < kMaxSmemEntries) g_smem[g_smem_count++] = SmemEntry{kernel, dev, bytes};
+  if (g_smem_count < kMaxSmemEntries) g_smem[g_smem_count++] = SmemEntry{kernel, ctx, bytes};
   return cudaSuccess;
 }
 

@@ -28,8 +28,14 @@ int sm_count();
 // Current device index (0 if the query fails).
 int current_device();
 
-// Raises a kernel's dynamic shared-memory limit to `bytes` once per kernel,
-// device and process, so that later calls (including calls made while a
+// A unique non-zero id of the calling thread's current CUDA context (driver
+// cuCtxGetId), 0 when there is none or the driver cannot say.  Per-context
+// caches key on it: a device reset destroys the primary context, and the
+// next one gets a new id, so nothing cached for the old one is reused.
+uint64_t context_id();
+
+// Raises a kernel's dynamic shared-memory limit to `bytes` once per kernel
+// and CUDA context, so that later calls (including calls made while a
 // stream is being captured into a CUDA graph) only launch.
 cudaError_t ensure_smem_raw(const void* kernel, size_t bytes);
 

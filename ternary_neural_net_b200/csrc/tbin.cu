@@ -134,10 +134,16 @@ extern "C" bnn_status bnn_tbin_load_ternary(const uint8_t* file_dev, uint64_t le
                                             uint16_t* packed, float* scale, float* bias, cudaStream_t s) {
   if (!file_dev || !rec || rec->kind != 0 || !packed) return BNN_ERR_INVALID_ARG;
   const uint64_t words = rec->weights_words, out_f = rec->out_features;
-  // every byte the kernel reads lies inside the file
-  if (rec->weights_offset > len || 2 * words > len - rec->weights_offset || rec->scales_offset > len ||
-      2 * out_f > len - rec->scales_offset ||
-      (rec->num_biases && (rec->biases_offset > len || 2 * out_f > len - rec->biases_offset)) ||
+  // The record may come from the caller rather than from bnn_tbin_parse, so
+  // nothing in it is trusted: the word count must be the documented output
+  // size, and every byte the kernel reads must lie inside the file.  Counts
+  // are compared against halved byte lengths (never doubled), so no product
+  // can wrap.
+  const uint64_t row_words = (static_cast<uint64_t>(rec->in_features) + 9) / 10;
+  if (words != out_f * row_words) return BNN_ERR_INVALID_ARG;  // out_f, row_words < 2^32: no wrap
+  if (rec->weights_offset > len || words > (len - rec->weights_offset) / 2 || rec->scales_offset > len ||
+      out_f > (len - rec->scales_offset) / 2 ||
+      (rec->num_biases && (rec->biases_offset > len || out_f > (len - rec->biases_offset) / 2)) ||
       (rec->num_biases != 0 && rec->num_biases != out_f))
     return BNN_ERR_INVALID_ARG;
   if (!bnn::aligned(packed, 2) || (scale && !bnn::aligned(scale, 4)) || (bias && !bnn::aligned(bias, 4)))
@@ -154,7 +160,8 @@ extern "C" bnn_status bnn_tbin_load_ternary(const uint8_t* file_dev, uint64_t le
 extern "C" bnn_status bnn_tbin_load_raw(const uint8_t* file_dev, uint64_t len, const bnn_tbin_record* rec,
                                         float* out, cudaStream_t s) {
   if (!file_dev || !rec || rec->kind != 1 || !out) return BNN_ERR_INVALID_ARG;
-  if (rec->data_offset > len || 2 * rec->data_elems > len - rec->data_offset) return BNN_ERR_INVALID_ARG;
+  // a caller-supplied record is not trusted: halve the byte length instead of doubling the count
+  if (rec->data_offset > len || rec->data_elems > (len - rec->data_offset) / 2) return BNN_ERR_INVALID_ARG;
   if (!bnn::aligned(out, 4)) return BNN_ERR_MISALIGNED;
   if (rec->data_elems == 0) return BNN_OK;
   tbin_raw_kernel<<<grid_for(static_cast<int64_t>(rec->data_elems)), 256, 0, s>>>(

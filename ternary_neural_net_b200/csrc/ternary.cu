@@ -610,8 +610,8 @@ extern "C" bnn_status bnn_ternary_gemm(const uint16_t* x_bf16, const uint16_t* p
 // The float64 partial sums of |W| (one per 65536 weights) live in the
 // file-scope array below, which every GPU that loads this library holds
 // until the process exits.  Its host-side name is only a stand-in for the
-// symbol; the device address comes from cudaGetSymbolAddress, looked up once
-// per device (with that device current) on the first call and cached.
+// symbol; the device address comes from cudaGetSymbolAddress, looked up on
+// the first call in each CUDA context (with that device current) and cached.
 // ---------------------------------------------------------------------------
 constexpr int64_t kNoAllocMaxParts = 8192;  // 64 KiB of float64: up to 8192 * 65536 = 2^29 weights
 
@@ -620,22 +620,30 @@ static __device__ __align__(256) double g_twn_noalloc_partials[kNoAllocMaxParts]
 namespace {
 
 constexpr int kNoAllocMaxDevices = 64;
-double* g_noalloc_ptr[kNoAllocMaxDevices] = {nullptr};
+struct NoAllocSlot {
+  uint64_t ctx;  // bnn::context_id() the address was looked up in
+  double* ptr;
+};
+NoAllocSlot g_noalloc[kNoAllocMaxDevices] = {};
 std::mutex g_noalloc_mu;
 
-// Device address of g_twn_noalloc_partials on the current device.
+// Device address of g_twn_noalloc_partials on the current device.  Looked up
+// with cudaGetSymbolAddress on the first call in each CUDA context (with the
+// device current) and cached for that context: after a device reset the
+// context, and so the id, is new, and the address is looked up again.
 bnn_status noalloc_scratch(double** out) {
   int dev = -1;
   BNN_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= kNoAllocMaxDevices) return BNN_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  const uint64_t ctx = bnn::context_id();
+  if (ctx == 0 || g_noalloc[dev].ctx != ctx || !g_noalloc[dev].ptr) {
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_twn_noalloc_partials);
     if (e != cudaSuccess) return bnn::cuda_fail(e);
-    g_noalloc_ptr[dev] = static_cast<double*>(p);
+    g_noalloc[dev] = NoAllocSlot{bnn::context_id(), static_cast<double*>(p)};
   }
-  *out = g_noalloc_ptr[dev];
+  *out = g_noalloc[dev].ptr;
   return BNN_OK;
 }
 

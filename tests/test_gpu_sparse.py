@@ -80,3 +80,25 @@ def test_sparse_layer_full_size(bnn):
     dense = bnn.bnn_ternary_gemm(to_dev_bf16(xb), packed, scale, k)
     assert_ternary_close(dense.cpu().numpy(), want, mag, "dense on the same words")
     assert bnn.device_error_count() == 0
+
+
+def test_sparse_gemm_right_after_encode_with_device_x(bnn):
+    """The natural call sequence with everything already on the device and no
+    copy in between: pack -> encode -> sparse matmul.  The matmul starts early
+    (programmatic dependent launch) and reads row_ptr and entries before its
+    wait, so the binding's encode must return complete weights."""
+    n, k, m = 3000, 4096, 2
+    w = torch.from_numpy(synth.normal_f32(77, 3, (n, k))).cuda()
+    xd = to_dev_bf16(synth.bf16_bits_from_f32(synth.normal_f32(77, 4, (m, k))))
+    torch.cuda.synchronize()
+    packed, scale, _ = bnn.bnn_ternary_pack_mode(w, bnn.TERNARY_DELTA, 1.2)
+    torch.cuda.synchronize()
+    for _ in range(3):
+        row_ptr, ent = bnn.bnn_ternary_sparse_encode(packed, k)
+        got = bnn.bnn_ternary_sparse_gemm(xd, row_ptr, ent, scale)
+        trits, _ = oracle.base3_unpack(packed.cpu().numpy().view(np.uint16), k)
+        rp, en = oracle.sparse_encode(trits)
+        want, mag = oracle.sparse_gemm(xd.view(torch.int16).cpu().numpy().view(np.uint16), rp, en,
+                                       scale.cpu().numpy(), None, m, n, k)
+        assert_ternary_close(got.cpu().numpy(), want, mag, "sparse right after encode")
+        del row_ptr, ent

@@ -2,6 +2,8 @@
 base-3 pack, and the ternary matmul) against the CPU oracle.  Trits/words are
 bit-exact given the same threshold; scales within 1 ulp (float64 sums in a
 different order, rounded once); matmul outputs within 1e-3 of scale*sum|x t|."""
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -179,18 +181,73 @@ def test_workload_ternary_full(bnn, m):
     assert bnn.device_error_count() == 0
 
 
-@pytest.mark.parametrize("n,k", [(7, 4096), (64, 1000), (300, 4096 + 7), (1, 1)])
-def test_pack_mode_absmean_matches_oracle(bnn, n, k):
-    w = synth.normal_f32(n * 3 + k, 7, (n, k))
+def _check_absmean(bnn, w: np.ndarray, what: str):
+    """GPU absmean pack against the oracle.  gamma is the float64 mean of |W|
+    rounded once to float32; the GPU sums in another order, so its gamma may be
+    a neighbouring float32.  Then the trits and scales are compared with the
+    oracle's trit rule run at the GPU's gamma (the same float32 quotient and
+    rounding on both sides), and the number of weights whose trit the two
+    gammas would decide differently is reported."""
     packed, scale, gamma = bnn.bnn_ternary_pack_mode(to_dev_f32(w), bnn.TERNARY_ABSMEAN)
     torch.cuda.synchronize()
-    ot, os_, og = oracle.absmean_ternarize(w)
     gg = np.float32(gamma.cpu().numpy()[0])
-    if gg == og:
-        assert_bits_equal(host_u16(packed), oracle.base3_pack(ot), f"absmean {n}x{k} words")
-        assert _ulp_diff(scale.cpu().numpy(), os_) <= 1
-    else:  # float64 sums in another order rounded to a neighbouring float32
-        assert abs(float(gg) - float(og)) <= 2 * np.spacing(np.float32(og))
+    ot, os_, og = oracle.absmean_ternarize(w)
+    if gg != og:
+        assert abs(float(gg) - float(og)) <= 2 * np.spacing(np.float32(og)), (what, gg, og)
+        ot, os_ = oracle.absmean_apply(w, gg)
+        moved = int((oracle.absmean_apply(w, og)[0] != ot).sum())
+        print(f"{what}: gamma differs (gpu {gg!r}, oracle {og!r}); {moved} trits decided differently")
+    assert_bits_equal(host_u16(packed), oracle.base3_pack(ot), f"{what} words")
+    assert _ulp_diff(scale.cpu().numpy(), os_) <= 1, f"{what} scales"
+    return host_u16(packed), scale.cpu().numpy(), gg
+
+
+@pytest.mark.parametrize("n,k", [(7, 4096), (64, 1000), (300, 4096 + 7), (1, 1), (1000, 777)])
+def test_pack_mode_absmean_matches_oracle(bnn, n, k):
+    w = synth.normal_f32(n * 3 + k, 7, (n, k))
+    _check_absmean(bnn, w, f"absmean {n}x{k}")
+
+
+def test_pack_modes_full_size(bnn):
+    """absmean and delta (F = 0.5 and the 10%-density F = 1.6449) on the
+    11008 x 4096 layer: words bit-exact, scales within 1 ulp."""
+    w = synth.ternary(1, m=1)["w"]
+    gp, _, gg = _check_absmean(bnn, w, "absmean 11008x4096")
+    zero_frac = float((oracle.base3_unpack(gp, w.shape[1])[0] == 0).mean())
+    print(f"absmean 11008x4096: gamma={gg} zero fraction={zero_frac:.4f}")
+    # N(0,1): gamma -> sqrt(2/pi); |w / gamma| <= 0.5 with probability erf(gamma / (2 sqrt 2))
+    assert abs(zero_frac - math.erf(float(gg) / (2 * math.sqrt(2)))) < 2e-3
+    for F in (0.5, 1.6449):
+        packed, scale, thr = bnn.bnn_ternary_pack_mode(to_dev_f32(w), bnn.TERNARY_DELTA, F)
+        torch.cuda.synchronize()
+        ot, os_ = oracle.delta_ternarize(w, np.float32(F))
+        assert float(thr.cpu()[0]) == np.float32(F)
+        assert_bits_equal(host_u16(packed), oracle.base3_pack(ot), f"delta F={F} 11008x4096 words")
+        assert _ulp_diff(scale.cpu().numpy(), os_) <= 1, f"delta F={F} scales"
+
+
+def test_ternary_m256_full_size_sampled(bnn):
+    """The AUTO route for m > 64 (the tensor-core kernel that decodes into
+    shared memory) at 256 x 11008 x 4096: 4096 sampled outputs plus all of
+    row 0, row 255 and columns 0 and 11007 against the oracle, and a
+    property at every output: |y| <= |scale| * sum |x| (the largest value a
+    row of trits can give)."""
+    c = synth.ternary(1, m=256)
+    n, k = c["n"], c["k"]
+    gp, gs, _ = _check_pack(bnn, c["w"], "cfg5 pack (m=256)")
+    xd = to_dev_bf16(c["x_bf16"])
+    out = bnn.bnn_ternary_gemm(xd, to_dev_u16(gp), to_dev_f32(gs), k).cpu().numpy()
+    assert bnn.device_error_count() == 0
+    rng = np.random.default_rng(256)
+    rows = np.concatenate([rng.integers(0, 256, 4096), np.zeros(n, np.int64), np.full(n, 255),
+                           np.arange(256), np.arange(256)])
+    cols = np.concatenate([rng.integers(0, n, 4096), np.arange(n), np.arange(n), np.zeros(256, np.int64),
+                           np.full(256, n - 1)])
+    ref, mag = oracle.ternary_gemm_sampled(c["x_bf16"], gp, gs, 256, n, k, rows, cols)
+    assert_ternary_close(out[rows, cols], ref, mag, "cfg5 m=256 sampled")
+    xabs = np.abs((c["x_bf16"].astype(np.uint32) << 16).view(np.float32).astype(np.float64))
+    bound = np.abs(gs.astype(np.float64))[None, :] * xabs.sum(axis=1)[:, None]
+    assert np.all(np.isfinite(out)) and np.all(np.abs(out) <= bound * (1 + 1e-3) + 1e-30)
 
 
 @pytest.mark.parametrize("F", [0.0, 0.5, 1.3])

@@ -229,6 +229,58 @@ def test_absmean_and_delta_golden(case):
     assert np.array_equal(s, scales)
 
 
+@pytest.mark.parametrize("case", [c for c in _mode_cases() if c[2] is None], ids=lambda c: c[0])
+def test_absmean_apply_golden(case):
+    """The absmean trit rule at the golden gamma alone (the step the GPU
+    parity test re-runs when the GPU's gamma is a neighbouring float32)."""
+    name, w, _, th_bits, trits, scales = case
+    g = np.array([th_bits], np.uint32).view(np.float32)[0]
+    t, s = oracle.absmean_apply(w, g)
+    assert np.array_equal(t, trits) and np.array_equal(s, scales)
+
+
+@pytest.mark.parametrize("gamma", [0.3, 0.7978846, 1.0, 2.5])
+def test_absmean_apply_is_roundclip_at_any_gamma(gamma):
+    """At a gamma that is not the tensor's own mean, the trits are still
+    numpy's RoundClip of the float32 quotient (np.round: half to even), and
+    the scales the least-squares mean of |w| over the non-zero trits."""
+    w = synth.normal_f32(21, 4, (48, 301))
+    g = np.float32(gamma)
+    w[0, :4] = [g * np.float32(0.5), -g * np.float32(0.5), g * np.float32(1.5), -g * np.float32(2.5)]
+    t, s = oracle.absmean_apply(w, g)
+    want = np.clip(np.round((w / g).astype(np.float32)), -1, 1).astype(np.int8)
+    assert np.array_equal(t, want)
+    kept = np.abs(w.astype(np.float64)) * (t != 0)
+    cnt = (t != 0).sum(axis=1)
+    want_s = np.where(cnt > 0, kept.sum(axis=1) / np.maximum(cnt, 1), 0).astype(np.float32)
+    assert np.array_equal(s, want_s)
+    # a larger gamma can only zero more trits
+    t2, _ = oracle.absmean_apply(w, np.float32(gamma * 1.5))
+    assert np.all((t2 == 0) | (t2 == t)) and (t2 == 0).sum() >= (t == 0).sum()
+
+
+def test_absmean_apply_tells_neighbouring_gammas_apart():
+    """Re-running the trit rule at the GPU's gamma matters: a weight at exactly
+    half of the next float32 above gamma is a tie (trit 0) there and a
+    non-zero trit at gamma itself."""
+    g = np.float32(0.7978846)
+    g_up = np.nextafter(g, np.float32(np.inf))
+    w = np.array([[g_up * np.float32(0.5), -(g_up * np.float32(0.5)), 1.0]], np.float32)
+    t_g, _ = oracle.absmean_apply(w, g)
+    t_up, _ = oracle.absmean_apply(w, g_up)
+    assert t_g.tolist() == [[1, -1, 1]] and t_up.tolist() == [[0, 0, 1]]
+
+
+def test_absmean_ternarize_is_gamma_then_apply():
+    w = synth.normal_f32(22, 4, (17, 555))
+    t, s, g = oracle.absmean_ternarize(w)
+    assert g == np.float32(np.abs(w.astype(np.float64)).mean())
+    t2, s2 = oracle.absmean_apply(w, g)
+    assert np.array_equal(t, t2) and np.array_equal(s, s2)
+    t0, s0 = oracle.absmean_apply(w, np.float32(0))
+    assert not t0.any() and not s0.any()
+
+
 def test_absmean_is_roundclip_of_numpy():
     """The absmean trits equal numpy's own RoundClip (np.round is half-to-even)
     of the float32 quotient, with gamma the float64 mean rounded to float32."""

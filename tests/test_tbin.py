@@ -94,3 +94,38 @@ def test_raw_record_dims_must_match_its_data(bnn):
     for dims, n in (([3, 5], 14), ([65536, 65536, 65536, 65536], 0), ([0xFFFFFFFF, 2], 2), ([2 ** 31, 2], 0)):
         with pytest.raises(bnn.BnnError):
             bnn.bnn_tbin_parse(raw_file(dims, n))
+
+
+def test_loaders_reject_forged_records(bnn):
+    """bnn_tbin_load_ternary / bnn_tbin_load_raw take a record from the caller,
+    so they must not trust it: counts whose doubled byte length wraps modulo
+    2^64, a word count that is not out_features x ceil(in_features / 10) and
+    ranges past the end of the file are rejected on the host, before any CUDA
+    call (the file pointer here is a fake, never dereferenced)."""
+    import ctypes as C
+    lib = bnn.lib()
+    fake = C.c_void_p(0x10000)
+    length = 4096
+
+    def ternary(**kw):
+        r = bnn.TbinRecord()
+        r.kind, r.out_features, r.in_features = 0, 4, 20
+        r.scales_offset, r.weights_offset, r.weights_words = 16, 64, 8
+        for k, v in kw.items():
+            setattr(r, k, v)
+        return lib.bnn_tbin_load_ternary(fake, length, C.byref(r), fake, fake, fake, None)
+
+    two63 = 1 << 63
+    for kw in (dict(weights_words=two63), dict(weights_words=two63 + 8), dict(weights_words=9),
+               dict(out_features=0x80000000, in_features=10, weights_words=0x80000000),
+               dict(weights_offset=length - 8), dict(scales_offset=length - 4), dict(weights_offset=two63),
+               dict(num_biases=4, biases_offset=length - 6), dict(num_biases=3, biases_offset=32)):
+        assert ternary(**kw) == bnn.BNN_ERR_INVALID_ARG, kw
+
+    def raw(elems, off=16):
+        r = bnn.TbinRecord()
+        r.kind, r.data_offset, r.data_elems = 1, off, elems
+        return lib.bnn_tbin_load_raw(fake, length, C.byref(r), fake, None)
+
+    for elems, off in ((two63, 16), (two63 + 4, 16), ((1 << 64) - 1, 16), (2041, 16), (1, length)):
+        assert raw(elems, off) == bnn.BNN_ERR_INVALID_ARG, (elems, off)

@@ -4,8 +4,8 @@ allocator, a setup without stream-ordered memory pools, a loop that cannot
 risk an allocator call).  It keeps its partial sums in a fixed array inside
 libbnn.so; this test calls it through the C ABI and checks it against the
 allocating entry point bnn_ternary_pack on two calls in a row with different
-inputs, with the tolerances the other ternary-pack tests use (words and the
-threshold bit-exact, scales within 1 ulp).  The file sorts last so that a run
+inputs.  Both entry points run the same kernels in the same reduction order,
+so words, scales and the threshold must be bitwise equal.  The file sorts last so that a run
 stopping at the first failure has already run every other test."""
 import ctypes as C
 
@@ -51,7 +51,7 @@ def test_noalloc_matches_allocating_pack_twice(cuda_device):
         torch.cuda.synchronize()
         assert torch.equal(p, want_p)
         assert torch.equal(d, want_d)
-        assert _ulps(s, want_s) <= 1
+        assert torch.equal(s, want_s), f"scales differ by up to {_ulps(s, want_s)} ulp"
 
 
 def test_noalloc_rejects_sizes_beyond_its_array(cuda_device):
