@@ -15,6 +15,7 @@ import ctypes as C
 import numpy as np
 
 from .build import build as _build
+from .build import build_k1 as _build_k1
 
 _lib = None
 
@@ -255,3 +256,37 @@ def ternary_gemm_sampled(x_bf16, packed, scale, m: int, n: int, k: int, rows, co
     _L().oracle_ternary_gemm_sampled(_p(x_bf16), _p(packed), _p(scale), m, n, k, _p(rows), _p(cols),
                                      rows.size, _p(y), _p(mag))
     return y, mag
+
+
+# ----------------------------------------------------------------------------
+# CPU baseline (not the oracle): the pages' binary_gemm_u64 restated, XOR +
+# 64-bit popcount row by row (k1_popcount.cpp).  Checked against the oracle by
+# the tests; timed by the bench on one core and on all cores.
+# ----------------------------------------------------------------------------
+_k1 = None
+
+
+def _K1():
+    global _k1
+    if _k1 is None:
+        lib = C.CDLL(_build_k1())
+        i64, vp = C.c_int64, C.c_void_p
+        lib.k1_binary_gemm.argtypes = [vp, vp, vp, i64, i64, i64, C.c_int, vp, vp]
+        lib.k1_binary_gemm.restype = None
+        lib.k1_threads_used.argtypes = [C.c_int]
+        lib.k1_threads_used.restype = C.c_int
+        _k1 = lib
+    return _k1
+
+
+def k1_binary_gemm(xp, wp, alpha, m: int, n: int, k: int, threads: int = 1):
+    """(dots int32 [m,n], out float32 [m,n]) by XOR + popcount, on `threads` OpenMP threads."""
+    xp, wp, alpha = _c(xp, np.uint64), _c(wp, np.uint64), _c(alpha, np.float32)
+    dots = np.zeros((m, n), dtype=np.int32)
+    out = np.zeros((m, n), dtype=np.float32)
+    _K1().k1_binary_gemm(_p(xp), _p(wp), _p(alpha), m, n, k, int(threads), _p(dots), _p(out))
+    return dots, out
+
+
+def k1_threads_used(threads: int) -> int:
+    return int(_K1().k1_threads_used(int(threads)))
