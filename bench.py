@@ -1,30 +1,40 @@
 #!/usr/bin/env python
 """Benchmark of the packed 1-bit / balanced-ternary matmul on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl bnn|reference] [--workloads all|headline]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl bnn|reference]
+                    [--config 1,2,3,4,5] [--seeds 1,2,3] [--extras sparse,stack,probe]
+                    [--cpu-budget S] [--csv PATH]
 
-Headline (the JSON line's value): binary GEMM with fused activation packing,
-M=256 x K=4096 activations (float32, N(0,1), sign-packed on the device every
-step) against N=4096 x K=4096 packed weights (packed once, before timing) with
-per-channel alpha.  One step = bnn_pack_signs + bnn_binary_gemm (int32 dots and
-float32 scaled outputs); metric = GMAC/s (M*N*K / time).  The step's inputs
-and outputs rotate through enough copies that every step starts with a cold L2
-(copies totalling more than 2x the L2 size).
+Headline (the JSON line's value): the large compute-bound binary GEMM,
+M = N = K = 8192, fair-coin +-1 activations and weights pre-packed to uint64,
+per-channel alpha ~ U(0.5, 1.5); one step = one bnn_binary_gemm call writing
+int32 dots and float32 alpha-scaled outputs; metric = GMAC/s (M*N*K / time).
+Every step reads its own copy of the packed operands (copies totalling more
+than 2x the L2 size, so each step starts cold) and writes 512 MiB of outputs.
 
-The other workloads (batch-1 GEMVs, the 8192^3 GEMM, the ternary layer) are
-reported under "workloads" on the same line; they are measured after the
-headline's timed region.
+Every config of the workload list (1: GEMV 1x1024x1000; 2: sign-pack of
+256x4096 fp32 activations + GEMM 256x4096x4096; 3: FFN GEMV 1x28672x8192 with
+its activation pack; 4: the headline; 5: the balanced-ternary 11008x4096 layer
+at M = 1 and M = 64) also gets a record of its own under "configs" -- GPU
+figures for each seed, the roofline of its dominant kernel, and the CPU
+baselines -- and one CSV row per config and seed (--csv).
+
+CPU baselines (rank 0, N = 1 only; each a bounded sample, --cpu-budget
+seconds): the oracle (the plain unpack-and-sum definition the GPU is checked
+against) and K1 (the pages' row-by-row XOR + 64-bit popcount, restated), each
+on one core and on all host cores.
 
 Under torchrun (N > 1) every rank runs its own independent copy of the
-workload (weak scaling, no data-path collective); the job's time is the max
+headline (weak scaling, no data-path collective); the job's time is the max
 over ranks and value = all ranks' MACs / that time.
 
---impl reference times the CPU oracle (the plain definition the GPU path is
-checked against) on bounded samples of the same workload, on rank 0 only.
+--impl reference times the CPU oracle on bounded samples of the headline
+workload on the host cores (rank 0 only).
 """
 from __future__ import annotations
 
 import argparse
+import csv
 import ctypes as C
 import hashlib
 import json
@@ -33,6 +43,7 @@ import os
 import sys
 import threading
 import time
+from concurrent.futures import ThreadPoolExecutor
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
@@ -45,23 +56,36 @@ from ternary_neural_net_b200 import synth  # noqa: E402
 METRIC = "binary GEMM GMAC/s (M·N·K) and batch-1 GEMV HBM GB/s vs B200 peak"
 L2_BYTES = 126 * 1024 * 1024
 POPC32_PER_CLK_PER_SM = 16  # 32-bit population counts per clock per SM (integer pipe)
+HBM_SPEC_GBS = 8000.0       # B200 HBM3e specification (~8 TB/s)
+HEADLINE = ("binary GEMM M=N=K=8192: fair-coin +-1 activations and weights pre-packed to uint64, per-channel "
+            "alpha ~ U(0.5,1.5); int32 dots + fp32 alpha-scaled outputs")
 
 
 def log(*a):
     print(*a, file=sys.stderr, flush=True)
 
 
-def parse_args():
+def parse_args(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=2000)
-    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["bnn", "reference"], default="bnn")
-    p.add_argument("--workloads", default="all",
-                   help="all, or a comma list of: headline, gemv_small, gemv_ffn, gemm_large, ternary "
-                        "(without 'headline' no JSON headline is measured: for profiling runs)")
-    p.add_argument("--seed", type=int, default=1)
-    return p.parse_args()
+    p.add_argument("--config", default="1,2,3,4,5",
+                   help="comma list of the configs that get a record of their own (1..5), or 'none'")
+    p.add_argument("--seeds", default="1,2,3", help="seeds the per-config GPU figures are taken for")
+    p.add_argument("--extras", default="sparse,stack,probe",
+                   help="comma list of extra measurements: sparse, stack, probe (or 'none')")
+    p.add_argument("--cpu-budget", type=float, default=2.0,
+                   help="seconds of CPU work per CPU-baseline sample (0 = no CPU baselines)")
+    p.add_argument("--csv", default=None, help="write one CSV row per config and seed to this path")
+    p.add_argument("--no-headline", action="store_true", help="skip the headline (profiling runs)")
+    p.add_argument("--seed", type=int, default=1, help="seed of the headline's inputs")
+    a = p.parse_args(argv)
+    a.configs = [] if a.config == "none" else sorted({int(c) for c in a.config.split(",") if c})
+    a.seed_list = [int(s) for s in a.seeds.split(",") if s]
+    a.extra_set = set() if a.extras == "none" else set(a.extras.split(","))
+    return a
 
 
 # ----------------------------------------------------------------------------
@@ -224,64 +248,42 @@ def rotation_copies(bytes_per_set: int) -> int:
 
 
 # ----------------------------------------------------------------------------
-# the headline: binary GEMM with fused activation packing (M=256, N=K=4096)
+# the headline: binary GEMM M = N = K = 8192 (pre-packed operands)
 # ----------------------------------------------------------------------------
 def run_headline(cu: Cuda, args, dist: Dist):
-    torch = cu.torch
-    dev = cu.device
-    c = synth.gemm_fused_pack(args.seed + dist.rank)
+    torch, dev, lib = cu.torch, cu.device, cu.lib
+    c = synth.gemm_large(args.seed + dist.rank)
     m, n, k = c["m"], c["n"], c["k"]
     kw = synth.words_per_row(k)
-    x_host = torch.from_numpy(c["x"])
-    alpha = torch.from_numpy(c["alpha"]).to(dev)
-    w_dev = torch.from_numpy(c["w"]).to(dev)
-    wp0 = cu.bnn.bnn_pack_signs(w_dev)          # offline weight packing (not timed)
-    del w_dev
-    set_bytes = m * k * 4 + n * kw * 8 + m * kw * 8 + m * n * 8
-    R = rotation_copies(set_bytes)
-    X = [x_host.to(dev) for _ in range(R)]
-    WP = [wp0.clone() for _ in range(R)]
-    XP = [torch.empty((m, kw), dtype=torch.int64, device=dev) for _ in range(R)]
-    D = [torch.empty((m, n), dtype=torch.int32, device=dev) for _ in range(R)]
-    O = [torch.empty((m, n), dtype=torch.float32, device=dev) for _ in range(R)]
-    lib = cu.lib
+    R = rotation_copies((m + n) * kw * 8)
+    xp_h = torch.from_numpy(c["xp"].view(np.int64))
+    wp_h = torch.from_numpy(c["wp"].view(np.int64))
+    XP = [xp_h.to(dev) for _ in range(R)]
+    WP = [wp_h.to(dev) for _ in range(R)]
+    al = torch.from_numpy(c["alpha"]).to(dev)
+    D = [torch.empty((m, n), dtype=torch.int32, device=dev) for _ in range(2)]
+    O = [torch.empty((m, n), dtype=torch.float32, device=dev) for _ in range(2)]
+    torch.cuda.synchronize(dev)     # weights complete before any matmul is enqueued
     cap = torch.cuda.Stream(dev)
     cs = C.c_void_p(cap.cuda_stream)
-    pack_args = [(C.c_void_p(X[r].data_ptr()), m, k, C.c_void_p(XP[r].data_ptr()), cs) for r in range(R)]
-    gemm_args = [(C.c_void_p(XP[r].data_ptr()), C.c_void_p(WP[r].data_ptr()), C.c_void_p(alpha.data_ptr()),
-                  m, n, k, C.c_void_p(D[r].data_ptr()), C.c_void_p(O[r].data_ptr()), cs) for r in range(R)]
+    P = lambda t: C.c_void_p(t.data_ptr())  # noqa: E731
+    gemm_args = [(P(XP[r]), P(WP[r]), P(al), m, n, k, P(D[r % 2]), P(O[r % 2]), cs) for r in range(R)]
 
-    def step(i, ev=None):
-        r = i % R
-        if ev:
-            ev[0].record(cap)
-        st1 = lib.bnn_pack_signs(*pack_args[r])
-        if ev:
-            ev[1].record(cap)
-        st2 = lib.bnn_binary_gemm(*gemm_args[r])
-        if ev:
-            ev[2].record(cap)
-        if st1 or st2:
-            cu.check(st1 or st2, "headline step")
+    def step(i):
+        st = lib.bnn_binary_gemm(*gemm_args[i % R])
+        if st:
+            cu.check(st, "headline step")
 
-    # W eager warm-up steps, then the K timed steps captured once into a CUDA
-    # graph (so host launch overhead cannot leave gaps between kernels).  One
-    # step in EVERY carries external timing events around its two kernels:
-    # event nodes serialise the graph around them, so instrumenting every step
-    # would slow the whole timed region.
     cap.wait_stream(torch.cuda.current_stream(dev))
     with torch.cuda.stream(cap):
         for i in range(args.warmup):
             step(i)
     torch.cuda.synchronize(dev)
     K = args.steps
-    EVERY = 16
-    inst = list(range(0, K, EVERY))
-    evs = {i: [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for i in inst}
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=cap):
         for i in range(K):
-            step(args.warmup + i, evs.get(i))
+            step(args.warmup + i)
     g.replay()                                   # upload the graph (untimed)
     t0, t1 = cu.events(2)
     torch.cuda.synchronize(dev)
@@ -294,36 +296,34 @@ def run_headline(cu: Cuda, args, dist: Dist):
         torch.cuda.synchronize(dev)
     dist.barrier(dev)
     torch.cuda.synchronize(dev)
-    ms_local = t0.elapsed_time(t1)
-    ms = dist.max(ms_local, dev)
-    pack_ms = float(np.mean([evs[i][0].elapsed_time(evs[i][1]) for i in inst]))
-    gemm_ms = float(np.mean([evs[i][1].elapsed_time(evs[i][2]) for i in inst]))
+    ms = dist.max(t0.elapsed_time(t1), dev)
     del g
     macs = float(m) * n * k
-    res = dict(m=m, n=n, k=k, R=R, ms_total=ms, ms_per_step=ms / K, pack_ms=pack_ms, gemm_ms=gemm_ms,
-               macs=macs, clocks=clocks.summary())
-
-    # the same GEMM with the popcount kernel family (for its own roofline)
-    popc_args = [a[:-1] + (C.c_int(1), a[-1]) for a in gemm_args]
-    res["gemm_popc_ms"] = graph_time(cu, lambda i: lib.bnn_binary_gemm_algo(*popc_args[i % R]), 200, cap)
-    tc_args = [a[:-1] + (C.c_int(3), a[-1]) for a in gemm_args]
-    res["gemm_tc_ms"] = graph_time(cu, lambda i: lib.bnn_binary_gemm_algo(*tc_args[i % R]), 200, cap)
-    mma_args = [a[:-1] + (C.c_int(2), a[-1]) for a in gemm_args]
-    res["gemm_mma_ms"] = graph_time(cu, lambda i: lib.bnn_binary_gemm_algo(*mma_args[i % R]), 200, cap)
-    # each kernel alone, back to back in a graph without events in between
-    res["pack_graph_ms"] = graph_time(cu, lambda i: lib.bnn_pack_signs(*pack_args[i % R]), 200, cap)
-    res["gemm_graph_ms"] = graph_time(cu, lambda i: lib.bnn_binary_gemm(*gemm_args[i % R]), 200, cap)
+    res = dict(m=m, n=n, k=k, R=R, ms_total=ms, ms_per_step=ms / K, macs=macs, clocks=clocks.summary(),
+               kernel_ms=ms / K)
+    # per-launch events around a few eager launches (a cross-check of the
+    # graph-averaged kernel time; each launch is one kernel of ~0.6 ms)
+    evs = [cu.events(2) for _ in range(4)]
+    with torch.cuda.stream(cap):
+        for i, (a, b) in enumerate(evs):
+            a.record(cap)
+            step(i)
+            b.record(cap)
+    torch.cuda.synchronize(dev)
+    res["kernel_ms_events"] = float(np.median([a.elapsed_time(b) for a, b in evs]))
+    # the popcount kernel family on the same operands (its own roofline)
+    with ClockSampler(dev.index) as clk:
+        res["popc_ms"] = graph_time(cu, lambda i: lib.bnn_binary_gemm_algo(*gemm_args[i % R][:-1], 1, cs), 3, cap)
+    res["popc_clocks"] = clk.summary()
 
     # end to end through the public API: pinned host activations in, dots and
-    # outputs back to pinned host.  Steps are pipelined over two buffer slots
-    # and three streams (copy in, compute, copy out), so that one step's
-    # host->device copy, another's kernels and a third's device->host copies
-    # overlap (PCIe carries both directions at once); every step still moves
-    # its own inputs in and its own results out.
-    xh = x_host.pin_memory()
+    # outputs back to pinned host, pipelined over two buffer slots and three
+    # streams (copy in / compute / copy out).  Every step moves its own 8 MiB
+    # of packed activations in and its own 512 MiB of results out.
+    xh = xp_h.pin_memory()
     DH = [torch.empty((m, n), dtype=torch.int32).pin_memory() for _ in range(2)]
     OH = [torch.empty((m, n), dtype=torch.float32).pin_memory() for _ in range(2)]
-    Ke = max(3, min(K, 200))
+    Ke = max(3, min(K, 12))
     s_in, s_comp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_comp = [torch.cuda.Event() for _ in range(2)]
@@ -335,14 +335,13 @@ def run_headline(cu: Cuda, args, dist: Dist):
     def e2e_step(i):
         sl = i % 2
         with torch.cuda.stream(s_in):
-            s_in.wait_event(ev_comp[sl])            # step i-2 has packed this slot's activations
-            X[sl].copy_(xh, non_blocking=True)
+            s_in.wait_event(ev_comp[sl])            # step i-2's GEMM has read this slot's activations
+            XP[sl].copy_(xh, non_blocking=True)
             ev_in[sl].record(s_in)
         with torch.cuda.stream(s_comp):
             s_comp.wait_event(ev_in[sl])
             s_comp.wait_event(ev_out[sl])           # step i-2's results have left this slot
-            cu.bnn.bnn_pack_signs(X[sl], out=XP[sl])
-            cu.bnn.bnn_binary_gemm(XP[sl], WP[0], alpha, k, dots=D[sl], out=O[sl])
+            cu.bnn.bnn_binary_gemm(XP[sl], WP[0], al, k, dots=D[sl], out=O[sl])
             ev_comp[sl].record(s_comp)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_comp[sl])
@@ -350,7 +349,7 @@ def run_headline(cu: Cuda, args, dist: Dist):
             OH[sl].copy_(O[sl], non_blocking=True)
             ev_out[sl].record(s_out)
 
-    for i in range(3):
+    for i in range(2):
         e2e_step(i)
     e0, e1 = cu.events(2)
     torch.cuda.synchronize(dev)
@@ -359,17 +358,267 @@ def run_headline(cu: Cuda, args, dist: Dist):
     for st_ in (s_in, s_comp, s_out):
         st_.wait_event(e0)
     for i in range(Ke):
-        e2e_step(3 + i)
+        e2e_step(2 + i)
     for st_ in (s_in, s_comp, s_out):
         cu.stream.wait_stream(st_)
     e1.record(cu.stream)
     torch.cuda.synchronize(dev)
     e2e_ms = dist.max(e0.elapsed_time(e1), dev) / Ke
-    res["e2e"] = dict(ms_per_step=e2e_ms, steps=Ke, h2d=m * k * 4, d2h=m * n * 8,
+    res["e2e"] = dict(ms_per_step=e2e_ms, steps=Ke, h2d=m * kw * 8, d2h=m * n * 8,
                       pipelining="2 buffer slots, 3 streams (copy in / compute / copy out)")
-    for lst in (X, WP, XP, D, O):
+    # the last step's results on the host, checked against the CPU baseline
+    # on a few rows (a consistency check of the measured run, not the parity test)
+    torch.cuda.synchronize(dev)
+    res["host_result"] = (DH[(Ke + 1) % 2], OH[(Ke + 1) % 2])
+    for lst in (XP, WP, D, O):
         lst.clear()
     return res
+
+
+# ----------------------------------------------------------------------------
+# per-config GPU figures
+# ----------------------------------------------------------------------------
+def roofline(bound, achieved, peak, unit, kernel, basis, traffic=None, **extra):
+    d = {"bound": bound, "kernel": kernel, "achieved": achieved, "peak": peak, "unit": unit,
+         "frac": achieved / peak if peak else None, "traffic": traffic, "peak_basis": basis}
+    d.update(extra)
+    return d
+
+
+def check_within(kernel_ms, step_ms, what):
+    """A kernel's time cannot exceed the step it is part of."""
+    if kernel_ms > step_ms * 1.02:
+        raise RuntimeError(f"{what}: kernel time {kernel_ms:.4f} ms exceeds its step's {step_ms:.4f} ms")
+
+
+def gpu_cfg1(cu, seed, P, st, s, pk):
+    torch, dev, lib = cu.torch, cu.device, cu.lib
+    c = synth.gemv_small(seed)
+    n, k = c["n"], c["k"]
+    xp = torch.from_numpy(c["xp"].view(np.int64)).to(dev)
+    wp = torch.from_numpy(c["wp"].view(np.int64)).to(dev)
+    al = torch.from_numpy(c["alpha"]).to(dev)
+    d = torch.empty((1, n), dtype=torch.int32, device=dev)
+    o = torch.empty((1, n), dtype=torch.float32, device=dev)
+    torch.cuda.synchronize(dev)
+    ms_eager = time_calls(cu, lambda i: lib.bnn_binary_gemm(P(xp), P(wp), P(al), 1, n, k, P(d), P(o), cu.s), 2000)
+    ms_graph = graph_time(cu, lambda i: lib.bnn_binary_gemm(P(xp), P(wp), P(al), 1, n, k, P(d), P(o), s), 400, st)
+    alg = n * 16 * 8 + 16 * 8 + n * 4 * 3
+    gbs = alg / (ms_graph * 1e-3) / 1e9
+    return dict(value=ms_graph * 1e3, unit="us per call (graph)", us_eager=ms_eager * 1e3, gbs=gbs,
+                macs=float(n) * k, roofline=roofline(
+                    "hbm", gbs, pk["hbm_gbs"], "GB/s", "binary_gemv_kernel (m = 1)",
+                    f"HBM copy {pk['hbm_gbs']} GB/s ({pk['src']}); 143 KB per call: launch-latency bound",
+                    note="a 2 us call moves 143 KB; the fraction only shows that the call is latency bound"))
+
+
+def gpu_cfg2(cu, seed, P, st, s, pk):
+    torch, dev, lib = cu.torch, cu.device, cu.lib
+    c = synth.gemm_fused_pack(seed)
+    m, n, k = c["m"], c["n"], c["k"]
+    kw = synth.words_per_row(k)
+    w = torch.from_numpy(c["w"]).to(dev)
+    wp0 = cu.bnn.bnn_pack_signs(w)
+    del w
+    R = rotation_copies(m * k * 4 + n * kw * 8 + m * kw * 8 + m * n * 8)
+    x0 = torch.from_numpy(c["x"]).to(dev)
+    X = [x0.clone() for _ in range(R)]
+    WP = [wp0.clone() for _ in range(R)]
+    XP = [torch.empty((m, kw), dtype=torch.int64, device=dev) for _ in range(R)]
+    D = [torch.empty((m, n), dtype=torch.int32, device=dev) for _ in range(R)]
+    O = [torch.empty((m, n), dtype=torch.float32, device=dev) for _ in range(R)]
+    al = torch.from_numpy(c["alpha"]).to(dev)
+    torch.cuda.synchronize(dev)
+
+    def step(i):
+        r = i % R
+        return lib.bnn_pack_signs(P(X[r]), m, k, P(XP[r]), s) or \
+            lib.bnn_binary_gemm(P(XP[r]), P(WP[r]), P(al), m, n, k, P(D[r]), P(O[r]), s)
+    step_ms = graph_time(cu, step, 200, st)
+    gemm_ms = graph_time(cu, lambda i: lib.bnn_binary_gemm(P(XP[i % R]), P(WP[i % R]), P(al), m, n, k, P(D[i % R]),
+                                                           P(O[i % R]), s), 200, st)
+    pack_ms = graph_time(cu, lambda i: lib.bnn_pack_signs(P(X[i % R]), m, k, P(XP[i % R]), s), 200, st)
+    check_within(gemm_ms, step_ms, "config 2 GEMM")
+    macs = float(m) * n * k
+    mma_ms = graph_time(cu, lambda i: lib.bnn_binary_gemm_algo(P(XP[i % R]), P(WP[i % R]), P(al), m, n, k,
+                                                               P(D[i % R]), P(O[i % R]), 2, s), 100, st)
+    popc_ms = graph_time(cu, lambda i: lib.bnn_binary_gemm_algo(P(XP[i % R]), P(WP[i % R]), P(al), m, n, k,
+                                                                P(D[i % R]), P(O[i % R]), 1, s), 50, st)
+    int8 = 2.0 * pk["bf16_tflops"]
+    return dict(value=macs / (step_ms * 1e-3) / 1e9, unit="GMAC/s", us_step=step_ms * 1e3, us_gemm=gemm_ms * 1e3,
+                us_pack=pack_ms * 1e3, us_gemm_mma_s8=mma_ms * 1e3, us_gemm_popc=popc_ms * 1e3, macs=macs,
+                roofline=roofline(
+                    "tensor", 2 * macs / (gemm_ms * 1e-3) / 1e12, int8, "TOP/s",
+                    "binary_gemm_tc_kernel (AUTO for m >= 64): tcgen05.mma kind::i8 into tensor memory",
+                    f"int8 dense = 2 x bf16 {pk['bf16_tflops']} TFLOP/s ({pk['src']}; nominal int8:bf16 = 2)",
+                    traffic_for("binary_gemm_tc_128x2", "ternary_neural_net_b200/csrc/binary_gemm_tc.cu"),
+                    basis="kernel alone, back to back in a CUDA graph (inside the step: pack + GEMM)"),
+                rotation=R)
+
+
+def gpu_cfg3(cu, seed, P, st, s, pk):
+    torch, dev, lib = cu.torch, cu.device, cu.lib
+    c = synth.gemv_ffn(seed)
+    n, k = c["n"], c["k"]
+    kw = synth.words_per_row(k)
+    wp_bytes = n * kw * 8
+    R = rotation_copies(wp_bytes)
+    WP = [torch.from_numpy(c["wp"].view(np.int64)).to(dev)]
+    WP += [WP[0].clone() for _ in range(R - 1)]
+    x = torch.from_numpy(c["x"]).to(dev)
+    xp = torch.empty((1, kw), dtype=torch.int64, device=dev)
+    al = torch.from_numpy(c["alpha"]).to(dev)
+    o = torch.empty((1, n), dtype=torch.float32, device=dev)
+    lib.bnn_pack_signs(P(x), 1, k, P(xp), cu.s)
+    torch.cuda.synchronize(dev)
+    ms_gemv = graph_time(cu, lambda i: lib.bnn_binary_gemm(P(xp), P(WP[i % R]), P(al), 1, n, k, None, P(o), s),
+                         300, st)
+
+    def step(i):
+        return lib.bnn_pack_signs(P(x), 1, k, P(xp), s) or \
+            lib.bnn_binary_gemm(P(xp), P(WP[i % R]), P(al), 1, n, k, None, P(o), s)
+    ms_step = graph_time(cu, step, 300, st)
+    check_within(ms_gemv, ms_step, "config 3 GEMV")
+    alg = wp_bytes + kw * 8 + n * 4 + n * 4
+    gbs = alg / (ms_gemv * 1e-3) / 1e9
+    return dict(value=gbs, unit="GB/s", us_gemv=ms_gemv * 1e3, us_step=ms_step * 1e3,
+                step_gbs=(alg + k * 4 + kw * 8) / (ms_step * 1e-3) / 1e9, macs=float(n) * k,
+                frac_of_spec_8tbs=gbs / HBM_SPEC_GBS,
+                frac_of_read_stream=gbs / pk["read_gbs"] if pk.get("read_gbs") else None,
+                roofline=roofline("hbm", gbs, pk["hbm_gbs"], "GB/s", "binary_gemv_kernel (m = 1)",
+                                  f"HBM copy {pk['hbm_gbs']} GB/s ({pk['src']})",
+                                  traffic_for("binary_gemv", "ternary_neural_net_b200/csrc/binary_gemm.cu")),
+                rotation=R)
+
+
+def gpu_cfg4(cu, seed, P, st, s, pk, head=None):
+    """Seed 1 is the headline's own measurement; other seeds time the kernel in
+    a short graph on their own operands."""
+    torch, dev, lib = cu.torch, cu.device, cu.lib
+    int8 = 2.0 * pk["bf16_tflops"]
+    if head is not None:
+        ms, macs = head["kernel_ms"], head["macs"]
+    else:
+        c = synth.gemm_large(seed)
+        m, n, k = c["m"], c["n"], c["k"]
+        xp = torch.from_numpy(c["xp"].view(np.int64)).to(dev)
+        wp = torch.from_numpy(c["wp"].view(np.int64)).to(dev)
+        al = torch.from_numpy(c["alpha"]).to(dev)
+        d = torch.empty((m, n), dtype=torch.int32, device=dev)
+        o = torch.empty((m, n), dtype=torch.float32, device=dev)
+        torch.cuda.synchronize(dev)
+        ms = graph_time(cu, lambda i: lib.bnn_binary_gemm(P(xp), P(wp), P(al), m, n, k, P(d), P(o), s), 8, st)
+        macs = float(m) * n * k
+        del d, o
+    return dict(value=macs / (ms * 1e-3) / 1e9, unit="GMAC/s", ms_kernel=ms, macs=macs,
+                roofline=roofline("tensor", 2 * macs / (ms * 1e-3) / 1e12, int8, "TOP/s",
+                                  "binary_gemm_tc_kernel (m = 8192: 256-row activation tiles)",
+                                  f"int8 dense = 2 x bf16 {pk['bf16_tflops']} TFLOP/s ({pk['src']})",
+                                  traffic_for("binary_gemm_tc_256x1", "ternary_neural_net_b200/csrc/binary_gemm_tc.cu")))
+
+
+def gpu_cfg5(cu, seed, P, st, s, pk):
+    torch, dev, lib = cu.torch, cu.device, cu.lib
+    c = synth.ternary(seed, m=256)
+    n, k = c["n"], c["k"]
+    kt = synth.trit_words_per_row(k)
+    w = torch.from_numpy(c["w"]).to(dev)
+    packed = torch.empty((n, kt), dtype=torch.int16, device=dev)
+    scale = torch.empty((n,), dtype=torch.float32, device=dev)
+    delta = torch.empty((1,), dtype=torch.float32, device=dev)
+    ms_pack = time_calls(cu, lambda i: lib.bnn_ternary_pack(P(w), n, k, P(packed), P(scale), P(delta), cu.s), 10)
+    ms_pack_na = time_calls(cu, lambda i: lib.bnn_ternary_pack_noalloc(P(w), n, k, P(packed), P(scale), P(delta),
+                                                                        cu.s), 10)
+    ms_modes = {}
+    for mode, name, thr in ((1, "absmean", 0.0), (2, "delta", 0.5)):
+        ms_modes[name] = time_calls(cu, lambda i: lib.bnn_ternary_pack_mode(P(w), n, k, mode, thr, P(packed),
+                                                                            P(scale), P(delta), cu.s), 5, warm=2)
+    lib.bnn_ternary_pack(P(w), n, k, P(packed), P(scale), P(delta), cu.s)   # TWN: what the layer uses
+    del w
+    torch.cuda.synchronize(dev)
+    pbytes = n * kt * 2
+    R = rotation_copies(pbytes)
+    PK = [packed] + [packed.clone() for _ in range(R - 1)]
+    xb = torch.from_numpy(c["x_bf16"].view(np.int16)).to(dev).view(torch.bfloat16)
+    o = torch.empty((256, n), dtype=torch.float32, device=dev)
+    torch.cuda.synchronize(dev)
+
+    def t(m, iters, algo=0):
+        return graph_time(cu, lambda i: lib.bnn_ternary_gemm_algo(P(xb), P(PK[i % R]), P(scale), m, n, k, P(o), algo,
+                                                                  s), iters, st)
+    ms1, ms64, ms256 = t(1, 300), t(64, 100), t(256, 30)
+    ms64_mma = t(64, 50, 2)
+    alg1 = pbytes + k * 2 + n * 4 + n * 4
+    gbs1 = alg1 / (ms1 * 1e-3) / 1e9
+    fl64, fl256 = 2.0 * 64 * n * k, 2.0 * 256 * n * k
+    bf16 = pk["bf16_tflops"]
+    return dict(value=gbs1, unit="GB/s (M=1)", us_m1=ms1 * 1e3, us_m64=ms64 * 1e3, us_m256=ms256 * 1e3,
+                us_m64_mma_sync=ms64_mma * 1e3, m64_tflops=fl64 / (ms64 * 1e-3) / 1e12,
+                m256_tflops=fl256 / (ms256 * 1e-3) / 1e12, macs=float(n) * k,
+                pack_ms=ms_pack, pack_noalloc_ms=ms_pack_na, pack_mode_ms=ms_modes,
+                pack_gbs=(2 * n * k * 4 + pbytes) / (ms_pack * 1e-3) / 1e9,
+                roofline=roofline("hbm", gbs1, pk["hbm_gbs"], "GB/s", "ternary GEMV m = 1",
+                                  f"HBM copy {pk['hbm_gbs']} GB/s ({pk['src']})",
+                                  traffic_for("ternary_gemv_rows", "ternary_neural_net_b200/csrc/ternary.cu"),
+                                  frac_of_read_stream=gbs1 / pk["read_gbs"] if pk.get("read_gbs") else None),
+                roofline_m64=roofline("tensor", fl64 / (ms64 * 1e-3) / 1e12, bf16, "TFLOP/s",
+                                      "ternary GEMM m = 64 (tcgen05 kind::f16)",
+                                      f"bf16 dense {bf16} TFLOP/s ({pk['src']})",
+                                      traffic_for("ternary_gemm_tmem_m64",
+                                                  "ternary_neural_net_b200/csrc/ternary_gemm_tc.cu")),
+                rotation=R)
+
+
+GPU_CFG = {1: gpu_cfg1, 2: gpu_cfg2, 3: gpu_cfg3, 4: gpu_cfg4, 5: gpu_cfg5}
+CFG_NAME = {1: "gemv_small_m1_n1024_k1000", 2: "gemm_fused_pack_m256_n4096_k4096", 3: "gemv_ffn_m1_n28672_k8192",
+            4: "gemm_large_m8192_n8192_k8192", 5: "ternary_n11008_k4096"}
+
+
+def read_stream_peak(cu):
+    """Read-only HBM stream rate on this device (bnn_probe_stream_read over a
+    4 GiB buffer, far above the L2 size), best of a few launches."""
+    torch, dev, lib = cu.torch, cu.device, cu.lib
+    nbytes = 4 << 30
+    buf = torch.empty(nbytes // 4, dtype=torch.int32, device=dev)
+    buf.fill_(1)
+    sink = torch.zeros(1, dtype=torch.int32, device=dev)
+    lib.bnn_probe_stream_read.argtypes = [C.c_void_p, C.c_int64, C.c_int64, C.c_void_p, C.c_void_p]
+    lib.bnn_probe_stream_read.restype = C.c_int
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    best = 0.0
+    for blocks in (sms * 4, sms * 8):
+        for _ in range(4):
+            a, b = cu.events(2)
+            a.record(cu.stream)
+            cu.check(lib.bnn_probe_stream_read(C.c_void_p(buf.data_ptr()), nbytes, blocks,
+                                               C.c_void_p(sink.data_ptr()), cu.s), "stream read probe")
+            b.record(cu.stream)
+            torch.cuda.synchronize(dev)
+            best = max(best, nbytes / (a.elapsed_time(b) * 1e-3) / 1e9)
+    del buf
+    return best
+
+
+def run_configs(cu, args, pk, head):
+    torch, dev = cu.torch, cu.device
+    st = torch.cuda.Stream(dev)
+    s = C.c_void_p(st.cuda_stream)
+    P = lambda t: C.c_void_p(t.data_ptr()) if t is not None else None  # noqa: E731
+    out = {}
+    for cfg in args.configs:
+        per_seed = {}
+        for seed in args.seed_list:
+            if cfg == 4:
+                r = gpu_cfg4(cu, seed, P, st, s, pk, head if (head and seed == args.seed) else None)
+            else:
+                r = GPU_CFG[cfg](cu, seed, P, st, s, pk)
+            per_seed[seed] = r
+            torch.cuda.synchronize(dev)
+            torch.cuda.empty_cache()
+        vals = [r["value"] for r in per_seed.values()]
+        out[cfg] = dict(name=CFG_NAME[cfg], seeds=per_seed, value_median=float(np.median(vals)),
+                        value_min=float(min(vals)), value_max=float(max(vals)), unit=per_seed[args.seed_list[0]]["unit"])
+    return out
 
 
 def graph_time(cu: Cuda, fn, iters: int, stream=None) -> float:
@@ -428,9 +677,6 @@ def popc_probe(cu: Cuda, dev):
     return out
 
 
-# ----------------------------------------------------------------------------
-# the other workloads (after the headline's timed region)
-# ----------------------------------------------------------------------------
 def time_calls(cu, fn, iters, warm=3):
     """ms per call of eager launches on the current stream (host launch cost included)."""
     torch = cu.torch
@@ -444,31 +690,6 @@ def time_calls(cu, fn, iters, warm=3):
     b.record(cu.stream)
     torch.cuda.synchronize(cu.device)
     return a.elapsed_time(b) / iters
-
-
-def run_workloads(cu: Cuda, args, peaks, popc_peak_macs):
-    torch, dev, lib = cu.torch, cu.device, cu.lib
-    P = lambda t: C.c_void_p(t.data_ptr()) if t is not None else None  # noqa: E731
-    hbm = peaks["hbm_gbs"]
-    st = torch.cuda.Stream(dev)
-    s = C.c_void_p(st.cuda_stream)
-    out = {}
-
-    want = set(args.workloads.split(",")) if args.workloads != "all" else {"gemv_small", "gemv_ffn", "gemm_large",
-                                                                           "ternary", "stack", "sparse"}
-    if "gemv_small" in want:
-        out.update(wl_gemv_small(cu, args, P, st, s))
-    if "gemv_ffn" in want:
-        out.update(wl_gemv_ffn(cu, args, P, st, s, hbm))
-    if "gemm_large" in want:
-        out.update(wl_gemm_large(cu, args, P, st, s, popc_peak_macs, peaks))
-    if "ternary" in want:
-        out.update(wl_ternary(cu, args, P, st, s, hbm, peaks))
-    if "stack" in want:
-        out.update(wl_stack(cu, args, P, st, s))
-    if "sparse" in want:
-        out.update(wl_sparse(cu, args, P, st, s, hbm))
-    return out
 
 
 def wl_sparse(cu, args, P, st, s, hbm):
@@ -546,212 +767,201 @@ def wl_stack(cu, args, P, st, s):
              "(float32 out); unfused: pack x, GEMM, pack of the float32 layer-1 output, GEMM (no bias)")}
 
 
-def wl_gemv_small(cu, args, P, st, s):
-    torch, dev, lib = cu.torch, cu.device, cu.lib
-    out = {}
-    # 1. GEMV small: M=1, K=1000, N=1024 (launch-latency bound)
-    c = synth.gemv_small(args.seed)
-    xp = torch.from_numpy(c["xp"].view(np.int64)).to(dev)
-    wp = torch.from_numpy(c["wp"].view(np.int64)).to(dev)
-    al = torch.from_numpy(c["alpha"]).to(dev)
-    d = torch.empty((1, c["n"]), dtype=torch.int32, device=dev)
-    o = torch.empty((1, c["n"]), dtype=torch.float32, device=dev)
-    ms_eager = time_calls(cu, lambda i: lib.bnn_binary_gemm(P(xp), P(wp), P(al), 1, c["n"], c["k"], P(d), P(o),
-                                                            cu.s), 2000)
-    ms_graph = graph_time(cu, lambda i: lib.bnn_binary_gemm(P(xp), P(wp), P(al), 1, c["n"], c["k"], P(d), P(o), s),
-                          200, st)
-    bytes1 = c["n"] * 16 * 8 + 16 * 8 + c["n"] * 4 * 3
-    out["gemv_small_m1_n1024_k1000"] = dict(us_per_call_eager=ms_eager * 1e3, us_per_call_graph=ms_graph * 1e3,
-                                            gbs_graph=bytes1 / (ms_graph * 1e-3) / 1e9)
-    return out
-
-
-def wl_gemv_ffn(cu, args, P, st, s, hbm):
-    torch, dev, lib = cu.torch, cu.device, cu.lib
-    out = {}
-
-    # 3. GEMV FFN: M=1, K=8192, N=28672 (HBM-bound weight stream), x packed on device
-    c = synth.gemv_ffn(args.seed)
-    n, k = c["n"], c["k"]
-    kw = synth.words_per_row(k)
-    wp_bytes = n * kw * 8
-    R = rotation_copies(wp_bytes)
-    WP = [torch.from_numpy(c["wp"].view(np.int64)).to(dev)]
-    WP += [WP[0].clone() for _ in range(R - 1)]
-    x = torch.from_numpy(c["x"]).to(dev)
-    xp = torch.empty((1, kw), dtype=torch.int64, device=dev)
-    al = torch.from_numpy(c["alpha"]).to(dev)
-    o = torch.empty((1, n), dtype=torch.float32, device=dev)
-    lib.bnn_pack_signs(P(x), 1, k, P(xp), cu.s)
-    ms_gemv = graph_time(cu, lambda i: lib.bnn_binary_gemm(P(xp), P(WP[i % R]), P(al), 1, n, k, None, P(o), s),
-                         300, st)
-
-    def step3(i):
-        return lib.bnn_pack_signs(P(x), 1, k, P(xp), s) or \
-            lib.bnn_binary_gemm(P(xp), P(WP[i % R]), P(al), 1, n, k, None, P(o), s)
-    ms_step = graph_time(cu, step3, 300, st)
-    alg_kernel = wp_bytes + kw * 8 + n * 4 + n * 4
-    alg_step = alg_kernel + k * 4 + kw * 8
-    out["gemv_ffn_m1_n28672_k8192"] = dict(
-        us_gemv=ms_gemv * 1e3, gemv_gbs=alg_kernel / (ms_gemv * 1e-3) / 1e9,
-        gemv_frac_of_hbm=alg_kernel / (ms_gemv * 1e-3) / 1e9 / hbm,
-        us_step=ms_step * 1e3, step_gbs=alg_step / (ms_step * 1e-3) / 1e9, rotation=R,
-        gemv_traffic_bytes=traffic_for("binary_gemv", "ternary_neural_net_b200/csrc/binary_gemm.cu"))
-    del WP
-    return out
-
-
-def wl_gemm_large(cu, args, P, st, s, popc_peak_macs, peaks):
-    torch, dev, lib = cu.torch, cu.device, cu.lib
-    out = {}
-
-    # 4. GEMM large: M=N=K=8192 pre-packed, both kernel families
-    c = synth.gemm_large(args.seed)
-    m, n, k = c["m"], c["n"], c["k"]
-    xp = torch.from_numpy(c["xp"].view(np.int64)).to(dev)
-    wp = torch.from_numpy(c["wp"].view(np.int64)).to(dev)
-    al = torch.from_numpy(c["alpha"]).to(dev)
-    d = torch.empty((m, n), dtype=torch.int32, device=dev)
-    o = torch.empty((m, n), dtype=torch.float32, device=dev)
-    macs = float(m) * n * k
-    res4 = {}
-    for algo, name in ((3, "tc"), (2, "mma_s8"), (1, "popc")):
-        with ClockSampler(dev.index) as clk:
-            ms = graph_time(cu, lambda i: lib.bnn_binary_gemm_algo(P(xp), P(wp), P(al), m, n, k, P(d), P(o), algo, s),
-                            10 if algo == 2 else 5, st)
-        res4[name] = dict(ms=ms, gmacs=macs / (ms * 1e-3) / 1e9, clocks=clk.summary())
-    res4["popc"]["frac_of_popc_peak"] = res4["popc"]["gmacs"] / 1e3 / popc_peak_macs
-    res4["mma_s8"]["x_popc_peak"] = res4["mma_s8"]["gmacs"] / 1e3 / popc_peak_macs
-    res4["tc"]["x_popc_peak"] = res4["tc"]["gmacs"] / 1e3 / popc_peak_macs
-    int8_peak = 2.0 * peaks["bf16_tflops"]  # TOP/s: nominal int8:bf16 ratio 2 x the measured bf16 rate
-    res4["tc"]["frac_of_int8_peak"] = 2.0 * res4["tc"]["gmacs"] / 1e3 / int8_peak
-    res4["tc"]["traffic_bytes"] = traffic_for("binary_gemm_tc_256x1", "ternary_neural_net_b200/csrc/binary_gemm_tc.cu")
-    out["gemm_large_8192"] = res4
-    del d, o, xp, wp
-    return out
-
-
-def wl_ternary(cu, args, P, st, s, hbm, peaks):
-    torch, dev, lib = cu.torch, cu.device, cu.lib
-    out = {}
-
-    # 5. Ternary: TWN pack of N=11008 x K=4096 (offline), then M=1 and M=64
-    c = synth.ternary(args.seed, m=64)
-    n, k = c["n"], c["k"]
-    kt = synth.trit_words_per_row(k)
-    w = torch.from_numpy(c["w"]).to(dev)
-    packed = torch.empty((n, kt), dtype=torch.int16, device=dev)
-    scale = torch.empty((n,), dtype=torch.float32, device=dev)
-    delta = torch.empty((1,), dtype=torch.float32, device=dev)
-    ms_pack = time_calls(cu, lambda i: lib.bnn_ternary_pack(P(w), n, k, P(packed), P(scale), P(delta), cu.s), 20,
-                         warm=3)
-    lib.bnn_ternary_pack_noalloc.argtypes = [C.c_void_p, C.c_int64, C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p,
-                                             C.c_void_p]
-    ms_pack_na = time_calls(cu, lambda i: lib.bnn_ternary_pack_noalloc(P(w), n, k, P(packed), P(scale), P(delta),
-                                                                        cu.s), 20, warm=3)
-    lib.bnn_ternary_pack_mode.argtypes = [C.c_void_p, C.c_int64, C.c_int64, C.c_int, C.c_float, C.c_void_p,
-                                          C.c_void_p, C.c_void_p, C.c_void_p]
-    ms_modes = {}
-    for mode, name, thr in ((1, "absmean", 0.0), (2, "delta", 0.5)):
-        ms_modes[name] = time_calls(cu, lambda i: lib.bnn_ternary_pack_mode(P(w), n, k, mode, thr, P(packed), P(scale),
-                                                                            P(delta), cu.s), 10, warm=2)
-    # the TWN pack is what the layer below uses
-    lib.bnn_ternary_pack_noalloc(P(w), n, k, P(packed), P(scale), P(delta), cu.s)
-    del w
-    pbytes = n * kt * 2
-    R = rotation_copies(pbytes)
-    PK = [packed] + [packed.clone() for _ in range(R - 1)]
-    xb = torch.from_numpy(c["x_bf16"].view(np.int16)).to(dev).view(torch.bfloat16)
-    o1 = torch.empty((1, n), dtype=torch.float32, device=dev)
-    o64 = torch.empty((64, n), dtype=torch.float32, device=dev)
-    ms1 = graph_time(cu, lambda i: lib.bnn_ternary_gemm(P(xb), P(PK[i % R]), P(scale), 1, n, k, P(o1), s), 300, st)
-    ms64 = graph_time(cu, lambda i: lib.bnn_ternary_gemm(P(xb), P(PK[i % R]), P(scale), 64, n, k, P(o64), s), 100,
-                      st)
-    lib.bnn_ternary_gemm_algo.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int64, C.c_int64, C.c_int64,
-                                          C.c_void_p, C.c_int, C.c_void_p]
-    ms64_alg = {}
-    for algo, name in ((2, "mma"), (3, "tc")):
-        ms64_alg[name] = graph_time(
-            cu, lambda i: lib.bnn_ternary_gemm_algo(P(xb), P(PK[i % R]), P(scale), 64, n, k, P(o64), algo, s), 100, st)
-    alg1 = pbytes + k * 2 + n * 4 + n * 4
-    flops64 = 2.0 * 64 * n * k
-    out["ternary_n11008_k4096"] = dict(
-        pack_ms=ms_pack, pack_noalloc_ms=ms_pack_na, pack_mode_ms=ms_modes, pack_gbs=(2 * n * k * 4 + pbytes) / (ms_pack_na * 1e-3) / 1e9,
-        m1_us=ms1 * 1e3, m1_gbs=alg1 / (ms1 * 1e-3) / 1e9,
-        m1_frac_of_hbm=alg1 / (ms1 * 1e-3) / 1e9 / hbm,
-        m64_us=ms64 * 1e3, m64_tflops=flops64 / (ms64 * 1e-3) / 1e12,
-        m64_us_by_algo={a: v * 1e3 for a, v in ms64_alg.items()},
-        m64_tflops_by_algo={a: flops64 / (v * 1e-3) / 1e12 for a, v in ms64_alg.items()},
-        m64_frac_of_bf16=flops64 / (ms64 * 1e-3) / 1e12 / peaks["bf16_tflops"], rotation=R)
-    return out
-
-
 # ----------------------------------------------------------------------------
-# CPU baseline: the oracle, timed on a bounded sample of the headline workload
+# CPU baselines: the oracle (as it stands) and K1 (the pages' XOR + popcount
+# loop, restated), each on one core and on all host cores, bounded samples
 # ----------------------------------------------------------------------------
-def oracle_sample_rate(seed: int, budget_s: float):
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _timed_units(run_units, total, budget, threads):
+    """Calibrate on one unit, then run as many units as fit `budget` seconds
+    (at least one per thread, at most `total`), split into `threads`
+    contiguous chunks run concurrently (ctypes releases the GIL, so the
+    chunks run on separate cores).  Returns (units, seconds)."""
+    t = time.perf_counter()
+    run_units(0, 1)
+    t1 = max(time.perf_counter() - t, 1e-6)
+    units = int(max(threads, min(total, threads * budget / t1)))
+    units = min(units, total)
+    bounds = [(units * i // threads, units * (i + 1) // threads) for i in range(threads)]
+    t = time.perf_counter()
+    if threads == 1:
+        run_units(0, units)
+    else:
+        with ThreadPoolExecutor(max_workers=threads) as ex:
+            list(ex.map(lambda b: run_units(*b) if b[1] > b[0] else None, bounds))
+    return units, time.perf_counter() - t
+
+
+def cpu_baselines(cfg, budget, cores):
+    """Oracle and K1 rates for one config, GMAC/s, on 1 core and on `cores`.
+    The oracle (single-threaded code) runs on all cores as contiguous chunks of
+    units on a pool of threads; K1 runs each sample as one call that spreads
+    its (row, column) pairs over OpenMP threads."""
     import oracle
-    c = synth.gemm_fused_pack(seed)
+    res = {}
+    k1 = None
+    if cfg == 1:         # unit: one whole 1 x 1024 x 1000 call, repeated
+        c = synth.gemv_small(1)
+        n, k, xp, wp, al = c["n"], c["k"], c["xp"], c["wp"], c["alpha"]
+        total, unit_macs = 1 << 30, float(n) * k
+
+        def orc(a, b):
+            for _ in range(a, b):
+                oracle.binary_gemm(xp, wp, al, 1, n, k)
+
+        def k1(a, b, th):
+            for _ in range(a, b):
+                oracle.k1_binary_gemm(xp, wp, al, 1, n, k, th)
+    elif cfg == 3:       # unit: 256 output channels of the GEMV, with the activation pack
+        c = synth.gemv_ffn(1)
+        n, k, wp, al = c["n"], c["k"], c["wp"], c["alpha"]
+        xp = oracle.pack_signs(c["x"])
+        blk = 256
+        total, unit_macs = n // blk, float(blk) * k
+
+        def orc(a, b):
+            for u in range(a, b):
+                oracle.binary_gemm(oracle.pack_signs(c["x"]), wp[u * blk:(u + 1) * blk], al[u * blk:(u + 1) * blk],
+                                   1, blk, k)
+
+        def k1(a, b, th):
+            oracle.k1_binary_gemm(xp, wp[a * blk:b * blk], al[a * blk:b * blk], 1, (b - a) * blk, k, th)
+    elif cfg in (2, 4):  # unit: one activation row against all weight rows (cfg 2: with its sign-pack)
+        if cfg == 2:
+            c = synth.gemm_fused_pack(1)
+            x, wp = c["x"], oracle.pack_signs(c["w"])
+            xp = oracle.pack_signs(x)
+        else:
+            c = synth.gemm_large(1)
+            x, xp, wp = None, c["xp"], c["wp"]
+        m, n, k, al = c["m"], c["n"], c["k"], c["alpha"]
+        total, unit_macs = m, float(n) * k
+
+        def orc(a, b):
+            oracle.binary_gemm(oracle.pack_signs(x[a:b]) if x is not None else xp[a:b], wp, al, b - a, n, k)
+
+        def k1(a, b, th):
+            oracle.k1_binary_gemm(xp[a:b], wp, al, b - a, n, k, th)
+    else:                # ternary layer: M = 1 GEMV by blocks of 256 weight rows; M = 64 by activation rows
+        c = synth.ternary(1, m=64)
+        n, k = c["n"], c["k"]
+        trits, sc, _ = oracle.twn_ternarize(c["w"])
+        packed = oracle.base3_pack(trits)
+        xb = c["x_bf16"]
+        blk = 256
+        total, unit_macs = n // blk, float(blk) * k
+
+        def orc(a, b):
+            oracle.ternary_gemm(xb[:1], packed[a * blk:b * blk], sc[a * blk:b * blk], 1, (b - a) * blk, k)
+
+        def orc64(a, b):
+            oracle.ternary_gemm(xb[a:b], packed, sc, b - a, n, k)
+        for th, key in ((1, "1core"), (cores, "allcores")):
+            u, dt = _timed_units(orc64, 64, budget, th)
+            res[f"oracle_m64_{key}"] = dict(gmacs=u * float(n) * k / dt / 1e9, units=u, of=64, seconds=dt, threads=th)
+    for th, key in ((1, "1core"), (cores, "allcores")):
+        u, dt = _timed_units(orc, total, budget, th)
+        res[f"oracle_{key}"] = dict(gmacs=u * unit_macs / dt / 1e9, units=u, of=total, seconds=dt, threads=th)
+        if k1 is not None:
+            used = oracle.k1_threads_used(th)
+            t = time.perf_counter()
+            k1(0, 1, used)
+            t1 = max(time.perf_counter() - t, 1e-6)
+            u = int(max(1, min(total, budget / t1)))
+            t = time.perf_counter()
+            k1(0, u, used)
+            dt = time.perf_counter() - t
+            res[f"k1_{key}"] = dict(gmacs=u * unit_macs / dt / 1e9, units=u, of=total, seconds=dt, threads=used)
+    res["unit"] = {1: "one call (1 x 1024 x 1000)", 2: "one activation row: sign-pack + its 4096 x 4096 dots",
+                   3: "256 output channels of the GEMV (with the 8192-element activation pack)",
+                   4: "one activation row against all 8192 weight rows",
+                   5: "256 weight rows of the M = 1 ternary GEMV (bf16 x, base-3 words, float64 sums); "
+                      "m64: one activation row of the M = 64 layer"}[cfg]
+    if cfg in (2, 3):
+        res["k1_note"] = "K1 times the matmul on operands packed beforehand (the pages' kernel takes packed words)"
+    return res
+
+
+def oracle_headline_baseline(budget, cores):
+    """cpu_baseline of the JSON line: the oracle on all host cores over a
+    bounded sample of the headline workload (activation rows of the 8192^3
+    GEMM against all weight rows)."""
+    import oracle
+    c = synth.gemm_large(1)
     m, n, k = c["m"], c["n"], c["k"]
-    wp = oracle.pack_signs(c["w"])
-    rows = 1
-    t = time.perf_counter()
-    xp = oracle.pack_signs(c["x"][:rows])
-    oracle.binary_gemm(xp, wp, c["alpha"], rows, n, k)
-    t1 = time.perf_counter() - t
-    rows = int(max(1, min(m, budget_s / max(t1, 1e-6))))
-    t = time.perf_counter()
-    xp = oracle.pack_signs(c["x"][:rows])
-    oracle.binary_gemm(xp, wp, c["alpha"], rows, n, k)
-    dt = time.perf_counter() - t
-    macs = float(rows) * n * k
-    return dict(value=macs / dt / 1e9, unit="GMAC/s", cores=1, kind="oracle",
-                sample=f"sign-pack of {rows} of {m} activation rows (fp32, K={k}) + unpack-and-sum "
-                       f"binary matmul of those rows against all N={n} packed weight rows "
-                       f"({macs:.3g} MAC, {dt:.1f} s, single thread)")
+
+    def orc(a, b):
+        oracle.binary_gemm(c["xp"][a:b], c["wp"], c["alpha"], b - a, n, k)
+    u, dt = _timed_units(orc, m, budget, cores)
+    macs = u * float(n) * k
+    return dict(value=macs / dt / 1e9, unit="GMAC/s", cores=cores, kind="oracle",
+                sample=f"{u} of the {m} activation rows of the M=N=K=8192 GEMM, each against all {n} weight rows "
+                       f"(unpack-and-sum, int64; {macs:.3g} MAC in {dt:.1f} s on {cores} threads)")
+
+
+def e2e_consistency(head, rows=4):
+    """The last end-to-end step's host results against K1 on a few rows."""
+    import oracle
+    c = synth.gemm_large(1)
+    n, k = c["n"], c["k"]
+    d, o = head["host_result"]
+    d, o = d.numpy(), o.numpy()
+    idx = np.linspace(0, c["m"] - 1, rows).astype(np.int64)
+    kd, ko = oracle.k1_binary_gemm(c["xp"][idx], c["wp"], c["alpha"], rows, n, k, host_cores())
+    return dict(rows=idx.tolist(), dots_equal=bool(np.array_equal(d[idx], kd)),
+                out_equal=bool(np.array_equal(o[idx].view(np.uint32), ko.view(np.uint32))))
 
 
 def run_reference(args, dist: Dist):
     if dist.rank != 0:
         return 0
     import oracle
-    c = synth.gemm_fused_pack(args.seed)
+    c = synth.gemm_large(args.seed)
     m, n, k = c["m"], c["n"], c["k"]
-    wp = oracle.pack_signs(c["w"])
-    # calibrate: one activation row against `cols` weight rows per step, so the
-    # whole --steps/--warmup run stays within about two minutes
+    cores = host_cores()
+    # calibrate: one activation row against `cols` weight rows per thread per
+    # step, so the whole --steps/--warmup run stays within about two minutes
     t = time.perf_counter()
-    xp = oracle.pack_signs(c["x"][:1])
-    oracle.binary_gemm(xp, wp[:256], c["alpha"][:256], 1, 256, k)
+    oracle.binary_gemm(c["xp"][:1], c["wp"][:256], c["alpha"][:256], 1, 256, k)
     per_col = (time.perf_counter() - t) / 256
     budget = 90.0 / max(1, args.steps + args.warmup)
     cols = int(max(1, min(n, budget / max(per_col, 1e-9))))
 
-    def step(i):
-        r = i % m
-        xp = oracle.pack_signs(c["x"][r:r + 1])
-        c0 = (i * cols) % n
-        cc = min(cols, n - c0)
-        oracle.binary_gemm(xp, wp[c0:c0 + cc], c["alpha"][c0:c0 + cc], 1, cc, k)
-        return cc
+    def chunk(r, c0, cc):
+        oracle.binary_gemm(c["xp"][r:r + 1], c["wp"][c0:c0 + cc], c["alpha"][c0:c0 + cc], 1, cc, k)
 
-    for i in range(args.warmup):
-        step(i)
-    t = time.perf_counter()
-    macs = 0.0
-    for i in range(args.steps):
-        macs += step(args.warmup + i) * float(k)
-    dt = time.perf_counter() - t
+    def step(i, ex):
+        jobs = []
+        for t_ in range(cores):
+            r = (i * cores + t_) % m
+            c0 = ((i * cores + t_) * cols) % n
+            jobs.append((r, c0, min(cols, n - c0)))
+        list(ex.map(lambda j: chunk(*j), jobs))
+        return sum(j[2] for j in jobs)
+
+    with ThreadPoolExecutor(max_workers=cores) as ex:
+        for i in range(args.warmup):
+            step(i, ex)
+        t = time.perf_counter()
+        macs = 0.0
+        for i in range(args.steps):
+            macs += step(args.warmup + i, ex) * float(k)
+        dt = time.perf_counter() - t
     value = macs / dt / 1e9
-    sample = (f"per step: sign-pack of 1 activation row (fp32, K={k}) and its unpack-and-sum binary matmul "
-              f"against {cols} of the N={n} weight rows of the M={m} x N={n} x K={k} workload; single thread")
+    sample = (f"per step and per host thread ({cores} threads): one activation row of the M=N=K=8192 workload "
+              f"against {cols} of its {n} weight rows, unpack-and-sum in int64 (the oracle as it stands)")
     line = {
         "metric": METRIC, "value": value, "unit": "GMAC/s", "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": dt * 1e3 / max(1, args.steps), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "u64", "data": "synthetic", "impl": "reference",
-        "config": {"workload": "binary GEMM with fused activation sign-packing, M=256 N=4096 K=4096 "
-                               "(oracle on a bounded sample)", "m": m, "n": n, "k": k},
-        "cpu_baseline": {"value": value, "unit": "GMAC/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "config": {"workload": HEADLINE + " (oracle on a bounded sample)", "m": m, "n": n, "k": k},
+        "cpu_baseline": {"value": value, "unit": "GMAC/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "GMAC/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -759,8 +969,25 @@ def run_reference(args, dist: Dist):
 
 
 # ----------------------------------------------------------------------------
-def main():
-    args = parse_args()
+def write_csv(path, configs, cpu):
+    cols = ["config", "name", "seed", "value", "unit", "roofline_bound", "roofline_achieved", "roofline_peak",
+            "roofline_unit", "roofline_frac", "cpu_oracle_1core_gmacs", "cpu_oracle_allcores_gmacs",
+            "cpu_k1_1core_gmacs", "cpu_k1_allcores_gmacs", "cpu_threads"]
+    with open(path, "w", newline="") as f:
+        wr = csv.writer(f)
+        wr.writerow(cols)
+        for cfg, rec in configs.items():
+            cb = cpu.get(cfg, {}) if cpu else {}
+            for seed, r in rec["seeds"].items():
+                rf = r["roofline"]
+                wr.writerow([cfg, rec["name"], seed, r["value"], r["unit"], rf["bound"], rf["achieved"], rf["peak"],
+                             rf["unit"], rf["frac"], cb.get("oracle_1core", {}).get("gmacs"),
+                             cb.get("oracle_allcores", {}).get("gmacs"), cb.get("k1_1core", {}).get("gmacs"),
+                             cb.get("k1_allcores", {}).get("gmacs"), cb.get("oracle_allcores", {}).get("threads")])
+
+
+def main(argv=None):
+    args = parse_args(argv)
     dist = Dist()
     if args.impl == "reference":
         return run_reference(args, dist)
@@ -772,77 +999,87 @@ def main():
     dist.init("nccl")
     cu = Cuda(torch, dev)
     peaks, peak_src = measured_peaks()
-
+    pk = dict(peaks, src=peak_src)
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    with_headline = args.workloads == "all" or "headline" in args.workloads.split(",")
-    if not with_headline:   # profiling runs of single workloads: no headline line
-        popc_peak_macs = sms * POPC32_PER_CLK_PER_SM * 32 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
-        print(json.dumps({"workloads": run_workloads(cu, args, peaks, popc_peak_macs)}), flush=True)
+    N, K, W = dist.world, args.steps, args.warmup
+    lead = dist.rank == 0 and N == 1
+
+    head = None if args.no_headline else run_headline(cu, args, dist)
+    extras = {}
+    if lead and "probe" in args.extra_set:
+        pk["read_gbs"] = read_stream_peak(cu)
+        extras["popc_probe"] = popc_probe(cu, dev)
+    configs = run_configs(cu, args, pk, head) if lead else {}
+    if lead:
+        st = torch.cuda.Stream(dev)
+        s = C.c_void_p(st.cuda_stream)
+        P = lambda t: C.c_void_p(t.data_ptr()) if t is not None else None  # noqa: E731
+        if "sparse" in args.extra_set:
+            extras.update(wl_sparse(cu, args, P, st, s, pk["hbm_gbs"]))
+        if "stack" in args.extra_set:
+            extras.update(wl_stack(cu, args, P, st, s))
+    torch.cuda.synchronize(dev)
+    cores = host_cores()
+    cpu = {}
+    if lead and args.cpu_budget > 0:
+        for cfg in args.configs:
+            cpu[cfg] = cpu_baselines(cfg, args.cpu_budget, cores)
+    for cfg, rec in configs.items():
+        rec["cpu"] = cpu.get(cfg)
+    if args.csv and lead:
+        write_csv(args.csv, configs, cpu)
+    if head is None:
+        if dist.rank == 0:
+            print(json.dumps({"configs": configs, "extras": extras, "peaks": pk}), flush=True)
         dist.close()
         return 0
-    res = run_headline(cu, args, dist)
-    probe = popc_probe(cu, dev)
-    max_mhz = res["clocks"]["sm_max_mhz"] or peaks.get("sm_max_mhz", 1965.0)
-    popc_peak_macs = sms * POPC32_PER_CLK_PER_SM * 32 * max_mhz * 1e6 / 1e12  # TMAC/s at max clock
-    int8_peak = 2.0 * peaks["bf16_tflops"]                                     # TOP/s (1 MAC = 2 ops)
-    workloads = run_workloads(cu, args, peaks, popc_peak_macs) if args.workloads != "headline" else {}
-    torch.cuda.synchronize(dev)
 
-    K, W, N = args.steps, args.warmup, dist.world
-    ms_step = res["ms_per_step"]
-    value = job_throughput(res["macs"], N, ms_step) / 1e9
-    gemm_achieved = res["macs"] / (res["gemm_ms"] * 1e-3) / 1e12           # TMAC/s
-    popc_achieved = res["macs"] / (res["gemm_popc_ms"] * 1e-3) / 1e12
-    cpu = oracle_sample_rate(args.seed, 10.0) if (dist.rank == 0 and N == 1) else None
-    e2e = res["e2e"]
+    ms_step = head["ms_per_step"]
+    check_within(head["kernel_ms_events"] * 0.98, ms_step, "headline GEMM (event-bracketed launches)")
+    value = job_throughput(head["macs"], N, ms_step) / 1e9
+    int8_peak = 2.0 * peaks["bf16_tflops"]                     # TOP/s (1 MAC = 2 ops)
+    achieved = 2 * head["macs"] / (head["kernel_ms"] * 1e-3) / 1e12
+    max_mhz = head["clocks"]["sm_max_mhz"] or peaks.get("sm_max_mhz", 1965.0)
+    popc_peak = sms * POPC32_PER_CLK_PER_SM * 32 * max_mhz * 1e6 / 1e12   # TMAC/s at the max clock
+    popc_ach = head["macs"] / (head["popc_ms"] * 1e-3) / 1e12
+    e2e = head["e2e"]
+    cpu_line = oracle_headline_baseline(args.cpu_budget * 2, cores) if (lead and args.cpu_budget > 0) else None
     line = {
         "metric": METRIC, "value": value, "unit": "GMAC/s", "n_gpus": N, "steps": K, "warmup": W,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "u64", "data": "synthetic",
-        "config": {"workload": "binary GEMM with fused activation sign-packing: fp32 N(0,1) activations "
-                               "M=256 x K=4096 packed on device each step, packed N=4096 x K=4096 weights, "
-                               "per-channel alpha; int32 dots + fp32 scaled outputs",
-                   "m": res["m"], "n": res["n"], "k": res["k"],
-                   "l2": f"inputs and outputs rotate through {res['R']} copies (> 2x L2) so each step starts cold",
+        "config": {"workload": HEADLINE, "m": head["m"], "n": head["n"], "k": head["k"],
+                   "l2": f"packed operands rotate through {head['R']} copies (> 2x L2) and each step writes "
+                         f"512 MiB of outputs, so every step starts cold",
                    "parallelism": f"replicas x{N} (independent problems per GPU)"},
-        "roofline": {"bound": "tensor", "kernel": "binary_gemm_tc_kernel<128,2,TMA,deep> (bnn_binary_gemm, m >= 64: "
-                                                  "TMA-fed packed chunks -> 0/1 bytes in swizzled smem, tcgen05.mma "
-                                                  "kind::i8 into TMEM, 2-CTA cluster split-K)",
-                     "achieved": 2 * gemm_achieved, "peak": int8_peak, "unit": "TOP/s",
-                     "frac": 2 * gemm_achieved / int8_peak,
-                     "achieved_back_to_back": 2 * res["macs"] / (res["gemm_graph_ms"] * 1e-3) / 1e12,
-                     "achieved_basis": "achieved: CUDA events around the kernel on every 16th step of the timed "
-                                       "graph (includes the event nodes' serialisation); achieved_back_to_back: "
-                                       "a graph of the kernel alone launched back to back",
-                     "traffic": traffic_for("binary_gemm_tc_128x2", "ternary_neural_net_b200/csrc/binary_gemm_tc.cu"),
-                     "peak_basis": f"int8 dense tensor peak = measured bf16 {peaks['bf16_tflops']} TFLOP/s x 2 "
-                                   f"(nominal int8:bf16 ratio 4.5:2.25 PFLOP/s), {peak_src}"},
+        "roofline": {"bound": "tensor",
+                     "kernel": "binary_gemm_tc_kernel (bnn_binary_gemm AUTO, m >= 64): TMA-fed packed chunks -> 0/1 "
+                               "bytes in swizzled smem, tcgen05.mma kind::i8 into tensor memory",
+                     "achieved": achieved, "peak": int8_peak, "unit": "TOP/s", "frac": achieved / int8_peak,
+                     "achieved_basis": "2 ops x M*N*K per launch / the timed region's duration / K (the step is "
+                                       "this one kernel; CUDA events on the launching stream)",
+                     "kernel_ms": head["kernel_ms"], "kernel_ms_events": head["kernel_ms_events"],
+                     "traffic": traffic_for("binary_gemm_tc_256x1", "ternary_neural_net_b200/csrc/binary_gemm_tc.cu"),
+                     "peak_basis": f"int8 dense tensor peak = bf16 {peaks['bf16_tflops']} TFLOP/s x 2 (nominal "
+                                   f"int8:bf16 ratio 4.5:2.25 PFLOP/s), {peak_src} (burst figure: a kernel timed "
+                                   f"alone)"},
         "roofline_popc": {"bound": "alu", "kernel": "binary_gemm_tiled_kernel (bnn_binary_gemm_algo POPC)",
-                          "achieved": popc_achieved, "peak": popc_peak_macs, "unit": "TMAC/s",
-                          "frac": popc_achieved / popc_peak_macs,
-                          "traffic": traffic_for("binary_gemm_tiled_4x4",
-                                                 "ternary_neural_net_b200/csrc/binary_gemm.cu"),
-                          "peak_basis": f"{sms} SMs x {POPC32_PER_CLK_PER_SM} popc32/clk x 32 bit-MAC x {max_mhz} MHz "
-                                        f"(max SM clock); probe measured {probe['popc32']['per_sm_per_clk']:.2f} "
-                                        f"popc32/clk/SM and {probe['word_step']['per_sm_per_clk']:.2f} "
-                                        f"word-steps/clk/SM"},
-        "kernels_ms": {"bnn_pack_signs": res["pack_ms"], "bnn_binary_gemm": res["gemm_ms"],
-                       "bnn_binary_gemm_algo(POPC)": res["gemm_popc_ms"],
-                       "bnn_binary_gemm_algo(TC)": res["gemm_tc_ms"],
-                       "bnn_binary_gemm_algo(MMA_S8)": res["gemm_mma_ms"],
-                       "bnn_pack_signs(graph, alone)": res["pack_graph_ms"],
-                       "bnn_binary_gemm(graph, alone)": res["gemm_graph_ms"]},
-        "cpu_baseline": cpu,
-        "e2e": {"value": N * res["macs"] / (e2e["ms_per_step"] * 1e-3) / 1e9, "unit": "GMAC/s",
+                          "achieved": popc_ach, "peak": popc_peak, "unit": "TMAC/s", "frac": popc_ach / popc_peak,
+                          "ms": head["popc_ms"], "clocks": head["popc_clocks"],
+                          "peak_basis": f"{sms} SMs x {POPC32_PER_CLK_PER_SM} popc32/clk x 32 bit-MACs x {max_mhz} "
+                                        f"MHz (max SM clock)"},
+        "cpu_baseline": cpu_line,
+        "e2e": {"value": N * head["macs"] / (e2e["ms_per_step"] * 1e-3) / 1e9, "unit": "GMAC/s",
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
-                "ms_per_step": e2e["ms_per_step"], "pipelining": e2e["pipelining"]},
-        "gpu_launches": 2 * K,
-        "timing": "K steps captured in one CUDA graph, replayed once untimed to upload, then once between events; "
-                  "every 16th step carries external events around its two kernels (kernels_ms)",
-        "clocks": res["clocks"],
-        "peaks": {"source": peak_src, "hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"]},
-        "popc_probe": probe,
-        "workloads": workloads,
+                "ms_per_step": e2e["ms_per_step"], "pipelining": e2e["pipelining"],
+                "check": e2e_consistency(head) if lead else None},
+        "gpu_launches": K,
+        "timing": "W eager warm-up steps, then K steps captured in one CUDA graph, replayed once untimed and once "
+                  "between CUDA events on the launching stream (barrier + synchronize on both sides)",
+        "clocks": head["clocks"],
+        "peaks": pk,
+        "configs": configs,
+        "extras": extras,
     }
     if dist.rank == 0:
         print(json.dumps(line), flush=True)

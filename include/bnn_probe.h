@@ -1,8 +1,9 @@
 /*
- * bnn_probe.h -- measurement helper exported by libbnn.so next to the four
- * matmul calls of bnn.h.  It is not a step of the method; the bench uses it to
- * measure the integer-pipe rate that the XOR + popcount matmul is bounded by,
- * so the roofline denominator is a number taken on the same device.
+ * bnn_probe.h -- measurement helpers exported by libbnn.so next to the matmul
+ * calls of bnn.h.  They are not steps of the method; the bench uses them to
+ * measure, on the same device, the roofline denominators the kernels are
+ * bounded by: the integer-pipe rate of the XOR + popcount matmul and the
+ * read-only HBM stream rate of the batch-1 GEMVs (which only read weights).
  */
 #ifndef BNN_PROBE_H
 #define BNN_PROBE_H
@@ -32,6 +33,35 @@ extern "C" {
  */
 bnn_status bnn_probe_popc(int mode, int64_t blocks, int64_t iters, int32_t* sink, double* ops,
                           cudaStream_t s);
+
+/*
+ * bnn_probe_stream_read -- enqueue one kernel of `blocks` x 512 threads that
+ * reads `bytes` bytes of `buf` once with 16-byte streaming loads (four in
+ * flight per thread, grid-stride, coalesced) and writes nothing else.
+ *   buf    device, 16-byte aligned; bytes a multiple of 16 (>= 0).
+ *   sink   uint32 [1] device; written only when the fold of the data equals
+ *          a fixed key (so the loads cannot be optimised away).
+ * Time it with events around the call: bytes / time is the read-only HBM
+ * bandwidth when bytes is well above the L2 size.  BNN_ERR_INVALID_ARG /
+ * BNN_ERR_MISALIGNED for bad arguments.  A diagnostic of this library.
+ */
+bnn_status bnn_probe_stream_read(const void* buf, int64_t bytes, int64_t blocks, uint32_t* sink,
+                                 cudaStream_t s);
+
+/*
+ * bnn_probe_wait_limit -- bound, in polls, the main mbarrier waits of the
+ * tensor-core binary GEMM kernel (bnn_binary_gemm for m >= 64,
+ * BNN_ALGO_TC, bnn_binary_linear) launched after this call; 0 restores the
+ * normal bound (2^24 polls).  The final waits for copies and MMAs already in
+ * flight keep the normal bound whatever the setting.  A wait that runs out
+ * makes its CTA skip every store, wait for its copies and MMAs, free its
+ * tensor memory and return; bnn_device_error_count() counts it.  With a
+ * small limit (a few polls) the first waits run out before the first copies
+ * land, which is how a test exercises that path without any GPU fault.
+ * Process-wide, host only; always BNN_OK.  A diagnostic of this library (no
+ * counterpart on the pages).
+ */
+bnn_status bnn_probe_wait_limit(uint32_t polls);
 
 /*
  * bnn_probe_ternary_plan -- the launch plan bnn_ternary_gemm uses for one

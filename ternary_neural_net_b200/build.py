@@ -47,18 +47,37 @@ def _stale() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False, extra=()) -> str:
+    """Compile every stale object (its .cu, or any shared header, newer than
+    it) in parallel, then link the library."""
     if not force and not _stale():
         return LIB
     objdir = os.path.join(ROOT, "_build")
     os.makedirs(objdir, exist_ok=True)
-    objs = []
+    headers = glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h"))
+    newest_header = max((os.path.getmtime(p) for p in headers), default=0.0)
+    jobs, objs = [], []
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
-        cmd = [nvcc(), *NVCC_FLAGS, *extra, "-I", INCLUDE, "-I", CSRC, "-dc" if False else "-c", src, "-o", obj]
+        objs.append(obj)
+        if force or extra or not os.path.exists(obj) or \
+                os.path.getmtime(obj) < max(os.path.getmtime(src), newest_header):
+            jobs.append([nvcc(), *NVCC_FLAGS, *extra, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj])
+
+    def run(cmd):
         if verbose:
             print(" ".join(cmd))
-        subprocess.run(cmd, check=True)
-        objs.append(obj)
+        return subprocess.run(cmd, capture_output=not verbose, text=True)
+
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=max(1, min(len(jobs), os.cpu_count() or 1))) as ex:
+        results = list(ex.map(run, jobs))
+    for cmd, r in zip(jobs, results):
+        if r.returncode != 0:
+            if r.stdout or r.stderr:
+                sys.stderr.write((r.stdout or "") + (r.stderr or ""))
+            raise subprocess.CalledProcessError(r.returncode, cmd)
+        if not verbose and r.stderr and ("warning" in r.stderr or "ptxas" in r.stderr):
+            sys.stderr.write(r.stderr)
     tmp = LIB + ".tmp"
     cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs]
     if verbose:

@@ -1,4 +1,5 @@
-// bnn_probe_popc: integer-pipe rate probe (measurement helper, see bnn_probe.h).
+// Measurement helpers (see bnn_probe.h): the integer-pipe rate probe and a
+// read-only HBM stream.
 #include "bnn_internal.cuh"
 #include "bnn_probe.h"
 
@@ -36,7 +37,39 @@ __global__ void __launch_bounds__(256) probe_popc_kernel(int mode, int64_t iters
   sink[tid] = static_cast<int32_t>(r);
 }
 
+// Read-only stream: every thread keeps four 16-byte streaming loads in flight
+// per step (grid-stride, so consecutive threads read consecutive 16-byte
+// pieces: fully coalesced) and folds them into one register.  The fold is
+// written only when it equals a value no input of the bench produces, so the
+// kernel's DRAM traffic is the buffer's bytes read once.
+__global__ void __launch_bounds__(512) probe_read_kernel(const uint4* __restrict__ p, int64_t n16,
+                                                         uint32_t key, uint32_t* __restrict__ sink) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  uint32_t acc = 0;
+  for (; i + 3 * stride < n16; i += 4 * stride) {
+    const uint4 a = __ldcs(p + i), b = __ldcs(p + i + stride), c = __ldcs(p + i + 2 * stride),
+                d = __ldcs(p + i + 3 * stride);
+    acc ^= (a.x ^ a.y ^ a.z ^ a.w) + (b.x ^ b.y ^ b.z ^ b.w) + (c.x ^ c.y ^ c.z ^ c.w) + (d.x ^ d.y ^ d.z ^ d.w);
+  }
+  for (; i < n16; i += stride) {
+    const uint4 a = __ldcs(p + i);
+    acc ^= a.x ^ a.y ^ a.z ^ a.w;
+  }
+  if (acc == key) sink[0] = acc;
+}
+
 }  // namespace
+
+extern "C" bnn_status bnn_probe_stream_read(const void* buf, int64_t bytes, int64_t blocks, uint32_t* sink,
+                                            cudaStream_t s) {
+  if (!buf || !sink || bytes < 0 || bytes % 16 != 0 || blocks <= 0 || blocks > (1 << 22)) return BNN_ERR_INVALID_ARG;
+  if (!bnn::aligned(buf, 16) || !bnn::aligned(sink, 4)) return BNN_ERR_MISALIGNED;
+  if (bytes == 0) return BNN_OK;
+  probe_read_kernel<<<static_cast<unsigned>(blocks), 512, 0, s>>>(static_cast<const uint4*>(buf), bytes / 16,
+                                                                   0x9E3779B9u, sink);
+  return bnn::check_launch();
+}
 
 extern "C" bnn_status bnn_probe_popc(int mode, int64_t blocks, int64_t iters, int32_t* sink, double* ops,
                                      cudaStream_t s) {
