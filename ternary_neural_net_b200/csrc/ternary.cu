@@ -307,6 +307,188 @@ size_t rows_smem_bytes(int64_t kt) {
 }
 
 // ---------------------------------------------------------------------------
+// Ternary GEMV, m = 1, k <= 4160: activation tables over 4 + 3 + 3 trits.
+//
+// A word's ten trits split into a 4-trit group (digits 0..3, the word mod 81),
+// a 3-trit group (digits 4..6) and a 3-trit group (digits 7..9).  For word
+// position j of the rows, table A_j holds, for each of the 81 digit patterns
+// e of the first group, the partial dot sum_{i<4} x[10j+i] (d_i(e) - 1); B_j
+// and C_j (27 patterns each) the same for the other two groups.  A word then
+// costs three shared-memory loads and three adds: y = scale * sum_j
+// (A_j[e_A] + B_j[e_B] + C_j[e_C]).  The group codes come from two exact
+// multiply-shift divisions (by 81, then by 27; the constants are checked
+// against every word at compile time below).
+//
+// One CTA per SM holds all 135 tables of the row length (135 x ktp floats,
+// ktp = kt rounded up to 32: 218 KiB at k = 4096) and takes a contiguous
+// block of rows.  Work unit = (row, pass): a warp's 32 lanes load 32
+// consecutive 32-bit pairs of words of one row (128 coalesced bytes), so
+// lane l of pass p holds words j = 64p + 2l + t, t = 0, 1.  Tables are stored
+// entry-major with word column sigma(j) = 64p + t L + l (L = the pass's lane
+// count), so for each of the six loads of a unit the 32 lanes read 32
+// consecutive columns: 32 different banks, whatever patterns they decode.
+// Lanes past the row's end decode the all-zero-trit pair, whose entries are 0
+// in every column.  Each unit's lane sums are added by a shuffle tree and
+// stored per (row, pass); the rows' pass sums are added in pass order, so the
+// result does not depend on the launch shape.  Eight units per warp are in
+// flight (their words loaded a group ahead); the first group is loaded
+// before the programmatic-launch wait (weights do not depend on the kernel
+// ahead), the tables are built after it (they depend on x).
+// ---------------------------------------------------------------------------
+constexpr int kLutThreads = 1024;
+constexpr int kLutMaxKt = 416;         // 32-bit pairs of words need kt even; 135 x 416 floats = 219.4 KiB
+constexpr int kLutRowsChunk = 256;     // rows whose pass sums are held at once
+constexpr int kLutMaxPasses = (kLutMaxKt / 2 + 31) / 32;
+constexpr int kLutGroup = 8;           // units per warp in flight
+constexpr uint32_t kDiv81Mul = 25891u, kDiv81Shift = 21;  // floor(w / 81) for w < 3^10
+constexpr uint32_t kDiv27Mul = 607u, kDiv27Shift = 14;    // floor(q / 27) for q < 3^6
+constexpr uint32_t kZeroPair = 29524u | (29524u << 16);   // two all-zero-trit words
+
+constexpr bool lut_divisions_exact() {
+  for (uint32_t w = 0; w < 59049u; ++w)
+    if ((w * kDiv81Mul) >> kDiv81Shift != w / 81u) return false;
+  for (uint32_t q = 0; q < 729u; ++q)
+    if ((q * kDiv27Mul) >> kDiv27Shift != q / 27u) return false;
+  return true;
+}
+static_assert(lut_divisions_exact(), "multiply-shift division constants");
+
+__host__ __device__ constexpr int lut_pitch(int kt) { return (kt + 31) & ~31; }
+
+size_t lut_smem_bytes(int64_t kt) {
+  return static_cast<size_t>(135 * lut_pitch(static_cast<int>(kt)) + kLutRowsChunk * kLutMaxPasses) * sizeof(float);
+}
+
+__device__ __forceinline__ float bf16f(const uint16_t* x, int e, int k) {
+  return e < k ? __uint_as_float(static_cast<uint32_t>(__ldg(x + e)) << 16) : 0.0f;
+}
+
+__global__ void __launch_bounds__(kLutThreads, 1)
+ternary_gemv_lut_kernel(const uint16_t* __restrict__ x, const uint32_t* __restrict__ packed2,
+                        const float* __restrict__ scale, int64_t n, int k, int kt, float* __restrict__ out,
+                        const float* __restrict__ bias) {
+  extern __shared__ float T[];  // [135][ktp] tables, then [kLutRowsChunk][passes] pass sums
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int kWarps = kLutThreads / 32;
+  const int ktp = lut_pitch(kt);
+  const int kt2 = kt >> 1;                       // 32-bit pairs per row
+  const int passes = (kt2 + 31) >> 5;
+  float* psum = T + 135 * ktp;
+  const int64_t r_begin = n * blockIdx.x / gridDim.x, r_end = n * (blockIdx.x + 1) / gridDim.x;
+  bnn::pdl_trigger();
+
+  // word pair of unit u (row r_chunk + u / passes, pass u % passes) for this lane
+  auto fetch = [&](int64_t r_chunk, int units, int u) -> uint32_t {
+    if (u >= units) return kZeroPair;
+    const int rl = u / passes, p = u - rl * passes;
+    const int c = 32 * p + lane;
+    return c < kt2 ? __ldcs(packed2 + (r_chunk + rl) * kt2 + c) : kZeroPair;
+  };
+
+  int64_t r_chunk = r_begin;
+  int units = static_cast<int>((r_end - r_begin < kLutRowsChunk ? r_end - r_begin : kLutRowsChunk) * passes);
+  uint32_t cur[kLutGroup];
+#pragma unroll
+  for (int g = 0; g < kLutGroup; ++g) cur[g] = fetch(r_chunk, units, warp + kWarps * g);
+
+  bnn::pdl_wait();  // x may come from the kernel ahead
+  // Tables.  Task f = part * kt + column: parts 0..8 fill A's entries
+  // 9 part .. 9 part + 8, parts 9..11 B's, 12..14 C's.  Consecutive threads
+  // write consecutive columns of one entry row (distinct banks).
+  for (int f = tid; f < 15 * kt; f += kLutThreads) {
+    const int part = f / kt, c = f - part * kt;
+    const int p = c >> 6, o = c & 63;
+    const int L = kt2 - 32 * p < 32 ? kt2 - 32 * p : 32;
+    const int t = o >= L ? 1 : 0, l = o - t * L;
+    const int j = 64 * p + 2 * l + t;          // the word position stored in column c
+    const int e0 = 10 * j;
+    float lo[9];
+    float hi;
+    int row0;
+    if (part < 9) {                             // A: digits 0, 1 run over e_lo; digits 2, 3 fixed by part
+      const float x0 = bf16f(x, e0, k), x1 = bf16f(x, e0 + 1, k);
+      const float x2 = bf16f(x, e0 + 2, k), x3 = bf16f(x, e0 + 3, k);
+#pragma unroll
+      for (int v = 0; v < 9; ++v) lo[v] = x0 * static_cast<float>(v % 3 - 1) + x1 * static_cast<float>(v / 3 - 1);
+      hi = x2 * static_cast<float>(part % 3 - 1) + x3 * static_cast<float>(part / 3 - 1);
+      row0 = 9 * part;
+    } else {                                    // B (digits 4..6) or C (digits 7..9): last digit fixed by part
+      const int g = part < 12 ? 0 : 1, d = part - 9 - 3 * g;
+      const int b = e0 + 4 + 3 * g;
+      const float x0 = bf16f(x, b, k), x1 = bf16f(x, b + 1, k), x2 = bf16f(x, b + 2, k);
+#pragma unroll
+      for (int v = 0; v < 9; ++v) lo[v] = x0 * static_cast<float>(v % 3 - 1) + x1 * static_cast<float>(v / 3 - 1);
+      hi = x2 * static_cast<float>(d - 1);
+      row0 = 81 + 27 * g + 9 * d;
+    }
+    float* dst = T + row0 * ktp + c;
+#pragma unroll
+    for (int v = 0; v < 9; ++v) dst[v * ktp] = lo[v] + hi;
+  }
+  __syncthreads();
+
+  const uint32_t stride = 4u * static_cast<uint32_t>(ktp);
+  const uint32_t tbase = static_cast<uint32_t>(__cvta_generic_to_shared(T));
+  const uint32_t offB = 81u * stride, offC = 108u * stride;
+  auto lookup = [&](uint32_t w, uint32_t col) -> float {
+    const uint32_t q = (w * kDiv81Mul) >> kDiv81Shift;   // digits 4..9
+    const uint32_t eA = w - 81u * q;                     // digits 0..3
+    const uint32_t eC = (q * kDiv27Mul) >> kDiv27Shift;  // digits 7..9
+    const uint32_t eB = q - 27u * eC;                    // digits 4..6
+    float a, b, c;
+    asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(a) : "r"(col + eA * stride));
+    asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(b) : "r"(col + offB + eB * stride));
+    asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(c) : "r"(col + offC + eC * stride));
+    return (a + b) + c;
+  };
+
+  while (true) {
+    for (int u0 = warp; u0 < units; u0 += kWarps * kLutGroup) {
+      uint32_t nxt[kLutGroup];
+#pragma unroll
+      for (int g = 0; g < kLutGroup; ++g) nxt[g] = fetch(r_chunk, units, u0 + kWarps * (kLutGroup + g));
+      float sum[kLutGroup];
+#pragma unroll
+      for (int g = 0; g < kLutGroup; ++g) {
+        const int u = u0 + kWarps * g;
+        const int p = u % passes;               // warp-uniform
+        const int L = kt2 - 32 * p < 32 ? kt2 - 32 * p : 32;
+        const int l = lane < L ? lane : L - 1;  // lanes past the row end read a valid column (their pair is zero)
+        const uint32_t col0 = tbase + 4u * static_cast<uint32_t>(64 * p + l);
+        const uint32_t col1 = col0 + 4u * static_cast<uint32_t>(L);
+        const uint32_t pr = cur[g];
+        sum[g] = lookup(pr & 0xFFFFu, col0) + lookup(pr >> 16, col1);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+        for (int g = 0; g < kLutGroup; ++g) sum[g] += __shfl_xor_sync(0xffffffffu, sum[g], off);
+      if (lane == 0) {
+#pragma unroll
+        for (int g = 0; g < kLutGroup; ++g)
+          if (u0 + kWarps * g < units) psum[u0 + kWarps * g] = sum[g];
+      }
+#pragma unroll
+      for (int g = 0; g < kLutGroup; ++g) cur[g] = nxt[g];
+    }
+    __syncthreads();  // every unit's pass sum of this chunk is stored
+    const int rows = units / passes;
+    for (int rl = tid; rl < rows; rl += kLutThreads) {
+      float acc = 0.0f;
+      for (int p = 0; p < passes; ++p) acc += psum[rl * passes + p];
+      const int64_t r = r_chunk + rl;
+      out[r] = bias ? __ldg(scale + r) * acc + __ldg(bias + r) : __ldg(scale + r) * acc;
+    }
+    r_chunk += rows;
+    if (r_chunk >= r_end) break;
+    __syncthreads();  // pass sums read before the next chunk overwrites them
+    units = static_cast<int>((r_end - r_chunk < kLutRowsChunk ? r_end - r_chunk : kLutRowsChunk) * passes);
+#pragma unroll
+    for (int g = 0; g < kLutGroup; ++g) cur[g] = fetch(r_chunk, units, warp + kWarps * g);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Ternary GEMM (m > 8): trits decoded to bf16 tiles in shared memory, bf16
 // mma.sync m16n8k16 with fp32 accumulation.
 //
@@ -547,6 +729,16 @@ bnn_status ternary_gemm_impl(const uint16_t* x_bf16, const uint16_t* packed, con
   // for one activation tile, into shared memory above that)
   if (algo == BNN_TALGO_AUTO && m > 8 && k % 8 == 0 && bnn::aligned(x_bf16, 16))
     return bnn::ternary_gemm_tc(x_bf16, packed, scale, bias, m, n, k, out, s);
+  if (algo != BNN_TALGO_MMA && m == 1 && kt > 0 && kt <= kLutMaxKt && kt % 2 == 0 && bnn::aligned(packed, 4)) {
+    const size_t smem = lut_smem_bytes(kt);
+    BNN_TRY(bnn::ensure_smem(ternary_gemv_lut_kernel, smem));
+    const int64_t sms = bnn::sm_count();
+    const int grid = static_cast<int>(n < sms ? n : sms);
+    BNN_TRY(bnn::launch_pdl(ternary_gemv_lut_kernel, dim3(grid), dim3(kLutThreads), smem, s, 1, x_bf16,
+                            reinterpret_cast<const uint32_t*>(packed), scale, n, static_cast<int>(k),
+                            static_cast<int>(kt), out, bias));
+    return bnn::check_launch();
+  }
   if (algo != BNN_TALGO_MMA && m == 1 && kt > 0 && rows_smem_bytes(kt) <= 200 * 1024) {
     const size_t smem = rows_smem_bytes(kt);
     BNN_TRY(bnn::ensure_smem(ternary_gemv_rows_kernel, smem));

@@ -157,6 +157,62 @@ def test_every_base3_word_decodes_row_kernel(bnn):
     _gemm_case(bnn, 1, 60, k, seed=23, trits=trits, algos=(0, 1))
 
 
+def test_every_base3_word_decodes_lut_kernel(bnn):
+    """All 3^10 words in 145 rows of 410 words (k = 4100, even word count: the
+    m = 1 kernel on 4 + 3 + 3-trit activation tables), every code through its
+    decoder, with and without a bias."""
+    k, kt = 4100, 410
+    words = (np.arange(145 * kt) % 59049).astype(np.uint16).reshape(145, kt)
+    trits, bad = oracle.base3_unpack(words, k)
+    assert bad == 0
+    _gemm_case(bnn, 1, 145, k, seed=29, trits=trits, algos=(0,))
+    scale = synth.uniform_f32(29, 1, (145,), 0.25, 2.0)
+    bias = synth.normal_f32(29, 3, (145,))
+    xb = synth.bf16_bits_from_f32(synth.normal_f32(29, 2, (1, k)))
+    ref, mag = oracle.ternary_linear(xb, words, scale, bias, 1, 145, k)
+    out = bnn.bnn_ternary_linear(to_dev_bf16(xb), to_dev_u16(words), to_dev_f32(scale), to_dev_f32(bias), k)
+    assert_ternary_close(out.cpu().numpy(), ref, mag + np.abs(bias.astype(np.float64)), "lut kernel with bias")
+
+
+# m = 1 shapes around the table kernel's limits: word counts from 2 to its
+# maximum 416 (even) with ragged last passes, odd word counts and words 2
+# bytes off 4-byte alignment (other kernels), row blocks larger than one
+# chunk of 256 rows per CTA, fewer rows than SMs, and pad trits in the last word.
+@pytest.mark.parametrize("n,k", [(1, 11), (7, 20), (300, 640), (149, 4160), (1000, 4140), (40000, 100),
+                                 (5000, 4096), (500, 1300), (33, 4161), (64, 1290), (150, 4170)])
+def test_gemv_m1_lut_shapes(bnn, n, k):
+    _gemm_case(bnn, 1, n, k, seed=n + k)
+
+
+def test_gemv_m1_packed_two_bytes_off(bnn):
+    """Packed words 2 bytes off 4-byte alignment take the pair-table kernel,
+    with the same results."""
+    n, k = 300, 4096
+    rng = np.random.default_rng(5)
+    trits = rng.integers(-1, 2, (n, k)).astype(np.int8)
+    packed = oracle.base3_pack(trits)
+    scale = synth.uniform_f32(5, 1, (n,), 0.25, 2.0)
+    xb = synth.bf16_bits_from_f32(synth.normal_f32(5, 2, (1, k)))
+    ref, mag = oracle.ternary_gemm(xb, packed, scale, 1, n, k)
+    pbuf = torch.empty(packed.size + 1, dtype=torch.int16, device="cuda")
+    pbuf[1:] = to_dev_u16(packed).reshape(-1)
+    p_off = pbuf[1:].view(packed.shape)
+    assert p_off.data_ptr() % 4 == 2
+    for pd in (to_dev_u16(packed), p_off):
+        out = bnn.bnn_ternary_gemm(to_dev_bf16(xb), pd, to_dev_f32(scale), k)
+        assert_ternary_close(out.cpu().numpy(), ref, mag, "m = 1, packed alignment")
+
+
+def test_gemv_m1_is_deterministic(bnn):
+    c = synth.ternary(2, m=1)
+    trits = np.random.default_rng(3).integers(-1, 2, (2000, c["k"])).astype(np.int8)
+    pd = to_dev_u16(oracle.base3_pack(trits))
+    xd, sd = to_dev_bf16(c["x_bf16"]), to_dev_f32(np.ones(2000, np.float32))
+    a = bnn.bnn_ternary_gemm(xd, pd, sd, c["k"])
+    b = bnn.bnn_ternary_gemm(xd, pd, sd, c["k"])
+    assert torch.equal(a, b)
+
+
 def test_zero_trits_give_exact_zero(bnn):
     k = 300
     packed = np.full((4, 30), 29524, np.uint16)
