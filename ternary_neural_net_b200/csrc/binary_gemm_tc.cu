@@ -47,11 +47,19 @@
 // (bounded) for the MMAs it issued, frees its tensor memory and returns.
 #include <cooperative_groups.h>
 
+#include <atomic>
+
 #include "bnn_internal.cuh"
+#include "bnn_probe.h"
 #include "tc_common.cuh"
 
 // Bounded waits that ran out in this file's kernels (read by bnn_device_error_count).
 __device__ unsigned int g_bnn_device_errors = 0;
+
+// Polls of the main mbarrier waits of the kernel below (the final drains keep
+// the full bound): 0 = the normal bound; a small value is set only by the
+// diagnostic bnn_probe_wait_limit, so that a test can make the waits run out.
+static std::atomic<uint32_t> g_wait_limit{0};
 
 namespace {
 
@@ -112,7 +120,7 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
                       const uint64_t* __restrict__ xp, const uint64_t* __restrict__ wp,
                       const float* __restrict__ alpha, const float* __restrict__ bias, int64_t m, int64_t n,
                       int k, int kw, int32_t* __restrict__ dots, float* __restrict__ out,
-                      uint32_t* __restrict__ next, int64_t next_w32) {
+                      uint32_t* __restrict__ next, int64_t next_w32, uint32_t wait_limit) {
   using Cfg = TcCfg<BN, TMA, WIDE>;
   constexpr int S = Cfg::S;
   constexpr int P = TMA ? Cfg::P : 1;
@@ -200,7 +208,7 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
       for (int j = 0; j < nst; ++j) {
         const int c = j / kChunkStages, s = j % kChunkStages, pb = c % P;
         if (s == 0 && !bnn::tc::mbar_wait(smem_u32(&chunk_full[pb]), static_cast<uint32_t>((c / P) & 1), &abort_flag,
-                                          &g_bnn_device_errors)) {
+                                          &g_bnn_device_errors, wait_limit)) {
           ok = false;
           break;
         }
@@ -210,7 +218,7 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
         const int b = j % S;
         // refill only after the tensor core has read the previous fill of this buffer
         if (j >= S && !bnn::tc::mbar_wait(smem_u32(&empty_bar[b]), static_cast<uint32_t>((j / S + 1) & 1), &abort_flag,
-                                          &g_bnn_device_errors)) {
+                                          &g_bnn_device_errors, wait_limit)) {
           ok = false;
           break;
         }
@@ -238,7 +246,7 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
           if (j >= nst) break;
           const int b = j % S;
           if (j >= S && !bnn::tc::mbar_wait(smem_u32(&empty_bar[b]), static_cast<uint32_t>((j / S + 1) & 1), &abort_flag,
-                                          &g_bnn_device_errors)) {
+                                          &g_bnn_device_errors, wait_limit)) {
             ok = false;
             break;
           }
@@ -261,7 +269,7 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
     for (int j = 0; j < nst; ++j) {
       const int b = j % S;
       if (!bnn::tc::mbar_wait(smem_u32(&full_bar[b]), static_cast<uint32_t>((j / S) & 1), &abort_flag,
-                              &g_bnn_device_errors))
+                              &g_bnn_device_errors, wait_limit))
         break;
       asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
       const uint64_t ad = sw128_desc(smem_base + b * kStageBytes);
@@ -302,7 +310,7 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
     for (int c = pre; c < nch; ++c) {
       const int pb = c % P;
       if (!bnn::tc::mbar_wait(smem_u32(&chunk_empty[pb]), static_cast<uint32_t>((c / P + 1) & 1), &abort_flag,
-                              &g_bnn_device_errors))
+                              &g_bnn_device_errors, wait_limit))
         break;
       const uint32_t dst = smem_u32(chunks + pb * Cfg::kChunkBytes);
       const uint32_t bar = smem_u32(&chunk_full[pb]);
@@ -487,7 +495,8 @@ bnn_status launch_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha,
                                         dim3(tma ? TcCfg<BN, true, WIDE>::kThreads : TcCfg<BN, false, WIDE>::kThreads),
                                         smem, s,
                                         KS, tw, tx, xp, wp, alpha, bias, m, n, k, kw, dots, out,
-                                        reinterpret_cast<uint32_t*>(next), 2 * bnn::words64(n));
+                                        reinterpret_cast<uint32_t*>(next), 2 * bnn::words64(n),
+                                        g_wait_limit.load() ? g_wait_limit.load() : bnn::tc::kSpinLimit);
   if (e != cudaSuccess) return bnn::cuda_fail(e);
   return bnn::check_launch();
 }
@@ -540,4 +549,9 @@ extern "C" int bnn_device_error_count(int reset) {
   const int t = bnn::ternary_tc_error_count(reset);
   if (t < 0) return -1;
   return static_cast<int>(v) + t;
+}
+
+extern "C" bnn_status bnn_probe_wait_limit(uint32_t polls) {
+  g_wait_limit.store(polls);
+  return BNN_OK;
 }

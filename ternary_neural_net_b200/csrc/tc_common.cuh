@@ -36,11 +36,12 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait; false when it ran out (counted in *errors, abort raised) or
-// when another thread of the CTA raised the abort flag.
+// Bounded wait of at most `limit` polls; false when it ran out (counted in
+// *errors, abort raised) or when another thread of the CTA raised the abort
+// flag.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          unsigned int* errors) {
-  for (uint32_t it = 0; it < kSpinLimit; ++it) {
+                                          unsigned int* errors, uint32_t limit = kSpinLimit) {
+  for (uint32_t it = 0; it < limit; ++it) {
     if (mbar_try(bar, parity)) return true;
     if ((it & 255u) == 255u && *abort_flag) return false;
   }
