@@ -452,7 +452,7 @@ def gpu_cfg2(cu, seed, P, st, s, pk):
                     "binary_gemm_tc_kernel (AUTO for m >= 64): tcgen05.mma kind::i8 into tensor memory",
                     f"int8 dense = 2 x bf16 {pk['bf16_tflops']} TFLOP/s ({pk['src']}; nominal int8:bf16 = 2)",
                     traffic_for("binary_gemm_tc_128x2", "ternary_neural_net_b200/csrc/binary_gemm_tc.cu"),
-                    basis="kernel alone, back to back in a CUDA graph (inside the step: pack + GEMM)"),
+                    achieved_basis="kernel alone, back to back in a CUDA graph (inside the step: pack + GEMM)"),
                 rotation=R)
 
 
@@ -1035,7 +1035,6 @@ def main(argv=None):
         return 0
 
     ms_step = head["ms_per_step"]
-    check_within(head["kernel_ms_events"] * 0.98, ms_step, "headline GEMM (event-bracketed launches)")
     value = job_throughput(head["macs"], N, ms_step) / 1e9
     int8_peak = 2.0 * peaks["bf16_tflops"]                     # TOP/s (1 MAC = 2 ops)
     achieved = 2 * head["macs"] / (head["kernel_ms"] * 1e-3) / 1e12

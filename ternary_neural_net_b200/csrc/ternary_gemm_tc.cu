@@ -678,15 +678,58 @@ constexpr int kT3Units = kT3N / 4;                     // activation columns in 
 static_assert(kT3N + 128 * kT3S <= static_cast<int>(kT3Cols), "tensor-memory columns");
 static_assert(kT3GU * 4 >= 2 + 2 * (kT3G * kT3K / 10 + 1), "a group's words (from a 2-byte offset) fit its units");
 
-// the 32 bf16 pairs of 64 trits starting at phase PH of word 0 (F[i] = word_i * kFix)
-template <int PH>
-__device__ __forceinline__ void decode64(const uint32_t (&F)[8], const uint32_t* lut, uint32_t (&a)[32]) {
-#pragma unroll
-  for (int p = 0; p < 32; ++p) {
-    const int kp = PH / 2 + p;         // pair index counted from word 0
-    const int j = kp / 5, q = kp % 5;  // word, base-9 digit
-    a[p] = lut[__umulhi(F[j] * pow9(4 - q), 9u)];
+// Word decode for this kernel: a word's five bf16 pairs from three table loads.
+// With F = w * kFix (the fixed-point fraction w / 3^10, see the file header),
+// the high word of 81 F is the base-81 number of digits 6..9, and of 81 times
+// the low word of 81 F that of digits 2..5; 9 times what remains gives digits
+// 0..1 (the errors stay below the digit boundaries for every w < 3^10; checked
+// at compile time below).  A 4-digit code indexes an 81-entry table of two
+// bf16 pairs (8 bytes: the pairs of its digits (0,1) and (2,3)), a 2-digit code
+// the 9-entry pair table.  The 81-entry table is stored 16 times, copy c in the
+// 8-byte bank pair c (entry v of copy c at byte 128 v + 8 c), and lane l reads
+// copy l % 16: the 16 lanes of each half-warp then hit 16 different bank pairs
+// whatever codes they decode.
+constexpr bool quad_digits_exact() {
+  for (uint32_t w = 0; w < 59049u; ++w) {
+    const uint32_t F = w * kFix;
+    const uint32_t va = static_cast<uint32_t>((static_cast<uint64_t>(F) * 81u) >> 32);
+    const uint32_t F1 = F * 81u;
+    const uint32_t vb = static_cast<uint32_t>((static_cast<uint64_t>(F1) * 81u) >> 32);
+    const uint32_t F2 = F1 * 81u;
+    const uint32_t vc = static_cast<uint32_t>((static_cast<uint64_t>(F2) * 9u) >> 32);
+    if (va != w / 729u || vb != (w / 9u) % 81u || vc != w % 9u) return false;
   }
+  return true;
+}
+static_assert(quad_digits_exact(), "base-81 / base-9 digit extraction from the fixed-point fraction");
+
+constexpr uint32_t kQuadTableBytes = 81u * 128u;  // 16 interleaved copies of 81 x 8 bytes
+
+// the 32 bf16 pairs of 64 trits starting at phase PH of word 0 (w[i] = word i)
+template <int PH>
+__device__ __forceinline__ void decode64(const uint32_t (&w)[8], const uint32_t* lut, uint32_t quad_lane,
+                                         uint32_t (&a)[32]) {
+  constexpr int P0 = PH / 2;            // first pair, counted from word 0
+  constexpr int W1 = (P0 + 31) / 5;     // last word needed
+  uint32_t pr[8][5];
+#pragma unroll
+  for (int j = 0; j <= W1; ++j) {
+    const uint32_t F = w[j] * kFix;
+    const uint32_t va = __umulhi(F, 81u);        // digits 6..9
+    const uint32_t F1 = F * 81u;
+    const uint32_t vb = __umulhi(F1, 81u);       // digits 2..5
+    const uint32_t vc = __umulhi(F1 * 81u, 9u);  // digits 0..1
+    uint32_t a0, a1, b0, b1;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];\n" : "=r"(a0), "=r"(a1) : "r"(quad_lane + va * 128u));
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];\n" : "=r"(b0), "=r"(b1) : "r"(quad_lane + vb * 128u));
+    pr[j][0] = lut[vc];
+    pr[j][1] = b0;
+    pr[j][2] = b1;
+    pr[j][3] = a0;
+    pr[j][4] = a1;
+  }
+#pragma unroll
+  for (int p = 0; p < 32; ++p) a[p] = pr[(P0 + p) / 5][(P0 + p) % 5];
 }
 
 __device__ __forceinline__ void tmem_st32(uint32_t addr, const uint32_t (&a)[32]) {
@@ -732,6 +775,7 @@ ternary_gemm_tmem_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint1
   __shared__ uint32_t lut[9];
   uint8_t* const bsm = t3_raw + ((1024u - (smem_u32(t3_raw) & 1023u)) & 1023u);  // kT3S activation stages
   uint8_t* const wbuf = bsm + kT3S * kT3BStage;                                   // [2][kT3M][kT3GU] units
+  uint2* const quad = reinterpret_cast<uint2*>(wbuf + 2 * kT3WBuf + 16);          // 81-entry table, 16 copies
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rank = KS > 1 ? static_cast<int>(blockIdx.x % KS) : 0;
@@ -752,6 +796,13 @@ ternary_gemm_tmem_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint1
     const uint32_t blo = lo == 0 ? 0xBF80u : (lo == 2 ? 0x3F80u : 0u);
     const uint32_t bhi = hi == 0 ? 0xBF80u : (hi == 2 ? 0x3F80u : 0u);
     lut[tid] = blo | (bhi << 16);
+  }
+  for (int e = tid; e < 81 * 16; e += kT3Threads) {  // entry v (digits d0..d3 of v), copy c
+    const int v = e >> 4;
+    uint32_t h[4];
+#pragma unroll
+    for (int i = 0, t = v; i < 4; ++i, t /= 3) h[i] = t % 3 == 0 ? 0xBF80u : (t % 3 == 2 ? 0x3F80u : 0u);
+    quad[e] = make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
   }
   if (tid == 0) {
     for (int i = 0; i < kT3S; ++i) {
@@ -788,6 +839,7 @@ ternary_gemm_tmem_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint1
     const int row = 32 * (warp & 3) + lane;  // weight row of the tile = tensor-memory lane
     const int qk = warp >> 2;                // 64-trit quarter of each stage
     const uint32_t lane_field = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    const uint32_t quad_lane = smem_u32(quad) + 8u * static_cast<uint32_t>(lane & 15);  // this lane's table copy
     bool ok = 32 * (warp & 3) < rows_cta;
     for (int g = 0; g < ngroups && ok; ++g) {
       const int buf = g & 1;
@@ -815,16 +867,16 @@ ternary_gemm_tmem_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint1
         const int64_t t0 = kT3K * (sb + jj) + 64 * qk;  // first trit of this quarter
         const int64_t jw = t0 / 10;
         const uint16_t* wr = wrow + (jw - w0);
-        uint32_t F[8];
+        uint32_t W[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) F[i] = static_cast<uint32_t>(wr[i]) * kFix;
+        for (int i = 0; i < 8; ++i) W[i] = wr[i];
         uint32_t av[32];
         switch (static_cast<int>(t0 - 10 * jw)) {  // the phase, warp-uniform
-          case 0: decode64<0>(F, lut, av); break;
-          case 2: decode64<2>(F, lut, av); break;
-          case 4: decode64<4>(F, lut, av); break;
-          case 6: decode64<6>(F, lut, av); break;
-          default: decode64<8>(F, lut, av); break;
+          case 0: decode64<0>(W, lut, quad_lane, av); break;
+          case 2: decode64<2>(W, lut, quad_lane, av); break;
+          case 4: decode64<4>(W, lut, quad_lane, av); break;
+          case 6: decode64<6>(W, lut, quad_lane, av); break;
+          default: decode64<8>(W, lut, quad_lane, av); break;
         }
         tmem_st32(tmem + lane_field + static_cast<uint32_t>(kT3N + 128 * slot + 32 * qk), av);
         asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
@@ -1006,9 +1058,9 @@ ternary_gemm_tmem_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint1
 }
 
 // dynamic shared memory: 1024-byte alignment slack, the activation stages, two
-// word buffers and 16 bytes past them (a producer may read, and not use, the
-// word after its row's window)
-size_t tmem_smem_bytes() { return 1024 + static_cast<size_t>(kT3S) * kT3BStage + 2u * kT3WBuf + 16; }
+// word buffers, 16 bytes past them (a producer may read, and not use, the word
+// after its row's window) and the interleaved copies of the 81-entry table
+size_t tmem_smem_bytes() { return 1024 + static_cast<size_t>(kT3S) * kT3BStage + 2u * kT3WBuf + 16 + kQuadTableBytes; }
 
 // clusters of KS CTAs of the tensor-memory kernel that can run at once (0 when unknown)
 template <int KS>

@@ -170,7 +170,7 @@ def test_every_base3_word_decodes_lut_kernel(bnn):
     bias = synth.normal_f32(29, 3, (145,))
     xb = synth.bf16_bits_from_f32(synth.normal_f32(29, 2, (1, k)))
     ref, mag = oracle.ternary_linear(xb, words, scale, bias, 1, 145, k)
-    out = bnn.bnn_ternary_linear(to_dev_bf16(xb), to_dev_u16(words), to_dev_f32(scale), to_dev_f32(bias), k)
+    out = bnn.bnn_ternary_linear(to_dev_bf16(xb), to_dev_u16(words), to_dev_f32(scale), to_dev_f32(bias))
     assert_ternary_close(out.cpu().numpy(), ref, mag + np.abs(bias.astype(np.float64)), "lut kernel with bias")
 
 
