@@ -16,10 +16,12 @@
 //     its word, a warp prefix sum of the mask popcounts gives each lane its
 //     first slot, and the lane writes its entries in position order.
 //   - layer: the lanes stride over the row's entries (64-byte coalesced
-//     loads), gather x at each position (bf16, through L1) and add or subtract
-//     it in float32; the warp sum is scaled (and biased) once.  Launched with
-//     programmatic dependent launch: the row's first entries are read before
-//     waiting for the kernel that produced x.
+//     loads), gather x at each position and add or subtract it in float32;
+//     the warp sum is scaled (and biased) once.  At m = 1, x is staged in
+//     shared memory as float32 and the next row's entries load while this
+//     row's are gathered; for m > 1 the gathers read bf16 x through L1.
+//     Launched with programmatic dependent launch: the row's first entries
+//     are read before waiting for the kernel that produced x.
 #include "bnn_internal.cuh"
 
 namespace {
@@ -200,6 +202,86 @@ sparse_gemm_kernel(const uint16_t* __restrict__ x, const int64_t* __restrict__ r
   }
 }
 
+// The layer at m = 1: x staged once per CTA in shared memory as float32 (k
+// floats, k <= 32768), so every gather is a shared-memory load.  One CTA per
+// SM takes a contiguous block of rows; a warp takes every 32nd of them.  Per
+// row the lanes hold up to 512 entries in registers (16 per lane, 64-byte
+// coalesced loads), and the first 512 entries of the warp's next row are
+// loaded while this row's are gathered, so each warp keeps 32 loads in
+// flight.  The row's sum is added by a shuffle tree (a fixed order), scaled
+// once (and biased).  Row ptr and entries are read before the programmatic-
+// launch wait, x after it.
+constexpr int kSpThreads = 1024;
+constexpr int kSpU = 16;  // entries per lane per pass
+
+__global__ void __launch_bounds__(kSpThreads, 1)
+sparse_gemv_smem_kernel(const uint16_t* __restrict__ x, const int64_t* __restrict__ row_ptr,
+                        const uint16_t* __restrict__ entries, const float* __restrict__ scale,
+                        const float* __restrict__ bias, int64_t n, int k, float* __restrict__ out) {
+  extern __shared__ float xs[];  // [k]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int kWarps = kSpThreads / 32;
+  const int64_t r_begin = n * blockIdx.x / gridDim.x, r_end = n * (blockIdx.x + 1) / gridDim.x;
+  bnn::pdl_trigger();
+
+  // entries [b + 32 u + lane] of one pass (0xFFFFFFFF past the end)
+  auto fetch = [&](int64_t q0, int64_t e, uint32_t (&v)[kSpU]) {
+#pragma unroll
+    for (int u = 0; u < kSpU; ++u) {
+      const int64_t q = q0 + 32 * u + lane;
+      v[u] = q < e ? static_cast<uint32_t>(__ldcs(entries + q)) : 0xFFFFFFFFu;
+    }
+  };
+  int64_t r = r_begin + warp;
+  int64_t b = 0, e = 0;
+  uint32_t cur[kSpU];
+  if (r < r_end) {
+    b = row_ptr[r];
+    e = row_ptr[r + 1];
+  }
+  fetch(b, e, cur);
+
+  bnn::pdl_wait();  // x may come from the kernel ahead
+  for (int i = tid; i < k; i += kSpThreads) xs[i] = __uint_as_float(static_cast<uint32_t>(__ldg(x + i)) << 16);
+  __syncthreads();
+
+  while (r < r_end) {
+    const int64_t rn = r + kWarps;
+    int64_t bn = 0, en = 0;
+    if (rn < r_end) {
+      bn = row_ptr[rn];
+      en = row_ptr[rn + 1];
+    }
+    uint32_t nxt[kSpU];
+    fetch(bn, en, nxt);  // the next row's first pass, in flight during this row
+    float acc0 = 0.0f, acc1 = 0.0f;
+    for (int64_t q0 = b;;) {
+#pragma unroll
+      for (int u = 0; u < kSpU; ++u) {
+        const uint32_t v = cur[u];
+        const int pos = static_cast<int>(v & 0x7FFFu);
+        if (v != 0xFFFFFFFFu && pos < k) {  // positions >= k are malformed: skipped
+          const float xv = xs[pos];
+          if (u & 1) acc1 += (v & 0x8000u) ? -xv : xv;
+          else acc0 += (v & 0x8000u) ? -xv : xv;
+        }
+      }
+      q0 += 32 * kSpU;
+      if (q0 >= e) break;
+      fetch(q0, e, cur);  // rows longer than one pass
+    }
+    float sum = acc0 + acc1;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (lane == 0) out[r] = bias ? __ldg(scale + r) * sum + __ldg(bias + r) : __ldg(scale + r) * sum;
+    r = rn;
+    b = bn;
+    e = en;
+#pragma unroll
+    for (int u = 0; u < kSpU; ++u) cur[u] = nxt[u];
+  }
+}
+
 int warp_grid(int64_t rows) {
   const int64_t need = (rows + kWarpsPerBlock - 1) / kWarpsPerBlock;
   const int64_t cap = static_cast<int64_t>(bnn::sm_count()) * 8;
@@ -243,6 +325,15 @@ extern "C" bnn_status bnn_ternary_sparse_gemm(const uint16_t* x_bf16, const int6
   if ((x_bf16 && !bnn::aligned(x_bf16, 2)) || !bnn::aligned(row_ptr, 8) || (entries && !bnn::aligned(entries, 2)) ||
       !bnn::aligned(scale, 4) || (bias && !bnn::aligned(bias, 4)) || !bnn::aligned(out, 4))
     return BNN_ERR_MISALIGNED;
+  if (m == 1 && k > 0) {
+    const size_t smem = static_cast<size_t>(k) * sizeof(float);
+    BNN_TRY(bnn::ensure_smem(sparse_gemv_smem_kernel, smem));
+    const int64_t sms = bnn::sm_count();
+    const int grid = static_cast<int>(n < sms ? n : sms);
+    BNN_TRY(bnn::launch_pdl(sparse_gemv_smem_kernel, dim3(grid), dim3(kSpThreads), smem, s, 1, x_bf16, row_ptr,
+                            entries, scale, bias, n, static_cast<int>(k), out));
+    return bnn::check_launch();
+  }
   const dim3 grid(warp_grid(n)), block(kWarpsPerBlock * 32);
   cudaError_t e;
   if (m == 1)

@@ -102,3 +102,24 @@ def test_sparse_gemm_right_after_encode_with_device_x(bnn):
                                        scale.cpu().numpy(), None, m, n, k)
         assert_ternary_close(got.cpu().numpy(), want, mag, "sparse right after encode")
         del row_ptr, ent
+
+
+@pytest.mark.parametrize("n,k,density", [(150, 32768, 0.1), (300, 1000, 0.0), (1000, 777, 0.7), (5, 3, 1.0)])
+def test_sparse_gemv_m1_shapes(bnn, n, k, density):
+    """m = 1 (x staged in shared memory): the longest rows k allows (several
+    passes of 512 entries per row), empty rows, dense rows and tiny k, with
+    every other row emptied."""
+    rng = np.random.default_rng(n + k)
+    trits = ((rng.integers(0, 2, (n, k)) * 2 - 1) * (rng.random((n, k)) < density)).astype(np.int8)
+    trits[::2] = 0
+    scale = (rng.random(n) + 0.5).astype(np.float32)
+    bias = rng.standard_normal(n).astype(np.float32)
+    xb = synth.bf16_bits_from_f32(synth.normal_f32(n + k, 1, (1, k)))
+    _, row_ptr, ent = _encode(bnn, trits, k)
+    rp, en = oracle.sparse_encode(trits)
+    for b in (None, bias):
+        got = bnn.bnn_ternary_sparse_gemm(to_dev_bf16(xb), row_ptr, ent, to_dev_f32(scale),
+                                          None if b is None else to_dev_f32(b))
+        want, mag = oracle.sparse_gemm(xb, rp, en, scale, b, 1, n, k)
+        lim = mag + (0 if b is None else np.abs(b.astype(np.float64)))
+        assert_ternary_close(got.cpu().numpy(), want, lim, f"sparse m=1 {n}x{k}")
