@@ -96,7 +96,10 @@ def test_tiled_matches_oracle(bnn, m, n, k):
                                    (70, 9600, 512), (65, 2, 64 * 20 + 1), (256, 4096 + 3, 4096 - 64),
                                    (257, 383, 2048 * 2 + 64), (2304, 4219, 130), (600, 9000, 760), (50, 700, 2000),
                                    (64, 1000, 300), (64, 2000, 500), (200, 1000, 2048), (300, 3000, 256),
-                                   (384, 6400, 128), (250, 700, 2048 + 130)])
+                                   (384, 6400, 128), (250, 700, 2048 + 130),
+                                   # two tiles or more per SM (the persistent kernel): ragged m and n, one
+                                   # activation tile, a single stage and several
+                                   (2304, 4219, 128), (2000, 4800, 256), (200, 38000, 128), (300, 40000, 128)])
 def test_tc_tile_configs(bnn, m, n, k):
     _gemm_case(bnn, m, n, k, seed=5 * m + n + 3 * k, algos=(3,))
 

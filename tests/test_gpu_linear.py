@@ -32,7 +32,7 @@ def _case(seed, m, n, k):
 # tiles, TMA and plain loads), small m, and n off the 64- and 32-bit boundaries
 @pytest.mark.parametrize("m,n,k", [(1, 100, 640), (5, 64, 64), (40, 300, 2048 + 37), (64, 1000, 1000),
                                    (100, 500, 4096), (128, 129, 1100), (70, 9600, 512), (257, 383, 4160),
-                                   (600, 9000, 760), (2304, 4219, 130), (33, 31, 3000)])
+                                   (600, 9000, 760), (2304, 4219, 130), (33, 31, 3000), (2304, 4219, 128)])
 @pytest.mark.parametrize("with_bias", [True, False])
 def test_linear_matches_oracle(bnn, m, n, k, with_bias):
     xp, wp, alpha, bias = _case(m + 3 * n + k, m, n, k)
