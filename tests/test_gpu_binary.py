@@ -209,6 +209,12 @@ def test_workload_gemm_large(bnn, algo):
     assert np.all((d - k) % 2 == 0) and np.abs(d).max() <= k
     o = out.cpu().numpy()
     assert_bits_equal(o, c["alpha"][None, :] * d.astype(np.float32), "cfg4 epilogue everywhere")
+    if algo == 0:
+        # every output against the CPU baseline restated from the pages' XOR + popcount
+        # loop (itself checked bitwise against the oracle), on all host cores
+        import os
+        kd, _ = oracle.k1_binary_gemm(c["xp"], c["wp"], c["alpha"], c["m"], c["n"], k, os.cpu_count() or 1)
+        assert np.array_equal(d, kd), "cfg4 dots differ from the CPU XOR + popcount baseline"
 
 
 def test_algos_agree_bitwise_on_random_shapes(bnn):
