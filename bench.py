@@ -512,9 +512,9 @@ def gpu_cfg4(cu, seed, P, st, s, pk, head=None):
         del d, o
     return dict(value=macs / (ms * 1e-3) / 1e9, unit="GMAC/s", ms_kernel=ms, macs=macs,
                 roofline=roofline("tensor", 2 * macs / (ms * 1e-3) / 1e12, int8, "TOP/s",
-                                  "binary_gemm_tc_kernel (m = 8192: 256-row activation tiles)",
+                                  "binary_gemm_tcp_kernel (persistent, 128x256 tiles)",
                                   f"int8 dense = 2 x bf16 {pk['bf16_tflops']} TFLOP/s ({pk['src']})",
-                                  traffic_for("binary_gemm_tc_256x1", "ternary_neural_net_b200/csrc/binary_gemm_tc.cu")))
+                                  traffic_for("binary_gemm_tcp_m8192", "ternary_neural_net_b200/csrc/binary_gemm_tc.cu")))
 
 
 def gpu_cfg5(cu, seed, P, st, s, pk):
@@ -559,7 +559,7 @@ def gpu_cfg5(cu, seed, P, st, s, pk):
                 pack_gbs=(2 * n * k * 4 + pbytes) / (ms_pack * 1e-3) / 1e9,
                 roofline=roofline("hbm", gbs1, pk["hbm_gbs"], "GB/s", "ternary GEMV m = 1",
                                   f"HBM copy {pk['hbm_gbs']} GB/s ({pk['src']})",
-                                  traffic_for("ternary_gemv_rows", "ternary_neural_net_b200/csrc/ternary.cu"),
+                                  traffic_for("ternary_gemv_lut", "ternary_neural_net_b200/csrc/ternary.cu"),
                                   frac_of_read_stream=gbs1 / pk["read_gbs"] if pk.get("read_gbs") else None),
                 roofline_m64=roofline("tensor", fl64 / (ms64 * 1e-3) / 1e12, bf16, "TFLOP/s",
                                       "ternary GEMM m = 64 (tcgen05 kind::f16)",
@@ -1052,13 +1052,14 @@ def main(argv=None):
                          f"512 MiB of outputs, so every step starts cold",
                    "parallelism": f"replicas x{N} (independent problems per GPU)"},
         "roofline": {"bound": "tensor",
-                     "kernel": "binary_gemm_tc_kernel (bnn_binary_gemm AUTO, m >= 64): TMA-fed packed chunks -> 0/1 "
-                               "bytes in swizzled smem, tcgen05.mma kind::i8 into tensor memory",
+                     "kernel": "binary_gemm_tcp_kernel (bnn_binary_gemm AUTO at two tiles or more per SM): persistent "
+                               "CTAs, TMA-fed packed chunks -> 0/1 bytes in swizzled smem, tcgen05.mma kind::i8 into "
+                               "double-buffered tensor memory, epilogue warps overlapping the next tile",
                      "achieved": achieved, "peak": int8_peak, "unit": "TOP/s", "frac": achieved / int8_peak,
                      "achieved_basis": "2 ops x M*N*K per launch / the timed region's duration / K (the step is "
                                        "this one kernel; CUDA events on the launching stream)",
                      "kernel_ms": head["kernel_ms"], "kernel_ms_events": head["kernel_ms_events"],
-                     "traffic": traffic_for("binary_gemm_tc_256x1", "ternary_neural_net_b200/csrc/binary_gemm_tc.cu"),
+                     "traffic": traffic_for("binary_gemm_tcp_m8192", "ternary_neural_net_b200/csrc/binary_gemm_tc.cu"),
                      "peak_basis": f"int8 dense tensor peak = bf16 {peaks['bf16_tflops']} TFLOP/s x 2 (nominal "
                                    f"int8:bf16 ratio 4.5:2.25 PFLOP/s), {peak_src} (burst figure: a kernel timed "
                                    f"alone)"},
