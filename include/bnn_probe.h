@@ -36,8 +36,9 @@ bnn_status bnn_probe_popc(int mode, int64_t blocks, int64_t iters, int32_t* sink
 
 /*
  * bnn_probe_stream_read -- enqueue one kernel of `blocks` x 512 threads that
- * reads `bytes` bytes of `buf` once with 16-byte streaming loads (four in
- * flight per thread, grid-stride, coalesced) and writes nothing else.
+ * reads `bytes` bytes of `buf` once with 16-byte streaming loads (each warp a
+ * contiguous 2 KiB block per step, four loads in flight per thread, blocks
+ * strided across the grid) and writes nothing else.
  *   buf    device, 16-byte aligned; bytes a multiple of 16 (>= 0).
  *   sink   uint32 [1] device; written only when the fold of the data equals
  *          a fixed key (so the loads cannot be optimised away).

@@ -112,6 +112,35 @@ __device__ __forceinline__ void expand_word(uint8_t* dst_row, uint32_t swz, int 
   }
 }
 
+// The same mapping with the bit left in the top bit of its byte (0 or 0x80):
+// per 4 bytes one multiply by a power of two and one AND, where expand_word
+// takes a shift and an AND (both on the integer ALU).  The multipliers
+// mul[t - 1] = 2^t arrive as run-time values, so the multiplies stay integer
+// multiply-adds on the FMA pipe and the two pipes share the expansion.  As
+// signed int8 both operands then hold 0 or -128, every product is 0 or
+// +16384, and the int32 accumulator holds 16384 popcount(a AND b) -- exact
+// while the tile's K stays below 2^17 bits (2^31 / 16384).
+__device__ __forceinline__ void expand_word_hi(uint8_t* dst_row, uint32_t swz, int part, uint64_t cw,
+                                               const uint32_t (&mul)[7]) {
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    const int h = 2 * part + hh;
+    const uint32_t hw = static_cast<uint32_t>(cw >> (32 * hh));
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      // byte j of word s: bit 8j + 4q + s of hw, moved up to bit 7 of the byte
+      uint32_t v[4];
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const int t = 7 - 4 * q - w;
+        v[w] = (t == 0 ? hw : hw * mul[t > 0 ? t - 1 : 0]) & 0x80808080u;
+      }
+      const uint32_t chunk = static_cast<uint32_t>(2 * h + q);
+      *reinterpret_cast<uint4*>(dst_row + ((chunk ^ swz) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
+    }
+  }
+}
+
 // grid: x = KS * (weight tiles of 128 rows), y = activation tiles of BN rows;
 // clusters of KS CTAs along x
 template <int BN, int KS, bool TMA, bool WIDE>
@@ -498,11 +527,14 @@ constexpr int kPThreads = kPProducers + 64 + 128;          // + MMA warp + TMA w
 constexpr uint32_t kPSmem = kPS * kPStageBytes + kPP * kPChunkBytes + 2u * kPProducers * 4u;  // + popcounts
 static_assert(kPSmem + 1024 <= 227u * 1024u, "persistent tile fits shared memory");
 
+// HI: bits expanded to 0/0x80 bytes (expand_word_hi; k < 2^17), else 0/1 bytes.
+// mul_one is 1 at run time (the base of expand_word_hi's multipliers).
+template <bool HI>
 __global__ void __launch_bounds__(kPThreads, 1)
 binary_gemm_tcp_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                        const float* __restrict__ alpha, const float* __restrict__ bias, int64_t m, int64_t n, int k,
                        int kw, int64_t mtiles, int64_t ntiles, int32_t* __restrict__ dots, float* __restrict__ out,
-                       uint32_t* __restrict__ next, int64_t next_w32, uint32_t wait_limit) {
+                       uint32_t* __restrict__ next, int64_t next_w32, uint32_t wait_limit, uint32_t mul_one) {
   using bnn::tc::mbar_drain;
   using bnn::tc::mbar_wait;
   using bnn::tc::mbar_wait_idle;
@@ -574,6 +606,9 @@ binary_gemm_tcp_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_
     const uint32_t swz = static_cast<uint32_t>(row & 7);
     const uint32_t rd_off = static_cast<uint32_t>(r2) * 64u + 8u * static_cast<uint32_t>(part);
     const uint32_t rd_swz = static_cast<uint32_t>((r2 >> 1) & 3);
+    uint32_t mul[7];
+#pragma unroll
+    for (int t = 0; t < 7; ++t) mul[t] = mul_one << (t + 1);
     int64_t gs = 0, gc = 0;  // stages and chunks consumed so far (all tiles)
     bool ok = true;
     int ti = 0;
@@ -598,7 +633,8 @@ binary_gemm_tcp_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_
           break;
         }
         my_pop += __popcll(cw);
-        expand_word(smem + b * kPStageBytes + row_off, swz, part, cw);
+        if constexpr (HI) expand_word_hi(smem + b * kPStageBytes + row_off, swz, part, cw, mul);
+        else expand_word(smem + b * kPStageBytes + row_off, swz, part, cw);
         asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
         mbar_arrive(smem_u32(&full_bar[b]));
       }
@@ -726,7 +762,8 @@ binary_gemm_tcp_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           const int px = 2 * (kTm + c0 + c);
-          const int32_t dv = base - 2 * (pops[px] + pops[px + 1]) + 4 * static_cast<int32_t>(r[c]);
+          const int32_t s4 = HI ? static_cast<int32_t>(r[c] >> 12) : 4 * static_cast<int32_t>(r[c]);  // 4 popc(a&b)
+          const int32_t dv = base - 2 * (pops[px] + pops[px + 1]) + s4;
           const float y0 = __fmul_rn(a_j, static_cast<float>(dv));
           const float y = bias ? __fadd_rn(y0, b_j) : y0;
           if (store && c < nc && jlive) {
@@ -774,11 +811,13 @@ bnn_status launch_tcp(const uint64_t* xp, const uint64_t* wp, const float* alpha
   const int64_t sms = bnn::sm_count();
   const int64_t grid = mtiles * ntiles < sms ? mtiles * ntiles : sms;
   const size_t smem = static_cast<size_t>(kPSmem) + 1024;
-  BNN_TRY(bnn::ensure_smem(binary_gemm_tcp_kernel, smem));
-  const cudaError_t e = bnn::launch_pdl(binary_gemm_tcp_kernel, dim3(static_cast<unsigned>(grid)), dim3(kPThreads),
+  const bool hi = 64 * static_cast<int64_t>(kw) < (int64_t{1} << 17);  // 16384 popc(a AND b) fits int32
+  auto kern = hi ? binary_gemm_tcp_kernel<true> : binary_gemm_tcp_kernel<false>;
+  BNN_TRY(bnn::ensure_smem(kern, smem));
+  const cudaError_t e = bnn::launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(kPThreads),
                                         smem, s, 1, tw, tx, alpha, bias, m, n, k, kw, mtiles, ntiles, dots, out,
                                         reinterpret_cast<uint32_t*>(next), 2 * bnn::words64(n),
-                                        g_wait_limit.load() ? g_wait_limit.load() : bnn::tc::kSpinLimit);
+                                        g_wait_limit.load() ? g_wait_limit.load() : bnn::tc::kSpinLimit, 1u);
   if (e != cudaSuccess) return bnn::cuda_fail(e);
   *launched = true;
   return bnn::check_launch();

@@ -37,24 +37,24 @@ __global__ void __launch_bounds__(256) probe_popc_kernel(int mode, int64_t iters
   sink[tid] = static_cast<int32_t>(r);
 }
 
-// Read-only stream: every thread keeps four 16-byte streaming loads in flight
-// per step (grid-stride, so consecutive threads read consecutive 16-byte
-// pieces: fully coalesced) and folds them into one register.  The fold is
-// written only when it equals a value no input of the bench produces, so the
-// kernel's DRAM traffic is the buffer's bytes read once.
+// Read-only stream: each warp reads one contiguous 2 KiB block per step (four
+// 16-byte streaming loads per lane, 512 consecutive bytes per load
+// instruction), blocks strided by the number of warps in the grid.  The loads
+// are folded into one register, which is written only when it equals a value
+// no input of the bench produces, so the kernel's DRAM traffic is the
+// buffer's bytes read once.
 __global__ void __launch_bounds__(512) probe_read_kernel(const uint4* __restrict__ p, int64_t n16,
                                                          uint32_t key, uint32_t* __restrict__ sink) {
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   uint32_t acc = 0;
-  for (; i + 3 * stride < n16; i += 4 * stride) {
-    const uint4 a = __ldcs(p + i), b = __ldcs(p + i + stride), c = __ldcs(p + i + 2 * stride),
-                d = __ldcs(p + i + 3 * stride);
-    acc ^= (a.x ^ a.y ^ a.z ^ a.w) + (b.x ^ b.y ^ b.z ^ b.w) + (c.x ^ c.y ^ c.z ^ c.w) + (d.x ^ d.y ^ d.z ^ d.w);
-  }
-  for (; i < n16; i += stride) {
-    const uint4 a = __ldcs(p + i);
-    acc ^= a.x ^ a.y ^ a.z ^ a.w;
+  for (int64_t b = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; 128 * b < n16; b += warps) {
+    const int64_t i = 128 * b + lane;
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = i + 32 * u < n16 ? __ldcs(p + i + 32 * u) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) acc ^= v[u].x + v[u].y + v[u].z + v[u].w;
   }
   if (acc == key) sink[0] = acc;
 }

@@ -337,9 +337,10 @@ size_t rows_smem_bytes(int64_t kt) {
 // ---------------------------------------------------------------------------
 constexpr int kLutThreads = 1024;
 constexpr int kLutMaxKt = 416;         // 32-bit pairs of words need kt even; 135 x 416 floats = 219.4 KiB
-constexpr int kLutRowsChunk = 256;     // rows whose pass sums are held at once
+constexpr int kLutRowsChunk = 256;     // rows whose unit sums are held at once
 constexpr int kLutMaxPasses = (kLutMaxKt / 2 + 31) / 32;
-constexpr int kLutGroup = 8;           // units per warp in flight
+constexpr int kLutMaxUnits = (kLutMaxPasses + 1) / 2;  // units (two passes each) per row
+constexpr int kLutGroup = 4;           // units per warp in flight (two 32-bit loads each)
 constexpr uint32_t kDiv81Mul = 25891u, kDiv81Shift = 21;  // floor(w / 81) for w < 3^10
 constexpr uint32_t kDiv27Mul = 607u, kDiv27Shift = 14;    // floor(q / 27) for q < 3^6
 constexpr uint32_t kZeroPair = 29524u | (29524u << 16);   // two all-zero-trit words
@@ -356,40 +357,73 @@ static_assert(lut_divisions_exact(), "multiply-shift division constants");
 __host__ __device__ constexpr int lut_pitch(int kt) { return (kt + 31) & ~31; }
 
 size_t lut_smem_bytes(int64_t kt) {
-  return static_cast<size_t>(135 * lut_pitch(static_cast<int>(kt)) + kLutRowsChunk * kLutMaxPasses) * sizeof(float);
+  return static_cast<size_t>(135 * lut_pitch(static_cast<int>(kt)) + kLutRowsChunk * kLutMaxUnits) * sizeof(float);
 }
 
 __device__ __forceinline__ float bf16f(const uint16_t* x, int e, int k) {
   return e < k ? __uint_as_float(static_cast<uint32_t>(__ldg(x + e)) << 16) : 0.0f;
 }
 
+// One word's three table entries, summed: colA/colB/colC are the byte
+// addresses of the word's column in tables A, B and C, stride one entry row.
+__device__ __forceinline__ float lut_word(uint32_t w, uint32_t colA, uint32_t colB, uint32_t colC, uint32_t stride) {
+  const uint32_t q = (w * kDiv81Mul) >> kDiv81Shift;   // digits 4..9
+  const uint32_t eA = w - 81u * q;                     // digits 0..3
+  const uint32_t eC = (q * kDiv27Mul) >> kDiv27Shift;  // digits 7..9
+  const uint32_t eB = q - 27u * eC;                    // digits 4..6
+  float a, b, c;
+  asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(a) : "r"(colA + eA * stride));
+  asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(b) : "r"(colB + eB * stride));
+  asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(c) : "r"(colC + eC * stride));
+  return (a + b) + c;
+}
+
 __global__ void __launch_bounds__(kLutThreads, 1)
 ternary_gemv_lut_kernel(const uint16_t* __restrict__ x, const uint32_t* __restrict__ packed2,
                         const float* __restrict__ scale, int64_t n, int k, int kt, float* __restrict__ out,
                         const float* __restrict__ bias) {
-  extern __shared__ float T[];  // [135][ktp] tables, then [kLutRowsChunk][passes] pass sums
+  extern __shared__ float T[];  // [135][ktp] tables, then [kLutRowsChunk][units per row] unit sums
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int kWarps = kLutThreads / 32;
   const int ktp = lut_pitch(kt);
   const int kt2 = kt >> 1;                       // 32-bit pairs per row
-  const int passes = (kt2 + 31) >> 5;
-  float* psum = T + 135 * ktp;
+  const int passes = (kt2 + 31) >> 5;            // 32 pairs (64 words) per pass
+  const int upr = (passes + 1) >> 1;             // units per row: passes 2u and 2u + 1
+  const int l_last = kt2 - 32 * (passes - 1);    // lanes of the last pass
+  float* usum = T + 135 * ktp;
   const int64_t r_begin = n * blockIdx.x / gridDim.x, r_end = n * (blockIdx.x + 1) / gridDim.x;
+  // warp-uniform walk over the units u = warp + kWarps i as (row, unit-of-row) pairs
+  const int d_row = kWarps / upr, d_unit = kWarps - d_row * upr;
+  auto advance = [&](int& rl, int& ur) {
+    ur += d_unit;
+    rl += d_row;
+    if (ur >= upr) {
+      ur -= upr;
+      ++rl;
+    }
+  };
   bnn::pdl_trigger();
 
-  // word pair of unit u (row r_chunk + u / passes, pass u % passes) for this lane
-  auto fetch = [&](int64_t r_chunk, int units, int u) -> uint32_t {
-    if (u >= units) return kZeroPair;
-    const int rl = u / passes, p = u - rl * passes;
-    const int c = 32 * p + lane;
-    return c < kt2 ? __ldcs(packed2 + (r_chunk + rl) * kt2 + c) : kZeroPair;
+  // this lane's pairs of unit (rl, ur): passes 2 ur and 2 ur + 1 (zero pairs past the row)
+  auto fetch = [&](int64_t r_chunk, int rows, int rl, int ur, uint32_t& v0, uint32_t& v1) {
+    v0 = v1 = kZeroPair;
+    if (rl < rows) {
+      const uint32_t* src = packed2 + (r_chunk + rl) * kt2 + 64 * ur + lane;
+      if (64 * ur + lane < kt2) v0 = __ldcs(src);
+      if (64 * ur + 32 + lane < kt2) v1 = __ldcs(src + 32);
+    }
   };
 
   int64_t r_chunk = r_begin;
-  int units = static_cast<int>((r_end - r_begin < kLutRowsChunk ? r_end - r_begin : kLutRowsChunk) * passes);
-  uint32_t cur[kLutGroup];
+  int rows = static_cast<int>(r_end - r_begin < kLutRowsChunk ? r_end - r_begin : kLutRowsChunk);
+  int rl0 = warp / upr, ur0 = warp - rl0 * upr;  // the warp's first unit
+  uint32_t cur[kLutGroup][2];
+  int frl = rl0, fur = ur0;  // fetch cursor (runs kLutGroup units ahead of the compute cursor)
 #pragma unroll
-  for (int g = 0; g < kLutGroup; ++g) cur[g] = fetch(r_chunk, units, warp + kWarps * g);
+  for (int g = 0; g < kLutGroup; ++g) {
+    fetch(r_chunk, rows, frl, fur, cur[g][0], cur[g][1]);
+    advance(frl, fur);
+  }
 
   bnn::pdl_wait();  // x may come from the kernel ahead
   // Tables.  Task f = part * kt + column: parts 0..8 fill A's entries
@@ -428,36 +462,37 @@ ternary_gemv_lut_kernel(const uint16_t* __restrict__ x, const uint32_t* __restri
   __syncthreads();
 
   const uint32_t stride = 4u * static_cast<uint32_t>(ktp);
-  const uint32_t tbase = static_cast<uint32_t>(__cvta_generic_to_shared(T));
+  const uint32_t tA = static_cast<uint32_t>(__cvta_generic_to_shared(T));
   const uint32_t offB = 81u * stride, offC = 108u * stride;
-  auto lookup = [&](uint32_t w, uint32_t col) -> float {
-    const uint32_t q = (w * kDiv81Mul) >> kDiv81Shift;   // digits 4..9
-    const uint32_t eA = w - 81u * q;                     // digits 0..3
-    const uint32_t eC = (q * kDiv27Mul) >> kDiv27Shift;  // digits 7..9
-    const uint32_t eB = q - 27u * eC;                    // digits 4..6
-    float a, b, c;
-    asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(a) : "r"(col + eA * stride));
-    asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(b) : "r"(col + offB + eB * stride));
-    asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(c) : "r"(col + offC + eC * stride));
-    return (a + b) + c;
+  const uint32_t lane_full = 4u * static_cast<uint32_t>(lane);
+  const uint32_t lane_last = 4u * static_cast<uint32_t>(lane < l_last ? lane : l_last - 1);  // valid column
+  // the two words of pair v in pass p (warp-uniform p), added to acc
+  auto pass_sum = [&](uint32_t v, int p) -> float {
+    const bool last = p == passes - 1;
+    const uint32_t c0 = tA + 256u * static_cast<uint32_t>(p) + (last ? lane_last : lane_full);
+    const uint32_t c1 = c0 + 4u * static_cast<uint32_t>(last ? l_last : 32);
+    return lut_word(v & 0xFFFFu, c0, c0 + offB, c0 + offC, stride) +
+           lut_word(v >> 16, c1, c1 + offB, c1 + offC, stride);
   };
 
   while (true) {
-    for (int u0 = warp; u0 < units; u0 += kWarps * kLutGroup) {
-      uint32_t nxt[kLutGroup];
-#pragma unroll
-      for (int g = 0; g < kLutGroup; ++g) nxt[g] = fetch(r_chunk, units, u0 + kWarps * (kLutGroup + g));
-      float sum[kLutGroup];
+    int rl = rl0, ur = ur0;
+    while (rl < rows) {
+      uint32_t nxt[kLutGroup][2];
 #pragma unroll
       for (int g = 0; g < kLutGroup; ++g) {
-        const int u = u0 + kWarps * g;
-        const int p = u % passes;               // warp-uniform
-        const int L = kt2 - 32 * p < 32 ? kt2 - 32 * p : 32;
-        const int l = lane < L ? lane : L - 1;  // lanes past the row end read a valid column (their pair is zero)
-        const uint32_t col0 = tbase + 4u * static_cast<uint32_t>(64 * p + l);
-        const uint32_t col1 = col0 + 4u * static_cast<uint32_t>(L);
-        const uint32_t pr = cur[g];
-        sum[g] = lookup(pr & 0xFFFFu, col0) + lookup(pr >> 16, col1);
+        fetch(r_chunk, rows, frl, fur, nxt[g][0], nxt[g][1]);
+        advance(frl, fur);
+      }
+      float sum[kLutGroup];
+      int idx[kLutGroup];
+#pragma unroll
+      for (int g = 0; g < kLutGroup; ++g) {
+        idx[g] = rl < rows ? rl * upr + ur : -1;
+        const int p = 2 * ur;
+        sum[g] = pass_sum(cur[g][0], p);
+        if (p + 1 < passes) sum[g] += pass_sum(cur[g][1], p + 1);
+        advance(rl, ur);
       }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1)
@@ -466,25 +501,32 @@ ternary_gemv_lut_kernel(const uint16_t* __restrict__ x, const uint32_t* __restri
       if (lane == 0) {
 #pragma unroll
         for (int g = 0; g < kLutGroup; ++g)
-          if (u0 + kWarps * g < units) psum[u0 + kWarps * g] = sum[g];
+          if (idx[g] >= 0) usum[idx[g]] = sum[g];
       }
 #pragma unroll
-      for (int g = 0; g < kLutGroup; ++g) cur[g] = nxt[g];
+      for (int g = 0; g < kLutGroup; ++g) {
+        cur[g][0] = nxt[g][0];
+        cur[g][1] = nxt[g][1];
+      }
     }
-    __syncthreads();  // every unit's pass sum of this chunk is stored
-    const int rows = units / passes;
-    for (int rl = tid; rl < rows; rl += kLutThreads) {
+    __syncthreads();  // every unit sum of this chunk is stored
+    for (int r = tid; r < rows; r += kLutThreads) {
       float acc = 0.0f;
-      for (int p = 0; p < passes; ++p) acc += psum[rl * passes + p];
-      const int64_t r = r_chunk + rl;
-      out[r] = bias ? __ldg(scale + r) * acc + __ldg(bias + r) : __ldg(scale + r) * acc;
+      for (int u = 0; u < upr; ++u) acc += usum[r * upr + u];
+      const int64_t gr = r_chunk + r;
+      out[gr] = bias ? __ldg(scale + gr) * acc + __ldg(bias + gr) : __ldg(scale + gr) * acc;
     }
     r_chunk += rows;
     if (r_chunk >= r_end) break;
-    __syncthreads();  // pass sums read before the next chunk overwrites them
-    units = static_cast<int>((r_end - r_chunk < kLutRowsChunk ? r_end - r_chunk : kLutRowsChunk) * passes);
+    __syncthreads();  // unit sums read before the next chunk overwrites them
+    rows = static_cast<int>(r_end - r_chunk < kLutRowsChunk ? r_end - r_chunk : kLutRowsChunk);
+    frl = rl0;
+    fur = ur0;
 #pragma unroll
-    for (int g = 0; g < kLutGroup; ++g) cur[g] = fetch(r_chunk, units, warp + kWarps * g);
+    for (int g = 0; g < kLutGroup; ++g) {
+      fetch(r_chunk, rows, frl, fur, cur[g][0], cur[g][1]);
+      advance(frl, fur);
+    }
   }
 }
 
