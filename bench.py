@@ -548,11 +548,18 @@ def gpu_cfg5(cu, seed, P, st, s, pk):
                                                                   s), iters, st)
     ms1, ms64, ms256 = t(1, 300), t(64, 100), t(256, 30)
     ms64_mma = t(64, 50, 2)
+    # m = 1 on the pair-table kernel (the words 2 bytes off 4-byte alignment, so the table kernel does not apply)
+    pbuf = torch.empty(packed.numel() + 2, dtype=torch.int16, device=dev)
+    pbuf[1:1 + packed.numel()] = packed.reshape(-1)
+    p_off = pbuf[1:1 + packed.numel()]
+    torch.cuda.synchronize(dev)
+    ms1_pairs = graph_time(cu, lambda i: lib.bnn_ternary_gemm(P(xb), P(p_off), P(scale), 1, n, k, P(o), s), 300, st)
     alg1 = pbytes + k * 2 + n * 4 + n * 4
     gbs1 = alg1 / (ms1 * 1e-3) / 1e9
     fl64, fl256 = 2.0 * 64 * n * k, 2.0 * 256 * n * k
     bf16 = pk["bf16_tflops"]
-    return dict(value=gbs1, unit="GB/s (M=1)", us_m1=ms1 * 1e3, us_m64=ms64 * 1e3, us_m256=ms256 * 1e3,
+    return dict(value=gbs1, unit="GB/s (M=1)", us_m1=ms1 * 1e3, us_m1_pair_tables=ms1_pairs * 1e3,
+                us_m64=ms64 * 1e3, us_m256=ms256 * 1e3,
                 us_m64_mma_sync=ms64_mma * 1e3, m64_tflops=fl64 / (ms64 * 1e-3) / 1e12,
                 m256_tflops=fl256 / (ms256 * 1e-3) / 1e12, macs=float(n) * k,
                 pack_ms=ms_pack, pack_noalloc_ms=ms_pack_na, pack_mode_ms=ms_modes,

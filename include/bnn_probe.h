@@ -51,10 +51,11 @@ bnn_status bnn_probe_stream_read(const void* buf, int64_t bytes, int64_t blocks,
 
 /*
  * bnn_probe_wait_limit -- bound, in polls, the main mbarrier waits of the
- * tensor-core binary GEMM kernel (bnn_binary_gemm for m >= 64,
+ * tensor-core binary GEMM kernels (bnn_binary_gemm for m >= 64,
  * BNN_ALGO_TC, bnn_binary_linear) launched after this call; 0 restores the
- * normal bound (2^24 polls).  The final waits for copies and MMAs already in
- * flight keep the normal bound whatever the setting.  A wait that runs out
+ * normal bound (suspending polls for up to one second of wall time).  The
+ * final waits for copies and MMAs already in flight keep the normal bound
+ * whatever the setting.  A wait that runs out
  * makes its CTA skip every store, wait for its copies and MMAs, free its
  * tensor memory and return; bnn_device_error_count() counts it.  With a
  * small limit (a few polls) the first waits run out before the first copies

@@ -56,8 +56,8 @@
 // Bounded waits that ran out in this file's kernels (read by bnn_device_error_count).
 __device__ unsigned int g_bnn_device_errors = 0;
 
-// Polls of the main mbarrier waits of the kernel below (the final drains keep
-// the full bound): 0 = the normal bound; a small value is set only by the
+// Polls of the main mbarrier waits of the kernels below (the final drains keep
+// the full bound): 0 = the normal time bound; a small value is set only by the
 // diagnostic bnn_probe_wait_limit, so that a test can make the waits run out.
 static std::atomic<uint32_t> g_wait_limit{0};
 
@@ -817,7 +817,7 @@ bnn_status launch_tcp(const uint64_t* xp, const uint64_t* wp, const float* alpha
   const cudaError_t e = bnn::launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(kPThreads),
                                         smem, s, 1, tw, tx, alpha, bias, m, n, k, kw, mtiles, ntiles, dots, out,
                                         reinterpret_cast<uint32_t*>(next), 2 * bnn::words64(n),
-                                        g_wait_limit.load() ? g_wait_limit.load() : bnn::tc::kSpinLimit, 1u);
+                                        g_wait_limit.load(), 1u);
   if (e != cudaSuccess) return bnn::cuda_fail(e);
   *launched = true;
   return bnn::check_launch();
@@ -849,7 +849,7 @@ bnn_status launch_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha,
                                         smem, s,
                                         KS, tw, tx, xp, wp, alpha, bias, m, n, k, kw, dots, out,
                                         reinterpret_cast<uint32_t*>(next), 2 * bnn::words64(n),
-                                        g_wait_limit.load() ? g_wait_limit.load() : bnn::tc::kSpinLimit);
+                                        g_wait_limit.load());
   if (e != cudaSuccess) return bnn::cuda_fail(e);
   return bnn::check_launch();
 }

@@ -8,10 +8,17 @@
 namespace bnn {
 namespace tc {
 
-constexpr uint32_t kSpinLimit = 1u << 24;  // iterations of a bounded mbarrier wait
+constexpr uint64_t kWaitNs = 1000000000ull;  // a bounded mbarrier wait gives up after 1 s
+constexpr uint32_t kSuspendNs = 10000000u;   // suspend-time hint of one poll (10 ms; woken when the phase completes)
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
+  return t;
 }
 
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, 8-row
@@ -26,6 +33,7 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
   return d;
 }
 
+// One poll of an mbarrier phase, without suspending.
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -36,39 +44,54 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait of at most `limit` polls; false when it ran out (counted in
-// *errors, abort raised) or when another thread of the CTA raised the abort
-// flag.
+// One poll that suspends the thread until the phase completes or kSuspendNs
+// pass, so that waiting threads do not take issue slots from working ones.
+__device__ __forceinline__ bool mbar_try_suspend(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\nselp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(kSuspendNs)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for an mbarrier phase.  polls == 0: suspending polls for up to
+// kWaitNs of wall time (%globaltimer); polls > 0: at most that many polls
+// without suspension (the short bound of the diagnostic bnn_probe_wait_limit).
+// False when it ran out (counted in *errors, abort raised) or when another
+// thread of the CTA raised the abort flag.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          unsigned int* errors, uint32_t limit = kSpinLimit) {
-  for (uint32_t it = 0; it < limit; ++it) {
-    if (mbar_try(bar, parity)) return true;
-    if ((it & 255u) == 255u && *abort_flag) return false;
+                                          unsigned int* errors, uint32_t polls = 0) {
+  if (polls) {
+    for (uint32_t it = 0; it < polls; ++it)
+      if (mbar_try(bar, parity)) return true;
+  } else {
+    const uint64_t t0 = global_ns();
+    while (true) {
+      if (mbar_try_suspend(bar, parity)) return true;
+      if (*abort_flag) return false;
+      if (global_ns() - t0 > kWaitNs) break;
+    }
   }
   *abort_flag = 1;
   atomicAdd(errors, 1u);
   return false;
 }
 
-// mbar_wait for threads that only wait (MMA issue, copies): between polls the
-// thread sleeps, leaving the issue slots of its SM sub-partition to the warps
-// that compute.
+// The same wait for threads that only wait (MMA issue, copies, epilogue).
 __device__ __forceinline__ bool mbar_wait_idle(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                                unsigned int* errors) {
-  for (uint32_t it = 0; it < (kSpinLimit >> 4); ++it) {
-    if (mbar_try(bar, parity)) return true;
-    if ((it & 15u) == 15u && *abort_flag) return false;
-    __nanosleep(32);
-  }
-  *abort_flag = 1;
-  atomicAdd(errors, 1u);
-  return false;
+  return mbar_wait(bar, parity, abort_flag, errors);
 }
 
 // Bounded wait that ignores the abort flag (the final drains).
 __device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity, unsigned int* errors) {
-  for (uint32_t it = 0; it < kSpinLimit; ++it)
-    if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
+    if (mbar_try_suspend(bar, parity)) return true;
+    if (global_ns() - t0 > kWaitNs) break;
+  }
   atomicAdd(errors, 1u);
   return false;
 }

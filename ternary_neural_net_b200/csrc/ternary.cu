@@ -404,13 +404,15 @@ ternary_gemv_lut_kernel(const uint16_t* __restrict__ x, const uint32_t* __restri
   };
   bnn::pdl_trigger();
 
-  // this lane's pairs of unit (rl, ur): passes 2 ur and 2 ur + 1 (zero pairs past the row)
+  // this lane's pairs of unit (rl, ur): passes 2 ur and 2 ur + 1 (zero pairs past the row);
+  // offsets in 32 bits (the host keeps n * kt / 2 below 2^31)
   auto fetch = [&](int64_t r_chunk, int rows, int rl, int ur, uint32_t& v0, uint32_t& v1) {
     v0 = v1 = kZeroPair;
     if (rl < rows) {
-      const uint32_t* src = packed2 + (r_chunk + rl) * kt2 + 64 * ur + lane;
-      if (64 * ur + lane < kt2) v0 = __ldcs(src);
-      if (64 * ur + 32 + lane < kt2) v1 = __ldcs(src + 32);
+      const int c = 64 * ur + lane;
+      const uint32_t* src = packed2 + static_cast<uint32_t>(static_cast<int>(r_chunk) + rl) * static_cast<uint32_t>(kt2) + c;
+      if (c < kt2) v0 = __ldcs(src);
+      if (c + 32 < kt2) v1 = __ldcs(src + 32);
     }
   };
 
@@ -488,10 +490,14 @@ ternary_gemv_lut_kernel(const uint16_t* __restrict__ x, const uint32_t* __restri
       int idx[kLutGroup];
 #pragma unroll
       for (int g = 0; g < kLutGroup; ++g) {
-        idx[g] = rl < rows ? rl * upr + ur : -1;
-        const int p = 2 * ur;
-        sum[g] = pass_sum(cur[g][0], p);
-        if (p + 1 < passes) sum[g] += pass_sum(cur[g][1], p + 1);
+        idx[g] = -1;
+        sum[g] = 0.0f;
+        if (rl < rows) {  // warp-uniform: units past the chunk's rows cost nothing
+          idx[g] = rl * upr + ur;
+          const int p = 2 * ur;
+          sum[g] = pass_sum(cur[g][0], p);
+          if (p + 1 < passes) sum[g] += pass_sum(cur[g][1], p + 1);
+        }
         advance(rl, ur);
       }
 #pragma unroll
@@ -771,7 +777,8 @@ bnn_status ternary_gemm_impl(const uint16_t* x_bf16, const uint16_t* packed, con
   // for one activation tile, into shared memory above that)
   if (algo == BNN_TALGO_AUTO && m > 8 && k % 8 == 0 && bnn::aligned(x_bf16, 16))
     return bnn::ternary_gemm_tc(x_bf16, packed, scale, bias, m, n, k, out, s);
-  if (algo != BNN_TALGO_MMA && m == 1 && kt > 0 && kt <= kLutMaxKt && kt % 2 == 0 && bnn::aligned(packed, 4)) {
+  if (algo != BNN_TALGO_MMA && m == 1 && kt > 0 && kt <= kLutMaxKt && kt % 2 == 0 && bnn::aligned(packed, 4) &&
+      n * (kt / 2) < (int64_t{1} << 31)) {
     const size_t smem = lut_smem_bytes(kt);
     BNN_TRY(bnn::ensure_smem(ternary_gemv_lut_kernel, smem));
     const int64_t sms = bnn::sm_count();

@@ -46,7 +46,6 @@ constexpr int kTcK = 2;        // CTAs per cluster (split of the trits)
 constexpr int kTcThreads = 256;
 constexpr int kPreT = 4;       // stages of weight words prefetched in registers
 constexpr uint32_t kFix = 72736u;  // ceil(2^32 / 3^10)
-constexpr uint32_t kSpin = 1u << 24;
 constexpr int kAStage = kTcMW * 128;  // bytes per stage of the weight tile
 constexpr int kBStage = kTcNX * 128;  // bytes per stage of the activation tile
 
@@ -62,17 +61,13 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
   return d;
 }
 
+// bounded wait (suspending polls, at most bnn::tc::kWaitNs of wall time)
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity) {
-  for (uint32_t it = 0; it < kSpin; ++it) {
-    uint32_t ok;
-    asm volatile(
-        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    if (ok) return true;
+  const uint64_t t0 = bnn::tc::global_ns();
+  while (true) {
+    if (bnn::tc::mbar_try_suspend(bar, parity)) return true;
+    if (bnn::tc::global_ns() - t0 > bnn::tc::kWaitNs) return false;
   }
-  return false;
 }
 
 // byte offset of element (row, k) (k < 64, 2-byte elements) in a 128B-swizzled K-major tile
