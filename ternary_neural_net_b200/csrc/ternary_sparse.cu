@@ -218,18 +218,19 @@ __global__ void __launch_bounds__(kSpThreads, 1)
 sparse_gemv_smem_kernel(const uint16_t* __restrict__ x, const int64_t* __restrict__ row_ptr,
                         const uint16_t* __restrict__ entries, const float* __restrict__ scale,
                         const float* __restrict__ bias, int64_t n, int k, float* __restrict__ out) {
-  extern __shared__ float xs[];  // [k]
+  extern __shared__ float xs[];  // [k + 1]: x as float32, then xs[k] = 0 (the slot of padding and malformed entries)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int kWarps = kSpThreads / 32;
   const int64_t r_begin = n * blockIdx.x / gridDim.x, r_end = n * (blockIdx.x + 1) / gridDim.x;
   bnn::pdl_trigger();
 
-  // entries [b + 32 u + lane] of one pass (0xFFFFFFFF past the end)
+  // entries [b + 32 u + lane] of one pass (position k, a zero term, past the row's end)
+  const uint32_t pad = static_cast<uint32_t>(k);
   auto fetch = [&](int64_t q0, int64_t e, uint32_t (&v)[kSpU]) {
 #pragma unroll
     for (int u = 0; u < kSpU; ++u) {
       const int64_t q = q0 + 32 * u + lane;
-      v[u] = q < e ? static_cast<uint32_t>(__ldcs(entries + q)) : 0xFFFFFFFFu;
+      v[u] = q < e ? static_cast<uint32_t>(__ldcs(entries + q)) : pad;
     }
   };
   int64_t r = r_begin + warp;
@@ -243,6 +244,7 @@ sparse_gemv_smem_kernel(const uint16_t* __restrict__ x, const int64_t* __restric
 
   bnn::pdl_wait();  // x may come from the kernel ahead
   for (int i = tid; i < k; i += kSpThreads) xs[i] = __uint_as_float(static_cast<uint32_t>(__ldg(x + i)) << 16);
+  if (tid == 0) xs[k] = 0.0f;
   __syncthreads();
 
   while (r < r_end) {
@@ -259,12 +261,11 @@ sparse_gemv_smem_kernel(const uint16_t* __restrict__ x, const int64_t* __restric
 #pragma unroll
       for (int u = 0; u < kSpU; ++u) {
         const uint32_t v = cur[u];
-        const int pos = static_cast<int>(v & 0x7FFFu);
-        if (v != 0xFFFFFFFFu && pos < k) {  // positions >= k are malformed: skipped
-          const float xv = xs[pos];
-          if (u & 1) acc1 += (v & 0x8000u) ? -xv : xv;
-          else acc0 += (v & 0x8000u) ? -xv : xv;
-        }
+        // positions >= k (malformed, or the padding past the row) read the zero slot xs[k]
+        const uint32_t pos = min(v & 0x7FFFu, pad);
+        const float t = __uint_as_float(__float_as_uint(xs[pos]) ^ ((v << 16) & 0x80000000u));  // sign bit 15
+        if (u & 1) acc1 += t;
+        else acc0 += t;
       }
       q0 += 32 * kSpU;
       if (q0 >= e) break;
@@ -326,7 +327,7 @@ extern "C" bnn_status bnn_ternary_sparse_gemm(const uint16_t* x_bf16, const int6
       !bnn::aligned(scale, 4) || (bias && !bnn::aligned(bias, 4)) || !bnn::aligned(out, 4))
     return BNN_ERR_MISALIGNED;
   if (m == 1 && k > 0) {
-    const size_t smem = static_cast<size_t>(k) * sizeof(float);
+    const size_t smem = static_cast<size_t>(k + 1) * sizeof(float);
     BNN_TRY(bnn::ensure_smem(sparse_gemv_smem_kernel, smem));
     const int64_t sms = bnn::sm_count();
     const int grid = static_cast<int>(n < sms ? n : sms);
