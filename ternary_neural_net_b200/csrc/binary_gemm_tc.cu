@@ -48,6 +48,7 @@
 #include <cooperative_groups.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "bnn_internal.cuh"
 #include "bnn_probe.h"
@@ -893,6 +894,33 @@ bnn_status binary_gemm_tc(const uint64_t* xp, const uint64_t* wp, const float* a
     return launch_tc<64, 2, false>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
   if (tiles <= sms) return launch_tc<64, 1, true>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
   return launch_tc<64, 1, false>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
+}
+
+}  // namespace bnn
+
+namespace bnn {
+
+namespace {
+constexpr int kCounterDevices = 64;
+struct CounterSlot {
+  uint64_t ctx;
+  unsigned int* ptr;
+};
+CounterSlot g_counter[kCounterDevices] = {};
+std::mutex g_counter_mu;
+}  // namespace
+
+unsigned int* device_error_counter() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kCounterDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_counter_mu);
+  const uint64_t ctx = context_id();
+  if (ctx == 0 || g_counter[dev].ctx != ctx || !g_counter[dev].ptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_bnn_device_errors) != cudaSuccess) return nullptr;
+    g_counter[dev] = CounterSlot{context_id(), static_cast<unsigned int*>(p)};
+  }
+  return g_counter[dev].ptr;
 }
 
 }  // namespace bnn

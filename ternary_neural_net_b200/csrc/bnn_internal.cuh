@@ -87,6 +87,11 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 bnn_status binary_gemm_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha, const float* bias, int64_t m,
                           int64_t n, int k, int kw, int32_t* dots, float* out, uint64_t* next, cudaStream_t s);
 
+// Device address of the counter of bounded device-side waits that ran out
+// (the one bnn_device_error_count reads), looked up once per CUDA context;
+// nullptr when the lookup fails.
+unsigned int* device_error_counter();
+
 // Bounded waits that ran out in the ternary tensor-core kernel (reset != 0 clears).
 int ternary_tc_error_count(int reset);
 

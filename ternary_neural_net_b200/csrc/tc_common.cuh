@@ -9,7 +9,6 @@ namespace bnn {
 namespace tc {
 
 constexpr uint64_t kWaitNs = 1000000000ull;  // a bounded mbarrier wait gives up after 1 s
-constexpr uint32_t kSuspendNs = 10000000u;   // suspend-time hint of one poll (10 ms; woken when the phase completes)
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -44,23 +43,11 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// One poll that suspends the thread until the phase completes or kSuspendNs
-// pass, so that waiting threads do not take issue slots from working ones.
-__device__ __forceinline__ bool mbar_try_suspend(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\nselp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(kSuspendNs)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait for an mbarrier phase.  polls == 0: suspending polls for up to
-// kWaitNs of wall time (%globaltimer); polls > 0: at most that many polls
-// without suspension (the short bound of the diagnostic bnn_probe_wait_limit).
-// False when it ran out (counted in *errors, abort raised) or when another
-// thread of the CTA raised the abort flag.
+// Bounded wait for an mbarrier phase.  polls == 0: polls for up to kWaitNs of
+// wall time (%globaltimer, read every 64 polls); polls > 0: at most that many
+// polls (the short bound of the diagnostic bnn_probe_wait_limit).  False when
+// it ran out (counted in *errors, abort raised) or when another thread of the
+// CTA raised the abort flag.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           unsigned int* errors, uint32_t polls = 0) {
   if (polls) {
@@ -68,10 +55,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
       if (mbar_try(bar, parity)) return true;
   } else {
     const uint64_t t0 = global_ns();
-    while (true) {
-      if (mbar_try_suspend(bar, parity)) return true;
-      if (*abort_flag) return false;
-      if (global_ns() - t0 > kWaitNs) break;
+    for (uint32_t it = 1;; ++it) {
+      if (mbar_try(bar, parity)) return true;
+      if ((it & 63u) == 0) {
+        if (*abort_flag) return false;
+        if (global_ns() - t0 > kWaitNs) break;
+      }
     }
   }
   *abort_flag = 1;
@@ -79,18 +68,31 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   return false;
 }
 
-// The same wait for threads that only wait (MMA issue, copies, epilogue).
+// The same wait for threads that only wait (MMA issue, copies, epilogue):
+// between polls the thread sleeps, leaving the issue slots of its SM
+// sub-partition to the warps that compute.
 __device__ __forceinline__ bool mbar_wait_idle(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                                unsigned int* errors) {
-  return mbar_wait(bar, parity, abort_flag, errors);
+  const uint64_t t0 = global_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try(bar, parity)) return true;
+    if ((it & 15u) == 0) {
+      if (*abort_flag) return false;
+      if (global_ns() - t0 > kWaitNs) break;
+    }
+    __nanosleep(32);
+  }
+  *abort_flag = 1;
+  atomicAdd(errors, 1u);
+  return false;
 }
 
 // Bounded wait that ignores the abort flag (the final drains).
 __device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity, unsigned int* errors) {
   const uint64_t t0 = global_ns();
-  while (true) {
-    if (mbar_try_suspend(bar, parity)) return true;
-    if (global_ns() - t0 > kWaitNs) break;
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try(bar, parity)) return true;
+    if ((it & 63u) == 0 && global_ns() - t0 > kWaitNs) break;
   }
   atomicAdd(errors, 1u);
   return false;

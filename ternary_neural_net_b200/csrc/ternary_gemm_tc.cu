@@ -61,12 +61,12 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
   return d;
 }
 
-// bounded wait (suspending polls, at most bnn::tc::kWaitNs of wall time)
+// bounded wait (polls for at most bnn::tc::kWaitNs of wall time)
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = bnn::tc::global_ns();
-  while (true) {
-    if (bnn::tc::mbar_try_suspend(bar, parity)) return true;
-    if (bnn::tc::global_ns() - t0 > bnn::tc::kWaitNs) return false;
+  for (uint32_t it = 1;; ++it) {
+    if (bnn::tc::mbar_try(bar, parity)) return true;
+    if ((it & 63u) == 0 && bnn::tc::global_ns() - t0 > bnn::tc::kWaitNs) return false;
   }
 }
 

@@ -81,6 +81,14 @@ def test_skinny_matches_oracle(bnn, m, n, k):
     _gemm_case(bnn, m, n, k, seed=m * 1000 + n + k)
 
 
+# m = 1 with 16-byte aligned rows of at most 256 words streams the weights by
+# bulk copies: one to four 64-word passes per row, rows per chunk from 512 down
+# to 16, several chunks per CTA (the ring wraps), fewer rows than SMs.
+@pytest.mark.parametrize("n,k", [(5000, 16384), (3000, 12000), (70000, 128), (100, 8192), (20000, 640), (7, 4096)])
+def test_gemv_bulk_shapes(bnn, n, k):
+    _gemm_case(bnn, 1, n, k, seed=n + k, algos=(0,))
+
+
 @pytest.mark.parametrize("m,n,k", [(9, 33, 64), (64, 64, 128), (130, 257, 1000), (300, 129, 4096 + 100),
                                    (129, 1000, 63), (512, 640, 512), (17, 3, 130), (16, 8, 32), (1000, 2500, 257),
                                    (2400, 2500, 640)])
