@@ -537,6 +537,146 @@ ternary_gemv_lut_kernel(const uint16_t* __restrict__ x, const uint32_t* __restri
 }
 
 // ---------------------------------------------------------------------------
+// Ternary GEMV, m = 1, k <= 4800: 5 + 5-trit activation tables, the row
+// length split over a cluster of kC5 CTAs.
+//
+// A word's low five digits (w mod 243) and high five (w div 243, one exact
+// multiply-shift) index two 243-entry tables of word position j: lo_j[e] =
+// sum_{i<5} x[10j+i] (d_i(e) - 1) and hi_j[e] the same over x[10j+5..10j+9], so
+// a word costs two shared-memory loads and two adds.  The tables of a whole row
+// do not fit one SM (2 x 243 entries per word), so the kC5 CTAs of a cluster
+// take one slice of at most 96 word positions each and hold only that slice's
+// tables (two [243][96] float arrays, 182 KiB), and every CTA of the cluster
+// runs over the same block of rows: a warp takes whole rows, its 32 lanes
+// consecutive word positions (so a lookup's 32 lanes read 32 consecutive
+// columns: 32 banks), one 16-bit load per word, the next row's words in
+// registers while this row is added.  Each row's slice sum (a shuffle tree) is
+// stored in the CTA's shared memory; after a cluster barrier CTA q adds, for
+// its share of the block's rows, the kC5 slice sums in rank order through
+// distributed shared memory, scales once and writes.  Deterministic for a
+// given launch shape.  The first row's words are loaded before the
+// programmatic-launch wait, the tables (which depend on x) after it.
+// ---------------------------------------------------------------------------
+constexpr int kC5 = 5;                 // CTAs per cluster (slices of the row)
+constexpr int kC5Threads = 1024;
+constexpr int kC5Pitch = 96;           // table columns (word positions) per slice; a multiple of 32
+constexpr int kC5Rows = 1024;          // rows of a block (slice sums held at once)
+constexpr uint32_t kDiv243Mul = 69043u, kDiv243Shift = 24;  // floor(w / 243) for w < 3^10
+
+constexpr bool div243_exact() {
+  for (uint32_t w = 0; w < 59049u; ++w)
+    if ((w * kDiv243Mul) >> kDiv243Shift != w / 243u) return false;
+  return true;
+}
+static_assert(div243_exact(), "multiply-shift division by 243");
+
+size_t c5_smem_bytes() { return (2u * 243u * kC5Pitch + kC5Rows) * sizeof(float); }
+
+__global__ void __launch_bounds__(kC5Threads, 1)
+ternary_gemv_c5_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ packed,
+                       const float* __restrict__ scale, int64_t n, int k, int kt, int slice, int64_t block_rows,
+                       float* __restrict__ out, const float* __restrict__ bias) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  extern __shared__ float c5sm[];  // lo [243][kC5Pitch], hi [243][kC5Pitch], slice sums [kC5Rows]
+  float* const lo = c5sm;
+  float* const hi = c5sm + 243 * kC5Pitch;
+  float* const psum = c5sm + 2 * 243 * kC5Pitch;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int kWarps = kC5Threads / 32;
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int64_t cl = blockIdx.x / kC5, nclusters = gridDim.x / kC5;
+  const int w0 = rank * slice;                                  // this CTA's first word position
+  const int sw = kt - w0 < slice ? (kt - w0 > 0 ? kt - w0 : 0) : slice;  // its word count (<= kC5Pitch)
+  const int64_t nblocks = (n + block_rows - 1) / block_rows;
+  bnn::pdl_trigger();
+
+  // the words of row r at positions w0 + lane + 32 p (29524 = all-zero trits past the slice)
+  auto fetch = [&](int64_t r, bool live, uint32_t (&v)[3]) {
+#pragma unroll
+    for (int p = 0; p < 3; ++p) {
+      const int o = lane + 32 * p;
+      v[p] = (live && o < sw) ? static_cast<uint32_t>(__ldcs(packed + r * kt + w0 + o)) : 29524u;
+    }
+  };
+  int64_t blk = cl;
+  int64_t b0 = blk * block_rows;
+  int64_t b1 = b0 + block_rows < n ? b0 + block_rows : n;
+  uint32_t cur[3];
+  fetch(b0 + warp, blk < nblocks && b0 + warp < b1, cur);
+
+  bnn::pdl_wait();  // x may come from the kernel ahead
+  // Tables: task = (table t, high digits e_hi of the 5, word position o), nine
+  // entries each (the two low digits run over 0..8); consecutive threads take
+  // consecutive positions of one entry row (distinct banks).  Every column is
+  // built, those past the slice with x = 0 (all their entries 0), since the
+  // lanes past the slice look up the all-zero-trit word there.
+  for (int f = tid; f < 2 * 27 * kC5Pitch; f += kC5Threads) {
+    const int o = f % kC5Pitch, g = f / kC5Pitch, t = g / 27, eh = g - 27 * t;
+    const int e0 = 10 * (w0 + o) + 5 * t;
+    float xv[5];
+#pragma unroll
+    for (int i = 0; i < 5; ++i)
+      xv[i] = (o < sw && e0 + i < k) ? __uint_as_float(static_cast<uint32_t>(__ldg(x + e0 + i)) << 16) : 0.0f;
+    const float base = xv[2] * static_cast<float>(eh % 3 - 1) + xv[3] * static_cast<float>((eh / 3) % 3 - 1) +
+                       xv[4] * static_cast<float>(eh / 9 - 1);
+    float* dst = (t == 0 ? lo : hi) + (9 * eh) * kC5Pitch + o;
+#pragma unroll
+    for (int v = 0; v < 9; ++v)
+      dst[v * kC5Pitch] = (xv[0] * static_cast<float>(v % 3 - 1) + xv[1] * static_cast<float>(v / 3 - 1)) + base;
+  }
+  __syncthreads();
+
+  const uint32_t stride = 4u * kC5Pitch;
+  const uint32_t lo_lane = static_cast<uint32_t>(__cvta_generic_to_shared(lo)) + 4u * static_cast<uint32_t>(lane);
+  const uint32_t hi_lane = static_cast<uint32_t>(__cvta_generic_to_shared(hi)) + 4u * static_cast<uint32_t>(lane);
+  for (; blk < nblocks; blk += nclusters) {
+    const int rows = static_cast<int>(b1 - b0);
+    for (int rl = warp; rl < rows; rl += kWarps) {
+      // the next row of this warp (in this block, else the first of the next block)
+      int64_t nr = b0 + rl + kWarps;
+      bool nlive = rl + kWarps < rows;
+      if (!nlive) {
+        const int64_t nb = blk + nclusters;
+        nr = nb * block_rows + warp;
+        nlive = nb < nblocks && nr < (nb * block_rows + block_rows < n ? nb * block_rows + block_rows : n);
+      }
+      uint32_t nxt[3];
+      fetch(nr, nlive, nxt);
+      float acc = 0.0f;
+#pragma unroll
+      for (int p = 0; p < 3; ++p) {
+        const uint32_t w = cur[p];
+        const uint32_t qh = (w * kDiv243Mul) >> kDiv243Shift;  // digits 5..9
+        const uint32_t ql = w - 243u * qh;                     // digits 0..4
+        float a, b;
+        asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(a) : "r"(lo_lane + 128u * p + ql * stride));
+        asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(b) : "r"(hi_lane + 128u * p + qh * stride));
+        acc += a + b;
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      if (lane == 0) psum[rl] = acc;
+#pragma unroll
+      for (int p = 0; p < 3; ++p) cur[p] = nxt[p];
+    }
+    cluster.sync();  // every CTA's slice sums of this block are stored
+    // this CTA finalises rows [q0, q1) of the block: slice sums added in rank order
+    const int q0 = rows * rank / kC5, q1 = rows * (rank + 1) / kC5;
+    for (int rl = q0 + tid; rl < q1; rl += kC5Threads) {
+      float sum = 0.0f;
+#pragma unroll
+      for (int q = 0; q < kC5; ++q) sum += cluster.map_shared_rank(psum, q)[rl];
+      const int64_t r = b0 + rl;
+      out[r] = bias ? __ldg(scale + r) * sum + __ldg(bias + r) : __ldg(scale + r) * sum;
+    }
+    cluster.sync();  // slice sums read before the next block overwrites them (and before any CTA exits)
+    b0 = (blk + nclusters) * block_rows;
+    b1 = b0 + block_rows < n ? b0 + block_rows : n;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Ternary GEMM (m > 8): trits decoded to bf16 tiles in shared memory, bf16
 // mma.sync m16n8k16 with fp32 accumulation.
 //
@@ -760,6 +900,36 @@ extern "C" bnn_status bnn_ternary_pack(const float* w, int64_t n, int64_t k, uin
 }
 
 namespace {
+// Clusters of the c5 GEMV kernel that fit the GPU at once (cached per CUDA
+// context; 0 when the occupancy query fails: the other m = 1 kernels are used).
+int c5_clusters() {
+  static std::mutex mu;
+  static uint64_t ctx_cached = 0;
+  static int cached = 0;
+  std::lock_guard<std::mutex> lock(mu);
+  const uint64_t ctx = bnn::context_id();
+  if (ctx != 0 && ctx == ctx_cached) return cached;
+  int num = 0;
+  if (bnn::ensure_smem(ternary_gemv_c5_kernel, c5_smem_bytes()) == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kC5 * 64);
+    cfg.blockDim = dim3(kC5Threads);
+    cfg.dynamicSmemBytes = c5_smem_bytes();
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kC5;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&num, ternary_gemv_c5_kernel, &cfg) != cudaSuccess) num = 0;
+  }
+  cudaGetLastError();  // a failed query leaves no error behind
+  cached = num;
+  ctx_cached = bnn::context_id();
+  return num;
+}
+
 bnn_status ternary_gemm_impl(const uint16_t* x_bf16, const uint16_t* packed, const float* scale, const float* bias,
                              int64_t m, int64_t n, int64_t k, float* out, int algo, cudaStream_t s) {
   if (algo != BNN_TALGO_AUTO && algo != BNN_TALGO_CUDA_CORES && algo != BNN_TALGO_MMA && algo != BNN_TALGO_TC)
@@ -777,6 +947,21 @@ bnn_status ternary_gemm_impl(const uint16_t* x_bf16, const uint16_t* packed, con
   // for one activation tile, into shared memory above that)
   if (algo == BNN_TALGO_AUTO && m > 8 && k % 8 == 0 && bnn::aligned(x_bf16, 16))
     return bnn::ternary_gemm_tc(x_bf16, packed, scale, bias, m, n, k, out, s);
+  if (algo != BNN_TALGO_MMA && m == 1 && kt > 0 && kt <= kC5 * kC5Pitch) {
+    const int clusters = c5_clusters();
+    if (clusters > 0) {
+      const int slice = static_cast<int>((kt + kC5 - 1) / kC5);
+      const int64_t g = (n + 63) / 64 < clusters ? (n + 63) / 64 : clusters;  // at least 64 rows per cluster
+      int64_t block_rows = (n + g - 1) / g;
+      if (block_rows > kC5Rows) block_rows = kC5Rows;
+      const size_t smem = c5_smem_bytes();
+      BNN_TRY(bnn::ensure_smem(ternary_gemv_c5_kernel, smem));
+      BNN_TRY(bnn::launch_pdl(ternary_gemv_c5_kernel, dim3(static_cast<unsigned>(kC5 * g)), dim3(kC5Threads), smem, s,
+                              kC5, x_bf16, packed, scale, n, static_cast<int>(k), static_cast<int>(kt), slice,
+                              block_rows, out, bias));
+      return bnn::check_launch();
+    }
+  }
   if (algo != BNN_TALGO_MMA && m == 1 && kt > 0 && kt <= kLutMaxKt && kt % 2 == 0 && bnn::aligned(packed, 4) &&
       n * (kt / 2) < (int64_t{1} << 31)) {
     const size_t smem = lut_smem_bytes(kt);
