@@ -643,13 +643,15 @@ bnn_status launch_tc2(const CUtensorMap& tx, const uint16_t* packed, const float
 // tcgen05.st.32x32b.x32 into the stage's A slot of tensor memory; the MMA reads
 // A from there ([a-tmem] operand) and B, the activations, from shared memory
 // (four TMA boxes of 64 x 64 bf16 per stage, 128-byte swizzle).  The packed
-// words reach shared memory without passing through registers: four loader
+// words reach shared memory without passing through registers: the loader
 // warps copy, per group of five stages (1280 trits = 128 words, 129 when the
 // group starts inside a word), every row's window as 4-byte cp.async units
 // (the row's bytes from the 4-byte boundary at or below its first word; units
 // past the end of the matrix are zero-filled) into a [row][65 units] buffer
 // (odd stride: a warp's 32 rows read 32 different banks), double-buffered and
-// completed on an mbarrier by cp.async.mbarrier.arrive.  Per stage a producer
+// completed on an mbarrier by cp.async.mbarrier.arrive (eight loader warps; the
+// producers sleep between polls while a group's words arrive, leaving the
+// issue slots to the loaders).  Per stage a producer
 // waits for its slot to be free, decodes, stores, waits for the store and
 // arrives once per warp; one thread waits for the A slot and the B tile and
 // issues 16 tcgen05.mma (K = 16).  A cluster of KS CTAs splits the stages;
@@ -663,7 +665,7 @@ constexpr int kT3S = 3;                                // stages in flight
 constexpr int kT3G = 5;                                // stages per word group (1280 trits)
 constexpr int kT3GU = 65;                              // 4-byte units staged per row and group (129 words + offset)
 constexpr int kT3Prod = 512;                           // producer threads (16 warps)
-constexpr int kT3Load = 128;                           // loader threads (4 warps)
+constexpr int kT3Load = 256;                           // loader threads (8 warps)
 constexpr int kT3Threads = kT3Prod + 64 + kT3Load;     // + MMA warp + TMA warp + loaders
 constexpr uint32_t kT3BAtom = kT3N * 128u;             // one 64-trit box of activations
 constexpr uint32_t kT3BStage = 4 * kT3BAtom;
@@ -838,8 +840,9 @@ ternary_gemm_tmem_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint1
     bool ok = 32 * (warp & 3) < rows_cta;
     for (int g = 0; g < ngroups && ok; ++g) {
       const int buf = g & 1;
-      bool fine = mbar_wait(smem_u32(&w_full[buf]), static_cast<uint32_t>((g >> 1) & 1), &abort_flag,
-                            &g_bnn_tc_ternary_errors);
+      // sleeping between polls: the loaders need the issue slots while the group's words arrive
+      bool fine = mbar_wait_idle(smem_u32(&w_full[buf]), static_cast<uint32_t>((g >> 1) & 1), &abort_flag,
+                                 &g_bnn_tc_ternary_errors);
       if (!__all_sync(0xffffffffu, fine)) break;
       const int64_t s0 = sb + kT3G * static_cast<int64_t>(g);  // first stage of the group
       const int64_t w0 = (kT3K * s0) / 10;                     // first word staged
@@ -887,6 +890,9 @@ ternary_gemm_tmem_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint1
     const int lt = tid - kLoadWarp0 * 32;
     const uint8_t* gbase = reinterpret_cast<const uint8_t*>(packed);
     const int64_t total_bytes = n * kt * 2;
+    // this thread's units idx = lt + kT3Load i, walked as (row, unit) without divisions
+    const int r_first = lt / kT3GU, u_first = lt - r_first * kT3GU;
+    constexpr int kDr = kT3Load / kT3GU, kDu = kT3Load % kT3GU;
     for (int g = 0; g < ngroups; ++g) {
       const int buf = g & 1;
       if (g >= 2 && !mbar_wait_idle(smem_u32(&w_empty[buf]), static_cast<uint32_t>(((g >> 1) + 1) & 1), &abort_flag,
@@ -894,12 +900,19 @@ ternary_gemm_tmem_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint1
         break;
       const int64_t w0 = (kT3K * (sb + kT3G * static_cast<int64_t>(g))) / 10;
       const uint32_t dbase = smem_u32(wbuf + buf * kT3WBuf);
+      const int64_t first = 2 * (j0 * kt + w0);  // byte of the group's first word in row 0 of the tile
+      int r = r_first, un = u_first;
       for (int idx = lt; idx < rows_cta * kT3GU; idx += kT3Load) {
-        const int r = idx / kT3GU, un = idx - r * kT3GU;
-        const int64_t a = ((((j0 + r) * kt + w0) * 2) & ~int64_t{3}) + 4 * un;  // 4-byte unit of the matrix
+        const int64_t a = ((first + 2 * static_cast<int64_t>(r) * kt) & ~int64_t{3}) + 4 * un;  // 4-byte unit
         const int64_t left = r < rows_live ? total_bytes - a : 0;
         const uint32_t bytes = left >= 4 ? 4u : (left > 0 ? static_cast<uint32_t>(left) : 0u);
         cp_async4(dbase + static_cast<uint32_t>(idx) * 4u, gbase + (bytes ? a : 0), bytes);
+        un += kDu;
+        r += kDr;
+        if (un >= kT3GU) {
+          un -= kT3GU;
+          ++r;
+        }
       }
       asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(smem_u32(&w_full[buf])) : "memory");
     }
