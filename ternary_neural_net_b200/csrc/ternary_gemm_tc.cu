@@ -638,8 +638,9 @@ bnn_status launch_tc2(const CUtensorMap& tx, const uint16_t* packed, const float
 // With one activation tile every packed word is decoded exactly once, so the
 // decode is the whole cost.  Here it writes no shared memory: each producer
 // thread owns one weight row (its tensor-memory lane) and one 64-trit quarter
-// of a 256-trit stage, decodes its 32 bf16 pairs into registers (five base-9
-// digit phases, warp-uniform, as above) and stores them with one
+// of a 256-trit stage, decodes its 32 bf16 pairs into registers (each word's
+// five pairs from two 81-entry quad-table loads and one pair-table load,
+// specialised per warp-uniform phase) and stores them with one
 // tcgen05.st.32x32b.x32 into the stage's A slot of tensor memory; the MMA reads
 // A from there ([a-tmem] operand) and B, the activations, from shared memory
 // (four TMA boxes of 64 x 64 bf16 per stage, 128-byte swizzle).  The packed
