@@ -190,7 +190,7 @@ void dispatch_gemv(const uint64_t* xp, const uint64_t* wp, const float* alpha, i
 // refilled once every warp has passed the barrier after it.  The weights'
 // first chunks are requested before the programmatic-launch wait.
 // ---------------------------------------------------------------------------
-constexpr int kGvThreads = 256;
+constexpr int kGvThreads = 512;
 constexpr int kGvStages = 4;
 constexpr int kGvChunkBytes = 32 * 1024;
 
@@ -249,15 +249,19 @@ binary_gemv_bulk_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restr
     const int w = 2 * (32 * p + lane);
     xv[p] = w < kw ? __ldg(reinterpret_cast<const ulonglong2*>(xp + w)) : make_ulonglong2(0, 0);
   }
+  constexpr int kWarps = kGvThreads / 32;
   int c = 0;
   for (; c < nch; ++c) {
     const int st = c % kGvStages;
-    const bool ok = gv_wait(bar(st), static_cast<uint32_t>((c / kGvStages) & 1));
-    if (!__syncthreads_and(ok)) break;  // the chunk did not land in time: every thread stops here
     const int64_t first = r0 + static_cast<int64_t>(c) * rows_chunk;
     const int rows = static_cast<int>(r1 - first < rows_chunk ? r1 - first : rows_chunk);
+    // the scales of this warp's rows of the chunk (lane i: row warp + kWarps i), loaded before the wait
+    float a_lane = 0.0f;
+    if (out && warp + kWarps * lane < rows) a_lane = __ldg(alpha + first + warp + kWarps * lane);
+    const bool ok = gv_wait(bar(st), static_cast<uint32_t>((c / kGvStages) & 1));
+    if (!__syncthreads_and(ok)) break;  // the chunk did not land in time: every thread stops here
     const uint8_t* buf = gsm + st * chunk_bytes;
-    for (int rr = warp; rr < rows; rr += kGvThreads / 32) {
+    for (int rr = warp, i = 0; rr < rows; rr += kWarps, ++i) {
       uint32_t acc = 0;
 #pragma unroll
       for (int p = 0; p < PASSES; ++p) {
@@ -269,11 +273,12 @@ binary_gemv_bulk_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restr
       }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      const float a = __shfl_sync(0xffffffffu, a_lane, i & 31);
       if (lane == 0) {
         const int64_t row = first + rr;
         const int32_t d = k - 2 * static_cast<int32_t>(acc);
         if (dots) dots[row] = d;
-        if (out) out[row] = alpha[row] * static_cast<float>(d);
+        if (out) out[row] = (i < 32 ? a : __ldg(alpha + row)) * static_cast<float>(d);
       }
     }
     __syncthreads();  // every warp is done with this buffer
@@ -685,7 +690,8 @@ extern "C" bnn_status bnn_binary_gemm_algo(const uint64_t* xp, const uint64_t* w
     return vec2 ? dispatch_mma<2>(xp, wp, alpha, m, n, ki, kw, dots, out, s)
                 : dispatch_mma<1>(xp, wp, alpha, m, n, ki, kw, dots, out, s);
   }
-  if (m == 1 && vec2 && kw <= 256 && algo == BNN_ALGO_AUTO) {
+  // large weight streams only (at least 4 MiB: about 28 KiB per SM); smaller ones are launch-latency bound
+  if (m == 1 && vec2 && kw > 0 && kw <= 256 && algo == BNN_ALGO_AUTO && n * kw >= (int64_t{1} << 19)) {
     const int rows_chunk = kGvChunkBytes / (8 * kw) < 1 ? 1 : kGvChunkBytes / (8 * kw);
     const int64_t sms = bnn::sm_count();
     const int64_t want = (n + rows_chunk - 1) / rows_chunk;  // at least one chunk per CTA

@@ -619,8 +619,11 @@ binary_gemm_tcp_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_
         const int s = j % kChunkStages;
         const int64_t cc = gc + j / kChunkStages;
         const int pb = static_cast<int>(cc % kPP);
-        if (s == 0 && !mbar_wait(smem_u32(&chunk_full[pb]), static_cast<uint32_t>((cc / kPP) & 1), &abort_flag,
-                                 &g_bnn_device_errors, wait_limit)) {
+        // waits sleep between polls: the epilogue warps of the previous tile need the issue slots
+        if (s == 0 && !(wait_limit ? mbar_wait(smem_u32(&chunk_full[pb]), static_cast<uint32_t>((cc / kPP) & 1),
+                                               &abort_flag, &g_bnn_device_errors, wait_limit)
+                                   : mbar_wait_idle(smem_u32(&chunk_full[pb]), static_cast<uint32_t>((cc / kPP) & 1),
+                                                    &abort_flag, &g_bnn_device_errors))) {
           ok = false;
           break;
         }
@@ -628,8 +631,10 @@ binary_gemm_tcp_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_
             chunks + pb * kPChunkBytes + rd_off + ((static_cast<uint32_t>(s) ^ rd_swz) << 4));
         if (s == kChunkStages - 1 || j == nst - 1) mbar_arrive(smem_u32(&chunk_empty[pb]));
         const int b = static_cast<int>(gs % kPS);
-        if (gs >= kPS && !mbar_wait(smem_u32(&empty_bar[b]), static_cast<uint32_t>((gs / kPS + 1) & 1), &abort_flag,
-                                    &g_bnn_device_errors, wait_limit)) {
+        if (gs >= kPS && !(wait_limit ? mbar_wait(smem_u32(&empty_bar[b]), static_cast<uint32_t>((gs / kPS + 1) & 1),
+                                                  &abort_flag, &g_bnn_device_errors, wait_limit)
+                                      : mbar_wait_idle(smem_u32(&empty_bar[b]), static_cast<uint32_t>((gs / kPS + 1) & 1),
+                                                       &abort_flag, &g_bnn_device_errors))) {
           ok = false;
           break;
         }
