@@ -512,9 +512,9 @@ def gpu_cfg4(cu, seed, P, st, s, pk, head=None):
         del d, o
     return dict(value=macs / (ms * 1e-3) / 1e9, unit="GMAC/s", ms_kernel=ms, macs=macs,
                 roofline=roofline("tensor", 2 * macs / (ms * 1e-3) / 1e12, int8, "TOP/s",
-                                  "binary_gemm_tcp_kernel (persistent, 128x256 tiles)",
+                                  "binary_gemm_tc_kernel<256,1> (128x256 tiles)",
                                   f"int8 dense = 2 x bf16 {pk['bf16_tflops']} TFLOP/s ({pk['src']})",
-                                  traffic_for("binary_gemm_tcp_m8192", "ternary_neural_net_b200/csrc/binary_gemm_tc.cu")))
+                                  traffic_for("binary_gemm_tc_256x1", "ternary_neural_net_b200/csrc/binary_gemm_tc.cu")))
 
 
 def gpu_cfg5(cu, seed, P, st, s, pk):
@@ -548,25 +548,20 @@ def gpu_cfg5(cu, seed, P, st, s, pk):
                                                                   s), iters, st)
     ms1, ms64, ms256 = t(1, 300), t(64, 100), t(256, 30)
     ms64_mma = t(64, 50, 2)
-    # m = 1 on the pair-table kernel (the words 2 bytes off 4-byte alignment, so the table kernel does not apply)
-    pbuf = torch.empty(packed.numel() + 2, dtype=torch.int16, device=dev)
-    pbuf[1:1 + packed.numel()] = packed.reshape(-1)
-    p_off = pbuf[1:1 + packed.numel()]
-    torch.cuda.synchronize(dev)
-    ms1_pairs = graph_time(cu, lambda i: lib.bnn_ternary_gemm(P(xb), P(p_off), P(scale), 1, n, k, P(o), s), 300, st)
     alg1 = pbytes + k * 2 + n * 4 + n * 4
     gbs1 = alg1 / (ms1 * 1e-3) / 1e9
     fl64, fl256 = 2.0 * 64 * n * k, 2.0 * 256 * n * k
     bf16 = pk["bf16_tflops"]
-    return dict(value=gbs1, unit="GB/s (M=1)", us_m1=ms1 * 1e3, us_m1_pair_tables=ms1_pairs * 1e3,
+    return dict(value=gbs1, unit="GB/s (M=1)", us_m1=ms1 * 1e3,
                 us_m64=ms64 * 1e3, us_m256=ms256 * 1e3,
                 us_m64_mma_sync=ms64_mma * 1e3, m64_tflops=fl64 / (ms64 * 1e-3) / 1e12,
                 m256_tflops=fl256 / (ms256 * 1e-3) / 1e12, macs=float(n) * k,
                 pack_ms=ms_pack, pack_noalloc_ms=ms_pack_na, pack_mode_ms=ms_modes,
                 pack_gbs=(2 * n * k * 4 + pbytes) / (ms_pack * 1e-3) / 1e9,
-                roofline=roofline("hbm", gbs1, pk["hbm_gbs"], "GB/s", "ternary GEMV m = 1",
+                roofline=roofline("hbm", gbs1, pk["hbm_gbs"], "GB/s",
+                                  "ternary_gemv_c5_kernel (m = 1, 5 + 5-trit tables over 5-CTA clusters)",
                                   f"HBM copy {pk['hbm_gbs']} GB/s ({pk['src']})",
-                                  traffic_for("ternary_gemv_lut", "ternary_neural_net_b200/csrc/ternary.cu"),
+                                  traffic_for("ternary_gemv_c5", "ternary_neural_net_b200/csrc/ternary.cu"),
                                   frac_of_read_stream=gbs1 / pk["read_gbs"] if pk.get("read_gbs") else None),
                 roofline_m64=roofline("tensor", fl64 / (ms64 * 1e-3) / 1e12, bf16, "TFLOP/s",
                                       "ternary GEMM m = 64 (tcgen05 kind::f16)",
@@ -1059,14 +1054,14 @@ def main(argv=None):
                          f"512 MiB of outputs, so every step starts cold",
                    "parallelism": f"replicas x{N} (independent problems per GPU)"},
         "roofline": {"bound": "tensor",
-                     "kernel": "binary_gemm_tcp_kernel (bnn_binary_gemm AUTO at two tiles or more per SM): persistent "
-                               "CTAs, TMA-fed packed chunks -> 0/1 bytes in swizzled smem, tcgen05.mma kind::i8 into "
-                               "double-buffered tensor memory, epilogue warps overlapping the next tile",
+                     "kernel": "binary_gemm_tc_kernel<256,1> (bnn_binary_gemm AUTO for m > 128 with 3/4 of a wave "
+                               "of 128x256 tiles or more): TMA-fed packed chunks -> 0/1 bytes in swizzled smem, "
+                               "tcgen05.mma kind::i8 into tensor memory, epilogue by the producer warps",
                      "achieved": achieved, "peak": int8_peak, "unit": "TOP/s", "frac": achieved / int8_peak,
                      "achieved_basis": "2 ops x M*N*K per launch / the timed region's duration / K (the step is "
                                        "this one kernel; CUDA events on the launching stream)",
                      "kernel_ms": head["kernel_ms"], "kernel_ms_events": head["kernel_ms_events"],
-                     "traffic": traffic_for("binary_gemm_tcp_m8192", "ternary_neural_net_b200/csrc/binary_gemm_tc.cu"),
+                     "traffic": traffic_for("binary_gemm_tc_256x1", "ternary_neural_net_b200/csrc/binary_gemm_tc.cu"),
                      "peak_basis": f"int8 dense tensor peak = bf16 {peaks['bf16_tflops']} TFLOP/s x 2 (nominal "
                                    f"int8:bf16 ratio 4.5:2.25 PFLOP/s), {peak_src} (burst figure: a kernel timed "
                                    f"alone)"},

@@ -178,122 +178,6 @@ void dispatch_gemv(const uint64_t* xp, const uint64_t* wp, const float* alpha, i
 }
 
 // ---------------------------------------------------------------------------
-// m = 1 with 16-byte aligned rows of at most 256 words: the weight stream
-// staged by bulk copies.  Each CTA (one per SM) owns a contiguous block of
-// rows, i.e. a contiguous range of bytes, and one thread streams it into a
-// ring of kGvStages chunks of about 32 KiB with cp.async.bulk completing on an
-// mbarrier, so that about 100 KiB per SM are in flight with a handful of
-// instructions; the eight warps take the rows of each landed chunk (a row is
-// read from shared memory by its 32 lanes, 16 bytes each per 64-word pass,
-// against the activation words held in registers), add the popcounts by a
-// shuffle tree and write dot and alpha * dot.  The buffer of a chunk is
-// refilled once every warp has passed the barrier after it.  The weights'
-// first chunks are requested before the programmatic-launch wait.
-// ---------------------------------------------------------------------------
-constexpr int kGvThreads = 512;
-constexpr int kGvStages = 4;
-constexpr int kGvChunkBytes = 32 * 1024;
-
-__device__ __forceinline__ bool gv_wait(uint32_t bar, uint32_t parity) {
-  uint64_t t0;
-  asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t0));
-  while (true) {
-    uint32_t ok;
-    asm volatile("{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
-                 : "=r"(ok)
-                 : "r"(bar), "r"(parity)
-                 : "memory");
-    if (ok) return true;
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
-    if (t - t0 > 1000000000ull) return false;  // one second
-  }
-}
-
-template <int PASSES>
-__global__ void __launch_bounds__(kGvThreads, 1)
-binary_gemv_bulk_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restrict__ wp,
-                        const float* __restrict__ alpha, int64_t n, int k, int kw, int rows_chunk,
-                        int32_t* __restrict__ dots, float* __restrict__ out, unsigned int* __restrict__ errors) {
-  extern __shared__ __align__(128) uint8_t gsm[];  // kGvStages chunks of rows_chunk rows
-  __shared__ __align__(8) uint64_t full[kGvStages];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t r0 = n * blockIdx.x / gridDim.x, r1 = n * (blockIdx.x + 1) / gridDim.x;
-  const int nch = static_cast<int>((r1 - r0 + rows_chunk - 1) / rows_chunk);
-  const uint32_t row_bytes = static_cast<uint32_t>(kw) * 8u;
-  const uint32_t chunk_bytes = static_cast<uint32_t>(rows_chunk) * row_bytes;
-  auto bar = [&](int st) { return static_cast<uint32_t>(__cvta_generic_to_shared(&full[st])); };
-  auto issue = [&](int c) {  // chunk c of this CTA's rows into buffer c % kGvStages
-    const int64_t first = r0 + static_cast<int64_t>(c) * rows_chunk;
-    const int64_t rows = r1 - first < rows_chunk ? r1 - first : rows_chunk;
-    const uint32_t bytes = static_cast<uint32_t>(rows) * row_bytes;
-    const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(gsm + (c % kGvStages) * chunk_bytes));
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar(c % kGvStages)), "r"(bytes)
-                 : "memory");
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
-                 "l"(wp + first * kw), "r"(bytes), "r"(bar(c % kGvStages))
-                 : "memory");
-  };
-  if (tid == 0) {
-    for (int i = 0; i < kGvStages; ++i) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(bar(i)));
-    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-  }
-  __syncthreads();
-  if (tid == 0)
-    for (int c = 0; c < nch && c < kGvStages; ++c) issue(c);  // weights before the wait
-  bnn::pdl_trigger();
-  bnn::pdl_wait();  // x may come from the kernel ahead
-  ulonglong2 xv[PASSES];
-#pragma unroll
-  for (int p = 0; p < PASSES; ++p) {
-    const int w = 2 * (32 * p + lane);
-    xv[p] = w < kw ? __ldg(reinterpret_cast<const ulonglong2*>(xp + w)) : make_ulonglong2(0, 0);
-  }
-  constexpr int kWarps = kGvThreads / 32;
-  int c = 0;
-  for (; c < nch; ++c) {
-    const int st = c % kGvStages;
-    const int64_t first = r0 + static_cast<int64_t>(c) * rows_chunk;
-    const int rows = static_cast<int>(r1 - first < rows_chunk ? r1 - first : rows_chunk);
-    // the scales of this warp's rows of the chunk (lane i: row warp + kWarps i), loaded before the wait
-    float a_lane = 0.0f;
-    if (out && warp + kWarps * lane < rows) a_lane = __ldg(alpha + first + warp + kWarps * lane);
-    const bool ok = gv_wait(bar(st), static_cast<uint32_t>((c / kGvStages) & 1));
-    if (!__syncthreads_and(ok)) break;  // the chunk did not land in time: every thread stops here
-    const uint8_t* buf = gsm + st * chunk_bytes;
-    for (int rr = warp, i = 0; rr < rows; rr += kWarps, ++i) {
-      uint32_t acc = 0;
-#pragma unroll
-      for (int p = 0; p < PASSES; ++p) {
-        const int w = 2 * (32 * p + lane);
-        if (w < kw) {
-          const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(buf + rr * row_bytes + 8u * static_cast<uint32_t>(w));
-          acc += __popcll(v.x ^ xv[p].x) + __popcll(v.y ^ xv[p].y);
-        }
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-      const float a = __shfl_sync(0xffffffffu, a_lane, i & 31);
-      if (lane == 0) {
-        const int64_t row = first + rr;
-        const int32_t d = k - 2 * static_cast<int32_t>(acc);
-        if (dots) dots[row] = d;
-        if (out) out[row] = (i < 32 ? a : __ldg(alpha + row)) * static_cast<float>(d);
-      }
-    }
-    __syncthreads();  // every warp is done with this buffer
-    if (tid == 0 && c + kGvStages < nch) issue(c + kGvStages);
-  }
-  if (c < nch) {  // stopped early: no copy may still be in flight when the CTA retires
-    if (tid == 0) {
-      if (errors) atomicAdd(errors, 1u);
-      for (int cc = c; cc < nch && cc < c + kGvStages; ++cc) gv_wait(bar(cc % kGvStages), static_cast<uint32_t>((cc / kGvStages) & 1));
-    }
-    __syncthreads();
-  }
-}
-
-// ---------------------------------------------------------------------------
 // tiled kernel
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void cp_async_16(void* smem, const void* gmem, bool valid) {
@@ -689,35 +573,6 @@ extern "C" bnn_status bnn_binary_gemm_algo(const uint64_t* xp, const uint64_t* w
   if (algo == BNN_ALGO_MMA_S8 || (algo == BNN_ALGO_AUTO && m > 8)) {
     return vec2 ? dispatch_mma<2>(xp, wp, alpha, m, n, ki, kw, dots, out, s)
                 : dispatch_mma<1>(xp, wp, alpha, m, n, ki, kw, dots, out, s);
-  }
-  // large weight streams only (at least 4 MiB: about 28 KiB per SM); smaller ones are launch-latency bound
-  if (m == 1 && vec2 && kw > 0 && kw <= 256 && algo == BNN_ALGO_AUTO && n * kw >= (int64_t{1} << 19)) {
-    const int rows_chunk = kGvChunkBytes / (8 * kw) < 1 ? 1 : kGvChunkBytes / (8 * kw);
-    const int64_t sms = bnn::sm_count();
-    const int64_t want = (n + rows_chunk - 1) / rows_chunk;  // at least one chunk per CTA
-    const int grid = static_cast<int>(want < sms ? want : sms);
-    const size_t smem = static_cast<size_t>(kGvStages) * rows_chunk * kw * 8;
-    unsigned int* errors = bnn::device_error_counter();
-    cudaError_t e;
-    if (kw <= 64) {
-      BNN_TRY(bnn::ensure_smem(binary_gemv_bulk_kernel<1>, smem));
-      e = bnn::launch_pdl(binary_gemv_bulk_kernel<1>, dim3(grid), dim3(kGvThreads), smem, s, 1, xp, wp, alpha, n, ki,
-                          kw, rows_chunk, dots, out, errors);
-    } else if (kw <= 128) {
-      BNN_TRY(bnn::ensure_smem(binary_gemv_bulk_kernel<2>, smem));
-      e = bnn::launch_pdl(binary_gemv_bulk_kernel<2>, dim3(grid), dim3(kGvThreads), smem, s, 1, xp, wp, alpha, n, ki,
-                          kw, rows_chunk, dots, out, errors);
-    } else if (kw <= 192) {
-      BNN_TRY(bnn::ensure_smem(binary_gemv_bulk_kernel<3>, smem));
-      e = bnn::launch_pdl(binary_gemv_bulk_kernel<3>, dim3(grid), dim3(kGvThreads), smem, s, 1, xp, wp, alpha, n, ki,
-                          kw, rows_chunk, dots, out, errors);
-    } else {
-      BNN_TRY(bnn::ensure_smem(binary_gemv_bulk_kernel<4>, smem));
-      e = bnn::launch_pdl(binary_gemv_bulk_kernel<4>, dim3(grid), dim3(kGvThreads), smem, s, 1, xp, wp, alpha, n, ki,
-                          kw, rows_chunk, dots, out, errors);
-    }
-    if (e != cudaSuccess) return bnn::cuda_fail(e);
-    return bnn::check_launch();
   }
   if (m <= 8) {
     if (vec2) dispatch_gemv<2>(xp, wp, alpha, static_cast<int>(m), n, ki, kw, dots, out, s);

@@ -113,35 +113,6 @@ __device__ __forceinline__ void expand_word(uint8_t* dst_row, uint32_t swz, int 
   }
 }
 
-// The same mapping with the bit left in the top bit of its byte (0 or 0x80):
-// per 4 bytes one multiply by a power of two and one AND, where expand_word
-// takes a shift and an AND (both on the integer ALU).  The multipliers
-// mul[t - 1] = 2^t arrive as run-time values, so the multiplies stay integer
-// multiply-adds on the FMA pipe and the two pipes share the expansion.  As
-// signed int8 both operands then hold 0 or -128, every product is 0 or
-// +16384, and the int32 accumulator holds 16384 popcount(a AND b) -- exact
-// while the tile's K stays below 2^17 bits (2^31 / 16384).
-__device__ __forceinline__ void expand_word_hi(uint8_t* dst_row, uint32_t swz, int part, uint64_t cw,
-                                               const uint32_t (&mul)[7]) {
-#pragma unroll
-  for (int hh = 0; hh < 2; ++hh) {
-    const int h = 2 * part + hh;
-    const uint32_t hw = static_cast<uint32_t>(cw >> (32 * hh));
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      // byte j of word s: bit 8j + 4q + s of hw, moved up to bit 7 of the byte
-      uint32_t v[4];
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const int t = 7 - 4 * q - w;
-        v[w] = (t == 0 ? hw : hw * mul[t > 0 ? t - 1 : 0]) & 0x80808080u;
-      }
-      const uint32_t chunk = static_cast<uint32_t>(2 * h + q);
-      *reinterpret_cast<uint4*>(dst_row + ((chunk ^ swz) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
-    }
-  }
-}
-
 // grid: x = KS * (weight tiles of 128 rows), y = activation tiles of BN rows;
 // clusters of KS CTAs along x
 template <int BN, int KS, bool TMA, bool WIDE>
@@ -500,335 +471,6 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(BN));
 }
 
-// ---------------------------------------------------------------------------
-// Persistent variant for GEMMs with many tiles (at least two per SM): one CTA
-// per SM walks its tiles (128 weight rows x 256 activation rows; tile t of the
-// CTA is blockIdx.x + t gridDim.x, consecutive CTAs on the same weight rows),
-// and the epilogue of one tile overlaps the mainloop of the next.  Roles as
-// above (768 producer threads, an MMA thread, a TMA thread), plus four
-// epilogue warps of their own, one per quarter of the tensor-memory lanes.
-// The accumulator is double-buffered in tensor memory (2 x 256 columns): the
-// MMA thread commits buffer t % 2 to acc_full after a tile's last stage and
-// waits on acc_empty before reusing it; the epilogue warps arrive on
-// acc_empty once they have read it.  The stage ring, the chunk ring and their
-// mbarrier phases run on across tiles.  The producers' row popcounts of a
-// tile go to a double-buffered array, published with pop_full (the producers
-// first wait, on acc_empty, for the epilogue that read that buffer two tiles
-// back).  Every wait is bounded as above; a wait that runs out stops every
-// role and leaves the outputs unspecified.
-// ---------------------------------------------------------------------------
-constexpr int kPBN = 256;                                   // activation rows per tile
-constexpr int kPRows = kTm + kPBN;                          // stacked rows per stage
-constexpr uint32_t kPStageBytes = kPRows * 128u;            // one expanded stage (48 KiB)
-constexpr uint32_t kPChunkBytes = kPRows * 16u * kChunkStages;  // one packed chunk (24 KiB)
-constexpr int kPS = 3, kPP = 2;                             // expanded stages, packed chunks
-constexpr int kPProducers = 2 * kPRows;                     // 768
-constexpr int kPMmaWarp = kPProducers / 32, kPTmaWarp = kPMmaWarp + 1, kPEpiWarp0 = kPMmaWarp + 2;
-constexpr int kPThreads = kPProducers + 64 + 128;          // + MMA warp + TMA warp + 4 epilogue warps
-constexpr uint32_t kPSmem = kPS * kPStageBytes + kPP * kPChunkBytes + 2u * kPProducers * 4u;  // + popcounts
-static_assert(kPSmem + 1024 <= 227u * 1024u, "persistent tile fits shared memory");
-
-// HI: bits expanded to 0/0x80 bytes (expand_word_hi; k < 2^17), else 0/1 bytes.
-// mul_one is 1 at run time (the base of expand_word_hi's multipliers).
-template <bool HI>
-__global__ void __launch_bounds__(kPThreads, 1)
-binary_gemm_tcp_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
-                       const float* __restrict__ alpha, const float* __restrict__ bias, int64_t m, int64_t n, int k,
-                       int kw, int64_t mtiles, int64_t ntiles, int32_t* __restrict__ dots, float* __restrict__ out,
-                       uint32_t* __restrict__ next, int64_t next_w32, uint32_t wait_limit, uint32_t mul_one) {
-  using bnn::tc::mbar_drain;
-  using bnn::tc::mbar_wait;
-  using bnn::tc::mbar_wait_idle;
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full_bar[kPS];
-  __shared__ __align__(8) uint64_t empty_bar[kPS];
-  __shared__ __align__(8) uint64_t chunk_full[kPP];
-  __shared__ __align__(8) uint64_t chunk_empty[kPP];
-  __shared__ __align__(8) uint64_t acc_full[2];
-  __shared__ __align__(8) uint64_t acc_empty[2];
-  __shared__ __align__(8) uint64_t pop_full[2];
-  __shared__ __align__(8) uint64_t done_bar;
-  __shared__ uint32_t tmem_holder;
-  __shared__ volatile int abort_flag;
-  uint8_t* const smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint8_t* const chunks = smem + kPS * kPStageBytes;
-  int* const pop_part = reinterpret_cast<int*>(chunks + kPP * kPChunkBytes);  // [2][kPProducers]
-
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5;
-  const int nst = (kw + 1) / 2;                          // 128-bit stages per tile
-  const int nch = (nst + kChunkStages - 1) / kChunkStages;
-  const int64_t tiles = mtiles * ntiles;
-  const uint32_t smem_base = smem_u32(smem);
-
-  if (tid == 0) {
-    for (int i = 0; i < kPS; ++i) {
-      bnn::tc::mbar_init(smem_u32(&full_bar[i]), kPProducers);
-      bnn::tc::mbar_init(smem_u32(&empty_bar[i]), 1);
-    }
-    for (int i = 0; i < kPP; ++i) {
-      bnn::tc::mbar_init(smem_u32(&chunk_full[i]), 1);
-      bnn::tc::mbar_init(smem_u32(&chunk_empty[i]), kPProducers);
-    }
-    for (int i = 0; i < 2; ++i) {
-      bnn::tc::mbar_init(smem_u32(&acc_full[i]), 1);
-      bnn::tc::mbar_init(smem_u32(&acc_empty[i]), 128);
-      bnn::tc::mbar_init(smem_u32(&pop_full[i]), kPProducers);
-    }
-    bnn::tc::mbar_init(smem_u32(&done_bar), 1);
-    abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-  }
-  if (tid == kPTmaWarp * 32) {
-    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tmap_w)) : "memory");
-    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
-  }
-  if (warp == kPMmaWarp) {  // the MMA warp owns the tensor memory: two 256-column accumulators
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(&tmem_holder)),
-                 "r"(2 * kPBN));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::);
-  }
-  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
-  __syncthreads();
-  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-  const uint32_t tmem = tmem_holder;
-  bnn::pdl_trigger();
-
-  auto tile_rows = [&](int64_t t, int64_t& j0, int64_t& i0) {
-    j0 = (t / mtiles) * kTm;
-    i0 = (t % mtiles) * kPBN;
-  };
-
-  if (tid < kPProducers) {
-    // ------------------------------------------------------------ producers
-    const int r2 = tid >> 1, part = tid & 1;
-    const int row = r2 < kTm ? r2 : r2 - kTm;
-    const uint32_t row_off = static_cast<uint32_t>(r2) * 128u;
-    const uint32_t swz = static_cast<uint32_t>(row & 7);
-    const uint32_t rd_off = static_cast<uint32_t>(r2) * 64u + 8u * static_cast<uint32_t>(part);
-    const uint32_t rd_swz = static_cast<uint32_t>((r2 >> 1) & 3);
-    uint32_t mul[7];
-#pragma unroll
-    for (int t = 0; t < 7; ++t) mul[t] = mul_one << (t + 1);
-    int64_t gs = 0, gc = 0;  // stages and chunks consumed so far (all tiles)
-    bool ok = true;
-    int ti = 0;
-    for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++ti) {
-      int my_pop = 0;
-      for (int j = 0; j < nst; ++j, ++gs) {
-        const int s = j % kChunkStages;
-        const int64_t cc = gc + j / kChunkStages;
-        const int pb = static_cast<int>(cc % kPP);
-        // waits sleep between polls: the epilogue warps of the previous tile need the issue slots
-        if (s == 0 && !(wait_limit ? mbar_wait(smem_u32(&chunk_full[pb]), static_cast<uint32_t>((cc / kPP) & 1),
-                                               &abort_flag, &g_bnn_device_errors, wait_limit)
-                                   : mbar_wait_idle(smem_u32(&chunk_full[pb]), static_cast<uint32_t>((cc / kPP) & 1),
-                                                    &abort_flag, &g_bnn_device_errors))) {
-          ok = false;
-          break;
-        }
-        const uint64_t cw = *reinterpret_cast<const uint64_t*>(
-            chunks + pb * kPChunkBytes + rd_off + ((static_cast<uint32_t>(s) ^ rd_swz) << 4));
-        if (s == kChunkStages - 1 || j == nst - 1) mbar_arrive(smem_u32(&chunk_empty[pb]));
-        const int b = static_cast<int>(gs % kPS);
-        if (gs >= kPS && !(wait_limit ? mbar_wait(smem_u32(&empty_bar[b]), static_cast<uint32_t>((gs / kPS + 1) & 1),
-                                                  &abort_flag, &g_bnn_device_errors, wait_limit)
-                                      : mbar_wait_idle(smem_u32(&empty_bar[b]), static_cast<uint32_t>((gs / kPS + 1) & 1),
-                                                       &abort_flag, &g_bnn_device_errors))) {
-          ok = false;
-          break;
-        }
-        my_pop += __popcll(cw);
-        if constexpr (HI) expand_word_hi(smem + b * kPStageBytes + row_off, swz, part, cw, mul);
-        else expand_word(smem + b * kPStageBytes + row_off, swz, part, cw);
-        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-        mbar_arrive(smem_u32(&full_bar[b]));
-      }
-      gc += nch;
-      if (!ok) break;
-      const int tb = ti & 1;
-      // the epilogue two tiles back has read this popcount buffer
-      if (ti >= 2 && !mbar_wait(smem_u32(&acc_empty[tb]), static_cast<uint32_t>(((ti >> 1) - 1) & 1), &abort_flag,
-                                &g_bnn_device_errors, wait_limit)) {
-        ok = false;
-        break;
-      }
-      pop_part[tb * kPProducers + tid] = my_pop;
-      mbar_arrive(smem_u32(&pop_full[tb]));
-    }
-  } else if (tid == kPMmaWarp * 32) {
-    // ------------------------------------------------------------ MMA issue
-    const uint32_t idesc = (2u << 4) | (1u << 7) | (1u << 10) | ((static_cast<uint32_t>(kPBN) >> 3) << 17) |
-                           ((static_cast<uint32_t>(kTm) >> 4) << 24);
-    int64_t gs = 0;
-    int ti = 0;
-    bool ok = true;
-    for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++ti) {
-      const int tb = ti & 1;
-      if (ti >= 2 && !mbar_wait_idle(smem_u32(&acc_empty[tb]), static_cast<uint32_t>(((ti >> 1) - 1) & 1),
-                                     &abort_flag, &g_bnn_device_errors))
-        break;
-      asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-      const uint32_t d = tmem + static_cast<uint32_t>(tb * kPBN);
-      for (int j = 0; j < nst; ++j, ++gs) {
-        const int b = static_cast<int>(gs % kPS);
-        if (!mbar_wait(smem_u32(&full_bar[b]), static_cast<uint32_t>((gs / kPS) & 1), &abort_flag,
-                       &g_bnn_device_errors, wait_limit)) {
-          ok = false;
-          break;
-        }
-        asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-        const uint64_t ad = sw128_desc(smem_base + b * kPStageBytes);
-        const uint64_t bd = sw128_desc(smem_base + b * kPStageBytes + kTm * 128u);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-          asm volatile(
-              "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
-              "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
-              "l"(ad + static_cast<uint64_t>(2 * kk)), "l"(bd + static_cast<uint64_t>(2 * kk)), "r"(idesc), "r"(acc));
-        }
-        bnn::tc::mma_commit(smem_u32(&empty_bar[b]));
-      }
-      if (!ok) break;
-      bnn::tc::mma_commit(smem_u32(&acc_full[tb]));  // the tile's accumulator is final when this arrives
-    }
-    bnn::tc::mma_commit(smem_u32(&done_bar));  // every MMA issued above has completed
-  } else if (tid == kPTmaWarp * 32) {
-    // ------------------------------------------------------------ TMA copies
-    int64_t gc = 0;
-    bool waited = false;
-    bool ok = true;
-    for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-      int64_t j0, i0;
-      tile_rows(t, j0, i0);
-      for (int c = 0; c < nch; ++c, ++gc) {
-        const int pb = static_cast<int>(gc % kPP);
-        if (gc >= kPP && !mbar_wait_idle(smem_u32(&chunk_empty[pb]), static_cast<uint32_t>((gc / kPP + 1) & 1),
-                                         &abort_flag, &g_bnn_device_errors)) {
-          ok = false;
-          break;
-        }
-        const uint32_t dst = smem_u32(chunks + pb * kPChunkBytes);
-        const uint32_t bar = smem_u32(&chunk_full[pb]);
-        const int cx = 2 * kChunkStages * c;
-        mbar_expect_tx(bar, kPChunkBytes);
-        tma_load_2d(dst, &tmap_w, cx, static_cast<int>(j0), bar);
-        if (!waited) {  // the weights do not depend on the kernel ahead; the activations may
-          bnn::pdl_wait();
-          waited = true;
-        }
-        tma_load_2d(dst + kTm * 16u * kChunkStages, &tmap_x, cx, static_cast<int>(i0), bar);
-      }
-    }
-    // no copy may be in flight when the CTA retires
-    for (int64_t g = gc - kPP; g < gc; ++g)
-      if (g >= 0) mbar_drain(smem_u32(&chunk_full[g % kPP]), static_cast<uint32_t>((g / kPP) & 1), &g_bnn_device_errors);
-  } else if (warp >= kPEpiWarp0) {
-    // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;                       // tensor-memory lane quarter this warp may access
-    const int erow = 32 * q + (tid & 31);         // weight row of the tile
-    const uint32_t lane_field = static_cast<uint32_t>(32 * q) << 16;
-    const bool need_y = out || next;
-    int ti = 0;
-    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++ti) {
-      const int tb = ti & 1;
-      const uint32_t par = static_cast<uint32_t>((ti >> 1) & 1);
-      if (!mbar_wait_idle(smem_u32(&acc_full[tb]), par, &abort_flag, &g_bnn_device_errors) ||
-          !mbar_wait_idle(smem_u32(&pop_full[tb]), par, &abort_flag, &g_bnn_device_errors))
-        break;
-      asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-      int64_t j0, i0;
-      tile_rows(t, j0, i0);
-      const int* pops = pop_part + tb * kPProducers;
-      const int64_t jrow = j0 + erow;
-      const bool jlive = jrow < n;
-      const float a_j = (need_y && jlive) ? __ldg(alpha + jrow) : 0.0f;
-      const float b_j = (bias && jlive) ? __ldg(bias + jrow) : 0.0f;
-      const int base = k - 2 * (pops[2 * erow] + pops[2 * erow + 1]);
-      const int64_t half = (j0 + 32 * q) / 32;
-      const bool pack = next && half < next_w32;  // uniform across the warp
-      const uint32_t taddr = tmem + lane_field + static_cast<uint32_t>(tb * kPBN);
-      for (int c0 = 0; c0 < kPBN; c0 += 16) {
-        uint32_t r[16];
-        if (nst > 0) {
-          tmem_ld16(taddr + static_cast<uint32_t>(c0), r);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int c = 0; c < 16; ++c) r[c] = 0u;
-        }
-        const int64_t rows_left = m - (i0 + c0);
-        const int nc = rows_left <= 0 ? 0 : (rows_left < 16 ? static_cast<int>(rows_left) : 16);
-        const int64_t off = (i0 + c0) * n + jrow;
-        int32_t* dp = dots ? dots + off : nullptr;
-        float* op = out ? out + off : nullptr;
-        uint32_t* np = pack ? next + (i0 + c0) * next_w32 + half : nullptr;
-        const bool store = abort_flag == 0;
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int px = 2 * (kTm + c0 + c);
-          const int32_t s4 = HI ? static_cast<int32_t>(r[c] >> 12) : 4 * static_cast<int32_t>(r[c]);  // 4 popc(a&b)
-          const int32_t dv = base - 2 * (pops[px] + pops[px + 1]) + s4;
-          const float y0 = __fmul_rn(a_j, static_cast<float>(dv));
-          const float y = bias ? __fadd_rn(y0, b_j) : y0;
-          if (store && c < nc && jlive) {
-            if (dp) *dp = dv;
-            if (op) *op = y;
-          }
-          if (np) {
-            const unsigned bits = __ballot_sync(0xffffffffu, jlive && !(y > 0.0f));
-            if (store && (tid & 31) == 0 && c < nc) *np = bits;
-            np += next_w32;
-          }
-          dp += n;
-          op += n;
-        }
-      }
-      asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
-      mbar_arrive(smem_u32(&acc_empty[tb]));
-    }
-  }
-  __syncwarp();
-  if (tid == kPMmaWarp * 32) mbar_drain(smem_u32(&done_bar), 0u, &g_bnn_device_errors);
-  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
-  __syncthreads();
-  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-  if (warp == kPMmaWarp)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(2 * kPBN));
-}
-
-bnn_status launch_tcp(const uint64_t* xp, const uint64_t* wp, const float* alpha, const float* bias, int64_t m,
-                      int64_t n, int k, int kw, int32_t* dots, float* out, uint64_t* next, cudaStream_t s,
-                      bool* launched) {
-  *launched = false;
-  if (kw <= 0 || kw % 2 != 0 || !bnn::aligned(xp, 16) || !bnn::aligned(wp, 16) || n >= (1LL << 31) ||
-      m >= (1LL << 31))
-    return BNN_OK;  // no TMA: the caller takes the per-tile kernel
-  CUtensorMap tw, tx;
-  if (!bnn::encode_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT64, wp, static_cast<uint64_t>(kw),
-                           static_cast<uint64_t>(n), static_cast<uint64_t>(kw) * 8u, 2 * kChunkStages, kTm,
-                           CU_TENSOR_MAP_SWIZZLE_64B) ||
-      !bnn::encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT64, xp, static_cast<uint64_t>(kw),
-                           static_cast<uint64_t>(m), static_cast<uint64_t>(kw) * 8u, 2 * kChunkStages, kPBN,
-                           CU_TENSOR_MAP_SWIZZLE_64B))
-    return BNN_OK;
-  const int64_t mtiles = (m + kPBN - 1) / kPBN, ntiles = (n + kTm - 1) / kTm;
-  const int64_t sms = bnn::sm_count();
-  const int64_t grid = mtiles * ntiles < sms ? mtiles * ntiles : sms;
-  const size_t smem = static_cast<size_t>(kPSmem) + 1024;
-  const bool hi = 64 * static_cast<int64_t>(kw) < (int64_t{1} << 17);  // 16384 popc(a AND b) fits int32
-  auto kern = hi ? binary_gemm_tcp_kernel<true> : binary_gemm_tcp_kernel<false>;
-  BNN_TRY(bnn::ensure_smem(kern, smem));
-  const cudaError_t e = bnn::launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(kPThreads),
-                                        smem, s, 1, tw, tx, alpha, bias, m, n, k, kw, mtiles, ntiles, dots, out,
-                                        reinterpret_cast<uint32_t*>(next), 2 * bnn::words64(n),
-                                        g_wait_limit.load(), 1u);
-  if (e != cudaSuccess) return bnn::cuda_fail(e);
-  *launched = true;
-  return bnn::check_launch();
-}
-
 template <int BN, int KS, bool WIDE = false>
 bnn_status launch_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha, const float* bias, int64_t m,
                      int64_t n, int k, int kw, int32_t* dots, float* out, uint64_t* next, cudaStream_t s) {
@@ -877,11 +519,6 @@ bnn_status binary_gemm_tc(const uint64_t* xp, const uint64_t* wp, const float* a
   const int64_t sms = sm_count();
   const int ktiles = (kw + 1) / 2;
   if (m > 128) {
-    if (wt * ((m + 255) / 256) >= 2 * sms) {  // two tiles or more per SM: the persistent kernel
-      bool launched = false;
-      const bnn_status st = launch_tcp(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s, &launched);
-      if (st != BNN_OK || launched) return st;
-    }
     if (4 * wt * ((m + 255) / 256) >= 3 * sms)
       return launch_tc<256, 1>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
     const int64_t t128 = wt * ((m + 127) / 128);

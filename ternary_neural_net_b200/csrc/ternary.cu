@@ -307,236 +307,6 @@ size_t rows_smem_bytes(int64_t kt) {
 }
 
 // ---------------------------------------------------------------------------
-// Ternary GEMV, m = 1, k <= 4160: activation tables over 4 + 3 + 3 trits.
-//
-// A word's ten trits split into a 4-trit group (digits 0..3, the word mod 81),
-// a 3-trit group (digits 4..6) and a 3-trit group (digits 7..9).  For word
-// position j of the rows, table A_j holds, for each of the 81 digit patterns
-// e of the first group, the partial dot sum_{i<4} x[10j+i] (d_i(e) - 1); B_j
-// and C_j (27 patterns each) the same for the other two groups.  A word then
-// costs three shared-memory loads and three adds: y = scale * sum_j
-// (A_j[e_A] + B_j[e_B] + C_j[e_C]).  The group codes come from two exact
-// multiply-shift divisions (by 81, then by 27; the constants are checked
-// against every word at compile time below).
-//
-// One CTA per SM holds all 135 tables of the row length (135 x ktp floats,
-// ktp = kt rounded up to 32: 218 KiB at k = 4096) and takes a contiguous
-// block of rows.  Work unit = (row, pass): a warp's 32 lanes load 32
-// consecutive 32-bit pairs of words of one row (128 coalesced bytes), so
-// lane l of pass p holds words j = 64p + 2l + t, t = 0, 1.  Tables are stored
-// entry-major with word column sigma(j) = 64p + t L + l (L = the pass's lane
-// count), so for each of the six loads of a unit the 32 lanes read 32
-// consecutive columns: 32 different banks, whatever patterns they decode.
-// Lanes past the row's end decode the all-zero-trit pair, whose entries are 0
-// in every column.  Each unit's lane sums are added by a shuffle tree and
-// stored per (row, pass); the rows' pass sums are added in pass order, so the
-// result does not depend on the launch shape.  Eight units per warp are in
-// flight (their words loaded a group ahead); the first group is loaded
-// before the programmatic-launch wait (weights do not depend on the kernel
-// ahead), the tables are built after it (they depend on x).
-// ---------------------------------------------------------------------------
-constexpr int kLutThreads = 1024;
-constexpr int kLutMaxKt = 416;         // 32-bit pairs of words need kt even; 135 x 416 floats = 219.4 KiB
-constexpr int kLutRowsChunk = 256;     // rows whose unit sums are held at once
-constexpr int kLutMaxPasses = (kLutMaxKt / 2 + 31) / 32;
-constexpr int kLutMaxUnits = (kLutMaxPasses + 1) / 2;  // units (two passes each) per row
-constexpr int kLutGroup = 4;           // units per warp in flight (two 32-bit loads each)
-constexpr uint32_t kDiv81Mul = 25891u, kDiv81Shift = 21;  // floor(w / 81) for w < 3^10
-constexpr uint32_t kDiv27Mul = 607u, kDiv27Shift = 14;    // floor(q / 27) for q < 3^6
-constexpr uint32_t kZeroPair = 29524u | (29524u << 16);   // two all-zero-trit words
-
-constexpr bool lut_divisions_exact() {
-  for (uint32_t w = 0; w < 59049u; ++w)
-    if ((w * kDiv81Mul) >> kDiv81Shift != w / 81u) return false;
-  for (uint32_t q = 0; q < 729u; ++q)
-    if ((q * kDiv27Mul) >> kDiv27Shift != q / 27u) return false;
-  return true;
-}
-static_assert(lut_divisions_exact(), "multiply-shift division constants");
-
-__host__ __device__ constexpr int lut_pitch(int kt) { return (kt + 31) & ~31; }
-
-size_t lut_smem_bytes(int64_t kt) {
-  return static_cast<size_t>(135 * lut_pitch(static_cast<int>(kt)) + kLutRowsChunk * kLutMaxUnits) * sizeof(float);
-}
-
-__device__ __forceinline__ float bf16f(const uint16_t* x, int e, int k) {
-  return e < k ? __uint_as_float(static_cast<uint32_t>(__ldg(x + e)) << 16) : 0.0f;
-}
-
-// One word's three table entries, summed: colA/colB/colC are the byte
-// addresses of the word's column in tables A, B and C, stride one entry row.
-__device__ __forceinline__ float lut_word(uint32_t w, uint32_t colA, uint32_t colB, uint32_t colC, uint32_t stride) {
-  const uint32_t q = (w * kDiv81Mul) >> kDiv81Shift;   // digits 4..9
-  const uint32_t eA = w - 81u * q;                     // digits 0..3
-  const uint32_t eC = (q * kDiv27Mul) >> kDiv27Shift;  // digits 7..9
-  const uint32_t eB = q - 27u * eC;                    // digits 4..6
-  float a, b, c;
-  asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(a) : "r"(colA + eA * stride));
-  asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(b) : "r"(colB + eB * stride));
-  asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(c) : "r"(colC + eC * stride));
-  return (a + b) + c;
-}
-
-__global__ void __launch_bounds__(kLutThreads, 1)
-ternary_gemv_lut_kernel(const uint16_t* __restrict__ x, const uint32_t* __restrict__ packed2,
-                        const float* __restrict__ scale, int64_t n, int k, int kt, float* __restrict__ out,
-                        const float* __restrict__ bias) {
-  extern __shared__ float T[];  // [135][ktp] tables, then [kLutRowsChunk][units per row] unit sums
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int kWarps = kLutThreads / 32;
-  const int ktp = lut_pitch(kt);
-  const int kt2 = kt >> 1;                       // 32-bit pairs per row
-  const int passes = (kt2 + 31) >> 5;            // 32 pairs (64 words) per pass
-  const int upr = (passes + 1) >> 1;             // units per row: passes 2u and 2u + 1
-  const int l_last = kt2 - 32 * (passes - 1);    // lanes of the last pass
-  float* usum = T + 135 * ktp;
-  const int64_t r_begin = n * blockIdx.x / gridDim.x, r_end = n * (blockIdx.x + 1) / gridDim.x;
-  // warp-uniform walk over the units u = warp + kWarps i as (row, unit-of-row) pairs
-  const int d_row = kWarps / upr, d_unit = kWarps - d_row * upr;
-  auto advance = [&](int& rl, int& ur) {
-    ur += d_unit;
-    rl += d_row;
-    if (ur >= upr) {
-      ur -= upr;
-      ++rl;
-    }
-  };
-  bnn::pdl_trigger();
-
-  // this lane's pairs of unit (rl, ur): passes 2 ur and 2 ur + 1 (zero pairs past the row);
-  // offsets in 32 bits (the host keeps n * kt / 2 below 2^31)
-  auto fetch = [&](int64_t r_chunk, int rows, int rl, int ur, uint32_t& v0, uint32_t& v1) {
-    v0 = v1 = kZeroPair;
-    if (rl < rows) {
-      const int c = 64 * ur + lane;
-      const uint32_t* src = packed2 + static_cast<uint32_t>(static_cast<int>(r_chunk) + rl) * static_cast<uint32_t>(kt2) + c;
-      if (c < kt2) v0 = __ldcs(src);
-      if (c + 32 < kt2) v1 = __ldcs(src + 32);
-    }
-  };
-
-  int64_t r_chunk = r_begin;
-  int rows = static_cast<int>(r_end - r_begin < kLutRowsChunk ? r_end - r_begin : kLutRowsChunk);
-  int rl0 = warp / upr, ur0 = warp - rl0 * upr;  // the warp's first unit
-  uint32_t cur[kLutGroup][2];
-  int frl = rl0, fur = ur0;  // fetch cursor (runs kLutGroup units ahead of the compute cursor)
-#pragma unroll
-  for (int g = 0; g < kLutGroup; ++g) {
-    fetch(r_chunk, rows, frl, fur, cur[g][0], cur[g][1]);
-    advance(frl, fur);
-  }
-
-  bnn::pdl_wait();  // x may come from the kernel ahead
-  // Tables.  Task f = part * kt + column: parts 0..8 fill A's entries
-  // 9 part .. 9 part + 8, parts 9..11 B's, 12..14 C's.  Consecutive threads
-  // write consecutive columns of one entry row (distinct banks).
-  for (int f = tid; f < 15 * kt; f += kLutThreads) {
-    const int part = f / kt, c = f - part * kt;
-    const int p = c >> 6, o = c & 63;
-    const int L = kt2 - 32 * p < 32 ? kt2 - 32 * p : 32;
-    const int t = o >= L ? 1 : 0, l = o - t * L;
-    const int j = 64 * p + 2 * l + t;          // the word position stored in column c
-    const int e0 = 10 * j;
-    float lo[9];
-    float hi;
-    int row0;
-    if (part < 9) {                             // A: digits 0, 1 run over e_lo; digits 2, 3 fixed by part
-      const float x0 = bf16f(x, e0, k), x1 = bf16f(x, e0 + 1, k);
-      const float x2 = bf16f(x, e0 + 2, k), x3 = bf16f(x, e0 + 3, k);
-#pragma unroll
-      for (int v = 0; v < 9; ++v) lo[v] = x0 * static_cast<float>(v % 3 - 1) + x1 * static_cast<float>(v / 3 - 1);
-      hi = x2 * static_cast<float>(part % 3 - 1) + x3 * static_cast<float>(part / 3 - 1);
-      row0 = 9 * part;
-    } else {                                    // B (digits 4..6) or C (digits 7..9): last digit fixed by part
-      const int g = part < 12 ? 0 : 1, d = part - 9 - 3 * g;
-      const int b = e0 + 4 + 3 * g;
-      const float x0 = bf16f(x, b, k), x1 = bf16f(x, b + 1, k), x2 = bf16f(x, b + 2, k);
-#pragma unroll
-      for (int v = 0; v < 9; ++v) lo[v] = x0 * static_cast<float>(v % 3 - 1) + x1 * static_cast<float>(v / 3 - 1);
-      hi = x2 * static_cast<float>(d - 1);
-      row0 = 81 + 27 * g + 9 * d;
-    }
-    float* dst = T + row0 * ktp + c;
-#pragma unroll
-    for (int v = 0; v < 9; ++v) dst[v * ktp] = lo[v] + hi;
-  }
-  __syncthreads();
-
-  const uint32_t stride = 4u * static_cast<uint32_t>(ktp);
-  const uint32_t tA = static_cast<uint32_t>(__cvta_generic_to_shared(T));
-  const uint32_t offB = 81u * stride, offC = 108u * stride;
-  const uint32_t lane_full = 4u * static_cast<uint32_t>(lane);
-  const uint32_t lane_last = 4u * static_cast<uint32_t>(lane < l_last ? lane : l_last - 1);  // valid column
-  // the two words of pair v in pass p (warp-uniform p), added to acc
-  auto pass_sum = [&](uint32_t v, int p) -> float {
-    const bool last = p == passes - 1;
-    const uint32_t c0 = tA + 256u * static_cast<uint32_t>(p) + (last ? lane_last : lane_full);
-    const uint32_t c1 = c0 + 4u * static_cast<uint32_t>(last ? l_last : 32);
-    return lut_word(v & 0xFFFFu, c0, c0 + offB, c0 + offC, stride) +
-           lut_word(v >> 16, c1, c1 + offB, c1 + offC, stride);
-  };
-
-  while (true) {
-    int rl = rl0, ur = ur0;
-    while (rl < rows) {
-      uint32_t nxt[kLutGroup][2];
-#pragma unroll
-      for (int g = 0; g < kLutGroup; ++g) {
-        fetch(r_chunk, rows, frl, fur, nxt[g][0], nxt[g][1]);
-        advance(frl, fur);
-      }
-      float sum[kLutGroup];
-      int idx[kLutGroup];
-#pragma unroll
-      for (int g = 0; g < kLutGroup; ++g) {
-        idx[g] = -1;
-        sum[g] = 0.0f;
-        if (rl < rows) {  // warp-uniform: units past the chunk's rows cost nothing
-          idx[g] = rl * upr + ur;
-          const int p = 2 * ur;
-          sum[g] = pass_sum(cur[g][0], p);
-          if (p + 1 < passes) sum[g] += pass_sum(cur[g][1], p + 1);
-        }
-        advance(rl, ur);
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1)
-#pragma unroll
-        for (int g = 0; g < kLutGroup; ++g) sum[g] += __shfl_xor_sync(0xffffffffu, sum[g], off);
-      if (lane == 0) {
-#pragma unroll
-        for (int g = 0; g < kLutGroup; ++g)
-          if (idx[g] >= 0) usum[idx[g]] = sum[g];
-      }
-#pragma unroll
-      for (int g = 0; g < kLutGroup; ++g) {
-        cur[g][0] = nxt[g][0];
-        cur[g][1] = nxt[g][1];
-      }
-    }
-    __syncthreads();  // every unit sum of this chunk is stored
-    for (int r = tid; r < rows; r += kLutThreads) {
-      float acc = 0.0f;
-      for (int u = 0; u < upr; ++u) acc += usum[r * upr + u];
-      const int64_t gr = r_chunk + r;
-      out[gr] = bias ? __ldg(scale + gr) * acc + __ldg(bias + gr) : __ldg(scale + gr) * acc;
-    }
-    r_chunk += rows;
-    if (r_chunk >= r_end) break;
-    __syncthreads();  // unit sums read before the next chunk overwrites them
-    rows = static_cast<int>(r_end - r_chunk < kLutRowsChunk ? r_end - r_chunk : kLutRowsChunk);
-    frl = rl0;
-    fur = ur0;
-#pragma unroll
-    for (int g = 0; g < kLutGroup; ++g) {
-      fetch(r_chunk, rows, frl, fur, cur[g][0], cur[g][1]);
-      advance(frl, fur);
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------
 // Ternary GEMV, m = 1, k <= 4800: 5 + 5-trit activation tables, the row
 // length split over a cluster of kC5 CTAs.
 //
@@ -546,22 +316,38 @@ ternary_gemv_lut_kernel(const uint16_t* __restrict__ x, const uint32_t* __restri
 // a word costs two shared-memory loads and two adds.  The tables of a whole row
 // do not fit one SM (2 x 243 entries per word), so the kC5 CTAs of a cluster
 // take one slice of at most 96 word positions each and hold only that slice's
-// tables (two [243][96] float arrays, 182 KiB), and every CTA of the cluster
-// runs over the same block of rows: a warp takes whole rows, its 32 lanes
-// consecutive word positions (so a lookup's 32 lanes read 32 consecutive
-// columns: 32 banks), one 16-bit load per word, the next row's words in
-// registers while this row is added.  Each row's slice sum (a shuffle tree) is
-// stored in the CTA's shared memory; after a cluster barrier CTA q adds, for
-// its share of the block's rows, the kC5 slice sums in rank order through
-// distributed shared memory, scales once and writes.  Deterministic for a
-// given launch shape.  The first row's words are loaded before the
-// programmatic-launch wait, the tables (which depend on x) after it.
+// tables (two [243][96] float arrays, 182 KiB); every CTA of the cluster runs
+// over the cluster's contiguous range of rows.
+//
+// Lanes and columns: in one row, lane l holds the words of slice columns 2l and
+// 2l + 1 (one 32-bit load where kt and the slice start are even, else two
+// 16-bit loads) and of column 64 + l (a 16-bit load).  Table rows store column
+// c < 64 at position (c & 1) * 32 + c / 2 and column c >= 64 at c, so each of
+// the six lookups of a row reads 32 consecutive positions of one table row
+// chosen per lane: 32 different banks, whatever the words are.  Columns past
+// the slice hold x = 0 (all entries 0); lanes there look up the all-zero-trit
+// word.
+//
+// A warp takes four consecutive rows per round and keeps the words of the two
+// rounds after it in flight (the first two rounds are loaded before the
+// programmatic-launch wait, while x is staged and the tables are built).  The
+// four rows' lane sums are added in one transposed shuffle tree (six shuffles
+// for four rows) and stored as the CTA's slice sums; at the end of each chunk
+// of kC5Rows rows, after a cluster barrier, CTA q adds for its share of the
+// chunk the kC5 slice sums in rank order through distributed shared memory,
+// scales once and writes.  Deterministic for a given launch shape.
 // ---------------------------------------------------------------------------
 constexpr int kC5 = 5;                 // CTAs per cluster (slices of the row)
 constexpr int kC5Threads = 1024;
-constexpr int kC5Pitch = 96;           // table columns (word positions) per slice; a multiple of 32
-constexpr int kC5Rows = 1024;          // rows of a block (slice sums held at once)
+constexpr int kC5Warps = kC5Threads / 32;
+constexpr int kC5Pitch = 96;           // table positions per slice (64 in pairs + 32 single)
+constexpr int kC5D = 4;                // rows per warp round
+constexpr int kC5Round = kC5Warps * kC5D;          // rows per CTA round
+constexpr int kC5Rows = 1024;          // rows of a chunk (slice sums held at once)
+static_assert(kC5Rows % kC5Round == 0, "a chunk is a whole number of rounds");
 constexpr uint32_t kDiv243Mul = 69043u, kDiv243Shift = 24;  // floor(w / 243) for w < 3^10
+constexpr uint32_t kZeroWord = 29524u;                      // all ten digits 1: trits 0
+constexpr uint32_t kZeroPair = kZeroWord | (kZeroWord << 16);
 
 constexpr bool div243_exact() {
   for (uint32_t w = 0; w < 59049u; ++w)
@@ -570,109 +356,185 @@ constexpr bool div243_exact() {
 }
 static_assert(div243_exact(), "multiply-shift division by 243");
 
-size_t c5_smem_bytes() { return (2u * 243u * kC5Pitch + kC5Rows) * sizeof(float); }
+// floats: lo [243][96], hi [243][96], slice sums [kC5Rows], x [10][96] by table position
+size_t c5_smem_bytes() { return (2u * 243u * kC5Pitch + kC5Rows + 10u * kC5Pitch) * sizeof(float); }
 
+// slice column of table position p
+__device__ __forceinline__ int c5_column(int p) { return p < 64 ? (p < 32 ? 2 * p : 2 * (p - 32) + 1) : p; }
+
+// The words of one row at this lane's three columns: VEC, one 32-bit load for
+// columns 2l, 2l + 1 (w[0]; w[1] unused); else two 16-bit loads (w[0], w[1]).
+// w[2] = column 64 + l.
+template <bool VEC>
+struct C5Words {
+  uint32_t w[VEC ? 2 : 3];
+};
+
+template <bool VEC>
+__device__ __forceinline__ void c5_fetch(const uint16_t* __restrict__ row, bool live, int lane, int sw,
+                                         C5Words<VEC>& o) {
+  const bool a = live && 2 * lane < sw, b = live && 2 * lane + 1 < sw, c = live && 64 + lane < sw;
+  if constexpr (VEC) {
+    o.w[0] = a ? __ldcs(reinterpret_cast<const uint32_t*>(row + 2 * lane)) : kZeroPair;
+    o.w[1] = c ? static_cast<uint32_t>(__ldcs(row + 64 + lane)) : kZeroWord;
+  } else {
+    o.w[0] = a ? static_cast<uint32_t>(__ldcs(row + 2 * lane)) : kZeroWord;
+    o.w[1] = b ? static_cast<uint32_t>(__ldcs(row + 2 * lane + 1)) : kZeroWord;
+    o.w[2] = c ? static_cast<uint32_t>(__ldcs(row + 64 + lane)) : kZeroWord;
+  }
+}
+
+// lo_p[ql] + hi_p[qh] of one word; tl / th = this lane's table positions (bytes)
+__device__ __forceinline__ float c5_lookup(uint32_t w, uint32_t tl, uint32_t th) {
+  const uint32_t qh = (w * kDiv243Mul) >> kDiv243Shift;  // digits 5..9
+  const uint32_t ql = w - 243u * qh;                     // digits 0..4
+  float a, b;
+  asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(a) : "r"(tl + ql * (4u * kC5Pitch)));
+  asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(b) : "r"(th + qh * (4u * kC5Pitch)));
+  return a + b;
+}
+
+// One row's three words at this lane.  Words are clamped to 3^10 - 1 first, so
+// a word outside the format (its result unspecified) still looks up inside the
+// tables.
+template <bool VEC>
+__device__ __forceinline__ float c5_row(const C5Words<VEC>& v, uint32_t lo0, uint32_t hi0) {
+  constexpr uint32_t kMaxWord = 59048u;
+  float s;
+  if constexpr (VEC) {
+    const uint32_t pr = __vminu2(v.w[0], kMaxWord | (kMaxWord << 16));
+    s = c5_lookup(pr & 0xFFFFu, lo0, hi0) + c5_lookup(pr >> 16, lo0 + 128u, hi0 + 128u);
+    s += c5_lookup(min(v.w[1], kMaxWord), lo0 + 256u, hi0 + 256u);
+  } else {
+    s = c5_lookup(min(v.w[0], kMaxWord), lo0, hi0) + c5_lookup(min(v.w[1], kMaxWord), lo0 + 128u, hi0 + 128u);
+    s += c5_lookup(min(v.w[2], kMaxWord), lo0 + 256u, hi0 + 256u);
+  }
+  return s;
+}
+
+// base + x0 (d0 - 1) + x1 (d1 - 1) for the digits d0 = a % 3, d1 = a / 3 (a is
+// a compile-time constant once the caller's loop is unrolled: one add)
+__device__ __forceinline__ float c5_entry(int a, float base, float x0, float x1) {
+  switch (a) {
+    case 0: return base - (x0 + x1);
+    case 1: return base - x1;
+    case 2: return base + (x0 - x1);
+    case 3: return base - x0;
+    case 4: return base;
+    case 5: return base + x0;
+    case 6: return base - (x0 - x1);
+    case 7: return base + x1;
+    default: return base + (x0 + x1);
+  }
+}
+
+template <bool VEC>
 __global__ void __launch_bounds__(kC5Threads, 1)
 ternary_gemv_c5_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ packed,
-                       const float* __restrict__ scale, int64_t n, int k, int kt, int slice, int64_t block_rows,
+                       const float* __restrict__ scale, int64_t n, int k, int kt, int slice,
                        float* __restrict__ out, const float* __restrict__ bias) {
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
-  extern __shared__ float c5sm[];  // lo [243][kC5Pitch], hi [243][kC5Pitch], slice sums [kC5Rows]
+  extern __shared__ __align__(16) float c5sm[];
   float* const lo = c5sm;
   float* const hi = c5sm + 243 * kC5Pitch;
   float* const psum = c5sm + 2 * 243 * kC5Pitch;
+  float* const xs = psum + kC5Rows;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int kWarps = kC5Threads / 32;
   const int rank = static_cast<int>(cluster.block_rank());
-  const int64_t cl = blockIdx.x / kC5, nclusters = gridDim.x / kC5;
-  const int w0 = rank * slice;                                  // this CTA's first word position
+  const int64_t cl = blockIdx.x / kC5, ncl = gridDim.x / kC5;
+  const int w0 = rank * slice;                                            // this CTA's first word position
   const int sw = kt - w0 < slice ? (kt - w0 > 0 ? kt - w0 : 0) : slice;  // its word count (<= kC5Pitch)
-  const int64_t nblocks = (n + block_rows - 1) / block_rows;
+  const int64_t c0 = n * cl / ncl, c1 = n * (cl + 1) / ncl;              // the cluster's rows
+  const int rounds = static_cast<int>((c1 - c0 + kC5Round - 1) / kC5Round);
   bnn::pdl_trigger();
 
-  // the words of row r at positions w0 + lane + 32 p (29524 = all-zero trits past the slice)
-  auto fetch = [&](int64_t r, bool live, uint32_t (&v)[3]) {
+  const uint16_t* const wbase = packed + w0;
+  auto fetch_round = [&](int i, C5Words<VEC> (&buf)[kC5D]) {
+    const int64_t r0 = c0 + static_cast<int64_t>(i) * kC5Round + warp * kC5D;
 #pragma unroll
-    for (int p = 0; p < 3; ++p) {
-      const int o = lane + 32 * p;
-      v[p] = (live && o < sw) ? static_cast<uint32_t>(__ldcs(packed + r * kt + w0 + o)) : 29524u;
-    }
+    for (int j = 0; j < kC5D; ++j) c5_fetch<VEC>(wbase + (r0 + j) * kt, i < rounds && r0 + j < c1, lane, sw, buf[j]);
   };
-  int64_t blk = cl;
-  int64_t b0 = blk * block_rows;
-  int64_t b1 = b0 + block_rows < n ? b0 + block_rows : n;
-  uint32_t cur[3];
-  fetch(b0 + warp, blk < nblocks && b0 + warp < b1, cur);
+  C5Words<VEC> bufA[kC5D], bufB[kC5D], bufC[kC5D];
+  fetch_round(0, bufA);
+  fetch_round(1, bufB);
 
   bnn::pdl_wait();  // x may come from the kernel ahead
-  // Tables: task = (table t, high digits e_hi of the 5, word position o), nine
-  // entries each (the two low digits run over 0..8); consecutive threads take
-  // consecutive positions of one entry row (distinct banks).  Every column is
-  // built, those past the slice with x = 0 (all their entries 0), since the
-  // lanes past the slice look up the all-zero-trit word there.
-  for (int f = tid; f < 2 * 27 * kC5Pitch; f += kC5Threads) {
-    const int o = f % kC5Pitch, g = f / kC5Pitch, t = g / 27, eh = g - 27 * t;
-    const int e0 = 10 * (w0 + o) + 5 * t;
-    float xv[5];
+  // x of the slice as float32, [digit i][table position p]
+  for (int f = tid; f < 10 * kC5Pitch; f += kC5Threads) {
+    const int i = f / kC5Pitch, p = f - kC5Pitch * i, c = c5_column(p), e = 10 * (w0 + c) + i;
+    xs[f] = (c < sw && e < k) ? __uint_as_float(static_cast<uint32_t>(__ldg(x + e)) << 16) : 0.0f;
+  }
+  __syncthreads();
+  // Tables: task = (table t, digits 2..4 of the five as b, four table positions
+  // 4q..4q+3); the nine entries 9b + a (a = digits 0, 1) of each position, one
+  // add each, stored four positions at a time.
+  for (int f = tid; f < 2 * 27 * (kC5Pitch / 4); f += kC5Threads) {
+    const int q = f % (kC5Pitch / 4), g = f / (kC5Pitch / 4), t = g / 27, b = g - 27 * t;
+    const float4* xq = reinterpret_cast<const float4*>(xs + (5 * t) * kC5Pitch) + q;
+    const float4 x0 = xq[0], x1 = xq[kC5Pitch / 4], x2 = xq[2 * kC5Pitch / 4], x3 = xq[3 * kC5Pitch / 4],
+                 x4 = xq[4 * kC5Pitch / 4];
+    const float c2 = static_cast<float>(b % 3 - 1), c3 = static_cast<float>((b / 3) % 3 - 1),
+                c4 = static_cast<float>(b / 9 - 1);
+    const float bx = x2.x * c2 + x3.x * c3 + x4.x * c4, by = x2.y * c2 + x3.y * c3 + x4.y * c4,
+                bz = x2.z * c2 + x3.z * c3 + x4.z * c4, bw = x2.w * c2 + x3.w * c3 + x4.w * c4;
+    float4* dst = reinterpret_cast<float4*>((t == 0 ? lo : hi) + (9 * b) * kC5Pitch) + q;
 #pragma unroll
-    for (int i = 0; i < 5; ++i)
-      xv[i] = (o < sw && e0 + i < k) ? __uint_as_float(static_cast<uint32_t>(__ldg(x + e0 + i)) << 16) : 0.0f;
-    const float base = xv[2] * static_cast<float>(eh % 3 - 1) + xv[3] * static_cast<float>((eh / 3) % 3 - 1) +
-                       xv[4] * static_cast<float>(eh / 9 - 1);
-    float* dst = (t == 0 ? lo : hi) + (9 * eh) * kC5Pitch + o;
-#pragma unroll
-    for (int v = 0; v < 9; ++v)
-      dst[v * kC5Pitch] = (xv[0] * static_cast<float>(v % 3 - 1) + xv[1] * static_cast<float>(v / 3 - 1)) + base;
+    for (int a = 0; a < 9; ++a) {
+      float4 v;
+      v.x = c5_entry(a, bx, x0.x, x1.x);
+      v.y = c5_entry(a, by, x0.y, x1.y);
+      v.z = c5_entry(a, bz, x0.z, x1.z);
+      v.w = c5_entry(a, bw, x0.w, x1.w);
+      dst[a * (kC5Pitch / 4)] = v;
+    }
   }
   __syncthreads();
 
-  const uint32_t stride = 4u * kC5Pitch;
-  const uint32_t lo_lane = static_cast<uint32_t>(__cvta_generic_to_shared(lo)) + 4u * static_cast<uint32_t>(lane);
-  const uint32_t hi_lane = static_cast<uint32_t>(__cvta_generic_to_shared(hi)) + 4u * static_cast<uint32_t>(lane);
-  for (; blk < nblocks; blk += nclusters) {
-    const int rows = static_cast<int>(b1 - b0);
-    for (int rl = warp; rl < rows; rl += kWarps) {
-      // the next row of this warp (in this block, else the first of the next block)
-      int64_t nr = b0 + rl + kWarps;
-      bool nlive = rl + kWarps < rows;
-      if (!nlive) {
-        const int64_t nb = blk + nclusters;
-        nr = nb * block_rows + warp;
-        nlive = nb < nblocks && nr < (nb * block_rows + block_rows < n ? nb * block_rows + block_rows : n);
+  const uint32_t lo0 = static_cast<uint32_t>(__cvta_generic_to_shared(lo)) + 4u * static_cast<uint32_t>(lane);
+  const uint32_t hi0 = static_cast<uint32_t>(__cvta_generic_to_shared(hi)) + 4u * static_cast<uint32_t>(lane);
+  const bool upper = (lane & 16) != 0, mid = (lane & 8) != 0;
+  // round i: the rows of bufX, with the round two ahead loaded into bufY
+  auto round = [&](int i, C5Words<VEC> (&cur)[kC5D], C5Words<VEC> (&ahead)[kC5D]) {
+    fetch_round(i + 2, ahead);
+    const int64_t r0 = c0 + static_cast<int64_t>(i) * kC5Round + warp * kC5D;
+    float acc[kC5D];
+#pragma unroll
+    for (int j = 0; j < kC5D; ++j) acc[j] = r0 + j < c1 ? c5_row<VEC>(cur[j], lo0, hi0) : 0.0f;
+    // four rows over 32 lanes: halves exchange rows (0,1) / (2,3), then quarters
+    // row 0 / 1 of their pair; lane group (lane >> 3) ends with row 2 (lane >> 4) + (lane >> 3 & 1)
+    float k0 = upper ? acc[2] : acc[0], k1 = upper ? acc[3] : acc[1];
+    const float s0 = upper ? acc[0] : acc[2], s1 = upper ? acc[1] : acc[3];
+    k0 += __shfl_xor_sync(0xffffffffu, s0, 16);
+    k1 += __shfl_xor_sync(0xffffffffu, s1, 16);
+    float v = mid ? k1 : k0;
+    v += __shfl_xor_sync(0xffffffffu, mid ? k0 : k1, 8);
+    v += __shfl_xor_sync(0xffffffffu, v, 4);
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    const int j = lane >> 3;
+    const int64_t cs = c0 + static_cast<int64_t>(i / (kC5Rows / kC5Round)) * kC5Rows;  // the chunk's first row
+    if ((lane & 7) == 0 && r0 + j < c1) psum[r0 + j - cs] = v;
+    if (i % (kC5Rows / kC5Round) == kC5Rows / kC5Round - 1 || i == rounds - 1) {
+      // end of a chunk: its slice sums added in rank order by the CTA that owns the row
+      cluster.sync();
+      const int64_t ce = cs + kC5Rows < c1 ? cs + kC5Rows : c1;
+      const int rows = static_cast<int>(ce - cs);
+      const int q0 = rows * rank / kC5, q1 = rows * (rank + 1) / kC5;
+      for (int rl = q0 + tid; rl < q1; rl += kC5Threads) {
+        float sum = 0.0f;
+#pragma unroll
+        for (int q = 0; q < kC5; ++q) sum += cluster.map_shared_rank(psum, q)[rl];
+        const int64_t r = cs + rl;
+        out[r] = bias ? __ldg(scale + r) * sum + __ldg(bias + r) : __ldg(scale + r) * sum;
       }
-      uint32_t nxt[3];
-      fetch(nr, nlive, nxt);
-      float acc = 0.0f;
-#pragma unroll
-      for (int p = 0; p < 3; ++p) {
-        const uint32_t w = cur[p];
-        const uint32_t qh = (w * kDiv243Mul) >> kDiv243Shift;  // digits 5..9
-        const uint32_t ql = w - 243u * qh;                     // digits 0..4
-        float a, b;
-        asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(a) : "r"(lo_lane + 128u * p + ql * stride));
-        asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(b) : "r"(hi_lane + 128u * p + qh * stride));
-        acc += a + b;
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-      if (lane == 0) psum[rl] = acc;
-#pragma unroll
-      for (int p = 0; p < 3; ++p) cur[p] = nxt[p];
+      cluster.sync();  // slice sums read before the next chunk overwrites them (and before any CTA exits)
     }
-    cluster.sync();  // every CTA's slice sums of this block are stored
-    // this CTA finalises rows [q0, q1) of the block: slice sums added in rank order
-    const int q0 = rows * rank / kC5, q1 = rows * (rank + 1) / kC5;
-    for (int rl = q0 + tid; rl < q1; rl += kC5Threads) {
-      float sum = 0.0f;
-#pragma unroll
-      for (int q = 0; q < kC5; ++q) sum += cluster.map_shared_rank(psum, q)[rl];
-      const int64_t r = b0 + rl;
-      out[r] = bias ? __ldg(scale + r) * sum + __ldg(bias + r) : __ldg(scale + r) * sum;
-    }
-    cluster.sync();  // slice sums read before the next block overwrites them (and before any CTA exits)
-    b0 = (blk + nclusters) * block_rows;
-    b1 = b0 + block_rows < n ? b0 + block_rows : n;
+  };
+  for (int i = 0; i < rounds; i += 3) {
+    round(i, bufA, bufC);
+    if (i + 1 < rounds) round(i + 1, bufB, bufA);
+    if (i + 2 < rounds) round(i + 2, bufC, bufB);
   }
 }
 
@@ -910,7 +772,7 @@ int c5_clusters() {
   const uint64_t ctx = bnn::context_id();
   if (ctx != 0 && ctx == ctx_cached) return cached;
   int num = 0;
-  if (bnn::ensure_smem(ternary_gemv_c5_kernel, c5_smem_bytes()) == cudaSuccess) {
+  if (bnn::ensure_smem(ternary_gemv_c5_kernel<true>, c5_smem_bytes()) == cudaSuccess) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(kC5 * 64);
     cfg.blockDim = dim3(kC5Threads);
@@ -922,7 +784,7 @@ int c5_clusters() {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&num, ternary_gemv_c5_kernel, &cfg) != cudaSuccess) num = 0;
+    if (cudaOccupancyMaxActiveClusters(&num, ternary_gemv_c5_kernel<true>, &cfg) != cudaSuccess) num = 0;
   }
   cudaGetLastError();  // a failed query leaves no error behind
   cached = num;
@@ -950,28 +812,25 @@ bnn_status ternary_gemm_impl(const uint16_t* x_bf16, const uint16_t* packed, con
   if (algo != BNN_TALGO_MMA && m == 1 && kt > 0 && kt <= kC5 * kC5Pitch) {
     const int clusters = c5_clusters();
     if (clusters > 0) {
-      const int slice = static_cast<int>((kt + kC5 - 1) / kC5);
+      // 32-bit word pairs where every row's slices start 4-byte aligned: kt even, the slice even
+      const bool vec = kt % 2 == 0 && bnn::aligned(packed, 4);
+      int slice = static_cast<int>((kt + kC5 - 1) / kC5);
+      if (vec) slice += slice & 1;  // at most 96: kt <= 480
       const int64_t g = (n + 63) / 64 < clusters ? (n + 63) / 64 : clusters;  // at least 64 rows per cluster
-      int64_t block_rows = (n + g - 1) / g;
-      if (block_rows > kC5Rows) block_rows = kC5Rows;
       const size_t smem = c5_smem_bytes();
-      BNN_TRY(bnn::ensure_smem(ternary_gemv_c5_kernel, smem));
-      BNN_TRY(bnn::launch_pdl(ternary_gemv_c5_kernel, dim3(static_cast<unsigned>(kC5 * g)), dim3(kC5Threads), smem, s,
-                              kC5, x_bf16, packed, scale, n, static_cast<int>(k), static_cast<int>(kt), slice,
-                              block_rows, out, bias));
+      if (vec) {
+        BNN_TRY(bnn::ensure_smem(ternary_gemv_c5_kernel<true>, smem));
+        BNN_TRY(bnn::launch_pdl(ternary_gemv_c5_kernel<true>, dim3(static_cast<unsigned>(kC5 * g)),
+                                dim3(kC5Threads), smem, s, kC5, x_bf16, packed, scale, n, static_cast<int>(k),
+                                static_cast<int>(kt), slice, out, bias));
+      } else {
+        BNN_TRY(bnn::ensure_smem(ternary_gemv_c5_kernel<false>, smem));
+        BNN_TRY(bnn::launch_pdl(ternary_gemv_c5_kernel<false>, dim3(static_cast<unsigned>(kC5 * g)),
+                                dim3(kC5Threads), smem, s, kC5, x_bf16, packed, scale, n, static_cast<int>(k),
+                                static_cast<int>(kt), slice, out, bias));
+      }
       return bnn::check_launch();
     }
-  }
-  if (algo != BNN_TALGO_MMA && m == 1 && kt > 0 && kt <= kLutMaxKt && kt % 2 == 0 && bnn::aligned(packed, 4) &&
-      n * (kt / 2) < (int64_t{1} << 31)) {
-    const size_t smem = lut_smem_bytes(kt);
-    BNN_TRY(bnn::ensure_smem(ternary_gemv_lut_kernel, smem));
-    const int64_t sms = bnn::sm_count();
-    const int grid = static_cast<int>(n < sms ? n : sms);
-    BNN_TRY(bnn::launch_pdl(ternary_gemv_lut_kernel, dim3(grid), dim3(kLutThreads), smem, s, 1, x_bf16,
-                            reinterpret_cast<const uint32_t*>(packed), scale, n, static_cast<int>(k),
-                            static_cast<int>(kt), out, bias));
-    return bnn::check_launch();
   }
   if (algo != BNN_TALGO_MMA && m == 1 && kt > 0 && rows_smem_bytes(kt) <= 200 * 1024) {
     const size_t smem = rows_smem_bytes(kt);

@@ -224,8 +224,10 @@ sparse_gemv_smem_kernel(const uint16_t* __restrict__ x, const int64_t* __restric
   const int64_t r_begin = n * blockIdx.x / gridDim.x, r_end = n * (blockIdx.x + 1) / gridDim.x;
   bnn::pdl_trigger();
 
-  // entries [b + 32 u + lane] of one pass (position k, a zero term, past the row's end)
-  const uint32_t pad = static_cast<uint32_t>(k);
+  // entries [b + 32 u + lane] of one pass; past the row's end the value 2^16, which no
+  // 16-bit entry holds and which the position clamp below sends to the zero slot (at
+  // k = 32768 every 15-bit position is a real one, so the padding cannot be one)
+  const uint32_t pad = 0x10000u, kk = static_cast<uint32_t>(k);
   auto fetch = [&](int64_t q0, int64_t e, uint32_t (&v)[kSpU]) {
 #pragma unroll
     for (int u = 0; u < kSpU; ++u) {
@@ -261,8 +263,8 @@ sparse_gemv_smem_kernel(const uint16_t* __restrict__ x, const int64_t* __restric
 #pragma unroll
       for (int u = 0; u < kSpU; ++u) {
         const uint32_t v = cur[u];
-        // positions >= k (malformed, or the padding past the row) read the zero slot xs[k]
-        const uint32_t pos = min(v & 0x7FFFu, pad);
+        // positions >= k (malformed) and the padding (bit 16 kept by the mask) read the zero slot xs[k]
+        const uint32_t pos = min(v & 0x17FFFu, kk);
         const float t = __uint_as_float(__float_as_uint(xs[pos]) ^ ((v << 16) & 0x80000000u));  // sign bit 15
         if (u & 1) acc1 += t;
         else acc0 += t;

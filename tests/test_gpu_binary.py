@@ -81,11 +81,10 @@ def test_skinny_matches_oracle(bnn, m, n, k):
     _gemm_case(bnn, m, n, k, seed=m * 1000 + n + k)
 
 
-# m = 1 with 16-byte aligned rows of at most 256 words streams the weights by
-# bulk copies: one to four 64-word passes per row, rows per chunk from 512 down
-# to 16, several chunks per CTA (the ring wraps), fewer rows than SMs.
+# m = 1 GEMV shapes: long rows (several 16-byte passes per lane), short rows
+# with many of them, ragged word counts, fewer rows than SMs.
 @pytest.mark.parametrize("n,k", [(5000, 16384), (3000, 12000), (70000, 128), (100, 8192), (20000, 640), (7, 4096)])
-def test_gemv_bulk_shapes(bnn, n, k):
+def test_gemv_m1_shapes(bnn, n, k):
     _gemm_case(bnn, 1, n, k, seed=n + k, algos=(0,))
 
 
@@ -105,8 +104,8 @@ def test_tiled_matches_oracle(bnn, m, n, k):
                                    (257, 383, 2048 * 2 + 64), (2304, 4219, 130), (600, 9000, 760), (50, 700, 2000),
                                    (64, 1000, 300), (64, 2000, 500), (200, 1000, 2048), (300, 3000, 256),
                                    (384, 6400, 128), (250, 700, 2048 + 130),
-                                   # two tiles or more per SM (the persistent kernel): ragged m and n, one
-                                   # activation tile, a single stage and several
+                                   # two tiles or more per SM: ragged m and n, one activation tile,
+                                   # a single stage and several
                                    (2304, 4219, 128), (2000, 4800, 256), (200, 38000, 128), (300, 40000, 128)])
 def test_tc_tile_configs(bnn, m, n, k):
     _gemm_case(bnn, m, n, k, seed=5 * m + n + 3 * k, algos=(3,))

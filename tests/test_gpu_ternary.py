@@ -157,36 +157,40 @@ def test_every_base3_word_decodes_row_kernel(bnn):
     _gemm_case(bnn, 1, 60, k, seed=23, trits=trits, algos=(0, 1))
 
 
-def test_every_base3_word_decodes_lut_kernel(bnn):
-    """All 3^10 words in 145 rows of 410 words (k = 4100, even word count: the
-    m = 1 kernel on 4 + 3 + 3-trit activation tables), every code through its
-    decoder, with and without a bias."""
-    k, kt = 4100, 410
-    words = (np.arange(145 * kt) % 59049).astype(np.uint16).reshape(145, kt)
+@pytest.mark.parametrize("k,kt", [(4100, 410), (4090, 409)])
+def test_every_base3_word_decodes_table_kernel(bnn, k, kt):
+    """All 3^10 words in 145 rows (k = 4100: 410 words a row, the m = 1
+    kernel on 5 + 5-trit activation tables with 32-bit word pairs; k = 4090:
+    409 words, the same kernel on 16-bit loads), every code through both
+    tables of every lane position, with and without a bias."""
+    rows = (59049 + kt - 1) // kt
+    words = (np.arange(rows * kt) % 59049).astype(np.uint16).reshape(rows, kt)
     trits, bad = oracle.base3_unpack(words, k)
     assert bad == 0
-    _gemm_case(bnn, 1, 145, k, seed=29, trits=trits, algos=(0,))
-    scale = synth.uniform_f32(29, 1, (145,), 0.25, 2.0)
-    bias = synth.normal_f32(29, 3, (145,))
+    _gemm_case(bnn, 1, rows, k, seed=29, trits=trits, algos=(0,))
+    scale = synth.uniform_f32(29, 1, (rows,), 0.25, 2.0)
+    bias = synth.normal_f32(29, 3, (rows,))
     xb = synth.bf16_bits_from_f32(synth.normal_f32(29, 2, (1, k)))
-    ref, mag = oracle.ternary_linear(xb, words, scale, bias, 1, 145, k)
+    ref, mag = oracle.ternary_linear(xb, words, scale, bias, 1, rows, k)
     out = bnn.bnn_ternary_linear(to_dev_bf16(xb), to_dev_u16(words), to_dev_f32(scale), to_dev_f32(bias))
-    assert_ternary_close(out.cpu().numpy(), ref, mag + np.abs(bias.astype(np.float64)), "lut kernel with bias")
+    assert_ternary_close(out.cpu().numpy(), ref, mag + np.abs(bias.astype(np.float64)), "table kernel with bias")
 
 
 # m = 1 shapes around the table kernel's limits: word counts from 2 to its
-# maximum 416 (even) with ragged last passes, odd word counts and words 2
-# bytes off 4-byte alignment (other kernels), row blocks larger than one
-# chunk of 256 rows per CTA, fewer rows than SMs, and pad trits in the last word.
+# maximum 480 (k = 4800; 4801 takes the pair-table kernel), even (32-bit word
+# pairs) and odd (16-bit loads), clusters with more rows than one chunk of
+# 1024, fewer rows than a round of 128, one cluster, and pad trits in the last
+# word.
 @pytest.mark.parametrize("n,k", [(1, 11), (7, 20), (300, 640), (149, 4160), (1000, 4140), (40000, 100),
-                                 (5000, 4096), (500, 1300), (33, 4161), (64, 1290), (150, 4170)])
-def test_gemv_m1_lut_shapes(bnn, n, k):
+                                 (5000, 4096), (500, 1300), (33, 4161), (64, 1290), (150, 4170),
+                                 (2000, 4800), (300, 4801), (129, 4791)])
+def test_gemv_m1_table_shapes(bnn, n, k):
     _gemm_case(bnn, 1, n, k, seed=n + k)
 
 
 def test_gemv_m1_packed_two_bytes_off(bnn):
-    """Packed words 2 bytes off 4-byte alignment take the pair-table kernel,
-    with the same results."""
+    """Packed words 2 bytes off 4-byte alignment take the table kernel's
+    16-bit loads, with the same results."""
     n, k = 300, 4096
     rng = np.random.default_rng(5)
     trits = rng.integers(-1, 2, (n, k)).astype(np.int8)
