@@ -471,6 +471,293 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(BN));
 }
 
+// ---------------------------------------------------------------------------
+// Two-SM variant for large GEMMs: a cluster of two CTAs computes one tile of
+// 256 weight rows x 256 activation rows with tcgen05.mma.cta_group::2 (UMMA
+// M = 256, N = 256).  CTA q of the pair holds weight rows 128q.. of the tile
+// (its half of operand A, and the tensor-memory lanes of those rows) and
+// activation rows 128q.. (its half of operand B); one MMA reads both CTAs'
+// shared memory, so each SM expands and feeds only 256 rows per stage instead
+// of the 384 of a 128 x 256 tile on one SM, and its tensor memory receives all
+// 256 accumulator columns of its 128 weight rows.
+//
+// Roles per CTA as in the kernel above (two producer threads per stacked row,
+// a TMA thread for the packed chunks of its own rows), with these changes:
+//   - producers signal per warp (fence to the async proxy, a warp barrier,
+//     then lane 0 arrives) on the stage's "full" mbarrier of CTA 0, at cluster
+//     scope, so that barrier completes once both CTAs' 32 producer warps have
+//     written the stage;
+//   - only CTA 0 issues the MMAs; tcgen05.commit with a two-CTA mask arrives
+//     on the "empty" barrier of the stage in both CTAs (and on "done" after the
+//     last stage);
+//   - the epilogue reads the other CTA's activation-row popcounts through
+//     distributed shared memory.
+// Every wait is bounded; an abort in either CTA leaves the whole tile unwritten.
+// ---------------------------------------------------------------------------
+constexpr int kQRows = 256;                                  // stacked rows per CTA (128 weight + 128 activation)
+constexpr uint32_t kQStageBytes = kQRows * 128u;             // one expanded stage (32 KiB)
+constexpr uint32_t kQChunkBytes = kQRows * 16u * kChunkStages;  // one packed chunk (16 KiB)
+constexpr int kQS = 5, kQP = 2;                              // expanded stages, packed chunks
+constexpr int kQProducers = 2 * kQRows;                      // 512
+constexpr int kQWarps = kQProducers / 32;                    // producer warps per CTA
+constexpr int kQMmaWarp = kQWarps, kQTmaWarp = kQWarps + 1;
+constexpr int kQThreads = kQProducers + 64;
+constexpr uint32_t kQSmem = kQS * kQStageBytes + kQP * kQChunkBytes;
+constexpr uint32_t kQTmemCols = 256;
+
+__global__ void __launch_bounds__(kQThreads, 1)
+binary_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
+                        const float* __restrict__ alpha, const float* __restrict__ bias, int64_t m, int64_t n, int k,
+                        int kw, int32_t* __restrict__ dots, float* __restrict__ out, uint32_t* __restrict__ next,
+                        int64_t next_w32, uint32_t wait_limit) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[kQS];   // CTA 0's: both CTAs' producer warps arrive
+  __shared__ __align__(8) uint64_t empty_bar[kQS];
+  __shared__ __align__(8) uint64_t chunk_full[kQP];
+  __shared__ __align__(8) uint64_t chunk_empty[kQP];
+  __shared__ __align__(8) uint64_t done_bar;
+  __shared__ uint32_t tmem_holder;
+  __shared__ volatile int abort_flag;
+  __shared__ int any_bad;
+  __shared__ int pop_w[kTm];
+  __shared__ int pop_x[kTm];        // this CTA's 128 activation rows
+  __shared__ int pop_xt[2 * kTm];   // the tile's 256 activation rows
+  uint8_t* const smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* const chunks = smem + kQS * kQStageBytes;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster.block_rank();
+  const int64_t j0 = static_cast<int64_t>(blockIdx.x >> 1) * 256 + 128 * rank;  // this CTA's weight rows
+  const int64_t i0 = static_cast<int64_t>(blockIdx.y) * 256;                      // the tile's activation rows
+  const int nst = (kw + 1) / 2;
+  const uint32_t smem_base = smem_u32(smem);
+
+  for (int i = tid; i < kTm; i += blockDim.x) pop_w[i] = pop_x[i] = 0;
+  if (tid == 0) {
+    for (int i = 0; i < kQS; ++i) {
+      bnn::tc::mbar_init(smem_u32(&full_bar[i]), 2 * kQWarps);
+      bnn::tc::mbar_init(smem_u32(&empty_bar[i]), 1);
+    }
+    for (int i = 0; i < kQP; ++i) {
+      bnn::tc::mbar_init(smem_u32(&chunk_full[i]), 1);
+      bnn::tc::mbar_init(smem_u32(&chunk_empty[i]), kQWarps);
+    }
+    bnn::tc::mbar_init(smem_u32(&done_bar), 1);
+    abort_flag = 0;
+    any_bad = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  if (tid == kQTmaWarp * 32) {
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tmap_w)) : "memory");
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
+  }
+  if (warp == kQMmaWarp) {  // the same warp of both CTAs allocates the pair's tensor memory
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(&tmem_holder)),
+                 "r"(kQTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;\n" ::);
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+  cluster.sync();  // both CTAs' barriers exist before any arrival from the other CTA
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+  const uint32_t tmem = tmem_holder;
+  bnn::pdl_trigger();
+
+  if (tid < kQProducers) {
+    // ------------------------------------------------------------ producers
+    const int r2 = tid >> 1, part = tid & 1;
+    const bool is_w = r2 < kTm;
+    const int row = is_w ? r2 : r2 - kTm;
+    const uint32_t row_off = static_cast<uint32_t>(r2) * 128u;
+    const uint32_t swz = static_cast<uint32_t>(row & 7);
+    const uint32_t rd_off = static_cast<uint32_t>(r2) * 64u + 8u * static_cast<uint32_t>(part);
+    const uint32_t rd_swz = static_cast<uint32_t>((r2 >> 1) & 3);
+    int my_pop = 0;
+    for (int j = 0; j < nst; ++j) {
+      const int c = j / kChunkStages, s = j % kChunkStages, pb = c % kQP;
+      bool ok = true;
+      if (s == 0)
+        ok = bnn::tc::mbar_wait(smem_u32(&chunk_full[pb]), static_cast<uint32_t>((c / kQP) & 1), &abort_flag,
+                                &g_bnn_device_errors, wait_limit);
+      const int b = j % kQS;
+      // refill only after the tensor core has read the previous fill of this buffer
+      if (ok && j >= kQS)
+        ok = bnn::tc::mbar_wait(smem_u32(&empty_bar[b]), static_cast<uint32_t>((j / kQS + 1) & 1), &abort_flag,
+                                &g_bnn_device_errors, wait_limit);
+      if (!__all_sync(0xffffffffu, ok)) break;  // the warp stops together
+      const uint64_t cw = *reinterpret_cast<const uint64_t*>(
+          chunks + pb * kQChunkBytes + rd_off + ((static_cast<uint32_t>(s) ^ rd_swz) << 4));
+      my_pop += __popcll(cw);
+      expand_word(smem + b * kQStageBytes + row_off, swz, part, cw);
+      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+      __syncwarp();
+      if (lane == 0) {
+        if (s == kChunkStages - 1 || j == nst - 1) mbar_arrive(smem_u32(&chunk_empty[pb]));
+        bnn::tc::mbar_arrive_rank(smem_u32(&full_bar[b]), 0u);
+      }
+    }
+    atomicAdd(is_w ? &pop_w[row] : &pop_x[row], my_pop);
+  } else if (tid == kQMmaWarp * 32 && rank == 0) {
+    // ------------------------------------------------------------ MMA issue
+    // D s32, A and B 8-bit integers, both K-major, N = 256, M = 256 (two CTAs)
+    const uint32_t idesc = (2u << 4) | (1u << 7) | (1u << 10) | ((256u >> 3) << 17) | ((256u >> 4) << 24);
+    for (int j = 0; j < nst; ++j) {
+      const int b = j % kQS;
+      if (!bnn::tc::mbar_wait_cluster(smem_u32(&full_bar[b]), static_cast<uint32_t>((j / kQS) & 1), &abort_flag,
+                                      &g_bnn_device_errors, wait_limit))
+        break;
+      asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+      const uint64_t ad = sw128_desc(smem_base + b * kQStageBytes);
+      const uint64_t bd = sw128_desc(smem_base + b * kQStageBytes + kTm * 128u);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+        asm volatile(
+            "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+            "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem),
+            "l"(ad + static_cast<uint64_t>(2 * kk)), "l"(bd + static_cast<uint64_t>(2 * kk)), "r"(idesc), "r"(acc));
+      }
+      asm volatile(
+          "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n" ::"r"(
+              smem_u32(&empty_bar[b])),
+          "h"(static_cast<uint16_t>(3))
+          : "memory");
+    }
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n" ::"r"(
+            smem_u32(&done_bar)),
+        "h"(static_cast<uint16_t>(3))
+        : "memory");
+  } else if (tid == kQTmaWarp * 32) {
+    // ------------------------------------------------------------ TMA copies
+    const int nch = (nst + kChunkStages - 1) / kChunkStages;
+    const int pre = nch < kQP ? nch : kQP;
+    const int iq = static_cast<int>(i0) + 128 * static_cast<int>(rank);  // this CTA's activation rows
+    auto chunk_x = [&](int c) { return 2 * kChunkStages * c; };
+    for (int c = 0; c < pre; ++c) {
+      mbar_expect_tx(smem_u32(&chunk_full[c]), kQChunkBytes);
+      tma_load_2d(smem_u32(chunks + c * kQChunkBytes), &tmap_w, chunk_x(c), static_cast<int>(j0),
+                  smem_u32(&chunk_full[c]));
+    }
+    bnn::pdl_wait();
+    for (int c = 0; c < pre; ++c)
+      tma_load_2d(smem_u32(chunks + c * kQChunkBytes) + kTm * 16u * kChunkStages, &tmap_x, chunk_x(c), iq,
+                  smem_u32(&chunk_full[c]));
+    int issued = pre;
+    for (int c = pre; c < nch; ++c) {
+      const int pb = c % kQP;
+      if (!bnn::tc::mbar_wait(smem_u32(&chunk_empty[pb]), static_cast<uint32_t>((c / kQP + 1) & 1), &abort_flag,
+                              &g_bnn_device_errors, wait_limit))
+        break;
+      const uint32_t dst = smem_u32(chunks + pb * kQChunkBytes);
+      const uint32_t bar = smem_u32(&chunk_full[pb]);
+      mbar_expect_tx(bar, kQChunkBytes);
+      tma_load_2d(dst, &tmap_w, chunk_x(c), static_cast<int>(j0), bar);
+      tma_load_2d(dst + kTm * 16u * kChunkStages, &tmap_x, chunk_x(c), iq, bar);
+      issued = c + 1;
+    }
+    for (int c = issued - kQP; c < issued; ++c)
+      if (c >= 0)
+        bnn::tc::mbar_drain(smem_u32(&chunk_full[c % kQP]), static_cast<uint32_t>((c / kQP) & 1),
+                            &g_bnn_device_errors);
+  }
+  __syncwarp();
+
+  // -------------------------------------------------------------- epilogue
+  if (tid < kQProducers) asm volatile("bar.sync 1, %0;\n" ::"r"(kQProducers) : "memory");
+  bool drained = true;
+  if (warp < 8) {
+    drained = bnn::tc::mbar_drain(smem_u32(&done_bar), 0u, &g_bnn_device_errors);
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+  }
+  const bool good = __syncthreads_and(drained && abort_flag == 0) != 0;
+  if (tid == 0 && !good)  // the tile is incomplete: neither CTA writes it
+    for (uint32_t q = 0; q < 2; ++q) atomicExch(cluster.map_shared_rank(&any_bad, q), 1);
+  cluster.sync();  // popcounts final in both CTAs; abort flags exchanged
+  for (int i = tid; i < 2 * kTm; i += blockDim.x) pop_xt[i] = cluster.map_shared_rank(pop_x, i / kTm)[i % kTm];
+  __syncthreads();
+
+  const int erow = 32 * (warp & 3) + lane;
+  const int ecol0 = (warp >> 2) * 128;
+  const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+  const bool need_y = out || next;
+  if (warp < 8 && any_bad == 0) {
+    const int64_t jrow = j0 + erow;
+    const bool jlive = jrow < n;
+    const float a_j = (need_y && jlive) ? __ldg(alpha + jrow) : 0.0f;
+    const float b_j = (bias && jlive) ? __ldg(bias + jrow) : 0.0f;
+    const int base = k - 2 * pop_w[erow];
+    const int64_t half = (j0 + 32 * (warp & 3)) / 32;
+    const bool pack = next && half < next_w32;
+    for (int c0 = ecol0; c0 < ecol0 + 128; c0 += 16) {
+      uint32_t r[16];
+      if (nst > 0) {
+        tmem_ld16(taddr + static_cast<uint32_t>(c0), r);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int c = 0; c < 16; ++c) r[c] = 0u;
+      }
+      const int64_t rows_left = m - (i0 + c0);
+      const int nc = rows_left <= 0 ? 0 : (rows_left < 16 ? static_cast<int>(rows_left) : 16);
+      const int64_t off = (i0 + c0) * n + jrow;
+      int32_t* dp = dots ? dots + off : nullptr;
+      float* op = out ? out + off : nullptr;
+      uint32_t* np = pack ? next + (i0 + c0) * next_w32 + half : nullptr;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const int32_t d = base - 2 * pop_xt[c0 + c] + 4 * static_cast<int32_t>(r[c]);
+        const float y0 = __fmul_rn(a_j, static_cast<float>(d));
+        const float y = bias ? __fadd_rn(y0, b_j) : y0;
+        if (c < nc && jlive) {
+          if (dp) *dp = d;
+          if (op) *op = y;
+        }
+        if (np) {
+          const unsigned bits = __ballot_sync(0xffffffffu, jlive && !(y > 0.0f));
+          if (lane == 0 && c < nc) *np = bits;
+          np += next_w32;
+        }
+        dp += n;
+        op += n;
+      }
+    }
+  }
+
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+  cluster.sync();  // neither CTA leaves while the pair's tensor memory or shared memory is in use
+  if (warp == kQMmaWarp)
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kQTmemCols));
+}
+
+bnn_status launch_pair(const uint64_t* xp, const uint64_t* wp, const float* alpha, const float* bias, int64_t m,
+                       int64_t n, int k, int kw, int32_t* dots, float* out, uint64_t* next, cudaStream_t s,
+                       bool* launched) {
+  *launched = false;
+  const int64_t gx = 2 * ((n + 255) / 256), gy = (m + 255) / 256;
+  if (gx > 2147483647LL || gy > 65535 || kw <= 0 || kw % 2 != 0 || !bnn::aligned(xp, 16) || !bnn::aligned(wp, 16) ||
+      n >= (1LL << 31) || m >= (1LL << 31))
+    return BNN_OK;
+  CUtensorMap tw, tx;
+  if (!bnn::encode_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT64, wp, static_cast<uint64_t>(kw),
+                           static_cast<uint64_t>(n), static_cast<uint64_t>(kw) * 8u, 2 * kChunkStages, kTm,
+                           CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !bnn::encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT64, xp, static_cast<uint64_t>(kw),
+                           static_cast<uint64_t>(m), static_cast<uint64_t>(kw) * 8u, 2 * kChunkStages, kTm,
+                           CU_TENSOR_MAP_SWIZZLE_64B))
+    return BNN_OK;
+  const size_t smem = static_cast<size_t>(kQSmem) + 1024;
+  BNN_TRY(bnn::ensure_smem(binary_gemm_pair_kernel, smem));
+  const cudaError_t e = bnn::launch_pdl(binary_gemm_pair_kernel, dim3(static_cast<unsigned>(gx),
+                                        static_cast<unsigned>(gy)), dim3(kQThreads), smem, s, 2u, tw, tx, alpha,
+                                        bias, m, n, k, kw, dots, out, reinterpret_cast<uint32_t*>(next),
+                                        2 * bnn::words64(n), g_wait_limit.load());
+  if (e != cudaSuccess) return bnn::cuda_fail(e);
+  *launched = true;
+  return bnn::check_launch();
+}
+
 template <int BN, int KS, bool WIDE = false>
 bnn_status launch_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha, const float* bias, int64_t m,
                      int64_t n, int k, int kw, int32_t* dots, float* out, uint64_t* next, cudaStream_t s) {
@@ -508,8 +795,10 @@ namespace bnn {
 
 // Tensor-core (tcgen05) binary GEMM; tiles chosen from a sweep over M = 64 ..
 // 8192 at N = K = 4096 and 8192.  m <= 128: 64-row activation tiles.  Larger
-// m: 256-row tiles (the widest MMA, the fewest re-expansions of the operands)
-// once they make three quarters of a wave, otherwise 128-row tiles.  When the
+// m: two-SM 256 x 256 tiles when they make two waves of CTA pairs or more
+// (16-byte aligned rows), else 256-row tiles on one SM (the widest one-SM MMA,
+// the fewest re-expansions of the operands) once they make three quarters of
+// a wave, otherwise 128-row tiles.  When the
 // tiles leave SMs idle a cluster of 4 or 2 CTAs splits each tile's stages (at
 // least 4 stages per CTA).  CTAs that fit one per SM take the deep ring (more
 // stages in flight); otherwise 64-row-tile CTAs pair up on an SM.
@@ -519,6 +808,11 @@ bnn_status binary_gemm_tc(const uint64_t* xp, const uint64_t* wp, const float* a
   const int64_t sms = sm_count();
   const int ktiles = (kw + 1) / 2;
   if (m > 128) {
+    if (((n + 255) / 256) * ((m + 255) / 256) >= sms) {  // at least two waves of 256 x 256 pair tiles
+      bool launched = false;
+      const bnn_status st = launch_pair(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s, &launched);
+      if (st != BNN_OK || launched) return st;
+    }
     if (4 * wt * ((m + 255) / 256) >= 3 * sms)
       return launch_tc<256, 1>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
     const int64_t t128 = wt * ((m + 127) / 128);

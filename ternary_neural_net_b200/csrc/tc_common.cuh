@@ -87,6 +87,49 @@ __device__ __forceinline__ bool mbar_wait_idle(uint32_t bar, uint32_t parity, vo
   return false;
 }
 
+// One poll with acquire semantics at cluster scope: the arrivals it observes
+// may come from the other CTA of a cluster (see mbar_arrive_rank), whose
+// shared-memory writes before its arrival are then visible here.
+__device__ __forceinline__ bool mbar_try_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n.reg .pred p;\nmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+      "selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// mbar_wait with cluster-scope acquire (same bounds and abort protocol).
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                                  unsigned int* errors, uint32_t polls = 0) {
+  if (polls) {
+    for (uint32_t it = 0; it < polls; ++it)
+      if (mbar_try_cluster(bar, parity)) return true;
+  } else {
+    const uint64_t t0 = global_ns();
+    for (uint32_t it = 1;; ++it) {
+      if (mbar_try_cluster(bar, parity)) return true;
+      if ((it & 63u) == 0) {
+        if (*abort_flag) return false;
+        if (global_ns() - t0 > kWaitNs) break;
+      }
+    }
+  }
+  *abort_flag = 1;
+  atomicAdd(errors, 1u);
+  return false;
+}
+
+// Arrive, with release semantics at cluster scope, on the mbarrier at the same
+// shared-memory offset in CTA `rank` of the cluster (this CTA's own included).
+__device__ __forceinline__ void mbar_arrive_rank(uint32_t bar, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(remote) : "r"(bar), "r"(rank));
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n" ::"r"(remote) : "memory");
+}
+
 // Bounded wait that ignores the abort flag (the final drains).
 __device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity, unsigned int* errors) {
   const uint64_t t0 = global_ns();

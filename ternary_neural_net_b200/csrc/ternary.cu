@@ -345,16 +345,17 @@ constexpr int kC5D = 4;                // rows per warp round
 constexpr int kC5Round = kC5Warps * kC5D;          // rows per CTA round
 constexpr int kC5Rows = 1024;          // rows of a chunk (slice sums held at once)
 static_assert(kC5Rows % kC5Round == 0, "a chunk is a whole number of rounds");
-constexpr uint32_t kDiv243Mul = 69043u, kDiv243Shift = 24;  // floor(w / 243) for w < 3^10
-constexpr uint32_t kZeroWord = 29524u;                      // all ten digits 1: trits 0
+constexpr uint32_t kDiv243Hi = 17674763u;   // ceil(2^32 / 243): floor(w / 243) = high word of w * kDiv243Hi
+constexpr uint32_t kZeroWord = 29524u;      // all ten digits 1: trits 0
 constexpr uint32_t kZeroPair = kZeroWord | (kZeroWord << 16);
+constexpr uint32_t kC5HiOff = 243u * kC5Pitch * 4u;  // bytes from the lo table to the hi table
 
 constexpr bool div243_exact() {
-  for (uint32_t w = 0; w < 59049u; ++w)
-    if ((w * kDiv243Mul) >> kDiv243Shift != w / 243u) return false;
+  for (uint64_t w = 0; w < 59049u; ++w)
+    if (((w * kDiv243Hi) >> 32) != w / 243u) return false;
   return true;
 }
-static_assert(div243_exact(), "multiply-shift division by 243");
+static_assert(div243_exact(), "multiply-high division by 243");
 
 // floats: lo [243][96], hi [243][96], slice sums [kC5Rows], x [10][96] by table position
 size_t c5_smem_bytes() { return (2u * 243u * kC5Pitch + kC5Rows + 10u * kC5Pitch) * sizeof(float); }
@@ -362,35 +363,36 @@ size_t c5_smem_bytes() { return (2u * 243u * kC5Pitch + kC5Rows + 10u * kC5Pitch
 // slice column of table position p
 __device__ __forceinline__ int c5_column(int p) { return p < 64 ? (p < 32 ? 2 * p : 2 * (p - 32) + 1) : p; }
 
-// The words of one row at this lane's three columns: VEC, one 32-bit load for
-// columns 2l, 2l + 1 (w[0]; w[1] unused); else two 16-bit loads (w[0], w[1]).
-// w[2] = column 64 + l.
+// The words of one row at this lane's three columns (o = the row's offset in
+// 16-bit words from `packed`, at column 2l): VEC, one 32-bit load for columns
+// 2l, 2l + 1 (w[0]; w[1] unused); else two 16-bit loads (w[0], w[1]).  The last
+// word is column 64 + l.  Lanes or rows outside the slice get the zero word.
 template <bool VEC>
 struct C5Words {
   uint32_t w[VEC ? 2 : 3];
 };
 
 template <bool VEC>
-__device__ __forceinline__ void c5_fetch(const uint16_t* __restrict__ row, bool live, int lane, int sw,
-                                         C5Words<VEC>& o) {
-  const bool a = live && 2 * lane < sw, b = live && 2 * lane + 1 < sw, c = live && 64 + lane < sw;
+__device__ __forceinline__ void c5_fetch(const uint16_t* __restrict__ packed, uint32_t o, uint32_t oc, bool live,
+                                         bool la, bool lb, bool lc, C5Words<VEC>& v) {
   if constexpr (VEC) {
-    o.w[0] = a ? __ldcs(reinterpret_cast<const uint32_t*>(row + 2 * lane)) : kZeroPair;
-    o.w[1] = c ? static_cast<uint32_t>(__ldcs(row + 64 + lane)) : kZeroWord;
+    v.w[0] = (live && la) ? __ldcs(reinterpret_cast<const uint32_t*>(packed + o)) : kZeroPair;
+    v.w[1] = (live && lc) ? static_cast<uint32_t>(__ldcs(packed + o + oc)) : kZeroWord;
   } else {
-    o.w[0] = a ? static_cast<uint32_t>(__ldcs(row + 2 * lane)) : kZeroWord;
-    o.w[1] = b ? static_cast<uint32_t>(__ldcs(row + 2 * lane + 1)) : kZeroWord;
-    o.w[2] = c ? static_cast<uint32_t>(__ldcs(row + 64 + lane)) : kZeroWord;
+    v.w[0] = (live && la) ? static_cast<uint32_t>(__ldcs(packed + o)) : kZeroWord;
+    v.w[1] = (live && lb) ? static_cast<uint32_t>(__ldcs(packed + o + 1)) : kZeroWord;
+    v.w[2] = (live && lc) ? static_cast<uint32_t>(__ldcs(packed + o + oc)) : kZeroWord;
   }
 }
 
-// lo_p[ql] + hi_p[qh] of one word; tl / th = this lane's table positions (bytes)
-__device__ __forceinline__ float c5_lookup(uint32_t w, uint32_t tl, uint32_t th) {
-  const uint32_t qh = (w * kDiv243Mul) >> kDiv243Shift;  // digits 5..9
-  const uint32_t ql = w - 243u * qh;                     // digits 0..4
+// lo_p[ql] + hi_p[qh] of one word; t = this lane's lo-table position (bytes),
+// plus 128 per 32 positions; the hi table sits kC5HiOff bytes above.
+__device__ __forceinline__ float c5_lookup(uint32_t w, uint32_t t) {
+  const uint32_t qh = __umulhi(w, kDiv243Hi);  // digits 5..9
+  const uint32_t ql = w - 243u * qh;          // digits 0..4
   float a, b;
-  asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(a) : "r"(tl + ql * (4u * kC5Pitch)));
-  asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(b) : "r"(th + qh * (4u * kC5Pitch)));
+  asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(a) : "r"(t + ql * (4u * kC5Pitch)));
+  asm volatile("ld.shared.f32 %0, [%1+%2];\n" : "=f"(b) : "r"(t + qh * (4u * kC5Pitch)), "n"(kC5HiOff));
   return a + b;
 }
 
@@ -398,16 +400,16 @@ __device__ __forceinline__ float c5_lookup(uint32_t w, uint32_t tl, uint32_t th)
 // a word outside the format (its result unspecified) still looks up inside the
 // tables.
 template <bool VEC>
-__device__ __forceinline__ float c5_row(const C5Words<VEC>& v, uint32_t lo0, uint32_t hi0) {
+__device__ __forceinline__ float c5_row(const C5Words<VEC>& v, uint32_t t) {
   constexpr uint32_t kMaxWord = 59048u;
   float s;
   if constexpr (VEC) {
     const uint32_t pr = __vminu2(v.w[0], kMaxWord | (kMaxWord << 16));
-    s = c5_lookup(pr & 0xFFFFu, lo0, hi0) + c5_lookup(pr >> 16, lo0 + 128u, hi0 + 128u);
-    s += c5_lookup(min(v.w[1], kMaxWord), lo0 + 256u, hi0 + 256u);
+    s = c5_lookup(pr & 0xFFFFu, t) + c5_lookup(pr >> 16, t + 128u);
+    s += c5_lookup(min(v.w[1], kMaxWord), t + 256u);
   } else {
-    s = c5_lookup(min(v.w[0], kMaxWord), lo0, hi0) + c5_lookup(min(v.w[1], kMaxWord), lo0 + 128u, hi0 + 128u);
-    s += c5_lookup(min(v.w[2], kMaxWord), lo0 + 256u, hi0 + 256u);
+    s = c5_lookup(min(v.w[0], kMaxWord), t) + c5_lookup(min(v.w[1], kMaxWord), t + 128u);
+    s += c5_lookup(min(v.w[2], kMaxWord), t + 256u);
   }
   return s;
 }
@@ -449,11 +451,19 @@ ternary_gemv_c5_kernel(const uint16_t* __restrict__ x, const uint16_t* __restric
   const int rounds = static_cast<int>((c1 - c0 + kC5Round - 1) / kC5Round);
   bnn::pdl_trigger();
 
-  const uint16_t* const wbase = packed + w0;
+  // 16-bit word offsets from `packed` (the launch keeps n * kt below 2^31):
+  // this warp's rows of round i start at local row 128 i + 4 warp
+  const int rows_c = static_cast<int>(c1 - c0);
+  const uint32_t ktu = static_cast<uint32_t>(kt);
+  const uint32_t off0 = (static_cast<uint32_t>(c0) + 4u * static_cast<uint32_t>(warp)) * ktu +
+                        static_cast<uint32_t>(w0 + 2 * lane);
+  const uint32_t oc = 64u - static_cast<uint32_t>(lane);  // column 64 + l from column 2l
+  const bool la = 2 * lane < sw, lb = 2 * lane + 1 < sw, lc = 64 + lane < sw;
   auto fetch_round = [&](int i, C5Words<VEC> (&buf)[kC5D]) {
-    const int64_t r0 = c0 + static_cast<int64_t>(i) * kC5Round + warp * kC5D;
+    const uint32_t o = off0 + static_cast<uint32_t>(i) * (static_cast<uint32_t>(kC5Round) * ktu);
+    const int nl = rows_c - (i * kC5Round + warp * kC5D);  // live rows of the four
 #pragma unroll
-    for (int j = 0; j < kC5D; ++j) c5_fetch<VEC>(wbase + (r0 + j) * kt, i < rounds && r0 + j < c1, lane, sw, buf[j]);
+    for (int j = 0; j < kC5D; ++j) c5_fetch<VEC>(packed, o + j * ktu, oc, j < nl, la, lb, lc, buf[j]);
   };
   C5Words<VEC> bufA[kC5D], bufB[kC5D], bufC[kC5D];
   fetch_round(0, bufA);
@@ -491,16 +501,16 @@ ternary_gemv_c5_kernel(const uint16_t* __restrict__ x, const uint16_t* __restric
   }
   __syncthreads();
 
-  const uint32_t lo0 = static_cast<uint32_t>(__cvta_generic_to_shared(lo)) + 4u * static_cast<uint32_t>(lane);
-  const uint32_t hi0 = static_cast<uint32_t>(__cvta_generic_to_shared(hi)) + 4u * static_cast<uint32_t>(lane);
+  const uint32_t tl = static_cast<uint32_t>(__cvta_generic_to_shared(lo)) + 4u * static_cast<uint32_t>(lane);
   const bool upper = (lane & 16) != 0, mid = (lane & 8) != 0;
-  // round i: the rows of bufX, with the round two ahead loaded into bufY
+  // round i: the rows of `cur`, with the round two ahead loaded into `ahead`
   auto round = [&](int i, C5Words<VEC> (&cur)[kC5D], C5Words<VEC> (&ahead)[kC5D]) {
     fetch_round(i + 2, ahead);
-    const int64_t r0 = c0 + static_cast<int64_t>(i) * kC5Round + warp * kC5D;
+    const int rl0 = i * kC5Round + warp * kC5D;  // local row of cur[0]
+    const int nl = rows_c - rl0;
     float acc[kC5D];
 #pragma unroll
-    for (int j = 0; j < kC5D; ++j) acc[j] = r0 + j < c1 ? c5_row<VEC>(cur[j], lo0, hi0) : 0.0f;
+    for (int j = 0; j < kC5D; ++j) acc[j] = j < nl ? c5_row<VEC>(cur[j], tl) : 0.0f;
     // four rows over 32 lanes: halves exchange rows (0,1) / (2,3), then quarters
     // row 0 / 1 of their pair; lane group (lane >> 3) ends with row 2 (lane >> 4) + (lane >> 3 & 1)
     float k0 = upper ? acc[2] : acc[0], k1 = upper ? acc[3] : acc[1];
@@ -513,19 +523,19 @@ ternary_gemv_c5_kernel(const uint16_t* __restrict__ x, const uint16_t* __restric
     v += __shfl_xor_sync(0xffffffffu, v, 2);
     v += __shfl_xor_sync(0xffffffffu, v, 1);
     const int j = lane >> 3;
-    const int64_t cs = c0 + static_cast<int64_t>(i / (kC5Rows / kC5Round)) * kC5Rows;  // the chunk's first row
-    if ((lane & 7) == 0 && r0 + j < c1) psum[r0 + j - cs] = v;
-    if (i % (kC5Rows / kC5Round) == kC5Rows / kC5Round - 1 || i == rounds - 1) {
+    if ((lane & 7) == 0 && j < nl) psum[(rl0 + j) & (kC5Rows - 1)] = v;  // chunks start at multiples of kC5Rows
+    constexpr int kRoundsPerChunk = kC5Rows / kC5Round;
+    if (i % kRoundsPerChunk == kRoundsPerChunk - 1 || i == rounds - 1) {
       // end of a chunk: its slice sums added in rank order by the CTA that owns the row
       cluster.sync();
-      const int64_t ce = cs + kC5Rows < c1 ? cs + kC5Rows : c1;
-      const int rows = static_cast<int>(ce - cs);
+      const int cb = (i / kRoundsPerChunk) * kC5Rows;  // the chunk's first local row
+      const int rows = rows_c - cb < kC5Rows ? rows_c - cb : kC5Rows;
       const int q0 = rows * rank / kC5, q1 = rows * (rank + 1) / kC5;
       for (int rl = q0 + tid; rl < q1; rl += kC5Threads) {
         float sum = 0.0f;
 #pragma unroll
         for (int q = 0; q < kC5; ++q) sum += cluster.map_shared_rank(psum, q)[rl];
-        const int64_t r = cs + rl;
+        const int64_t r = c0 + cb + rl;
         out[r] = bias ? __ldg(scale + r) * sum + __ldg(bias + r) : __ldg(scale + r) * sum;
       }
       cluster.sync();  // slice sums read before the next chunk overwrites them (and before any CTA exits)
@@ -809,7 +819,8 @@ bnn_status ternary_gemm_impl(const uint16_t* x_bf16, const uint16_t* packed, con
   // for one activation tile, into shared memory above that)
   if (algo == BNN_TALGO_AUTO && m > 8 && k % 8 == 0 && bnn::aligned(x_bf16, 16))
     return bnn::ternary_gemm_tc(x_bf16, packed, scale, bias, m, n, k, out, s);
-  if (algo != BNN_TALGO_MMA && m == 1 && kt > 0 && kt <= kC5 * kC5Pitch) {
+  // (the table kernel addresses the words with 32-bit offsets)
+  if (algo != BNN_TALGO_MMA && m == 1 && kt > 0 && kt <= kC5 * kC5Pitch && (n + 512) * kt < (int64_t{1} << 31)) {
     const int clusters = c5_clusters();
     if (clusters > 0) {
       // 32-bit word pairs where every row's slices start 4-byte aligned: kt even, the slice even
