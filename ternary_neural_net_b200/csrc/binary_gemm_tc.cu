@@ -498,7 +498,9 @@ constexpr int kQRows = 256;                                  // stacked rows per
 constexpr uint32_t kQStageBytes = kQRows * 128u;             // one expanded stage (32 KiB)
 constexpr uint32_t kQChunkBytes = kQRows * 16u * kChunkStages;  // one packed chunk (16 KiB)
 constexpr int kQS = 5, kQP = 2;                              // expanded stages, packed chunks
-constexpr int kQProducers = 2 * kQRows;                      // 512
+constexpr int kQG = kChunkStages;                            // producer groups (one stage of every chunk each)
+constexpr int kQGroup = kTm;                                 // threads per group (one weight + one activation row each)
+constexpr int kQProducers = kQG * kQGroup;                   // 512
 constexpr int kQWarps = kQProducers / 32;                    // producer warps per CTA
 constexpr int kQMmaWarp = kQWarps, kQTmaWarp = kQWarps + 1;
 constexpr int kQThreads = kQProducers + 64;
@@ -537,12 +539,12 @@ binary_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
   for (int i = tid; i < kTm; i += blockDim.x) pop_w[i] = pop_x[i] = 0;
   if (tid == 0) {
     for (int i = 0; i < kQS; ++i) {
-      bnn::tc::mbar_init(smem_u32(&full_bar[i]), 2 * kQWarps);
+      bnn::tc::mbar_init(smem_u32(&full_bar[i]), 2);  // one arrival per CTA: the group that wrote the stage
       bnn::tc::mbar_init(smem_u32(&empty_bar[i]), 1);
     }
     for (int i = 0; i < kQP; ++i) {
       bnn::tc::mbar_init(smem_u32(&chunk_full[i]), 1);
-      bnn::tc::mbar_init(smem_u32(&chunk_empty[i]), kQWarps);
+      bnn::tc::mbar_init(smem_u32(&chunk_empty[i]), kQG);  // one arrival per group
     }
     bnn::tc::mbar_init(smem_u32(&done_bar), 1);
     abort_flag = 0;
@@ -566,38 +568,44 @@ binary_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
 
   if (tid < kQProducers) {
     // ------------------------------------------------------------ producers
-    const int r2 = tid >> 1, part = tid & 1;
-    const bool is_w = r2 < kTm;
-    const int row = is_w ? r2 : r2 - kTm;
-    const uint32_t row_off = static_cast<uint32_t>(r2) * 128u;
-    const uint32_t swz = static_cast<uint32_t>(row & 7);
-    const uint32_t rd_off = static_cast<uint32_t>(r2) * 64u + 8u * static_cast<uint32_t>(part);
-    const uint32_t rd_swz = static_cast<uint32_t>((r2 >> 1) & 3);
-    int my_pop = 0;
-    for (int j = 0; j < nst; ++j) {
-      const int c = j / kChunkStages, s = j % kChunkStages, pb = c % kQP;
-      bool ok = true;
-      if (s == 0)
-        ok = bnn::tc::mbar_wait(smem_u32(&chunk_full[pb]), static_cast<uint32_t>((c / kQP) & 1), &abort_flag,
-                                &g_bnn_device_errors, wait_limit);
-      const int b = j % kQS;
+    // group g = tid / kQGroup takes the stages j = g (mod kQG); its thread t
+    // takes weight row t and activation row t (stacked row kTm + t), both
+    // 64-bit words of the stage
+    const int g = tid / kQGroup, t = tid % kQGroup;
+    const uint32_t swz = static_cast<uint32_t>(t & 7);
+    int pop_a = 0, pop_b = 0;
+    for (int j = g; j < nst; j += kQG) {
+      const int c = j / kChunkStages, s = j % kChunkStages, pb = c % kQP, b = j % kQS;
+      bool ok = bnn::tc::mbar_wait(smem_u32(&chunk_full[pb]), static_cast<uint32_t>((c / kQP) & 1), &abort_flag,
+                                   &g_bnn_device_errors, wait_limit);
       // refill only after the tensor core has read the previous fill of this buffer
       if (ok && j >= kQS)
         ok = bnn::tc::mbar_wait(smem_u32(&empty_bar[b]), static_cast<uint32_t>((j / kQS + 1) & 1), &abort_flag,
                                 &g_bnn_device_errors, wait_limit);
-      if (!__all_sync(0xffffffffu, ok)) break;  // the warp stops together
-      const uint64_t cw = *reinterpret_cast<const uint64_t*>(
-          chunks + pb * kQChunkBytes + rd_off + ((static_cast<uint32_t>(s) ^ rd_swz) << 4));
-      my_pop += __popcll(cw);
-      expand_word(smem + b * kQStageBytes + row_off, swz, part, cw);
-      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-      __syncwarp();
-      if (lane == 0) {
-        if (s == kChunkStages - 1 || j == nst - 1) mbar_arrive(smem_u32(&chunk_empty[pb]));
+      if (ok) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {  // h = 0: the weight row, 1: the activation row
+          const int r2 = t + h * kTm;
+          // the row's 16 bytes of stage s in the chunk (64-byte swizzle: unit s ^ bits 1-2 of the row)
+          const uint4 v = *reinterpret_cast<const uint4*>(chunks + pb * kQChunkBytes + r2 * 64u +
+                                                          ((static_cast<uint32_t>(s) ^ ((r2 >> 1) & 3)) << 4));
+          const uint64_t w0 = (static_cast<uint64_t>(v.y) << 32) | v.x, w1 = (static_cast<uint64_t>(v.w) << 32) | v.z;
+          (h == 0 ? pop_a : pop_b) += __popcll(w0) + __popcll(w1);
+          uint8_t* dst = smem + b * kQStageBytes + static_cast<uint32_t>(r2) * 128u;
+          expand_word(dst, swz, 0, w0);
+          expand_word(dst, swz, 1, w1);
+        }
+        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+      }
+      // the group's rows of stage j are written (or some wait ran out: the group stops together)
+      if (!bnn::tc::named_barrier_and(ok, 2 + g, kQGroup)) break;
+      if (t == 0) {
+        mbar_arrive(smem_u32(&chunk_empty[pb]));  // this group's stage of chunk c is read
         bnn::tc::mbar_arrive_rank(smem_u32(&full_bar[b]), 0u);
       }
     }
-    atomicAdd(is_w ? &pop_w[row] : &pop_x[row], my_pop);
+    atomicAdd(&pop_w[t], pop_a);
+    atomicAdd(&pop_x[t], pop_b);
   } else if (tid == kQMmaWarp * 32 && rank == 0) {
     // ------------------------------------------------------------ MMA issue
     // D s32, A and B 8-bit integers, both K-major, N = 256, M = 256 (two CTAs)

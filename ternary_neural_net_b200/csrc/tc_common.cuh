@@ -165,6 +165,18 @@ __device__ __forceinline__ bool producer_barrier_and(bool pred, int count) {
   return r != 0;
 }
 
+// Named barrier `id` over `count` threads (whole warps) returning the AND of
+// every participant's `pred`.
+__device__ __forceinline__ bool named_barrier_and(bool pred, int id, int count) {
+  uint32_t r;
+  asm volatile(
+      "{\n.reg .pred p, q;\nsetp.ne.u32 p, %1, 0;\nbar.red.and.pred q, %2, %3, p;\nselp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"(pred ? 1u : 0u), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+
 // 2-D tiled TMA load of one box into this CTA's shared memory (x = innermost
 // element index, y = row), completing its bytes on the mbarrier.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* map, int x, int y, uint32_t bar) {
