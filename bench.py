@@ -512,9 +512,9 @@ def gpu_cfg4(cu, seed, P, st, s, pk, head=None):
         del d, o
     return dict(value=macs / (ms * 1e-3) / 1e9, unit="GMAC/s", ms_kernel=ms, macs=macs,
                 roofline=roofline("tensor", 2 * macs / (ms * 1e-3) / 1e12, int8, "TOP/s",
-                                  "binary_gemm_tc_kernel<256,1> (128x256 tiles)",
+                                  "binary_gemm_pair_kernel (persistent CTA pairs, 256x256 tiles)",
                                   f"int8 dense = 2 x bf16 {pk['bf16_tflops']} TFLOP/s ({pk['src']})",
-                                  traffic_for("binary_gemm_tc_256x1", "ternary_neural_net_b200/csrc/binary_gemm_tc.cu")))
+                                  traffic_for("binary_gemm_pair_m8192", "ternary_neural_net_b200/csrc/binary_gemm_tc.cu")))
 
 
 def gpu_cfg5(cu, seed, P, st, s, pk):
@@ -1054,14 +1054,16 @@ def main(argv=None):
                          f"512 MiB of outputs, so every step starts cold",
                    "parallelism": f"replicas x{N} (independent problems per GPU)"},
         "roofline": {"bound": "tensor",
-                     "kernel": "binary_gemm_tc_kernel<256,1> (bnn_binary_gemm AUTO for m > 128 with 3/4 of a wave "
-                               "of 128x256 tiles or more): TMA-fed packed chunks -> 0/1 bytes in swizzled smem, "
-                               "tcgen05.mma kind::i8 into tensor memory, epilogue by the producer warps",
+                     "kernel": "binary_gemm_pair_kernel (bnn_binary_gemm AUTO at two waves of 256x256 CTA-pair "
+                               "tiles or more): persistent 2-CTA clusters, TMA-fed packed chunks -> 0/1 bytes in "
+                               "swizzled smem by four producer groups, tcgen05.mma.cta_group::2 kind::i8 into a "
+                               "double-buffered tensor-memory accumulator, epilogue warps overlapping the next tile "
+                               "(+ row_popcount_kernel, ~1% of the step)",
                      "achieved": achieved, "peak": int8_peak, "unit": "TOP/s", "frac": achieved / int8_peak,
                      "achieved_basis": "2 ops x M*N*K per launch / the timed region's duration / K (the step is "
                                        "this one kernel; CUDA events on the launching stream)",
                      "kernel_ms": head["kernel_ms"], "kernel_ms_events": head["kernel_ms_events"],
-                     "traffic": traffic_for("binary_gemm_tc_256x1", "ternary_neural_net_b200/csrc/binary_gemm_tc.cu"),
+                     "traffic": traffic_for("binary_gemm_pair_m8192", "ternary_neural_net_b200/csrc/binary_gemm_tc.cu"),
                      "peak_basis": f"int8 dense tensor peak = bf16 {peaks['bf16_tflops']} TFLOP/s x 2 (nominal "
                                    f"int8:bf16 ratio 4.5:2.25 PFLOP/s), {peak_src} (burst figure: a kernel timed "
                                    f"alone)"},
@@ -1075,7 +1077,7 @@ def main(argv=None):
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                 "ms_per_step": e2e["ms_per_step"], "pipelining": e2e["pipelining"],
                 "check": e2e_consistency(head) if lead else None},
-        "gpu_launches": K,
+        "gpu_launches": 2 * K,  # per step: row_popcount_kernel + binary_gemm_pair_kernel
         "timing": "W eager warm-up steps, then K steps captured in one CUDA graph, replayed once untimed and once "
                   "between CUDA events on the launching stream (barrier + synchronize on both sides)",
         "clocks": head["clocks"],

@@ -80,6 +80,44 @@ cudaError_t ensure_smem_raw(const void* kernel, size_t bytes) {
 }
 
 namespace {
+struct PoolSlot {
+  uint64_t ctx;
+  cudaMemPool_t pool;
+};
+constexpr int kPoolDevices = 64;
+PoolSlot g_pool[kPoolDevices] = {};
+std::mutex g_pool_mu;
+}  // namespace
+
+cudaError_t scratch_alloc(void** p, size_t bytes, cudaStream_t s) {
+  const int dev = current_device();
+  cudaMemPool_t pool = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_pool_mu);
+    const uint64_t ctx = context_id();
+    const bool cacheable = dev >= 0 && dev < kPoolDevices && ctx != 0;
+    if (cacheable && g_pool[dev].ctx == ctx && g_pool[dev].pool) {
+      pool = g_pool[dev].pool;
+    } else {
+      cudaMemPoolProps props = {};
+      props.allocType = cudaMemAllocationTypePinned;
+      props.location.type = cudaMemLocationTypeDevice;
+      props.location.id = dev;
+      cudaError_t e = cudaMemPoolCreate(&pool, &props);
+      if (e != cudaSuccess) return e;
+      uint64_t keep = ~uint64_t{0};  // never trim at synchronisation
+      e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+      if (e != cudaSuccess) {
+        cudaMemPoolDestroy(pool);
+        return e;
+      }
+      if (cacheable) g_pool[dev] = PoolSlot{ctx, pool};
+    }
+  }
+  return cudaMallocFromPoolAsync(p, bytes, pool, s);
+}
+
+namespace {
 using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);

@@ -472,83 +472,97 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
 }
 
 // ---------------------------------------------------------------------------
-// Two-SM variant for large GEMMs: a cluster of two CTAs computes one tile of
-// 256 weight rows x 256 activation rows with tcgen05.mma.cta_group::2 (UMMA
-// M = 256, N = 256).  CTA q of the pair holds weight rows 128q.. of the tile
-// (its half of operand A, and the tensor-memory lanes of those rows) and
+// Two-SM persistent variant for large GEMMs.  A cluster of two CTAs computes
+// tiles of 256 weight rows x 256 activation rows with tcgen05.mma.cta_group::2
+// (UMMA M = 256, N = 256): CTA q of the pair holds weight rows 128q.. of the
+// tile (its half of operand A, and the tensor-memory lanes of those rows) and
 // activation rows 128q.. (its half of operand B); one MMA reads both CTAs'
-// shared memory, so each SM expands and feeds only 256 rows per stage instead
-// of the 384 of a 128 x 256 tile on one SM, and its tensor memory receives all
-// 256 accumulator columns of its 128 weight rows.
+// shared memory, so each SM expands only 256 rows per stage instead of the
+// 384 of a 128 x 256 tile on one SM, and its tensor memory receives all 256
+// accumulator columns of its 128 weight rows.  The pairs are persistent: pair
+// p takes tiles p, p + P, ... (P pairs, at most as many as fit the GPU at
+// once), and the accumulator is double-buffered in tensor memory (2 x 256
+// columns), so the epilogue of one tile overlaps the mainloop of the next.
 //
-// Roles per CTA as in the kernel above (two producer threads per stacked row,
-// a TMA thread for the packed chunks of its own rows), with these changes:
-//   - producers signal per warp (fence to the async proxy, a warp barrier,
-//     then lane 0 arrives) on the stage's "full" mbarrier of CTA 0, at cluster
-//     scope, so that barrier completes once both CTAs' 32 producer warps have
-//     written the stage;
-//   - only CTA 0 issues the MMAs; tcgen05.commit with a two-CTA mask arrives
-//     on the "empty" barrier of the stage in both CTAs (and on "done" after the
-//     last stage);
-//   - the epilogue reads the other CTA's activation-row popcounts through
-//     distributed shared memory.
-// Every wait is bounded; an abort in either CTA leaves the whole tile unwritten.
+// Roles per CTA:
+//   - a TMA thread copies the packed chunks (4 stages of its own 128 weight and
+//     128 activation rows) into a two-chunk ring;
+//   - four producer groups of 128 threads; group g takes stage g of every
+//     chunk, thread t weight row t and activation row t (both 64-bit words of
+//     the stage), so four stages are expanded at once and the latency of one
+//     (loads, stores, proxy fence, barrier) hides behind the others.  After a
+//     named barrier of its 128 threads a group arrives once on the stage's
+//     "full" mbarrier of CTA 0 (at cluster scope), which thus completes once
+//     both CTAs' groups have written the stage;
+//   - CTA 0's MMA thread waits for "full", issues 4 tcgen05.mma (K = 32) into
+//     accumulator buffer t % 2, and commits with a two-CTA mask to the stage's
+//     "empty" barrier in both CTAs (and to "acc_full" after a tile's last
+//     stage); before a tile it waits on "acc_empty" for the epilogue that read
+//     the buffer two tiles back;
+//   - four epilogue warps (one per quarter of the tensor-memory lanes) read
+//     the accumulator, apply the popcount correction (row popcounts from a
+//     pass before the kernel), alpha and the optional bias, store, and arrive
+//     on CTA 0's "acc_empty".
+// The stage, chunk and accumulator rings run on across tiles.  Every wait is
+// bounded; a wait that runs out stops every role of the CTA (the other CTA's
+// waits then run out too) and leaves the outputs unspecified.
 // ---------------------------------------------------------------------------
-constexpr int kQRows = 256;                                  // stacked rows per CTA (128 weight + 128 activation)
-constexpr uint32_t kQStageBytes = kQRows * 128u;             // one expanded stage (32 KiB)
+constexpr int kQRows = 256;                                     // stacked rows per CTA (128 weight + 128 activation)
+constexpr uint32_t kQStageBytes = kQRows * 128u;                // one expanded stage (32 KiB)
 constexpr uint32_t kQChunkBytes = kQRows * 16u * kChunkStages;  // one packed chunk (16 KiB)
-constexpr int kQS = 5, kQP = 2;                              // expanded stages, packed chunks
-constexpr int kQG = kChunkStages;                            // producer groups (one stage of every chunk each)
-constexpr int kQGroup = kTm;                                 // threads per group (one weight + one activation row each)
-constexpr int kQProducers = kQG * kQGroup;                   // 512
-constexpr int kQWarps = kQProducers / 32;                    // producer warps per CTA
-constexpr int kQMmaWarp = kQWarps, kQTmaWarp = kQWarps + 1;
-constexpr int kQThreads = kQProducers + 64;
+constexpr int kQS = 5, kQP = 2;                                 // expanded stages, packed chunks
+constexpr int kQG = kChunkStages;                               // producer groups (one stage of every chunk each)
+constexpr int kQGroup = kTm;                                    // threads per group
+constexpr int kQProducers = kQG * kQGroup;                      // 512
+constexpr int kQMmaWarp = kQProducers / 32, kQTmaWarp = kQMmaWarp + 1, kQEpiWarp0 = kQMmaWarp + 2;
+constexpr int kQThreads = kQProducers + 64 + 128;               // + MMA warp + TMA warp + 4 epilogue warps
 constexpr uint32_t kQSmem = kQS * kQStageBytes + kQP * kQChunkBytes;
-constexpr uint32_t kQTmemCols = 256;
+constexpr uint32_t kQTmemCols = 512;                            // two 256-column accumulators
+constexpr int kQEpiBar = 2 + kQG;                               // named barrier of the epilogue warps
 
 __global__ void __launch_bounds__(kQThreads, 1)
 binary_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
-                        const float* __restrict__ alpha, const float* __restrict__ bias, int64_t m, int64_t n, int k,
+                        const float* __restrict__ alpha, const float* __restrict__ bias,
+                        const int* __restrict__ pop_x, const int* __restrict__ pop_w, int64_t m, int64_t n, int k,
                         int kw, int32_t* __restrict__ dots, float* __restrict__ out, uint32_t* __restrict__ next,
                         int64_t next_w32, uint32_t wait_limit) {
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full_bar[kQS];   // CTA 0's: both CTAs' producer warps arrive
+  __shared__ __align__(8) uint64_t full_bar[kQS];   // CTA 0's: one arrival per CTA
   __shared__ __align__(8) uint64_t empty_bar[kQS];
   __shared__ __align__(8) uint64_t chunk_full[kQP];
   __shared__ __align__(8) uint64_t chunk_empty[kQP];
+  __shared__ __align__(8) uint64_t acc_full[2];
+  __shared__ __align__(8) uint64_t acc_empty[2];    // CTA 0's: one arrival per CTA
   __shared__ __align__(8) uint64_t done_bar;
   __shared__ uint32_t tmem_holder;
   __shared__ volatile int abort_flag;
-  __shared__ int any_bad;
-  __shared__ int pop_w[kTm];
-  __shared__ int pop_x[kTm];        // this CTA's 128 activation rows
-  __shared__ int pop_xt[2 * kTm];   // the tile's 256 activation rows
   uint8_t* const smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* const chunks = smem + kQS * kQStageBytes;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster.block_rank();
-  const int64_t j0 = static_cast<int64_t>(blockIdx.x >> 1) * 256 + 128 * rank;  // this CTA's weight rows
-  const int64_t i0 = static_cast<int64_t>(blockIdx.y) * 256;                      // the tile's activation rows
-  const int nst = (kw + 1) / 2;
+  const int64_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int64_t ntn = (n + 255) / 256, ntiles = ntn * ((m + 255) / 256);
+  const int nst = (kw + 1) / 2, nch = (nst + kChunkStages - 1) / kChunkStages;
   const uint32_t smem_base = smem_u32(smem);
 
-  for (int i = tid; i < kTm; i += blockDim.x) pop_w[i] = pop_x[i] = 0;
   if (tid == 0) {
     for (int i = 0; i < kQS; ++i) {
-      bnn::tc::mbar_init(smem_u32(&full_bar[i]), 2);  // one arrival per CTA: the group that wrote the stage
+      bnn::tc::mbar_init(smem_u32(&full_bar[i]), 2);
       bnn::tc::mbar_init(smem_u32(&empty_bar[i]), 1);
     }
     for (int i = 0; i < kQP; ++i) {
       bnn::tc::mbar_init(smem_u32(&chunk_full[i]), 1);
-      bnn::tc::mbar_init(smem_u32(&chunk_empty[i]), kQG);  // one arrival per group
+      bnn::tc::mbar_init(smem_u32(&chunk_empty[i]), kQG);
+    }
+    for (int i = 0; i < 2; ++i) {
+      bnn::tc::mbar_init(smem_u32(&acc_full[i]), 1);
+      bnn::tc::mbar_init(smem_u32(&acc_empty[i]), 2);
     }
     bnn::tc::mbar_init(smem_u32(&done_bar), 1);
     abort_flag = 0;
-    any_bad = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
   if (tid == kQTmaWarp * 32) {
@@ -568,185 +582,253 @@ binary_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
 
   if (tid < kQProducers) {
     // ------------------------------------------------------------ producers
-    // group g = tid / kQGroup takes the stages j = g (mod kQG); its thread t
-    // takes weight row t and activation row t (stacked row kTm + t), both
-    // 64-bit words of the stage
     const int g = tid / kQGroup, t = tid % kQGroup;
     const uint32_t swz = static_cast<uint32_t>(t & 7);
-    int pop_a = 0, pop_b = 0;
-    for (int j = g; j < nst; j += kQG) {
-      const int c = j / kChunkStages, s = j % kChunkStages, pb = c % kQP, b = j % kQS;
-      bool ok = bnn::tc::mbar_wait(smem_u32(&chunk_full[pb]), static_cast<uint32_t>((c / kQP) & 1), &abort_flag,
-                                   &g_bnn_device_errors, wait_limit);
-      // refill only after the tensor core has read the previous fill of this buffer
-      if (ok && j >= kQS)
-        ok = bnn::tc::mbar_wait(smem_u32(&empty_bar[b]), static_cast<uint32_t>((j / kQS + 1) & 1), &abort_flag,
+    const uint32_t rd = ((static_cast<uint32_t>(g) ^ ((t >> 1) & 3)) << 4);  // stage g's unit in a chunk row
+    bool ok = true;
+    int64_t gc = 0;  // chunks consumed so far (all tiles)
+    for (int64_t tile = pair, ti = 0; tile < ntiles && ok; tile += npairs, ++ti) {
+      for (int c = 0; c < nch; ++c, ++gc) {
+        const int pb = static_cast<int>(gc % kQP);
+        const int j = kChunkStages * c + g;           // this group's stage of the chunk
+        const bool has = j < nst;
+        const int64_t gs = ti * nst + j;              // stage count over all tiles
+        const int b = static_cast<int>(gs % kQS);
+        ok = bnn::tc::mbar_wait(smem_u32(&chunk_full[pb]), static_cast<uint32_t>((gc / kQP) & 1), &abort_flag,
                                 &g_bnn_device_errors, wait_limit);
-      if (ok) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {  // h = 0: the weight row, 1: the activation row
-          const int r2 = t + h * kTm;
-          // the row's 16 bytes of stage s in the chunk (64-byte swizzle: unit s ^ bits 1-2 of the row)
-          const uint4 v = *reinterpret_cast<const uint4*>(chunks + pb * kQChunkBytes + r2 * 64u +
-                                                          ((static_cast<uint32_t>(s) ^ ((r2 >> 1) & 3)) << 4));
-          const uint64_t w0 = (static_cast<uint64_t>(v.y) << 32) | v.x, w1 = (static_cast<uint64_t>(v.w) << 32) | v.z;
-          (h == 0 ? pop_a : pop_b) += __popcll(w0) + __popcll(w1);
-          uint8_t* dst = smem + b * kQStageBytes + static_cast<uint32_t>(r2) * 128u;
-          expand_word(dst, swz, 0, w0);
-          expand_word(dst, swz, 1, w1);
+        // refill only after the tensor core has read the previous fill of this buffer
+        if (ok && has && gs >= kQS)
+          ok = bnn::tc::mbar_wait(smem_u32(&empty_bar[b]), static_cast<uint32_t>((gs / kQS + 1) & 1), &abort_flag,
+                                  &g_bnn_device_errors, wait_limit);
+        if (ok && has) {
+          const uint8_t* ck = chunks + pb * kQChunkBytes + rd;
+          const uint4 vw = *reinterpret_cast<const uint4*>(ck + t * 64u);
+          const uint4 vx = *reinterpret_cast<const uint4*>(ck + (t + kTm) * 64u);  // same swizzle unit as row t
+          uint8_t* dst = smem + b * kQStageBytes + static_cast<uint32_t>(t) * 128u;
+          expand_word(dst, swz, 0, (static_cast<uint64_t>(vw.y) << 32) | vw.x);
+          expand_word(dst, swz, 1, (static_cast<uint64_t>(vw.w) << 32) | vw.z);
+          expand_word(dst + kTm * 128u, swz, 0, (static_cast<uint64_t>(vx.y) << 32) | vx.x);
+          expand_word(dst + kTm * 128u, swz, 1, (static_cast<uint64_t>(vx.w) << 32) | vx.z);
+          asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
         }
-        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-      }
-      // the group's rows of stage j are written (or some wait ran out: the group stops together)
-      if (!bnn::tc::named_barrier_and(ok, 2 + g, kQGroup)) break;
-      if (t == 0) {
-        mbar_arrive(smem_u32(&chunk_empty[pb]));  // this group's stage of chunk c is read
-        bnn::tc::mbar_arrive_rank(smem_u32(&full_bar[b]), 0u);
+        // the group's rows of the stage are written (or a wait ran out: the group stops together)
+        ok = bnn::tc::named_barrier_and(ok, 2 + g, kQGroup);
+        if (!ok) break;
+        if (t == 0) {
+          mbar_arrive(smem_u32(&chunk_empty[pb]));  // this group is done with the chunk
+          if (has) bnn::tc::mbar_arrive_rank(smem_u32(&full_bar[b]), 0u);
+        }
       }
     }
-    atomicAdd(&pop_w[t], pop_a);
-    atomicAdd(&pop_x[t], pop_b);
-  } else if (tid == kQMmaWarp * 32 && rank == 0) {
-    // ------------------------------------------------------------ MMA issue
-    // D s32, A and B 8-bit integers, both K-major, N = 256, M = 256 (two CTAs)
-    const uint32_t idesc = (2u << 4) | (1u << 7) | (1u << 10) | ((256u >> 3) << 17) | ((256u >> 4) << 24);
-    for (int j = 0; j < nst; ++j) {
-      const int b = j % kQS;
-      if (!bnn::tc::mbar_wait_cluster(smem_u32(&full_bar[b]), static_cast<uint32_t>((j / kQS) & 1), &abort_flag,
-                                      &g_bnn_device_errors, wait_limit))
-        break;
-      asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-      const uint64_t ad = sw128_desc(smem_base + b * kQStageBytes);
-      const uint64_t bd = sw128_desc(smem_base + b * kQStageBytes + kTm * 128u);
+  } else if (warp == kQMmaWarp) {
+    // ------------------------------------------------------------ MMA issue (CTA 0)
+    if (rank == 0 && lane == 0) {
+      // D s32, A and B 8-bit integers, both K-major, N = 256, M = 256 (two CTAs)
+      const uint32_t idesc = (2u << 4) | (1u << 7) | (1u << 10) | ((256u >> 3) << 17) | ((256u >> 4) << 24);
+      bool ok = true;
+      for (int64_t tile = pair, ti = 0; tile < ntiles && ok; tile += npairs, ++ti) {
+        const int tb = static_cast<int>(ti & 1);
+        // the epilogues (both CTAs) have read this buffer's previous tile
+        if (ti >= 2)
+          ok = bnn::tc::mbar_wait_cluster(smem_u32(&acc_empty[tb]), static_cast<uint32_t>((ti / 2 + 1) & 1),
+                                          &abort_flag, &g_bnn_device_errors, wait_limit);
+        const uint32_t d = tmem + 256u * static_cast<uint32_t>(tb);
+        for (int j = 0; j < nst && ok; ++j) {
+          const int64_t gs = ti * nst + j;
+          const int b = static_cast<int>(gs % kQS);
+          ok = bnn::tc::mbar_wait_cluster(smem_u32(&full_bar[b]), static_cast<uint32_t>((gs / kQS) & 1),
+                                          &abort_flag, &g_bnn_device_errors, wait_limit);
+          if (!ok) break;
+          asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+          const uint64_t ad = sw128_desc(smem_base + b * kQStageBytes);
+          const uint64_t bd = sw128_desc(smem_base + b * kQStageBytes + kTm * 128u);
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+            asm volatile(
+                "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+                "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
+                "l"(ad + static_cast<uint64_t>(2 * kk)), "l"(bd + static_cast<uint64_t>(2 * kk)), "r"(idesc),
+                "r"(acc));
+          }
+          asm volatile(
+              "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n" ::
+                  "r"(smem_u32(&empty_bar[b])),
+              "h"(static_cast<uint16_t>(3))
+              : "memory");
+        }
+        if (!ok) break;
         asm volatile(
-            "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
-            "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem),
-            "l"(ad + static_cast<uint64_t>(2 * kk)), "l"(bd + static_cast<uint64_t>(2 * kk)), "r"(idesc), "r"(acc));
+            "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n" ::"r"(
+                smem_u32(&acc_full[tb])),
+            "h"(static_cast<uint16_t>(3))
+            : "memory");
       }
+      // arrives (in both CTAs) once every MMA issued above has completed
       asm volatile(
           "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n" ::"r"(
-              smem_u32(&empty_bar[b])),
+              smem_u32(&done_bar)),
           "h"(static_cast<uint16_t>(3))
           : "memory");
     }
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n" ::"r"(
-            smem_u32(&done_bar)),
-        "h"(static_cast<uint16_t>(3))
-        : "memory");
-  } else if (tid == kQTmaWarp * 32) {
+  } else if (warp == kQTmaWarp) {
     // ------------------------------------------------------------ TMA copies
-    const int nch = (nst + kChunkStages - 1) / kChunkStages;
-    const int pre = nch < kQP ? nch : kQP;
-    const int iq = static_cast<int>(i0) + 128 * static_cast<int>(rank);  // this CTA's activation rows
-    auto chunk_x = [&](int c) { return 2 * kChunkStages * c; };
-    for (int c = 0; c < pre; ++c) {
-      mbar_expect_tx(smem_u32(&chunk_full[c]), kQChunkBytes);
-      tma_load_2d(smem_u32(chunks + c * kQChunkBytes), &tmap_w, chunk_x(c), static_cast<int>(j0),
-                  smem_u32(&chunk_full[c]));
+    if (lane == 0) {
+      bnn::pdl_wait();  // the activations may come from the preceding kernel
+      int64_t gc = 0;
+      bool ok = true;
+      for (int64_t tile = pair; tile < ntiles && ok; tile += npairs) {
+        const int j0 = static_cast<int>((tile % ntn) * 256 + 128 * rank);
+        const int iq = static_cast<int>((tile / ntn) * 256 + 128 * rank);
+        for (int c = 0; c < nch; ++c, ++gc) {
+          const int pb = static_cast<int>(gc % kQP);
+          if (gc >= kQP &&
+              !bnn::tc::mbar_wait(smem_u32(&chunk_empty[pb]), static_cast<uint32_t>((gc / kQP + 1) & 1), &abort_flag,
+                                  &g_bnn_device_errors, wait_limit)) {
+            ok = false;
+            break;
+          }
+          const uint32_t dst = smem_u32(chunks + pb * kQChunkBytes);
+          const uint32_t bar = smem_u32(&chunk_full[pb]);
+          mbar_expect_tx(bar, kQChunkBytes);
+          tma_load_2d(dst, &tmap_w, 2 * kChunkStages * c, j0, bar);
+          tma_load_2d(dst + kTm * 16u * kChunkStages, &tmap_x, 2 * kChunkStages * c, iq, bar);
+        }
+      }
+      // the CTA must not retire with copies in flight: wait for the last chunk issued into each buffer
+      for (int64_t c = gc - kQP; c < gc; ++c)
+        if (c >= 0)
+          bnn::tc::mbar_drain(smem_u32(&chunk_full[c % kQP]), static_cast<uint32_t>((c / kQP) & 1),
+                              &g_bnn_device_errors);
     }
-    bnn::pdl_wait();
-    for (int c = 0; c < pre; ++c)
-      tma_load_2d(smem_u32(chunks + c * kQChunkBytes) + kTm * 16u * kChunkStages, &tmap_x, chunk_x(c), iq,
-                  smem_u32(&chunk_full[c]));
-    int issued = pre;
-    for (int c = pre; c < nch; ++c) {
-      const int pb = c % kQP;
-      if (!bnn::tc::mbar_wait(smem_u32(&chunk_empty[pb]), static_cast<uint32_t>((c / kQP + 1) & 1), &abort_flag,
-                              &g_bnn_device_errors, wait_limit))
-        break;
-      const uint32_t dst = smem_u32(chunks + pb * kQChunkBytes);
-      const uint32_t bar = smem_u32(&chunk_full[pb]);
-      mbar_expect_tx(bar, kQChunkBytes);
-      tma_load_2d(dst, &tmap_w, chunk_x(c), static_cast<int>(j0), bar);
-      tma_load_2d(dst + kTm * 16u * kChunkStages, &tmap_x, chunk_x(c), iq, bar);
-      issued = c + 1;
+  } else {
+    // ------------------------------------------------------------ epilogue warps
+    bnn::pdl_wait();  // the row popcounts come from the preceding kernel
+    const int q = warp & 3;                         // tensor-memory lanes 32q..32q+31
+    const int erow = 32 * q + lane;
+    const uint32_t lane_field = static_cast<uint32_t>(32 * q) << 16;
+    const bool need_y = out || next;
+    for (int64_t tile = pair, ti = 0; tile < ntiles; tile += npairs, ++ti) {
+      const int tb = static_cast<int>(ti & 1);
+      const int64_t j0 = (tile % ntn) * 256 + 128 * rank, i0 = (tile / ntn) * 256;
+      const bool ok = bnn::tc::mbar_wait_idle(smem_u32(&acc_full[tb]), static_cast<uint32_t>((ti / 2) & 1),
+                                              &abort_flag, &g_bnn_device_errors);
+      if (!bnn::tc::named_barrier_and(ok, kQEpiBar, 128)) break;  // the four warps stop together
+      asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+      const int64_t jrow = j0 + erow;
+      const bool jlive = jrow < n;
+      const float a_j = (need_y && jlive) ? __ldg(alpha + jrow) : 0.0f;
+      const float b_j = (bias && jlive) ? __ldg(bias + jrow) : 0.0f;
+      const int base = k - 2 * (jlive ? __ldg(pop_w + jrow) : 0);
+      const int64_t half = (j0 + 32 * q) / 32;
+      const bool pack = next && half < next_w32;
+      const uint32_t taddr = tmem + lane_field + 256u * static_cast<uint32_t>(tb);
+      for (int c0 = 0; c0 < 256; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld16(taddr + static_cast<uint32_t>(c0), r);
+        const int64_t rows_left = m - (i0 + c0);
+        const int nc = rows_left <= 0 ? 0 : (rows_left < 16 ? static_cast<int>(rows_left) : 16);
+        int px[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) px[c] = c < nc ? __ldg(pop_x + i0 + c0 + c) : 0;
+        tmem_wait_ld();
+        const int64_t off = (i0 + c0) * n + jrow;
+        int32_t* dp = dots ? dots + off : nullptr;
+        float* op = out ? out + off : nullptr;
+        uint32_t* np = pack ? next + (i0 + c0) * next_w32 + half : nullptr;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int32_t dv = base - 2 * px[c] + 4 * static_cast<int32_t>(r[c]);
+          const float y0 = __fmul_rn(a_j, static_cast<float>(dv));
+          const float y = bias ? __fadd_rn(y0, b_j) : y0;
+          if (c < nc && jlive) {
+            if (dp) *dp = dv;
+            if (op) *op = y;
+          }
+          if (np) {
+            const unsigned bits = __ballot_sync(0xffffffffu, jlive && !(y > 0.0f));
+            if (lane == 0 && c < nc) *np = bits;
+            np += next_w32;
+          }
+          dp += n;
+          op += n;
+        }
+      }
+      // this CTA's four epilogue warps have read the buffer: one arrival on CTA 0's acc_empty
+      asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+      asm volatile("bar.sync %0, 128;\n" ::"r"(kQEpiBar) : "memory");
+      if (warp == kQEpiWarp0 && lane == 0) bnn::tc::mbar_arrive_rank(smem_u32(&acc_empty[tb]), 0u);
     }
-    for (int c = issued - kQP; c < issued; ++c)
-      if (c >= 0)
-        bnn::tc::mbar_drain(smem_u32(&chunk_full[c % kQP]), static_cast<uint32_t>((c / kQP) & 1),
-                            &g_bnn_device_errors);
   }
   __syncwarp();
 
-  // -------------------------------------------------------------- epilogue
-  if (tid < kQProducers) asm volatile("bar.sync 1, %0;\n" ::"r"(kQProducers) : "memory");
-  bool drained = true;
-  if (warp < 8) {
-    drained = bnn::tc::mbar_drain(smem_u32(&done_bar), 0u, &g_bnn_device_errors);
-    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-  }
-  const bool good = __syncthreads_and(drained && abort_flag == 0) != 0;
-  if (tid == 0 && !good)  // the tile is incomplete: neither CTA writes it
-    for (uint32_t q = 0; q < 2; ++q) atomicExch(cluster.map_shared_rank(&any_bad, q), 1);
-  cluster.sync();  // popcounts final in both CTAs; abort flags exchanged
-  for (int i = tid; i < 2 * kTm; i += blockDim.x) pop_xt[i] = cluster.map_shared_rank(pop_x, i / kTm)[i % kTm];
-  __syncthreads();
-
-  const int erow = 32 * (warp & 3) + lane;
-  const int ecol0 = (warp >> 2) * 128;
-  const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
-  const bool need_y = out || next;
-  if (warp < 8 && any_bad == 0) {
-    const int64_t jrow = j0 + erow;
-    const bool jlive = jrow < n;
-    const float a_j = (need_y && jlive) ? __ldg(alpha + jrow) : 0.0f;
-    const float b_j = (bias && jlive) ? __ldg(bias + jrow) : 0.0f;
-    const int base = k - 2 * pop_w[erow];
-    const int64_t half = (j0 + 32 * (warp & 3)) / 32;
-    const bool pack = next && half < next_w32;
-    for (int c0 = ecol0; c0 < ecol0 + 128; c0 += 16) {
-      uint32_t r[16];
-      if (nst > 0) {
-        tmem_ld16(taddr + static_cast<uint32_t>(c0), r);
-        tmem_wait_ld();
-      } else {
-#pragma unroll
-        for (int c = 0; c < 16; ++c) r[c] = 0u;
-      }
-      const int64_t rows_left = m - (i0 + c0);
-      const int nc = rows_left <= 0 ? 0 : (rows_left < 16 ? static_cast<int>(rows_left) : 16);
-      const int64_t off = (i0 + c0) * n + jrow;
-      int32_t* dp = dots ? dots + off : nullptr;
-      float* op = out ? out + off : nullptr;
-      uint32_t* np = pack ? next + (i0 + c0) * next_w32 + half : nullptr;
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const int32_t d = base - 2 * pop_xt[c0 + c] + 4 * static_cast<int32_t>(r[c]);
-        const float y0 = __fmul_rn(a_j, static_cast<float>(d));
-        const float y = bias ? __fadd_rn(y0, b_j) : y0;
-        if (c < nc && jlive) {
-          if (dp) *dp = d;
-          if (op) *op = y;
-        }
-        if (np) {
-          const unsigned bits = __ballot_sync(0xffffffffu, jlive && !(y > 0.0f));
-          if (lane == 0 && c < nc) *np = bits;
-          np += next_w32;
-        }
-        dp += n;
-        op += n;
-      }
-    }
-  }
-
+  // every MMA issued has completed before the tensor memory is freed
+  if (tid == 0) bnn::tc::mbar_drain(smem_u32(&done_bar), 0u, &g_bnn_device_errors);
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+  __syncthreads();
   cluster.sync();  // neither CTA leaves while the pair's tensor memory or shared memory is in use
   if (warp == kQMmaWarp)
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kQTmemCols));
+}
+
+// Popcount of every packed row of x (rows 0..m-1) and w (rows m..m+n-1), one
+// warp per row, for the CTA-pair kernel's epilogue.
+__global__ void row_popcount_kernel(const uint64_t* __restrict__ xp, const uint64_t* __restrict__ wp, int64_t m,
+                                    int64_t n, int kw, int* __restrict__ pop) {
+  bnn::pdl_trigger();
+  bnn::pdl_wait();  // the activations may come from the preceding kernel
+  const int lane = threadIdx.x & 31;
+  for (int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < m + n;
+       r += (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5) {
+    const uint64_t* row = r < m ? xp + r * kw : wp + (r - m) * kw;
+    int c = 0;
+    for (int i = lane; i < kw; i += 32) c += __popcll(__ldg(row + i));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
+    if (lane == 0) pop[r] = c;
+  }
+}
+
+// Clusters of the pair kernel that fit the GPU at once (cached per context).
+int pair_clusters() {
+  static std::mutex mu;
+  static uint64_t ctx_cached = 0;
+  static int cached = 0;
+  std::lock_guard<std::mutex> lock(mu);
+  const uint64_t ctx = bnn::context_id();
+  if (ctx != 0 && ctx == ctx_cached) return cached;
+  int num = 0;
+  const size_t smem = static_cast<size_t>(kQSmem) + 1024;
+  if (bnn::ensure_smem(binary_gemm_pair_kernel, smem) == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * 128);
+    cfg.blockDim = dim3(kQThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&num, binary_gemm_pair_kernel, &cfg) != cudaSuccess) num = 0;
+  }
+  cudaGetLastError();  // a failed query leaves no error behind
+  cached = num;
+  ctx_cached = bnn::context_id();
+  return num;
 }
 
 bnn_status launch_pair(const uint64_t* xp, const uint64_t* wp, const float* alpha, const float* bias, int64_t m,
                        int64_t n, int k, int kw, int32_t* dots, float* out, uint64_t* next, cudaStream_t s,
                        bool* launched) {
   *launched = false;
-  const int64_t gx = 2 * ((n + 255) / 256), gy = (m + 255) / 256;
-  if (gx > 2147483647LL || gy > 65535 || kw <= 0 || kw % 2 != 0 || !bnn::aligned(xp, 16) || !bnn::aligned(wp, 16) ||
-      n >= (1LL << 31) || m >= (1LL << 31))
+  const int64_t ntiles = ((n + 255) / 256) * ((m + 255) / 256);
+  if (kw <= 0 || kw % 2 != 0 || !bnn::aligned(xp, 16) || !bnn::aligned(wp, 16) || n >= (1LL << 31) ||
+      m >= (1LL << 31))
     return BNN_OK;
+  const int clusters = pair_clusters();
+  if (clusters <= 0) return BNN_OK;
   CUtensorMap tw, tx;
   if (!bnn::encode_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT64, wp, static_cast<uint64_t>(kw),
                            static_cast<uint64_t>(n), static_cast<uint64_t>(kw) * 8u, 2 * kChunkStages, kTm,
@@ -755,13 +837,24 @@ bnn_status launch_pair(const uint64_t* xp, const uint64_t* wp, const float* alph
                            static_cast<uint64_t>(m), static_cast<uint64_t>(kw) * 8u, 2 * kChunkStages, kTm,
                            CU_TENSOR_MAP_SWIZZLE_64B))
     return BNN_OK;
-  const size_t smem = static_cast<size_t>(kQSmem) + 1024;
-  BNN_TRY(bnn::ensure_smem(binary_gemm_pair_kernel, smem));
-  const cudaError_t e = bnn::launch_pdl(binary_gemm_pair_kernel, dim3(static_cast<unsigned>(gx),
-                                        static_cast<unsigned>(gy)), dim3(kQThreads), smem, s, 2u, tw, tx, alpha,
-                                        bias, m, n, k, kw, dots, out, reinterpret_cast<uint32_t*>(next),
-                                        2 * bnn::words64(n), g_wait_limit.load());
+  int* pop = nullptr;
+  BNN_TRY(bnn::scratch_alloc(reinterpret_cast<void**>(&pop), static_cast<size_t>(m + n) * sizeof(int), s));
+  const int64_t warps = m + n, blocks = (warps + 7) / 8;
+  const int pgrid = static_cast<int>(blocks < 4 * bnn::sm_count() ? blocks : 4 * bnn::sm_count());
+  cudaError_t e = bnn::launch_pdl(row_popcount_kernel, dim3(pgrid), dim3(256), 0, s, 1u, xp, wp, m, n, kw, pop);
+  if (e == cudaSuccess) {
+    const size_t smem = static_cast<size_t>(kQSmem) + 1024;
+    const int64_t np = ntiles < clusters ? ntiles : clusters;
+    e = bnn::ensure_smem(binary_gemm_pair_kernel, smem);
+    if (e == cudaSuccess)
+      e = bnn::launch_pdl(binary_gemm_pair_kernel, dim3(static_cast<unsigned>(2 * np)), dim3(kQThreads), smem, s, 2u,
+                          tw, tx, alpha, bias, static_cast<const int*>(pop), static_cast<const int*>(pop + m), m, n,
+                          k, kw, dots, out, reinterpret_cast<uint32_t*>(next), 2 * bnn::words64(n),
+                          g_wait_limit.load());
+  }
+  const cudaError_t ef = cudaFreeAsync(pop, s);
   if (e != cudaSuccess) return bnn::cuda_fail(e);
+  if (ef != cudaSuccess) return bnn::cuda_fail(ef);
   *launched = true;
   return bnn::check_launch();
 }

@@ -34,6 +34,12 @@ int current_device();
 // next one gets a new id, so nothing cached for the old one is reused.
 uint64_t context_id();
 
+// Stream-ordered scratch memory from a pool of this library (one per device
+// and CUDA context) that keeps its memory between calls, where the default
+// pool would hand it back to the driver at each synchronisation and map it
+// again on the next call.  Free with cudaFreeAsync on the same stream.
+cudaError_t scratch_alloc(void** p, size_t bytes, cudaStream_t s);
+
 // Raises a kernel's dynamic shared-memory limit to `bytes` once per kernel
 // and CUDA context, so that later calls (including calls made while a
 // stream is being captured into a CUDA graph) only launch.

@@ -752,7 +752,7 @@ extern "C" bnn_status bnn_ternary_pack(const float* w, int64_t n, int64_t k, uin
   const int64_t nparts = (total + kChunk - 1) / kChunk;
   double* partial = nullptr;
   if (nparts > 0) {
-    BNN_TRY(cudaMallocAsync(reinterpret_cast<void**>(&partial), static_cast<size_t>(nparts) * sizeof(double), s));
+    BNN_TRY(bnn::scratch_alloc(reinterpret_cast<void**>(&partial), static_cast<size_t>(nparts) * sizeof(double), s));
     twn_abs_partial_kernel<<<static_cast<unsigned>(nparts), kRedThreads, 0, s>>>(w, total, partial);
     const bnn_status st = bnn::check_launch();
     if (st != BNN_OK) {
@@ -1001,7 +1001,7 @@ extern "C" bnn_status bnn_ternary_pack_mode(const float* w, int64_t n, int64_t k
   const int64_t nparts = (total + kChunk - 1) / kChunk;
   double* partial = nullptr;
   if (nparts > 0) {
-    BNN_TRY(cudaMallocAsync(reinterpret_cast<void**>(&partial), static_cast<size_t>(nparts) * sizeof(double), s));
+    BNN_TRY(bnn::scratch_alloc(reinterpret_cast<void**>(&partial), static_cast<size_t>(nparts) * sizeof(double), s));
     twn_abs_partial_kernel<<<static_cast<unsigned>(nparts), kRedThreads, 0, s>>>(w, total, partial);
     const bnn_status st = bnn::check_launch();
     if (st != BNN_OK) {
