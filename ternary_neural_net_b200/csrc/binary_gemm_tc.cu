@@ -71,6 +71,7 @@ using bnn::tc::smem_u32;
 using bnn::tc::sw128_desc;
 using bnn::tc::tma_load_2d;
 using bnn::tc::tmem_ld16;
+using bnn::tc::tmem_ld32;
 using bnn::tc::tmem_wait_ld;
 
 constexpr int kTm = 128;                   // weight rows per tile (UMMA M)
@@ -510,7 +511,7 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
 constexpr int kQRows = 256;                                     // stacked rows per CTA (128 weight + 128 activation)
 constexpr uint32_t kQStageBytes = kQRows * 128u;                // one expanded stage (32 KiB)
 constexpr uint32_t kQChunkBytes = kQRows * 16u * kChunkStages;  // one packed chunk (16 KiB)
-constexpr int kQS = 5, kQP = 2;                                 // expanded stages, packed chunks
+constexpr int kQS = 6, kQP = 2;                                 // expanded stages, packed chunks
 constexpr int kQG = kChunkStages;                               // producer groups (one stage of every chunk each)
 constexpr int kQGroup = kTm;                                    // threads per group
 constexpr int kQProducers = kQG * kQGroup;                      // 512
@@ -538,6 +539,7 @@ binary_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
   __shared__ __align__(8) uint64_t done_bar;
   __shared__ uint32_t tmem_holder;
   __shared__ volatile int abort_flag;
+  __shared__ int pop_xs[256];                      // the epilogue's tile: activation-row popcounts
   uint8_t* const smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* const chunks = smem + kQS * kQStageBytes;
 
@@ -586,20 +588,21 @@ binary_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
     const uint32_t swz = static_cast<uint32_t>(t & 7);
     const uint32_t rd = ((static_cast<uint32_t>(g) ^ ((t >> 1) & 3)) << 4);  // stage g's unit in a chunk row
     bool ok = true;
-    int64_t gc = 0;  // chunks consumed so far (all tiles)
-    for (int64_t tile = pair, ti = 0; tile < ntiles && ok; tile += npairs, ++ti) {
+    uint32_t gc = 0;  // chunks consumed so far (all tiles)
+    uint32_t ts = 0;  // first stage of the tile, counted over all tiles (the launch keeps it below 2^31)
+    for (int64_t tile = pair; tile < ntiles && ok; tile += npairs, ts += static_cast<uint32_t>(nst)) {
       for (int c = 0; c < nch; ++c, ++gc) {
         const int pb = static_cast<int>(gc % kQP);
         const int j = kChunkStages * c + g;           // this group's stage of the chunk
         const bool has = j < nst;
-        const int64_t gs = ti * nst + j;              // stage count over all tiles
+        const uint32_t gs = ts + static_cast<uint32_t>(j);
         const int b = static_cast<int>(gs % kQS);
-        ok = bnn::tc::mbar_wait(smem_u32(&chunk_full[pb]), static_cast<uint32_t>((gc / kQP) & 1), &abort_flag,
-                                &g_bnn_device_errors, wait_limit);
+        ok = bnn::tc::mbar_wait(smem_u32(&chunk_full[pb]), (gc / kQP) & 1u, &abort_flag, &g_bnn_device_errors,
+                                wait_limit);
         // refill only after the tensor core has read the previous fill of this buffer
-        if (ok && has && gs >= kQS)
-          ok = bnn::tc::mbar_wait(smem_u32(&empty_bar[b]), static_cast<uint32_t>((gs / kQS + 1) & 1), &abort_flag,
-                                  &g_bnn_device_errors, wait_limit);
+        if (ok && has && gs >= static_cast<uint32_t>(kQS))
+          ok = bnn::tc::mbar_wait(smem_u32(&empty_bar[b]), (gs / kQS + 1) & 1u, &abort_flag, &g_bnn_device_errors,
+                                  wait_limit);
         if (ok && has) {
           const uint8_t* ck = chunks + pb * kQChunkBytes + rd;
           const uint4 vw = *reinterpret_cast<const uint4*>(ck + t * 64u);
@@ -634,10 +637,10 @@ binary_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
                                           &abort_flag, &g_bnn_device_errors, wait_limit);
         const uint32_t d = tmem + 256u * static_cast<uint32_t>(tb);
         for (int j = 0; j < nst && ok; ++j) {
-          const int64_t gs = ti * nst + j;
+          const uint32_t gs = static_cast<uint32_t>(ti) * static_cast<uint32_t>(nst) + static_cast<uint32_t>(j);
           const int b = static_cast<int>(gs % kQS);
-          ok = bnn::tc::mbar_wait_cluster(smem_u32(&full_bar[b]), static_cast<uint32_t>((gs / kQS) & 1),
-                                          &abort_flag, &g_bnn_device_errors, wait_limit);
+          ok = bnn::tc::mbar_wait_cluster(smem_u32(&full_bar[b]), (gs / kQS) & 1u, &abort_flag,
+                                          &g_bnn_device_errors, wait_limit);
           if (!ok) break;
           asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
           const uint64_t ad = sw128_desc(smem_base + b * kQStageBytes);
@@ -675,15 +678,15 @@ binary_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
     // ------------------------------------------------------------ TMA copies
     if (lane == 0) {
       bnn::pdl_wait();  // the activations may come from the preceding kernel
-      int64_t gc = 0;
+      uint32_t gc = 0;
       bool ok = true;
       for (int64_t tile = pair; tile < ntiles && ok; tile += npairs) {
         const int j0 = static_cast<int>((tile % ntn) * 256 + 128 * rank);
         const int iq = static_cast<int>((tile / ntn) * 256 + 128 * rank);
         for (int c = 0; c < nch; ++c, ++gc) {
           const int pb = static_cast<int>(gc % kQP);
-          if (gc >= kQP &&
-              !bnn::tc::mbar_wait(smem_u32(&chunk_empty[pb]), static_cast<uint32_t>((gc / kQP + 1) & 1), &abort_flag,
+          if (gc >= static_cast<uint32_t>(kQP) &&
+              !bnn::tc::mbar_wait(smem_u32(&chunk_empty[pb]), (gc / kQP + 1) & 1u, &abort_flag,
                                   &g_bnn_device_errors, wait_limit)) {
             ok = false;
             break;
@@ -696,14 +699,13 @@ binary_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
         }
       }
       // the CTA must not retire with copies in flight: wait for the last chunk issued into each buffer
-      for (int64_t c = gc - kQP; c < gc; ++c)
-        if (c >= 0)
-          bnn::tc::mbar_drain(smem_u32(&chunk_full[c % kQP]), static_cast<uint32_t>((c / kQP) & 1),
-                              &g_bnn_device_errors);
+      for (uint32_t c = gc >= static_cast<uint32_t>(kQP) ? gc - kQP : 0; c < gc; ++c)
+        bnn::tc::mbar_drain(smem_u32(&chunk_full[c % kQP]), (c / kQP) & 1u, &g_bnn_device_errors);
     }
   } else {
     // ------------------------------------------------------------ epilogue warps
     bnn::pdl_wait();  // the row popcounts come from the preceding kernel
+    const int et = tid - kQEpiWarp0 * 32;           // 0..127
     const int q = warp & 3;                         // tensor-memory lanes 32q..32q+31
     const int erow = 32 * q + lane;
     const uint32_t lane_field = static_cast<uint32_t>(32 * q) << 16;
@@ -713,6 +715,8 @@ binary_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
       const int64_t j0 = (tile % ntn) * 256 + 128 * rank, i0 = (tile / ntn) * 256;
       const bool ok = bnn::tc::mbar_wait_idle(smem_u32(&acc_full[tb]), static_cast<uint32_t>((ti / 2) & 1),
                                               &abort_flag, &g_bnn_device_errors);
+      // the tile's 256 activation-row popcounts (0 past m) into shared memory
+      for (int i = et; i < 256; i += 128) pop_xs[i] = i0 + i < m ? __ldg(pop_x + i0 + i) : 0;
       if (!bnn::tc::named_barrier_and(ok, kQEpiBar, 128)) break;  // the four warps stop together
       asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
       const int64_t jrow = j0 + erow;
@@ -723,22 +727,19 @@ binary_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
       const int64_t half = (j0 + 32 * q) / 32;
       const bool pack = next && half < next_w32;
       const uint32_t taddr = tmem + lane_field + 256u * static_cast<uint32_t>(tb);
-      for (int c0 = 0; c0 < 256; c0 += 16) {
-        uint32_t r[16];
-        tmem_ld16(taddr + static_cast<uint32_t>(c0), r);
-        const int64_t rows_left = m - (i0 + c0);
-        const int nc = rows_left <= 0 ? 0 : (rows_left < 16 ? static_cast<int>(rows_left) : 16);
-        int px[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) px[c] = c < nc ? __ldg(pop_x + i0 + c0 + c) : 0;
+      for (int c0 = 0; c0 < 256; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(taddr + static_cast<uint32_t>(c0), r);
         tmem_wait_ld();
+        const int64_t rows_left = m - (i0 + c0);
+        const int nc = rows_left <= 0 ? 0 : (rows_left < 32 ? static_cast<int>(rows_left) : 32);
         const int64_t off = (i0 + c0) * n + jrow;
         int32_t* dp = dots ? dots + off : nullptr;
         float* op = out ? out + off : nullptr;
         uint32_t* np = pack ? next + (i0 + c0) * next_w32 + half : nullptr;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int32_t dv = base - 2 * px[c] + 4 * static_cast<int32_t>(r[c]);
+        for (int c = 0; c < 32; ++c) {
+          const int32_t dv = base - 2 * pop_xs[c0 + c] + 4 * static_cast<int32_t>(r[c]);
           const float y0 = __fmul_rn(a_j, static_cast<float>(dv));
           const float y = bias ? __fadd_rn(y0, b_j) : y0;
           if (c < nc && jlive) {
@@ -829,6 +830,9 @@ bnn_status launch_pair(const uint64_t* xp, const uint64_t* wp, const float* alph
     return BNN_OK;
   const int clusters = pair_clusters();
   if (clusters <= 0) return BNN_OK;
+  // the kernel counts stages over a pair's tiles in 32 bits
+  const int64_t nst = (kw + 1) / 2, per_pair = (ntiles + clusters - 1) / clusters;
+  if (per_pair * nst >= (int64_t{1} << 31)) return BNN_OK;
   CUtensorMap tw, tx;
   if (!bnn::encode_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT64, wp, static_cast<uint64_t>(kw),
                            static_cast<uint64_t>(n), static_cast<uint64_t>(kw) * 8u, 2 * kChunkStages, kTm,
