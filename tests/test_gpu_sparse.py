@@ -104,11 +104,13 @@ def test_sparse_gemm_right_after_encode_with_device_x(bnn):
         del row_ptr, ent
 
 
-@pytest.mark.parametrize("n,k,density", [(150, 32768, 0.1), (300, 1000, 0.0), (1000, 777, 0.7), (5, 3, 1.0)])
+@pytest.mark.parametrize("n,k,density", [(150, 32768, 0.1), (300, 1000, 0.0), (1000, 777, 0.7), (5, 3, 1.0),
+                                         (1000, 32768, 0.9), (700000, 20, 0.5), (11008, 4096, 0.1)])
 def test_sparse_gemv_m1_shapes(bnn, n, k, density):
     """m = 1 (x staged in shared memory): the longest rows k allows (several
     passes of 512 entries per row), empty rows, dense rows and tiny k, with
-    every other row emptied."""
+    every other row emptied; long dense rows at the largest k, thousands of
+    rows per CTA, and the full 11008 x 4096 layer at 10% density."""
     rng = np.random.default_rng(n + k)
     trits = ((rng.integers(0, 2, (n, k)) * 2 - 1) * (rng.random((n, k)) < density)).astype(np.int8)
     trits[::2] = 0
