@@ -644,8 +644,13 @@ bnn_status launch_tc2(const CUtensorMap& tx, const uint16_t* packed, const float
 // tcgen05.st.32x32b.x32 into the stage's A slot of tensor memory; the MMA reads
 // A from there ([a-tmem] operand) and B, the activations, from shared memory
 // (four TMA boxes of 64 x 64 bf16 per stage, 128-byte swizzle).  The packed
-// words reach shared memory without passing through registers: the loader
-// warps copy, per group of five stages (1280 trits = 128 words, 129 when the
+// words reach shared memory without passing through registers.  When the
+// tile's rows fit the word region (a CTA that takes every stage of its rows,
+// rows x k <= about 600 K trits), they are one contiguous byte range of the
+// matrix, which one thread bulk-copies at the start (before the programmatic-
+// launch wait: weights do not depend on the kernel ahead), so the decode never
+// waits for words again.  Otherwise the loader warps copy, per group of five
+// stages (1280 trits = 128 words, 129 when the
 // group starts inside a word), every row's window as 4-byte cp.async units
 // (the row's bytes from the 4-byte boundary at or below its first word; units
 // past the end of the matrix are zero-filled) into a [row][65 units] buffer
@@ -671,6 +676,8 @@ constexpr int kT3Threads = kT3Prod + 64 + kT3Load;     // + MMA warp + TMA warp 
 constexpr uint32_t kT3BAtom = kT3N * 128u;             // one 64-trit box of activations
 constexpr uint32_t kT3BStage = 4 * kT3BAtom;
 constexpr uint32_t kT3WBuf = kT3M * kT3GU * 4u;        // one group's words
+constexpr uint32_t kT3WRegion = 120000u;               // packed words: two groups, or a whole tile (+ slack)
+static_assert(2 * kT3WBuf <= kT3WRegion, "two word groups fit the word region");
 constexpr uint32_t kT3Cols = 512;                      // D (64 columns) + kT3S A slots of 128
 constexpr int kT3Units = kT3N / 4;                     // activation columns in units of 4
 static_assert(kT3N + 128 * kT3S <= static_cast<int>(kT3Cols), "tensor-memory columns");
@@ -754,7 +761,7 @@ template <int KS>
 __global__ void __launch_bounds__(kT3Threads, 1)
 ternary_gemm_tmem_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t* __restrict__ packed,
                          const float* __restrict__ scale, const float* __restrict__ bias, int64_t m, int64_t n,
-                         int64_t kt, int rows_cta, float* __restrict__ out) {
+                         int64_t kt, int rows_cta, int preload, float* __restrict__ out) {
   using namespace bnn::tc;
   constexpr int kMaxCols = 4 * ((kT3Units + KS - 1) / KS);
   constexpr int kPitch = kMaxCols + 4;  // padded receive row (floats)
@@ -772,8 +779,9 @@ ternary_gemm_tmem_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint1
   __shared__ int any_bad;
   __shared__ uint32_t lut[9];
   uint8_t* const bsm = t3_raw + ((1024u - (smem_u32(t3_raw) & 1023u)) & 1023u);  // kT3S activation stages
-  uint8_t* const wbuf = bsm + kT3S * kT3BStage;                                   // [2][kT3M][kT3GU] units
-  uint2* const quad = reinterpret_cast<uint2*>(wbuf + 2 * kT3WBuf + 16);          // 81-entry table, 16 copies
+  // the packed words: the whole tile's rows (preload) or [2][kT3M][kT3GU] units of a word group
+  uint8_t* const wbuf = bsm + kT3S * kT3BStage;
+  uint2* const quad = reinterpret_cast<uint2*>(wbuf + kT3WRegion + 16);           // 81-entry table, 16 copies
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rank = KS > 1 ? static_cast<int>(blockIdx.x % KS) : 0;
@@ -809,7 +817,7 @@ ternary_gemm_tmem_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint1
       mbar_init(smem_u32(&empty_bar[i]), 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&w_full[i]), kT3Load);
+      mbar_init(smem_u32(&w_full[i]), preload ? 1 : kT3Load);  // preload: the copying thread's expect_tx
       mbar_init(smem_u32(&w_empty[i]), prod_warps);
     }
     mbar_init(smem_u32(&done_bar), 1);
@@ -839,58 +847,102 @@ ternary_gemm_tmem_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint1
     const uint32_t lane_field = static_cast<uint32_t>(32 * (warp & 3)) << 16;
     const uint32_t quad_lane = smem_u32(quad) + 8u * static_cast<uint32_t>(lane & 15);  // this lane's table copy
     bool ok = 32 * (warp & 3) < rows_cta;
-    for (int g = 0; g < ngroups && ok; ++g) {
-      const int buf = g & 1;
-      // sleeping between polls: the loaders need the issue slots while the group's words arrive
-      bool fine = mbar_wait_idle(smem_u32(&w_full[buf]), static_cast<uint32_t>((g >> 1) & 1), &abort_flag,
-                                 &g_bnn_tc_ternary_errors);
-      if (!__all_sync(0xffffffffu, fine)) break;
-      const int64_t s0 = sb + kT3G * static_cast<int64_t>(g);  // first stage of the group
-      const int64_t w0 = (kT3K * s0) / 10;                     // first word staged
-      // this row's words in the buffer: its first staged byte sits at the row's
-      // byte offset mod 4 within its units
-      const int64_t rbyte = ((j0 + row) * kt + w0) * 2;
-      const uint16_t* wrow =
-          reinterpret_cast<const uint16_t*>(wbuf + buf * kT3WBuf + row * (kT3GU * 4) + (rbyte & 3));
-      for (int u = 0; u < kT3G; ++u) {
-        const int jj = kT3G * g + u;
-        if (jj >= nst) break;
-        const int slot = jj % kT3S;
-        fine = jj < kT3S || mbar_wait(smem_u32(&empty_bar[slot]), static_cast<uint32_t>((jj / kT3S + 1) & 1),
-                                      &abort_flag, &g_bnn_tc_ternary_errors);
-        if (!__all_sync(0xffffffffu, fine)) {  // the tensor-memory store below is warp-collective
-          ok = false;
-          break;
-        }
-        asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+    // stage jj of this quarter from the words at wr (the word holding its first trit)
+    auto stage = [&](int jj, const uint16_t* wr, int64_t jw, int64_t t0) -> bool {
+      const int slot = jj % kT3S;
+      const bool fine = jj < kT3S || mbar_wait(smem_u32(&empty_bar[slot]), static_cast<uint32_t>((jj / kT3S + 1) & 1),
+                                               &abort_flag, &g_bnn_tc_ternary_errors);
+      if (!__all_sync(0xffffffffu, fine)) return false;  // the tensor-memory store below is warp-collective
+      asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+      uint32_t W[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) W[i] = wr[i];
+      uint32_t av[32];
+      switch (static_cast<int>(t0 - 10 * jw)) {  // the phase, warp-uniform
+        case 0: decode64<0>(W, lut, quad_lane, av); break;
+        case 2: decode64<2>(W, lut, quad_lane, av); break;
+        case 4: decode64<4>(W, lut, quad_lane, av); break;
+        case 6: decode64<6>(W, lut, quad_lane, av); break;
+        default: decode64<8>(W, lut, quad_lane, av); break;
+      }
+      tmem_st32(tmem + lane_field + static_cast<uint32_t>(kT3N + 128 * slot + 32 * qk), av);
+      asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
+      asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&a_full[slot]));
+      return true;
+    };
+    if (preload) {
+      // every word of the tile's rows is in shared memory once the copy lands
+      // (row r at byte pre_off + 2 kt r, pre_off = the tile's offset from a
+      // 16-byte boundary)
+      const bool fine = ok && mbar_wait_idle(smem_u32(&w_full[0]), 0u, &abort_flag, &g_bnn_tc_ternary_errors);
+      if (!__all_sync(0xffffffffu, fine)) ok = false;
+      const uint32_t pre_off = static_cast<uint32_t>((2 * j0 * kt) & 15);
+      const uint16_t* wrow = reinterpret_cast<const uint16_t*>(wbuf + pre_off) + static_cast<int64_t>(row) * kt;
+      for (int jj = 0; jj < nst && ok; ++jj) {
         const int64_t t0 = kT3K * (sb + jj) + 64 * qk;  // first trit of this quarter
         const int64_t jw = t0 / 10;
-        const uint16_t* wr = wrow + (jw - w0);
-        uint32_t W[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) W[i] = wr[i];
-        uint32_t av[32];
-        switch (static_cast<int>(t0 - 10 * jw)) {  // the phase, warp-uniform
-          case 0: decode64<0>(W, lut, quad_lane, av); break;
-          case 2: decode64<2>(W, lut, quad_lane, av); break;
-          case 4: decode64<4>(W, lut, quad_lane, av); break;
-          case 6: decode64<6>(W, lut, quad_lane, av); break;
-          default: decode64<8>(W, lut, quad_lane, av); break;
-        }
-        tmem_st32(tmem + lane_field + static_cast<uint32_t>(kT3N + 128 * slot + 32 * qk), av);
-        asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
-        asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&a_full[slot]));
+        ok = stage(jj, wrow + jw, jw, t0);
       }
-      __syncwarp();
-      if (ok && lane == 0) mbar_arrive(smem_u32(&w_empty[buf]));  // this warp is done with the group's words
+    } else {
+      for (int g = 0; g < ngroups && ok; ++g) {
+        const int buf = g & 1;
+        // sleeping between polls: the loaders need the issue slots while the group's words arrive
+        const bool fine = mbar_wait_idle(smem_u32(&w_full[buf]), static_cast<uint32_t>((g >> 1) & 1), &abort_flag,
+                                         &g_bnn_tc_ternary_errors);
+        if (!__all_sync(0xffffffffu, fine)) break;
+        const int64_t s0 = sb + kT3G * static_cast<int64_t>(g);  // first stage of the group
+        const int64_t w0 = (kT3K * s0) / 10;                     // first word staged
+        // this row's words in the buffer: its first staged byte sits at the row's
+        // byte offset mod 4 within its units
+        const int64_t rbyte = ((j0 + row) * kt + w0) * 2;
+        const uint16_t* wrow =
+            reinterpret_cast<const uint16_t*>(wbuf + buf * kT3WBuf + row * (kT3GU * 4) + (rbyte & 3));
+        for (int u = 0; u < kT3G && ok; ++u) {
+          const int jj = kT3G * g + u;
+          if (jj >= nst) break;
+          const int64_t t0 = kT3K * (sb + jj) + 64 * qk;  // first trit of this quarter
+          const int64_t jw = t0 / 10;
+          ok = stage(jj, wrow + (jw - w0), jw, t0);
+        }
+        __syncwarp();
+        if (ok && lane == 0) mbar_arrive(smem_u32(&w_empty[buf]));  // this warp is done with the group's words
+      }
     }
   } else if (warp >= kLoadWarp0) {
     // ------------------------------------------------------------ loaders of the packed words
     const int lt = tid - kLoadWarp0 * 32;
     const uint8_t* gbase = reinterpret_cast<const uint8_t*>(packed);
     const int64_t total_bytes = n * kt * 2;
+    if (preload) {
+      // one thread: the tile's rows are one contiguous byte range [a0, a1) of the
+      // matrix; bulk-copy it from the 16-byte boundary at or below a0 (pieces of
+      // at most 32 KiB, ending at the last 16-byte boundary inside the matrix),
+      // the bytes after that boundary (fewer than 16) by plain loads
+      if (lt == 0) {
+        const uint64_t base = reinterpret_cast<uint64_t>(gbase);
+        const uint64_t a0 = base + static_cast<uint64_t>(2 * j0 * kt);
+        const uint64_t a1 = base + static_cast<uint64_t>(2 * (j0 + rows_live) * kt);
+        const uint64_t f0 = a0 & ~uint64_t{15};
+        const uint64_t t16 = (base + static_cast<uint64_t>(total_bytes)) & ~uint64_t{15};
+        uint64_t f1 = (a1 + 15u) & ~uint64_t{15};
+        if (f1 > t16) f1 = t16;
+        if (f1 < f0) f1 = f0;
+        for (uint64_t p = (f1 > a0 ? f1 : a0); p < a1; ++p) wbuf[p - f0] = gbase[p - base];
+        const uint32_t bar = smem_u32(&w_full[0]);
+        mbar_expect_tx(bar, static_cast<uint32_t>(f1 - f0));  // after the plain stores: they are released with it
+        for (uint64_t p = f0; p < f1; p += 32768u) {
+          const uint32_t bytes = static_cast<uint32_t>(f1 - p < 32768u ? f1 - p : 32768u);
+          asm volatile(
+              "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                  smem_u32(wbuf + (p - f0))),
+              "l"(p), "r"(bytes), "r"(bar)
+              : "memory");
+        }
+        mbar_drain(bar, 0u, &g_bnn_tc_ternary_errors);  // no copy in flight when the CTA retires
+      }
+    } else {
     // this thread's units idx = lt + kT3Load i, walked as (row, unit) without divisions
     const int r_first = lt / kT3GU, u_first = lt - r_first * kT3GU;
     constexpr int kDr = kT3Load / kT3GU, kDu = kT3Load % kT3GU;
@@ -918,6 +970,7 @@ ternary_gemm_tmem_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint1
       asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(smem_u32(&w_full[buf])) : "memory");
     }
     asm volatile("cp.async.wait_all;\n" ::: "memory");  // no copy in flight when the CTA retires
+    }
   } else if (tid == kMmaWarp * 32) {
     // ------------------------------------------------------------ MMA issue
     // D f32, A (tensor memory) and B bf16, K-major, N = 64, M = 128
@@ -1069,7 +1122,13 @@ ternary_gemm_tmem_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint1
 // dynamic shared memory: 1024-byte alignment slack, the activation stages, two
 // word buffers, 16 bytes past them (a producer may read, and not use, the word
 // after its row's window) and the interleaved copies of the 81-entry table
-size_t tmem_smem_bytes() { return 1024 + static_cast<size_t>(kT3S) * kT3BStage + 2u * kT3WBuf + 16 + kQuadTableBytes; }
+size_t tmem_smem_bytes() { return 1024 + static_cast<size_t>(kT3S) * kT3BStage + kT3WRegion + 16 + kQuadTableBytes; }
+
+// whether a tile of rows_cta rows fits the word region whole (with 16 bytes of
+// alignment and 32 bytes read past the last word)
+bool tmem_preload_fits(int rows_cta, int64_t kt) {
+  return static_cast<int64_t>(rows_cta) * kt * 2 + 16 + 32 <= static_cast<int64_t>(kT3WRegion);
+}
 
 // clusters of KS CTAs of the tensor-memory kernel that can run at once (0 when unknown)
 template <int KS>
@@ -1111,9 +1170,11 @@ bnn_status launch_tmem(const CUtensorMap& tx, const uint16_t* packed, const floa
   auto kern = ternary_gemm_tmem_kernel<KS>;
   const size_t smem = tmem_smem_bytes();
   BNN_TRY(bnn::ensure_smem(kern, smem));
+  // (a rank of a split-K cluster needs only its share of each row's words: group loads)
+  const int preload = (KS == 1 && tmem_preload_fits(rows_cta, kt)) ? 1 : 0;
   const cudaError_t e = bnn::launch_pdl(kern, dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)),
                                         dim3(kT3Threads), smem, s, KS, tx, packed, scale, bias, m, n, kt, rows_cta,
-                                        out);
+                                        preload, out);
   if (e != cudaSuccess) return bnn::cuda_fail(e);
   return bnn::check_launch();
 }

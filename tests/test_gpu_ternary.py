@@ -372,3 +372,13 @@ def test_auto_one_tile_edge_cases(bnn):
                          (x_off, to_dev_u16(packed), "x +2")):
         out = bnn.bnn_ternary_gemm(xd, pd, sc, k)
         assert_ternary_close(out.cpu().numpy(), ref, mag, f"AUTO one tile, {what}")
+
+
+# The tensor-memory kernel (9 <= m <= 64, k % 8 == 0): tiles whose rows fit
+# shared memory whole (one bulk copy of the tile's words, the matrix end not on
+# a 16-byte boundary, odd word counts), long rows that take the word-group
+# loads, and split-K plans.
+@pytest.mark.parametrize("m,n,k", [(64, 999, 4100), (48, 5000, 1288), (64, 300, 32000), (17, 2000, 4096),
+                                   (64, 150, 8000)])
+def test_tmem_word_sources(bnn, m, n, k):
+    _gemm_case(bnn, m, n, k, seed=3 * m + n + k)
