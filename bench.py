@@ -81,7 +81,11 @@ def parse_args(argv=None):
     p.add_argument("--csv", default=None, help="write one CSV row per config and seed to this path")
     p.add_argument("--no-headline", action="store_true", help="skip the headline (profiling runs)")
     p.add_argument("--seed", type=int, default=1, help="seed of the headline's inputs")
+    p.add_argument("--gemm-shape", default=None,
+                   help="M,N,K of config 4's binary GEMM in its per-seed records (profiling of smaller cases; the "
+                        "headline keeps 8192^3)")
     a = p.parse_args(argv)
+    a.gemm_shape = tuple(int(v) for v in a.gemm_shape.split(",")) if a.gemm_shape else None
     a.configs = [] if a.config == "none" else sorted({int(c) for c in a.config.split(",") if c})
     a.seed_list = [int(s) for s in a.seeds.split(",") if s]
     a.extra_set = set() if a.extras == "none" else set(a.extras.split(","))
@@ -491,7 +495,7 @@ def gpu_cfg3(cu, seed, P, st, s, pk):
                 rotation=R)
 
 
-def gpu_cfg4(cu, seed, P, st, s, pk, head=None):
+def gpu_cfg4(cu, seed, P, st, s, pk, head=None, shape=None):
     """Seed 1 is the headline's own measurement; other seeds time the kernel in
     a short graph on their own operands."""
     torch, dev, lib = cu.torch, cu.device, cu.lib
@@ -499,7 +503,7 @@ def gpu_cfg4(cu, seed, P, st, s, pk, head=None):
     if head is not None:
         ms, macs = head["kernel_ms"], head["macs"]
     else:
-        c = synth.gemm_large(seed)
+        c = synth.gemm_large(seed, *shape) if shape else synth.gemm_large(seed)
         m, n, k = c["m"], c["n"], c["k"]
         xp = torch.from_numpy(c["xp"].view(np.int64)).to(dev)
         wp = torch.from_numpy(c["wp"].view(np.int64)).to(dev)
@@ -511,9 +515,11 @@ def gpu_cfg4(cu, seed, P, st, s, pk, head=None):
         macs = float(m) * n * k
         del d, o
     return dict(value=macs / (ms * 1e-3) / 1e9, unit="GMAC/s", ms_kernel=ms, macs=macs,
+                shape=list(shape) if shape else [8192, 8192, 8192],
                 roofline=roofline("tensor", 2 * macs / (ms * 1e-3) / 1e12, int8, "TOP/s",
                                   "binary_gemm_pair_kernel (persistent CTA pairs, 256x256 tiles)",
                                   f"int8 dense = 2 x bf16 {pk['bf16_tflops']} TFLOP/s ({pk['src']})",
+                                  None if shape else
                                   traffic_for("binary_gemm_pair_m8192", "ternary_neural_net_b200/csrc/binary_gemm_tc.cu")))
 
 
@@ -611,7 +617,9 @@ def run_configs(cu, args, pk, head):
         per_seed = {}
         for seed in args.seed_list:
             if cfg == 4:
-                r = gpu_cfg4(cu, seed, P, st, s, pk, head if (head and seed == args.seed) else None)
+                r = gpu_cfg4(cu, seed, P, st, s, pk,
+                             head if (head and seed == args.seed and not args.gemm_shape) else None,
+                             args.gemm_shape)
             else:
                 r = GPU_CFG[cfg](cu, seed, P, st, s, pk)
             per_seed[seed] = r
