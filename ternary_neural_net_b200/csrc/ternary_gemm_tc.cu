@@ -301,8 +301,11 @@ ternary_gemm_tc_kernel(const uint16_t* __restrict__ x, const uint16_t* __restric
 // ---------------------------------------------------------------------------
 // Warp-specialised version (activation rows 16-byte aligned: TMA).
 //
-// Roles: one thread copies the stage's 64 x 64 bf16 activation box by TMA
-// straight into the 128-byte-swizzled tile; 512 producer threads copy the
+// Tile: 128 weight rows x BN activation rows (BN = 64 with two CTAs per SM,
+// or 128 / 256 with one, so that each weight tile is decoded once per 128 or
+// 256 activation rows instead of per 64), K stages of 64 trits.
+// Roles: one thread copies the stage's 64-trit x BN-row bf16 activation box by
+// TMA straight into the 128-byte-swizzled tile; 512 producer threads copy the
 // stage's 8-word window of each weight row into shared memory (coalesced along
 // the rows, one stage ahead) and then decode: warp w takes quarter w % 4 (16
 // trits, 8 pairs) of 32 weight rows, reads the (up to) three words covering
@@ -324,7 +327,7 @@ constexpr int kT2N = 64;                             // activation rows (UMMA N)
 constexpr int kT2S = 4;                              // stages of 64 trits
 constexpr int kT2Prod = 4 * kT2M;                    // producer threads
 constexpr int kT2Threads = kT2Prod + 64;             // + MMA warp + TMA warp
-constexpr uint32_t kT2AStage = kT2M * 128u, kT2Stage = kT2AStage + kT2N * 128u;
+constexpr uint32_t kT2AStage = kT2M * 128u;          // one stage of decoded weights
 constexpr int kT2Pre = 4;                            // stages of words prefetched in registers
 constexpr uint32_t kZeroWord = 29524u;               // all ten trits 0 (every digit 1)
 
@@ -351,13 +354,14 @@ __device__ __forceinline__ void decode16(const uint32_t (&F)[3], const uint32_t*
   hi = make_uint4(v[4], v[5], v[6], v[7]);
 }
 
-template <int KS>
-__global__ void __launch_bounds__(kT2Threads, 2)
+template <int KS, int BN>
+__global__ void __launch_bounds__(kT2Threads, BN == 64 ? 2 : 1)
 ternary_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t* __restrict__ packed,
                         const float* __restrict__ scale, const float* __restrict__ bias, int64_t m, int64_t n,
                         int64_t k, int64_t kt, float* __restrict__ out) {
   using namespace bnn::tc;
-  constexpr int kCols = kT2N / KS;
+  constexpr uint32_t kT2Stage = kT2AStage + BN * 128u;  // decoded weights + BN activation rows
+  constexpr int kCols = BN / KS;
   constexpr int kPitch = kCols + 4;  // padded receive row (floats)
   static_assert(KS * kT2M * kPitch * 4 <= kT2S * kT2Stage, "split-K shares must fit the stage memory");
 
@@ -375,7 +379,7 @@ ternary_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16
   const int tid = threadIdx.x, warp = tid >> 5;
   const int rank = KS > 1 ? static_cast<int>(blockIdx.x % KS) : 0;
   const int64_t j0 = static_cast<int64_t>(blockIdx.x / KS) * kT2M;  // first weight row
-  const int64_t i0 = static_cast<int64_t>(blockIdx.y) * kT2N;        // first activation row
+  const int64_t i0 = static_cast<int64_t>(blockIdx.y) * BN;        // first activation row
   const int64_t total = (10 * kt + 63) / 64;                         // 64-trit stages covering every word
   const int64_t share = (total + KS - 1) / KS;
   const int64_t sb = rank * share < total ? rank * share : total;
@@ -403,7 +407,7 @@ ternary_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16
     asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
   if (warp == kMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(&tmem_holder)),
-                 "r"(kT2N));
+                 "r"(BN));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::);
   }
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
@@ -488,7 +492,7 @@ ternary_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16
   } else if (tid == kMmaWarp * 32) {
     // ------------------------------------------------------------ MMA issue
     // D f32, A and B bf16, both K-major, N = 64, M = 128
-    const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((static_cast<uint32_t>(kT2N) >> 3) << 17) |
+    const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((static_cast<uint32_t>(BN) >> 3) << 17) |
                            ((static_cast<uint32_t>(kT2M) >> 4) << 24);
     const uint32_t base = smem_u32(smem);
     for (int jj = 0; jj < nst; ++jj) {
@@ -518,7 +522,7 @@ ternary_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16
                                    &abort_flag, &g_bnn_tc_ternary_errors))
         break;
       const uint32_t bar = smem_u32(&full_bar[b]);
-      mbar_expect_tx(bar, kT2N * 128u);
+      mbar_expect_tx(bar, BN * 128u);
       tma_load_2d(smem_u32(smem + b * kT2Stage + kT2AStage), &tmap_x, static_cast<int>(64 * (sb + jj)),
                   static_cast<int>(i0), bar);
     }
@@ -533,14 +537,14 @@ ternary_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16
   }
   const bool good = __syncthreads_and(drained && abort_flag == 0) != 0;
   const int erow = 32 * (warp & 3) + (tid & 31);       // weight row (tensor-memory lane)
-  const int ecol0 = (warp >> 2) * (kT2N / 2);          // half of the activation columns
+  const int ecol0 = (warp >> 2) * (BN / 2);          // half of the activation columns
   const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
   const int64_t jrow = j0 + erow;
   if constexpr (KS == 1) {
     if (warp < 8 && good) {
       const bool jlive = jrow < n;
       const float sc = jlive ? __ldg(scale + jrow) : 0.0f, bv = (bias && jlive) ? __ldg(bias + jrow) : 0.0f;
-      for (int c0 = ecol0; c0 < ecol0 + kT2N / 2; c0 += 16) {
+      for (int c0 = ecol0; c0 < ecol0 + BN / 2; c0 += 16) {
         uint32_t r[16];
         if (nst > 0) {  // every lane of the warp takes part in the collective load
           tmem_ld16(taddr + static_cast<uint32_t>(c0), r);
@@ -567,7 +571,7 @@ ternary_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16
     if (tid == 0 && !good)
       for (int q = 0; q < KS; ++q) atomicExch(cluster.map_shared_rank(&any_bad, q), 1);
     if (warp < 8 && good) {
-      for (int c0 = ecol0; c0 < ecol0 + kT2N / 2; c0 += 16) {
+      for (int c0 = ecol0; c0 < ecol0 + BN / 2; c0 += 16) {
         uint32_t r[16];
         if (nst > 0) {
           tmem_ld16(taddr + static_cast<uint32_t>(c0), r);
@@ -614,16 +618,16 @@ ternary_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
   __syncthreads();
   if (warp == kMmaWarp)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kT2N));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(BN));
 }
 
-template <int KS>
+template <int KS, int BN>
 bnn_status launch_tc2(const CUtensorMap& tx, const uint16_t* packed, const float* scale, const float* bias, int64_t m,
                       int64_t n, int64_t k, int64_t kt, float* out, cudaStream_t s) {
-  const int64_t gx = KS * ((n + kT2M - 1) / kT2M), gy = (m + kT2N - 1) / kT2N;
+  const int64_t gx = KS * ((n + kT2M - 1) / kT2M), gy = (m + BN - 1) / BN;
   if (gx > 2147483647LL || gy > 65535) return BNN_ERR_INVALID_ARG;
-  const size_t smem = static_cast<size_t>(kT2S) * kT2Stage + 1024;
-  auto kern = ternary_gemm_tc2_kernel<KS>;
+  const size_t smem = static_cast<size_t>(kT2S) * (kT2AStage + BN * 128u) + 1024;
+  auto kern = ternary_gemm_tc2_kernel<KS, BN>;
   BNN_TRY(bnn::ensure_smem(kern, smem));
   const cudaError_t e = bnn::launch_pdl(kern, dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)),
                                    dim3(kT2Threads), smem, s, KS, tx, packed, scale, bias, m, n, k, kt, out);
@@ -1241,12 +1245,32 @@ bnn_status ternary_gemm_tc(const uint16_t* x_bf16, const uint16_t* packed, const
         default: return launch_tmem<1>(tx, packed, scale, bias, m, n, kt, rows, out, s);
       }
     }
-    const int64_t tiles = ((n + kT2M - 1) / kT2M) * ((m + kT2N - 1) / kT2N);
+    // activation tiles of 256 rows above m = 128, 128 above m = 64 (each weight
+    // tile is decoded once per activation tile), else 64 (two CTAs per SM)
+    const int bn = m > 128 ? 256 : (m > 64 ? 128 : 64);
+    CUtensorMap txw;
+    if (bn != 64 &&
+        !encode_tmap_2d(&txw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x_bf16, static_cast<uint64_t>(k),
+                        static_cast<uint64_t>(m), static_cast<uint64_t>(k) * 2u, 64, static_cast<uint32_t>(bn),
+                        CU_TENSOR_MAP_SWIZZLE_128B))
+      return BNN_ERR_CUDA;
+    const int64_t tiles = ((n + kT2M - 1) / kT2M) * ((m + bn - 1) / bn);
     const int64_t stages = (10 * kt + 63) / 64;
-    const int64_t slots = 2LL * sm_count();  // two CTAs per SM
-    if (tiles * 4 <= slots && stages >= 16) return launch_tc2<4>(tx, packed, scale, bias, m, n, k, kt, out, s);
-    if (tiles * 2 <= slots && stages >= 8) return launch_tc2<2>(tx, packed, scale, bias, m, n, k, kt, out, s);
-    return launch_tc2<1>(tx, packed, scale, bias, m, n, k, kt, out, s);
+    const int64_t slots = (bn == 64 ? 2LL : 1LL) * sm_count();
+    const int ks = (tiles * 4 <= slots && stages >= 16) ? 4 : ((tiles * 2 <= slots && stages >= 8) ? 2 : 1);
+    if (bn == 256) {
+      if (ks == 4) return launch_tc2<4, 256>(txw, packed, scale, bias, m, n, k, kt, out, s);
+      if (ks == 2) return launch_tc2<2, 256>(txw, packed, scale, bias, m, n, k, kt, out, s);
+      return launch_tc2<1, 256>(txw, packed, scale, bias, m, n, k, kt, out, s);
+    }
+    if (bn == 128) {
+      if (ks == 4) return launch_tc2<4, 128>(txw, packed, scale, bias, m, n, k, kt, out, s);
+      if (ks == 2) return launch_tc2<2, 128>(txw, packed, scale, bias, m, n, k, kt, out, s);
+      return launch_tc2<1, 128>(txw, packed, scale, bias, m, n, k, kt, out, s);
+    }
+    if (ks == 4) return launch_tc2<4, 64>(tx, packed, scale, bias, m, n, k, kt, out, s);
+    if (ks == 2) return launch_tc2<2, 64>(tx, packed, scale, bias, m, n, k, kt, out, s);
+    return launch_tc2<1, 64>(tx, packed, scale, bias, m, n, k, kt, out, s);
   }
   const int64_t ntiles = (n + kTcMW - 1) / kTcMW, gy = (m + kTcNX - 1) / kTcNX;
   if (ntiles * kTcK > 2147483647LL || gy > 65535) return BNN_ERR_INVALID_ARG;
