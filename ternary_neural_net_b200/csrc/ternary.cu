@@ -325,29 +325,33 @@ size_t rows_smem_bytes(int64_t kt) {
 // c < 64 at position (c & 1) * 32 + c / 2 and column c >= 64 at c, so each of
 // the six lookups of a row reads 32 consecutive positions of one table row
 // chosen per lane: 32 different banks, whatever the words are.  Columns past
-// the slice hold x = 0 (all entries 0); lanes there look up the all-zero-trit
-// word.
+// the slice hold x = 0 (all entries 0); lanes there read the row's first
+// word(s) instead and look them up in those zero columns.
 //
-// A warp takes four consecutive rows per round and keeps the words of the two
-// rounds after it in flight (the first two rounds are loaded before the
-// programmatic-launch wait, while x is staged and the tables are built).  The
-// four rows' lane sums are added in one transposed shuffle tree (six shuffles
-// for four rows) and stored as the CTA's slice sums; at the end of each chunk
-// of kC5Rows rows, after a cluster barrier, CTA q adds for its share of the
-// chunk the kC5 slice sums in rank order through distributed shared memory,
-// scales once and writes.  Deterministic for a given launch shape.
+// A warp takes 16 consecutive rows per round (four without 32-bit pairs) and
+// holds the words of two rounds: the first two are loaded before the
+// programmatic-launch wait, while x is staged and the tables are built (for a
+// cluster's first 512 rows, every word it reads), and each round's registers
+// are refilled with the round two ahead once its lookups are done.  Rows past
+// the cluster's last are read as that last row and dropped, so nothing in the
+// loop is predicated per row.  The rows' lane sums are added in one transposed
+// shuffle tree (16 shuffles for 16 rows) and stored as the CTA's slice
+// sums; at the end of each chunk of kC5Rows rows, after a cluster barrier, CTA q
+// adds for its share of the chunk the kC5 slice sums in rank order through
+// distributed shared memory, scales once and writes.  Deterministic for a given launch shape.
 // ---------------------------------------------------------------------------
 constexpr int kC5 = 5;                 // CTAs per cluster (slices of the row)
-constexpr int kC5Threads = 1024;
+constexpr int kC5Threads = 512;
 constexpr int kC5Warps = kC5Threads / 32;
 constexpr int kC5Pitch = 96;           // table positions per slice (64 in pairs + 32 single)
-constexpr int kC5D = 4;                // rows per warp round
-constexpr int kC5Round = kC5Warps * kC5D;          // rows per CTA round
 constexpr int kC5Rows = 1024;          // rows of a chunk (slice sums held at once)
-static_assert(kC5Rows % kC5Round == 0, "a chunk is a whole number of rounds");
+// rows per warp round: 16 with 32-bit word pairs (2 registers a row), 4 with
+// three 16-bit words (3 registers a row); two rounds of words are held at once
+template <bool VEC>
+constexpr int c5_rows_per_warp() { return VEC ? 16 : 4; }
+static_assert(kC5Rows % (2 * kC5Warps * 16) == 0 && kC5Rows % (2 * kC5Warps * 4) == 0,
+              "a chunk is an even number of rounds");
 constexpr uint32_t kDiv243Hi = 17674763u;   // ceil(2^32 / 243): floor(w / 243) = high word of w * kDiv243Hi
-constexpr uint32_t kZeroWord = 29524u;      // all ten digits 1: trits 0
-constexpr uint32_t kZeroPair = kZeroWord | (kZeroWord << 16);
 constexpr uint32_t kC5HiOff = 243u * kC5Pitch * 4u;  // bytes from the lo table to the hi table
 
 constexpr bool div243_exact() {
@@ -363,25 +367,27 @@ size_t c5_smem_bytes() { return (2u * 243u * kC5Pitch + kC5Rows + 10u * kC5Pitch
 // slice column of table position p
 __device__ __forceinline__ int c5_column(int p) { return p < 64 ? (p < 32 ? 2 * p : 2 * (p - 32) + 1) : p; }
 
-// The words of one row at this lane's three columns (o = the row's offset in
-// 16-bit words from `packed`, at column 2l): VEC, one 32-bit load for columns
-// 2l, 2l + 1 (w[0]; w[1] unused); else two 16-bit loads (w[0], w[1]).  The last
-// word is column 64 + l.  Lanes or rows outside the slice get the zero word.
+// The words of one row at this lane's three columns: VEC, one 32-bit load for
+// columns 2l, 2l + 1 (w[0]) and one 16-bit load for column 64 + l (w[1]);
+// else three 16-bit loads.  pa, pb, pc point at the lane's columns in the
+// cluster's first row (at that row's first word where a column lies past the
+// slice: the lane then looks up a real word in a table column of zeros), ro is
+// the row's offset from there in 16-bit words.
 template <bool VEC>
 struct C5Words {
   uint32_t w[VEC ? 2 : 3];
 };
 
 template <bool VEC>
-__device__ __forceinline__ void c5_fetch(const uint16_t* __restrict__ packed, uint32_t o, uint32_t oc, bool live,
-                                         bool la, bool lb, bool lc, C5Words<VEC>& v) {
+__device__ __forceinline__ void c5_fetch(const uint16_t* __restrict__ pa, const uint16_t* __restrict__ pb,
+                                         const uint16_t* __restrict__ pc, uint32_t ro, C5Words<VEC>& v) {
   if constexpr (VEC) {
-    v.w[0] = (live && la) ? __ldcs(reinterpret_cast<const uint32_t*>(packed + o)) : kZeroPair;
-    v.w[1] = (live && lc) ? static_cast<uint32_t>(__ldcs(packed + o + oc)) : kZeroWord;
+    v.w[0] = __ldcs(reinterpret_cast<const uint32_t*>(pa + ro));
+    v.w[1] = static_cast<uint32_t>(__ldcs(pc + ro));
   } else {
-    v.w[0] = (live && la) ? static_cast<uint32_t>(__ldcs(packed + o)) : kZeroWord;
-    v.w[1] = (live && lb) ? static_cast<uint32_t>(__ldcs(packed + o + 1)) : kZeroWord;
-    v.w[2] = (live && lc) ? static_cast<uint32_t>(__ldcs(packed + o + oc)) : kZeroWord;
+    v.w[0] = static_cast<uint32_t>(__ldcs(pa + ro));
+    v.w[1] = static_cast<uint32_t>(__ldcs(pb + ro));
+    v.w[2] = static_cast<uint32_t>(__ldcs(pc + ro));
   }
 }
 
@@ -412,6 +418,28 @@ __device__ __forceinline__ float c5_row(const C5Words<VEC>& v, uint32_t t) {
     s += c5_lookup(min(v.w[2], kMaxWord), t + 256u);
   }
   return s;
+}
+
+// Sums of D rows (a[j] = this lane's part of row j) over the warp: D / 2 + ... +
+// 1 shuffles exchange halves of the rows (masks 16, 8, ...), after which lane l
+// holds a part of row l >> (5 - log2 D); plain shuffles finish the sum.  The
+// result is row (lane >> (5 - log2 D))'s total, in every lane of its group.
+template <int D>
+__device__ __forceinline__ float c5_reduce(float (&a)[D], int lane) {
+#pragma unroll
+  for (int h = D / 2, mask = 16; h >= 1; h /= 2, mask >>= 1) {
+    const bool up = (lane & mask) != 0;
+#pragma unroll
+    for (int i = 0; i < h; ++i) {
+      const float keep = up ? a[h + i] : a[i];
+      const float send = up ? a[i] : a[h + i];
+      a[i] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
+    }
+  }
+  float v = a[0];
+#pragma unroll
+  for (int mask = 16 / D; mask >= 1; mask >>= 1) v += __shfl_xor_sync(0xffffffffu, v, mask);
+  return v;
 }
 
 // base + x0 (d0 - 1) + x1 (d1 - 1) for the digits d0 = a % 3, d1 = a / 3 (a is
@@ -448,26 +476,35 @@ ternary_gemv_c5_kernel(const uint16_t* __restrict__ x, const uint16_t* __restric
   const int w0 = rank * slice;                                            // this CTA's first word position
   const int sw = kt - w0 < slice ? (kt - w0 > 0 ? kt - w0 : 0) : slice;  // its word count (<= kC5Pitch)
   const int64_t c0 = n * cl / ncl, c1 = n * (cl + 1) / ncl;              // the cluster's rows
-  const int rounds = static_cast<int>((c1 - c0 + kC5Round - 1) / kC5Round);
+  constexpr int D = c5_rows_per_warp<VEC>();  // rows per warp round
+  constexpr int R = kC5Warps * D;             // rows per CTA round
+  constexpr int kRoundsPerChunk = kC5Rows / R;
+  const int rows_c = static_cast<int>(c1 - c0);
+  const int rounds = (rows_c + R - 1) / R;
   bnn::pdl_trigger();
 
-  // 16-bit word offsets from `packed` (the launch keeps n * kt below 2^31):
-  // this warp's rows of round i start at local row 128 i + 4 warp
-  const int rows_c = static_cast<int>(c1 - c0);
+  // Row offsets are 32-bit (the launch keeps n * kt below 2^31).  A warp's rows
+  // of round i are the local rows R i + D warp + j; rows past the cluster's
+  // last are read as that last row (their sums are dropped), and a warp whose
+  // D rows all lie past it skips the round.
   const uint32_t ktu = static_cast<uint32_t>(kt);
-  const uint32_t off0 = (static_cast<uint32_t>(c0) + 4u * static_cast<uint32_t>(warp)) * ktu +
-                        static_cast<uint32_t>(w0 + 2 * lane);
-  const uint32_t oc = 64u - static_cast<uint32_t>(lane);  // column 64 + l from column 2l
-  const bool la = 2 * lane < sw, lb = 2 * lane + 1 < sw, lc = 64 + lane < sw;
-  auto fetch_round = [&](int i, C5Words<VEC> (&buf)[kC5D]) {
-    const uint32_t o = off0 + static_cast<uint32_t>(i) * (static_cast<uint32_t>(kC5Round) * ktu);
-    const int nl = rows_c - (i * kC5Round + warp * kC5D);  // live rows of the four
+  const uint16_t* const row0 = packed + c0 * static_cast<int64_t>(kt);
+  const uint16_t* const pa = row0 + (2 * lane < sw ? w0 + 2 * lane : 0);
+  const uint16_t* const pb = row0 + (2 * lane + 1 < sw ? w0 + 2 * lane + 1 : 0);
+  const uint16_t* const pc = row0 + (64 + lane < sw ? w0 + 64 + lane : 0);
+  auto fetch_round = [&](int i, C5Words<VEC> (&buf)[D]) {
+    const int rb = i * R + warp * D;
 #pragma unroll
-    for (int j = 0; j < kC5D; ++j) c5_fetch<VEC>(packed, o + j * ktu, oc, j < nl, la, lb, lc, buf[j]);
+    for (int j = 0; j < D; ++j) {
+      const uint32_t rl = static_cast<uint32_t>(rb + j < rows_c ? rb + j : rows_c - 1);
+      c5_fetch<VEC>(pa, pb, pc, rl * ktu, buf[j]);
+    }
   };
-  C5Words<VEC> bufA[kC5D], bufB[kC5D], bufC[kC5D];
-  fetch_round(0, bufA);
-  fetch_round(1, bufB);
+  // rounds 0 and 1 are loaded before the programmatic-launch wait, while x is
+  // staged and the tables are built
+  C5Words<VEC> bufA[D], bufB[D];
+  if (warp * D < rows_c) fetch_round(0, bufA);
+  if (R + warp * D < rows_c) fetch_round(1, bufB);
 
   bnn::pdl_wait();  // x may come from the kernel ahead
   // x of the slice as float32, [digit i][table position p]
@@ -502,49 +539,36 @@ ternary_gemv_c5_kernel(const uint16_t* __restrict__ x, const uint16_t* __restric
   __syncthreads();
 
   const uint32_t tl = static_cast<uint32_t>(__cvta_generic_to_shared(lo)) + 4u * static_cast<uint32_t>(lane);
-  const bool upper = (lane & 16) != 0, mid = (lane & 8) != 0;
-  // round i: the rows of `cur`, with the round two ahead loaded into `ahead`
-  auto round = [&](int i, C5Words<VEC> (&cur)[kC5D], C5Words<VEC> (&ahead)[kC5D]) {
-    fetch_round(i + 2, ahead);
-    const int rl0 = i * kC5Round + warp * kC5D;  // local row of cur[0]
-    const int nl = rows_c - rl0;
-    float acc[kC5D];
+  // round i from the words in cur; round i + 2 is then loaded into cur
+  auto step = [&](int i, C5Words<VEC> (&cur)[D]) {
+    const int rl0 = i * R + warp * D;  // local row of cur[0]
+    if (rl0 >= rows_c) return;
+    float acc[D];
 #pragma unroll
-    for (int j = 0; j < kC5D; ++j) acc[j] = j < nl ? c5_row<VEC>(cur[j], tl) : 0.0f;
-    // four rows over 32 lanes: halves exchange rows (0,1) / (2,3), then quarters
-    // row 0 / 1 of their pair; lane group (lane >> 3) ends with row 2 (lane >> 4) + (lane >> 3 & 1)
-    float k0 = upper ? acc[2] : acc[0], k1 = upper ? acc[3] : acc[1];
-    const float s0 = upper ? acc[0] : acc[2], s1 = upper ? acc[1] : acc[3];
-    k0 += __shfl_xor_sync(0xffffffffu, s0, 16);
-    k1 += __shfl_xor_sync(0xffffffffu, s1, 16);
-    float v = mid ? k1 : k0;
-    v += __shfl_xor_sync(0xffffffffu, mid ? k0 : k1, 8);
-    v += __shfl_xor_sync(0xffffffffu, v, 4);
-    v += __shfl_xor_sync(0xffffffffu, v, 2);
-    v += __shfl_xor_sync(0xffffffffu, v, 1);
-    const int j = lane >> 3;
-    if ((lane & 7) == 0 && j < nl) psum[(rl0 + j) & (kC5Rows - 1)] = v;  // chunks start at multiples of kC5Rows
-    constexpr int kRoundsPerChunk = kC5Rows / kC5Round;
-    if (i % kRoundsPerChunk == kRoundsPerChunk - 1 || i == rounds - 1) {
-      // end of a chunk: its slice sums added in rank order by the CTA that owns the row
-      cluster.sync();
-      const int cb = (i / kRoundsPerChunk) * kC5Rows;  // the chunk's first local row
-      const int rows = rows_c - cb < kC5Rows ? rows_c - cb : kC5Rows;
-      const int q0 = rows * rank / kC5, q1 = rows * (rank + 1) / kC5;
-      for (int rl = q0 + tid; rl < q1; rl += kC5Threads) {
-        float sum = 0.0f;
-#pragma unroll
-        for (int q = 0; q < kC5; ++q) sum += cluster.map_shared_rank(psum, q)[rl];
-        const int64_t r = c0 + cb + rl;
-        out[r] = bias ? __ldg(scale + r) * sum + __ldg(bias + r) : __ldg(scale + r) * sum;
-      }
-      cluster.sync();  // slice sums read before the next chunk overwrites them (and before any CTA exits)
-    }
+    for (int j = 0; j < D; ++j) acc[j] = c5_row<VEC>(cur[j], tl);
+    if (rl0 + 2 * R < rows_c) fetch_round(i + 2, cur);
+    const float v = c5_reduce<D>(acc, lane);
+    const int j = lane / (32 / D);
+    if ((lane & (32 / D - 1)) == 0 && rl0 + j < rows_c) psum[(rl0 + j) & (kC5Rows - 1)] = v;  // chunks start at multiples of kC5Rows
   };
-  for (int i = 0; i < rounds; i += 3) {
-    round(i, bufA, bufC);
-    if (i + 1 < rounds) round(i + 1, bufB, bufA);
-    if (i + 2 < rounds) round(i + 2, bufC, bufB);
+  for (int cb = 0, i0 = 0; i0 < rounds; cb += kC5Rows, i0 += kRoundsPerChunk) {
+    const int i1 = i0 + kRoundsPerChunk < rounds ? i0 + kRoundsPerChunk : rounds;
+    for (int i = i0; i < i1; i += 2) {  // chunks hold an even number of rounds: round i's words are in bufA
+      step(i, bufA);
+      if (i + 1 < i1) step(i + 1, bufB);
+    }
+    // end of a chunk: its slice sums added in rank order by the CTA that owns the row
+    cluster.sync();
+    const int rows = rows_c - cb < kC5Rows ? rows_c - cb : kC5Rows;
+    const int q0 = rows * rank / kC5, q1 = rows * (rank + 1) / kC5;
+    for (int rl = q0 + tid; rl < q1; rl += kC5Threads) {
+      float sum = 0.0f;
+#pragma unroll
+      for (int q = 0; q < kC5; ++q) sum += cluster.map_shared_rank(psum, q)[rl];
+      const int64_t r = c0 + cb + rl;
+      out[r] = bias ? __ldg(scale + r) * sum + __ldg(bias + r) : __ldg(scale + r) * sum;
+    }
+    cluster.sync();  // slice sums read before the next chunk overwrites them (and before any CTA exits)
   }
 }
 
