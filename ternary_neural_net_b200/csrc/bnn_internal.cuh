@@ -104,10 +104,10 @@ int ternary_tc_error_count(int reset);
 // Tensor-core (tcgen05 kind::f16) ternary GEMM, in ternary_gemm_tc.cu.
 // Plan of the ternary kernel that decodes into tensor memory (one activation
 // tile): rows of weights per CTA (32, 64, 96 or 128) and CTAs per cluster
-// splitting the stages (1..4), for n weight rows of kt words, given how many
-// clusters of each size fit the GPU at once (active[ks - 1]; 0 = unusable).
-// Host only.
-void ternary_tmem_plan(int64_t n, int64_t kt, const int active[4], int* rows, int* ks);
+// splitting the stages (1..4), for n weight rows of k trits (ceil(k / 256)
+// stages), given how many clusters of each size fit the GPU at once
+// (active[ks - 1]; 0 = unusable).  Host only.
+void ternary_tmem_plan(int64_t n, int64_t k, const int active[4], int* rows, int* ks);
 bnn_status ternary_gemm_tc(const uint16_t* x_bf16, const uint16_t* packed, const float* scale, const float* bias,
                            int64_t m, int64_t n, int64_t k, float* out, cudaStream_t s);
 

@@ -83,6 +83,6 @@ extern "C" bnn_status bnn_probe_popc(int mode, int64_t blocks, int64_t iters, in
 
 extern "C" bnn_status bnn_probe_ternary_plan(int64_t n, int64_t k, const int* active, int* rows, int* ks) {
   if (n < 1 || k < 1 || !active || !rows || !ks) return BNN_ERR_INVALID_ARG;
-  bnn::ternary_tmem_plan(n, bnn::words10(k), active, rows, ks);
+  bnn::ternary_tmem_plan(n, k, active, rows, ks);
   return BNN_OK;
 }

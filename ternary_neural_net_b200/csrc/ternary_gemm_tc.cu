@@ -380,7 +380,7 @@ ternary_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16
   const int rank = KS > 1 ? static_cast<int>(blockIdx.x % KS) : 0;
   const int64_t j0 = static_cast<int64_t>(blockIdx.x / KS) * kT2M;  // first weight row
   const int64_t i0 = static_cast<int64_t>(blockIdx.y) * BN;        // first activation row
-  const int64_t total = (10 * kt + 63) / 64;                         // 64-trit stages covering every word
+  const int64_t total = (k + 63) / 64;  // 64-trit stages up to trit k (past it, only pad trits of the last word)
   const int64_t share = (total + KS - 1) / KS;
   const int64_t sb = rank * share < total ? rank * share : total;
   const int64_t se = sb + share < total ? sb + share : total;
@@ -765,7 +765,7 @@ template <int KS>
 __global__ void __launch_bounds__(kT3Threads, 1)
 ternary_gemm_tmem_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t* __restrict__ packed,
                          const float* __restrict__ scale, const float* __restrict__ bias, int64_t m, int64_t n,
-                         int64_t kt, int rows_cta, int preload, float* __restrict__ out) {
+                         int64_t k, int64_t kt, int rows_cta, int preload, float* __restrict__ out) {
   using namespace bnn::tc;
   constexpr int kMaxCols = 4 * ((kT3Units + KS - 1) / KS);
   constexpr int kPitch = kMaxCols + 4;  // padded receive row (floats)
@@ -791,7 +791,7 @@ ternary_gemm_tmem_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint1
   const int rank = KS > 1 ? static_cast<int>(blockIdx.x % KS) : 0;
   const int64_t j0 = static_cast<int64_t>(blockIdx.x / KS) * rows_cta;  // first weight row (rows_cta: 32..128)
   const int64_t i0 = static_cast<int64_t>(blockIdx.y) * kT3N;        // first activation row
-  const int64_t total = (10 * kt + kT3K - 1) / kT3K;                 // stages covering every word
+  const int64_t total = (k + kT3K - 1) / kT3K;  // stages up to trit k (past it, only pad trits of the last word)
   const int64_t share = (total + KS - 1) / KS;
   const int64_t sb = rank * share < total ? rank * share : total;
   const int64_t se = sb + share < total ? sb + share : total;
@@ -1168,7 +1168,7 @@ int tmem_active_clusters() {
 
 template <int KS>
 bnn_status launch_tmem(const CUtensorMap& tx, const uint16_t* packed, const float* scale, const float* bias, int64_t m,
-                       int64_t n, int64_t kt, int rows_cta, float* out, cudaStream_t s) {
+                       int64_t n, int64_t k, int64_t kt, int rows_cta, float* out, cudaStream_t s) {
   const int64_t gx = KS * ((n + rows_cta - 1) / rows_cta), gy = (m + kT3N - 1) / kT3N;
   if (gx > 2147483647LL || gy > 65535) return BNN_ERR_INVALID_ARG;
   auto kern = ternary_gemm_tmem_kernel<KS>;
@@ -1177,7 +1177,7 @@ bnn_status launch_tmem(const CUtensorMap& tx, const uint16_t* packed, const floa
   // (a rank of a split-K cluster needs only its share of each row's words: group loads)
   const int preload = (KS == 1 && tmem_preload_fits(rows_cta, kt)) ? 1 : 0;
   const cudaError_t e = bnn::launch_pdl(kern, dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)),
-                                        dim3(kT3Threads), smem, s, KS, tx, packed, scale, bias, m, n, kt, rows_cta,
+                                        dim3(kT3Threads), smem, s, KS, tx, packed, scale, bias, m, n, k, kt, rows_cta,
                                         preload, out);
   if (e != cudaSuccess) return bnn::cuda_fail(e);
   return bnn::check_launch();
@@ -1203,8 +1203,8 @@ int ternary_tc_error_count(int reset) {
 // latency), and every CTA pays about two stages of start-up (its first words),
 // plus two for the exchange of a split.  CTAs of a cluster take whole SMs, so
 // few clusters of 3 or 4 run at once.
-void ternary_tmem_plan(int64_t n, int64_t kt, const int active[4], int* rows, int* ks) {
-  const int64_t stages = (10 * kt + kT3K - 1) / kT3K;
+void ternary_tmem_plan(int64_t n, int64_t k, const int active[4], int* rows, int* ks) {
+  const int64_t stages = (k + kT3K - 1) / kT3K;
   int best_ks = 1, best_rows = kT3M;
   int64_t best_cost = INT64_MAX;
   for (int r = kT3M; r >= 32; r -= 32) {
@@ -1237,12 +1237,12 @@ bnn_status ternary_gemm_tc(const uint16_t* x_bf16, const uint16_t* packed, const
       const int active[4] = {tmem_active_clusters<1>(), tmem_active_clusters<2>(), tmem_active_clusters<3>(),
                              tmem_active_clusters<4>()};
       int rows = kT3M, ks = 1;
-      ternary_tmem_plan(n, kt, active, &rows, &ks);
+      ternary_tmem_plan(n, k, active, &rows, &ks);
       switch (ks) {
-        case 4: return launch_tmem<4>(tx, packed, scale, bias, m, n, kt, rows, out, s);
-        case 3: return launch_tmem<3>(tx, packed, scale, bias, m, n, kt, rows, out, s);
-        case 2: return launch_tmem<2>(tx, packed, scale, bias, m, n, kt, rows, out, s);
-        default: return launch_tmem<1>(tx, packed, scale, bias, m, n, kt, rows, out, s);
+        case 4: return launch_tmem<4>(tx, packed, scale, bias, m, n, k, kt, rows, out, s);
+        case 3: return launch_tmem<3>(tx, packed, scale, bias, m, n, k, kt, rows, out, s);
+        case 2: return launch_tmem<2>(tx, packed, scale, bias, m, n, k, kt, rows, out, s);
+        default: return launch_tmem<1>(tx, packed, scale, bias, m, n, k, kt, rows, out, s);
       }
     }
     // activation tiles of 256 rows above m = 128, 128 above m = 64 (each weight
