@@ -204,84 +204,109 @@ sparse_gemm_kernel(const uint16_t* __restrict__ x, const int64_t* __restrict__ r
 
 // The layer at m = 1: x staged once per CTA in shared memory as float32 (k
 // floats, k <= 32768), so every gather is a shared-memory load.  One CTA per
-// SM takes a contiguous block of rows; a warp takes every 32nd of them.  Per
-// row the lanes hold up to 512 entries in registers (16 per lane, 64-byte
-// coalesced loads), and the first 512 entries of the warp's next row are
-// loaded while this row's are gathered, so each warp keeps 32 loads in
-// flight.  The row's sum is added by a shuffle tree (a fixed order), scaled
-// once (and biased).  Row ptr and entries are read before the programmatic-
-// launch wait, x after it.
+// SM takes a contiguous block of rows, in chunks of kSpChunk = 96: the chunk's
+// row_ptr values are read into shared memory once, and warp w takes rows w,
+// w + 32 and w + 64 of it.  A warp issues the loads of all its rows' first
+// 511..512 entries at once, before the programmatic-launch wait and the
+// staging of x (each lane eight 32-bit entry pairs per row, 128-byte coalesced
+// loads from the even entry at or below the row's first), so the whole
+// chunk's entries are in flight together.  A pair's halves outside the row
+// contribute nothing (the gathered value is masked in the same logic op that
+// applies the sign).  Longer rows take further passes of 512 entries.  The
+// row's sum is added by a shuffle tree (a fixed order), scaled once (and
+// biased).  VEC: entries 4-byte aligned (one 32-bit load per pair), else two
+// 16-bit loads.
 constexpr int kSpThreads = 1024;
-constexpr int kSpU = 16;  // entries per lane per pass
+constexpr int kSpR = 3;                         // rows per warp and chunk
+constexpr int kSpChunk = kSpThreads / 32 * kSpR;
+constexpr int kSpW = 8;                         // entry pairs per lane per pass
 
+// entries q, q + 1 (bits 0..15 and 16..31; q even relative to the row's pass
+// start); entries at or past e are not read (their halves are masked off, and
+// e may be the end of the array)
+template <bool VEC>
+__device__ __forceinline__ uint32_t sp_pair(const uint16_t* __restrict__ entries, int64_t q, int64_t e) {
+  if (q >= e) return 0u;
+  if (VEC && q + 1 < e) return __ldcs(reinterpret_cast<const uint32_t*>(entries + q));
+  const uint32_t lo = __ldcs(entries + q);
+  return q + 1 < e ? lo | (static_cast<uint32_t>(__ldcs(entries + q + 1)) << 16) : lo;
+}
+
+// the contributions of one pass of a row: pairs v[i] hold entries a + 2 (32 i
+// + lane) and the one after; only those in [b, e) count (offsets within the
+// pass are 32-bit: 0 <= max(b - a, 0) and min(e - a, 64 W) <= 64 W)
+template <int W>
+__device__ __forceinline__ float sp_gather(const float* xs, const uint32_t (&v)[W], int64_t a, int64_t b, int64_t e,
+                                           int lane, uint32_t kk) {
+  const int lo = b > a ? static_cast<int>(b - a) : 0;
+  const int hi = e - a < 64 * W ? static_cast<int>(e - a) : 64 * W;
+  const int span = hi > lo ? hi - lo : 0;  // entries of the row in this pass
+  const int base = 2 * lane - lo;    // offset of pair 0's first entry from the row's first in the pass
+  float acc0 = 0.0f, acc1 = 0.0f;
+#pragma unroll
+  for (int i = 0; i < W; ++i) {
+    const uint32_t d = static_cast<uint32_t>(base + 64 * i);
+    const uint32_t p0 = min(v[i] & 0x7FFFu, kk), p1 = min((v[i] >> 16) & 0x7FFFu, kk);  // >= k: the zero slot
+    const float t0 = __uint_as_float(__float_as_uint(xs[p0]) ^ ((v[i] << 16) & 0x80000000u));  // sign: bit 15
+    const float t1 = __uint_as_float(__float_as_uint(xs[p1]) ^ (v[i] & 0x80000000u));          // sign: bit 31
+    if (d < static_cast<uint32_t>(span)) acc0 += t0;
+    if (d + 1u < static_cast<uint32_t>(span)) acc1 += t1;
+  }
+  return acc0 + acc1;
+}
+
+template <bool VEC>
 __global__ void __launch_bounds__(kSpThreads, 1)
 sparse_gemv_smem_kernel(const uint16_t* __restrict__ x, const int64_t* __restrict__ row_ptr,
                         const uint16_t* __restrict__ entries, const float* __restrict__ scale,
                         const float* __restrict__ bias, int64_t n, int k, float* __restrict__ out) {
-  extern __shared__ float xs[];  // [k + 1]: x as float32, then xs[k] = 0 (the slot of padding and malformed entries)
+  extern __shared__ float xs[];  // [k + 1]: x as float32, then xs[k] = 0
+  __shared__ int64_t rp[kSpChunk + 1];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int kWarps = kSpThreads / 32;
   const int64_t r_begin = n * blockIdx.x / gridDim.x, r_end = n * (blockIdx.x + 1) / gridDim.x;
+  const uint32_t kk = static_cast<uint32_t>(k);
   bnn::pdl_trigger();
-
-  // entries [b + 32 u + lane] of one pass; past the row's end the value 2^16, which no
-  // 16-bit entry holds and which the position clamp below sends to the zero slot (at
-  // k = 32768 every 15-bit position is a real one, so the padding cannot be one)
-  const uint32_t pad = 0x10000u, kk = static_cast<uint32_t>(k);
-  auto fetch = [&](int64_t q0, int64_t e, uint32_t (&v)[kSpU]) {
+  bool staged = false;
+  for (int64_t cb = r_begin; cb < r_end; cb += kSpChunk) {
+    const int rows = static_cast<int>(r_end - cb < kSpChunk ? r_end - cb : kSpChunk);
+    if (tid <= rows) rp[tid] = row_ptr[cb + tid];
+    __syncthreads();
+    // every row's first pass, in flight together
+    uint32_t v[kSpR][kSpW];
 #pragma unroll
-    for (int u = 0; u < kSpU; ++u) {
-      const int64_t q = q0 + 32 * u + lane;
-      v[u] = q < e ? static_cast<uint32_t>(__ldcs(entries + q)) : pad;
-    }
-  };
-  int64_t r = r_begin + warp;
-  int64_t b = 0, e = 0;
-  uint32_t cur[kSpU];
-  if (r < r_end) {
-    b = row_ptr[r];
-    e = row_ptr[r + 1];
-  }
-  fetch(b, e, cur);
-
-  bnn::pdl_wait();  // x may come from the kernel ahead
-  for (int i = tid; i < k; i += kSpThreads) xs[i] = __uint_as_float(static_cast<uint32_t>(__ldg(x + i)) << 16);
-  if (tid == 0) xs[k] = 0.0f;
-  __syncthreads();
-
-  while (r < r_end) {
-    const int64_t rn = r + kWarps;
-    int64_t bn = 0, en = 0;
-    if (rn < r_end) {
-      bn = row_ptr[rn];
-      en = row_ptr[rn + 1];
-    }
-    uint32_t nxt[kSpU];
-    fetch(bn, en, nxt);  // the next row's first pass, in flight during this row
-    float acc0 = 0.0f, acc1 = 0.0f;
-    for (int64_t q0 = b;;) {
+    for (int j = 0; j < kSpR; ++j) {
+      const int rl = warp + 32 * j;
+      const int64_t b = rl < rows ? rp[rl] : 0, e = rl < rows ? rp[rl + 1] : 0;
+      const int64_t a = b & ~int64_t{1};
 #pragma unroll
-      for (int u = 0; u < kSpU; ++u) {
-        const uint32_t v = cur[u];
-        // positions >= k (malformed) and the padding (bit 16 kept by the mask) read the zero slot xs[k]
-        const uint32_t pos = min(v & 0x17FFFu, kk);
-        const float t = __uint_as_float(__float_as_uint(xs[pos]) ^ ((v << 16) & 0x80000000u));  // sign bit 15
-        if (u & 1) acc1 += t;
-        else acc0 += t;
+      for (int i = 0; i < kSpW; ++i) v[j][i] = sp_pair<VEC>(entries, a + 2 * (32 * i + lane), e);
+    }
+    if (!staged) {
+      bnn::pdl_wait();  // x may come from the kernel ahead
+      for (int i = tid; i < k; i += kSpThreads) xs[i] = __uint_as_float(static_cast<uint32_t>(__ldg(x + i)) << 16);
+      if (tid == 0) xs[k] = 0.0f;
+      __syncthreads();
+      staged = true;
+    }
+#pragma unroll
+    for (int j = 0; j < kSpR; ++j) {
+      const int rl = warp + 32 * j;
+      if (rl >= rows) break;
+      const int64_t b = rp[rl], e = rp[rl + 1];
+      int64_t a = b & ~int64_t{1};
+      float sum = sp_gather<kSpW>(xs, v[j], a, b, e, lane, kk);
+      for (a += 64 * kSpW; a < e; a += 64 * kSpW) {  // rows of more than one pass
+        uint32_t w[kSpW];
+#pragma unroll
+        for (int i = 0; i < kSpW; ++i) w[i] = sp_pair<VEC>(entries, a + 2 * (32 * i + lane), e);
+        sum += sp_gather<kSpW>(xs, w, a, b, e, lane, kk);
       }
-      q0 += 32 * kSpU;
-      if (q0 >= e) break;
-      fetch(q0, e, cur);  // rows longer than one pass
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+      const int64_t r = cb + rl;
+      if (lane == 0) out[r] = bias ? __ldg(scale + r) * sum + __ldg(bias + r) : __ldg(scale + r) * sum;
     }
-    float sum = acc0 + acc1;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-    if (lane == 0) out[r] = bias ? __ldg(scale + r) * sum + __ldg(bias + r) : __ldg(scale + r) * sum;
-    r = rn;
-    b = bn;
-    e = en;
-#pragma unroll
-    for (int u = 0; u < kSpU; ++u) cur[u] = nxt[u];
+    __syncthreads();  // rp is refilled by the next chunk
   }
 }
 
@@ -330,11 +355,17 @@ extern "C" bnn_status bnn_ternary_sparse_gemm(const uint16_t* x_bf16, const int6
     return BNN_ERR_MISALIGNED;
   if (m == 1 && k > 0) {
     const size_t smem = static_cast<size_t>(k + 1) * sizeof(float);
-    BNN_TRY(bnn::ensure_smem(sparse_gemv_smem_kernel, smem));
     const int64_t sms = bnn::sm_count();
     const int grid = static_cast<int>(n < sms ? n : sms);
-    BNN_TRY(bnn::launch_pdl(sparse_gemv_smem_kernel, dim3(grid), dim3(kSpThreads), smem, s, 1, x_bf16, row_ptr,
-                            entries, scale, bias, n, static_cast<int>(k), out));
+    if (entries && bnn::aligned(entries, 4)) {
+      BNN_TRY(bnn::ensure_smem(sparse_gemv_smem_kernel<true>, smem));
+      BNN_TRY(bnn::launch_pdl(sparse_gemv_smem_kernel<true>, dim3(grid), dim3(kSpThreads), smem, s, 1, x_bf16,
+                              row_ptr, entries, scale, bias, n, static_cast<int>(k), out));
+    } else {
+      BNN_TRY(bnn::ensure_smem(sparse_gemv_smem_kernel<false>, smem));
+      BNN_TRY(bnn::launch_pdl(sparse_gemv_smem_kernel<false>, dim3(grid), dim3(kSpThreads), smem, s, 1, x_bf16,
+                              row_ptr, entries, scale, bias, n, static_cast<int>(k), out));
+    }
     return bnn::check_launch();
   }
   const dim3 grid(warp_grid(n)), block(kWarpsPerBlock * 32);

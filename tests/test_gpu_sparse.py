@@ -125,3 +125,26 @@ def test_sparse_gemv_m1_shapes(bnn, n, k, density):
         want, mag = oracle.sparse_gemm(xb, rp, en, scale, b, 1, n, k)
         lim = mag + (0 if b is None else np.abs(b.astype(np.float64)))
         assert_ternary_close(got.cpu().numpy(), want, lim, f"sparse m=1 {n}x{k}")
+
+
+@pytest.mark.parametrize("n,k,density", [(11008, 4096, 0.1), (300, 5000, 0.6)])
+def test_sparse_gemv_m1_entries_two_bytes_off(bnn, n, k, density):
+    """m = 1 with the entries 2 bytes off a 4-byte boundary (16-bit loads of
+    each pair instead of one 32-bit load): the same sums in the same order, so
+    bit-identical outputs, and both match the oracle."""
+    rng = np.random.default_rng(3 * n + k)
+    trits = ((rng.integers(0, 2, (n, k)) * 2 - 1) * (rng.random((n, k)) < density)).astype(np.int8)
+    scale = (rng.random(n) + 0.5).astype(np.float32)
+    xb = synth.bf16_bits_from_f32(synth.normal_f32(n + k, 2, (1, k)))
+    _, row_ptr, ent = _encode(bnn, trits, k)
+    buf = torch.empty(ent.numel() + 1, dtype=ent.dtype, device="cuda")
+    buf[1:] = ent
+    ent_off = buf[1:]
+    assert ent.data_ptr() % 4 == 0 and ent_off.data_ptr() % 4 == 2
+    xd, sd = to_dev_bf16(xb), to_dev_f32(scale)
+    got = bnn.bnn_ternary_sparse_gemm(xd, row_ptr, ent, sd)
+    got_off = bnn.bnn_ternary_sparse_gemm(xd, row_ptr, ent_off, sd)
+    assert torch.equal(got.view(torch.int32), got_off.view(torch.int32))
+    rp, en = oracle.sparse_encode(trits)
+    want, mag = oracle.sparse_gemm(xb, rp, en, scale, None, 1, n, k)
+    assert_ternary_close(got.cpu().numpy(), want, mag, f"sparse m=1 {n}x{k} entries +2")
