@@ -473,53 +473,88 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
 }
 
 // ---------------------------------------------------------------------------
-// Two-SM persistent variant for large GEMMs.  A cluster of two CTAs computes
-// tiles of 256 weight rows x 256 activation rows with tcgen05.mma.cta_group::2
-// (UMMA M = 256, N = 256): CTA q of the pair holds weight rows 128q.. of the
-// tile (its half of operand A, and the tensor-memory lanes of those rows) and
-// activation rows 128q.. (its half of operand B); one MMA reads both CTAs'
-// shared memory, so each SM expands only 256 rows per stage instead of the
-// 384 of a 128 x 256 tile on one SM, and its tensor memory receives all 256
-// accumulator columns of its 128 weight rows.  The pairs are persistent: pair
-// p takes tiles p, p + P, ... (P pairs, at most as many as fit the GPU at
-// once), and the accumulator is double-buffered in tensor memory (2 x 256
-// columns), so the epilogue of one tile overlaps the mainloop of the next.
+// Two-SM persistent variant for large GEMMs, on the 4-bit float tensor cores.
+//
+// The AND count popc(a AND b) is a dot product of 0/1 vectors.  Here each bit
+// becomes an e2m1 float, 1.0 (code 0b0010) or 0.0, and the pair runs
+// tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 with every ue8m0
+// scale factor 127 (2^0): the products are exactly 0 or 1 and the float32
+// accumulator holds the count exactly while it stays below 2^24 (k < 2^24,
+// checked on the host).  Per instruction K = 64 at twice the int8 rate, and
+// an expanded bit takes half a byte.
+//
+// A cluster of two CTAs computes tiles of 256 weight rows x kPN = 224
+// activation rows (UMMA M = 256, N = 224): CTA q of the pair holds weight
+// rows 128q.. of the tile (its half of operand A, and the tensor-memory lanes
+// of those rows) and activation rows 112q.. (its half of operand B); one MMA
+// reads both CTAs' shared memory.  The pairs are persistent: pair p takes
+// tiles p, p + P, ... (P pairs, at most as many as fit the GPU at once).  The
+// accumulator is double-buffered in tensor memory (2 x 224 columns, so the
+// epilogue of one tile overlaps the mainloop of the next); columns 448..511
+// hold the scale factors, written once by the epilogue warps of both CTAs
+// before the first MMA (every byte 127, so their layout within those columns
+// does not matter).
 //
 // Roles per CTA:
-//   - a TMA thread copies the packed chunks (4 stages of its own 128 weight and
-//     128 activation rows) into a two-chunk ring;
+//   - a TMA thread copies the packed chunks (4 stages of 4 words, 128 bytes of
+//     each of its own 128 weight and 112 activation rows, 128-byte swizzle)
+//     into a two-chunk ring;
 //   - four producer groups of 128 threads; group g takes stage g of every
-//     chunk, thread t weight row t and activation row t (both 64-bit words of
-//     the stage), so four stages are expanded at once and the latency of one
-//     (loads, stores, proxy fence, barrier) hides behind the others.  After a
-//     named barrier of its 128 threads a group arrives once on the stage's
-//     "full" mbarrier of CTA 0 (at cluster scope), which thus completes once
-//     both CTAs' groups have written the stage;
-//   - CTA 0's MMA thread waits for "full", issues 4 tcgen05.mma (K = 32) into
+//     chunk, thread t weight row t and activation row t (t < 112): each 32
+//     bits of a row's four words become one 16-byte unit of nibbles (word s
+//     of the unit holds bits s, s + 4, ... as 0 or 2, the same permutation of
+//     k in both operands), so four stages are expanded at once and the latency
+//     of one (loads, stores, proxy fence, barrier) hides behind the others.
+//     After a named barrier of its 128 threads a group arrives once on the
+//     stage's "full" mbarrier of CTA 0 (at cluster scope), which thus
+//     completes once both CTAs' groups have written the stage;
+//   - CTA 0's MMA thread waits for "full", issues 4 MMAs (K = 64) into
 //     accumulator buffer t % 2, and commits with a two-CTA mask to the stage's
 //     "empty" barrier in both CTAs (and to "acc_full" after a tile's last
 //     stage); before a tile it waits on "acc_empty" for the epilogue that read
 //     the buffer two tiles back;
-//   - four epilogue warps (one per quarter of the tensor-memory lanes) read
-//     the accumulator, apply the popcount correction (row popcounts from a
-//     pass before the kernel), alpha and the optional bias, store, and arrive
-//     on CTA 0's "acc_empty".
+//   - eight epilogue warps (two per quarter of the tensor-memory lanes, each
+//     half of the columns) read the accumulator (the count, exact in float32),
+//     apply the popcount correction (row popcounts from a pass before the
+//     kernel), alpha and the optional bias, store, and arrive on CTA 0's
+//     "acc_empty".
 // The stage, chunk and accumulator rings run on across tiles.  Every wait is
 // bounded; a wait that runs out stops every role of the CTA (the other CTA's
 // waits then run out too) and leaves the outputs unspecified.
 // ---------------------------------------------------------------------------
-constexpr int kQRows = 256;                                     // stacked rows per CTA (128 weight + 128 activation)
-constexpr uint32_t kQStageBytes = kQRows * 128u;                // one expanded stage (32 KiB)
-constexpr uint32_t kQChunkBytes = kQRows * 16u * kChunkStages;  // one packed chunk (16 KiB)
-constexpr int kQS = 6, kQP = 2;                                 // expanded stages, packed chunks
+constexpr int kPX = 112;                                        // activation rows per CTA (N / 2)
+constexpr int kPN = 2 * kPX;                                    // activation rows per tile (UMMA N)
+constexpr int kQRows = kTm + kPX;                               // stacked rows per CTA (128 weight + 112 activation)
+constexpr int kQWords = 4;                                      // packed words per row and stage (K = 256 bits)
+constexpr uint32_t kQRowBytes = 8u * kQWords * kChunkStages;    // a packed chunk row (128 bytes)
+constexpr uint32_t kQStageBytes = kQRows * 128u;                // one expanded stage (30 KiB)
+constexpr uint32_t kQChunkBytes = kQRows * kQRowBytes;          // one packed chunk (30 KiB)
+constexpr int kQS = 5, kQP = 2;                                 // expanded stages, packed chunks
 constexpr int kQG = kChunkStages;                               // producer groups (one stage of every chunk each)
 constexpr int kQGroup = kTm;                                    // threads per group
 constexpr int kQProducers = kQG * kQGroup;                      // 512
 constexpr int kQMmaWarp = kQProducers / 32, kQTmaWarp = kQMmaWarp + 1, kQEpiWarp0 = kQMmaWarp + 2;
-constexpr int kQThreads = kQProducers + 64 + 128;               // + MMA warp + TMA warp + 4 epilogue warps
+constexpr int kQEpi = 8;                                        // epilogue warps (two per lane quarter)
+constexpr int kQThreads = kQProducers + 64 + 32 * kQEpi;        // + MMA warp + TMA warp + epilogue warps
 constexpr uint32_t kQSmem = kQS * kQStageBytes + kQP * kQChunkBytes;
-constexpr uint32_t kQTmemCols = 512;                            // two 256-column accumulators
+constexpr uint32_t kQTmemCols = 512;                            // two 224-column accumulators + scale factors
+constexpr uint32_t kQSfCol = 2 * kPN;                           // scale factors: columns [448, 512)
 constexpr int kQEpiBar = 2 + kQG;                               // named barrier of the epilogue warps
+static_assert(kPX % 8 == 0 && kPN % 32 == 0 && kPN % 16 == 0 && kPN <= 256, "UMMA N and the epilogue's column blocks");
+static_assert(kQStageBytes % 1024 == 0 && kQChunkBytes % 1024 == 0, "128-byte swizzle atoms stay 1024-byte aligned");
+static_assert(kQSfCol + 64 <= kQTmemCols, "scale-factor columns");
+
+// 32 bits of a packed row as one 16-byte unit of e2m1 nibbles (0 or 2 = 1.0):
+// word s of the unit holds bits s, s + 4, ..., s + 28 of hw (nibble j = bit
+// 4j + s), the same permutation of k in both operands
+__device__ __forceinline__ uint4 nibbles_of(uint32_t hw) {
+  uint4 v;
+  v.x = (hw << 1) & 0x22222222u;
+  v.y = hw & 0x22222222u;
+  v.z = (hw >> 1) & 0x22222222u;
+  v.w = (hw >> 2) & 0x22222222u;
+  return v;
+}
 
 __global__ void __launch_bounds__(kQThreads, 1)
 binary_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
@@ -539,15 +574,15 @@ binary_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
   __shared__ __align__(8) uint64_t done_bar;
   __shared__ uint32_t tmem_holder;
   __shared__ volatile int abort_flag;
-  __shared__ int pop_xs[256];                      // the epilogue's tile: activation-row popcounts
+  __shared__ int pop_xs[kPN];                      // the epilogue's tile: activation-row popcounts
   uint8_t* const smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* const chunks = smem + kQS * kQStageBytes;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster.block_rank();
   const int64_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-  const int64_t ntn = (n + 255) / 256, ntiles = ntn * ((m + 255) / 256);
-  const int nst = (kw + 1) / 2, nch = (nst + kChunkStages - 1) / kChunkStages;
+  const int64_t ntn = (n + 255) / 256, ntiles = ntn * ((m + kPN - 1) / kPN);
+  const int nst = (kw + kQWords - 1) / kQWords, nch = (nst + kChunkStages - 1) / kChunkStages;
   const uint32_t smem_base = smem_u32(smem);
 
   if (tid == 0) {
@@ -577,16 +612,29 @@ binary_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;\n" ::);
   }
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
-  cluster.sync();  // both CTAs' barriers exist before any arrival from the other CTA
+  __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
   const uint32_t tmem = tmem_holder;
+  if (warp >= kQEpiWarp0 && warp < kQEpiWarp0 + 4) {  // scale factors: 127 in every byte of columns [448, 512)
+    const uint32_t lanes = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    for (uint32_t c = kQSfCol; c < kQTmemCols; c += 8)
+      asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1};\n" ::"r"(tmem + lanes + c),
+                   "r"(0x7F7F7F7Fu)
+                   : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+  cluster.sync();  // both CTAs' barriers and scale factors exist before any arrival or MMA
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
   bnn::pdl_trigger();
 
   if (tid < kQProducers) {
     // ------------------------------------------------------------ producers
     const int g = tid / kQGroup, t = tid % kQGroup;
-    const uint32_t swz = static_cast<uint32_t>(t & 7);
-    const uint32_t rd = ((static_cast<uint32_t>(g) ^ ((t >> 1) & 3)) << 4);  // stage g's unit in a chunk row
+    const uint32_t swz = static_cast<uint32_t>(t & 7);  // 128-byte swizzle phase of rows t and 128 + t
+    // stage g's two 16-byte units of a chunk row under the 128-byte swizzle
+    const uint32_t rd0 = ((2u * g) ^ swz) << 4, rd1 = ((2u * g + 1u) ^ swz) << 4;
+    const bool has_x = t < kPX;
     bool ok = true;
     uint32_t gc = 0;  // chunks consumed so far (all tiles)
     uint32_t ts = 0;  // first stage of the tile, counted over all tiles (the launch keeps it below 2^31)
@@ -604,14 +652,19 @@ binary_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
           ok = bnn::tc::mbar_wait(smem_u32(&empty_bar[b]), (gs / kQS + 1) & 1u, &abort_flag, &g_bnn_device_errors,
                                   wait_limit);
         if (ok && has) {
-          const uint8_t* ck = chunks + pb * kQChunkBytes + rd;
-          const uint4 vw = *reinterpret_cast<const uint4*>(ck + t * 64u);
-          const uint4 vx = *reinterpret_cast<const uint4*>(ck + (t + kTm) * 64u);  // same swizzle unit as row t
-          uint8_t* dst = smem + b * kQStageBytes + static_cast<uint32_t>(t) * 128u;
-          expand_word(dst, swz, 0, (static_cast<uint64_t>(vw.y) << 32) | vw.x);
-          expand_word(dst, swz, 1, (static_cast<uint64_t>(vw.w) << 32) | vw.z);
-          expand_word(dst + kTm * 128u, swz, 0, (static_cast<uint64_t>(vx.y) << 32) | vx.x);
-          expand_word(dst + kTm * 128u, swz, 1, (static_cast<uint64_t>(vx.w) << 32) | vx.z);
+          // row r's four words of the stage (eight 32-bit halves) -> units 0..7 of its stage row
+          auto expand_row = [&](int r) {
+            const uint8_t* ck = chunks + pb * kQChunkBytes + static_cast<uint32_t>(r) * kQRowBytes;
+            const uint4 v0 = *reinterpret_cast<const uint4*>(ck + rd0);
+            const uint4 v1 = *reinterpret_cast<const uint4*>(ck + rd1);
+            uint8_t* dst = smem + b * kQStageBytes + static_cast<uint32_t>(r) * 128u;
+            const uint32_t h[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              *reinterpret_cast<uint4*>(dst + ((static_cast<uint32_t>(u) ^ swz) << 4)) = nibbles_of(h[u]);
+          };
+          expand_row(t);
+          if (has_x) expand_row(kTm + t);
           asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
         }
         // the group's rows of the stage are written (or a wait ran out: the group stops together)
@@ -626,8 +679,11 @@ binary_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
   } else if (warp == kQMmaWarp) {
     // ------------------------------------------------------------ MMA issue (CTA 0)
     if (rank == 0 && lane == 0) {
-      // D s32, A and B 8-bit integers, both K-major, N = 256, M = 256 (two CTAs)
-      const uint32_t idesc = (2u << 4) | (1u << 7) | (1u << 10) | ((256u >> 3) << 17) | ((256u >> 4) << 24);
+      // D f32; A and B e2m1 (format 1), K-major; ue8m0 scales (bit 23); N = 224, M = 256 (two CTAs);
+      // dense K = 64; scale-factor ids 0
+      const uint32_t idesc = (1u << 7) | (1u << 10) | ((static_cast<uint32_t>(kPN) >> 3) << 17) | (1u << 23) |
+                             ((256u >> 4) << 24);
+      const uint32_t sfa = tmem + kQSfCol, sfb = tmem + kQSfCol + 32u;
       bool ok = true;
       for (int64_t tile = pair, ti = 0; tile < ntiles && ok; tile += npairs, ++ti) {
         const int tb = static_cast<int>(ti & 1);
@@ -635,7 +691,7 @@ binary_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
         if (ti >= 2)
           ok = bnn::tc::mbar_wait_cluster(smem_u32(&acc_empty[tb]), static_cast<uint32_t>((ti / 2 + 1) & 1),
                                           &abort_flag, &g_bnn_device_errors, wait_limit);
-        const uint32_t d = tmem + 256u * static_cast<uint32_t>(tb);
+        const uint32_t d = tmem + static_cast<uint32_t>(kPN) * static_cast<uint32_t>(tb);
         for (int j = 0; j < nst && ok; ++j) {
           const uint32_t gs = static_cast<uint32_t>(ti) * static_cast<uint32_t>(nst) + static_cast<uint32_t>(j);
           const int b = static_cast<int>(gs % kQS);
@@ -650,9 +706,10 @@ binary_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
             const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
             asm volatile(
                 "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
-                "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
+                "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n}\n" ::"r"(
+                    d),
                 "l"(ad + static_cast<uint64_t>(2 * kk)), "l"(bd + static_cast<uint64_t>(2 * kk)), "r"(idesc),
-                "r"(acc));
+                "r"(acc), "r"(sfa), "r"(sfb));
           }
           asm volatile(
               "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n" ::
@@ -682,7 +739,7 @@ binary_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
       bool ok = true;
       for (int64_t tile = pair; tile < ntiles && ok; tile += npairs) {
         const int j0 = static_cast<int>((tile % ntn) * 256 + 128 * rank);
-        const int iq = static_cast<int>((tile / ntn) * 256 + 128 * rank);
+        const int iq = static_cast<int>((tile / ntn) * kPN + kPX * rank);
         for (int c = 0; c < nch; ++c, ++gc) {
           const int pb = static_cast<int>(gc % kQP);
           if (gc >= static_cast<uint32_t>(kQP) &&
@@ -694,8 +751,8 @@ binary_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
           const uint32_t dst = smem_u32(chunks + pb * kQChunkBytes);
           const uint32_t bar = smem_u32(&chunk_full[pb]);
           mbar_expect_tx(bar, kQChunkBytes);
-          tma_load_2d(dst, &tmap_w, 2 * kChunkStages * c, j0, bar);
-          tma_load_2d(dst + kTm * 16u * kChunkStages, &tmap_x, 2 * kChunkStages * c, iq, bar);
+          tma_load_2d(dst, &tmap_w, kQWords * kChunkStages * c, j0, bar);
+          tma_load_2d(dst + kTm * kQRowBytes, &tmap_x, kQWords * kChunkStages * c, iq, bar);
         }
       }
       // the CTA must not retire with copies in flight: wait for the last chunk issued into each buffer
@@ -704,20 +761,23 @@ binary_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
     }
   } else {
     // ------------------------------------------------------------ epilogue warps
+    // warp ew reads lanes 32 q.. (q = warp % 4) of activation columns
+    // [112 h, 112 h + 112), h = ew / 4
     bnn::pdl_wait();  // the row popcounts come from the preceding kernel
-    const int et = tid - kQEpiWarp0 * 32;           // 0..127
+    const int et = tid - kQEpiWarp0 * 32;           // 0..255
     const int q = warp & 3;                         // tensor-memory lanes 32q..32q+31
+    const int cbeg = (et / 128) * (kPN / 2);        // this warp's first column
     const int erow = 32 * q + lane;
     const uint32_t lane_field = static_cast<uint32_t>(32 * q) << 16;
     const bool need_y = out || next;
     for (int64_t tile = pair, ti = 0; tile < ntiles; tile += npairs, ++ti) {
       const int tb = static_cast<int>(ti & 1);
-      const int64_t j0 = (tile % ntn) * 256 + 128 * rank, i0 = (tile / ntn) * 256;
+      const int64_t j0 = (tile % ntn) * 256 + 128 * rank, i0 = (tile / ntn) * kPN;
       const bool ok = bnn::tc::mbar_wait_idle(smem_u32(&acc_full[tb]), static_cast<uint32_t>((ti / 2) & 1),
                                               &abort_flag, &g_bnn_device_errors);
-      // the tile's 256 activation-row popcounts (0 past m) into shared memory
-      for (int i = et; i < 256; i += 128) pop_xs[i] = i0 + i < m ? __ldg(pop_x + i0 + i) : 0;
-      if (!bnn::tc::named_barrier_and(ok, kQEpiBar, 128)) break;  // the four warps stop together
+      // the tile's kPN activation-row popcounts (0 past m) into shared memory
+      for (int i = et; i < kPN; i += 32 * kQEpi) pop_xs[i] = i0 + i < m ? __ldg(pop_x + i0 + i) : 0;
+      if (!bnn::tc::named_barrier_and(ok, kQEpiBar, 32 * kQEpi)) break;  // the epilogue warps stop together
       asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
       const int64_t jrow = j0 + erow;
       const bool jlive = jrow < n;
@@ -726,20 +786,21 @@ binary_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
       const int base = k - 2 * (jlive ? __ldg(pop_w + jrow) : 0);
       const int64_t half = (j0 + 32 * q) / 32;
       const bool pack = next && half < next_w32;
-      const uint32_t taddr = tmem + lane_field + 256u * static_cast<uint32_t>(tb);
-      for (int c0 = 0; c0 < 256; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(taddr + static_cast<uint32_t>(c0), r);
+      const uint32_t taddr = tmem + lane_field + static_cast<uint32_t>(kPN) * static_cast<uint32_t>(tb);
+      for (int c0 = cbeg; c0 < cbeg + kPN / 2; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld16(taddr + static_cast<uint32_t>(c0), r);
         tmem_wait_ld();
         const int64_t rows_left = m - (i0 + c0);
-        const int nc = rows_left <= 0 ? 0 : (rows_left < 32 ? static_cast<int>(rows_left) : 32);
+        const int nc = rows_left <= 0 ? 0 : (rows_left < 16 ? static_cast<int>(rows_left) : 16);
         const int64_t off = (i0 + c0) * n + jrow;
         int32_t* dp = dots ? dots + off : nullptr;
         float* op = out ? out + off : nullptr;
         uint32_t* np = pack ? next + (i0 + c0) * next_w32 + half : nullptr;
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const int32_t dv = base - 2 * pop_xs[c0 + c] + 4 * static_cast<int32_t>(r[c]);
+        for (int c = 0; c < 16; ++c) {
+          // the AND count: an integer below 2^24, exact in the float32 accumulator
+          const int32_t dv = base - 2 * pop_xs[c0 + c] + 4 * static_cast<int32_t>(__uint_as_float(r[c]));
           const float y0 = __fmul_rn(a_j, static_cast<float>(dv));
           const float y = bias ? __fadd_rn(y0, b_j) : y0;
           if (c < nc && jlive) {
@@ -755,9 +816,9 @@ binary_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
           op += n;
         }
       }
-      // this CTA's four epilogue warps have read the buffer: one arrival on CTA 0's acc_empty
+      // this CTA's epilogue warps have read the buffer: one arrival on CTA 0's acc_empty
       asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
-      asm volatile("bar.sync %0, 128;\n" ::"r"(kQEpiBar) : "memory");
+      asm volatile("bar.sync %0, %1;\n" ::"r"(kQEpiBar), "r"(32 * kQEpi) : "memory");
       if (warp == kQEpiWarp0 && lane == 0) bnn::tc::mbar_arrive_rank(smem_u32(&acc_empty[tb]), 0u);
     }
   }
@@ -824,22 +885,24 @@ bnn_status launch_pair(const uint64_t* xp, const uint64_t* wp, const float* alph
                        int64_t n, int k, int kw, int32_t* dots, float* out, uint64_t* next, cudaStream_t s,
                        bool* launched) {
   *launched = false;
-  const int64_t ntiles = ((n + 255) / 256) * ((m + 255) / 256);
+  const int64_t ntiles = ((n + 255) / 256) * ((m + kPN - 1) / kPN);
+  // TMA rows (16-byte aligned: even kw, aligned bases), int32 coordinates, and
+  // AND counts (at most k) exact in float32
   if (kw <= 0 || kw % 2 != 0 || !bnn::aligned(xp, 16) || !bnn::aligned(wp, 16) || n >= (1LL << 31) ||
-      m >= (1LL << 31))
+      m >= (1LL << 31) || k >= (1 << 24))
     return BNN_OK;
   const int clusters = pair_clusters();
   if (clusters <= 0) return BNN_OK;
   // the kernel counts stages over a pair's tiles in 32 bits
-  const int64_t nst = (kw + 1) / 2, per_pair = (ntiles + clusters - 1) / clusters;
+  const int64_t nst = (kw + kQWords - 1) / kQWords, per_pair = (ntiles + clusters - 1) / clusters;
   if (per_pair * nst >= (int64_t{1} << 31)) return BNN_OK;
   CUtensorMap tw, tx;
   if (!bnn::encode_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT64, wp, static_cast<uint64_t>(kw),
-                           static_cast<uint64_t>(n), static_cast<uint64_t>(kw) * 8u, 2 * kChunkStages, kTm,
-                           CU_TENSOR_MAP_SWIZZLE_64B) ||
+                           static_cast<uint64_t>(n), static_cast<uint64_t>(kw) * 8u, kQWords * kChunkStages, kTm,
+                           CU_TENSOR_MAP_SWIZZLE_128B) ||
       !bnn::encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT64, xp, static_cast<uint64_t>(kw),
-                           static_cast<uint64_t>(m), static_cast<uint64_t>(kw) * 8u, 2 * kChunkStages, kTm,
-                           CU_TENSOR_MAP_SWIZZLE_64B))
+                           static_cast<uint64_t>(m), static_cast<uint64_t>(kw) * 8u, kQWords * kChunkStages, kPX,
+                           CU_TENSOR_MAP_SWIZZLE_128B))
     return BNN_OK;
   int* pop = nullptr;
   BNN_TRY(bnn::scratch_alloc(reinterpret_cast<void**>(&pop), static_cast<size_t>(m + n) * sizeof(int), s));
@@ -913,7 +976,7 @@ bnn_status binary_gemm_tc(const uint64_t* xp, const uint64_t* wp, const float* a
   const int64_t sms = sm_count();
   const int ktiles = (kw + 1) / 2;
   if (m > 128) {
-    if (((n + 255) / 256) * ((m + 255) / 256) >= sms) {  // at least two waves of 256 x 256 pair tiles
+    if (((n + 255) / 256) * ((m + kPN - 1) / kPN) >= sms) {  // at least two waves of 256 x 224 pair tiles
       bool launched = false;
       const bnn_status st = launch_pair(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s, &launched);
       if (st != BNN_OK || launched) return st;
