@@ -499,7 +499,7 @@ def gpu_cfg4(cu, seed, P, st, s, pk, head=None, shape=None):
     """Seed 1 is the headline's own measurement; other seeds time the kernel in
     a short graph on their own operands."""
     torch, dev, lib = cu.torch, cu.device, cu.lib
-    int8 = 2.0 * pk["bf16_tflops"]
+    fp4 = 4.0 * pk["bf16_tflops"]
     if head is not None:
         ms, macs = head["kernel_ms"], head["macs"]
     else:
@@ -516,9 +516,10 @@ def gpu_cfg4(cu, seed, P, st, s, pk, head=None, shape=None):
         del d, o
     return dict(value=macs / (ms * 1e-3) / 1e9, unit="GMAC/s", ms_kernel=ms, macs=macs,
                 shape=list(shape) if shape else [8192, 8192, 8192],
-                roofline=roofline("tensor", 2 * macs / (ms * 1e-3) / 1e12, int8, "TOP/s",
-                                  "binary_gemm_pair_kernel (persistent CTA pairs, 256x256 tiles)",
-                                  f"int8 dense = 2 x bf16 {pk['bf16_tflops']} TFLOP/s ({pk['src']})",
+                roofline=roofline("tensor", 2 * macs / (ms * 1e-3) / 1e12, fp4, "TOP/s",
+                                  "binary_gemm_pair_kernel (persistent CTA pairs, 256x224 tiles, tcgen05 kind::mxf4)",
+                                  f"fp4 dense = 4 x bf16 {pk['bf16_tflops']} TFLOP/s ({pk['src']}; nominal fp4:bf16 "
+                                  f"= 9:2.25 PFLOP/s)",
                                   None if shape else
                                   traffic_for("binary_gemm_pair_m8192", "ternary_neural_net_b200/csrc/binary_gemm_tc.cu")))
 
@@ -1046,7 +1047,7 @@ def main(argv=None):
 
     ms_step = head["ms_per_step"]
     value = job_throughput(head["macs"], N, ms_step) / 1e9
-    int8_peak = 2.0 * peaks["bf16_tflops"]                     # TOP/s (1 MAC = 2 ops)
+    fp4_peak = 4.0 * peaks["bf16_tflops"]                      # TOP/s (1 MAC = 2 ops)
     achieved = 2 * head["macs"] / (head["kernel_ms"] * 1e-3) / 1e12
     max_mhz = head["clocks"]["sm_max_mhz"] or peaks.get("sm_max_mhz", 1965.0)
     popc_peak = sms * POPC32_PER_CLK_PER_SM * 32 * max_mhz * 1e6 / 1e12   # TMAC/s at the max clock
@@ -1062,19 +1063,21 @@ def main(argv=None):
                          f"512 MiB of outputs, so every step starts cold",
                    "parallelism": f"replicas x{N} (independent problems per GPU)"},
         "roofline": {"bound": "tensor",
-                     "kernel": "binary_gemm_pair_kernel (bnn_binary_gemm AUTO at two waves of 256x256 CTA-pair "
-                               "tiles or more): persistent 2-CTA clusters, TMA-fed packed chunks -> 0/1 bytes in "
-                               "swizzled smem by four producer groups, tcgen05.mma.cta_group::2 kind::i8 into a "
-                               "double-buffered tensor-memory accumulator, epilogue warps overlapping the next tile "
-                               "(+ row_popcount_kernel, ~1% of the step)",
-                     "achieved": achieved, "peak": int8_peak, "unit": "TOP/s", "frac": achieved / int8_peak,
+                     "kernel": "binary_gemm_pair_kernel (bnn_binary_gemm AUTO at two waves of 256x224 CTA-pair "
+                               "tiles or more): persistent 2-CTA clusters, TMA-fed packed chunks -> e2m1 nibbles "
+                               "(1.0 or 0) in swizzled smem by four producer groups, "
+                               "tcgen05.mma.cta_group::2.kind::mxf4.block_scale (unit scale factors; the AND count "
+                               "is exact in the float32 accumulator) into a double-buffered tensor-memory "
+                               "accumulator, eight epilogue warps overlapping the next tile (+ row_popcount_kernel, "
+                               "~1% of the step)",
+                     "achieved": achieved, "peak": fp4_peak, "unit": "TOP/s", "frac": achieved / fp4_peak,
                      "achieved_basis": "2 ops x M*N*K per launch / the timed region's duration / K (the step is "
                                        "this one kernel; CUDA events on the launching stream)",
                      "kernel_ms": head["kernel_ms"], "kernel_ms_events": head["kernel_ms_events"],
                      "traffic": traffic_for("binary_gemm_pair_m8192", "ternary_neural_net_b200/csrc/binary_gemm_tc.cu"),
-                     "peak_basis": f"int8 dense tensor peak = bf16 {peaks['bf16_tflops']} TFLOP/s x 2 (nominal "
-                                   f"int8:bf16 ratio 4.5:2.25 PFLOP/s), {peak_src} (burst figure: a kernel timed "
-                                   f"alone)"},
+                     "peak_basis": f"fp4 dense tensor peak (the MMA kind the kernel runs) = bf16 "
+                                   f"{peaks['bf16_tflops']} TFLOP/s x 4 (nominal fp4:bf16 ratio 9:2.25 PFLOP/s), "
+                                   f"{peak_src} (burst figure: a kernel timed alone)"},
         "roofline_popc": {"bound": "alu", "kernel": "binary_gemm_tiled_kernel (bnn_binary_gemm_algo POPC)",
                           "achieved": popc_ach, "peak": popc_peak, "unit": "TMAC/s", "frac": popc_ach / popc_peak,
                           "ms": head["popc_ms"], "clocks": head["popc_clocks"],

@@ -543,6 +543,7 @@ constexpr int kQEpiBar = 2 + kQG;                               // named barrier
 static_assert(kPX % 8 == 0 && kPN % 32 == 0 && kPN % 16 == 0 && kPN <= 256, "UMMA N and the epilogue's column blocks");
 static_assert(kQStageBytes % 1024 == 0 && kQChunkBytes % 1024 == 0, "128-byte swizzle atoms stay 1024-byte aligned");
 static_assert(kQSfCol + 64 <= kQTmemCols, "scale-factor columns");
+static_assert(kQS > kQG, "the four groups expand four stages of a chunk at once: one buffer each, and one ahead");
 
 // 32 bits of a packed row as one 16-byte unit of e2m1 nibbles (0 or 2 = 1.0):
 // word s of the unit holds bits s, s + 4, ..., s + 28 of hw (nibble j = bit
