@@ -293,7 +293,7 @@ def run_headline(cu: Cuda, args, dist: Dist):
     torch.cuda.synchronize(dev)
     dist.barrier(dev)
     torch.cuda.synchronize(dev)
-    with ClockSampler(dev.index) as clocks:
+    with ClockSampler(dev.index, 0.0005) as clocks:  # every 0.5 ms: several samples in a region of K steps
         t0.record(cu.stream)
         g.replay()
         t1.record(cu.stream)
