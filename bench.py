@@ -448,13 +448,14 @@ def gpu_cfg2(cu, seed, P, st, s, pk):
                                                                P(D[i % R]), P(O[i % R]), 2, s), 100, st)
     popc_ms = graph_time(cu, lambda i: lib.bnn_binary_gemm_algo(P(XP[i % R]), P(WP[i % R]), P(al), m, n, k,
                                                                 P(D[i % R]), P(O[i % R]), 1, s), 50, st)
-    int8 = 2.0 * pk["bf16_tflops"]
+    fp4 = 4.0 * pk["bf16_tflops"]
     return dict(value=macs / (step_ms * 1e-3) / 1e9, unit="GMAC/s", us_step=step_ms * 1e3, us_gemm=gemm_ms * 1e3,
                 us_pack=pack_ms * 1e3, us_gemm_mma_s8=mma_ms * 1e3, us_gemm_popc=popc_ms * 1e3, macs=macs,
                 roofline=roofline(
-                    "tensor", 2 * macs / (gemm_ms * 1e-3) / 1e12, int8, "TOP/s",
-                    "binary_gemm_tc_kernel (AUTO for m >= 64): tcgen05.mma kind::i8 into tensor memory",
-                    f"int8 dense = 2 x bf16 {pk['bf16_tflops']} TFLOP/s ({pk['src']}; nominal int8:bf16 = 2)",
+                    "tensor", 2 * macs / (gemm_ms * 1e-3) / 1e12, fp4, "TOP/s",
+                    "binary_gemm_tc_kernel (AUTO for m >= 64): bits as e2m1 nibbles, tcgen05.mma kind::mxf4 "
+                    "(unit block scales) into tensor memory",
+                    f"fp4 dense = 4 x bf16 {pk['bf16_tflops']} TFLOP/s ({pk['src']}; nominal fp4:bf16 = 9:2.25)",
                     traffic_for("binary_gemm_tc_128x2", "ternary_neural_net_b200/csrc/binary_gemm_tc.cu"),
                     achieved_basis="kernel alone, back to back in a CUDA graph (inside the step: pack + GEMM)"),
                 rotation=R)

@@ -5,33 +5,41 @@
 // for the bits of x and w, popcount(x XOR w) = pa + pb - 2 popcount(a AND b),
 // so <x,w> = k - 2 pa - 2 pb + 4 popcount(a AND b), where pa and pb are the
 // row popcounts.  popcount(a AND b) is the dot product of the rows' bits as
-// 0/1 bytes, which an int8 MMA sums exactly into int32.  Pad bits are 0 in
-// both rows and so add nothing to any of the three counts.
+// 0/1 values.  Here each bit becomes an e2m1 float, 1.0 (code 0b0010) or 0.0,
+// and the tensor cores run tcgen05.mma.kind::mxf4.block_scale.block32 with
+// every ue8m0 scale factor 127 (2^0): the products are exactly 0 or 1 and the
+// float32 accumulator holds the count exactly (every integer up to 2^24 is a
+// float32, and the ABI bounds k by 2^24).  Pad bits are 0 in both rows and so
+// add nothing to any of the three counts.
 //
-// Tile: UMMA M = 128 weight rows (operand A) x N = BN activation rows (operand
-// B), K in stages of 128 bits.  Roles inside a CTA:
+// One-SM kernel.  Tile: UMMA M = 128 weight rows (operand A) x N = BN
+// activation rows (operand B), K in stages of 256 bits (4 words, 128 bytes of
+// nibbles per row).  Tensor memory holds the accumulator (BN columns) and the
+// scale factors (the next BN columns, 127 in every byte).  Roles inside a CTA:
 //   - a TMA thread (when every row is 16-byte aligned): copies the packed words
-//     of 4 stages of all the tile's rows (a 64-byte-swizzled box of each
+//     of 2 stages of all the tile's rows (a 64-byte-swizzled box of each
 //     operand) into a double-buffered chunk ring, signalling an mbarrier with
 //     the byte count;
 //   - producer threads, two per row of the stacked (weight, activation) tile,
-//     each owning one 64-bit word of the row per stage: read it (from the
+//     each owning two 64-bit words of the row per stage: read them (from the
 //     chunk ring, or without TMA straight from global memory, prefetched kPre
-//     stages ahead in registers), count its bits, and write its 64 0/1 bytes
-//     (per 4 bytes a shift and an AND) in the 128-byte-swizzled K-major layout
-//     the tensor core reads, then arrive on the stage's "full" mbarrier;
-//   - one MMA thread: waits for "full", issues 4 tcgen05.mma.kind::i8 (K = 32)
-//     into the int32 accumulator in tensor memory and commits to the stage's
-//     "empty" mbarrier, which the producers wait on before refilling it;
+//     stages ahead in registers), count their bits, and write their 64 bytes
+//     of nibbles (per 4 bytes a shift and an AND) in the 128-byte-swizzled
+//     K-major layout the tensor core reads, then arrive on the stage's "full"
+//     mbarrier;
+//   - one MMA thread: waits for "full", issues 4 MMAs (K = 64) into the float32
+//     accumulator in tensor memory and commits to the stage's "empty"
+//     mbarrier, which the producers wait on before refilling it;
 //   - the epilogue (warps 0-7; warp w reads tensor-memory lanes 32(w%4).. and
-//     half w/4 of the columns): tcgen05.ld, the popcount correction, alpha,
-//     the optional bias, and stores in which the 32 lanes of a warp write 32
-//     consecutive weight columns of one output row.  Those 32 columns are also
-//     one 32-bit half of a word of the next layer's packed input, so the
-//     optional sign pack of the layer output is one __ballot_sync per row.
-// Any bijection between the 128 bits and the 128 k-slots of a stage gives the
-// same sum when both operands use it; here byte j of word s of 16-byte chunk
-// 2h+q holds bit 32h + 8j + 4q + s.
+//     half w/4 of the columns): tcgen05.ld, the count as an integer, the
+//     popcount correction, alpha, the optional bias, and stores in which the
+//     32 lanes of a warp write 32 consecutive weight columns of one output
+//     row.  Those 32 columns are also one 32-bit half of a word of the next
+//     layer's packed input, so the optional sign pack of the layer output is
+//     one __ballot_sync per row.
+// Any bijection between the 256 bits and the 256 k-slots of a stage gives the
+// same sum when both operands use it; here nibble j of word s of the 16-byte
+// unit built from 32-bit half h holds bit 32h + 4j + s.
 //
 // Split K: a cluster of KS CTAs shares one output tile, each taking a
 // contiguous share of the stages.  Each CTA turns its accumulator into its
@@ -75,8 +83,11 @@ using bnn::tc::tmem_ld32;
 using bnn::tc::tmem_wait_ld;
 
 constexpr int kTm = 128;                   // weight rows per tile (UMMA M)
-constexpr int kPre = 8;                    // without TMA: stages of words prefetched in registers
-constexpr int kChunkStages = 4;            // with TMA: stages per packed chunk (64 bytes of every row)
+constexpr int kPre = 4;                    // without TMA: stages of words prefetched in registers
+constexpr int kChunkStages = 4;            // CTA pairs: stages per packed chunk (128 bytes of every row)
+constexpr int kTcWords = 4;                // one-SM kernel: packed words per row and stage (256 bits of k)
+constexpr int kTcChunkStages = 2;          // one-SM kernel with TMA: stages per packed chunk (64 bytes of every row)
+static_assert(BNN_MAX_K_BINARY <= (1 << 24), "AND counts accumulated in float32 stay exact integers");
 
 // WIDE (64- and 128-row tiles): one CTA per SM with a deeper ring of expanded
 // stages; otherwise 64-row tiles keep 96 KB so that two CTAs share an SM.
@@ -85,7 +96,7 @@ struct TcCfg {
   static_assert(!WIDE || BN <= 128, "deep rings for the 64- and 128-row tiles");
   static constexpr int kRows = kTm + BN;                             // stacked weight + activation rows
   static constexpr uint32_t kStageBytes = kRows * 128u;              // one expanded stage
-  static constexpr uint32_t kChunkBytes = kRows * 16u * kChunkStages; // one packed chunk (2 words per stage)
+  static constexpr uint32_t kChunkBytes = kRows * 8u * kTcWords * kTcChunkStages;  // one packed chunk (64 B a row)
   static constexpr int S = !WIDE ? (TMA ? 3 : 4)                     // expanded stages
                                  : (BN == 64 ? (TMA ? 6 : 8) : (TMA ? 5 : 6));
   static constexpr int P = TMA ? 2 : 0;                              // packed chunks
@@ -95,23 +106,25 @@ struct TcCfg {
   static constexpr int kMinBlocks = (BN <= 64 && !WIDE) ? 2 : 1;
 };
 
-// 4 bytes per 16-byte chunk word: byte j of word s holds bit 8j + s of hw
-__device__ __forceinline__ void expand_word(uint8_t* dst_row, uint32_t swz, int part, uint64_t cw) {
+// 32 bits of a packed row as one 16-byte unit of e2m1 nibbles (0 or 2 = 1.0):
+// word s of the unit holds bits s, s + 4, ..., s + 28 of hw (nibble j = bit
+// 4j + s), the same permutation of k in both operands
+__device__ __forceinline__ uint4 nibbles_of(uint32_t hw) {
+  uint4 v;
+  v.x = (hw << 1) & 0x22222222u;
+  v.y = hw & 0x22222222u;
+  v.z = (hw >> 1) & 0x22222222u;
+  v.w = (hw >> 2) & 0x22222222u;
+  return v;
+}
+
+// one-SM kernel: a thread's two words of a stage (v: four 32-bit halves) ->
+// units 4 part .. 4 part + 3 of its row of the expanded stage (128-byte swizzle)
+__device__ __forceinline__ void expand_pair(uint8_t* dst_row, uint32_t swz, int part, const uint4& v) {
+  const uint32_t h[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-  for (int hh = 0; hh < 2; ++hh) {
-    const int h = 2 * part + hh;  // half-word of the stage's 128 bits
-    const uint32_t hw = static_cast<uint32_t>(cw >> (32 * hh));
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      uint4 v;
-      v.x = (hw >> (4 * q + 0)) & 0x01010101u;
-      v.y = (hw >> (4 * q + 1)) & 0x01010101u;
-      v.z = (hw >> (4 * q + 2)) & 0x01010101u;
-      v.w = (hw >> (4 * q + 3)) & 0x01010101u;
-      const uint32_t chunk = static_cast<uint32_t>(2 * h + q);
-      *reinterpret_cast<uint4*>(dst_row + ((chunk ^ swz) << 4)) = v;
-    }
-  }
+  for (int q = 0; q < 4; ++q)
+    *reinterpret_cast<uint4*>(dst_row + ((static_cast<uint32_t>(4 * part + q) ^ swz) << 4)) = nibbles_of(h[q]);
 }
 
 // grid: x = KS * (weight tiles of 128 rows), y = activation tiles of BN rows;
@@ -155,7 +168,7 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
   const int rank = KS > 1 ? static_cast<int>(blockIdx.x % KS) : 0;
   const int64_t j0 = static_cast<int64_t>(blockIdx.x / KS) * kTm;  // first weight row
   const int64_t i0 = static_cast<int64_t>(blockIdx.y) * BN;        // first activation row
-  const int ktiles = (kw + 1) / 2;                                 // 2 words (128 bits) per stage
+  const int ktiles = (kw + kTcWords - 1) / kTcWords;               // 4 words (256 bits) per stage
   const int share = (ktiles + KS - 1) / KS;
   const int kb = rank * share < ktiles ? rank * share : ktiles;
   const int ke = kb + share < ktiles ? kb + share : ktiles;
@@ -184,13 +197,26 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
   }
   if (warp == kMmaWarp) {  // the MMA warp owns the tensor memory
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(&tmem_holder)),
-                 "r"(BN));
+                 "r"(2 * BN));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::);
   }
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+  // accumulator: columns [0, BN); the MMA's scale factors: 127 (2^0) in every
+  // byte of columns [BN, 2 BN), written by warps 0-3 before the first MMA
   const uint32_t tmem = tmem_holder;
+  if (warp < 4) {
+    const uint32_t lanes = static_cast<uint32_t>(32 * warp) << 16;
+    for (uint32_t c = BN; c < 2u * BN; c += 8)
+      asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1};\n" ::"r"(tmem + lanes + c),
+                   "r"(0x7F7F7F7Fu)
+                   : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
   bnn::pdl_trigger();
 
   if (tid < kProducers) {
@@ -203,20 +229,20 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
     int my_pop = 0;
     bool ok = true;
     if constexpr (TMA) {
-      // this thread's word of stage s of a chunk: row r2 (64 bytes), 16-byte unit
-      // s under the 64-byte swizzle (unit ^ bits 7-8 of the address), half `part`
-      const uint32_t rd_off = static_cast<uint32_t>(r2) * 64u + 8u * static_cast<uint32_t>(part);
+      // this thread's two words of stage s of a chunk: row r2 (64 bytes), 16-byte
+      // unit 2 s + part under the 64-byte swizzle (unit ^ bits 7-8 of the address)
+      const uint32_t rd_off = static_cast<uint32_t>(r2) * 64u;
       const uint32_t rd_swz = static_cast<uint32_t>((r2 >> 1) & 3);
       for (int j = 0; j < nst; ++j) {
-        const int c = j / kChunkStages, s = j % kChunkStages, pb = c % P;
+        const int c = j / kTcChunkStages, s = j % kTcChunkStages, pb = c % P;
         if (s == 0 && !bnn::tc::mbar_wait(smem_u32(&chunk_full[pb]), static_cast<uint32_t>((c / P) & 1), &abort_flag,
                                           &g_bnn_device_errors, wait_limit)) {
           ok = false;
           break;
         }
-        const uint64_t cw = *reinterpret_cast<const uint64_t*>(
-            chunks + pb * Cfg::kChunkBytes + rd_off + ((static_cast<uint32_t>(s) ^ rd_swz) << 4));
-        if (s == kChunkStages - 1 || j == nst - 1) mbar_arrive(smem_u32(&chunk_empty[pb]));
+        const uint4 cw = *reinterpret_cast<const uint4*>(
+            chunks + pb * Cfg::kChunkBytes + rd_off + ((static_cast<uint32_t>(2 * s + part) ^ rd_swz) << 4));
+        if (s == kTcChunkStages - 1 || j == nst - 1) mbar_arrive(smem_u32(&chunk_empty[pb]));
         const int b = j % S;
         // refill only after the tensor core has read the previous fill of this buffer
         if (j >= S && !bnn::tc::mbar_wait(smem_u32(&empty_bar[b]), static_cast<uint32_t>((j / S + 1) & 1), &abort_flag,
@@ -224,21 +250,26 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
           ok = false;
           break;
         }
-        my_pop += __popcll(cw);
-        expand_word(smem + b * kStageBytes + row_off, swz, part, cw);
+        my_pop += __popc(cw.x) + __popc(cw.y) + __popc(cw.z) + __popc(cw.w);
+        expand_pair(smem + b * kStageBytes + row_off, swz, part, cw);
         asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
         mbar_arrive(smem_u32(&full_bar[b]));
       }
     } else {
       const int64_t grow = is_w ? j0 + row : i0 + row;
       const bool live = grow < (is_w ? n : m);
-      const uint64_t* src = (is_w ? wp : xp) + (live ? grow : 0) * static_cast<int64_t>(kw) + part;
+      const uint64_t* src = (is_w ? wp : xp) + (live ? grow : 0) * static_cast<int64_t>(kw) + 2 * part;
       if (!is_w) bnn::pdl_wait();  // the activations may come from the preceding kernel
-      auto fetch = [&](int jj) -> uint64_t {
-        const int w = 2 * (kb + jj) + part;
-        return (live && jj < nst && w < kw) ? __ldg(src + 2 * (kb + jj)) : 0ull;
+      // this thread's two words of stage jj (words 4 (kb + jj) + 2 part and the next; 0 past the row)
+      auto fetch = [&](int jj) -> uint4 {
+        const int w = kTcWords * (kb + jj) + 2 * part;
+        const bool in = live && jj < nst;
+        const uint64_t a = (in && w < kw) ? __ldg(src + kTcWords * (kb + jj)) : 0ull;
+        const uint64_t b2 = (in && w + 1 < kw) ? __ldg(src + kTcWords * (kb + jj) + 1) : 0ull;
+        return make_uint4(static_cast<uint32_t>(a), static_cast<uint32_t>(a >> 32), static_cast<uint32_t>(b2),
+                          static_cast<uint32_t>(b2 >> 32));
       };
-      uint64_t ring[kPre];
+      uint4 ring[kPre];
 #pragma unroll
       for (int u = 0; u < kPre; ++u) ring[u] = fetch(u);
       for (int js = 0; js < nst && ok; js += kPre) {
@@ -252,10 +283,10 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
             ok = false;
             break;
           }
-          const uint64_t cw = ring[u];
+          const uint4 cw = ring[u];
           ring[u] = fetch(j + kPre);
-          my_pop += __popcll(cw);
-          expand_word(smem + b * kStageBytes + row_off, swz, part, cw);
+          my_pop += __popc(cw.x) + __popc(cw.y) + __popc(cw.z) + __popc(cw.w);
+          expand_pair(smem + b * kStageBytes + row_off, swz, part, cw);
           asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
           mbar_arrive(smem_u32(&full_bar[b]));
         }
@@ -264,10 +295,11 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
     atomicAdd(is_w ? &pop_w[row] : &pop_x[row], my_pop);
   } else if (tid == kMmaWarp * 32) {
     // ------------------------------------------------------------ MMA issue
-    // instruction descriptor: D s32, A and B 8-bit integers (0/1 bytes read
-    // the same signed or unsigned), both K-major, N = BN, M = 128
-    const uint32_t idesc = (2u << 4) | (1u << 7) | (1u << 10) | ((static_cast<uint32_t>(BN) >> 3) << 17) |
+    // instruction descriptor: D f32; A and B e2m1 (format 1), K-major; ue8m0
+    // scale factors (bit 23, every one 127 = 2^0); N = BN, M = 128; dense K = 64
+    const uint32_t idesc = (1u << 7) | (1u << 10) | ((static_cast<uint32_t>(BN) >> 3) << 17) | (1u << 23) |
                            ((static_cast<uint32_t>(kTm) >> 4) << 24);
+    const uint32_t sfa = tmem + static_cast<uint32_t>(BN), sfb = tmem + static_cast<uint32_t>(BN + BN / 2);
     for (int j = 0; j < nst; ++j) {
       const int b = j % S;
       if (!bnn::tc::mbar_wait(smem_u32(&full_bar[b]), static_cast<uint32_t>((j / S) & 1), &abort_flag,
@@ -281,8 +313,10 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
         const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
         asm volatile(
             "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
-            "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem),
-            "l"(ad + static_cast<uint64_t>(2 * kk)), "l"(bd + static_cast<uint64_t>(2 * kk)), "r"(idesc), "r"(acc));
+            "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n}\n" ::"r"(
+                tmem),
+            "l"(ad + static_cast<uint64_t>(2 * kk)), "l"(bd + static_cast<uint64_t>(2 * kk)), "r"(idesc), "r"(acc),
+            "r"(sfa), "r"(sfb));
       }
       asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
                        smem_u32(&empty_bar[b]))
@@ -294,9 +328,10 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
                  : "memory");
   } else if (TMA && tid == kTmaWarp * 32) {
     // ------------------------------------------------------------ TMA copies
-    const int nch = (nst + kChunkStages - 1) / kChunkStages;
+    const int nch = (nst + kTcChunkStages - 1) / kTcChunkStages;
     const int pre = nch < P ? nch : P;
-    auto chunk_x = [&](int c) { return 2 * kb + 2 * kChunkStages * c; };  // first word (even: 16-byte aligned)
+    // first word of chunk c (even: 16-byte aligned)
+    auto chunk_x = [&](int c) { return kTcWords * kb + kTcWords * kTcChunkStages * c; };
     // the weights do not depend on the preceding kernel: their first chunks
     // are copied before waiting for it, the activations after
     for (int c = 0; c < pre; ++c) {
@@ -306,7 +341,7 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
     }
     bnn::pdl_wait();
     for (int c = 0; c < pre; ++c)
-      tma_load_2d(smem_u32(chunks + c * Cfg::kChunkBytes) + kTm * 16u * kChunkStages, &tmap_x, chunk_x(c),
+      tma_load_2d(smem_u32(chunks + c * Cfg::kChunkBytes) + kTm * 64u, &tmap_x, chunk_x(c),
                   static_cast<int>(i0), smem_u32(&chunk_full[c]));
     int issued = pre;
     for (int c = pre; c < nch; ++c) {
@@ -318,7 +353,7 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
       const uint32_t bar = smem_u32(&chunk_full[pb]);
       mbar_expect_tx(bar, Cfg::kChunkBytes);
       tma_load_2d(dst, &tmap_w, chunk_x(c), static_cast<int>(j0), bar);
-      tma_load_2d(dst + kTm * 16u * kChunkStages, &tmap_x, chunk_x(c), static_cast<int>(i0), bar);
+      tma_load_2d(dst + kTm * 64u, &tmap_x, chunk_x(c), static_cast<int>(i0), bar);
       issued = c + 1;
     }
     // the CTA must not retire with copies in flight (producers that aborted no
@@ -344,11 +379,14 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
   const int erow = 32 * (warp & 3) + (tid & 31);
   const int ecol0 = (warp >> 2) * (BN / 2);
   const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
-  // the tile's accumulated popc(a AND b) for 16 columns from c0
+  // the tile's accumulated popc(a AND b) for 16 columns from c0 (the float32
+  // counts, exact integers, converted)
   auto load16 = [&](int c0, uint32_t (&r)[16]) {
     if (nst > 0) {
       tmem_ld16(taddr + static_cast<uint32_t>(c0), r);
       tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 16; ++c) r[c] = static_cast<uint32_t>(static_cast<int32_t>(__uint_as_float(r[c])));
     } else {
 #pragma unroll
       for (int c = 0; c < 16; ++c) r[c] = 0u;
@@ -469,7 +507,7 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
   __syncthreads();
   if (warp == kMmaWarp)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(BN));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(2 * BN));
 }
 
 // ---------------------------------------------------------------------------
@@ -479,9 +517,9 @@ binary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_c
 // becomes an e2m1 float, 1.0 (code 0b0010) or 0.0, and the pair runs
 // tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 with every ue8m0
 // scale factor 127 (2^0): the products are exactly 0 or 1 and the float32
-// accumulator holds the count exactly while it stays below 2^24 (k < 2^24,
-// checked on the host).  Per instruction K = 64 at twice the int8 rate, and
-// an expanded bit takes half a byte.
+// accumulator holds the count exactly (every integer up to 2^24 is a float32,
+// and the ABI bounds k by BNN_MAX_K_BINARY = 2^24).  Per instruction K = 64
+// at twice the int8 rate, and an expanded bit takes half a byte.
 //
 // A cluster of two CTAs computes tiles of 256 weight rows x kPN = 224
 // activation rows (UMMA M = 256, N = 224): CTA q of the pair holds weight
@@ -544,18 +582,6 @@ static_assert(kPX % 8 == 0 && kPN % 32 == 0 && kPN % 16 == 0 && kPN <= 256, "UMM
 static_assert(kQStageBytes % 1024 == 0 && kQChunkBytes % 1024 == 0, "128-byte swizzle atoms stay 1024-byte aligned");
 static_assert(kQSfCol + 64 <= kQTmemCols, "scale-factor columns");
 static_assert(kQS > kQG, "the four groups expand four stages of a chunk at once: one buffer each, and one ahead");
-
-// 32 bits of a packed row as one 16-byte unit of e2m1 nibbles (0 or 2 = 1.0):
-// word s of the unit holds bits s, s + 4, ..., s + 28 of hw (nibble j = bit
-// 4j + s), the same permutation of k in both operands
-__device__ __forceinline__ uint4 nibbles_of(uint32_t hw) {
-  uint4 v;
-  v.x = (hw << 1) & 0x22222222u;
-  v.y = hw & 0x22222222u;
-  v.z = (hw >> 1) & 0x22222222u;
-  v.w = (hw >> 2) & 0x22222222u;
-  return v;
-}
 
 __global__ void __launch_bounds__(kQThreads, 1)
 binary_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
@@ -800,7 +826,7 @@ binary_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
         uint32_t* np = pack ? next + (i0 + c0) * next_w32 + half : nullptr;
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          // the AND count: an integer below 2^24, exact in the float32 accumulator
+          // the AND count: an integer of at most 2^24, exact in the float32 accumulator
           const int32_t dv = base - 2 * pop_xs[c0 + c] + 4 * static_cast<int32_t>(__uint_as_float(r[c]));
           const float y0 = __fmul_rn(a_j, static_cast<float>(dv));
           const float y = bias ? __fadd_rn(y0, b_j) : y0;
@@ -887,10 +913,10 @@ bnn_status launch_pair(const uint64_t* xp, const uint64_t* wp, const float* alph
                        bool* launched) {
   *launched = false;
   const int64_t ntiles = ((n + 255) / 256) * ((m + kPN - 1) / kPN);
-  // TMA rows (16-byte aligned: even kw, aligned bases), int32 coordinates, and
-  // AND counts (at most k) exact in float32
+  // TMA rows (16-byte aligned: even kw, aligned bases) and int32 coordinates
+  // (the AND counts, at most k <= BNN_MAX_K_BINARY = 2^24, are exact in float32)
   if (kw <= 0 || kw % 2 != 0 || !bnn::aligned(xp, 16) || !bnn::aligned(wp, 16) || n >= (1LL << 31) ||
-      m >= (1LL << 31) || k >= (1 << 24))
+      m >= (1LL << 31))
     return BNN_OK;
   const int clusters = pair_clusters();
   if (clusters <= 0) return BNN_OK;
@@ -938,11 +964,11 @@ bnn_status launch_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha,
              m < (1LL << 31);
   if (tma)
     tma = bnn::encode_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT64, wp, static_cast<uint64_t>(kw),
-                              static_cast<uint64_t>(n), static_cast<uint64_t>(kw) * 8u, 2 * kChunkStages, kTm,
-                              CU_TENSOR_MAP_SWIZZLE_64B) &&
+                              static_cast<uint64_t>(n), static_cast<uint64_t>(kw) * 8u, kTcWords * kTcChunkStages,
+                              kTm, CU_TENSOR_MAP_SWIZZLE_64B) &&
           bnn::encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT64, xp, static_cast<uint64_t>(kw),
-                              static_cast<uint64_t>(m), static_cast<uint64_t>(kw) * 8u, 2 * kChunkStages, BN,
-                              CU_TENSOR_MAP_SWIZZLE_64B);
+                              static_cast<uint64_t>(m), static_cast<uint64_t>(kw) * 8u, kTcWords * kTcChunkStages,
+                              BN, CU_TENSOR_MAP_SWIZZLE_64B);
   if (!tma) memset(&tw, 0, sizeof(tw)), memset(&tx, 0, sizeof(tx));
   const size_t smem =
       static_cast<size_t>(tma ? TcCfg<BN, true, WIDE>::kSmem : TcCfg<BN, false, WIDE>::kSmem) + 1024;
