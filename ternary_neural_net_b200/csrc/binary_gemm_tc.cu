@@ -988,15 +988,18 @@ bnn_status launch_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha,
 
 namespace bnn {
 
-// Tensor-core (tcgen05) binary GEMM; tiles chosen from a sweep over M = 64 ..
-// 8192 at N = K = 4096 and 8192.  m <= 128: 64-row activation tiles.  Larger
-// m: two-SM 256 x 256 tiles when they make two waves of CTA pairs or more
-// (16-byte aligned rows), else 256-row tiles on one SM (the widest one-SM MMA,
-// the fewest re-expansions of the operands) once they make three quarters of
-// a wave, otherwise 128-row tiles.  When the
-// tiles leave SMs idle a cluster of 4 or 2 CTAs splits each tile's stages (at
-// least 4 stages per CTA).  CTAs that fit one per SM take the deep ring (more
-// stages in flight); otherwise 64-row-tile CTAs pair up on an SM.
+// Tensor-core (tcgen05) binary GEMM.  m <= 128: 64-row activation tiles (from
+// a sweep over M = 64 .. 8192 at N = K = 4096 and 8192); when the tiles leave
+// SMs idle a cluster of 4 or 2 CTAs splits each tile's stages (at least 4
+// 128-bit stages' worth per CTA).  Larger m: two-SM 256 x 224 tiles when they
+// make two waves of CTA pairs or more (16-byte aligned rows); else the one-SM
+// plan (activation tile 128 or 256 rows, cluster split 1 or 2) of least
+// modelled time: waves x 256-bit stages per CTA x the rows a CTA expands per
+// stage (128 + BN), at ~3.3 ns per row-stage, plus ~3 us per 128 activation
+// rows of a split's exchange (fitted to 256..1024 x 4096 x 4096 and 256 x 11008
+// x 4096, where it picks the measured best).  CTAs that fit one per SM take
+// the deep ring (more stages in flight); otherwise 64-row-tile CTAs pair up on
+// an SM.
 bnn_status binary_gemm_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha, const float* bias, int64_t m,
                           int64_t n, int k, int kw, int32_t* dots, float* out, uint64_t* next, cudaStream_t s) {
   const int64_t wt = (n + kTm - 1) / kTm;
@@ -1008,13 +1011,33 @@ bnn_status binary_gemm_tc(const uint64_t* xp, const uint64_t* wp, const float* a
       const bnn_status st = launch_pair(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s, &launched);
       if (st != BNN_OK || launched) return st;
     }
-    if (4 * wt * ((m + 255) / 256) >= 3 * sms)
-      return launch_tc<256, 1>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
-    const int64_t t128 = wt * ((m + 127) / 128);
-    if (t128 * 2 <= sms && ktiles >= 8)
-      return launch_tc<128, 2, true>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
-    if (t128 <= sms) return launch_tc<128, 1, true>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
-    return launch_tc<128, 1, false>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
+    const int64_t st = (kw + kTcWords - 1) / kTcWords;  // 256-bit stages
+    auto modelled_us = [&](int bn, int ks) -> double {
+      const int64_t ctas = ks * wt * ((m + bn - 1) / bn);
+      const int64_t waves = (ctas + sms - 1) / sms, per = (st + ks - 1) / ks;
+      return static_cast<double>(waves * per * (kTm + bn)) * 3.3e-3 + (ks > 1 ? 3.0 * bn / 128.0 : 0.0);
+    };
+    int bn = 256, ks = 1;
+    double best = modelled_us(256, 1);
+    const int plans[3][2] = {{128, 1}, {128, 2}, {256, 2}};
+    for (const auto& pl : plans) {
+      if (pl[1] > 1 && st < 4 * pl[1]) continue;  // at least 4 stages per CTA of a split
+      const double us = modelled_us(pl[0], pl[1]);
+      if (us < best) {
+        best = us;
+        bn = pl[0];
+        ks = pl[1];
+      }
+    }
+    const int64_t ctas = ks * wt * ((m + bn - 1) / bn);
+    if (bn == 256)
+      return ks == 2 ? launch_tc<256, 2>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s)
+                     : launch_tc<256, 1>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
+    if (ks == 2)
+      return ctas <= sms ? launch_tc<128, 2, true>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s)
+                         : launch_tc<128, 2, false>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
+    return ctas <= sms ? launch_tc<128, 1, true>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s)
+                       : launch_tc<128, 1, false>(xp, wp, alpha, bias, m, n, k, kw, dots, out, next, s);
   }
   const int64_t tiles = wt * ((m + 63) / 64);
   if (tiles * 4 <= sms && ktiles >= 16)

@@ -112,6 +112,27 @@ def test_tc_tile_configs(bnn, m, n, k):
     _gemm_case(bnn, m, n, k, seed=5 * m + n + 3 * k, algos=(3,))
 
 
+@pytest.mark.parametrize("m,n,k", [(512, 2431, 8192), (1024, 4096, 1024), (256, 11008, 4096)])
+def test_one_sm_plans_sampled(bnn, m, n, k):
+    """Shapes where the one-SM plan model picks the split 256-row tiles (512 x
+    2431 x 8192: 2-CTA clusters of 256-row activation tiles), one wave of
+    256-row tiles, and 256-row tiles over an FFN-sized weight: every output
+    against the popcount properties (|dot| <= k, dot = k mod 2), the rows at
+    the tile and cluster boundaries bit-exact against the oracle."""
+    xp = synth.fair_coin_words(m + 7, 1, m, k)
+    wp = synth.fair_coin_words(m + 7, 2, n, k)
+    alpha = synth.uniform_f32(m + 7, 3, (n,), 0.5, 1.5)
+    dots, out = bnn.bnn_binary_gemm(to_dev_u64(xp), to_dev_u64(wp), to_dev_f32(alpha), k, algo=3)
+    d = dots.cpu().numpy()
+    assert np.all(np.abs(d) <= k) and np.all((d - k) % 2 == 0)
+    rows = np.array(sorted(r for r in {0, 127, 128, 255, 256, m // 2, m - 1} if r < m), dtype=np.int64)
+    rr = np.repeat(rows, n)
+    cc = np.tile(np.arange(n, dtype=np.int64), rows.size)
+    sd, so = oracle.binary_gemm_sampled(xp, wp, alpha, m, n, k, rr, cc)
+    assert_bits_equal(d[rr, cc], sd, f"dots {m}x{n}x{k} sampled rows")
+    assert_bits_equal(out.cpu().numpy()[rr, cc], so, f"out {m}x{n}x{k} sampled rows")
+
+
 @pytest.mark.parametrize("m,n,k", [(1, 100, 200), (3, 50, 640), (40, 70, 128), (200, 300, 1024)])
 def test_unaligned_operands_use_the_8_byte_path(bnn, m, n, k):
     _gemm_case(bnn, m, n, k, seed=99 + m, offset_words=1)
