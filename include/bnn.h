@@ -122,10 +122,11 @@ typedef enum {
                           register-tiled GEMM otherwise) */
   BNN_ALGO_MMA_S8 = 2, /* packed bits expanded in registers to 0/-1 int8 fragments of
                           m16n8k32 s8 mma.sync; popc(a AND b) summed exactly in int32 */
-  BNN_ALGO_TC = 3      /* packed bits expanded to 0/1 bytes in shared memory; tcgen05.mma
-                          kind::i8 sums popc(a AND b) exactly into an int32 tensor-memory
-                          accumulator, and k - 2 popc(a) - 2 popc(b) + 4 popc(a AND b) is
-                          the dot */
+  BNN_ALGO_TC = 3      /* packed bits expanded to 4-bit floats (1.0 or 0) in shared memory;
+                          tcgen05.mma kind::mxf4 with unit scale factors sums popc(a AND b)
+                          exactly into a float32 tensor-memory accumulator (every count up
+                          to k <= 2^24 is a float32), and k - 2 popc(a) - 2 popc(b) +
+                          4 popc(a AND b) is the dot */
 } bnn_binary_algo;
 
 /*

@@ -87,7 +87,7 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
 }
 
-// Tensor-core (tcgen05 kind::i8) binary GEMM, in binary_gemm_tc.cu, with the
+// Tensor-core (tcgen05 kind::mxf4) binary GEMM, in binary_gemm_tc.cu, with the
 // optional layer epilogue: bias (may be null) and the sign-packed output for
 // the next layer (next, may be null; ceil(n/64) words per row).
 bnn_status binary_gemm_tc(const uint64_t* xp, const uint64_t* wp, const float* alpha, const float* bias, int64_t m,

@@ -104,7 +104,7 @@ def test_tiled_matches_oracle(bnn, m, n, k):
                                    (257, 383, 2048 * 2 + 64), (2304, 4219, 130), (600, 9000, 760), (50, 700, 2000),
                                    (64, 1000, 300), (64, 2000, 500), (200, 1000, 2048), (300, 3000, 256),
                                    (384, 6400, 128), (250, 700, 2048 + 130),
-                                   # two waves of 256 x 256 CTA-pair tiles (the two-SM kernel): ragged m and
+                                   # two waves of 256 x 224 CTA-pair tiles (the two-SM kernel): ragged m and
                                    # n, one activation tile, a single stage and several, ragged K
                                    (2304, 4219, 128), (2000, 4800, 256), (200, 38000, 128), (300, 40000, 128),
                                    (2048, 4800, 1000), (4100, 2500, 4096)])

@@ -63,7 +63,7 @@ def test_main_waits_run_out_then_a_normal_call_is_exact(bnn):
 
 
 def test_pair_kernel_waits_run_out_then_a_normal_call_is_exact(bnn):
-    # the persistent CTA-pair kernel (two waves of 256 x 256 pair tiles: m = 256, n = 148 x 256);
+    # the persistent CTA-pair kernel (two waves of 256 x 224 pair tiles: m = 256, n = 148 x 256);
     # its epilogue warps wait for a tile that never comes, up to their one-second bound
     m, n, k = 256, 148 * 256, 128
     xp = synth.fair_coin_words(4, 1, m, k)
