@@ -203,10 +203,14 @@ sparse_gemm_kernel(const uint16_t* __restrict__ x, const int64_t* __restrict__ r
 }
 
 // The layer at m = 1: x staged once per CTA in shared memory as float32 (k
-// floats, k <= 32768), so every gather is a shared-memory load.  One CTA per
-// SM takes a contiguous block of rows, in chunks of kSpChunk = 96: the chunk's
-// row_ptr values are read into shared memory once, and warp w takes rows w,
-// w + 32 and w + 64 of it.  A warp issues the loads of all its rows' first
+// floats, k <= 32768), so every gather is a shared-memory load.  Two CTAs of
+// 512 threads per SM (one where k leaves room for only one) each take a
+// contiguous block of rows, in chunks of kSpChunk = 48: the chunk's row_ptr
+// values are read into shared memory once, and warp w takes rows w, w + 16
+// and w + 32 of it.  (With two CTAs per SM, the next launch's CTAs start
+// their row_ptr and entry loads while this launch's last CTAs finish: 5.8
+// against 6.2 µs for one 1024-thread CTA per SM at 11008 x 4096, 10% of the
+// trits non-zero; four 256-thread CTAs lost on long rows.)  A warp issues the loads of all its rows' first
 // 511..512 entries at once, before the programmatic-launch wait and the
 // staging of x (each lane eight 32-bit entry pairs per row, 128-byte coalesced
 // loads from the even entry at or below the row's first), so the whole
@@ -216,9 +220,12 @@ sparse_gemm_kernel(const uint16_t* __restrict__ x, const int64_t* __restrict__ r
 // row's sum is added by a shuffle tree (a fixed order), scaled once (and
 // biased).  VEC: entries 4-byte aligned (one 32-bit load per pair), else two
 // 16-bit loads.
-constexpr int kSpThreads = 1024;
+constexpr int kSpThreads = 512;
+constexpr int kSpWarps = kSpThreads / 32;
+constexpr int kSpPerSm = 2;                     // CTAs per SM (register budget: 64 per thread)
 constexpr int kSpR = 3;                         // rows per warp and chunk
-constexpr int kSpChunk = kSpThreads / 32 * kSpR;
+constexpr int kSpChunk = kSpWarps * kSpR;
+static_assert(kSpChunk + 1 <= kSpThreads, "one thread per row_ptr value of a chunk");
 constexpr int kSpW = 8;                         // entry pairs per lane per pass
 
 // entries q, q + 1 (bits 0..15 and 16..31; q even relative to the row's pass
@@ -256,7 +263,7 @@ __device__ __forceinline__ float sp_gather(const float* xs, const uint32_t (&v)[
 }
 
 template <bool VEC>
-__global__ void __launch_bounds__(kSpThreads, 1)
+__global__ void __launch_bounds__(kSpThreads, kSpPerSm)
 sparse_gemv_smem_kernel(const uint16_t* __restrict__ x, const int64_t* __restrict__ row_ptr,
                         const uint16_t* __restrict__ entries, const float* __restrict__ scale,
                         const float* __restrict__ bias, int64_t n, int k, float* __restrict__ out) {
@@ -275,7 +282,7 @@ sparse_gemv_smem_kernel(const uint16_t* __restrict__ x, const int64_t* __restric
     uint32_t v[kSpR][kSpW];
 #pragma unroll
     for (int j = 0; j < kSpR; ++j) {
-      const int rl = warp + 32 * j;
+      const int rl = warp + kSpWarps * j;
       const int64_t b = rl < rows ? rp[rl] : 0, e = rl < rows ? rp[rl + 1] : 0;
       const int64_t a = b & ~int64_t{1};
 #pragma unroll
@@ -290,7 +297,7 @@ sparse_gemv_smem_kernel(const uint16_t* __restrict__ x, const int64_t* __restric
     }
 #pragma unroll
     for (int j = 0; j < kSpR; ++j) {
-      const int rl = warp + 32 * j;
+      const int rl = warp + kSpWarps * j;
       if (rl >= rows) break;
       const int64_t b = rp[rl], e = rp[rl + 1];
       int64_t a = b & ~int64_t{1};
@@ -355,8 +362,10 @@ extern "C" bnn_status bnn_ternary_sparse_gemm(const uint16_t* x_bf16, const int6
     return BNN_ERR_MISALIGNED;
   if (m == 1 && k > 0) {
     const size_t smem = static_cast<size_t>(k + 1) * sizeof(float);
-    const int64_t sms = bnn::sm_count();
-    const int grid = static_cast<int>(n < sms ? n : sms);
+    // two CTAs per SM where their x copies fit one SM's shared memory together
+    const int per_sm = 2 * (smem + 2048) <= 228u * 1024u ? kSpPerSm : 1;
+    const int64_t slots = bnn::sm_count() * static_cast<int64_t>(per_sm);
+    const int grid = static_cast<int>(n < slots ? n : slots);
     if (entries && bnn::aligned(entries, 4)) {
       BNN_TRY(bnn::ensure_smem(sparse_gemv_smem_kernel<true>, smem));
       BNN_TRY(bnn::launch_pdl(sparse_gemv_smem_kernel<true>, dim3(grid), dim3(kSpThreads), smem, s, 1, x_bf16,
