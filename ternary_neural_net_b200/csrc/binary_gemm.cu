@@ -150,7 +150,11 @@ void launch_gemv(const uint64_t* xp, const uint64_t* wp, const float* alpha, int
   constexpr int threads = 256;
   constexpr int64_t rows_per_block = (threads / 32) * (32 / LPR) * R;
   const int64_t blocks_needed = (n + rows_per_block - 1) / rows_per_block;
-  const int64_t cap = static_cast<int64_t>(bnn::sm_count()) * 8;
+  // One block per row block (waves of 8 per SM): blocks that finish early
+  // take the next ones, so the stream ends evenly.  A grid capped at one wave
+  // (grid-stride) left half the warps a second pass at 1 x 28672 x 8192: 6.45
+  // against 5.91 us.  The cap only bounds the grid for very large n.
+  const int64_t cap = static_cast<int64_t>(bnn::sm_count()) * 64;
   const int grid = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
   bnn::launch_pdl(binary_gemv_kernel<VEC, LPR, R, MT, P>, dim3(grid), dim3(threads), 0, s, 1, xp, wp, alpha, m, n,
                   k, kw, dots, out);
